@@ -1,0 +1,205 @@
+/*
+ * hkv.h -- C ABI of libhkv, a B200 (sm_100a) library for head-aware
+ * key-value cache compression in autoregressive image generation (HeadKV).
+ *
+ * The operations follow the technical summary of the explainer pages of
+ * "Head-Aware Key-Value Compression for Efficient Autoregressive Image
+ * Generation" (Liang, Zhang, Wen, Ye; gist.science, ja/de/fr/ko/es pages).
+ * Passages are named by that summary's parts:
+ *   Methodology step 1 (cache prefilling), step 2 (head grouping),
+ *   step 3 (head-specific compression: Local sliding window; Global
+ *   Stratified Token Eviction), Main contributions (asymmetric budgets),
+ *   Problem statement (the KV cache of autoregressive decoding).
+ *
+ * Conventions for every call:
+ *  - Pointers named *_host are host memory; all others are device memory of
+ *    the GPU the context was created on.  The library allocates nothing: the
+ *    state lives in one caller-owned device buffer (the pool) and inputs and
+ *    outputs are caller-owned.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *    call that takes one only enqueues work on it; calls on one context must
+ *    be ordered (one stream, or explicit dependencies): they share scratch.
+ *  - Argument errors are reported synchronously and enqueue nothing.
+ *    Errors found on the device (a numeric fault, an index out of range) are
+ *    latched in a device status word, never trap, and are read back by
+ *    hkv_check.
+ *  - Tensors are row-major.  S = num_seqs, H = num_heads, d = head_dim.
+ *    Element type is the config's dtype (fp32 or bf16) unless stated.
+ */
+#ifndef HKV_H
+#define HKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HKV_API __attribute__((visibility("default")))
+#else
+#define HKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HKV_OK = 0,
+    HKV_ERR_INVALID_ARG = 1, /* bad pointer, size, layer or config value */
+    HKV_ERR_STATE = 2,       /* call out of order (e.g. decode before classify) */
+    HKV_ERR_CAPACITY = 3,    /* pool too small, sequence longer than max_len */
+    HKV_ERR_NUMERIC = 4,     /* NaN/inf met in a softmax or a score */
+    HKV_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
+    HKV_ERR_TIMEOUT = 6      /* a bounded device wait gave up */
+} hkv_status;
+
+typedef enum { HKV_DTYPE_F32 = 0, HKV_DTYPE_BF16 = 1 } hkv_dtype;
+
+typedef enum {
+    HKV_MODE_HEADKV = 0,  /* the method: Local window / Global STE */
+    HKV_MODE_FULL = 1,    /* full cache, no compression (comparison baseline) */
+    HKV_MODE_UNIFORM = 2  /* one uniform budget for every head, STE eviction */
+} hkv_mode;
+
+typedef struct {
+    int32_t num_seqs;     /* S: independent sequences (CFG halves included) */
+    int32_t num_layers;   /* layers; each keeps its own cache */
+    int32_t num_heads;    /* H: attention heads (as many KV heads) */
+    int32_t head_dim;     /* d: 64 or 128 */
+    int32_t dtype;        /* hkv_dtype of q, k, v, outputs and the cache */
+    int32_t max_len;      /* L: longest sequence (prefix + all image tokens) */
+    int32_t local_window; /* W: Local heads keep the W most recent tokens */
+    int32_t ste_m;        /* M: tokens one STE evicts (even; M/2 per stratum) */
+    int32_t near_dist;    /* D: near stratum = distance 1..D, far = beyond */
+    int32_t score_window; /* r: queries of the last r steps score tokens, r <= M */
+    int32_t rho_num;      /* rho = rho_num / rho_den: kept share of the full cache */
+    int32_t rho_den;
+    int32_t mode;         /* hkv_mode */
+    int32_t stratified;   /* 1: near/far strata (STE); 0: one pool */
+    double tau;           /* grouping threshold, 0.9 on the pages */
+} hkv_config;
+
+typedef struct hkv_ctx hkv_ctx;
+
+/* Human-readable name of a status code (static string). */
+HKV_API const char* hkv_status_string(hkv_status s);
+
+/* Bytes of device memory the pool of `cfg` needs (state + scratch).
+ * Budgets [Main contributions]: each (sequence, layer) region holds
+ * floor(H * L * rho) + H * M slots for HKV_MODE_HEADKV.
+ * Errors: HKV_ERR_INVALID_ARG for an unusable config, including
+ * floor(H * L * rho) < H * W (the budget cannot give every head W). */
+HKV_API hkv_status hkv_pool_bytes(const hkv_config* cfg, size_t* bytes);
+
+/* Binds a context to `pool` (device memory on the current CUDA device,
+ * >= hkv_pool_bytes bytes, 256-byte aligned, owned by the caller and kept
+ * alive until hkv_destroy).  Enqueues the clearing of the pool's control
+ * words on `stream`.  *out receives the context (host memory owned by the
+ * library until hkv_destroy). */
+HKV_API hkv_status hkv_create(const hkv_config* cfg, void* pool, size_t bytes, void* stream,
+                      hkv_ctx** out);
+
+/* Cache prefilling and head grouping for one layer [Methodology steps 1-2],
+ * then compression at classification time [step 3].  Must be called once
+ * per layer before any append or decode on it.
+ *  q, k, v: S*H blocks of [prefill_len][d]; block b = s*H + h starts at
+ *           element b * block_stride (block_stride >= prefill_len * d).
+ *  out:     [S][H][prefill_len][d] causal attention outputs, or NULL.
+ * Causal softmax(q k^T / sqrt(d)) v over the prefill tokens.  Each head is
+ * then labelled from the weights of the last prefill query: Local iff the
+ * newest tokens reach tau in fewer than W tokens.  Budgets follow: Local
+ * heads keep W, Global heads split floor(H*L*rho) - nL*W evenly (rounded
+ * down) per (sequence, layer).  Local heads keep their last W prefill
+ * tokens; Global heads keep all, or, beyond their budget, run one
+ * Stratified Token Eviction (E = prefill_len - budget: floor(E/2) near,
+ * ceil(E/2) far) scored by the last r prefill queries.
+ * Requirements: W <= prefill_len < max_len, r <= prefill_len.
+ * Errors: INVALID_ARG (pointers, sizes), STATE (layer already classified). */
+HKV_API hkv_status hkv_prefill_classify(hkv_ctx* ctx, int32_t layer, const void* q, const void* k,
+                                const void* v, int32_t prefill_len, int64_t block_stride,
+                                void* out, void* stream);
+
+/* Appends the next token's key and value ([S][H][d] each) to every head of
+ * `layer` [step 3]: Local heads overwrite their oldest token (sliding
+ * window), Global heads add it at the tail.  Errors: STATE (layer not
+ * classified), CAPACITY (sequence already max_len long). */
+HKV_API hkv_status hkv_append(hkv_ctx* ctx, int32_t layer, const void* k_t, const void* v_t,
+                      void* stream);
+
+/* Decode attention of the newest token over each head's compressed cache
+ * [Problem statement; step 3]: o_t = softmax(q_t K^T / sqrt(d)) V over the
+ * head's kept tokens (the newest included).  q_t, o_t: [S][H][d].  For a
+ * Global head within r steps of its next eviction the same pass records the
+ * logits the STE scores are built from [step 3, STE scores].
+ * Errors: STATE (layer not classified or nothing appended yet). */
+HKV_API hkv_status hkv_decode_attend(hkv_ctx* ctx, int32_t layer, const void* q_t, void* o_t,
+                             void* stream);
+
+/* hkv_append followed by hkv_decode_attend in one kernel. */
+HKV_API hkv_status hkv_decode_step(hkv_ctx* ctx, int32_t layer, const void* q_t, const void* k_t,
+                           const void* v_t, void* o_t, void* stream);
+
+/* Stratified Token Eviction [step 3, Global heads] on layers
+ * [layer_begin, layer_end): every Global head whose cache reached
+ * budget + M tokens splits its past tokens (distance >= 1 from the newest)
+ * into near (distance <= D) and far strata, scores each token by the summed
+ * softmax weight the last r queries gave it, and evicts the M/2 lowest
+ * (score, position) of each stratum, ties going to the lower position; the
+ * cache is compacted in place.  Heads that are not due are left untouched,
+ * so one call per decode step serves every step.
+ * Errors: INVALID_ARG (layer range), STATE (a layer not classified). */
+HKV_API hkv_status hkv_ste_evict(hkv_ctx* ctx, int32_t layer_begin, int32_t layer_end, void* stream);
+
+/* Head labels of one layer (1 = Local, 0 = Global, 2 = full mode) and the
+ * token counts n_tau that decided them, [S][H] each (n_tau_host nullable).
+ * Waits for `stream`. */
+HKV_API hkv_status hkv_get_labels(hkv_ctx* ctx, int32_t layer, uint8_t* labels_host,
+                          int32_t* n_tau_host, void* stream);
+
+/* Cache lengths [S][H] and per-head budgets [S][H] (nullable) of one layer
+ * as of the work enqueued so far.  Waits for `stream`. */
+HKV_API hkv_status hkv_get_lens(hkv_ctx* ctx, int32_t layer, int32_t* len_host, int32_t* budget_host,
+                        void* stream);
+
+/* Positions cached by one head, ascending, into pos_host[0..capacity);
+ * *len_out = how many.  Waits for `stream`.  CAPACITY if capacity < len. */
+HKV_API hkv_status hkv_get_kept(hkv_ctx* ctx, int32_t seq, int32_t layer, int32_t head,
+                        int32_t* pos_host, int32_t capacity, int32_t* len_out, void* stream);
+
+/* Reads the device status word (waits for `stream`) and returns the first
+ * error latched on the device, or HKV_OK.  *detail_host (nullable) gets a
+ * code-specific detail (e.g. the head index). */
+HKV_API hkv_status hkv_check(hkv_ctx* ctx, int32_t* detail_host, void* stream);
+
+/* Clears a latched device error. */
+HKV_API hkv_status hkv_clear_error(hkv_ctx* ctx, void* stream);
+
+/* Releases the context (not the pool). */
+HKV_API void hkv_destroy(hkv_ctx* ctx);
+
+/* ---- Standalone primitives on caller-supplied device arrays -------------- */
+
+/* Head grouping rule [step 2] on n_rows weight rows (fp32, [n_rows][n]): row
+ * i holds the weights of a query at position n-1 over positions 0..n-1.
+ * n_tau[i] (int32) = tokens the backward accumulation needs to reach tau
+ * (n if never); label[i] (uint8) = 1 iff n_tau[i] < W.  Accumulation in
+ * double.  Errors: INVALID_ARG. */
+HKV_API hkv_status hkv_classify_rows(const float* rows, int32_t n_rows, int32_t n, int32_t W,
+                             double tau, int32_t* n_tau, uint8_t* label, void* stream);
+
+/* Stratified selection [step 3, STE] on n_probs independent problems.
+ * Problem i has count[i] <= n tokens: score[i*n + j] (fp32, >= 0) and
+ * pos[i*n + j] (int32, distinct); the newest position is t[i].  Evicts
+ * k_near lowest (score, position) of the near stratum (distance 1..D) and
+ * k_far of the far one (distance > D); a stratum short of candidates hands
+ * the shortfall to the other; stratified = 0 pools them.  evict[i*n + j]
+ * (uint8) = 1 for evicted tokens.  n <= 4096.  Errors: INVALID_ARG; a NaN
+ * score latches nothing here (no context) and selects as the largest key. */
+HKV_API hkv_status hkv_ste_select_batch(const float* score, const int32_t* pos, const int32_t* count,
+                                const int32_t* t, int32_t n_probs, int32_t n, int32_t D,
+                                int32_t k_near, int32_t k_far, int32_t stratified,
+                                uint8_t* evict, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HKV_H */

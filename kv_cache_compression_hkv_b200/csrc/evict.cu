@@ -1,0 +1,219 @@
+// evict.cu -- Stratified Token Eviction for Global heads (HeadKV technical
+// summary, Methodology step 3, global heads) and the standalone grouping and
+// selection primitives.
+//
+// One warp per due head: it turns the logits the decode kernel stored over
+// the last r steps into scores (summed softmax weights, each step normalised
+// by its own (max, sum) and counting only tokens already cached at that
+// step), selects the M/2 lowest (score, position) of the near and the far
+// strata with a warp bisection, and compacts the cache in place by moving
+// the surviving tail tokens into the holes below the budget.
+#include <math.h>
+
+#include "hkv_internal.cuh"
+#include "kernels.h"
+
+namespace hkv {
+
+template <typename T>
+__global__ void __launch_bounds__(128) evict_kernel(Layout L, int l0, int l1, int n_max) {
+    extern __shared__ __align__(16) unsigned char esm[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int NW = blockDim.x >> 5;
+    SelectScratch sc = carve_select_scratch(esm + (size_t)warp * select_scratch_bytes(n_max), n_max);
+    const int n_heads = L.S * L.H;
+    const int total = (l1 - l0) * n_heads;
+    const int d = L.d;
+    const int r = L.r;
+    T* Kp = reinterpret_cast<T*>(L.K);
+    T* Vp = reinterpret_cast<T*>(L.V);
+    constexpr int PIECE = 16 / sizeof(T);  // elements per 16-byte piece
+    const int per_row = d / PIECE;
+
+    for (int base = (blockIdx.x * NW + warp) * 32; base < total; base += gridDim.x * NW * 32) {
+        const int i = base + lane;
+        bool due = false;
+        if (i < total && L.mode != HKV_MODE_FULL) {
+            const int l = l0 + i / n_heads;
+            const size_t hx = (size_t)l * n_heads + (i % n_heads);
+            const int t = L.t_next[l] - 1;
+            due = L.label[hx] == 0 && len_at(L, hx, t) >= L.cap[hx];
+        }
+        unsigned todo = __ballot_sync(FULL_MASK, due);
+        while (todo) {
+            const int lead = __ffs(todo) - 1;
+            todo &= todo - 1;
+            const int j = base + lead;
+            const int l = l0 + j / n_heads;
+            const int hs = j % n_heads;
+            const int s = hs / L.H;
+            const size_t hx = (size_t)l * n_heads + hs;
+            const int t = L.t_next[l] - 1;
+            const int n = len_at(L, hx, t);
+            const int target = L.budget[hx];
+            if (n > n_max || n != L.cap[hx]) {
+                if (lane == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
+                continue;
+            }
+            const size_t slot0 = region_slot0(L, l, s) + L.off[hx];
+            const float2* mlh = L.ml + hx * r;  // (max, sum) of each scoring step
+            bool bad = false;
+            // called only by lanes that hold a token: no warp collectives here
+            auto key_of = [&](int q, uint32_t& sb, int32_t& p) {
+                p = L.pos[slot0 + q];
+                const float* lg = L.logit + (slot0 + q) * r;
+                float sc_ = 0.f;
+                for (int step = t - r + 1; step <= t; ++step) {
+                    if (p > step) continue;  // not yet cached at that step
+                    const int col = step % r;
+                    const float2 ml = mlh[col];
+                    sc_ += exp2f(lg[col] - ml.x) / ml.y;
+                }
+                if (isnan(sc_)) bad = true;
+                sb = __float_as_uint(sc_);
+            };
+            const int E = n - target;
+            warp_stratified_select(sc, n, t, L.D, E / 2, E - E / 2, L.stratified, key_of);
+            if (__any_sync(FULL_MASK, bad) && lane == 0) latch_error(L, HKV_ERR_NUMERIC, (int)hx);
+            // holes: evicted slots below the budget; movers: survivors above it
+            int nh = 0, nm = 0;
+            for (int b0 = 0; b0 < n; b0 += 32) {
+                const int q = b0 + lane;
+                const bool ev = q < n && ((sc.evict_bits[q >> 5] >> (q & 31)) & 1u);
+                const bool hole = q < target && ev;
+                const bool mover = q >= target && q < n && !ev;
+                const unsigned bh = __ballot_sync(FULL_MASK, hole);
+                const unsigned bm = __ballot_sync(FULL_MASK, mover);
+                const unsigned lt = (1u << lane) - 1u;
+                if (hole) sc.moves[nh + __popc(bh & lt)] = (uint16_t)q;
+                if (mover) sc.moves[sc.n_max - 1 - (nm + __popc(bm & lt))] = (uint16_t)q;
+                nh += __popc(bh);
+                nm += __popc(bm);
+            }
+            __syncwarp();
+            if (nh != nm) {
+                if (lane == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
+                continue;
+            }
+            // move rows: K and V, 16-byte pieces, four per lane in flight
+            const int pieces = nh * per_row * 2;
+            for (int w0 = 0; w0 < pieces; w0 += 32 * 4) {
+                uint4 buf[4];
+                size_t dst[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int w = w0 + u * 32 + lane;
+                    if (w < pieces) {
+                        const int mv = w / (per_row * 2);
+                        const int rem = w % (per_row * 2);
+                        const bool isv = rem >= per_row;
+                        const int pc = (isv ? rem - per_row : rem) * PIECE;
+                        const size_t src = (slot0 + sc.moves[sc.n_max - 1 - mv]) * d + pc;
+                        dst[u] = (slot0 + sc.moves[mv]) * d + pc;
+                        buf[u] = *reinterpret_cast<const uint4*>((isv ? Vp : Kp) + src);
+                        dst[u] |= (size_t)isv << 62;
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int w = w0 + u * 32 + lane;
+                    if (w < pieces) {
+                        const bool isv = (dst[u] >> 62) & 1;
+                        const size_t o = dst[u] & ~(3ull << 62);
+                        *reinterpret_cast<uint4*>((isv ? Vp : Kp) + o) = buf[u];
+                    }
+                }
+            }
+            for (int mv = lane; mv < nh; mv += 32)
+                L.pos[slot0 + sc.moves[mv]] = L.pos[slot0 + sc.moves[sc.n_max - 1 - mv]];
+            __syncwarp();
+            if (lane == 0) {
+                L.base_len[hx] = target;
+                L.base_t[hx] = t;
+            }
+        }
+    }
+}
+
+// Standalone grouping rule over weight rows, one warp per row.
+__global__ void classify_rows_kernel(const float* __restrict__ rows, int n_rows, int n, int W,
+                                     double tau, int32_t* __restrict__ n_tau,
+                                     uint8_t* __restrict__ label) {
+    const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (row >= n_rows) return;
+    const int need = warp_tokens_to_tau(rows + (size_t)row * n, n, tau);
+    if ((threadIdx.x & 31) == 0) {
+        n_tau[row] = need;
+        label[row] = need < W ? 1 : 0;
+    }
+}
+
+// Standalone stratified select, one warp per problem.
+__global__ void __launch_bounds__(128) select_batch_kernel(
+    const float* __restrict__ score, const int32_t* __restrict__ pos, const int32_t* __restrict__ count,
+    const int32_t* __restrict__ tt, int n_probs, int n, int D, int k_near, int k_far, int stratified,
+    uint8_t* __restrict__ evict) {
+    extern __shared__ __align__(16) unsigned char ssm[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int prob = blockIdx.x * (blockDim.x >> 5) + warp;
+    if (prob >= n_probs) return;
+    SelectScratch sc = carve_select_scratch(ssm + (size_t)warp * select_scratch_bytes(n), n);
+    const int m = min(max(count[prob], 0), n);
+    const float* sp = score + (size_t)prob * n;
+    const int32_t* pp = pos + (size_t)prob * n;
+    auto key_of = [&](int i, uint32_t& sb, int32_t& p) {
+        sb = __float_as_uint(sp[i]);
+        p = pp[i];
+    };
+    warp_stratified_select(sc, m, tt[prob], D, k_near, k_far, stratified, key_of);
+    for (int i = lane; i < n; i += 32)
+        evict[(size_t)prob * n + i] = i < m ? (uint8_t)((sc.evict_bits[i >> 5] >> (i & 31)) & 1u) : 0;
+}
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+
+static int evict_warps(int n_max) {
+    const size_t per = select_scratch_bytes(n_max);
+    int w = (int)((200 * 1024) / per);
+    return w < 1 ? 1 : (w > 4 ? 4 : w);
+}
+
+cudaError_t launch_evict(const Layout& L, int l0, int l1, int grid, cudaStream_t st) {
+    const int n_max = L.L;
+    const int nw = evict_warps(n_max);
+    const size_t sm = (size_t)nw * select_scratch_bytes(n_max);
+    cudaError_t e;
+    if (L.dtype == HKV_DTYPE_BF16) {
+        e = cudaFuncSetAttribute(evict_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+        evict_kernel<__nv_bfloat16><<<grid, 32 * nw, sm, st>>>(L, l0, l1, n_max);
+    } else {
+        e = cudaFuncSetAttribute(evict_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+        evict_kernel<float><<<grid, 32 * nw, sm, st>>>(L, l0, l1, n_max);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_classify_rows(const float* rows, int n_rows, int n, int W, double tau,
+                                 int32_t* n_tau, uint8_t* label, cudaStream_t st) {
+    const int grid = (n_rows + 7) / 8;
+    classify_rows_kernel<<<grid, 256, 0, st>>>(rows, n_rows, n, W, tau, n_tau, label);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select_batch(const float* score, const int32_t* pos, const int32_t* count,
+                                const int32_t* t, int n_probs, int n, int D, int k_near, int k_far,
+                                int stratified, uint8_t* evict, cudaStream_t st) {
+    const int nw = 4;
+    const size_t sm = (size_t)nw * select_scratch_bytes(n);
+    cudaError_t e = cudaFuncSetAttribute(select_batch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    select_batch_kernel<<<(n_probs + nw - 1) / nw, 32 * nw, sm, st>>>(
+        score, pos, count, t, n_probs, n, D, k_near, k_far, stratified, evict);
+    return cudaGetLastError();
+}
+
+}  // namespace hkv

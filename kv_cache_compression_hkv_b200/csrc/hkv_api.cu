@@ -1,0 +1,365 @@
+// hkv_api.cu -- the C ABI declared in include/hkv.h: argument checks, the
+// carving of the caller-owned pool, call-order bookkeeping and launches.
+// Every function here only validates and enqueues; the arithmetic of the
+// hot path runs in the kernels.
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+#include <vector>
+
+#include "hkv_internal.cuh"
+#include "kernels.h"
+
+using hkv::Layout;
+
+struct hkv_ctx {
+    hkv_config cfg;
+    Layout lay;
+    int device;
+    int n_sm;
+    int decode_grid;
+    int evict_grid;
+    int64_t t_total;
+    std::vector<int> classified;  // per layer
+    std::vector<int> t_host;      // per layer: next position, as enqueued by API calls
+    std::vector<int> prefill_len;
+};
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+size_t elem_size(int dtype) { return dtype == HKV_DTYPE_F32 ? 4 : 2; }
+
+bool config_ok(const hkv_config* c, int64_t* T_out, int32_t* R_out) {
+    if (!c) return false;
+    if (c->num_seqs < 1 || c->num_layers < 1 || c->num_heads < 1 || c->num_heads > 32) return false;
+    if (c->head_dim != 64 && c->head_dim != 128) return false;
+    if (c->dtype != HKV_DTYPE_F32 && c->dtype != HKV_DTYPE_BF16) return false;
+    if (c->max_len < 2 || c->max_len > 8192) return false;
+    if (c->local_window < 1 || c->local_window > c->max_len) return false;
+    if (c->ste_m < 2 || (c->ste_m & 1)) return false;
+    if (c->near_dist < 0) return false;
+    if (c->score_window < 1 || c->score_window > c->ste_m || c->score_window > 32) return false;
+    if (c->rho_num < 1 || c->rho_den < c->rho_num) return false;
+    if (c->mode < HKV_MODE_HEADKV || c->mode > HKV_MODE_UNIFORM) return false;
+    if (c->stratified != 0 && c->stratified != 1) return false;
+    if (!(c->tau > 0.0 && c->tau <= 1.0)) return false;
+    if ((int64_t)c->num_seqs * c->num_heads > 12288) return false;
+    const int64_t H = c->num_heads, L = c->max_len;
+    const int64_t T = H * L * c->rho_num / c->rho_den;
+    int64_t R;
+    if (c->mode == HKV_MODE_HEADKV) {
+        if (T < H * c->local_window) return false;
+        R = T + H * c->ste_m;
+    } else if (c->mode == HKV_MODE_UNIFORM) {
+        if (T / H < 1) return false;
+        R = (T / H + c->ste_m) * H;
+    } else {
+        R = H * L;
+    }
+    if (R > (int64_t)1 << 30) return false;
+    if (T_out) *T_out = T;
+    if (R_out) *R_out = (int32_t)R;
+    return true;
+}
+
+// Carves the pool.  With base == nullptr only sizes are computed.
+size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Layout* L) {
+    const size_t S = c->num_seqs, Ly = c->num_layers, H = c->num_heads, d = c->head_dim;
+    const size_t r = c->score_window, Lmax = c->max_len;
+    const size_t es = elem_size(c->dtype);
+    const size_t nh = Ly * S * H;
+    const size_t slots = Ly * S * (size_t)R;
+    const size_t max_chunks = S * ((size_t)R / hkv::CHUNK + H + 1);
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o = align_up(o + bytes);
+        return base ? base + at : nullptr;
+    };
+    Layout l;
+    memset(&l, 0, sizeof(l));
+    l.status = (int32_t*)take(16);
+    l.t_next = (int32_t*)take(Ly * 4);
+    l.done_ctr = (int32_t*)take(Ly * 4);
+    l.ticket = (int32_t*)take(S * H * 4);
+    const size_t ctrl_end = o;
+    l.off = (int32_t*)take(nh * 4);
+    l.cap = (int32_t*)take(nh * 4);
+    l.budget = (int32_t*)take(nh * 4);
+    l.base_len = (int32_t*)take(nh * 4);
+    l.base_t = (int32_t*)take(nh * 4);
+    l.n_tau = (int32_t*)take(nh * 4);
+    l.label = (uint8_t*)take(nh);
+    l.due_t = (int32_t*)take(Ly * S * 4);
+    l.K = take(slots * d * es);
+    l.V = take(slots * d * es);
+    l.pos = (int32_t*)take(slots * 4);
+    l.logit = (float*)take(slots * r * 4);
+    l.ml = (float2*)take(nh * r * 8);
+    l.rows = (float*)take(S * H * r * Lmax * 4);
+    l.partial = (float*)take(max_chunks * (d + 2) * 4);
+    l.S = c->num_seqs; l.Ly = c->num_layers; l.H = c->num_heads; l.d = c->head_dim;
+    l.L = c->max_len; l.W = c->local_window; l.M = c->ste_m; l.D = c->near_dist;
+    l.r = c->score_window; l.mode = c->mode; l.stratified = c->stratified; l.dtype = c->dtype;
+    l.R = R; l.T_total = T; l.tau = c->tau; l.max_chunks = (int32_t)max_chunks;
+    if (L) *L = l;
+    (void)ctrl_end;
+    return o;
+}
+
+size_t ctrl_bytes(const hkv_config* c) {
+    // status, t_next, done_ctr and ticket are laid out first (see carve)
+    size_t o = 0;
+    o = align_up(o + 16);
+    o = align_up(o + (size_t)c->num_layers * 4);
+    o = align_up(o + (size_t)c->num_layers * 4);
+    o = align_up(o + (size_t)c->num_seqs * c->num_heads * 4);
+    return o;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+hkv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HKV_OK : HKV_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* hkv_status_string(hkv_status s) {
+    switch (s) {
+        case HKV_OK: return "HKV_OK";
+        case HKV_ERR_INVALID_ARG: return "HKV_ERR_INVALID_ARG";
+        case HKV_ERR_STATE: return "HKV_ERR_STATE";
+        case HKV_ERR_CAPACITY: return "HKV_ERR_CAPACITY";
+        case HKV_ERR_NUMERIC: return "HKV_ERR_NUMERIC";
+        case HKV_ERR_CUDA: return "HKV_ERR_CUDA";
+        case HKV_ERR_TIMEOUT: return "HKV_ERR_TIMEOUT";
+    }
+    return "HKV_ERR_UNKNOWN";
+}
+
+hkv_status hkv_pool_bytes(const hkv_config* cfg, size_t* bytes) {
+    int64_t T;
+    int32_t R;
+    if (!bytes || !config_ok(cfg, &T, &R)) return HKV_ERR_INVALID_ARG;
+    *bytes = carve(cfg, T, R, nullptr, nullptr);
+    return HKV_OK;
+}
+
+hkv_status hkv_create(const hkv_config* cfg, void* pool, size_t bytes, void* stream, hkv_ctx** out) {
+    int64_t T;
+    int32_t R;
+    if (!out || !pool || ((uintptr_t)pool % kAlign) != 0 || !config_ok(cfg, &T, &R))
+        return HKV_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (bytes < carve(cfg, T, R, nullptr, nullptr)) return HKV_ERR_CAPACITY;
+    hkv_ctx* c = new (std::nothrow) hkv_ctx();
+    if (!c) return HKV_ERR_CAPACITY;
+    c->cfg = *cfg;
+    c->t_total = T;
+    carve(cfg, T, R, (unsigned char*)pool, &c->lay);
+    c->classified.assign(cfg->num_layers, 0);
+    c->t_host.assign(cfg->num_layers, 0);
+    c->prefill_len.assign(cfg->num_layers, 0);
+    cudaError_t e = cudaGetDevice(&c->device);
+    if (e == cudaSuccess)
+        e = cudaDeviceGetAttribute(&c->n_sm, cudaDevAttrMultiProcessorCount, c->device);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(pool, 0, ctrl_bytes(cfg), (cudaStream_t)stream);
+    if (e != cudaSuccess) {
+        delete c;
+        return HKV_ERR_CUDA;
+    }
+    c->decode_grid = c->n_sm;      // one 256-thread block per SM (register-bound)
+    c->evict_grid = c->n_sm * 2;
+    *out = c;
+    return HKV_OK;
+}
+
+hkv_status hkv_prefill_classify(hkv_ctx* c, int32_t layer, const void* q, const void* k,
+                                const void* v, int32_t prefill_len, int64_t block_stride,
+                                void* out, void* stream) {
+    if (!c || !q || !k || !v) return HKV_ERR_INVALID_ARG;
+    const hkv_config& g = c->cfg;
+    if (layer < 0 || layer >= g.num_layers) return HKV_ERR_INVALID_ARG;
+    const int P = prefill_len;
+    if (P < g.local_window || P >= g.max_len || P < g.score_window || P < 2)
+        return HKV_ERR_INVALID_ARG;
+    const size_t es = elem_size(g.dtype);
+    if (block_stride < (int64_t)P * g.head_dim || (block_stride * (int64_t)es) % 16 != 0)
+        return HKV_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || (out && !aligned16(out)))
+        return HKV_ERR_INVALID_ARG;
+    if (c->classified[layer]) return HKV_ERR_STATE;
+    if (hkv::pack_smem_bytes(P) > 200 * 1024) return HKV_ERR_INVALID_ARG;
+    cudaError_t e = hkv::launch_prefill(c->lay, layer, q, k, v, P, block_stride, out,
+                                        (cudaStream_t)stream);
+    if (e != cudaSuccess) return HKV_ERR_CUDA;
+    c->classified[layer] = 1;
+    c->t_host[layer] = P;
+    c->prefill_len[layer] = P;
+    return HKV_OK;
+}
+
+static hkv_status step_check(hkv_ctx* c, int32_t layer, bool appends) {
+    if (!c) return HKV_ERR_INVALID_ARG;
+    if (layer < 0 || layer >= c->cfg.num_layers) return HKV_ERR_INVALID_ARG;
+    if (!c->classified[layer]) return HKV_ERR_STATE;
+    if (appends && c->t_host[layer] >= c->cfg.max_len) return HKV_ERR_CAPACITY;
+    return HKV_OK;
+}
+
+hkv_status hkv_append(hkv_ctx* c, int32_t layer, const void* k_t, const void* v_t, void* stream) {
+    hkv_status s = step_check(c, layer, true);
+    if (s != HKV_OK) return s;
+    if (!k_t || !v_t || !aligned16(k_t) || !aligned16(v_t)) return HKV_ERR_INVALID_ARG;
+    cudaError_t e = hkv::launch_append(c->lay, layer, k_t, v_t, (cudaStream_t)stream);
+    if (e != cudaSuccess) return HKV_ERR_CUDA;
+    c->t_host[layer] += 1;
+    return HKV_OK;
+}
+
+hkv_status hkv_decode_attend(hkv_ctx* c, int32_t layer, const void* q_t, void* o_t, void* stream) {
+    hkv_status s = step_check(c, layer, false);
+    if (s != HKV_OK) return s;
+    if (!q_t || !o_t || !aligned16(q_t) || !aligned16(o_t)) return HKV_ERR_INVALID_ARG;
+    return cuda_status(hkv::launch_decode(c->lay, layer, q_t, nullptr, nullptr, o_t, 0,
+                                          c->decode_grid, (cudaStream_t)stream));
+}
+
+hkv_status hkv_decode_step(hkv_ctx* c, int32_t layer, const void* q_t, const void* k_t,
+                           const void* v_t, void* o_t, void* stream) {
+    hkv_status s = step_check(c, layer, true);
+    if (s != HKV_OK) return s;
+    if (!q_t || !k_t || !v_t || !o_t || !aligned16(q_t) || !aligned16(k_t) || !aligned16(v_t) ||
+        !aligned16(o_t))
+        return HKV_ERR_INVALID_ARG;
+    cudaError_t e = hkv::launch_decode(c->lay, layer, q_t, k_t, v_t, o_t, 1, c->decode_grid,
+                                       (cudaStream_t)stream);
+    if (e != cudaSuccess) return HKV_ERR_CUDA;
+    c->t_host[layer] += 1;
+    return HKV_OK;
+}
+
+hkv_status hkv_ste_evict(hkv_ctx* c, int32_t layer_begin, int32_t layer_end, void* stream) {
+    if (!c || layer_begin < 0 || layer_end > c->cfg.num_layers || layer_begin >= layer_end)
+        return HKV_ERR_INVALID_ARG;
+    for (int l = layer_begin; l < layer_end; ++l)
+        if (!c->classified[l]) return HKV_ERR_STATE;
+    if (c->cfg.mode == HKV_MODE_FULL) return HKV_OK;
+    return cuda_status(hkv::launch_evict(c->lay, layer_begin, layer_end, c->evict_grid,
+                                         (cudaStream_t)stream));
+}
+
+static hkv_status copy_back(void* dst, const void* src, size_t bytes, void* stream) {
+    cudaError_t e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    return cuda_status(e);
+}
+
+hkv_status hkv_get_labels(hkv_ctx* c, int32_t layer, uint8_t* labels_host, int32_t* n_tau_host,
+                          void* stream) {
+    if (!c || !labels_host || layer < 0 || layer >= c->cfg.num_layers) return HKV_ERR_INVALID_ARG;
+    if (!c->classified[layer]) return HKV_ERR_STATE;
+    const size_t nh = (size_t)c->cfg.num_seqs * c->cfg.num_heads;
+    hkv_status s = copy_back(labels_host, c->lay.label + layer * nh, nh, stream);
+    if (s == HKV_OK && n_tau_host) s = copy_back(n_tau_host, c->lay.n_tau + layer * nh, nh * 4, stream);
+    return s;
+}
+
+hkv_status hkv_get_lens(hkv_ctx* c, int32_t layer, int32_t* len_host, int32_t* budget_host,
+                        void* stream) {
+    if (!c || !len_host || layer < 0 || layer >= c->cfg.num_layers) return HKV_ERR_INVALID_ARG;
+    if (!c->classified[layer]) return HKV_ERR_STATE;
+    const size_t nh = (size_t)c->cfg.num_seqs * c->cfg.num_heads;
+    std::vector<int32_t> bl(nh), bt(nh), cap(nh), tn(1);
+    std::vector<uint8_t> lab(nh);
+    hkv_status s = copy_back(bl.data(), c->lay.base_len + layer * nh, nh * 4, stream);
+    if (s == HKV_OK) s = copy_back(bt.data(), c->lay.base_t + layer * nh, nh * 4, stream);
+    if (s == HKV_OK) s = copy_back(cap.data(), c->lay.cap + layer * nh, nh * 4, stream);
+    if (s == HKV_OK) s = copy_back(lab.data(), c->lay.label + layer * nh, nh, stream);
+    if (s == HKV_OK) s = copy_back(tn.data(), c->lay.t_next + layer, 4, stream);
+    if (s == HKV_OK && budget_host) s = copy_back(budget_host, c->lay.budget + layer * nh, nh * 4, stream);
+    if (s != HKV_OK) return s;
+    const int t = tn[0] - 1;  // newest cached position
+    for (size_t i = 0; i < nh; ++i) {
+        int n = bl[i] + (t - bt[i]);
+        if (lab[i] == 1 && n > cap[i]) n = cap[i];
+        len_host[i] = n;
+    }
+    return HKV_OK;
+}
+
+hkv_status hkv_get_kept(hkv_ctx* c, int32_t seq, int32_t layer, int32_t head, int32_t* pos_host,
+                        int32_t capacity, int32_t* len_out, void* stream) {
+    if (!c || !pos_host || !len_out || seq < 0 || seq >= c->cfg.num_seqs || layer < 0 ||
+        layer >= c->cfg.num_layers || head < 0 || head >= c->cfg.num_heads)
+        return HKV_ERR_INVALID_ARG;
+    if (!c->classified[layer]) return HKV_ERR_STATE;
+    const size_t nh = (size_t)c->cfg.num_seqs * c->cfg.num_heads;
+    std::vector<int32_t> lens(nh);
+    hkv_status s = hkv_get_lens(c, layer, lens.data(), nullptr, stream);
+    if (s != HKV_OK) return s;
+    const size_t hi = (size_t)layer * nh + (size_t)seq * c->cfg.num_heads + head;
+    int32_t off = 0;
+    s = copy_back(&off, c->lay.off + hi, 4, stream);
+    if (s != HKV_OK) return s;
+    const int n = lens[(size_t)seq * c->cfg.num_heads + head];
+    *len_out = n;
+    if (n > capacity) return HKV_ERR_CAPACITY;
+    const size_t slot0 = ((size_t)layer * c->cfg.num_seqs + seq) * (size_t)c->lay.R + off;
+    s = copy_back(pos_host, c->lay.pos + slot0, (size_t)n * 4, stream);
+    if (s != HKV_OK) return s;
+    // ascending order (slot order is a ring or a compacted set)
+    for (int i = 1; i < n; ++i) {
+        int32_t x = pos_host[i];
+        int j = i - 1;
+        while (j >= 0 && pos_host[j] > x) { pos_host[j + 1] = pos_host[j]; --j; }
+        pos_host[j + 1] = x;
+    }
+    return HKV_OK;
+}
+
+hkv_status hkv_check(hkv_ctx* c, int32_t* detail_host, void* stream) {
+    if (!c) return HKV_ERR_INVALID_ARG;
+    int32_t w[2] = {0, 0};
+    hkv_status s = copy_back(w, c->lay.status, 8, stream);
+    if (s != HKV_OK) return s;
+    if (detail_host) *detail_host = w[1];
+    return (hkv_status)w[0];
+}
+
+hkv_status hkv_clear_error(hkv_ctx* c, void* stream) {
+    if (!c) return HKV_ERR_INVALID_ARG;
+    return cuda_status(cudaMemsetAsync(c->lay.status, 0, 8, (cudaStream_t)stream));
+}
+
+void hkv_destroy(hkv_ctx* c) { delete c; }
+
+hkv_status hkv_classify_rows(const float* rows, int32_t n_rows, int32_t n, int32_t W, double tau,
+                             int32_t* n_tau, uint8_t* label, void* stream) {
+    if (!rows || !n_tau || !label || n_rows < 0 || n < 1 || W < 1 || !(tau > 0.0 && tau <= 1.0))
+        return HKV_ERR_INVALID_ARG;
+    if (n_rows == 0) return HKV_OK;
+    return cuda_status(hkv::launch_classify_rows(rows, n_rows, n, W, tau, n_tau, label,
+                                                 (cudaStream_t)stream));
+}
+
+hkv_status hkv_ste_select_batch(const float* score, const int32_t* pos, const int32_t* count,
+                                const int32_t* t, int32_t n_probs, int32_t n, int32_t D,
+                                int32_t k_near, int32_t k_far, int32_t stratified, uint8_t* evict,
+                                void* stream) {
+    if (!score || !pos || !count || !t || !evict || n_probs < 0 || n < 1 || n > 4096 || D < 0 ||
+        k_near < 0 || k_far < 0 || (stratified != 0 && stratified != 1))
+        return HKV_ERR_INVALID_ARG;
+    if (n_probs == 0) return HKV_OK;
+    return cuda_status(hkv::launch_select_batch(score, pos, count, t, n_probs, n, D, k_near, k_far,
+                                                stratified, evict, (cudaStream_t)stream));
+}
+
+}  // extern "C"

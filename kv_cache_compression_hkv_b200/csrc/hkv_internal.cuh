@@ -1,0 +1,298 @@
+// hkv_internal.cuh -- device-side layout of the cache pool and helpers shared
+// by the kernels of libhkv.  Everything here runs on sm_100a.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/hkv.h"
+
+namespace hkv {
+
+constexpr unsigned FULL_MASK = 0xffffffffu;
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr int CHUNK = 32;  // tokens one warp handles per decode work item
+
+// Everything a kernel needs to find the state of a (layer, sequence, head).
+// The pool is one caller-owned device buffer carved into these regions.
+struct Layout {
+    int32_t S, Ly, H, d, L, W, M, D, r;
+    int32_t mode, stratified, dtype;
+    int32_t R;          // slots per (sequence, layer) region
+    int64_t T_total;    // floor(H * L * rho): tokens one (sequence, layer) keeps
+    double tau;
+    // control words
+    int32_t* status;    // [0] first error code, [1] detail
+    int32_t* t_next;    // [Ly] position the next append writes
+    int32_t* done_ctr;  // [Ly] CTA arrivals of the running decode launch
+    // per (layer, sequence, head) metadata, index (l*S + s)*H + h
+    int32_t* off;       // first slot of the head inside its region
+    int32_t* cap;       // slots reserved for the head
+    int32_t* budget;    // tokens kept after an eviction (W for Local heads)
+    int32_t* base_len;  // cache length at step base_t
+    int32_t* base_t;    // the length grows by one per step after base_t
+    uint8_t* label;     // 1 Local, 0 Global, 2 full cache
+    int32_t* n_tau;
+    // per (layer, sequence): step at which its Global heads reach their cap
+    int32_t* due_t;
+    // cache rows, slot index (l*S + s)*R + slot
+    void* K;            // [Ly][S][R][d]
+    void* V;
+    int32_t* pos;       // [Ly][S][R]
+    float* logit;       // [Ly][S][R][r]   exp2-domain logits of scoring steps
+    float2* ml;         // [Ly][S][H][r]   (max, sum) of those steps' softmax
+    // scratch, reused by every call
+    float* rows;        // [S*H][r][prefill_len] weights of the last r prefill queries
+    float* partial;     // [max_chunks][d + 2] split-K partial states
+    int32_t* ticket;    // [S*H] arrivals per head of the running decode launch
+    int32_t max_chunks;
+};
+
+__device__ __forceinline__ size_t head_index(const Layout& L, int l, int s, int h) {
+    return ((size_t)l * L.S + s) * L.H + h;
+}
+__device__ __forceinline__ size_t region_slot0(const Layout& L, int l, int s) {
+    return ((size_t)l * L.S + s) * (size_t)L.R;
+}
+
+// Cache length of a head at step t: one token joins per step after base_t;
+// a Local head's ring stops growing at its capacity W.
+__device__ __forceinline__ int len_at(const Layout& L, size_t hi, int t) {
+    int n = L.base_len[hi] + (t - L.base_t[hi]);
+    if (L.label[hi] == 1 && n > L.cap[hi]) n = L.cap[hi];
+    return n;
+}
+
+// Slot (within the head) that the token of position t occupies when appended.
+__device__ __forceinline__ int append_slot(const Layout& L, size_t hi, int t, int len_after) {
+    return L.label[hi] == 1 ? t % L.cap[hi] : len_after - 1;
+}
+
+__device__ __forceinline__ void latch_error(const Layout& L, int code, int detail) {
+    if (atomicCAS(L.status, 0, code) == 0) atomicExch(L.status + 1, detail);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ float to_float(float x) { return x; }
+__device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ void from_float(float& dst, float x) { dst = x; }
+__device__ __forceinline__ void from_float(__nv_bfloat16& dst, float x) { dst = __float2bfloat16_rn(x); }
+
+// Loads DPL consecutive elements starting at p (aligned to DPL elements) as floats.
+template <typename T, int DPL> struct RowSlice;
+template <int DPL> struct RowSlice<float, DPL> {
+    __device__ static __forceinline__ void load(const float* p, float (&x)[DPL]) {
+        if constexpr (DPL == 4) {
+            float4 v = *reinterpret_cast<const float4*>(p);
+            x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+        } else if constexpr (DPL == 2) {
+            float2 v = *reinterpret_cast<const float2*>(p);
+            x[0] = v.x; x[1] = v.y;
+        } else {
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) x[i] = p[i];
+        }
+    }
+    __device__ static __forceinline__ void store(float* p, const float (&x)[DPL]) {
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) p[i] = x[i];
+    }
+};
+template <int DPL> struct RowSlice<__nv_bfloat16, DPL> {
+    __device__ static __forceinline__ void load(const __nv_bfloat16* p, float (&x)[DPL]) {
+        if constexpr (DPL == 4) {
+            uint2 v = *reinterpret_cast<const uint2*>(p);
+            x[0] = bf16_lo(v.x); x[1] = bf16_hi(v.x); x[2] = bf16_lo(v.y); x[3] = bf16_hi(v.y);
+        } else if constexpr (DPL == 2) {
+            uint32_t v = *reinterpret_cast<const uint32_t*>(p);
+            x[0] = bf16_lo(v); x[1] = bf16_hi(v);
+        } else {
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) x[i] = __bfloat162float(p[i]);
+        }
+    }
+    __device__ static __forceinline__ void store(__nv_bfloat16* p, const float (&x)[DPL]) {
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) p[i] = __float2bfloat16_rn(x[i]);
+    }
+};
+
+// ---------------------------------------------------------------------------
+// Warp-level bottom-k selection (Stratified Token Eviction).
+//
+// keys[i] = (bits(score) << 32) | position, score >= +0 so the bit pattern
+// orders like the value; the total order is (score, position), i.e. equal
+// scores evict the lower position first.  Finds the k-th smallest key of
+// keys[0..m) by bisection on the score bits, then on the positions of the
+// tied scores; returns it (every key <= it is evicted).  k >= 1, k <= m.
+// All 32 lanes must call it with the same arguments.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t warp_kth_key(const uint64_t* keys, int m, int k) {
+    const int lane = threadIdx.x & 31;
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    for (int i = lane; i < m; i += 32) {
+        uint32_t sb = (uint32_t)(keys[i] >> 32);
+        lo = min(lo, sb);
+        hi = max(hi, sb);
+    }
+    lo = __reduce_min_sync(FULL_MASK, lo);
+    hi = __reduce_max_sync(FULL_MASK, hi);
+    // smallest score pattern s with #{score <= s} >= k
+    while (lo < hi) {
+        uint32_t mid = lo + ((hi - lo) >> 1);
+        unsigned c = 0;
+        for (int i = lane; i < m; i += 32) c += (uint32_t)(keys[i] >> 32) <= mid;
+        c = __reduce_add_sync(FULL_MASK, c);
+        if ((int)c >= k) hi = mid; else lo = mid + 1;
+    }
+    const uint32_t s_star = lo;
+    unsigned c_lt = 0, c_eq = 0;
+    uint32_t plo = 0xffffffffu, phi = 0u;
+    for (int i = lane; i < m; i += 32) {
+        uint32_t sb = (uint32_t)(keys[i] >> 32);
+        uint32_t p = (uint32_t)keys[i];
+        c_lt += sb < s_star;
+        if (sb == s_star) { ++c_eq; plo = min(plo, p); phi = max(phi, p); }
+    }
+    c_lt = __reduce_add_sync(FULL_MASK, c_lt);
+    c_eq = __reduce_add_sync(FULL_MASK, c_eq);
+    plo = __reduce_min_sync(FULL_MASK, plo);
+    phi = __reduce_max_sync(FULL_MASK, phi);
+    const int need = k - (int)c_lt;  // 1 <= need <= c_eq
+    if (need < (int)c_eq) {
+        while (plo < phi) {
+            uint32_t mid = plo + ((phi - plo) >> 1);
+            unsigned c = 0;
+            for (int i = lane; i < m; i += 32)
+                c += ((uint32_t)(keys[i] >> 32) == s_star) && ((uint32_t)keys[i] <= mid);
+            c = __reduce_add_sync(FULL_MASK, c);
+            if ((int)c >= need) phi = mid; else plo = mid + 1;
+        }
+    } else {
+        plo = phi;  // every tied key goes
+    }
+    return ((uint64_t)s_star << 32) | plo;
+}
+
+// Scratch of one warp's stratified select over up to n_max tokens.  The
+// near keys fill keys[] from the front and the far keys from the back; the
+// same for slot[] and for the hole / mover lists of the compaction.
+struct SelectScratch {
+    uint64_t* keys;        // [n_max]
+    uint16_t* slot;        // [n_max]
+    uint32_t* evict_bits;  // [n_max / 32]
+    uint16_t* moves;       // [n_max]: holes from the front, movers from the back
+    int n_max;
+};
+
+__host__ __device__ inline int round32(int n) { return (n + 31) / 32 * 32; }
+
+__host__ __device__ inline size_t select_scratch_bytes(int n_max) {
+    size_t n = (size_t)round32(n_max);
+    return (n * 8 + n * 2 + (n / 32) * 4 + n * 2 + 15) / 16 * 16;  // 16-byte multiple
+}
+
+__device__ inline SelectScratch carve_select_scratch(unsigned char* base, int n_max) {
+    const int n = round32(n_max);
+    SelectScratch s;
+    s.keys = reinterpret_cast<uint64_t*>(base);
+    s.slot = reinterpret_cast<uint16_t*>(s.keys + n);
+    s.evict_bits = reinterpret_cast<uint32_t*>(s.slot + n);
+    s.moves = reinterpret_cast<uint16_t*>(s.evict_bits + n / 32);
+    s.n_max = n;
+    return s;
+}
+
+// Stratified select over tokens 0..n) whose keys a functor provides:
+// key_of(i, score_bits, pos).  Candidates: t - pos >= 1; near: t - pos <= D
+// (every candidate is "far" when !stratified).  k_near / k_far lowest keys
+// of each stratum are evicted, a stratum short of candidates handing its
+// shortfall to the other.  Sets evict_bits; returns the number evicted.
+// All 32 lanes call it; n <= 65535.
+template <typename KeyOf>
+__device__ int warp_stratified_select(const SelectScratch& sc, int n, int t, int D, int k_near,
+                                      int k_far, int stratified, KeyOf key_of) {
+    const int lane = threadIdx.x & 31;
+    int nn = 0, nf = 0;
+    for (int base = 0; base < n; base += 32) {
+        const int i = base + lane;
+        bool is_near = false, is_far = false;
+        uint64_t key = 0;
+        if (i < n) {
+            uint32_t sb;
+            int32_t p;
+            key_of(i, sb, p);
+            key = ((uint64_t)sb << 32) | (uint32_t)p;
+            const int delta = t - p;
+            if (delta >= 1) {
+                if (stratified && delta <= D) is_near = true; else is_far = true;
+            }
+        }
+        const unsigned bn = __ballot_sync(FULL_MASK, is_near);
+        const unsigned bf = __ballot_sync(FULL_MASK, is_far);
+        const unsigned lt = (1u << lane) - 1u;
+        if (is_near) {
+            const int o = nn + __popc(bn & lt);
+            sc.keys[o] = key;
+            sc.slot[o] = (uint16_t)i;
+        }
+        if (is_far) {
+            const int o = n - 1 - (nf + __popc(bf & lt));
+            sc.keys[o] = key;
+            sc.slot[o] = (uint16_t)i;
+        }
+        nn += __popc(bn);
+        nf += __popc(bf);
+        if (lane == 0) sc.evict_bits[base >> 5] = 0u;
+    }
+    __syncwarp();
+    int kn = k_near, kf = k_far;
+    if (stratified) {
+        if (kn > nn) { kf += kn - nn; kn = nn; }
+        if (kf > nf) { kn += kf - nf; kf = nf; if (kn > nn) kn = nn; }
+    } else {
+        kf = k_near + k_far;
+        kn = 0;
+        if (kf > nf) kf = nf;
+    }
+    for (int which = 0; which < 2; ++which) {
+        const int k = which == 0 ? kn : kf;
+        const int m = which == 0 ? nn : nf;
+        const uint64_t* keys = which == 0 ? sc.keys : sc.keys + (n - nf);
+        const uint16_t* slots = which == 0 ? sc.slot : sc.slot + (n - nf);
+        if (k <= 0) continue;
+        const uint64_t thr = k >= m ? ~0ull : warp_kth_key(keys, m, k);
+        for (int i = lane; i < m; i += 32)
+            if (keys[i] <= thr) atomicOr(&sc.evict_bits[slots[i] >> 5], 1u << (slots[i] & 31));
+    }
+    __syncwarp();
+    return kn + kf;
+}
+
+// Backward accumulation of the head-grouping rule on one weight row
+// (row[j] = weight of the query at position n-1 on position j): the number
+// of tokens, newest first, whose weights first sum to >= tau (n if never).
+// Double-precision running sum.  All lanes call it; all get the answer.
+__device__ __forceinline__ int warp_tokens_to_tau(const float* row, int n, double tau) {
+    const int lane = threadIdx.x & 31;
+    double carry = 0.0;
+    for (int base = 0; base < n; base += 32) {
+        const int delta = base + lane;
+        double x = delta < n ? (double)row[n - 1 - delta] : 0.0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double y = __shfl_up_sync(FULL_MASK, x, o);
+            if (lane >= o) x += y;
+        }
+        const double c = carry + x;
+        const unsigned hit = __ballot_sync(FULL_MASK, delta < n && c >= tau);
+        if (hit) return base + __ffs(hit);  // delta = 0 .. first hit
+        carry += __shfl_sync(FULL_MASK, x, 31);
+    }
+    return n;
+}
+
+}  // namespace hkv

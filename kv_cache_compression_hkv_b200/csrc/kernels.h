@@ -1,0 +1,23 @@
+// kernels.h -- launchers of libhkv's kernels (host side, internal).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "hkv_internal.cuh"
+
+namespace hkv {
+
+size_t pack_smem_bytes(int P);
+cudaError_t launch_prefill(const Layout& L, int layer, const void* q, const void* k, const void* v,
+                           int P, int64_t block_stride, void* out, cudaStream_t st);
+cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void* k, const void* v,
+                          void* o, int append, int grid, cudaStream_t st);
+cudaError_t launch_append(const Layout& L, int layer, const void* k, const void* v, cudaStream_t st);
+cudaError_t launch_evict(const Layout& L, int l0, int l1, int grid, cudaStream_t st);
+cudaError_t launch_classify_rows(const float* rows, int n_rows, int n, int W, double tau,
+                                 int32_t* n_tau, uint8_t* label, cudaStream_t st);
+cudaError_t launch_select_batch(const float* score, const int32_t* pos, const int32_t* count,
+                                const int32_t* t, int n_probs, int n, int D, int k_near, int k_far,
+                                int stratified, uint8_t* evict, cudaStream_t st);
+
+}  // namespace hkv

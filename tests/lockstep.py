@@ -1,0 +1,125 @@
+"""Lock-step comparison of the CUDA path with the CPU oracle (test helper).
+
+The GPU runs the whole hot path (prefill + classification for every layer,
+then per step: fused append + decode attention for every layer and one STE
+call).  For sampled (sequence, layer) units the harness records the decode
+outputs, the labels and the kept sets after every eviction, then replays the
+unit through the oracle with those decisions as hints: the oracle adopts a
+GPU decision only where its own differs by a near-tie inside the stated band,
+and counts every other difference as a hard mismatch.
+
+Bands (derivation in the design doc): fp32 logits carry an absolute error of at
+most ~1e-4 on these inputs (sequential fp32 dot products of length <= 128),
+so softmax weights carry a relative error <= ~1e-4; labels compare
+sum-of-weights with tau (band 1e-3 absolute) and selections compare two
+scores (band 1e-3 relative).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import kv_cache_compression_hkv_b200 as hkv
+from kv_cache_compression_hkv_b200.inputs import generate_layer
+from oracle import hkv_oracle as O
+
+LABEL_BAND = 1e-3
+SELECT_BAND = 1e-3
+
+
+def oracle_params(w, mode=O.MODE_HEADKV, stratified=True) -> O.UnitParams:
+    return O.UnitParams(num_heads=w.num_heads, head_dim=w.head_dim, max_len=w.max_len,
+                        prefill_len=w.prefill_len, local_window=w.local_window, ste_m=w.ste_m,
+                        near_dist=w.near_dist, score_window=w.score_window, rho_num=w.rho[0],
+                        rho_den=w.rho[1], mode=mode, stratified=stratified,
+                        label_band=LABEL_BAND, select_band=SELECT_BAND)
+
+
+def generate(w, seed, device, num_seqs=None):
+    return [generate_layer(w, l, seed, device, num_seqs=num_seqs) for l in range(w.num_layers)]
+
+
+def run_gpu(w, cfg, data, units, fused=True, with_prefill_out=False):
+    """Runs the pipeline; returns the cache and, per sampled unit (s, l),
+    {"labels", "o" [steps, H, d], "events" [(t, {h: kept positions})]}."""
+    dev = data[0][0].device
+    S, H, P, L, d = cfg.num_seqs, cfg.num_heads, w.prefill_len, w.max_len, cfg.head_dim
+    cache = hkv.HeadKVCache(cfg, device=dev)
+    rec = {u: {"o": torch.empty(L - P, H, d, dtype=cfg.torch_dtype, device=dev), "events": []}
+           for u in units}
+    pre_out = []
+    for l, (q, k, v) in enumerate(data):
+        out = torch.empty(S, H, P, d, dtype=cfg.torch_dtype, device=dev) if with_prefill_out else None
+        cache.prefill_classify(l, q[:, :, :P], k[:, :, :P], v[:, :, :P], out=out)
+        pre_out.append(out)
+    layers = sorted({l for (_, l) in units})
+    prev = {}
+    for l in layers:
+        lab, _ = cache.labels(l)
+        ln, bd = cache.lens(l)
+        prev[l] = ln
+        for (s, ll) in units:
+            if ll != l:
+                continue
+            rec[(s, l)]["labels"] = lab[s].copy()
+            glob = [h for h in range(H) if lab[s, h] == 0]
+            if cfg.mode != hkv.MODE_FULL and glob and ln[s, glob[0]] < P:
+                rec[(s, l)]["events"].append((P - 1, {h: cache.kept(s, l, h) for h in glob}))
+    o_t = [torch.empty(S, H, d, dtype=cfg.torch_dtype, device=dev) for _ in data]
+    for t in range(P, L):
+        for l, (q, k, v) in enumerate(data):
+            qt, kt, vt = (x[:, :, t].contiguous() for x in (q, k, v))
+            if fused:
+                cache.decode_step(l, qt, kt, vt, o_t[l])
+            else:
+                cache.append(l, kt, vt)
+                cache.decode_attend(l, qt, o_t[l])
+        cache.ste_evict()
+        for (s, l) in units:
+            rec[(s, l)]["o"][t - P] = o_t[l][s]
+        for l in layers:
+            ln, _ = cache.lens(l)
+            for (s, ll) in units:
+                if ll != l:
+                    continue
+                lab = rec[(s, l)]["labels"]
+                glob = [h for h in range(H) if lab[h] == 0]
+                if glob and ln[s, glob[0]] < prev[l][s, glob[0]] + 1:
+                    rec[(s, l)]["events"].append((t, {h: cache.kept(s, l, h) for h in glob}))
+            prev[l] = ln
+    torch.cuda.synchronize()
+    return cache, rec, pre_out
+
+
+def compare_unit(w, data, unit, r, mode=O.MODE_HEADKV, stratified=True):
+    """Replays one unit through the oracle with the GPU's decisions as hints.
+    Returns (oracle result, max relative output error per decode call)."""
+    s, l = unit
+    q, k, v = (x[s].double().cpu().numpy() for x in data[l])
+    H = w.num_heads
+    prm = oracle_params(w, mode, stratified)
+    hints = None
+    if mode != O.MODE_FULL:
+        ev = r["events"]
+        width = max([max((len(x) for x in kept.values()), default=0) for _, kept in ev] + [1])
+        kept = np.full((max(len(ev), 1), H, width), -1, np.int32)
+        for e, (_, km) in enumerate(ev):
+            for h, pos in km.items():
+                kept[e, h, : len(pos)] = pos
+        hints = {"labels": r["labels"], "event_step": np.array([t for t, _ in ev], np.int32),
+                 "kept": kept[: len(ev)] if ev else None}
+        if not ev:
+            hints.pop("kept")
+    res = O.run_unit(prm, q, k, v, hints=hints)
+    got = r["o"].double().cpu().numpy()
+    ref = res.o_decode
+    err = np.abs(got - ref).max(axis=(1, 2)) / np.abs(ref).max(axis=(1, 2))
+    return res, err
+
+
+def assert_lockstep(res, err, tol, n_events_gpu):
+    st = res.stats
+    assert st["n_label_hard"] == 0, st
+    assert st["n_select_hard"] == 0, st
+    assert st["n_events"] == n_events_gpu, (st, n_events_gpu)
+    assert err.max() <= tol, f"max relative output error {err.max():.3e} > {tol}"

@@ -1,0 +1,74 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/hkv.h declares, and sizes/validates configs."""
+import ctypes as C
+import subprocess
+
+import pytest
+
+import kv_cache_compression_hkv_b200 as hkv
+from kv_cache_compression_hkv_b200 import build
+from kv_cache_compression_hkv_b200.inputs import WORKLOADS
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build.build()
+
+
+def test_exports_every_declared_symbol():
+    names = hkv.declared_symbols()
+    assert len(names) >= 15
+    L = hkv.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    out = subprocess.check_output(["nm", "-D", "--defined-only", hkv.LIB_PATH], text=True)
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert set(names) <= exported
+    # nothing but the C ABI is exported
+    assert all(s.startswith("hkv_") or s.startswith("_") for s in exported), exported - set(names)
+
+
+def test_status_strings():
+    L = hkv.lib()
+    for code, name in hkv._lib.STATUS.items():
+        assert L.hkv_status_string(code).decode() == name
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_pool_bytes_for_every_workload(name):
+    w = WORKLOADS[name]
+    for mode in (hkv.MODE_HEADKV, hkv.MODE_FULL):
+        n = hkv.pool_bytes(hkv.config_for(w, mode=mode))
+        kv = 2 * w.num_layers * w.num_seqs * w.head_dim * (2 if w.dtype == "bf16" else 4)
+        H, L = w.num_heads, w.max_len
+        T = H * L * w.rho[0] // w.rho[1]
+        slots = T + H * w.ste_m if mode == hkv.MODE_HEADKV else H * L
+        assert n >= kv * slots
+        assert n < kv * slots * 1.6 + (64 << 20)
+    assert hkv.pool_bytes(hkv.config_for(w)) < hkv.pool_bytes(hkv.config_for(w, mode=hkv.MODE_FULL))
+
+
+def test_config_validation():
+    base = hkv.config_for(WORKLOADS["llamagen_xl"])
+    bad = [dict(num_heads=0), dict(num_heads=33), dict(head_dim=96), dict(ste_m=31), dict(ste_m=0),
+           dict(score_window=0), dict(score_window=40), dict(rho_num=2, rho_den=1), dict(tau=0.0),
+           dict(tau=1.5), dict(mode=7), dict(stratified=2), dict(max_len=1), dict(max_len=9000),
+           dict(local_window=0), dict(rho_num=1, rho_den=64)]  # last: budget below H*W
+    for kw in bad:
+        cfg = hkv.Config(**{**base.__dict__, **kw})
+        with pytest.raises(hkv.HkvError) as e:
+            hkv.pool_bytes(cfg)
+        assert e.value.code == 1, kw
+
+
+def test_create_rejects_bad_pool_without_touching_the_device():
+    cfg = hkv.config_for(WORKLOADS["llamagen_1layer_f32"])
+    cc = cfg.c()
+    ctx = C.c_void_p()
+    L = hkv.lib()
+    assert L.hkv_create(C.byref(cc), None, 1 << 20, None, C.byref(ctx)) == 1   # null pool
+    assert L.hkv_create(C.byref(cc), 0x1001, 1 << 30, None, C.byref(ctx)) == 1  # misaligned
+    assert L.hkv_create(C.byref(cc), 0x100000, 16, None, C.byref(ctx)) == 3  # too small
+    assert L.hkv_prefill_classify(None, 0, None, None, None, 10, 640, None, None) == 1
+    assert L.hkv_ste_evict(None, 0, 1, None) == 1
+    assert L.hkv_ste_select_batch(None, None, None, None, 1, 8, 4, 1, 1, 1, None, None) == 1

@@ -1,0 +1,217 @@
+"""GPU parity of the CUDA path (through the C ABI) against the CPU oracle.
+
+Integer decisions (labels, kept sets, evicted sets) are compared bit-exactly
+(outside the near-tie bands of tests/lockstep.py); attention outputs within
+the tolerance of the arithmetic: max-abs relative error per decode call
+<= 2e-2 for bf16 caches and <= 1e-5 for fp32.
+"""
+import numpy as np
+import pytest
+import torch
+
+import kv_cache_compression_hkv_b200 as hkv
+from kv_cache_compression_hkv_b200.inputs import WORKLOADS
+from oracle import hkv_oracle as O
+
+from lockstep import assert_lockstep, compare_unit, generate, run_gpu
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+TOL = {"f32": 1e-5, "bf16": 2e-2}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from kv_cache_compression_hkv_b200 import build
+    build.build()
+    assert torch.cuda.is_available(), "these tests need a CUDA device"
+
+
+# ---------------------------------------------------------------------------
+# standalone primitives: identical inputs on both sides, bit-exact answers
+# ---------------------------------------------------------------------------
+
+def test_classify_rows_bitexact():
+    g = np.random.default_rng(0)
+    rows, Ws = [], []
+    for i in range(600):
+        n = int(g.integers(2, 700))
+        a = float(g.choice([0.02, 0.2, 1.0, 5.0]))
+        x = g.dirichlet(np.full(n, a))
+        if i % 5 == 0:
+            x = np.zeros(n); x[-1 - int(g.integers(0, n))] = 1.0
+        rows.append(x.astype(np.float32)); Ws.append(int(g.integers(1, 60)))
+    for W in (1, 20, 28, 56):
+        for n in (65, 97, 384):
+            N = 13 if n == 65 else n
+            rows.append(np.full(n, 1.0 / N, np.float32) * (np.arange(n) >= n - N)); Ws.append(W)
+    n_max = max(r.size for r in rows)
+    for W in sorted(set(Ws)):
+        sel = [r for r, w in zip(rows, Ws) if w == W]
+        for n in sorted({r.size for r in sel}):
+            batch = np.stack([r for r in sel if r.size == n])
+            nt, lab = hkv.classify_rows(torch.tensor(batch, device=DEV), W)
+            nt, lab = nt.cpu().numpy(), lab.cpu().numpy()
+            for i, row in enumerate(batch):
+                e_nt, e_lab, _ = O.classify(row.astype(np.float64), W, 0.9)
+                assert (nt[i], lab[i]) == (e_nt, e_lab), (n, W, i)
+    assert n_max < 1000
+
+
+@pytest.mark.parametrize("n,stratified", [(40, True), (230, True), (834, True), (2480, True),
+                                          (230, False), (33, True), (1, True)])
+def test_select_batch_bitexact(n, stratified):
+    g = np.random.default_rng(n)
+    P = 96
+    score = np.zeros((P, n), np.float32)
+    pos = np.zeros((P, n), np.int32)
+    count = np.zeros(P, np.int32)
+    tt = np.zeros(P, np.int32)
+    for i in range(P):
+        m = n if i % 3 else int(g.integers(1, n + 1))
+        t = int(g.integers(m - 1, 3 * n + 5))
+        p = np.sort(g.choice(np.arange(t), size=m - 1, replace=False)) if m > 1 else np.zeros(0, int)
+        p = np.concatenate([p, [t]])
+        g.shuffle(p)
+        if i % 4 == 0:     # heavy ties
+            s = g.choice([0.0, 0.125, 0.25, 1.0], size=m)
+        elif i % 4 == 1:   # tiny and denormal-free spread
+            s = g.random(m) ** 8
+        else:
+            s = g.random(m)
+        score[i, :m] = s; pos[i, :m] = p; count[i] = m; tt[i] = t
+    D, kn, kf = 48, 16, 16
+    ev = hkv.ste_select_batch(*(torch.tensor(a, device=DEV) for a in (score, pos, count, tt)),
+                              D=D, k_near=kn, k_far=kf, stratified=stratified).cpu().numpy()
+    for i in range(P):
+        m = count[i]
+        e, _, _ = O.ste_select(score[i, :m].astype(np.float64), pos[i, :m], int(tt[i]), D, kn, kf,
+                               stratified)
+        np.testing.assert_array_equal(ev[i, :m].astype(bool), e, err_msg=f"problem {i}")
+        assert not ev[i, m:].any()
+
+
+# ---------------------------------------------------------------------------
+# whole hot path, lock-step with the oracle
+# ---------------------------------------------------------------------------
+
+def _lockstep(w, units, seed=0, fused=True, mode=hkv.MODE_HEADKV, stratified=True):
+    cfg = hkv.config_for(w, mode=mode, stratified=stratified)
+    data = generate(w, seed, DEV)
+    cache, rec, _ = run_gpu(w, cfg, data, units, fused=fused)
+    rc, detail = cache.check()
+    assert rc == 0, (rc, detail)
+    omode = {hkv.MODE_HEADKV: O.MODE_HEADKV, hkv.MODE_FULL: O.MODE_FULL,
+             hkv.MODE_UNIFORM: O.MODE_UNIFORM}[mode]
+    stats = []
+    for u in units:
+        res, err = compare_unit(w, data, u, rec[u], omode, stratified)
+        assert_lockstep(res, err, TOL[w.dtype], len(rec[u]["events"]))
+        if mode == hkv.MODE_HEADKV:
+            np.testing.assert_array_equal(res.labels, rec[u]["labels"])
+        stats.append(res.stats)
+    return stats
+
+
+def test_llamagen_1layer_f32_full_config():
+    w = WORKLOADS["llamagen_1layer_f32"]
+    stats = _lockstep(w, [(0, 0)])
+    assert stats[0]["n_events"] >= 1 and stats[0]["n_select"] > 0
+
+
+@pytest.mark.parametrize("name", ["llamagen_xl", "janus_pro_1b", "janus_pro_7b_rho6",
+                                  "janus_pro_7b_rho8", "lumina_mgpt_768"])
+def test_lockstep_scaled_stacks(name):
+    """Every shape of the stacks, full sequence length, few sequences/layers."""
+    w = WORKLOADS[name]
+    w = w.scaled(num_seqs=3 if w.max_len < 1000 else 2, num_layers=2)
+    units = [(s, l) for s in range(w.num_seqs) for l in range(w.num_layers)]
+    if w.max_len > 1000:
+        units = units[:2]
+    _lockstep(w, units, seed=11)
+
+
+def test_unfused_append_attend_matches_oracle():
+    w = WORKLOADS["janus_pro_1b"].scaled(num_seqs=2, num_layers=1)
+    _lockstep(w, [(0, 0), (1, 0)], seed=5, fused=False)
+
+
+def test_full_cache_mode_matches_oracle():
+    w = WORKLOADS["janus_pro_7b_rho4"].scaled(num_seqs=2, num_layers=1)
+    _lockstep(w, [(0, 0), (1, 0)], seed=6, mode=hkv.MODE_FULL)
+
+
+def test_unstratified_and_uniform_variants():
+    w = WORKLOADS["llamagen_xl"].scaled(num_seqs=2, num_layers=1)
+    _lockstep(w, [(0, 0), (1, 0)], seed=7, stratified=False)
+    _lockstep(w, [(0, 0)], seed=8, mode=hkv.MODE_UNIFORM)
+
+
+def test_prefill_outputs_match_oracle():
+    w = WORKLOADS["janus_pro_7b_rho6"].scaled(num_seqs=2, num_layers=1)
+    cfg = hkv.config_for(w)
+    data = generate(w, 3, DEV)
+    _, _, pre = run_gpu(w.scaled(image_tokens=w.prefill_image + 1), cfg, data, [], with_prefill_out=True)
+    q, k, v = data[0]
+    P = w.prefill_len
+    for s in range(2):
+        for h in range(0, w.num_heads, 7):
+            o, _ = O.causal_attention(q[s, h, :P].double().cpu().numpy(),
+                                      k[s, h, :P].double().cpu().numpy(),
+                                      v[s, h, :P].double().cpu().numpy())
+            got = pre[0][s, h].double().cpu().numpy()
+            assert np.abs(got - o).max() / np.abs(o).max() < 2e-2
+
+
+def test_full_size_sampled_units():
+    """The bench's workload at full size and launch configuration; two
+    sampled units go through the oracle in lock step."""
+    w = WORKLOADS["llamagen_xl"]
+    units = [(5, 0), (62, 35)]
+    _lockstep(w, units, seed=2024)
+
+
+# ---------------------------------------------------------------------------
+# errors: argument checks, call order, device-side status
+# ---------------------------------------------------------------------------
+
+def test_call_order_and_arguments():
+    w = WORKLOADS["llamagen_1layer_f32"]
+    cfg = hkv.config_for(w)
+    cache = hkv.HeadKVCache(cfg, device=DEV)
+    x = torch.zeros(1, 20, 64, device=DEV)
+    with pytest.raises(hkv.HkvError) as e:
+        cache.decode_step(0, x, x, x, x.clone())
+    assert e.value.code == 2  # STATE: not classified
+    with pytest.raises(hkv.HkvError) as e:
+        cache.ste_evict(0, 2)
+    assert e.value.code == 1
+    q = torch.randn(1, 20, 300, 64, device=DEV)
+    with pytest.raises(hkv.HkvError) as e:  # prefill longer than max_len
+        cache.prefill_classify(0, q[:, :, :257], q[:, :, :257], q[:, :, :257])
+    assert e.value.code == 1
+    cache.prefill_classify(0, q[:, :, :65], q[:, :, :65], q[:, :, :65])
+    with pytest.raises(hkv.HkvError) as e:
+        cache.prefill_classify(0, q[:, :, :65], q[:, :, :65], q[:, :, :65])
+    assert e.value.code == 2
+    for t in range(65, 257):
+        cache.decode_step(0, x, x, x, x.clone())
+        cache.ste_evict()
+    with pytest.raises(hkv.HkvError) as e:  # beyond max_len
+        cache.decode_step(0, x, x, x, x.clone())
+    assert e.value.code == 3
+    assert cache.check()[0] == 0
+
+
+def test_nan_input_latches_numeric_status():
+    w = WORKLOADS["llamagen_1layer_f32"]
+    cache = hkv.HeadKVCache(hkv.config_for(w), device=DEV)
+    q = torch.randn(1, 20, 65, 64, device=DEV)
+    cache.prefill_classify(0, q, q, q)
+    x = torch.randn(1, 20, 64, device=DEV)
+    bad = x.clone(); bad[0, 3, 5] = float("nan")
+    cache.decode_step(0, bad, x, x, x.clone())
+    rc, detail = cache.check()
+    assert rc == 4 and detail % 20 == 3
+    cache.clear_error()
+    assert cache.check()[0] == 0
