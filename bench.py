@@ -1,0 +1,484 @@
+#!/usr/bin/env python
+"""Benchmark of the HeadKV hot path on B200 (one JSON line on rank 0).
+
+One step = one pass of the whole hot path over one batch: reset, prefill +
+head grouping + compression for every layer, then every decode step
+(fused append + decode attention per layer, one STE call), replayed as one
+CUDA graph with the inputs resident in HBM.  value = decode image tokens/s
+over the whole pass (prefill time included).  Inputs are far larger than L2
+(the cache and the per-step inputs of all layers rotate through HBM).
+
+  python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own batch of
+the workload (weak scaling, no data-path collective); the time is the max
+over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "compressed decode image tokens/s and step µs; achieved HBM GB/s vs B200 peak"
+UNIT = "image tokens/s"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llamagen_xl")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-full", action="store_true", help="skip the full-cache comparator")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end arm")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the reported CPU baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(w, seed, seconds, threads=None):
+    """Runs whole (sequence, layer) units of the workload through the CPU
+    oracle on host threads for about `seconds`; returns (image tokens/s,
+    threads, units done)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    from kv_cache_compression_hkv_b200.inputs import generate_layer
+    from oracle import hkv_oracle as O
+
+    threads = threads or os.cpu_count() or 1
+    prm = O.UnitParams(num_heads=w.num_heads, head_dim=w.head_dim, max_len=w.max_len,
+                       prefill_len=w.prefill_len, local_window=w.local_window, ste_m=w.ste_m,
+                       near_dist=w.near_dist, score_window=w.score_window, rho_num=w.rho[0],
+                       rho_den=w.rho[1])
+    q, k, v = generate_layer(w, 0, seed, "cpu", num_seqs=min(w.num_seqs, threads))
+    units = [tuple(x[s].double().numpy() for x in (q, k, v)) for s in range(q.shape[0])]
+    O.build()
+    done = [0]
+    deadline = time.perf_counter() + seconds
+    lock = threading.Lock()
+
+    def worker(i):
+        n = 0
+        while True:
+            O.run_unit(prm, *units[i % len(units)], want_decode=True)
+            n += 1
+            if time.perf_counter() > deadline:
+                break
+        with lock:
+            done[0] += n
+
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(worker, range(threads)))
+    el = time.perf_counter() - t0
+    tokens_per_unit = w.images * w.decode_steps / (w.num_seqs * w.num_layers)
+    return done[0] * tokens_per_unit / el, threads, done[0], el
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+def gpu_id(dev) -> str:
+    """nvidia-smi id of a torch device (its UUID; indices may be remapped)."""
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev.index or 0)
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: str):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = [r.split(",") for r in (self.out or "").strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i]
+                          and "Not" not in r[5 + i]})
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+
+class Inputs:
+    """Per-layer prefill blocks [S, H, P, d] and per-step decode inputs
+    [steps, S, H, d], all resident in HBM."""
+
+    def __init__(self, w, seed, dev):
+        from kv_cache_compression_hkv_b200.inputs import generate_layer
+        P = w.prefill_len
+        self.pre, self.dec = [], []
+        for l in range(w.num_layers):
+            q, k, v = generate_layer(w, l, seed, dev)
+            self.pre.append(tuple(x[:, :, :P].contiguous() for x in (q, k, v)))
+            self.dec.append(tuple(x[:, :, P:].permute(2, 0, 1, 3).contiguous() for x in (q, k, v)))
+            del q, k, v
+        torch.cuda.synchronize()
+
+    def nbytes(self):
+        return sum(x.numel() * x.element_size() for t in self.pre + self.dec for x in t)
+
+
+def run_pass(cache, w, inp, outs, evict=True, pre_out=None, hooks=None):
+    """Enqueues one whole pass on the current stream (eagerly or under capture)."""
+    cache.reset()
+    for l in range(w.num_layers):
+        q, k, v = inp.pre[l]
+        cache.prefill_classify(l, q, k, v, out=None if pre_out is None else pre_out[l])
+    if hooks:
+        hooks("decode_begin", None, None)
+    for t in range(w.decode_steps):
+        for l in range(w.num_layers):
+            q, k, v = inp.dec[l]
+            if hooks:
+                hooks("pre_decode", t, l)
+            cache.decode_step(l, q[t], k[t], v[t], outs[l])
+            if hooks:
+                hooks("post_decode", t, l)
+        if evict:
+            if hooks:
+                hooks("pre_evict", t, None)
+            cache.ste_evict()
+            if hooks:
+                hooks("post_evict", t, None)
+    if hooks:
+        hooks("decode_end", None, None)
+
+
+def capture(fn):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def decode_tokens_per_launch(cache, w, inp, outs):
+    """Eager pass that reads back every layer's cache lengths right after its
+    decode launches: kv tokens each decode launch reads, [steps, layers]."""
+    S, H = w.num_seqs, w.num_heads
+    tok = np.zeros((w.decode_steps, w.num_layers), np.int64)
+    cache.reset()
+    for l in range(w.num_layers):
+        cache.prefill_classify(l, *inp.pre[l])
+    for t in range(w.decode_steps):
+        for l in range(w.num_layers):
+            q, k, v = inp.dec[l]
+            cache.decode_step(l, q[t], k[t], v[t], outs[l])
+        for l in range(w.num_layers):
+            ln, _ = cache.lens(l)
+            tok[t, l] = int(ln.sum())
+        cache.ste_evict()
+    torch.cuda.synchronize()
+    return tok
+
+
+def timed_replays(g, n):
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(s)
+    for _ in range(n):
+        g.replay()
+    e1.record(s)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / n  # ms per replay
+
+
+def gpu_arm(args, rank, world, dev):
+    import kv_cache_compression_hkv_b200 as hkv
+    from kv_cache_compression_hkv_b200.inputs import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    S, H, d, Ly = w.num_seqs, w.num_heads, w.head_dim, w.num_layers
+    es = 2 if w.dtype == "bf16" else 4
+    steps = w.decode_steps
+    inp = Inputs(w, args.seed + 1000 * rank, dev)
+    outs = [torch.empty(S, H, d, dtype=w.torch_dtype, device=dev) for _ in range(Ly)]
+    pre_out = [torch.empty(S, H, w.prefill_len, d, dtype=w.torch_dtype, device=dev) for _ in range(Ly)]
+    cfg = hkv.config_for(w)
+    cache = hkv.HeadKVCache(cfg, device=dev)
+
+    # one eager pass: warms every kernel and yields the bytes each decode launch reads
+    tokens = decode_tokens_per_launch(cache, w, inp, outs)
+    labels = np.stack([cache.labels(l)[0] for l in range(Ly)])
+    rc, detail = cache.check()
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} ({detail}) after the eager pass")
+
+    # main graph: the whole pass
+    ev_dec = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+
+    def hooks_main(what, t, l):
+        if what == "decode_begin":
+            ev_dec[0].record()
+        elif what == "decode_end":
+            ev_dec[1].record()
+
+    g_main = capture(lambda: run_pass(cache, w, inp, outs, pre_out=pre_out, hooks=hooks_main))
+    for _ in range(args.warmup):
+        g_main.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_id(dev)) as clk:
+        ms = timed_replays(g_main, args.steps)
+        decode_ms = ev_dec[0].elapsed_time(ev_dec[1])
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        torch.distributed.barrier()
+        ms = float(t.item())
+    rc, detail = cache.check()
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} ({detail}) after the timed passes")
+
+    # per-launch durations (same stream as the kernels: the capture stream)
+    n_ev = steps * (Ly + 1)
+    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * n_ev)]
+    slot = {}
+
+    def hooks_prof(what, t, l):
+        if what in ("pre_decode", "post_decode"):
+            i = t * (Ly + 1) + l
+        elif what in ("pre_evict", "post_evict"):
+            i = t * (Ly + 1) + Ly
+        else:
+            return
+        evs[2 * i + (0 if what.startswith("pre") else 1)].record()
+        slot[i] = True
+
+    g_prof = capture(lambda: run_pass(cache, w, inp, outs, pre_out=pre_out, hooks=hooks_prof))
+    g_prof.replay()
+    torch.cuda.synchronize()
+    dur = np.array([evs[2 * i].elapsed_time(evs[2 * i + 1]) for i in range(n_ev)]).reshape(steps, Ly + 1)
+    dec_us = dur[:, :Ly] * 1e3
+    evict_us = dur[:, Ly] * 1e3
+    kv_bytes = tokens * 2 * d * es                      # kept K + V read (new token included)
+    io_bytes = S * H * d * es * 4                        # q read, o written, new k/v row stored
+    alg = kv_bytes + io_bytes
+    achieved = float(alg.sum() / (dec_us.sum() * 1e-6) / 1e9)
+    del g_prof
+
+    peaks = {}
+    pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pk):
+        peaks = json.load(open(pk))
+    peak = peaks.get("hbm_gbs", 6650.0)
+    peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
+
+    res = {
+        "ms_per_step": ms,
+        "decode_step_us": decode_ms * 1e3 / steps,
+        "prefill_ms": ms - decode_ms,
+        "tokens_per_s": w.images * steps / (ms * 1e-3) * world,
+        "clocks": clk.summary(),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "kernel": "decode_kernel (fused append + split-K decode attention)",
+                     "peak_source": peak_src,
+                     "bytes_per_launch_avg": float(alg.mean()),
+                     "launch_us_avg": float(dec_us.mean())},
+        "evict_us_avg": float(evict_us.mean()),
+        "evict_us_max": float(evict_us.max()),
+        "labels_local_frac": float((labels == 1).mean()),
+        "gpu_launches": args.steps * (3 * Ly + steps * (Ly + 1)),
+        "kv_pool_bytes": cache.nbytes,
+    }
+    del g_main
+
+    # full-cache comparator (same kernels, no compression)
+    if not args.no_full:
+        cache_f = hkv.HeadKVCache(hkv.config_for(w, mode=hkv.MODE_FULL), device=dev)
+        g_full = capture(lambda: run_pass(cache_f, w, inp, outs, evict=False, pre_out=pre_out,
+                                          hooks=hooks_main))
+        for _ in range(2):
+            g_full.replay()
+        ms_f = timed_replays(g_full, max(1, min(args.steps, 3)))
+        dec_f = ev_dec[0].elapsed_time(ev_dec[1])
+        res["full"] = {"ms_per_step": ms_f, "decode_step_us": dec_f * 1e3 / steps,
+                       "kv_pool_bytes": cache_f.nbytes}
+        res["speedup_decode_vs_full"] = dec_f / decode_ms
+        res["speedup_pass_vs_full"] = ms_f / ms
+        del g_full, cache_f
+        torch.cuda.empty_cache()
+
+    # end to end through the C ABI from pinned host buffers
+    if not args.no_e2e:
+        res["e2e"] = e2e_arm(args, w, cache, inp, dev, world)
+    return res
+
+
+def e2e_arm(args, w, cache, inp, dev, world):
+    """Same pass with every input copied from pinned host memory inside the
+    timed region and every decode output copied back."""
+    S, H, d, Ly, steps = w.num_seqs, w.num_heads, w.head_dim, w.num_layers, w.decode_steps
+    host_pre = [tuple(torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in t) for t in inp.pre]
+    for hp, dp in zip(host_pre, inp.pre):
+        for hx, dx in zip(hp, dp):
+            hx.copy_(dx)
+    # one contiguous block per step: [steps][Ly][q, k, v][S][H][d]
+    host_dec = torch.empty(steps, Ly, 3, S, H, d, dtype=w.torch_dtype).pin_memory()
+    for l in range(Ly):
+        for j in range(3):
+            host_dec[:, l, j].copy_(inp.dec[l][j])
+    host_out = torch.empty(steps, Ly, S, H, d, dtype=w.torch_dtype).pin_memory()
+    dev_pre = [tuple(torch.empty_like(x) for x in t) for t in inp.pre]
+    stage = [torch.empty(Ly, 3, S, H, d, dtype=w.torch_dtype, device=dev) for _ in range(2)]
+    outs = torch.empty(Ly, S, H, d, dtype=w.torch_dtype, device=dev)
+
+    def body():
+        cache.reset()
+        for l in range(Ly):
+            for hx, dx in zip(host_pre[l], dev_pre[l]):
+                dx.copy_(hx, non_blocking=True)
+            cache.prefill_classify(l, *dev_pre[l])
+        for t in range(steps):
+            st = stage[t & 1]
+            st.copy_(host_dec[t], non_blocking=True)
+            for l in range(Ly):
+                cache.decode_step(l, st[l, 0], st[l, 1], st[l, 2], outs[l])
+            cache.ste_evict()
+            host_out[t].copy_(outs, non_blocking=True)
+
+    g = capture(body)
+    for _ in range(2):
+        g.replay()
+    ms = timed_replays(g, max(1, min(args.steps, 3)))
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    h2d = sum(x.numel() * x.element_size() for t in host_pre for x in t) + \
+        host_dec.numel() * host_dec.element_size()
+    d2h = host_out.numel() * host_out.element_size()
+    del g
+    return {"value": w.images * steps / (ms * 1e-3) * world, "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from kv_cache_compression_hkv_b200.inputs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    config = {"workload": w.name, "num_seqs": w.num_seqs, "images": w.images,
+              "num_layers": w.num_layers, "num_heads": w.num_heads, "head_dim": w.head_dim,
+              "max_len": w.max_len, "prefill_len": w.prefill_len, "decode_steps": w.decode_steps,
+              "rho": f"{w.rho[0]}/{w.rho[1]}", "local_window": w.local_window, "ste_m": w.ste_m,
+              "near_dist": w.near_dist, "l2": "inputs and cache larger than L2 (no flush needed)"}
+
+    if args.impl == "reference":
+        # the reference arm is the CPU oracle, on rank 0 only
+        if rank != 0:
+            return
+        vals = []
+        cores = 0
+        per = max(2.0, min(args.cpu_seconds, 20.0))
+        for i in range(args.warmup + args.steps):
+            v, cores, n, el = oracle_sample(w, args.seed, per if i >= args.warmup else 1.0)
+            if i >= args.warmup:
+                vals.append(v)
+        val = float(np.mean(vals))
+        sample = f"whole (sequence, layer) units of {w.name} through the oracle, ~{per:.0f} s per step"
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config,
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+        return
+
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    res = gpu_arm(args, rank, world, dev)
+    cpu = None
+    if rank == 0 and world == 1:
+        v, cores, n, el = oracle_sample(w, args.seed, args.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{n} whole (sequence, layer) units of {w.name} in {el:.1f} s "
+                         f"(one unit = 1/{w.num_seqs * w.num_layers} of a pass)"}
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": res["tokens_per_s"], "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic (seeded planted-attention Q/K/V, shapes of the workload)",
+            "config": config,
+            "decode_step_us": res["decode_step_us"], "prefill_ms": res["prefill_ms"],
+            "roofline": res["roofline"], "evict_us_avg": res["evict_us_avg"],
+            "evict_us_max": res["evict_us_max"],
+            "cpu_baseline": cpu, "e2e": res.get("e2e"), "gpu_launches": res["gpu_launches"],
+            "clocks": res["clocks"], "full": res.get("full"),
+            "speedup_decode_vs_full": res.get("speedup_decode_vs_full"),
+            "speedup_pass_vs_full": res.get("speedup_pass_vs_full"),
+            "kv_pool_bytes": res["kv_pool_bytes"], "labels_local_frac": res["labels_local_frac"],
+        }
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -173,6 +173,12 @@ HKV_API hkv_status hkv_check(hkv_ctx* ctx, int32_t* detail_host, void* stream);
 /* Clears a latched device error. */
 HKV_API hkv_status hkv_clear_error(hkv_ctx* ctx, void* stream);
 
+/* Starts a new generation on the same pool: enqueues the clearing of the
+ * control words (positions, counters, status) on `stream` and forgets every
+ * layer's classification, so prefill_classify must run again per layer.
+ * Cache contents are not cleared (they are rewritten by the next prefill). */
+HKV_API hkv_status hkv_reset(hkv_ctx* ctx, void* stream);
+
 /* Releases the context (not the pool). */
 HKV_API void hkv_destroy(hkv_ctx* ctx);
 

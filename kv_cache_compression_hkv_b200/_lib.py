@@ -64,6 +64,7 @@ def lib():
             "hkv_get_kept": [P, I, I, I, P, I, P, P],
             "hkv_check": [P, P, P],
             "hkv_clear_error": [P, P],
+            "hkv_reset": [P, P],
             "hkv_classify_rows": [P, I, I, I, D, P, P, P],
             "hkv_ste_select_batch": [P, P, P, P, I, I, I, I, I, I, P, P],
         }
@@ -162,6 +163,11 @@ class HeadKVCache:
             self.close()
         except Exception:
             pass
+
+    def reset(self, stream=None):
+        """Starts a new generation on the same pool (every layer must be
+        prefilled and classified again)."""
+        _check(lib().hkv_reset(self.ctx, _stream(stream)), "hkv_reset")
 
     # -- argument checks (shapes, dtypes, devices) ---------------------------
     def _tensor(self, x: torch.Tensor, name: str):

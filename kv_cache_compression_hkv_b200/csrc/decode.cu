@@ -332,11 +332,6 @@ template <typename T, int DPL>
 static cudaError_t launch_decode_t(const Layout& L, int layer, const void* q, const void* k,
                                    const void* v, void* o, int append, int grid, cudaStream_t st) {
     const size_t sm = (size_t)L.S * L.H * sizeof(int32_t);
-    if (sm > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, DPL>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        if (e != cudaSuccess) return e;
-    }
     decode_kernel<T, DPL><<<grid, 256, sm, st>>>(L, layer, (const T*)q, (const T*)k, (const T*)v,
                                                  (T*)o, append);
     return cudaGetLastError();
@@ -365,6 +360,14 @@ cudaError_t launch_append(const Layout& L, int layer, const void* k, const void*
         else append_kernel<float, 4><<<grid, 256, 0, st>>>(L, layer, (const float*)k, (const float*)v);
     }
     return cudaGetLastError();
+}
+
+cudaError_t prepare_decode(int smem) {
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<__nv_bfloat16, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(decode_kernel<__nv_bfloat16, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(decode_kernel<float, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(decode_kernel<float, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    return e;
 }
 
 }  // namespace hkv

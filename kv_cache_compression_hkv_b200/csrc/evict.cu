@@ -184,17 +184,18 @@ cudaError_t launch_evict(const Layout& L, int l0, int l1, int grid, cudaStream_t
     const int n_max = L.L;
     const int nw = evict_warps(n_max);
     const size_t sm = (size_t)nw * select_scratch_bytes(n_max);
-    cudaError_t e;
-    if (L.dtype == HKV_DTYPE_BF16) {
-        e = cudaFuncSetAttribute(evict_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        if (e != cudaSuccess) return e;
+    if (L.dtype == HKV_DTYPE_BF16)
         evict_kernel<__nv_bfloat16><<<grid, 32 * nw, sm, st>>>(L, l0, l1, n_max);
-    } else {
-        e = cudaFuncSetAttribute(evict_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        if (e != cudaSuccess) return e;
+    else
         evict_kernel<float><<<grid, 32 * nw, sm, st>>>(L, l0, l1, n_max);
-    }
     return cudaGetLastError();
+}
+
+cudaError_t prepare_evict(int smem) {
+    cudaError_t e = cudaFuncSetAttribute(evict_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(evict_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(select_batch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    return e;
 }
 
 cudaError_t launch_classify_rows(const float* rows, int n_rows, int n, int W, double tau,
@@ -209,11 +210,26 @@ cudaError_t launch_select_batch(const float* score, const int32_t* pos, const in
                                 int stratified, uint8_t* evict, cudaStream_t st) {
     const int nw = 4;
     const size_t sm = (size_t)nw * select_scratch_bytes(n);
-    cudaError_t e = cudaFuncSetAttribute(select_batch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    cudaError_t e = prepare_kernels();
     if (e != cudaSuccess) return e;
     select_batch_kernel<<<(n_probs + nw - 1) / nw, 32 * nw, sm, st>>>(
         score, pos, count, t, n_probs, n, D, k_near, k_far, stratified, evict);
     return cudaGetLastError();
+}
+
+cudaError_t prepare_kernels() {
+    // Every kernel may use up to the device's opt-in shared memory; set once
+    // per process (a host-side attribute call, kept out of stream captures).
+    static cudaError_t done = cudaErrorNotReady;
+    if (done == cudaSuccess) return done;
+    int dev = 0, optin = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e == cudaSuccess) e = prepare_prefill(optin);
+    if (e == cudaSuccess) e = prepare_decode(optin);
+    if (e == cudaSuccess) e = prepare_evict(optin);
+    done = e;
+    return e;
 }
 
 }  // namespace hkv

@@ -175,6 +175,10 @@ hkv_status hkv_create(const hkv_config* cfg, void* pool, size_t bytes, void* str
         delete c;
         return HKV_ERR_CUDA;
     }
+    if (hkv::prepare_kernels() != cudaSuccess) {
+        delete c;
+        return HKV_ERR_CUDA;
+    }
     c->decode_grid = c->n_sm;      // one 256-thread block per SM (register-bound)
     c->evict_grid = c->n_sm * 2;
     *out = c;
@@ -337,6 +341,18 @@ hkv_status hkv_check(hkv_ctx* c, int32_t* detail_host, void* stream) {
 hkv_status hkv_clear_error(hkv_ctx* c, void* stream) {
     if (!c) return HKV_ERR_INVALID_ARG;
     return cuda_status(cudaMemsetAsync(c->lay.status, 0, 8, (cudaStream_t)stream));
+}
+
+hkv_status hkv_reset(hkv_ctx* c, void* stream) {
+    if (!c) return HKV_ERR_INVALID_ARG;
+    cudaError_t e = cudaMemsetAsync(c->lay.status, 0, ctrl_bytes(&c->cfg), (cudaStream_t)stream);
+    if (e != cudaSuccess) return HKV_ERR_CUDA;
+    for (int l = 0; l < c->cfg.num_layers; ++l) {
+        c->classified[l] = 0;
+        c->t_host[l] = 0;
+        c->prefill_len[l] = 0;
+    }
+    return HKV_OK;
 }
 
 void hkv_destroy(hkv_ctx* c) { delete c; }

@@ -7,6 +7,12 @@
 
 namespace hkv {
 
+// Raises the dynamic shared-memory limits the kernels of this layout need
+// (a host call that must not run inside a stream capture; hkv_create makes it).
+cudaError_t prepare_kernels();
+cudaError_t prepare_prefill(int smem);
+cudaError_t prepare_decode(int smem);
+cudaError_t prepare_evict(int smem);
 size_t pack_smem_bytes(int P);
 cudaError_t launch_prefill(const Layout& L, int layer, const void* q, const void* k, const void* v,
                            int P, int64_t block_stride, void* out, cudaStream_t st);

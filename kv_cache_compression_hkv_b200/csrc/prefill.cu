@@ -228,12 +228,6 @@ cudaError_t launch_prefill(const Layout& L, int layer, const void* q, const void
     const int nb = L.S * L.H;
     dim3 grid(nb, (P + 3) / 4);
     size_t sm = (size_t)4 * (L.d + P) * sizeof(float);
-    if (sm > 48 * 1024) {
-        cudaError_t e = L.dtype == HKV_DTYPE_F32
-            ? cudaFuncSetAttribute(prefill_attn_simt<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)
-            : cudaFuncSetAttribute(prefill_attn_simt<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        if (e != cudaSuccess) return e;
-    }
     if (L.dtype == HKV_DTYPE_F32)
         prefill_attn_simt<float><<<grid, 128, sm, st>>>(
             (const float*)q, (const float*)k, (const float*)v, P, L.d, block_stride, L.r,
@@ -248,18 +242,21 @@ cudaError_t launch_prefill(const Layout& L, int layer, const void* q, const void
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     size_t psm = pack_smem_bytes(P);
-    if (L.dtype == HKV_DTYPE_F32) {
-        if (psm > 48 * 1024)
-            cudaFuncSetAttribute(pack_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm);
+    if (L.dtype == HKV_DTYPE_F32)
         pack_kernel<float><<<nb, 128, psm, st>>>(L, layer, (const float*)k, (const float*)v, P,
                                                   block_stride);
-    } else {
-        if (psm > 48 * 1024)
-            cudaFuncSetAttribute(pack_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm);
+    else
         pack_kernel<__nv_bfloat16><<<nb, 128, psm, st>>>(
             L, layer, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, P, block_stride);
-    }
     return cudaGetLastError();
+}
+
+cudaError_t prepare_prefill(int smem) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_attn_simt<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(pack_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_attn_simt<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(pack_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    return e;
 }
 
 }  // namespace hkv
