@@ -192,9 +192,9 @@ cudaError_t launch_evict(const Layout& L, int l0, int l1, int grid, cudaStream_t
 }
 
 cudaError_t prepare_evict(int smem) {
-    cudaError_t e = cudaFuncSetAttribute(evict_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(evict_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(select_batch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = allow_max_dynamic_smem(evict_kernel<__nv_bfloat16>, smem);
+    if (e == cudaSuccess) e = allow_max_dynamic_smem(evict_kernel<float>, smem);
+    if (e == cudaSuccess) e = allow_max_dynamic_smem(select_batch_kernel, smem);
     return e;
 }
 

@@ -295,4 +295,15 @@ __device__ __forceinline__ int warp_tokens_to_tau(const float* row, int n, doubl
     return n;
 }
 
+// Allows `func` as much dynamic shared memory as the device's opt-in limit
+// leaves next to its static shared memory.
+template <typename F>
+inline cudaError_t allow_max_dynamic_smem(F* func, int optin) {
+    cudaFuncAttributes a;
+    cudaError_t e = cudaFuncGetAttributes(&a, func);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                optin - (int)a.sharedSizeBytes);
+}
+
 }  // namespace hkv

@@ -252,10 +252,10 @@ cudaError_t launch_prefill(const Layout& L, int layer, const void* q, const void
 }
 
 cudaError_t prepare_prefill(int smem) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_attn_simt<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(pack_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_attn_simt<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(pack_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = allow_max_dynamic_smem(prefill_attn_simt<float>, smem);
+    if (e == cudaSuccess) e = allow_max_dynamic_smem(pack_kernel<float>, smem);
+    if (e == cudaSuccess) e = allow_max_dynamic_smem(prefill_attn_simt<__nv_bfloat16>, smem);
+    if (e == cudaSuccess) e = allow_max_dynamic_smem(pack_kernel<__nv_bfloat16>, smem);
     return e;
 }
 
