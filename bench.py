@@ -244,7 +244,8 @@ def gpu_arm(args, rank, world, dev):
     S, H, d, Ly = w.num_seqs, w.num_heads, w.head_dim, w.num_layers
     es = 2 if w.dtype == "bf16" else 4
     steps = w.decode_steps
-    inp = Inputs(w, args.seed + 1000 * rank, dev)
+    from kv_cache_compression_hkv_b200 import dist
+    inp = Inputs(w, dist.rank_seed(args.seed, rank), dev)
     outs = [torch.empty(S, H, d, dtype=w.torch_dtype, device=dev) for _ in range(Ly)]
     pre_out = [torch.empty(S, H, w.prefill_len, d, dtype=w.torch_dtype, device=dev) for _ in range(Ly)]
     cfg = hkv.config_for(w)
@@ -277,10 +278,8 @@ def gpu_arm(args, rank, world, dev):
         ms = timed_replays(g_main, args.steps)
         decode_ms = ev_dec[0].elapsed_time(ev_dec[1])
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = dist.max_over_ranks(ms, dev)
         torch.distributed.barrier()
-        ms = float(t.item())
     rc, detail = cache.check()
     if rc != 0:
         raise RuntimeError(f"device status {rc} ({detail}) after the timed passes")
@@ -398,9 +397,8 @@ def e2e_arm(args, w, cache, inp, dev, world):
         g.replay()
     ms = timed_replays(g, max(1, min(args.steps, 3)))
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+        from kv_cache_compression_hkv_b200 import dist
+        ms = dist.max_over_ranks(ms, dev)
     h2d = sum(x.numel() * x.element_size() for t in host_pre for x in t) + \
         host_dec.numel() * host_dec.element_size()
     d2h = host_out.numel() * host_out.element_size()

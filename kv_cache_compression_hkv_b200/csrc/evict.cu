@@ -226,6 +226,7 @@ cudaError_t prepare_kernels() {
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e == cudaSuccess) e = prepare_prefill(optin);
+    if (e == cudaSuccess) e = prepare_prefill_umma(optin);
     if (e == cudaSuccess) e = prepare_decode(optin);
     if (e == cudaSuccess) e = prepare_evict(optin);
     done = e;

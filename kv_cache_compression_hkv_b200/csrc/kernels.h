@@ -13,7 +13,10 @@ cudaError_t prepare_kernels();
 cudaError_t prepare_prefill(int smem);
 cudaError_t prepare_decode(int smem);
 cudaError_t prepare_evict(int smem);
+cudaError_t prepare_prefill_umma(int smem);
 size_t pack_smem_bytes(int P);
+cudaError_t launch_prefill_umma(const Layout& L, const void* q, const void* k, const void* v, int P,
+                                int64_t block_stride, void* out, cudaStream_t st);
 cudaError_t launch_prefill(const Layout& L, int layer, const void* q, const void* k, const void* v,
                            int P, int64_t block_stride, void* out, cudaStream_t st);
 cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void* k, const void* v,

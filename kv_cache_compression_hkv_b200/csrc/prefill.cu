@@ -228,15 +228,17 @@ cudaError_t launch_prefill(const Layout& L, int layer, const void* q, const void
     const int nb = L.S * L.H;
     dim3 grid(nb, (P + 3) / 4);
     size_t sm = (size_t)4 * (L.d + P) * sizeof(float);
-    if (L.dtype == HKV_DTYPE_F32)
+    cudaError_t e;
+    if (L.dtype == HKV_DTYPE_F32) {
+        // fp32 caches keep fp32 products: CUDA cores
         prefill_attn_simt<float><<<grid, 128, sm, st>>>(
             (const float*)q, (const float*)k, (const float*)v, P, L.d, block_stride, L.r,
             (float*)out, L.rows);
-    else
-        prefill_attn_simt<__nv_bfloat16><<<grid, 128, sm, st>>>(
-            (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, P, L.d,
-            block_stride, L.r, (__nv_bfloat16*)out, L.rows);
-    cudaError_t e = cudaGetLastError();
+        e = cudaGetLastError();
+    } else {
+        // bf16 caches: tcgen05 tensor cores
+        e = launch_prefill_umma(L, q, k, v, P, block_stride, out, st);
+    }
     if (e != cudaSuccess) return e;
     classify_kernel<<<L.S, 32 * L.H, 0, st>>>(L, layer, P);
     e = cudaGetLastError();

@@ -163,6 +163,37 @@ def test_prefill_outputs_match_oracle():
             assert np.abs(got - o).max() / np.abs(o).max() < 2e-2
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("P", [33, 65, 97, 128, 130, 192, 255, 384])
+def test_prefill_shapes_against_oracle(d, P):
+    """Tensor-core prefill: one or several 128-query tiles, ragged tails, the
+    last r rows straddling two tiles; outputs and labels against the oracle."""
+    w = WORKLOADS["janus_pro_1b"].scaled(num_seqs=2, num_layers=1, num_heads=6, local_heads=3,
+                                          head_dim=d, prefix_len=1, prefill_image=P - 1,
+                                          image_tokens=P + 39, local_window=min(28, P))
+    cfg = hkv.config_for(w, mode=hkv.MODE_HEADKV)
+    cfg.rho_num, cfg.rho_den = 1, 2
+    data = generate(w, 17 + P, DEV)
+    q, k, v = data[0]
+    cache = hkv.HeadKVCache(cfg, device=DEV)
+    out = torch.empty(2, 6, P, d, dtype=torch.bfloat16, device=DEV)
+    cache.prefill_classify(0, q[:, :, :P], k[:, :, :P], v[:, :, :P], out=out)
+    lab, ntau = cache.labels(0)
+    assert cache.check()[0] == 0
+    for s in range(2):
+        for h in range(6):
+            qq, kk, vv = (x[s, h, :P].double().cpu().numpy() for x in (q, k, v))
+            o, p = O.causal_attention(qq, kk, vv)
+            got = out[s, h].double().cpu().numpy()
+            assert np.abs(got - o).max() / np.abs(o).max() < 2e-2, (s, h)
+            e_nt, e_lab, cw = O.classify(p[-1], w.local_window, 0.9)
+            if abs(cw - 0.9) > 1e-3:
+                assert lab[s, h] == e_lab, (s, h, cw)
+            if e_nt > 1 and abs(np.cumsum(p[-1][::-1])[e_nt - 2] - 0.9) > 1e-3 and \
+                    abs(np.cumsum(p[-1][::-1])[e_nt - 1] - 0.9) > 1e-3:
+                assert ntau[s, h] == e_nt, (s, h)
+
+
 def test_full_size_sampled_units():
     """The bench's workload at full size and launch configuration; two
     sampled units go through the oracle in lock step."""
