@@ -45,6 +45,11 @@ def parse_args():
     ap.add_argument("--no-full", action="store_true", help="skip the full-cache comparator")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end arm")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--profile", action="store_true",
+                    help="eager run of a reduced workload for ncu captures (no timing line)")
+    ap.add_argument("--seqs", type=int, default=None, help="override the workload's sequences")
+    ap.add_argument("--layers", type=int, default=None, help="override the workload's layers")
+    ap.add_argument("--profile-steps", type=int, default=64)
     return ap.parse_args()
 
 
@@ -407,6 +412,31 @@ def e2e_arm(args, w, cache, inp, dev, world):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
 
 
+def profile_run(args, w):
+    """Eager prefill + decode steps of a reduced copy of the workload: the
+    command ncu captures single launches of (nothing is timed here)."""
+    import kv_cache_compression_hkv_b200 as hkv
+    dev = torch.device("cuda", 0)
+    w = w.scaled(num_seqs=args.seqs or w.num_seqs, num_layers=args.layers or w.num_layers)
+    inp = Inputs(w, args.seed, dev)
+    outs = [torch.empty(w.num_seqs, w.num_heads, w.head_dim, dtype=w.torch_dtype, device=dev)
+            for _ in range(w.num_layers)]
+    cache = hkv.HeadKVCache(hkv.config_for(w), device=dev)
+    for l in range(w.num_layers):
+        cache.prefill_classify(l, *inp.pre[l])
+    for t in range(min(args.profile_steps, w.decode_steps)):
+        for l in range(w.num_layers):
+            q, k, v = inp.dec[l]
+            cache.decode_step(l, q[t], k[t], v[t], outs[l])
+        cache.ste_evict()
+    torch.cuda.synchronize()
+    rc, detail = cache.check()
+    print(json.dumps({"profile_run": w.name, "seqs": w.num_seqs, "layers": w.num_layers,
+                      "steps": min(args.profile_steps, w.decode_steps), "status": rc}))
+    if rc != 0:
+        raise SystemExit(f"device status {rc} ({detail})")
+
+
 def main():
     args = parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -441,6 +471,10 @@ def main():
             "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+        return
+
+    if args.profile:
+        profile_run(args, w)
         return
 
     if world > 1:

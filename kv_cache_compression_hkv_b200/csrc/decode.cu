@@ -98,17 +98,25 @@ __device__ int chunk_prefix(const Layout& L, int layer, int t, int32_t* pre) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int NW = blockDim.x >> 5;
     const size_t hbase = (size_t)layer * n_heads;
-    const int per = (n_heads + blockDim.x - 1) / blockDim.x;
-    const int i0 = tid * per, i1 = min(i0 + per, n_heads);
-    int local = 0;
-    for (int i = i0; i < i1; ++i) {
-        const int n = len_at(L, hbase + i, t);
+    // chunk counts, coalesced (independent iterations: loads overlap)
+#pragma unroll 4
+    for (int i = tid; i < n_heads; i += blockDim.x) {
+        const size_t hx = hbase + i;
+        const int n = len_at(L, hx, t);
         int c = (n + CHUNK - 1) / CHUNK;
-        if (n > L.cap[hbase + i] || n < 0) {
-            if (blockIdx.x == 0) latch_error(L, HKV_ERR_CAPACITY, (int)(hbase + i));
+        if (n > L.cap[hx] || n < 0) {
+            if (blockIdx.x == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
             c = 0;
         }
-        local += c;
+        pre[i] = c;
+    }
+    __syncthreads();
+    // block-wide inclusive scan: contiguous runs per thread, then the warps
+    const int per = (n_heads + blockDim.x - 1) / blockDim.x;
+    const int i0 = min(tid * per, n_heads), i1 = min(i0 + per, n_heads);
+    int local = 0;
+    for (int i = i0; i < i1; ++i) {
+        local += pre[i];
         pre[i] = local;
     }
     int x = local;
@@ -259,17 +267,28 @@ __global__ void __launch_bounds__(256, 1)
         __threadfence();
         if (lane == 0) L.ticket[h] = 0;
         const float* pb = L.partial + (size_t)c0 * (d + 2);
+        // (max, sum) of the partials, lane-parallel; then the weighted sum
         float M = -INFINITY;
-        for (int i = 0; i < nch; ++i) M = fmaxf(M, __ldcg(pb + (size_t)i * (d + 2)));
-        float Ls = 0.f, o[DPL];
+        for (int i = lane; i < nch; i += 32) M = fmaxf(M, __ldcg(pb + (size_t)i * (d + 2)));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, o));
+        float Ls = 0.f;
+        for (int i = lane; i < nch; i += 32)
+            Ls += __ldcg(pb + (size_t)i * (d + 2) + 1) * exp2f(__ldcg(pb + (size_t)i * (d + 2)) - M);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(FULL_MASK, Ls, o);
+        float o[DPL];
 #pragma unroll
         for (int e = 0; e < DPL; ++e) o[e] = 0.f;
+#pragma unroll 4
         for (int i = 0; i < nch; ++i) {
             const float* pi = pb + (size_t)i * (d + 2);
             const float w = exp2f(__ldcg(pi) - M);
-            Ls = fmaf(__ldcg(pi + 1), w, Ls);
+            float a[DPL];
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) o[e] = fmaf(__ldcg(pi + 2 + lane * DPL + e), w, o[e]);
+            for (int e = 0; e < DPL; ++e) a[e] = __ldcg(pi + 2 + lane * DPL + e);
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) o[e] = fmaf(a[e], w, o[e]);
         }
         const float inv = 1.0f / Ls;
 #pragma unroll
