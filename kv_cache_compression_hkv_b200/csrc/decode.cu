@@ -16,6 +16,7 @@
 
 #include "hkv_internal.cuh"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace hkv {
 
@@ -30,6 +31,14 @@ template <int DPL> struct Raw<__nv_bfloat16, DPL> {
         else {
 #pragma unroll
             for (int i = 0; i < W; ++i) w[i] = __ldg(reinterpret_cast<const unsigned int*>(p) + i);
+        }
+    }
+    __device__ __forceinline__ void load_shared(const __nv_bfloat16* p) {
+        if constexpr (W == 2) { uint2 v = *reinterpret_cast<const uint2*>(p); w[0] = v.x; w[1] = v.y; }
+        else if constexpr (W == 1) { w[0] = *reinterpret_cast<const unsigned int*>(p); }
+        else {
+#pragma unroll
+            for (int i = 0; i < W; ++i) w[i] = reinterpret_cast<const unsigned int*>(p)[i];
         }
     }
     __device__ __forceinline__ void zero() {
@@ -54,6 +63,14 @@ template <int DPL> struct Raw<float, DPL> {
         else {
 #pragma unroll
             for (int i = 0; i < DPL; ++i) w[i] = __ldg(p + i);
+        }
+    }
+    __device__ __forceinline__ void load_shared(const float* p) {
+        if constexpr (DPL == 4) { float4 v = *reinterpret_cast<const float4*>(p); w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w; }
+        else if constexpr (DPL == 2) { float2 v = *reinterpret_cast<const float2*>(p); w[0] = v.x; w[1] = v.y; }
+        else {
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) w[i] = p[i];
         }
     }
     __device__ __forceinline__ void zero() {
@@ -89,35 +106,61 @@ __device__ __forceinline__ void store_row(T* p, const float (&x)[DPL]) {
     }
 }
 
-// Block-wide inclusive prefix of the chunk counts of all heads of a layer
-// into pre[0..n_heads).  Heads whose length exceeds their capacity latch
-// HKV_ERR_CAPACITY and contribute no work.
-__device__ int chunk_prefix(const Layout& L, int layer, int t, int32_t* pre) {
+// Per-head facts of one decode launch, cached in shared memory by every
+// block: inclusive prefix of chunk counts, slot offset in the layer, cache
+// length, slot of the appended token (-1: none) and whether the head records
+// STE logits this step.
+struct HeadTable {
+    int32_t* pre;
+    int64_t* slot0;
+    int16_t* len;
+    int16_t* jn;
+    uint8_t* scoring;
+    __host__ __device__ static size_t bytes(int n) { return (size_t)n * (4 + 8 + 2 + 2 + 1) + 64; }
+};
+
+__device__ HeadTable carve_table(unsigned char* p, int n) {
+    HeadTable t;
+    t.slot0 = reinterpret_cast<int64_t*>(p);
+    t.pre = reinterpret_cast<int32_t*>(t.slot0 + n);
+    t.len = reinterpret_cast<int16_t*>(t.pre + n);
+    t.jn = t.len + n;
+    t.scoring = reinterpret_cast<uint8_t*>(t.jn + n);
+    return t;
+}
+
+// Fills the table (coalesced, independent loads) and prefix-sums the chunk
+// counts; returns the layer's chunk count.  Heads past their capacity latch
+// HKV_ERR_CAPACITY and get no work.
+__device__ int build_table(const Layout& L, int layer, int t, int append, HeadTable tb) {
     __shared__ int wsum[32];
     const int n_heads = L.S * L.H;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int NW = blockDim.x >> 5;
     const size_t hbase = (size_t)layer * n_heads;
-    // chunk counts, coalesced (independent iterations: loads overlap)
 #pragma unroll 4
     for (int i = tid; i < n_heads; i += blockDim.x) {
         const size_t hx = hbase + i;
         const int n = len_at(L, hx, t);
+        const int cap = L.cap[hx];
         int c = (n + CHUNK - 1) / CHUNK;
-        if (n > L.cap[hx] || n < 0) {
+        if (n > cap || n < 1) {
             if (blockIdx.x == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
             c = 0;
         }
-        pre[i] = c;
+        tb.pre[i] = c;
+        tb.len[i] = (int16_t)n;
+        tb.slot0[i] = (int64_t)region_slot0(L, layer, i / L.H) + L.off[hx];
+        tb.jn[i] = (int16_t)(append ? append_slot(L, hx, t, n) : -1);
+        tb.scoring[i] = L.label[hx] == 0 && L.mode != HKV_MODE_FULL && n > cap - L.r;
     }
     __syncthreads();
-    // block-wide inclusive scan: contiguous runs per thread, then the warps
     const int per = (n_heads + blockDim.x - 1) / blockDim.x;
     const int i0 = min(tid * per, n_heads), i1 = min(i0 + per, n_heads);
     int local = 0;
     for (int i = i0; i < i1; ++i) {
-        local += pre[i];
-        pre[i] = local;
+        local += tb.pre[i];
+        tb.pre[i] = local;
     }
     int x = local;
 #pragma unroll
@@ -138,163 +181,274 @@ __device__ int chunk_prefix(const Layout& L, int layer, int t, int32_t* pre) {
     }
     __syncthreads();
     const int offset = x - local + (warp ? wsum[warp - 1] : 0);
-    for (int i = i0; i < i1; ++i) pre[i] += offset;
+    for (int i = i0; i < i1; ++i) tb.pre[i] += offset;
     __syncthreads();
-    return pre[n_heads - 1];
+    return tb.pre[n_heads - 1];
+}
+
+// Head holding chunk c: smallest h with pre[h] > c.
+__device__ __forceinline__ int head_of(const int32_t* pre, int n, int c) {
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (pre[mid] > c) hi = mid; else lo = mid + 1;
+    }
+    return lo;
+}
+
+// First chunk of warp w's range when `total` chunks go to `gw` warps.
+__device__ __forceinline__ int range_begin(int w, int total, int gw) {
+    return (int)((int64_t)w * total / gw);
+}
+// Warp whose range holds chunk c.
+__device__ __forceinline__ int range_owner(int c, int total, int gw) {
+    return (int)(((int64_t)(c + 1) * gw - 1) / total);
 }
 
 template <typename T, int DPL>
 __global__ void __launch_bounds__(256, 1)
     decode_kernel(Layout L, int layer, const T* __restrict__ q_t, const T* __restrict__ k_t,
-                  const T* __restrict__ v_t, T* __restrict__ o_t, int append) {
-    extern __shared__ int32_t pre[];
+                  const T* __restrict__ v_t, T* __restrict__ o_t, int append, int nstage) {
+    extern __shared__ __align__(128) unsigned char dsm[];
     const int n_heads = L.S * L.H;
-    const int d = L.d;
+    constexpr int D = DPL * 32;
+    constexpr int ROW = D * (int)sizeof(T);           // bytes of one cache row
+    constexpr int STAGE = (2 * CHUNK + 1) * ROW;       // K rows, V rows, the query
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int NW = blockDim.x >> 5;
     const int t = append ? L.t_next[layer] : L.t_next[layer] - 1;
-    const int total = chunk_prefix(L, layer, t, pre);
-    const size_t hbase = (size_t)layer * n_heads;
-    const float qscale = LOG2E / sqrtf((float)d);
-    T* Kp = reinterpret_cast<T*>(L.K);
-    T* Vp = reinterpret_cast<T*>(L.V);
     const int col = t % L.r;
 
-    for (int cid = blockIdx.x * NW + warp; cid < total; cid += gridDim.x * NW) {
-        int lo = 0, hi = n_heads - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (pre[mid] > cid) hi = mid; else lo = mid + 1;
-        }
-        const int h = lo;  // s * H + head
-        const int c0 = h ? pre[h - 1] : 0;
-        const int c = cid - c0;
-        const size_t hx = hbase + h;
-        const int len = len_at(L, hx, t);
-        const int nch = (len + CHUNK - 1) / CHUNK;
-        const int s = h / L.H;
-        const size_t slot0 = region_slot0(L, layer, s) + L.off[hx];
-        const int jn = append ? append_slot(L, hx, t, len) : -1;
-        const int tok0 = c * CHUNK;
-        const int n = min(CHUNK, len - tok0);
-        const bool scoring = L.label[hx] == 0 && L.mode != HKV_MODE_FULL && len > L.cap[hx] - L.r;
+    unsigned char* stages = dsm;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(stages + (size_t)NW * nstage * STAGE);
+    HeadTable tb = carve_table(reinterpret_cast<unsigned char*>(bars + NW * nstage), n_heads);
+    const int total = build_table(L, layer, t, append, tb);
 
-        float qv[DPL];
-        {
-            Raw<T, DPL> qr;
-            qr.load(q_t + (size_t)h * d + lane * DPL);
-#pragma unroll
-            for (int i = 0; i < DPL; ++i) qv[i] = qr.get(i) * qscale;
+    const int GW = gridDim.x * NW;
+    const int gw = blockIdx.x * NW + warp;
+    const int c_begin = total > 0 ? range_begin(gw, total, GW) : 0;
+    const int c_end = total > 0 ? range_begin(gw + 1, total, GW) : 0;
+    T* Kp = reinterpret_cast<T*>(L.K);
+    T* Vp = reinterpret_cast<T*>(L.V);
+    const size_t hbase = (size_t)layer * n_heads;
+    const float qscale = LOG2E / sqrtf((float)D);
+    constexpr uint64_t WAIT_NS = 2000000000ull;
+
+    if (c_begin < c_end) {
+        unsigned char* my = stages + (size_t)warp * nstage * STAGE;
+        uint64_t* bar = bars + warp * nstage;
+        if (lane == 0) {
+            for (int s = 0; s < nstage; ++s) ptx::mbar_init(bar + s, 1);
+            ptx::fence_mbar_init();
         }
-        // issue every load of the chunk first
-        Raw<T, DPL> kr[CHUNK], vr[CHUNK];
+        __syncwarp();
+
+        // producer cursor (lane 0 issues): chunk ip of head hp
+        int ip = c_begin, hp = head_of(tb.pre, n_heads, c_begin);
+        auto issue = [&](int stage) {
+            if (lane == 0) {
+                const int first = hp ? tb.pre[hp - 1] : 0;
+                const int tok0 = (ip - first) * CHUNK;
+                const int n = min(CHUNK, (int)tb.len[hp] - tok0);
+                const int jn = tb.jn[hp];
+                const size_t row0 = (size_t)tb.slot0[hp] + tok0;
+                unsigned char* kd = my + (size_t)stage * STAGE;
+                unsigned char* vd = kd + CHUNK * ROW;
+                unsigned char* qd = vd + CHUNK * ROW;
+                uint64_t* b = bar + stage;
+                ptx::mbar_expect_tx(b, (uint32_t)(2 * n + 1) * ROW);
+                ptx::bulk_g2s(qd, q_t + (size_t)hp * D, ROW, b);
+                const int a = jn - tok0;
+                if (a >= 0 && a < n) {
+                    if (a > 0) {
+                        ptx::bulk_g2s(kd, Kp + row0 * D, a * ROW, b);
+                        ptx::bulk_g2s(vd, Vp + row0 * D, a * ROW, b);
+                    }
+                    ptx::bulk_g2s(kd + a * ROW, k_t + (size_t)hp * D, ROW, b);
+                    ptx::bulk_g2s(vd + a * ROW, v_t + (size_t)hp * D, ROW, b);
+                    if (n - a - 1 > 0) {
+                        ptx::bulk_g2s(kd + (a + 1) * ROW, Kp + (row0 + a + 1) * D, (n - a - 1) * ROW, b);
+                        ptx::bulk_g2s(vd + (a + 1) * ROW, Vp + (row0 + a + 1) * D, (n - a - 1) * ROW, b);
+                    }
+                } else {
+                    ptx::bulk_g2s(kd, Kp + row0 * D, n * ROW, b);
+                    ptx::bulk_g2s(vd, Vp + row0 * D, n * ROW, b);
+                }
+            }
+            ++ip;
+            if (ip < c_end && tb.pre[hp] <= ip) hp = head_of(tb.pre, n_heads, ip);
+        };
+        for (int s = 0; s < nstage && ip < c_end; ++s) issue(s);
+
+        int hc = head_of(tb.pre, n_heads, c_begin);
+        int seg0 = c_begin;
+        float m = -INFINITY, l = 0.f, acc[DPL];
 #pragma unroll
-        for (int j = 0; j < CHUNK; ++j) {
-            const int sj = tok0 + j;
-            if (j < n) {
-                const T* kp = sj == jn ? k_t + (size_t)h * d : Kp + (slot0 + sj) * d;
-                const T* vp = sj == jn ? v_t + (size_t)h * d : Vp + (slot0 + sj) * d;
-                kr[j].load(kp + lane * DPL);
-                vr[j].load(vp + lane * DPL);
+        for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+        bool failed = false;
+
+        for (int i = c_begin; i < c_end; ++i) {
+            const int k = i - c_begin;
+            const int stage = k % nstage;
+            if (!ptx::mbar_wait(bar + stage, (uint32_t)((k / nstage) & 1), WAIT_NS)) {
+                failed = true;
+                break;
+            }
+            const int first = hc ? tb.pre[hc - 1] : 0;
+            const int tok0 = (i - first) * CHUNK;
+            const int len = tb.len[hc];
+            const int n = min(CHUNK, len - tok0);
+            const unsigned char* kst = my + (size_t)stage * STAGE;
+            const unsigned char* vst = kst + CHUNK * ROW;
+            const T* qs = reinterpret_cast<const T*>(vst + CHUNK * ROW);
+            float qv[DPL];
+            {
+                Raw<T, DPL> qr;
+                qr.load_shared(qs + lane * DPL);
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) qv[e] = qr.get(e) * qscale;
+            }
+            // partial dot products, lane-transposed butterfly: lane j ends
+            // with token j's logit
+            float part[CHUNK];
+#pragma unroll
+            for (int j = 0; j < CHUNK; ++j) {
+                float a = 0.f;
+                if (j < n) {
+                    Raw<T, DPL> kr;
+                    kr.load_shared(reinterpret_cast<const T*>(kst + j * ROW) + lane * DPL);
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) a = fmaf(qv[e], kr.get(e), a);
+                }
+                part[j] = a;
+            }
+#pragma unroll
+            for (int w = 16; w >= 1; w >>= 1) {
+                const bool upper = lane & w;
+#pragma unroll
+                for (int e = 0; e < w; ++e) {
+                    const float send = upper ? part[e] : part[e + w];
+                    const float keep = upper ? part[e + w] : part[e];
+                    part[e] = keep + __shfl_xor_sync(FULL_MASK, send, w);
+                }
+            }
+            const float sl = lane < n ? part[0] : -INFINITY;
+            const int64_t row0 = tb.slot0[hc] + tok0;
+            if (tb.scoring[hc] && lane < n) L.logit[(size_t)(row0 + lane) * L.r + col] = sl;
+            float cm = sl;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(FULL_MASK, cm, o));
+            const float mn = fmaxf(m, cm);
+            const float alpha = exp2f(m - mn);
+            const float p = lane < n ? exp2f(sl - mn) : 0.f;
+            float ps = p;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(FULL_MASK, ps, o);
+            l = l * alpha + ps;
+            m = mn;
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) acc[e] *= alpha;
+#pragma unroll
+            for (int j = 0; j < CHUNK; ++j) {
+                if (j < n) {
+                    const float pj = __shfl_sync(FULL_MASK, p, j);
+                    Raw<T, DPL> vr;
+                    vr.load_shared(reinterpret_cast<const T*>(vst + j * ROW) + lane * DPL);
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) acc[e] = fmaf(pj, vr.get(e), acc[e]);
+                }
+            }
+            // the appended token joins the cache
+            const int a = tb.jn[hc] - tok0;
+            if (a >= 0 && a < n) {
+                Raw<T, DPL> kr, vr;
+                kr.load_shared(reinterpret_cast<const T*>(kst + a * ROW) + lane * DPL);
+                vr.load_shared(reinterpret_cast<const T*>(vst + a * ROW) + lane * DPL);
+                kr.store(Kp + (size_t)(row0 + a) * D + lane * DPL);
+                vr.store(Vp + (size_t)(row0 + a) * D + lane * DPL);
+                if (lane == 0) L.pos[row0 + a] = t;
+            }
+            __syncwarp();
+            if (ip < c_end) {
+                ptx::fence_proxy_async();  // this stage's reads before its refill
+                issue(stage);
+            }
+            if (i + 1 < c_end && tb.pre[hc] > i + 1) continue;  // head goes on
+
+            // end of this warp's segment of head hc
+            const size_t hx = hbase + hc;
+            if (!(l > 0.f) || isinf(l)) latch_error(L, HKV_ERR_NUMERIC, (int)hx);
+            const bool whole = seg0 == first && i + 1 == tb.pre[hc];
+            if (whole) {
+                const float inv = 1.0f / l;
+                float o[DPL];
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) o[e] = acc[e] * inv;
+                store_row<T, DPL>(o_t + (size_t)hc * D + lane * DPL, o);
+                if (tb.scoring[hc] && lane == 0) L.ml[hx * L.r + col] = make_float2(m, l);
             } else {
-                kr[j].zero();
-                vr[j].zero();
+                float* pp = L.partial + (size_t)seg0 * (D + 2);
+                if (lane == 0) { pp[0] = m; pp[1] = l; }
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) pp[2 + lane * DPL + e] = acc[e];
+                __threadfence();
+                const int w_a = range_owner(first, total, GW);
+                const int w_b = range_owner(tb.pre[hc] - 1, total, GW);
+                int segs = 0;
+                for (int w = w_a; w <= w_b; ++w)
+                    segs += range_begin(w, total, GW) < range_begin(w + 1, total, GW);
+                int prev = 0;
+                if (lane == 0) prev = atomicAdd(&L.ticket[hc], 1);
+                prev = __shfl_sync(FULL_MASK, prev, 0);
+                if (prev == segs - 1) {
+                    // last segment in: merge (lane-parallel over segments)
+                    __threadfence();
+                    if (lane == 0) L.ticket[hc] = 0;
+                    float M = -INFINITY;
+                    for (int w = w_a + lane; w <= w_b; w += 32) {
+                        const int rb = range_begin(w, total, GW);
+                        if (rb < range_begin(w + 1, total, GW))
+                            M = fmaxf(M, __ldcg(L.partial + (size_t)max(rb, first) * (D + 2)));
+                    }
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, o));
+                    float Ls = 0.f, o[DPL];
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) o[e] = 0.f;
+                    for (int w = w_a; w <= w_b; ++w) {
+                        const int rb = range_begin(w, total, GW);
+                        if (rb >= range_begin(w + 1, total, GW)) continue;
+                        const float* pi = L.partial + (size_t)max(rb, first) * (D + 2);
+                        const float wt = exp2f(__ldcg(pi) - M);
+                        Ls = fmaf(__ldcg(pi + 1), wt, Ls);
+#pragma unroll
+                        for (int e = 0; e < DPL; ++e) o[e] = fmaf(__ldcg(pi + 2 + lane * DPL + e), wt, o[e]);
+                    }
+                    const float inv = 1.0f / Ls;
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) o[e] *= inv;
+                    store_row<T, DPL>(o_t + (size_t)hc * D + lane * DPL, o);
+                    if (tb.scoring[hc] && lane == 0) L.ml[hx * L.r + col] = make_float2(M, Ls);
+                }
+            }
+            // next head
+            seg0 = i + 1;
+            if (i + 1 < c_end) hc = head_of(tb.pre, n_heads, i + 1);
+            m = -INFINITY;
+            l = 0.f;
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+        }
+        if (failed) {
+            if (lane == 0) latch_error(L, HKV_ERR_TIMEOUT, (int)(hbase + hc));
+            // let this warp's outstanding copies land before the block exits
+            for (int k = 0; k < nstage; ++k) {
+                const int j = ip - 1 - k;
+                if (j < c_begin) break;
+                const int kk = j - c_begin;
+                ptx::mbar_wait(bar + kk % nstage, (uint32_t)((kk / nstage) & 1), WAIT_NS);
             }
         }
-        // partial dot products, then the lane-transposed butterfly sum:
-        // afterwards part[0] on lane j holds the logit of token j.
-        float part[CHUNK];
-#pragma unroll
-        for (int j = 0; j < CHUNK; ++j) {
-            float a = 0.f;
-#pragma unroll
-            for (int i = 0; i < DPL; ++i) a = fmaf(qv[i], kr[j].get(i), a);
-            part[j] = a;
-        }
-#pragma unroll
-        for (int w = 16; w >= 1; w >>= 1) {
-            const bool upper = lane & w;
-#pragma unroll
-            for (int i = 0; i < w; ++i) {
-                const float send = upper ? part[i] : part[i + w];
-                const float keep = upper ? part[i + w] : part[i];
-                part[i] = keep + __shfl_xor_sync(FULL_MASK, send, w);
-            }
-        }
-        const float sl = lane < n ? part[0] : -INFINITY;
-        if (scoring && lane < n) L.logit[(slot0 + tok0 + lane) * L.r + col] = sl;
-        float m = sl;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL_MASK, m, o));
-        const float p = lane < n ? exp2f(sl - m) : 0.f;
-        float l = p;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(FULL_MASK, l, o);
-        float acc[DPL];
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
-#pragma unroll
-        for (int j = 0; j < CHUNK; ++j) {
-            const float pj = __shfl_sync(FULL_MASK, p, j);
-#pragma unroll
-            for (int i = 0; i < DPL; ++i) acc[i] = fmaf(pj, vr[j].get(i), acc[i]);
-            if (tok0 + j == jn) {  // the appended token joins the cache
-                kr[j].store(Kp + (slot0 + jn) * d + lane * DPL);
-                vr[j].store(Vp + (slot0 + jn) * d + lane * DPL);
-                if (lane == 0) L.pos[slot0 + jn] = t;
-            }
-        }
-        if (!(l > 0.f) || isinf(l)) latch_error(L, HKV_ERR_NUMERIC, (int)hx);
-        if (nch == 1) {
-            const float inv = 1.0f / l;
-            float o[DPL];
-#pragma unroll
-            for (int i = 0; i < DPL; ++i) o[i] = acc[i] * inv;
-            store_row<T, DPL>(o_t + (size_t)h * d + lane * DPL, o);
-            if (scoring && lane == 0) L.ml[hx * L.r + col] = make_float2(m, l);
-            continue;
-        }
-        float* pp = L.partial + (size_t)cid * (d + 2);
-        if (lane == 0) { pp[0] = m; pp[1] = l; }
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) pp[2 + lane * DPL + i] = acc[i];
-        __threadfence();
-        int prev = 0;
-        if (lane == 0) prev = atomicAdd(&L.ticket[h], 1);
-        prev = __shfl_sync(FULL_MASK, prev, 0);
-        if (prev != nch - 1) continue;
-        // last arrival for this head: merge the partials
-        __threadfence();
-        if (lane == 0) L.ticket[h] = 0;
-        const float* pb = L.partial + (size_t)c0 * (d + 2);
-        // (max, sum) of the partials, lane-parallel; then the weighted sum
-        float M = -INFINITY;
-        for (int i = lane; i < nch; i += 32) M = fmaxf(M, __ldcg(pb + (size_t)i * (d + 2)));
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, o));
-        float Ls = 0.f;
-        for (int i = lane; i < nch; i += 32)
-            Ls += __ldcg(pb + (size_t)i * (d + 2) + 1) * exp2f(__ldcg(pb + (size_t)i * (d + 2)) - M);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(FULL_MASK, Ls, o);
-        float o[DPL];
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) o[e] = 0.f;
-#pragma unroll 4
-        for (int i = 0; i < nch; ++i) {
-            const float* pi = pb + (size_t)i * (d + 2);
-            const float w = exp2f(__ldcg(pi) - M);
-            float a[DPL];
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) a[e] = __ldcg(pi + 2 + lane * DPL + e);
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) o[e] = fmaf(a[e], w, o[e]);
-        }
-        const float inv = 1.0f / Ls;
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) o[e] *= inv;
-        store_row<T, DPL>(o_t + (size_t)h * d + lane * DPL, o);
-        if (scoring && lane == 0) L.ml[hx * L.r + col] = make_float2(M, Ls);
     }
     if (append) {
         __syncthreads();
@@ -347,12 +501,41 @@ __global__ void __launch_bounds__(256) append_kernel(Layout L, int layer, const 
 // launchers
 // ---------------------------------------------------------------------------
 
+// Launch shape of the decode kernel: warps per block and pipeline stages per
+// warp that fit the shared memory next to the head table.
+struct DecodeShape {
+    int warps, nstage;
+    size_t smem;
+};
+
+static DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
+    const size_t row = (size_t)L.d * (L.dtype == HKV_DTYPE_F32 ? 4 : 2);
+    const size_t stage = (2 * CHUNK + 1) * row;
+    const size_t fixed = HeadTable::bytes(L.S * L.H) + 128;
+    DecodeShape sh{0, 0, 0};
+    for (int ns = 3; ns >= 2 && sh.warps == 0; --ns) {
+        const size_t per = ns * (stage + 8);
+        int w = smem_limit > fixed ? (int)((smem_limit - fixed) / per) : 0;
+        if (w > 8) w = 8;
+        if (w >= (ns == 3 ? 6 : 1)) sh = DecodeShape{w, ns, fixed + (size_t)w * per};
+    }
+    return sh;
+}
+
 template <typename T, int DPL>
 static cudaError_t launch_decode_t(const Layout& L, int layer, const void* q, const void* k,
                                    const void* v, void* o, int append, int grid, cudaStream_t st) {
-    const size_t sm = (size_t)L.S * L.H * sizeof(int32_t);
-    decode_kernel<T, DPL><<<grid, 256, sm, st>>>(L, layer, (const T*)q, (const T*)k, (const T*)v,
-                                                 (T*)o, append);
+    static size_t limit = 0;
+    if (!limit) {
+        int dev = 0, optin = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        limit = (size_t)optin - 256;  // room for the kernel's static shared memory
+    }
+    const DecodeShape sh = decode_shape(L, limit);
+    if (sh.warps == 0) return cudaErrorInvalidConfiguration;
+    decode_kernel<T, DPL><<<grid, 32 * sh.warps, sh.smem, st>>>(L, layer, (const T*)q, (const T*)k,
+                                                                (const T*)v, (T*)o, append, sh.nstage);
     return cudaGetLastError();
 }
 

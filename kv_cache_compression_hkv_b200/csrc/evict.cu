@@ -15,12 +15,22 @@
 
 namespace hkv {
 
+// Per-warp scratch of the eviction: the select's own scratch, then the
+// head's scores and positions, then the (max, sum) of the scoring steps.
+__host__ __device__ inline size_t evict_warp_bytes(int n_max) {
+    return select_scratch_bytes(n_max) + (size_t)round32(n_max) * 8 + 32 * 8;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(128) evict_kernel(Layout L, int l0, int l1, int n_max) {
     extern __shared__ __align__(16) unsigned char esm[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int NW = blockDim.x >> 5;
-    SelectScratch sc = carve_select_scratch(esm + (size_t)warp * select_scratch_bytes(n_max), n_max);
+    unsigned char* wbase = esm + (size_t)warp * evict_warp_bytes(n_max);
+    SelectScratch sc = carve_select_scratch(wbase, n_max);
+    float* sc_s = reinterpret_cast<float*>(wbase + select_scratch_bytes(n_max));
+    int32_t* pos_s = reinterpret_cast<int32_t*>(sc_s + round32(n_max));
+    float2* ml_s = reinterpret_cast<float2*>(pos_s + round32(n_max));
     const int n_heads = L.S * L.H;
     const int total = (l1 - l0) * n_heads;
     const int d = L.d;
@@ -56,21 +66,41 @@ __global__ void __launch_bounds__(128) evict_kernel(Layout L, int l0, int l1, in
                 continue;
             }
             const size_t slot0 = region_slot0(L, l, s) + L.off[hx];
-            const float2* mlh = L.ml + hx * r;  // (max, sum) of each scoring step
+            // (max, sum) of each scoring step, by column = step mod r
+            if (lane < r) ml_s[lane] = L.ml[hx * r + lane];
+            __syncwarp();
+            // scores: summed softmax weight of the last r queries, each
+            // counting only tokens already cached at its step
             bool bad = false;
-            // called only by lanes that hold a token: no warp collectives here
-            auto key_of = [&](int q, uint32_t& sb, int32_t& p) {
-                p = L.pos[slot0 + q];
+#pragma unroll 4
+            for (int q = lane; q < n; q += 32) {
+                const int p = L.pos[slot0 + q];
                 const float* lg = L.logit + (slot0 + q) * r;
-                float sc_ = 0.f;
-                for (int step = t - r + 1; step <= t; ++step) {
-                    if (p > step) continue;  // not yet cached at that step
-                    const int col = step % r;
-                    const float2 ml = mlh[col];
-                    sc_ += exp2f(lg[col] - ml.x) / ml.y;
+                float v[32];
+                if (r == 8) {
+                    const float4 a = *reinterpret_cast<const float4*>(lg);
+                    const float4 b = *reinterpret_cast<const float4*>(lg + 4);
+                    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+                    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) if (c < r) v[c] = lg[c];
                 }
-                if (isnan(sc_)) bad = true;
-                sb = __float_as_uint(sc_);
+                float acc = 0.f;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    if (c >= r) break;
+                    const int step = t - (((t - c) % r) + r) % r;  // the window step of column c
+                    if (p <= step) acc += exp2f(v[c] - ml_s[c].x) / ml_s[c].y;
+                }
+                if (isnan(acc)) bad = true;
+                sc_s[q] = acc;
+                pos_s[q] = p;
+            }
+            __syncwarp();
+            auto key_of = [&](int q, uint32_t& sb, int32_t& p) {
+                sb = __float_as_uint(sc_s[q]);
+                p = pos_s[q];
             };
             const int E = n - target;
             warp_stratified_select(sc, n, t, L.D, E / 2, E - E / 2, L.stratified, key_of);
@@ -95,13 +125,12 @@ __global__ void __launch_bounds__(128) evict_kernel(Layout L, int l0, int l1, in
                 if (lane == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
                 continue;
             }
-            // move rows: K and V, 16-byte pieces, four per lane in flight
+            // move rows: K and V in 16-byte pieces, eight per lane in flight
             const int pieces = nh * per_row * 2;
-            for (int w0 = 0; w0 < pieces; w0 += 32 * 4) {
-                uint4 buf[4];
-                size_t dst[4];
+            for (int w0 = 0; w0 < pieces; w0 += 32 * 8) {
+                uint4 buf[8];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < 8; ++u) {
                     const int w = w0 + u * 32 + lane;
                     if (w < pieces) {
                         const int mv = w / (per_row * 2);
@@ -109,23 +138,24 @@ __global__ void __launch_bounds__(128) evict_kernel(Layout L, int l0, int l1, in
                         const bool isv = rem >= per_row;
                         const int pc = (isv ? rem - per_row : rem) * PIECE;
                         const size_t src = (slot0 + sc.moves[sc.n_max - 1 - mv]) * d + pc;
-                        dst[u] = (slot0 + sc.moves[mv]) * d + pc;
                         buf[u] = *reinterpret_cast<const uint4*>((isv ? Vp : Kp) + src);
-                        dst[u] |= (size_t)isv << 62;
                     }
                 }
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < 8; ++u) {
                     const int w = w0 + u * 32 + lane;
                     if (w < pieces) {
-                        const bool isv = (dst[u] >> 62) & 1;
-                        const size_t o = dst[u] & ~(3ull << 62);
-                        *reinterpret_cast<uint4*>((isv ? Vp : Kp) + o) = buf[u];
+                        const int mv = w / (per_row * 2);
+                        const int rem = w % (per_row * 2);
+                        const bool isv = rem >= per_row;
+                        const int pc = (isv ? rem - per_row : rem) * PIECE;
+                        const size_t dst = (slot0 + sc.moves[mv]) * d + pc;
+                        *reinterpret_cast<uint4*>((isv ? Vp : Kp) + dst) = buf[u];
                     }
                 }
             }
             for (int mv = lane; mv < nh; mv += 32)
-                L.pos[slot0 + sc.moves[mv]] = L.pos[slot0 + sc.moves[sc.n_max - 1 - mv]];
+                L.pos[slot0 + sc.moves[mv]] = pos_s[sc.moves[sc.n_max - 1 - mv]];
             __syncwarp();
             if (lane == 0) {
                 L.base_len[hx] = target;
@@ -175,7 +205,7 @@ __global__ void __launch_bounds__(128) select_batch_kernel(
 // ---------------------------------------------------------------------------
 
 static int evict_warps(int n_max) {
-    const size_t per = select_scratch_bytes(n_max);
+    const size_t per = evict_warp_bytes(n_max);
     int w = (int)((200 * 1024) / per);
     return w < 1 ? 1 : (w > 4 ? 4 : w);
 }
@@ -183,7 +213,7 @@ static int evict_warps(int n_max) {
 cudaError_t launch_evict(const Layout& L, int l0, int l1, int grid, cudaStream_t st) {
     const int n_max = L.L;
     const int nw = evict_warps(n_max);
-    const size_t sm = (size_t)nw * select_scratch_bytes(n_max);
+    const size_t sm = (size_t)nw * evict_warp_bytes(n_max);
     if (L.dtype == HKV_DTYPE_BF16)
         evict_kernel<__nv_bfloat16><<<grid, 32 * nw, sm, st>>>(L, l0, l1, n_max);
     else

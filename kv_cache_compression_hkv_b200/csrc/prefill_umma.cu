@@ -20,6 +20,7 @@
 
 #include "hkv_internal.cuh"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace hkv {
 namespace umma {
@@ -29,41 +30,11 @@ constexpr int KT = 64;    // keys per key tile (MMA N of S, K of P V)
 constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t O_COL = 128;  // O accumulator columns start here; S uses 0..63
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ uint64_t globaltimer() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-                 "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(phase)
-        : "memory");
-    return ok != 0;
-}
-// Waits for the phase with the given parity; gives up after `ns` nanoseconds.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, uint64_t ns) {
-    if (mbar_try_wait(bar, phase)) return true;
-    const uint64_t t0 = globaltimer();
-    while (!mbar_try_wait(bar, phase))
-        if (globaltimer() - t0 > ns) return false;
-    return true;
-}
+using ptx::smem_u32;
+using ptx::mbar_init;
+using ptx::mbar_expect_tx;
+using ptx::mbar_wait;
+
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0,
                                             int c1, int c2) {
     asm volatile(
@@ -74,7 +45,7 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
 }
 __device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+using ptx::fence_proxy_async;
 
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), version 1.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
