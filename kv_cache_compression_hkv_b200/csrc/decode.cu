@@ -221,8 +221,11 @@ __global__ void __launch_bounds__(256, 1)
 
     unsigned char* stages = dsm;
     uint64_t* bars = reinterpret_cast<uint64_t*>(stages + (size_t)NW * nstage * STAGE);
-    HeadTable tb = carve_table(reinterpret_cast<unsigned char*>(bars + NW * nstage), n_heads);
+    float* qbuf = reinterpret_cast<float*>(                     // [NW][D] fp32 queries
+        ((uintptr_t)(bars + NW * nstage) + 15) & ~(uintptr_t)15);
+    HeadTable tb = carve_table(reinterpret_cast<unsigned char*>(qbuf + NW * D), n_heads);
     const int total = build_table(L, layer, t, append, tb);
+    constexpr int NPIECE = ROW / 16;  // 16-byte pieces per row
 
     const int GW = gridDim.x * NW;
     const int gw = blockIdx.x * NW + warp;
@@ -237,6 +240,7 @@ __global__ void __launch_bounds__(256, 1)
     if (c_begin < c_end) {
         unsigned char* my = stages + (size_t)warp * nstage * STAGE;
         uint64_t* bar = bars + warp * nstage;
+        float* myq = qbuf + warp * D;
         if (lane == 0) {
             for (int s = 0; s < nstage; ++s) ptx::mbar_init(bar + s, 1);
             ptx::fence_mbar_init();
@@ -300,39 +304,46 @@ __global__ void __launch_bounds__(256, 1)
             const int n = min(CHUNK, len - tok0);
             const unsigned char* kst = my + (size_t)stage * STAGE;
             const unsigned char* vst = kst + CHUNK * ROW;
-            const T* qs = reinterpret_cast<const T*>(vst + CHUNK * ROW);
-            float qv[DPL];
-            {
+            if (i == seg0) {
+                // a new head: its query, pre-scaled, in fp32 shared memory
+                const T* qs = reinterpret_cast<const T*>(vst + CHUNK * ROW);
                 Raw<T, DPL> qr;
                 qr.load_shared(qs + lane * DPL);
 #pragma unroll
-                for (int e = 0; e < DPL; ++e) qv[e] = qr.get(e) * qscale;
+                for (int e = 0; e < DPL; ++e) myq[lane * DPL + e] = qr.get(e) * qscale;
+                __syncwarp();
             }
-            // partial dot products, lane-transposed butterfly: lane j ends
-            // with token j's logit
-            float part[CHUNK];
+            // lane j: dot product of the query with row j, reading the row's
+            // 16-byte pieces in a lane-rotated order (no bank conflicts)
+            float sl = -INFINITY;
+            if (lane < n) {
+                const unsigned char* krow = kst + lane * ROW;
+                float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int j = 0; j < CHUNK; ++j) {
-                float a = 0.f;
-                if (j < n) {
-                    Raw<T, DPL> kr;
-                    kr.load_shared(reinterpret_cast<const T*>(kst + j * ROW) + lane * DPL);
-#pragma unroll
-                    for (int e = 0; e < DPL; ++e) a = fmaf(qv[e], kr.get(e), a);
+                for (int cc = 0; cc < NPIECE; ++cc) {
+                    const int c = (cc + lane) & (NPIECE - 1);
+                    const uint4 kw = *reinterpret_cast<const uint4*>(krow + c * 16);
+                    if constexpr (sizeof(T) == 2) {
+                        const float4 qa = *reinterpret_cast<const float4*>(myq + c * 8);
+                        const float4 qb = *reinterpret_cast<const float4*>(myq + c * 8 + 4);
+                        a0 = fmaf(qa.x, bf16_lo(kw.x), a0);
+                        a1 = fmaf(qa.y, bf16_hi(kw.x), a1);
+                        a0 = fmaf(qa.z, bf16_lo(kw.y), a0);
+                        a1 = fmaf(qa.w, bf16_hi(kw.y), a1);
+                        a0 = fmaf(qb.x, bf16_lo(kw.z), a0);
+                        a1 = fmaf(qb.y, bf16_hi(kw.z), a1);
+                        a0 = fmaf(qb.z, bf16_lo(kw.w), a0);
+                        a1 = fmaf(qb.w, bf16_hi(kw.w), a1);
+                    } else {
+                        const float4 qa = *reinterpret_cast<const float4*>(myq + c * 4);
+                        a0 = fmaf(qa.x, __uint_as_float(kw.x), a0);
+                        a1 = fmaf(qa.y, __uint_as_float(kw.y), a1);
+                        a0 = fmaf(qa.z, __uint_as_float(kw.z), a0);
+                        a1 = fmaf(qa.w, __uint_as_float(kw.w), a1);
+                    }
                 }
-                part[j] = a;
+                sl = a0 + a1;
             }
-#pragma unroll
-            for (int w = 16; w >= 1; w >>= 1) {
-                const bool upper = lane & w;
-#pragma unroll
-                for (int e = 0; e < w; ++e) {
-                    const float send = upper ? part[e] : part[e + w];
-                    const float keep = upper ? part[e + w] : part[e];
-                    part[e] = keep + __shfl_xor_sync(FULL_MASK, send, w);
-                }
-            }
-            const float sl = lane < n ? part[0] : -INFINITY;
             const int64_t row0 = tb.slot0[hc] + tok0;
             if (tb.scoring[hc] && lane < n) L.logit[(size_t)(row0 + lane) * L.r + col] = sl;
             float cm = sl;
@@ -514,7 +525,7 @@ static DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
     const size_t fixed = HeadTable::bytes(L.S * L.H) + 128;
     DecodeShape sh{0, 0, 0};
     for (int ns = 3; ns >= 2 && sh.warps == 0; --ns) {
-        const size_t per = ns * (stage + 8);
+        const size_t per = ns * (stage + 8) + (size_t)L.d * 4;
         int w = smem_limit > fixed ? (int)((smem_limit - fixed) / per) : 0;
         if (w > 8) w = 8;
         if (w >= (ns == 3 ? 6 : 1)) sh = DecodeShape{w, ns, fixed + (size_t)w * per};
