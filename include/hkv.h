@@ -205,6 +205,40 @@ HKV_API hkv_status hkv_ste_select_batch(const float* score, const int32_t* pos, 
                                 int32_t k_near, int32_t k_far, int32_t stratified,
                                 uint8_t* evict, void* stream);
 
+/* ---- Allocation-free entry point ------------------------------------------ */
+
+/* Prefill attention and head grouping with no device allocation at all.
+ * The pages have no counterpart of this call: it exists for callers that
+ * cannot allocate device memory, not even the pool of hkv_create (code that
+ * runs during a global-mode CUDA graph capture, where cudaMalloc is refused;
+ * runtimes whose caching allocator owns all device memory; processes that
+ * may not allocate after start-up).  It computes, for n_blocks independent
+ * (sequence, head) blocks, what hkv_prefill_classify computes before it
+ * compresses anything: the causal attention outputs and each block's label.
+ *  q, k, v:  n_blocks blocks of [prefill_len][head_dim] elements of `dtype`,
+ *            block b at element b * block_stride (>= prefill_len * head_dim,
+ *            16-byte multiple); 16-byte aligned device pointers.
+ *  out:      [n_blocks][prefill_len][head_dim] outputs, or NULL.
+ *  n_tau:    int32[n_blocks] device output: tokens the backward accumulation
+ *            of the last query's weights needs to reach tau.
+ *  label:    uint8[n_blocks] device output: 1 (Local) iff n_tau < local_window.
+ *  status:   int32[2] device output (nullable): zeroed, then a device-side
+ *            fault (HKV_ERR_TIMEOUT, block index) if one occurs.
+ * Scratch: a fixed 8 MiB array inside the library, present on every GPU that
+ * loads it until the process exits.  Limit: n_blocks * prefill_len <=
+ * 2,097,088; larger calls return HKV_ERR_CAPACITY and enqueue nothing.  The
+ * first call on a device looks the array's address up and sets kernel
+ * attributes (host-side work): make it before any stream capture.  Every
+ * call reuses the same array, so calls that overlap on the GPU (other
+ * streams, other threads) race; order them.  Calls no cudaMalloc/cudaFree.
+ * Errors: INVALID_ARG, CAPACITY, CUDA. */
+HKV_API hkv_status hkv_prefill_classify_noalloc(int32_t dtype, int32_t head_dim, int32_t n_blocks,
+                                                const void* q, const void* k, const void* v,
+                                                int32_t prefill_len, int64_t block_stride,
+                                                int32_t local_window, double tau, void* out,
+                                                int32_t* n_tau, uint8_t* label, int32_t* status,
+                                                void* stream);
+
 #ifdef __cplusplus
 }
 #endif

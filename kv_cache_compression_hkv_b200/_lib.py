@@ -67,6 +67,7 @@ def lib():
             "hkv_reset": [P, P],
             "hkv_classify_rows": [P, I, I, I, D, P, P, P],
             "hkv_ste_select_batch": [P, P, P, P, I, I, I, I, I, I, P, P],
+            "hkv_prefill_classify_noalloc": [I, I, I, P, P, P, I, I64, I, D, P, P, P, P, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -287,3 +288,29 @@ def ste_select_batch(score: torch.Tensor, pos: torch.Tensor, count: torch.Tensor
                                       t.data_ptr(), n_probs, n, D, k_near, k_far, int(stratified),
                                       ev.data_ptr(), _stream(stream)), "hkv_ste_select_batch")
     return ev
+
+
+def prefill_classify_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, local_window: int,
+                             tau: float = 0.9, out: torch.Tensor | None = None, stream=None):
+    """Prefill attention + head grouping with no device allocation by the
+    library (see hkv_prefill_classify_noalloc).  q, k, v: [..., P, d] blocks
+    with unit stride in d, stride d in P and evenly spaced blocks.  Returns
+    (n_tau int32, label uint8, status int32[2]) device tensors; the caller's
+    tensors here are the outputs it passes."""
+    d, P = q.shape[-1], q.shape[-2]
+    nb = q.numel() // (P * d) if q.is_contiguous() else int(np.prod(q.shape[:-2]))
+    for x in (q, k, v):
+        if x.stride(-1) != 1 or x.stride(-2) != d or x.shape != q.shape or x.stride() != q.stride():
+            raise ValueError("q, k, v: unsupported layout")
+    bs = q.stride(-3) if q.dim() >= 3 else P * d
+    if q.dim() == 4 and q.stride(0) != q.shape[1] * q.stride(1):
+        raise ValueError("q, k, v: blocks must be evenly spaced")
+    dt = DTYPE_F32 if q.dtype == torch.float32 else DTYPE_BF16
+    n_tau = torch.empty(nb, dtype=torch.int32, device=q.device)
+    label = torch.empty(nb, dtype=torch.uint8, device=q.device)
+    status = torch.empty(2, dtype=torch.int32, device=q.device)
+    _check(lib().hkv_prefill_classify_noalloc(dt, d, nb, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                              P, bs, local_window, float(tau), _ptr(out),
+                                              n_tau.data_ptr(), label.data_ptr(), status.data_ptr(),
+                                              _stream(stream)), "hkv_prefill_classify_noalloc")
+    return n_tau, label, status

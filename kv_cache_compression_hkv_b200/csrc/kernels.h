@@ -21,6 +21,9 @@ cudaError_t launch_prefill(const Layout& L, int layer, const void* q, const void
                            int P, int64_t block_stride, void* out, cudaStream_t st);
 cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void* k, const void* v,
                           void* o, int append, int grid, cudaStream_t st);
+cudaError_t launch_prefill_rows_simt(int dtype, int d, int n_blocks, const void* q, const void* k,
+                                     const void* v, int P, int64_t block_stride, int r, void* out,
+                                     float* rows, cudaStream_t st);
 cudaError_t launch_append(const Layout& L, int layer, const void* k, const void* v, cudaStream_t st);
 cudaError_t launch_evict(const Layout& L, int l0, int l1, int grid, cudaStream_t st);
 cudaError_t launch_classify_rows(const float* rows, int n_rows, int n, int W, double tau,

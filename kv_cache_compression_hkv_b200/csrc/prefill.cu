@@ -253,6 +253,25 @@ cudaError_t launch_prefill(const Layout& L, int layer, const void* q, const void
     return cudaGetLastError();
 }
 
+// CUDA-core causal prefill of n_blocks caller blocks writing the weights of
+// their last r queries to `rows` ([n_blocks][r][P] fp32) and, if out is not
+// null, the outputs.  Used by the allocation-free entry point.
+cudaError_t launch_prefill_rows_simt(int dtype, int d, int n_blocks, const void* q, const void* k,
+                                     const void* v, int P, int64_t block_stride, int r, void* out,
+                                     float* rows, cudaStream_t st) {
+    dim3 grid(n_blocks, (P + 3) / 4);
+    const size_t sm = (size_t)4 * (d + P) * sizeof(float);
+    if (dtype == HKV_DTYPE_F32)
+        prefill_attn_simt<float><<<grid, 128, sm, st>>>((const float*)q, (const float*)k,
+                                                         (const float*)v, P, d, block_stride, r,
+                                                         (float*)out, rows);
+    else
+        prefill_attn_simt<__nv_bfloat16><<<grid, 128, sm, st>>>(
+            (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, P, d,
+            block_stride, r, (__nv_bfloat16*)out, rows);
+    return cudaGetLastError();
+}
+
 cudaError_t prepare_prefill(int smem) {
     cudaError_t e = allow_max_dynamic_smem(prefill_attn_simt<float>, smem);
     if (e == cudaSuccess) e = allow_max_dynamic_smem(pack_kernel<float>, smem);
