@@ -8,6 +8,7 @@ depend on which libcudart the Python process has loaded.
 """
 from __future__ import annotations
 
+import fcntl
 import glob
 import os
 import shutil
@@ -39,6 +40,13 @@ def _deps(src: str) -> list[str]:
 
 def build(verbose: bool = False, force: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
+    # one build at a time (parallel test workers may all ask for it)
+    with open(os.path.join(BUILD, ".lock"), "w") as lock:
+        fcntl.flock(lock, fcntl.LOCK_EX)
+        return _build_locked(verbose, force)
+
+
+def _build_locked(verbose: bool, force: bool) -> str:
     objs = []
     for src in sorted(glob.glob(os.path.join(CSRC, "*.cu"))):
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")

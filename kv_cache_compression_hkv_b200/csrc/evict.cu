@@ -2,7 +2,7 @@
 // summary, Methodology step 3, global heads) and the standalone grouping and
 // selection primitives.
 //
-// One warp per due head: it turns the logits the decode kernel stored over
+// One warp per due head (listed first by a scan): it turns the logits the decode kernel stored over
 // the last r steps into scores (summed softmax weights, each step normalised
 // by its own (max, sum) and counting only tokens already cached at that
 // step), selects the M/2 lowest (score, position) of the near and the far
@@ -21,8 +21,33 @@ __host__ __device__ inline size_t evict_warp_bytes(int n_max) {
     return select_scratch_bytes(n_max) + (size_t)round32(n_max) * 8 + 32 * 8;
 }
 
+// Lists the Global heads of layers [l0, l1) whose cache reached budget + M
+// (one thread per head; one atomic per warp).
+__global__ void __launch_bounds__(256) evict_scan_kernel(Layout L, int l0, int l1) {
+    const int n_heads = L.S * L.H;
+    const int total = (l1 - l0) * n_heads;
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    const int lane = threadIdx.x & 31;
+    bool due = false;
+    size_t hx = 0;
+    if (i < total && L.mode != HKV_MODE_FULL) {
+        const int l = l0 + i / n_heads;
+        hx = (size_t)l * n_heads + (i % n_heads);
+        due = L.label[hx] == 0 && len_at(L, hx, L.t_next[l] - 1) >= L.cap[hx];
+    }
+    const unsigned b = __ballot_sync(FULL_MASK, due);
+    if (!b) return;
+    const int leader = __ffs(b) - 1;  // every lane of the warp reaches here
+    int base = 0;
+    if (lane == leader) base = atomicAdd(L.due_ctl, __popc(b));
+    base = __shfl_sync(FULL_MASK, base, leader);
+    if (due) L.due_list[base + __popc(b & ((1u << lane) - 1u))] = (int)hx;
+}
+
+// Evicts every listed head, one warp per head: scores from the stored
+// logits, stratified select, compaction.  The last block clears the list.
 template <typename T>
-__global__ void __launch_bounds__(128) evict_kernel(Layout L, int l0, int l1, int n_max) {
+__global__ void __launch_bounds__(512) evict_run_kernel(Layout L, int n_max) {
     extern __shared__ __align__(16) unsigned char esm[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int NW = blockDim.x >> 5;
@@ -32,135 +57,133 @@ __global__ void __launch_bounds__(128) evict_kernel(Layout L, int l0, int l1, in
     int32_t* pos_s = reinterpret_cast<int32_t*>(sc_s + round32(n_max));
     float2* ml_s = reinterpret_cast<float2*>(pos_s + round32(n_max));
     const int n_heads = L.S * L.H;
-    const int total = (l1 - l0) * n_heads;
     const int d = L.d;
     const int r = L.r;
     T* Kp = reinterpret_cast<T*>(L.K);
     T* Vp = reinterpret_cast<T*>(L.V);
     constexpr int PIECE = 16 / sizeof(T);  // elements per 16-byte piece
     const int per_row = d / PIECE;
+    const int count = L.due_ctl[0];
 
-    for (int base = (blockIdx.x * NW + warp) * 32; base < total; base += gridDim.x * NW * 32) {
-        const int i = base + lane;
-        bool due = false;
-        if (i < total && L.mode != HKV_MODE_FULL) {
-            const int l = l0 + i / n_heads;
-            const size_t hx = (size_t)l * n_heads + (i % n_heads);
-            const int t = L.t_next[l] - 1;
-            due = L.label[hx] == 0 && len_at(L, hx, t) >= L.cap[hx];
+    for (int e = blockIdx.x * NW + warp; e < count; e += gridDim.x * NW) {
+        const size_t hx = (size_t)L.due_list[e];
+        const int l = (int)(hx / n_heads);
+        const int hs = (int)(hx % n_heads);
+        const int s = hs / L.H;
+        const int t = L.t_next[l] - 1;
+        const int n = len_at(L, hx, t);
+        const int target = L.budget[hx];
+        if (n > n_max || n != L.cap[hx]) {
+            if (lane == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
+            continue;
         }
-        unsigned todo = __ballot_sync(FULL_MASK, due);
-        while (todo) {
-            const int lead = __ffs(todo) - 1;
-            todo &= todo - 1;
-            const int j = base + lead;
-            const int l = l0 + j / n_heads;
-            const int hs = j % n_heads;
-            const int s = hs / L.H;
-            const size_t hx = (size_t)l * n_heads + hs;
-            const int t = L.t_next[l] - 1;
-            const int n = len_at(L, hx, t);
-            const int target = L.budget[hx];
-            if (n > n_max || n != L.cap[hx]) {
-                if (lane == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
-                continue;
-            }
-            const size_t slot0 = region_slot0(L, l, s) + L.off[hx];
-            // (max, sum) of each scoring step, by column = step mod r
-            if (lane < r) ml_s[lane] = L.ml[hx * r + lane];
-            __syncwarp();
-            // scores: summed softmax weight of the last r queries, each
-            // counting only tokens already cached at its step
-            bool bad = false;
+        const size_t slot0 = region_slot0(L, l, s) + L.off[hx];
+        // (max, 1/sum) of each scoring step, by column = step mod r
+        if (lane < r) {
+            const float2 ml = L.ml[hx * r + lane];
+            ml_s[lane] = make_float2(ml.x, 1.0f / ml.y);
+        }
+        __syncwarp();
+        // scores: summed softmax weight of the last r queries, each
+        // counting only tokens already cached at its step
+        bool bad = false;
 #pragma unroll 4
-            for (int q = lane; q < n; q += 32) {
-                const int p = L.pos[slot0 + q];
-                const float* lg = L.logit + (slot0 + q) * r;
-                float v[32];
-                if (r == 8) {
-                    const float4 a = *reinterpret_cast<const float4*>(lg);
-                    const float4 b = *reinterpret_cast<const float4*>(lg + 4);
-                    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-                    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-                } else {
+        for (int q = lane; q < n; q += 32) {
+            const int p = L.pos[slot0 + q];
+            const float* lg = L.logit + (slot0 + q) * r;
+            float v[32];
+            if (r == 8) {
+                const float4 a = *reinterpret_cast<const float4*>(lg);
+                const float4 b = *reinterpret_cast<const float4*>(lg + 4);
+                v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+                v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+            } else {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) if (c < r) v[c] = lg[c];
-                }
-                float acc = 0.f;
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    if (c >= r) break;
-                    const int step = t - (((t - c) % r) + r) % r;  // the window step of column c
-                    if (p <= step) acc += exp2f(v[c] - ml_s[c].x) / ml_s[c].y;
-                }
-                if (isnan(acc)) bad = true;
-                sc_s[q] = acc;
-                pos_s[q] = p;
+                for (int c = 0; c < 32; ++c) if (c < r) v[c] = lg[c];
             }
-            __syncwarp();
-            auto key_of = [&](int q, uint32_t& sb, int32_t& p) {
-                sb = __float_as_uint(sc_s[q]);
-                p = pos_s[q];
-            };
-            const int E = n - target;
-            warp_stratified_select(sc, n, t, L.D, E / 2, E - E / 2, L.stratified, key_of);
-            if (__any_sync(FULL_MASK, bad) && lane == 0) latch_error(L, HKV_ERR_NUMERIC, (int)hx);
-            // holes: evicted slots below the budget; movers: survivors above it
-            int nh = 0, nm = 0;
-            for (int b0 = 0; b0 < n; b0 += 32) {
-                const int q = b0 + lane;
-                const bool ev = q < n && ((sc.evict_bits[q >> 5] >> (q & 31)) & 1u);
-                const bool hole = q < target && ev;
-                const bool mover = q >= target && q < n && !ev;
-                const unsigned bh = __ballot_sync(FULL_MASK, hole);
-                const unsigned bm = __ballot_sync(FULL_MASK, mover);
-                const unsigned lt = (1u << lane) - 1u;
-                if (hole) sc.moves[nh + __popc(bh & lt)] = (uint16_t)q;
-                if (mover) sc.moves[sc.n_max - 1 - (nm + __popc(bm & lt))] = (uint16_t)q;
-                nh += __popc(bh);
-                nm += __popc(bm);
-            }
-            __syncwarp();
-            if (nh != nm) {
-                if (lane == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
-                continue;
-            }
-            // move rows: K and V in 16-byte pieces, eight per lane in flight
-            const int pieces = nh * per_row * 2;
-            for (int w0 = 0; w0 < pieces; w0 += 32 * 8) {
-                uint4 buf[8];
+            float acc = 0.f;
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int w = w0 + u * 32 + lane;
-                    if (w < pieces) {
-                        const int mv = w / (per_row * 2);
-                        const int rem = w % (per_row * 2);
-                        const bool isv = rem >= per_row;
-                        const int pc = (isv ? rem - per_row : rem) * PIECE;
-                        const size_t src = (slot0 + sc.moves[sc.n_max - 1 - mv]) * d + pc;
-                        buf[u] = *reinterpret_cast<const uint4*>((isv ? Vp : Kp) + src);
-                    }
-                }
+            for (int c = 0; c < 32; ++c) {
+                if (c >= r) break;
+                const int step = t - (((t - c) % r) + r) % r;  // the window step of column c
+                if (p <= step) acc += exp2f(v[c] - ml_s[c].x) * ml_s[c].y;
+            }
+            if (isnan(acc)) bad = true;
+            sc_s[q] = acc;
+            pos_s[q] = p;
+        }
+        __syncwarp();
+        auto key_of = [&](int q, uint32_t& sb, int32_t& p) {
+            sb = __float_as_uint(sc_s[q]);
+            p = pos_s[q];
+        };
+        const int E = n - target;
+        warp_stratified_select(sc, n, t, L.D, E / 2, E - E / 2, L.stratified, key_of);
+        if (__any_sync(FULL_MASK, bad) && lane == 0) latch_error(L, HKV_ERR_NUMERIC, (int)hx);
+        // holes: evicted slots below the budget; movers: survivors above it
+        int nh = 0, nm = 0;
+        for (int b0 = 0; b0 < n; b0 += 32) {
+            const int q = b0 + lane;
+            const bool ev = q < n && ((sc.evict_bits[q >> 5] >> (q & 31)) & 1u);
+            const bool hole = q < target && ev;
+            const bool mover = q >= target && q < n && !ev;
+            const unsigned bh = __ballot_sync(FULL_MASK, hole);
+            const unsigned bm = __ballot_sync(FULL_MASK, mover);
+            const unsigned lt = (1u << lane) - 1u;
+            if (hole) sc.moves[nh + __popc(bh & lt)] = (uint16_t)q;
+            if (mover) sc.moves[sc.n_max - 1 - (nm + __popc(bm & lt))] = (uint16_t)q;
+            nh += __popc(bh);
+            nm += __popc(bm);
+        }
+        __syncwarp();
+        if (nh != nm) {
+            if (lane == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
+            continue;
+        }
+        // move rows: K and V in 16-byte pieces, eight per lane in flight
+        const int pieces = nh * per_row * 2;
+        for (int w0 = 0; w0 < pieces; w0 += 32 * 8) {
+            uint4 buf[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int w = w0 + u * 32 + lane;
-                    if (w < pieces) {
-                        const int mv = w / (per_row * 2);
-                        const int rem = w % (per_row * 2);
-                        const bool isv = rem >= per_row;
-                        const int pc = (isv ? rem - per_row : rem) * PIECE;
-                        const size_t dst = (slot0 + sc.moves[mv]) * d + pc;
-                        *reinterpret_cast<uint4*>((isv ? Vp : Kp) + dst) = buf[u];
-                    }
+            for (int u = 0; u < 8; ++u) {
+                const int w = w0 + u * 32 + lane;
+                if (w < pieces) {
+                    const int mv = w / (per_row * 2);
+                    const int rem = w % (per_row * 2);
+                    const bool isv = rem >= per_row;
+                    const int pc = (isv ? rem - per_row : rem) * PIECE;
+                    const size_t src = (slot0 + sc.moves[sc.n_max - 1 - mv]) * d + pc;
+                    buf[u] = *reinterpret_cast<const uint4*>((isv ? Vp : Kp) + src);
                 }
             }
-            for (int mv = lane; mv < nh; mv += 32)
-                L.pos[slot0 + sc.moves[mv]] = pos_s[sc.moves[sc.n_max - 1 - mv]];
-            __syncwarp();
-            if (lane == 0) {
-                L.base_len[hx] = target;
-                L.base_t[hx] = t;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int w = w0 + u * 32 + lane;
+                if (w < pieces) {
+                    const int mv = w / (per_row * 2);
+                    const int rem = w % (per_row * 2);
+                    const bool isv = rem >= per_row;
+                    const int pc = (isv ? rem - per_row : rem) * PIECE;
+                    const size_t dst = (slot0 + sc.moves[mv]) * d + pc;
+                    *reinterpret_cast<uint4*>((isv ? Vp : Kp) + dst) = buf[u];
+                }
             }
+        }
+        for (int mv = lane; mv < nh; mv += 32)
+            L.pos[slot0 + sc.moves[mv]] = pos_s[sc.moves[sc.n_max - 1 - mv]];
+        __syncwarp();
+        if (lane == 0) {
+            L.base_len[hx] = target;
+            L.base_t[hx] = t;
+        }
+    }
+    // the last block out clears the list for the next step
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(L.due_ctl + 1, 1) == (int)gridDim.x - 1) {
+            L.due_ctl[0] = 0;
+            L.due_ctl[1] = 0;
         }
     }
 }
@@ -207,23 +230,27 @@ __global__ void __launch_bounds__(128) select_batch_kernel(
 static int evict_warps(int n_max) {
     const size_t per = evict_warp_bytes(n_max);
     int w = (int)((200 * 1024) / per);
-    return w < 1 ? 1 : (w > 4 ? 4 : w);
+    return w < 1 ? 1 : (w > 16 ? 16 : w);
 }
 
 cudaError_t launch_evict(const Layout& L, int l0, int l1, int grid, cudaStream_t st) {
+    const int heads = (l1 - l0) * L.S * L.H;
+    evict_scan_kernel<<<(heads + 255) / 256, 256, 0, st>>>(L, l0, l1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
     const int n_max = L.L;
     const int nw = evict_warps(n_max);
     const size_t sm = (size_t)nw * evict_warp_bytes(n_max);
     if (L.dtype == HKV_DTYPE_BF16)
-        evict_kernel<__nv_bfloat16><<<grid, 32 * nw, sm, st>>>(L, l0, l1, n_max);
+        evict_run_kernel<__nv_bfloat16><<<grid, 32 * nw, sm, st>>>(L, n_max);
     else
-        evict_kernel<float><<<grid, 32 * nw, sm, st>>>(L, l0, l1, n_max);
+        evict_run_kernel<float><<<grid, 32 * nw, sm, st>>>(L, n_max);
     return cudaGetLastError();
 }
 
 cudaError_t prepare_evict(int smem) {
-    cudaError_t e = allow_max_dynamic_smem(evict_kernel<__nv_bfloat16>, smem);
-    if (e == cudaSuccess) e = allow_max_dynamic_smem(evict_kernel<float>, smem);
+    cudaError_t e = allow_max_dynamic_smem(evict_run_kernel<__nv_bfloat16>, smem);
+    if (e == cudaSuccess) e = allow_max_dynamic_smem(evict_run_kernel<float>, smem);
     if (e == cudaSuccess) e = allow_max_dynamic_smem(select_batch_kernel, smem);
     return e;
 }

@@ -87,6 +87,7 @@ size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Lay
     l.t_next = (int32_t*)take(Ly * 4);
     l.done_ctr = (int32_t*)take(Ly * 4);
     l.ticket = (int32_t*)take(S * H * 4);
+    l.due_ctl = (int32_t*)take(16);
     const size_t ctrl_end = o;
     l.off = (int32_t*)take(nh * 4);
     l.cap = (int32_t*)take(nh * 4);
@@ -103,6 +104,7 @@ size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Lay
     l.ml = (float2*)take(nh * r * 8);
     l.rows = (float*)take(S * H * r * Lmax * 4);
     l.partial = (float*)take(max_chunks * (d + 2) * 4);
+    l.due_list = (int32_t*)take(nh * 4);
     l.S = c->num_seqs; l.Ly = c->num_layers; l.H = c->num_heads; l.d = c->head_dim;
     l.L = c->max_len; l.W = c->local_window; l.M = c->ste_m; l.D = c->near_dist;
     l.r = c->score_window; l.mode = c->mode; l.stratified = c->stratified; l.dtype = c->dtype;
@@ -113,12 +115,13 @@ size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Lay
 }
 
 size_t ctrl_bytes(const hkv_config* c) {
-    // status, t_next, done_ctr and ticket are laid out first (see carve)
+    // status, t_next, done_ctr, ticket and due_ctl are laid out first (see carve)
     size_t o = 0;
     o = align_up(o + 16);
     o = align_up(o + (size_t)c->num_layers * 4);
     o = align_up(o + (size_t)c->num_layers * 4);
     o = align_up(o + (size_t)c->num_seqs * c->num_heads * 4);
+    o = align_up(o + 16);
     return o;
 }
 

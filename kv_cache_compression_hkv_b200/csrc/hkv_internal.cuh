@@ -46,6 +46,8 @@ struct Layout {
     float* rows;        // [S*H][r][prefill_len] weights of the last r prefill queries
     float* partial;     // [max_chunks][d + 2] split-K partial states
     int32_t* ticket;    // [S*H] arrivals per head of the running decode launch
+    int32_t* due_ctl;   // [0] due heads listed, [1] blocks of the eviction done
+    int32_t* due_list;  // [Ly*S*H] heads due for eviction this step
     int32_t max_chunks;
 };
 
@@ -125,35 +127,37 @@ template <int DPL> struct RowSlice<__nv_bfloat16, DPL> {
 //
 // keys[i] = (bits(score) << 32) | position, score >= +0 so the bit pattern
 // orders like the value; the total order is (score, position), i.e. equal
-// scores evict the lower position first.  Finds the k-th smallest key of
-// keys[0..m) by bisection on the score bits, then on the positions of the
-// tied scores; returns it (every key <= it is evicted).  k >= 1, k <= m.
-// All 32 lanes must call it with the same arguments.
+// scores evict the lower position first.  The k-th smallest key of a set is
+// found by a 4-ary search on the score bits (three pivots per round), then,
+// only when scores tie at the boundary, by bisection on their positions.
+// Two independent sets (the near and the far stratum) are searched in the
+// same rounds.  Every key <= the returned threshold is evicted.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint64_t warp_kth_key(const uint64_t* keys, int m, int k) {
+struct KthSearch {
+    const uint64_t* keys;
+    int m, k;          // set size, rank wanted (1 <= k < m when active)
+    bool active;
+    uint32_t lo, hi;   // score bits of the k-th smallest lie in [lo, hi]
+    uint64_t thr;      // result
+};
+
+__device__ __forceinline__ void kth_round_update(KthSearch& s, uint32_t p1, uint32_t p2, uint32_t p3,
+                                                 unsigned c1, unsigned c2, unsigned c3) {
+    if ((int)c1 >= s.k) s.hi = p1;
+    else if ((int)c2 >= s.k) { s.lo = p1 + 1; s.hi = p2; }
+    else if ((int)c3 >= s.k) { s.lo = p2 + 1; s.hi = p3; }
+    else s.lo = p3 + 1;
+}
+
+// Resolves the position tie at score bits s.lo and sets s.thr.
+__device__ __forceinline__ void kth_finish(KthSearch& s) {
     const int lane = threadIdx.x & 31;
-    uint32_t lo = 0xffffffffu, hi = 0u;
-    for (int i = lane; i < m; i += 32) {
-        uint32_t sb = (uint32_t)(keys[i] >> 32);
-        lo = min(lo, sb);
-        hi = max(hi, sb);
-    }
-    lo = __reduce_min_sync(FULL_MASK, lo);
-    hi = __reduce_max_sync(FULL_MASK, hi);
-    // smallest score pattern s with #{score <= s} >= k
-    while (lo < hi) {
-        uint32_t mid = lo + ((hi - lo) >> 1);
-        unsigned c = 0;
-        for (int i = lane; i < m; i += 32) c += (uint32_t)(keys[i] >> 32) <= mid;
-        c = __reduce_add_sync(FULL_MASK, c);
-        if ((int)c >= k) hi = mid; else lo = mid + 1;
-    }
-    const uint32_t s_star = lo;
+    const uint32_t s_star = s.lo;
     unsigned c_lt = 0, c_eq = 0;
     uint32_t plo = 0xffffffffu, phi = 0u;
-    for (int i = lane; i < m; i += 32) {
-        uint32_t sb = (uint32_t)(keys[i] >> 32);
-        uint32_t p = (uint32_t)keys[i];
+    for (int i = lane; i < s.m; i += 32) {
+        const uint32_t sb = (uint32_t)(s.keys[i] >> 32);
+        const uint32_t p = (uint32_t)s.keys[i];
         c_lt += sb < s_star;
         if (sb == s_star) { ++c_eq; plo = min(plo, p); phi = max(phi, p); }
     }
@@ -161,20 +165,68 @@ __device__ __forceinline__ uint64_t warp_kth_key(const uint64_t* keys, int m, in
     c_eq = __reduce_add_sync(FULL_MASK, c_eq);
     plo = __reduce_min_sync(FULL_MASK, plo);
     phi = __reduce_max_sync(FULL_MASK, phi);
-    const int need = k - (int)c_lt;  // 1 <= need <= c_eq
+    const int need = s.k - (int)c_lt;  // 1 <= need <= c_eq
     if (need < (int)c_eq) {
         while (plo < phi) {
-            uint32_t mid = plo + ((phi - plo) >> 1);
+            const uint32_t mid = plo + ((phi - plo) >> 1);
             unsigned c = 0;
-            for (int i = lane; i < m; i += 32)
-                c += ((uint32_t)(keys[i] >> 32) == s_star) && ((uint32_t)keys[i] <= mid);
+            for (int i = lane; i < s.m; i += 32)
+                c += ((uint32_t)(s.keys[i] >> 32) == s_star) && ((uint32_t)s.keys[i] <= mid);
             c = __reduce_add_sync(FULL_MASK, c);
             if ((int)c >= need) phi = mid; else plo = mid + 1;
         }
     } else {
         plo = phi;  // every tied key goes
     }
-    return ((uint64_t)s_star << 32) | plo;
+    s.thr = ((uint64_t)s_star << 32) | plo;
+}
+
+// Threshold keys of two sets at once.  Inactive sets are skipped.
+__device__ inline void warp_kth_pair(KthSearch& a, KthSearch& b) {
+    const int lane = threadIdx.x & 31;
+    KthSearch* S[2] = {&a, &b};
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        KthSearch& s = *S[q];
+        uint32_t lo = 0xffffffffu, hi = 0u;
+        if (s.active)
+            for (int i = lane; i < s.m; i += 32) {
+                const uint32_t sb = (uint32_t)(s.keys[i] >> 32);
+                lo = min(lo, sb);
+                hi = max(hi, sb);
+            }
+        s.lo = __reduce_min_sync(FULL_MASK, lo);
+        s.hi = __reduce_max_sync(FULL_MASK, hi);
+        if (!s.active) s.lo = s.hi = 0;
+    }
+    const int mm = max(a.active ? a.m : 0, b.active ? b.m : 0);
+    while (a.lo < a.hi || b.lo < b.hi) {
+        const uint32_t a1 = a.lo + ((a.hi - a.lo) >> 2), a2 = a.lo + ((a.hi - a.lo) >> 1),
+                       a3 = a.lo + (uint32_t)(((uint64_t)(a.hi - a.lo) * 3) >> 2);
+        const uint32_t b1 = b.lo + ((b.hi - b.lo) >> 2), b2 = b.lo + ((b.hi - b.lo) >> 1),
+                       b3 = b.lo + (uint32_t)(((uint64_t)(b.hi - b.lo) * 3) >> 2);
+        unsigned ca1 = 0, ca2 = 0, ca3 = 0, cb1 = 0, cb2 = 0, cb3 = 0;
+        for (int i = lane; i < mm; i += 32) {
+            if (i < a.m && a.lo < a.hi) {
+                const uint32_t sb = (uint32_t)(a.keys[i] >> 32);
+                ca1 += sb <= a1; ca2 += sb <= a2; ca3 += sb <= a3;
+            }
+            if (i < b.m && b.lo < b.hi) {
+                const uint32_t sb = (uint32_t)(b.keys[i] >> 32);
+                cb1 += sb <= b1; cb2 += sb <= b2; cb3 += sb <= b3;
+            }
+        }
+        ca1 = __reduce_add_sync(FULL_MASK, ca1);
+        ca2 = __reduce_add_sync(FULL_MASK, ca2);
+        ca3 = __reduce_add_sync(FULL_MASK, ca3);
+        cb1 = __reduce_add_sync(FULL_MASK, cb1);
+        cb2 = __reduce_add_sync(FULL_MASK, cb2);
+        cb3 = __reduce_add_sync(FULL_MASK, cb3);
+        if (a.lo < a.hi) kth_round_update(a, a1, a2, a3, ca1, ca2, ca3);
+        if (b.lo < b.hi) kth_round_update(b, b1, b2, b3, cb1, cb2, cb3);
+    }
+    if (a.active) kth_finish(a);
+    if (b.active) kth_finish(b);
 }
 
 // Scratch of one warp's stratified select over up to n_max tokens.  The
@@ -258,13 +310,17 @@ __device__ int warp_stratified_select(const SelectScratch& sc, int n, int t, int
         kn = 0;
         if (kf > nf) kf = nf;
     }
+    // thresholds: none evicted (k <= 0), all evicted (k >= m), else searched
+    KthSearch a{sc.keys, nn, kn, kn > 0 && kn < nn, 0, 0, kn >= nn && kn > 0 ? ~0ull : 0ull};
+    KthSearch b{sc.keys + (n - nf), nf, kf, kf > 0 && kf < nf, 0, 0, kf >= nf && kf > 0 ? ~0ull : 0ull};
+    if (a.active || b.active) warp_kth_pair(a, b);
     for (int which = 0; which < 2; ++which) {
         const int k = which == 0 ? kn : kf;
         const int m = which == 0 ? nn : nf;
-        const uint64_t* keys = which == 0 ? sc.keys : sc.keys + (n - nf);
+        const uint64_t* keys = which == 0 ? a.keys : b.keys;
         const uint16_t* slots = which == 0 ? sc.slot : sc.slot + (n - nf);
+        const uint64_t thr = which == 0 ? a.thr : b.thr;
         if (k <= 0) continue;
-        const uint64_t thr = k >= m ? ~0ull : warp_kth_key(keys, m, k);
         for (int i = lane; i < m; i += 32)
             if (keys[i] <= thr) atomicOr(&sc.evict_bits[slots[i] >> 5], 1u << (slots[i] & 31));
     }
