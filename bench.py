@@ -346,7 +346,7 @@ def gpu_arm(args, rank, world, dev):
     # full-cache comparator (same kernels, no compression)
     if not args.no_full:
         cache_f = hkv.HeadKVCache(hkv.config_for(w, mode=hkv.MODE_FULL), device=dev)
-        g_full = capture(lambda: run_pass(cache_f, w, inp, outs, evict=False, pre_out=pre_out,
+        g_full = capture(lambda: run_pass(cache_f, w, inp, outs, pre_out=pre_out,
                                           hooks=hooks_main))
         for _ in range(2):
             g_full.replay()

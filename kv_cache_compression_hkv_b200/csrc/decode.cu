@@ -2,21 +2,21 @@
 // head-aware compressed cache (HeadKV technical summary: Problem statement;
 // Methodology step 3, Local sliding window and Global STE scoring).
 //
-// Work decomposition: every head's cache is cut into chunks of 32 tokens;
-// one warp owns one chunk.  A persistent grid walks the chunk list of the
-// layer (chunk counts prefix-summed per block from the device-side lengths,
-// so no host sync is needed).  Each warp computes its chunk's logits with a
-// lane-transposed reduction (lane j ends with token j's logit), its
-// softmax partial (max, sum, weighted V) and either finishes the head (one
-// chunk) or leaves a partial; the last warp to arrive for a head (atomic
-// ticket, no spinning) merges the partials.  Global heads within r steps of
-// their eviction also store their exp2-domain logits per slot, which the
-// eviction normalises with the (max, sum) stored here.
+// Work decomposition: every head's cache is cut into chunks of 32 tokens.
+// A plan (plan_kernel, once per step and layer) prefix-sums the heads' chunk
+// counts and cuts the layer's chunk list into equal contiguous ranges, one
+// per warp of the persistent decode grid.  Each warp walks its range with a
+// pipeline of shared-memory stages filled by per-lane 16-byte cp.async
+// copies, keeps the online softmax of the current head in registers across
+// that head's chunks, and finishes a head it holds entirely; a head split
+// between warps leaves one partial per warp and the last to arrive (atomic
+// ticket, no spinning) merges them.  Global heads within r steps of their
+// eviction also store their exp2-domain logits per slot, which the eviction
+// normalises with the (max, sum) stored here.
 #include <math.h>
 
 #include "hkv_internal.cuh"
 #include "kernels.h"
-#include "ptx.cuh"
 
 namespace hkv {
 
@@ -106,96 +106,6 @@ __device__ __forceinline__ void store_row(T* p, const float (&x)[DPL]) {
     }
 }
 
-// Per-head facts of one decode launch, cached in shared memory by every
-// block: inclusive prefix of chunk counts, slot offset in the layer, cache
-// length, slot of the appended token (-1: none) and whether the head records
-// STE logits this step.
-struct HeadTable {
-    int32_t* pre;
-    int64_t* slot0;
-    int16_t* len;
-    int16_t* jn;
-    uint8_t* scoring;
-    __host__ __device__ static size_t bytes(int n) { return (size_t)n * (4 + 8 + 2 + 2 + 1) + 64; }
-};
-
-__device__ HeadTable carve_table(unsigned char* p, int n) {
-    HeadTable t;
-    t.slot0 = reinterpret_cast<int64_t*>(p);
-    t.pre = reinterpret_cast<int32_t*>(t.slot0 + n);
-    t.len = reinterpret_cast<int16_t*>(t.pre + n);
-    t.jn = t.len + n;
-    t.scoring = reinterpret_cast<uint8_t*>(t.jn + n);
-    return t;
-}
-
-// Fills the table (coalesced, independent loads) and prefix-sums the chunk
-// counts; returns the layer's chunk count.  Heads past their capacity latch
-// HKV_ERR_CAPACITY and get no work.
-__device__ int build_table(const Layout& L, int layer, int t, int append, HeadTable tb) {
-    __shared__ int wsum[32];
-    const int n_heads = L.S * L.H;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int NW = blockDim.x >> 5;
-    const size_t hbase = (size_t)layer * n_heads;
-#pragma unroll 4
-    for (int i = tid; i < n_heads; i += blockDim.x) {
-        const size_t hx = hbase + i;
-        const int n = len_at(L, hx, t);
-        const int cap = L.cap[hx];
-        int c = (n + CHUNK - 1) / CHUNK;
-        if (n > cap || n < 1) {
-            if (blockIdx.x == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
-            c = 0;
-        }
-        tb.pre[i] = c;
-        tb.len[i] = (int16_t)n;
-        tb.slot0[i] = (int64_t)region_slot0(L, layer, i / L.H) + L.off[hx];
-        tb.jn[i] = (int16_t)(append ? append_slot(L, hx, t, n) : -1);
-        tb.scoring[i] = L.label[hx] == 0 && L.mode != HKV_MODE_FULL && n > cap - L.r;
-    }
-    __syncthreads();
-    const int per = (n_heads + blockDim.x - 1) / blockDim.x;
-    const int i0 = min(tid * per, n_heads), i1 = min(i0 + per, n_heads);
-    int local = 0;
-    for (int i = i0; i < i1; ++i) {
-        local += tb.pre[i];
-        tb.pre[i] = local;
-    }
-    int x = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        int y = __shfl_up_sync(FULL_MASK, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) wsum[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        int w = lane < NW ? wsum[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            int y = __shfl_up_sync(FULL_MASK, w, o);
-            if (lane >= o) w += y;
-        }
-        wsum[lane] = w;
-    }
-    __syncthreads();
-    const int offset = x - local + (warp ? wsum[warp - 1] : 0);
-    for (int i = i0; i < i1; ++i) tb.pre[i] += offset;
-    __syncthreads();
-    return tb.pre[n_heads - 1];
-}
-
-// Head holding chunk c: smallest h with pre[h] > c.
-__device__ __forceinline__ int head_of(const int32_t* pre, int n, int c) {
-    int lo = 0, hi = n - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (pre[mid] > c) hi = mid; else lo = mid + 1;
-    }
-    return lo;
-}
-
 // First chunk of warp w's range when `total` chunks go to `gw` warps.
 __device__ __forceinline__ int range_begin(int w, int total, int gw) {
     return (int)((int64_t)w * total / gw);
@@ -205,6 +115,123 @@ __device__ __forceinline__ int range_owner(int c, int total, int gw) {
     return (int)(((int64_t)(c + 1) * gw - 1) / total);
 }
 
+// ---------------------------------------------------------------------------
+// The plan of a layer's decode launch at step t (ahead = 1: the step of the
+// next append, t_next; ahead = 0: the newest cached position, t_next - 1).
+// One block per layer: per-head facts, the chunk-count prefix, and for every
+// warp of the decode grid its first chunk and the head holding it.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead) {
+    extern __shared__ int32_t cnt[];
+    __shared__ int wsum[32];
+    const int layer = l0 + blockIdx.x;
+    const int n = L.S * L.H;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, NW = blockDim.x >> 5;
+    const int t = L.t_next[layer] - 1 + ahead;
+    const size_t hbase = (size_t)layer * n;
+    for (int i = tid; i < n; i += blockDim.x) {
+        const size_t hx = hbase + i;
+        const int len = len_at(L, hx, t);
+        const int cap = L.cap[hx];
+        int c = (len + CHUNK - 1) / CHUNK;
+        if (len > cap || len < 1) {
+            latch_error(L, HKV_ERR_CAPACITY, (int)hx);
+            c = 0;
+        }
+        const int jn = append_slot(L, hx, t, len);
+        const int scoring = L.label[hx] == 0 && L.mode != HKV_MODE_FULL && len > cap - L.r;
+        const int slot = (i / L.H) * L.R + L.off[hx];
+        L.plan_head[hbase + i] = make_int4(slot, (len << 16) | (jn & 0xffff), scoring, 0);
+        cnt[i] = c;
+    }
+    __syncthreads();
+    // inclusive scan: contiguous runs per thread, then the warps
+    const int per = (n + blockDim.x - 1) / blockDim.x;
+    const int i0 = min(tid * per, n), i1 = min(i0 + per, n);
+    int local = 0;
+    for (int i = i0; i < i1; ++i) { local += cnt[i]; cnt[i] = local; }
+    int x = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(FULL_MASK, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < NW ? wsum[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(FULL_MASK, w, o);
+            if (lane >= o) w += y;
+        }
+        wsum[lane] = w;
+    }
+    __syncthreads();
+    const int offset = x - local + (warp ? wsum[warp - 1] : 0);
+    for (int i = i0; i < i1; ++i) cnt[i] += offset;
+    __syncthreads();
+    const int total = cnt[n - 1];
+    for (int i = tid; i < n; i += blockDim.x) L.plan_pre[hbase + i] = cnt[i];
+    const int GW = L.plan_gw;
+    int32_t* pw = L.plan_warp + (size_t)layer * (PLAN_MAX_WARPS + 1);
+    int32_t* ph = L.plan_whead + (size_t)layer * PLAN_MAX_WARPS;
+    for (int w = tid; w <= GW; w += blockDim.x) {
+        const int cb = range_begin(w, total, GW);
+        pw[w] = cb;
+        if (w < GW) {
+            int lo = 0, hi = n - 1;  // head holding chunk cb
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (cnt[mid] > cb) hi = mid; else lo = mid + 1;
+            }
+            ph[w] = lo;
+        }
+    }
+}
+
+// Head facts of the 32 heads [base, base + 32) of a layer, lane i holding
+// head base + i.
+struct HeadCache {
+    int base;
+    int slot, lenjn, scoring, pre, first;
+    __device__ void load(const Layout& L, size_t hbase, int n, int b) {
+        const int lane = threadIdx.x & 31;
+        base = b;
+        const int h = b + lane;
+        if (h < n) {
+            const int4 v = L.plan_head[hbase + h];
+            slot = v.x; lenjn = v.y; scoring = v.z;
+            pre = L.plan_pre[hbase + h];
+            first = h ? L.plan_pre[hbase + h - 1] : 0;
+        } else {
+            slot = 0; lenjn = 0; scoring = 0; pre = 0x7fffffff; first = 0x7fffffff;
+        }
+    }
+    // facts of head h (base <= h < base + 32), broadcast to every lane
+    __device__ void get(int h, int& o_slot, int& o_len, int& o_jn, int& o_scoring, int& o_pre,
+                        int& o_first) const {
+        const int src = h - base;
+        o_slot = __shfl_sync(FULL_MASK, slot, src);
+        const int lj = __shfl_sync(FULL_MASK, lenjn, src);
+        o_len = lj >> 16;
+        o_jn = (int)(int16_t)(lj & 0xffff);
+        o_scoring = __shfl_sync(FULL_MASK, scoring, src);
+        o_pre = __shfl_sync(FULL_MASK, pre, src);
+        o_first = __shfl_sync(FULL_MASK, first, src);
+    }
+};
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                     (uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 template <typename T, int DPL>
 __global__ void __launch_bounds__(256, 1)
     decode_kernel(Layout L, int layer, const T* __restrict__ q_t, const T* __restrict__ k_t,
@@ -213,94 +240,95 @@ __global__ void __launch_bounds__(256, 1)
     const int n_heads = L.S * L.H;
     constexpr int D = DPL * 32;
     constexpr int ROW = D * (int)sizeof(T);           // bytes of one cache row
-    constexpr int STAGE = (2 * CHUNK + 1) * ROW;       // K rows, V rows, the query
+    constexpr int PPR = ROW / 16;                     // 16-byte pieces per row
+    constexpr int STAGE = (2 * CHUNK + 1) * ROW;      // K rows, V rows, the query
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int NW = blockDim.x >> 5;
     const int t = append ? L.t_next[layer] : L.t_next[layer] - 1;
     const int col = t % L.r;
-
-    unsigned char* stages = dsm;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(stages + (size_t)NW * nstage * STAGE);
-    float* qbuf = reinterpret_cast<float*>(                     // [NW][D] fp32 queries
-        ((uintptr_t)(bars + NW * nstage) + 15) & ~(uintptr_t)15);
-    HeadTable tb = carve_table(reinterpret_cast<unsigned char*>(qbuf + NW * D), n_heads);
-    const int total = build_table(L, layer, t, append, tb);
-    constexpr int NPIECE = ROW / 16;  // 16-byte pieces per row
-
     const int GW = gridDim.x * NW;
     const int gw = blockIdx.x * NW + warp;
-    const int c_begin = total > 0 ? range_begin(gw, total, GW) : 0;
-    const int c_end = total > 0 ? range_begin(gw + 1, total, GW) : 0;
+    const size_t hbase = (size_t)layer * n_heads;
+    const size_t lrow = (size_t)layer * L.S * L.R;    // first slot of the layer
     T* Kp = reinterpret_cast<T*>(L.K);
     T* Vp = reinterpret_cast<T*>(L.V);
-    const size_t hbase = (size_t)layer * n_heads;
     const float qscale = LOG2E / sqrtf((float)D);
-    constexpr uint64_t WAIT_NS = 2000000000ull;
+
+    if (GW != L.plan_gw) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) latch_error(L, HKV_ERR_STATE, layer);
+        return;
+    }
+    const int32_t* pw = L.plan_warp + (size_t)layer * (PLAN_MAX_WARPS + 1);
+    const int c_begin = pw[gw], c_end = pw[gw + 1], total = pw[GW];
+
+    unsigned char* my = dsm + (size_t)warp * nstage * STAGE;
+    float* myq = reinterpret_cast<float*>(dsm + (size_t)NW * nstage * STAGE) + warp * D;
 
     if (c_begin < c_end) {
-        unsigned char* my = stages + (size_t)warp * nstage * STAGE;
-        uint64_t* bar = bars + warp * nstage;
-        float* myq = qbuf + warp * D;
-        if (lane == 0) {
-            for (int s = 0; s < nstage; ++s) ptx::mbar_init(bar + s, 1);
-            ptx::fence_mbar_init();
-        }
-        __syncwarp();
+        const int h_begin = L.plan_whead[(size_t)layer * PLAN_MAX_WARPS + gw];
+        HeadCache pc, cc;  // producer's and consumer's view of the heads
+        pc.load(L, hbase, n_heads, h_begin);
+        cc = pc;
 
-        // producer cursor (lane 0 issues): chunk ip of head hp
-        int ip = c_begin, hp = head_of(tb.pre, n_heads, c_begin);
+        // producer cursor: chunk ip of head hp
+        int ip = c_begin, hp = h_begin;
         auto issue = [&](int stage) {
-            if (lane == 0) {
-                const int first = hp ? tb.pre[hp - 1] : 0;
-                const int tok0 = (ip - first) * CHUNK;
-                const int n = min(CHUNK, (int)tb.len[hp] - tok0);
-                const int jn = tb.jn[hp];
-                const size_t row0 = (size_t)tb.slot0[hp] + tok0;
-                unsigned char* kd = my + (size_t)stage * STAGE;
-                unsigned char* vd = kd + CHUNK * ROW;
-                unsigned char* qd = vd + CHUNK * ROW;
-                uint64_t* b = bar + stage;
-                ptx::mbar_expect_tx(b, (uint32_t)(2 * n + 1) * ROW);
-                ptx::bulk_g2s(qd, q_t + (size_t)hp * D, ROW, b);
-                const int a = jn - tok0;
-                if (a >= 0 && a < n) {
-                    if (a > 0) {
-                        ptx::bulk_g2s(kd, Kp + row0 * D, a * ROW, b);
-                        ptx::bulk_g2s(vd, Vp + row0 * D, a * ROW, b);
-                    }
-                    ptx::bulk_g2s(kd + a * ROW, k_t + (size_t)hp * D, ROW, b);
-                    ptx::bulk_g2s(vd + a * ROW, v_t + (size_t)hp * D, ROW, b);
-                    if (n - a - 1 > 0) {
-                        ptx::bulk_g2s(kd + (a + 1) * ROW, Kp + (row0 + a + 1) * D, (n - a - 1) * ROW, b);
-                        ptx::bulk_g2s(vd + (a + 1) * ROW, Vp + (row0 + a + 1) * D, (n - a - 1) * ROW, b);
-                    }
-                } else {
-                    ptx::bulk_g2s(kd, Kp + row0 * D, n * ROW, b);
-                    ptx::bulk_g2s(vd, Vp + row0 * D, n * ROW, b);
-                }
+            int slot, len, jn, sc_, pre, first;
+            if (hp - pc.base >= 32) pc.load(L, hbase, n_heads, hp);
+            pc.get(hp, slot, len, jn, sc_, pre, first);
+            const int tok0 = (ip - first) * CHUNK;
+            const int n = min(CHUNK, len - tok0);
+            const int a = jn - tok0;  // appended row within the chunk (or outside)
+            const size_t row0 = lrow + slot + tok0;
+            unsigned char* kd = my + (size_t)stage * STAGE;
+            unsigned char* vd = kd + CHUNK * ROW;
+            unsigned char* qd = vd + CHUNK * ROW;
+            const int pieces = n * PPR;
+            for (int p = lane; p < pieces; p += 32) {
+                const int row = p / PPR, c = p % PPR;
+                const bool fresh = append && row == a;
+                const T* ks = (fresh ? k_t + (size_t)hp * D : Kp + (row0 + row) * D) + c * (16 / (int)sizeof(T));
+                const T* vs = (fresh ? v_t + (size_t)hp * D : Vp + (row0 + row) * D) + c * (16 / (int)sizeof(T));
+                cp_async16(kd + row * ROW + c * 16, ks);
+                cp_async16(vd + row * ROW + c * 16, vs);
             }
+            for (int c = lane; c < PPR; c += 32)
+                cp_async16(qd + c * 16, q_t + (size_t)hp * D + c * (16 / (int)sizeof(T)));
+            cp_async_commit();
             ++ip;
-            if (ip < c_end && tb.pre[hp] <= ip) hp = head_of(tb.pre, n_heads, ip);
+            if (ip < c_end && pre <= ip) ++hp;
+            while (ip < c_end) {  // skip heads with no chunk (capacity errors)
+                if (hp - pc.base >= 32) pc.load(L, hbase, n_heads, hp);
+                int s2, l2, j2, c2, p2, f2;
+                pc.get(hp, s2, l2, j2, c2, p2, f2);
+                if (p2 > ip) break;
+                ++hp;
+            }
         };
         for (int s = 0; s < nstage && ip < c_end; ++s) issue(s);
 
-        int hc = head_of(tb.pre, n_heads, c_begin);
+        int hc = h_begin;
         int seg0 = c_begin;
         float m = -INFINITY, l = 0.f, acc[DPL];
 #pragma unroll
         for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-        bool failed = false;
+        int slot, len, jn, scoring, pre, first;
+        cc.get(hc, slot, len, jn, scoring, pre, first);
+        while (pre <= c_begin) {  // heads with no chunk before the first one
+            ++hc;
+            if (hc - cc.base >= 32) cc.load(L, hbase, n_heads, hc);
+            cc.get(hc, slot, len, jn, scoring, pre, first);
+        }
 
         for (int i = c_begin; i < c_end; ++i) {
             const int k = i - c_begin;
             const int stage = k % nstage;
-            if (!ptx::mbar_wait(bar + stage, (uint32_t)((k / nstage) & 1), WAIT_NS)) {
-                failed = true;
-                break;
-            }
-            const int first = hc ? tb.pre[hc - 1] : 0;
+            const int pending = (ip - c_begin) - (k + 1);  // groups issued after this one
+            if (pending >= 2) cp_async_wait<2>();
+            else if (pending == 1) cp_async_wait<1>();
+            else cp_async_wait<0>();
+            __syncwarp();
             const int tok0 = (i - first) * CHUNK;
-            const int len = tb.len[hc];
             const int n = min(CHUNK, len - tok0);
             const unsigned char* kst = my + (size_t)stage * STAGE;
             const unsigned char* vst = kst + CHUNK * ROW;
@@ -320,8 +348,8 @@ __global__ void __launch_bounds__(256, 1)
                 const unsigned char* krow = kst + lane * ROW;
                 float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-                for (int cc = 0; cc < NPIECE; ++cc) {
-                    const int c = (cc + lane) & (NPIECE - 1);
+                for (int c2 = 0; c2 < PPR; ++c2) {
+                    const int c = (c2 + lane) & (PPR - 1);
                     const uint4 kw = *reinterpret_cast<const uint4*>(krow + c * 16);
                     if constexpr (sizeof(T) == 2) {
                         const float4 qa = *reinterpret_cast<const float4*>(myq + c * 8);
@@ -344,8 +372,8 @@ __global__ void __launch_bounds__(256, 1)
                 }
                 sl = a0 + a1;
             }
-            const int64_t row0 = tb.slot0[hc] + tok0;
-            if (tb.scoring[hc] && lane < n) L.logit[(size_t)(row0 + lane) * L.r + col] = sl;
+            const size_t row0 = lrow + slot + tok0;
+            if (scoring && lane < n) L.logit[(row0 + lane) * L.r + col] = sl;
             float cm = sl;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(FULL_MASK, cm, o));
@@ -370,33 +398,30 @@ __global__ void __launch_bounds__(256, 1)
                 }
             }
             // the appended token joins the cache
-            const int a = tb.jn[hc] - tok0;
-            if (a >= 0 && a < n) {
+            const int a = jn - tok0;
+            if (append && a >= 0 && a < n) {
                 Raw<T, DPL> kr, vr;
                 kr.load_shared(reinterpret_cast<const T*>(kst + a * ROW) + lane * DPL);
                 vr.load_shared(reinterpret_cast<const T*>(vst + a * ROW) + lane * DPL);
-                kr.store(Kp + (size_t)(row0 + a) * D + lane * DPL);
-                vr.store(Vp + (size_t)(row0 + a) * D + lane * DPL);
+                kr.store(Kp + (row0 + a) * D + lane * DPL);
+                vr.store(Vp + (row0 + a) * D + lane * DPL);
                 if (lane == 0) L.pos[row0 + a] = t;
             }
             __syncwarp();
-            if (ip < c_end) {
-                ptx::fence_proxy_async();  // this stage's reads before its refill
-                issue(stage);
-            }
-            if (i + 1 < c_end && tb.pre[hc] > i + 1) continue;  // head goes on
+            if (ip < c_end) issue(stage);
+            if (i + 1 < c_end && pre > i + 1) continue;  // head goes on
 
             // end of this warp's segment of head hc
             const size_t hx = hbase + hc;
             if (!(l > 0.f) || isinf(l)) latch_error(L, HKV_ERR_NUMERIC, (int)hx);
-            const bool whole = seg0 == first && i + 1 == tb.pre[hc];
+            const bool whole = seg0 == first && i + 1 == pre;
             if (whole) {
                 const float inv = 1.0f / l;
                 float o[DPL];
 #pragma unroll
                 for (int e = 0; e < DPL; ++e) o[e] = acc[e] * inv;
                 store_row<T, DPL>(o_t + (size_t)hc * D + lane * DPL, o);
-                if (tb.scoring[hc] && lane == 0) L.ml[hx * L.r + col] = make_float2(m, l);
+                if (scoring && lane == 0) L.ml[hx * L.r + col] = make_float2(m, l);
             } else {
                 float* pp = L.partial + (size_t)seg0 * (D + 2);
                 if (lane == 0) { pp[0] = m; pp[1] = l; }
@@ -404,7 +429,7 @@ __global__ void __launch_bounds__(256, 1)
                 for (int e = 0; e < DPL; ++e) pp[2 + lane * DPL + e] = acc[e];
                 __threadfence();
                 const int w_a = range_owner(first, total, GW);
-                const int w_b = range_owner(tb.pre[hc] - 1, total, GW);
+                const int w_b = range_owner(pre - 1, total, GW);
                 int segs = 0;
                 for (int w = w_a; w <= w_b; ++w)
                     segs += range_begin(w, total, GW) < range_begin(w + 1, total, GW);
@@ -439,27 +464,24 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
                     for (int e = 0; e < DPL; ++e) o[e] *= inv;
                     store_row<T, DPL>(o_t + (size_t)hc * D + lane * DPL, o);
-                    if (tb.scoring[hc] && lane == 0) L.ml[hx * L.r + col] = make_float2(M, Ls);
+                    if (scoring && lane == 0) L.ml[hx * L.r + col] = make_float2(M, Ls);
                 }
             }
-            // next head
+            // next head holding chunk i + 1
             seg0 = i + 1;
-            if (i + 1 < c_end) hc = head_of(tb.pre, n_heads, i + 1);
             m = -INFINITY;
             l = 0.f;
 #pragma unroll
             for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-        }
-        if (failed) {
-            if (lane == 0) latch_error(L, HKV_ERR_TIMEOUT, (int)(hbase + hc));
-            // let this warp's outstanding copies land before the block exits
-            for (int k = 0; k < nstage; ++k) {
-                const int j = ip - 1 - k;
-                if (j < c_begin) break;
-                const int kk = j - c_begin;
-                ptx::mbar_wait(bar + kk % nstage, (uint32_t)((kk / nstage) & 1), WAIT_NS);
+            if (i + 1 < c_end) {
+                do {
+                    ++hc;
+                    if (hc - cc.base >= 32) cc.load(L, hbase, n_heads, hc);
+                    cc.get(hc, slot, len, jn, scoring, pre, first);
+                } while (pre <= i + 1);
             }
         }
+        cp_async_wait<0>();
     }
     if (append) {
         __syncthreads();
@@ -512,54 +534,44 @@ __global__ void __launch_bounds__(256) append_kernel(Layout L, int layer, const 
 // launchers
 // ---------------------------------------------------------------------------
 
-// Launch shape of the decode kernel: warps per block and pipeline stages per
-// warp that fit the shared memory next to the head table.
-struct DecodeShape {
-    int warps, nstage;
-    size_t smem;
-};
-
-static DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
+DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
     const size_t row = (size_t)L.d * (L.dtype == HKV_DTYPE_F32 ? 4 : 2);
     const size_t stage = (2 * CHUNK + 1) * row;
-    const size_t fixed = HeadTable::bytes(L.S * L.H) + 128;
     DecodeShape sh{0, 0, 0};
     for (int ns = 3; ns >= 2 && sh.warps == 0; --ns) {
-        const size_t per = ns * (stage + 8) + (size_t)L.d * 4;
-        int w = smem_limit > fixed ? (int)((smem_limit - fixed) / per) : 0;
+        const size_t per = ns * stage + (size_t)L.d * 4;
+        int w = (int)((smem_limit - 1024) / per);
         if (w > 8) w = 8;
-        if (w >= (ns == 3 ? 6 : 1)) sh = DecodeShape{w, ns, fixed + (size_t)w * per};
+        if (w >= (ns == 3 ? 6 : 1)) sh = DecodeShape{w, ns, 1024 + (size_t)w * per};
     }
     return sh;
 }
 
 template <typename T, int DPL>
 static cudaError_t launch_decode_t(const Layout& L, int layer, const void* q, const void* k,
-                                   const void* v, void* o, int append, int grid, cudaStream_t st) {
-    static size_t limit = 0;
-    if (!limit) {
-        int dev = 0, optin = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-        limit = (size_t)optin - 256;  // room for the kernel's static shared memory
-    }
-    const DecodeShape sh = decode_shape(L, limit);
-    if (sh.warps == 0) return cudaErrorInvalidConfiguration;
-    decode_kernel<T, DPL><<<grid, 32 * sh.warps, sh.smem, st>>>(L, layer, (const T*)q, (const T*)k,
-                                                                (const T*)v, (T*)o, append, sh.nstage);
+                                   const void* v, void* o, int append, const DecodeShape& sh,
+                                   int grid, cudaStream_t st) {
+    decode_kernel<T, DPL><<<grid, 32 * sh.warps, sh.smem, st>>>(
+        L, layer, (const T*)q, (const T*)k, (const T*)v, (T*)o, append, sh.nstage);
     return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void* k, const void* v,
-                          void* o, int append, int grid, cudaStream_t st) {
+                          void* o, int append, const DecodeShape& sh, int grid, cudaStream_t st) {
     if (L.dtype == HKV_DTYPE_BF16) {
-        if (L.d == 64) return launch_decode_t<__nv_bfloat16, 2>(L, layer, q, k, v, o, append, grid, st);
-        if (L.d == 128) return launch_decode_t<__nv_bfloat16, 4>(L, layer, q, k, v, o, append, grid, st);
+        if (L.d == 64) return launch_decode_t<__nv_bfloat16, 2>(L, layer, q, k, v, o, append, sh, grid, st);
+        if (L.d == 128) return launch_decode_t<__nv_bfloat16, 4>(L, layer, q, k, v, o, append, sh, grid, st);
     } else {
-        if (L.d == 64) return launch_decode_t<float, 2>(L, layer, q, k, v, o, append, grid, st);
-        if (L.d == 128) return launch_decode_t<float, 4>(L, layer, q, k, v, o, append, grid, st);
+        if (L.d == 64) return launch_decode_t<float, 2>(L, layer, q, k, v, o, append, sh, grid, st);
+        if (L.d == 128) return launch_decode_t<float, 4>(L, layer, q, k, v, o, append, sh, grid, st);
     }
     return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_plan(const Layout& L, int l0, int l1, int ahead, cudaStream_t st) {
+    const size_t sm = (size_t)L.S * L.H * sizeof(int32_t);
+    plan_kernel<<<l1 - l0, 1024, sm, st>>>(L, l0, ahead);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_append(const Layout& L, int layer, const void* k, const void* v, cudaStream_t st) {
@@ -580,6 +592,7 @@ cudaError_t prepare_decode(int smem) {
     if (e == cudaSuccess) e = allow_max_dynamic_smem(decode_kernel<__nv_bfloat16, 4>, smem);
     if (e == cudaSuccess) e = allow_max_dynamic_smem(decode_kernel<float, 2>, smem);
     if (e == cudaSuccess) e = allow_max_dynamic_smem(decode_kernel<float, 4>, smem);
+    if (e == cudaSuccess) e = allow_max_dynamic_smem(plan_kernel, smem);
     return e;
 }
 

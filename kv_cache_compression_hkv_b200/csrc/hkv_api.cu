@@ -20,6 +20,8 @@ struct hkv_ctx {
     int n_sm;
     int decode_grid;
     int evict_grid;
+    hkv::DecodeShape decode_sh;
+    std::vector<int> plan_for;    // per layer: step its decode plan was made for (-1: none)
     int64_t t_total;
     std::vector<int> classified;  // per layer
     std::vector<int> t_host;      // per layer: next position, as enqueued by API calls
@@ -105,6 +107,10 @@ size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Lay
     l.rows = (float*)take(S * H * r * Lmax * 4);
     l.partial = (float*)take(max_chunks * (d + 2) * 4);
     l.due_list = (int32_t*)take(nh * 4);
+    l.plan_pre = (int32_t*)take(nh * 4);
+    l.plan_head = (int4*)take(nh * 16);
+    l.plan_warp = (int32_t*)take(Ly * (hkv::PLAN_MAX_WARPS + 1) * 4);
+    l.plan_whead = (int32_t*)take(Ly * hkv::PLAN_MAX_WARPS * 4);
     l.S = c->num_seqs; l.Ly = c->num_layers; l.H = c->num_heads; l.d = c->head_dim;
     l.L = c->max_len; l.W = c->local_window; l.M = c->ste_m; l.D = c->near_dist;
     l.r = c->score_window; l.mode = c->mode; l.stratified = c->stratified; l.dtype = c->dtype;
@@ -182,8 +188,17 @@ hkv_status hkv_create(const hkv_config* cfg, void* pool, size_t bytes, void* str
         delete c;
         return HKV_ERR_CUDA;
     }
-    c->decode_grid = c->n_sm;      // one 256-thread block per SM (register-bound)
-    c->evict_grid = c->n_sm * 2;
+    int optin = 0;
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, c->device);
+    c->decode_sh = hkv::decode_shape(c->lay, (size_t)optin - 256);
+    c->decode_grid = c->n_sm;  // persistent: one block per SM
+    if (c->decode_sh.warps == 0 || c->decode_grid * c->decode_sh.warps > hkv::PLAN_MAX_WARPS) {
+        delete c;
+        return HKV_ERR_INVALID_ARG;
+    }
+    c->lay.plan_gw = c->decode_grid * c->decode_sh.warps;
+    c->plan_for.assign(cfg->num_layers, -1);
+    c->evict_grid = c->n_sm;
     *out = c;
     return HKV_OK;
 }
@@ -206,7 +221,9 @@ hkv_status hkv_prefill_classify(hkv_ctx* c, int32_t layer, const void* q, const 
     if (hkv::pack_smem_bytes(P) > 200 * 1024) return HKV_ERR_INVALID_ARG;
     cudaError_t e = hkv::launch_prefill(c->lay, layer, q, k, v, P, block_stride, out,
                                         (cudaStream_t)stream);
+    if (e == cudaSuccess) e = hkv::launch_plan(c->lay, layer, layer + 1, 1, (cudaStream_t)stream);
     if (e != cudaSuccess) return HKV_ERR_CUDA;
+    c->plan_for[layer] = P;
     c->classified[layer] = 1;
     c->t_host[layer] = P;
     c->prefill_len[layer] = P;
@@ -235,8 +252,16 @@ hkv_status hkv_decode_attend(hkv_ctx* c, int32_t layer, const void* q_t, void* o
     hkv_status s = step_check(c, layer, false);
     if (s != HKV_OK) return s;
     if (!q_t || !o_t || !aligned16(q_t) || !aligned16(o_t)) return HKV_ERR_INVALID_ARG;
-    return cuda_status(hkv::launch_decode(c->lay, layer, q_t, nullptr, nullptr, o_t, 0,
-                                          c->decode_grid, (cudaStream_t)stream));
+    const int t = c->t_host[layer] - 1;  // newest cached position
+    cudaError_t e = cudaSuccess;
+    if (c->plan_for[layer] != t) {
+        e = hkv::launch_plan(c->lay, layer, layer + 1, 0, (cudaStream_t)stream);
+        c->plan_for[layer] = t;
+    }
+    if (e == cudaSuccess)
+        e = hkv::launch_decode(c->lay, layer, q_t, nullptr, nullptr, o_t, 0, c->decode_sh,
+                               c->decode_grid, (cudaStream_t)stream);
+    return cuda_status(e);
 }
 
 hkv_status hkv_decode_step(hkv_ctx* c, int32_t layer, const void* q_t, const void* k_t,
@@ -246,8 +271,15 @@ hkv_status hkv_decode_step(hkv_ctx* c, int32_t layer, const void* q_t, const voi
     if (!q_t || !k_t || !v_t || !o_t || !aligned16(q_t) || !aligned16(k_t) || !aligned16(v_t) ||
         !aligned16(o_t))
         return HKV_ERR_INVALID_ARG;
-    cudaError_t e = hkv::launch_decode(c->lay, layer, q_t, k_t, v_t, o_t, 1, c->decode_grid,
-                                       (cudaStream_t)stream);
+    const int t = c->t_host[layer];  // position this step appends
+    cudaError_t e = cudaSuccess;
+    if (c->plan_for[layer] != t) {
+        e = hkv::launch_plan(c->lay, layer, layer + 1, 1, (cudaStream_t)stream);
+        c->plan_for[layer] = t;
+    }
+    if (e == cudaSuccess)
+        e = hkv::launch_decode(c->lay, layer, q_t, k_t, v_t, o_t, 1, c->decode_sh, c->decode_grid,
+                               (cudaStream_t)stream);
     if (e != cudaSuccess) return HKV_ERR_CUDA;
     c->t_host[layer] += 1;
     return HKV_OK;
@@ -258,9 +290,15 @@ hkv_status hkv_ste_evict(hkv_ctx* c, int32_t layer_begin, int32_t layer_end, voi
         return HKV_ERR_INVALID_ARG;
     for (int l = layer_begin; l < layer_end; ++l)
         if (!c->classified[l]) return HKV_ERR_STATE;
-    if (c->cfg.mode == HKV_MODE_FULL) return HKV_OK;
-    return cuda_status(hkv::launch_evict(c->lay, layer_begin, layer_end, c->evict_grid,
-                                         (cudaStream_t)stream));
+    cudaError_t e = cudaSuccess;
+    if (c->cfg.mode != HKV_MODE_FULL)
+        e = hkv::launch_evict(c->lay, layer_begin, layer_end, c->evict_grid, (cudaStream_t)stream);
+    // plans of the next step, made once for all these layers
+    if (e == cudaSuccess)
+        e = hkv::launch_plan(c->lay, layer_begin, layer_end, 1, (cudaStream_t)stream);
+    if (e != cudaSuccess) return HKV_ERR_CUDA;
+    for (int l = layer_begin; l < layer_end; ++l) c->plan_for[l] = c->t_host[l];
+    return HKV_OK;
 }
 
 static hkv_status copy_back(void* dst, const void* src, size_t bytes, void* stream) {
@@ -354,6 +392,7 @@ hkv_status hkv_reset(hkv_ctx* c, void* stream) {
         c->classified[l] = 0;
         c->t_host[l] = 0;
         c->prefill_len[l] = 0;
+        c->plan_for[l] = -1;
     }
     return HKV_OK;
 }

@@ -13,6 +13,7 @@ namespace hkv {
 constexpr unsigned FULL_MASK = 0xffffffffu;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr int CHUNK = 32;  // tokens one warp handles per decode work item
+constexpr int PLAN_MAX_WARPS = 4096;  // capacity of a decode plan's warp table
 
 // Everything a kernel needs to find the state of a (layer, sequence, head).
 // The pool is one caller-owned device buffer carved into these regions.
@@ -48,6 +49,12 @@ struct Layout {
     int32_t* ticket;    // [S*H] arrivals per head of the running decode launch
     int32_t* due_ctl;   // [0] due heads listed, [1] blocks of the eviction done
     int32_t* due_list;  // [Ly*S*H] heads due for eviction this step
+    // decode plan per layer, for the step it was made for (see plan_kernel)
+    int32_t* plan_pre;   // [Ly][S*H] inclusive prefix of the heads' chunk counts
+    int4* plan_head;     // [Ly][S*H] {slot (layer-relative), len << 16 | jn, scoring, 0}
+    int32_t* plan_warp;  // [Ly][PLAN_MAX_WARPS + 1] first chunk of each warp's range
+    int32_t* plan_whead; // [Ly][PLAN_MAX_WARPS] head holding that chunk
+    int32_t plan_gw;     // warps of one decode launch
     int32_t max_chunks;
 };
 

@@ -19,8 +19,16 @@ cudaError_t launch_prefill_umma(const Layout& L, const void* q, const void* k, c
                                 int64_t block_stride, void* out, cudaStream_t st);
 cudaError_t launch_prefill(const Layout& L, int layer, const void* q, const void* k, const void* v,
                            int P, int64_t block_stride, void* out, cudaStream_t st);
+// Launch shape of the decode kernel: warps per block, pipeline stages per
+// warp, dynamic shared memory.
+struct DecodeShape {
+    int warps, nstage;
+    size_t smem;
+};
+DecodeShape decode_shape(const Layout& L, size_t smem_limit);
 cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void* k, const void* v,
-                          void* o, int append, int grid, cudaStream_t st);
+                          void* o, int append, const DecodeShape& sh, int grid, cudaStream_t st);
+cudaError_t launch_plan(const Layout& L, int l0, int l1, int ahead, cudaStream_t st);
 cudaError_t launch_prefill_rows_simt(int dtype, int d, int n_blocks, const void* q, const void* k,
                                      const void* v, int P, int64_t block_stride, int r, void* out,
                                      float* rows, cudaStream_t st);
