@@ -128,6 +128,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
     const int n = L.S * L.H;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, NW = blockDim.x >> 5;
     const int t = L.t_next[layer] - 1 + ahead;
+    if (t >= L.L) return;  // the sequence is complete: no step left to plan
     const size_t hbase = (size_t)layer * n;
     for (int i = tid; i < n; i += blockDim.x) {
         const size_t hx = hbase + i;

@@ -18,7 +18,7 @@ namespace hkv {
 // Per-warp scratch of the eviction: the select's own scratch, then the
 // head's scores and positions, then the (max, sum) of the scoring steps.
 __host__ __device__ inline size_t evict_warp_bytes(int n_max) {
-    return select_scratch_bytes(n_max) + (size_t)round32(n_max) * 8 + 32 * 8;
+    return select_scratch_bytes(n_max) + (size_t)round32(n_max) * 8 + 32 * 8 + 32 * 4;
 }
 
 // Lists the Global heads of layers [l0, l1) whose cache reached budget + M
@@ -56,6 +56,7 @@ __global__ void __launch_bounds__(512) evict_run_kernel(Layout L, int n_max) {
     float* sc_s = reinterpret_cast<float*>(wbase + select_scratch_bytes(n_max));
     int32_t* pos_s = reinterpret_cast<int32_t*>(sc_s + round32(n_max));
     float2* ml_s = reinterpret_cast<float2*>(pos_s + round32(n_max));
+    int32_t* step_s = reinterpret_cast<int32_t*>(ml_s + 32);
     const int n_heads = L.S * L.H;
     const int d = L.d;
     const int r = L.r;
@@ -78,10 +79,12 @@ __global__ void __launch_bounds__(512) evict_run_kernel(Layout L, int n_max) {
             continue;
         }
         const size_t slot0 = region_slot0(L, l, s) + L.off[hx];
-        // (max, 1/sum) of each scoring step, by column = step mod r
+        // (max, 1/sum) of each scoring step, by column = step mod r, and the
+        // step each column holds inside the window t-r+1 .. t
         if (lane < r) {
             const float2 ml = L.ml[hx * r + lane];
             ml_s[lane] = make_float2(ml.x, 1.0f / ml.y);
+            step_s[lane] = t - (((t - lane) % r) + r) % r;
         }
         __syncwarp();
         // scores: summed softmax weight of the last r queries, each
@@ -105,8 +108,7 @@ __global__ void __launch_bounds__(512) evict_run_kernel(Layout L, int n_max) {
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
                 if (c >= r) break;
-                const int step = t - (((t - c) % r) + r) % r;  // the window step of column c
-                if (p <= step) acc += exp2f(v[c] - ml_s[c].x) * ml_s[c].y;
+                if (p <= step_s[c]) acc += exp2f(v[c] - ml_s[c].x) * ml_s[c].y;
             }
             if (isnan(acc)) bad = true;
             sc_s[q] = acc;

@@ -14,6 +14,7 @@ constexpr unsigned FULL_MASK = 0xffffffffu;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr int CHUNK = 32;  // tokens one warp handles per decode work item
 constexpr int PLAN_MAX_WARPS = 4096;  // capacity of a decode plan's warp table
+constexpr int RANK_MAX = 256;         // strata up to this size are selected by ranking
 
 // Everything a kernel needs to find the state of a (layer, sequence, head).
 // The pool is one caller-owned device buffer carved into these regions.
@@ -317,9 +318,14 @@ __device__ int warp_stratified_select(const SelectScratch& sc, int n, int t, int
         kn = 0;
         if (kf > nf) kf = nf;
     }
-    // thresholds: none evicted (k <= 0), all evicted (k >= m), else searched
-    KthSearch a{sc.keys, nn, kn, kn > 0 && kn < nn, 0, 0, kn >= nn && kn > 0 ? ~0ull : 0ull};
-    KthSearch b{sc.keys + (n - nf), nf, kf, kf > 0 && kf < nf, 0, 0, kf >= nf && kf > 0 ? ~0ull : 0ull};
+    // Small strata: rank every key against all keys of its stratum (keys are
+    // distinct, so rank < k is exactly the k lowest).  Large strata: thresholds
+    // by the 4-ary search; none evicted (k <= 0), all evicted (k >= m).
+    const bool rank_n = kn > 0 && kn < nn && nn <= RANK_MAX;
+    const bool rank_f = kf > 0 && kf < nf && nf <= RANK_MAX;
+    KthSearch a{sc.keys, nn, kn, kn > 0 && kn < nn && !rank_n, 0, 0, kn >= nn && kn > 0 ? ~0ull : 0ull};
+    KthSearch b{sc.keys + (n - nf), nf, kf, kf > 0 && kf < nf && !rank_f, 0, 0,
+                kf >= nf && kf > 0 ? ~0ull : 0ull};
     if (a.active || b.active) warp_kth_pair(a, b);
     for (int which = 0; which < 2; ++which) {
         const int k = which == 0 ? kn : kf;
@@ -327,9 +333,20 @@ __device__ int warp_stratified_select(const SelectScratch& sc, int n, int t, int
         const uint64_t* keys = which == 0 ? a.keys : b.keys;
         const uint16_t* slots = which == 0 ? sc.slot : sc.slot + (n - nf);
         const uint64_t thr = which == 0 ? a.thr : b.thr;
+        const bool by_rank = which == 0 ? rank_n : rank_f;
         if (k <= 0) continue;
-        for (int i = lane; i < m; i += 32)
-            if (keys[i] <= thr) atomicOr(&sc.evict_bits[slots[i] >> 5], 1u << (slots[i] & 31));
+        if (by_rank) {
+            for (int i0 = 0; i0 < m; i0 += 32) {
+                const int i = i0 + lane;
+                const uint64_t ki = i < m ? keys[i] : ~0ull;
+                int rank = 0;
+                for (int j = 0; j < m; ++j) rank += keys[j] < ki;  // broadcast reads
+                if (i < m && rank < k) atomicOr(&sc.evict_bits[slots[i] >> 5], 1u << (slots[i] & 31));
+            }
+        } else {
+            for (int i = lane; i < m; i += 32)
+                if (keys[i] <= thr) atomicOr(&sc.evict_bits[slots[i] >> 5], 1u << (slots[i] & 31));
+        }
     }
     __syncwarp();
     return kn + kf;
