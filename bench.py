@@ -381,21 +381,49 @@ def e2e_arm(args, w, cache, inp, dev, world):
     host_out = torch.empty(steps, Ly, S, H, d, dtype=w.torch_dtype).pin_memory()
     dev_pre = [tuple(torch.empty_like(x) for x in t) for t in inp.pre]
     stage = [torch.empty(Ly, 3, S, H, d, dtype=w.torch_dtype, device=dev) for _ in range(2)]
-    outs = torch.empty(Ly, S, H, d, dtype=w.torch_dtype, device=dev)
+    outs2 = [torch.empty(Ly, S, H, d, dtype=w.torch_dtype, device=dev) for _ in range(2)]
+    h2d_s, d2h_s = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(steps)]    # step t's inputs landed
+    ev_done = [torch.cuda.Event() for _ in range(steps)]  # step t's kernels finished
+    ev_out = [torch.cuda.Event() for _ in range(steps)]   # step t's outputs copied out
 
     def body():
+        # step t+1's inputs go up and step t's outputs come down on two side
+        # streams while step t computes; staging and outputs double-buffered
+        main = torch.cuda.current_stream()
         cache.reset()
         for l in range(Ly):
             for hx, dx in zip(host_pre[l], dev_pre[l]):
                 dx.copy_(hx, non_blocking=True)
             cache.prefill_classify(l, *dev_pre[l])
+        h2d_s.wait_stream(main)
+        d2h_s.wait_stream(main)
+
+        def stage_in(t):
+            with torch.cuda.stream(h2d_s):
+                if t >= 2:
+                    h2d_s.wait_event(ev_done[t - 2])
+                stage[t & 1].copy_(host_dec[t], non_blocking=True)
+                ev_in[t].record(h2d_s)
+
+        stage_in(0)
         for t in range(steps):
-            st = stage[t & 1]
-            st.copy_(host_dec[t], non_blocking=True)
+            if t + 1 < steps:
+                stage_in(t + 1)
+            main.wait_event(ev_in[t])
+            if t >= 2:
+                main.wait_event(ev_out[t - 2])
+            st, ot = stage[t & 1], outs2[t & 1]
             for l in range(Ly):
-                cache.decode_step(l, st[l, 0], st[l, 1], st[l, 2], outs[l])
+                cache.decode_step(l, st[l, 0], st[l, 1], st[l, 2], ot[l])
             cache.ste_evict()
-            host_out[t].copy_(outs, non_blocking=True)
+            ev_done[t].record(main)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(ev_done[t])
+                host_out[t].copy_(ot, non_blocking=True)
+                ev_out[t].record(d2h_s)
+        main.wait_stream(h2d_s)
+        main.wait_stream(d2h_s)
 
     g = capture(body)
     for _ in range(2):

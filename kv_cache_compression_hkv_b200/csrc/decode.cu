@@ -263,7 +263,8 @@ __global__ void __launch_bounds__(256, 1)
     const int c_begin = pw[gw], c_end = pw[gw + 1], total = pw[GW];
 
     unsigned char* my = dsm + (size_t)warp * nstage * STAGE;
-    float* myq = reinterpret_cast<float*>(dsm + (size_t)NW * nstage * STAGE) + warp * D;
+    float* myq = reinterpret_cast<float*>(dsm + (size_t)NW * nstage * STAGE) + warp * (D + CHUNK);
+    float* myp = myq + D;  // this chunk's softmax numerators
 
     if (c_begin < c_end) {
         const int h_begin = L.plan_whead[(size_t)layer * PLAN_MAX_WARPS + gw];
@@ -347,7 +348,7 @@ __global__ void __launch_bounds__(256, 1)
             float sl = -INFINITY;
             if (lane < n) {
                 const unsigned char* krow = kst + lane * ROW;
-                float a0 = 0.f, a1 = 0.f;
+                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
                 for (int c2 = 0; c2 < PPR; ++c2) {
                     const int c = (c2 + lane) & (PPR - 1);
@@ -357,21 +358,21 @@ __global__ void __launch_bounds__(256, 1)
                         const float4 qb = *reinterpret_cast<const float4*>(myq + c * 8 + 4);
                         a0 = fmaf(qa.x, bf16_lo(kw.x), a0);
                         a1 = fmaf(qa.y, bf16_hi(kw.x), a1);
-                        a0 = fmaf(qa.z, bf16_lo(kw.y), a0);
-                        a1 = fmaf(qa.w, bf16_hi(kw.y), a1);
+                        a2 = fmaf(qa.z, bf16_lo(kw.y), a2);
+                        a3 = fmaf(qa.w, bf16_hi(kw.y), a3);
                         a0 = fmaf(qb.x, bf16_lo(kw.z), a0);
                         a1 = fmaf(qb.y, bf16_hi(kw.z), a1);
-                        a0 = fmaf(qb.z, bf16_lo(kw.w), a0);
-                        a1 = fmaf(qb.w, bf16_hi(kw.w), a1);
+                        a2 = fmaf(qb.z, bf16_lo(kw.w), a2);
+                        a3 = fmaf(qb.w, bf16_hi(kw.w), a3);
                     } else {
                         const float4 qa = *reinterpret_cast<const float4*>(myq + c * 4);
                         a0 = fmaf(qa.x, __uint_as_float(kw.x), a0);
                         a1 = fmaf(qa.y, __uint_as_float(kw.y), a1);
-                        a0 = fmaf(qa.z, __uint_as_float(kw.z), a0);
-                        a1 = fmaf(qa.w, __uint_as_float(kw.w), a1);
+                        a2 = fmaf(qa.z, __uint_as_float(kw.z), a2);
+                        a3 = fmaf(qa.w, __uint_as_float(kw.w), a3);
                     }
                 }
-                sl = a0 + a1;
+                sl = (a0 + a1) + (a2 + a3);
             }
             const size_t row0 = lrow + slot + tok0;
             if (scoring && lane < n) L.logit[(row0 + lane) * L.r + col] = sl;
@@ -386,18 +387,33 @@ __global__ void __launch_bounds__(256, 1)
             for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(FULL_MASK, ps, o);
             l = l * alpha + ps;
             m = mn;
+            // weighted V: p_j parked in shared memory and read back as float4
+            // broadcasts; four independent accumulator chains
+            myp[lane] = p;
+            __syncwarp();
+            float pa[4][DPL];
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) acc[e] *= alpha;
+            for (int u = 0; u < 4; ++u)
 #pragma unroll
-            for (int j = 0; j < CHUNK; ++j) {
-                if (j < n) {
-                    const float pj = __shfl_sync(FULL_MASK, p, j);
-                    Raw<T, DPL> vr;
-                    vr.load_shared(reinterpret_cast<const T*>(vst + j * ROW) + lane * DPL);
+                for (int e = 0; e < DPL; ++e) pa[u][e] = 0.f;
 #pragma unroll
-                    for (int e = 0; e < DPL; ++e) acc[e] = fmaf(pj, vr.get(e), acc[e]);
+            for (int j4 = 0; j4 < CHUNK; j4 += 4) {
+                if (j4 < n) {  // rows past n carry p = 0 and are never NaN-read
+                    const float4 p4 = *reinterpret_cast<const float4*>(myp + j4);
+                    const float pj[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        if (j4 + u < n) {
+                            Raw<T, DPL> vr;
+                            vr.load_shared(reinterpret_cast<const T*>(vst + (j4 + u) * ROW) + lane * DPL);
+#pragma unroll
+                            for (int e = 0; e < DPL; ++e) pa[u][e] = fmaf(pj[u], vr.get(e), pa[u][e]);
+                        }
+                    }
                 }
             }
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) acc[e] = acc[e] * alpha + ((pa[0][e] + pa[1][e]) + (pa[2][e] + pa[3][e]));
             // the appended token joins the cache
             const int a = jn - tok0;
             if (append && a >= 0 && a < n) {
@@ -540,7 +556,7 @@ DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
     const size_t stage = (2 * CHUNK + 1) * row;
     DecodeShape sh{0, 0, 0};
     for (int ns = 3; ns >= 2 && sh.warps == 0; --ns) {
-        const size_t per = ns * stage + (size_t)L.d * 4;
+        const size_t per = ns * stage + (size_t)(L.d + CHUNK) * 4;
         int w = (int)((smem_limit - 1024) / per);
         if (w > 8) w = 8;
         if (w >= (ns == 3 ? 6 : 1)) sh = DecodeShape{w, ns, 1024 + (size_t)w * per};
