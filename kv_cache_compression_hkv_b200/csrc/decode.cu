@@ -94,12 +94,15 @@ __device__ __forceinline__ void store_row(T* p, const float (&x)[DPL]) {
             __nv_bfloat162 b = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
             w[i] = *reinterpret_cast<uint32_t*>(&b);
         }
-        if constexpr (DPL == 4) *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
+        if constexpr (DPL == 8) *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+        else if constexpr (DPL == 4) *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
         else if constexpr (DPL == 2) *reinterpret_cast<uint32_t*>(p) = w[0];
         else {
 #pragma unroll
             for (int i = 0; i < DPL / 2; ++i) reinterpret_cast<uint32_t*>(p)[i] = w[i];
         }
+    } else if constexpr (DPL == 4) {
+        *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
     } else {
 #pragma unroll
         for (int i = 0; i < DPL; ++i) reinterpret_cast<float*>(p)[i] = x[i];
@@ -243,6 +246,9 @@ __global__ void __launch_bounds__(256, 1)
     constexpr int ROW = D * (int)sizeof(T);           // bytes of one cache row
     constexpr int PPR = ROW / 16;                     // 16-byte pieces per row
     constexpr int STAGE = (2 * CHUNK + 1) * ROW;      // K rows, V rows, the query
+    constexpr int E = 16 / (int)sizeof(T);            // elements per 16-byte piece
+    constexpr int G = PPR;                            // lanes covering one row (PV)
+    constexpr int TPI = 32 / G;                       // rows per PV step
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int NW = blockDim.x >> 5;
     const int t = append ? L.t_next[layer] : L.t_next[layer] - 1;
@@ -311,9 +317,13 @@ __global__ void __launch_bounds__(256, 1)
 
         int hc = h_begin;
         int seg0 = c_begin;
-        float m = -INFINITY, l = 0.f, acc[DPL];
+        // PV accumulators: lane (vg, vc) = (lane / G, lane % G) sums rows
+        // j = vg (mod TPI) of its 16-byte piece vc; the groups are added up once
+        // per head
+        const int vg = lane / G, vc = lane % G;
+        float m = -INFINITY, l = 0.f, acc[E];
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+        for (int e = 0; e < E; ++e) acc[e] = 0.f;
         int slot, len, jn, scoring, pre, first;
         cc.get(hc, slot, len, jn, scoring, pre, first);
         while (pre <= c_begin) {  // heads with no chunk before the first one
@@ -387,33 +397,37 @@ __global__ void __launch_bounds__(256, 1)
             for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(FULL_MASK, ps, o);
             l = l * alpha + ps;
             m = mn;
-            // weighted V: p_j parked in shared memory and read back as float4
-            // broadcasts; four independent accumulator chains
+            // weighted V: p_j parked in shared memory; each lane group reads
+            // whole 16-byte pieces of its rows; two accumulator chains
             myp[lane] = p;
             __syncwarp();
-            float pa[4][DPL];
+            float pa[2][E];
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
+            for (int u = 0; u < 2; ++u)
 #pragma unroll
-                for (int e = 0; e < DPL; ++e) pa[u][e] = 0.f;
+                for (int e = 0; e < E; ++e) pa[u][e] = 0.f;
 #pragma unroll
-            for (int j4 = 0; j4 < CHUNK; j4 += 4) {
-                if (j4 < n) {  // rows past n carry p = 0 and are never NaN-read
-                    const float4 p4 = *reinterpret_cast<const float4*>(myp + j4);
-                    const float pj[4] = {p4.x, p4.y, p4.z, p4.w};
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        if (j4 + u < n) {
-                            Raw<T, DPL> vr;
-                            vr.load_shared(reinterpret_cast<const T*>(vst + (j4 + u) * ROW) + lane * DPL);
-#pragma unroll
-                            for (int e = 0; e < DPL; ++e) pa[u][e] = fmaf(pj[u], vr.get(e), pa[u][e]);
-                        }
+            for (int jb = 0; jb < CHUNK; jb += TPI) {
+                const int j = jb + vg;
+                if (jb < n && j < n) {
+                    const float pj = myp[j];
+                    const uint4 vw = *reinterpret_cast<const uint4*>(vst + j * ROW + vc * 16);
+                    float* pu = pa[(jb / TPI) & 1];
+                    if constexpr (sizeof(T) == 2) {
+                        pu[0] = fmaf(pj, bf16_lo(vw.x), pu[0]); pu[1] = fmaf(pj, bf16_hi(vw.x), pu[1]);
+                        pu[2] = fmaf(pj, bf16_lo(vw.y), pu[2]); pu[3] = fmaf(pj, bf16_hi(vw.y), pu[3]);
+                        pu[4] = fmaf(pj, bf16_lo(vw.z), pu[4]); pu[5] = fmaf(pj, bf16_hi(vw.z), pu[5]);
+                        pu[6] = fmaf(pj, bf16_lo(vw.w), pu[6]); pu[7] = fmaf(pj, bf16_hi(vw.w), pu[7]);
+                    } else {
+                        pu[0] = fmaf(pj, __uint_as_float(vw.x), pu[0]);
+                        pu[1] = fmaf(pj, __uint_as_float(vw.y), pu[1]);
+                        pu[2] = fmaf(pj, __uint_as_float(vw.z), pu[2]);
+                        pu[3] = fmaf(pj, __uint_as_float(vw.w), pu[3]);
                     }
                 }
             }
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) acc[e] = acc[e] * alpha + ((pa[0][e] + pa[1][e]) + (pa[2][e] + pa[3][e]));
+            for (int e = 0; e < E; ++e) acc[e] = acc[e] * alpha + (pa[0][e] + pa[1][e]);
             // the appended token joins the cache
             const int a = jn - tok0;
             if (append && a >= 0 && a < n) {
@@ -428,22 +442,28 @@ __global__ void __launch_bounds__(256, 1)
             if (ip < c_end) issue(stage);
             if (i + 1 < c_end && pre > i + 1) continue;  // head goes on
 
-            // end of this warp's segment of head hc
+            // end of this warp's segment of head hc: add up the row groups
+#pragma unroll
+            for (int o = G; o < 32; o <<= 1)
+#pragma unroll
+                for (int e = 0; e < E; ++e) acc[e] += __shfl_xor_sync(FULL_MASK, acc[e], o);
             const size_t hx = hbase + hc;
             if (!(l > 0.f) || isinf(l)) latch_error(L, HKV_ERR_NUMERIC, (int)hx);
             const bool whole = seg0 == first && i + 1 == pre;
             if (whole) {
                 const float inv = 1.0f / l;
-                float o[DPL];
+                float o[E];
 #pragma unroll
-                for (int e = 0; e < DPL; ++e) o[e] = acc[e] * inv;
-                store_row<T, DPL>(o_t + (size_t)hc * D + lane * DPL, o);
+                for (int e = 0; e < E; ++e) o[e] = acc[e] * inv;
+                if (lane < G) store_row<T, E>(o_t + (size_t)hc * D + vc * E, o);
                 if (scoring && lane == 0) L.ml[hx * L.r + col] = make_float2(m, l);
             } else {
                 float* pp = L.partial + (size_t)seg0 * (D + 2);
                 if (lane == 0) { pp[0] = m; pp[1] = l; }
+                if (lane < G) {
 #pragma unroll
-                for (int e = 0; e < DPL; ++e) pp[2 + lane * DPL + e] = acc[e];
+                    for (int e = 0; e < E; ++e) pp[2 + vc * E + e] = acc[e];
+                }
                 __threadfence();
                 const int w_a = range_owner(first, total, GW);
                 const int w_b = range_owner(pre - 1, total, GW);
@@ -465,9 +485,9 @@ __global__ void __launch_bounds__(256, 1)
                     }
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, o));
-                    float Ls = 0.f, o[DPL];
+                    float Ls = 0.f, o[E];
 #pragma unroll
-                    for (int e = 0; e < DPL; ++e) o[e] = 0.f;
+                    for (int e = 0; e < E; ++e) o[e] = 0.f;
                     for (int w = w_a; w <= w_b; ++w) {
                         const int rb = range_begin(w, total, GW);
                         if (rb >= range_begin(w + 1, total, GW)) continue;
@@ -475,12 +495,12 @@ __global__ void __launch_bounds__(256, 1)
                         const float wt = exp2f(__ldcg(pi) - M);
                         Ls = fmaf(__ldcg(pi + 1), wt, Ls);
 #pragma unroll
-                        for (int e = 0; e < DPL; ++e) o[e] = fmaf(__ldcg(pi + 2 + lane * DPL + e), wt, o[e]);
+                        for (int e = 0; e < E; ++e) o[e] = fmaf(__ldcg(pi + 2 + vc * E + e), wt, o[e]);
                     }
                     const float inv = 1.0f / Ls;
 #pragma unroll
-                    for (int e = 0; e < DPL; ++e) o[e] *= inv;
-                    store_row<T, DPL>(o_t + (size_t)hc * D + lane * DPL, o);
+                    for (int e = 0; e < E; ++e) o[e] *= inv;
+                    if (lane < G) store_row<T, E>(o_t + (size_t)hc * D + vc * E, o);
                     if (scoring && lane == 0) L.ml[hx * L.r + col] = make_float2(M, Ls);
                 }
             }
@@ -489,7 +509,7 @@ __global__ void __launch_bounds__(256, 1)
             m = -INFINITY;
             l = 0.f;
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+            for (int e = 0; e < E; ++e) acc[e] = 0.f;
             if (i + 1 < c_end) {
                 do {
                     ++hc;
