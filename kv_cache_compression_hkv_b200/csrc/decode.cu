@@ -15,6 +15,8 @@
 // normalises with the (max, sum) stored here.
 #include <math.h>
 
+#include <cuda/atomic>
+
 #include "hkv_internal.cuh"
 #include "kernels.h"
 
@@ -464,18 +466,23 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
                     for (int e = 0; e < E; ++e) pp[2 + vc * E + e] = acc[e];
                 }
-                __threadfence();
+                __syncwarp();  // the lanes' partial stores precede lane 0's release
                 const int w_a = range_owner(first, total, GW);
                 const int w_b = range_owner(pre - 1, total, GW);
                 int segs = 0;
                 for (int w = w_a; w <= w_b; ++w)
                     segs += range_begin(w, total, GW) < range_begin(w + 1, total, GW);
                 int prev = 0;
-                if (lane == 0) prev = atomicAdd(&L.ticket[hc], 1);
+                if (lane == 0) {
+                    // release: this warp's partial before the ticket; acquire:
+                    // the other segments' partials for the last one in
+                    cuda::atomic_ref<int, cuda::thread_scope_device> tk(L.ticket[hc]);
+                    prev = tk.fetch_add(1, cuda::memory_order_acq_rel);
+                }
                 prev = __shfl_sync(FULL_MASK, prev, 0);
+                __syncwarp();  // lane 0's acquire before every lane's partial loads
                 if (prev == segs - 1) {
                     // last segment in: merge (lane-parallel over segments)
-                    __threadfence();
                     if (lane == 0) L.ticket[hc] = 0;
                     float M = -INFINITY;
                     for (int w = w_a + lane; w <= w_b; w += 32) {
