@@ -289,27 +289,28 @@ def gpu_arm(args, rank, world, dev):
     if rc != 0:
         raise RuntimeError(f"device status {rc} ({detail}) after the timed passes")
 
-    # per-launch durations (same stream as the kernels: the capture stream)
-    n_ev = steps * (Ly + 1)
+    # per step: the span of its Ly back-to-back decode launches (events only
+    # around the run, so consecutive launches may overlap as they do in the
+    # timed pass) and of its eviction; same stream as the kernels
+    n_ev = steps * 2
     evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * n_ev)]
-    slot = {}
 
     def hooks_prof(what, t, l):
-        if what in ("pre_decode", "post_decode"):
-            i = t * (Ly + 1) + l
-        elif what in ("pre_evict", "post_evict"):
-            i = t * (Ly + 1) + Ly
-        else:
-            return
-        evs[2 * i + (0 if what.startswith("pre") else 1)].record()
-        slot[i] = True
+        if what == "pre_decode" and l == 0:
+            evs[4 * t].record()
+        elif what == "post_decode" and l == Ly - 1:
+            evs[4 * t + 1].record()
+        elif what == "pre_evict":
+            evs[4 * t + 2].record()
+        elif what == "post_evict":
+            evs[4 * t + 3].record()
 
     g_prof = capture(lambda: run_pass(cache, w, inp, outs, pre_out=pre_out, hooks=hooks_prof))
     g_prof.replay()
     torch.cuda.synchronize()
-    dur = np.array([evs[2 * i].elapsed_time(evs[2 * i + 1]) for i in range(n_ev)]).reshape(steps, Ly + 1)
-    dec_us = dur[:, :Ly] * 1e3
-    evict_us = dur[:, Ly] * 1e3
+    dur = np.array([evs[2 * i].elapsed_time(evs[2 * i + 1]) for i in range(n_ev)]).reshape(steps, 2)
+    dec_us = np.repeat(dur[:, :1] * 1e3 / Ly, Ly, axis=1)  # average launch of each step
+    evict_us = dur[:, 1] * 1e3
     kv_bytes = tokens * 2 * d * es                      # kept K + V read (new token included)
     io_bytes = S * H * d * es * 4                        # q read, o written, new k/v row stored
     alg = kv_bytes + io_bytes

@@ -19,8 +19,15 @@
 
 #include "hkv_internal.cuh"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace hkv {
+
+// Headroom (log2 units) a logit may exceed the running softmax reference by
+// before the reference is raised: weights stay below 2^8, far from fp32 range.
+constexpr float RESCALE = 8.f;
+// Most pipeline stages a decode warp keeps in flight.
+constexpr int MAX_STAGES = 3;
 
 // Packed storage of DPL consecutive elements of one row.
 template <typename T, int DPL> struct Raw;
@@ -241,7 +248,8 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 template <typename T, int DPL>
 __global__ void __launch_bounds__(256, 1)
     decode_kernel(Layout L, int layer, const T* __restrict__ q_t, const T* __restrict__ k_t,
-                  const T* __restrict__ v_t, T* __restrict__ o_t, int append, int nstage) {
+                  const T* __restrict__ v_t, T* __restrict__ o_t, int append, int nstage,
+                  int early, int buf) {
     extern __shared__ __align__(128) unsigned char dsm[];
     const int n_heads = L.S * L.H;
     constexpr int D = DPL * 32;
@@ -251,6 +259,8 @@ __global__ void __launch_bounds__(256, 1)
     constexpr int E = 16 / (int)sizeof(T);            // elements per 16-byte piece
     constexpr int G = PPR;                            // lanes covering one row (PV)
     constexpr int TPI = 32 / G;                       // rows per PV step
+    constexpr int RPI = 32 / PPR;                     // rows per copy step
+    static_assert(PPR % 8 == 0 && PPR <= 32, "rows are 8, 16 or 32 pieces");
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int NW = blockDim.x >> 5;
     const int t = append ? L.t_next[layer] : L.t_next[layer] - 1;
@@ -263,7 +273,19 @@ __global__ void __launch_bounds__(256, 1)
     T* Vp = reinterpret_cast<T*>(L.V);
     const float qscale = LOG2E / sqrtf((float)D);
 
+    // Launched as a programmatic dependent of the previous launch in the
+    // stream.  With `early` the plan, the cache and t_next of this layer are
+    // read before the wait for that launch (the host sets it only when that
+    // launch is a decode launch of another layer, which writes none of them);
+    // q_t, k_t, v_t, o_t and the split-K buffers are touched only after it.
+    // Every thread waits before it triggers the next launch, so that launch
+    // can only ever overlap this one, whose split-K buffers (set `buf`) it
+    // does not share.
+    if (!early) ptx::grid_dep_wait();
+    int* ticket = L.ticket + (size_t)buf * n_heads;
+    float* partial = L.partial + (size_t)buf * L.max_chunks * (D + 2);
     if (GW != L.plan_gw) {
+        if (early) ptx::grid_dep_wait();
         if (threadIdx.x == 0 && blockIdx.x == 0) latch_error(L, HKV_ERR_STATE, layer);
         return;
     }
@@ -280,31 +302,40 @@ __global__ void __launch_bounds__(256, 1)
         pc.load(L, hbase, n_heads, h_begin);
         cc = pc;
 
-        // producer cursor: chunk ip of head hp
+        // producer cursor: chunk ip of head hp; lane copies piece pc_ of rows
+        // pr_, pr_ + RPI, ...
         int ip = c_begin, hp = h_begin;
-        auto issue = [&](int stage) {
+        const int pc_ = lane % PPR, pr_ = lane / PPR;
+        // Issues the copies of chunk ip into `stage`.  With `prior` (before the
+        // wait on the previous launch) the query and the appended row are left
+        // out; the returned (head, appended row or -1, query wanted) lets the
+        // caller put them in after the wait.
+        auto issue = [&](int stage, bool prior) -> int3 {
             int slot, len, jn, sc_, pre, first;
             if (hp - pc.base >= 32) pc.load(L, hbase, n_heads, hp);
             pc.get(hp, slot, len, jn, sc_, pre, first);
             const int tok0 = (ip - first) * CHUNK;
             const int n = min(CHUNK, len - tok0);
-            const int a = jn - tok0;  // appended row within the chunk (or outside)
+            const int a = append ? jn - tok0 : -1;  // appended row within the chunk (or outside)
             const size_t row0 = lrow + slot + tok0;
             unsigned char* kd = my + (size_t)stage * STAGE;
             unsigned char* vd = kd + CHUNK * ROW;
             unsigned char* qd = vd + CHUNK * ROW;
-            const int pieces = n * PPR;
-            for (int p = lane; p < pieces; p += 32) {
-                const int row = p / PPR, c = p % PPR;
-                const bool fresh = append && row == a;
-                const T* ks = (fresh ? k_t + (size_t)hp * D : Kp + (row0 + row) * D) + c * (16 / (int)sizeof(T));
-                const T* vs = (fresh ? v_t + (size_t)hp * D : Vp + (row0 + row) * D) + c * (16 / (int)sizeof(T));
-                cp_async16(kd + row * ROW + c * 16, ks);
-                cp_async16(vd + row * ROW + c * 16, vs);
+            const T* kf = k_t + (size_t)hp * D + pc_ * E;
+            const T* vf = v_t + (size_t)hp * D + pc_ * E;
+            const bool needq = ip == first || ip == c_begin;  // the head's first chunk here
+            for (int row = pr_; row < n; row += RPI) {
+                const bool fresh = row == a;
+                if (prior && fresh) continue;
+                const T* ks = fresh ? kf : Kp + (row0 + row) * D + pc_ * E;
+                const T* vs = fresh ? vf : Vp + (row0 + row) * D + pc_ * E;
+                cp_async16(kd + row * ROW + ((pc_ ^ (row & 7)) << 4), ks);
+                cp_async16(vd + row * ROW + (pc_ << 4), vs);
             }
-            for (int c = lane; c < PPR; c += 32)
-                cp_async16(qd + c * 16, q_t + (size_t)hp * D + c * (16 / (int)sizeof(T)));
+            if (!prior && needq)
+                for (int c = lane; c < PPR; c += 32) cp_async16(qd + c * 16, q_t + (size_t)hp * D + c * E);
             cp_async_commit();
+            const int3 rec = make_int3(hp, (a >= 0 && a < n) ? a : -1, needq);
             ++ip;
             if (ip < c_end && pre <= ip) ++hp;
             while (ip < c_end) {  // skip heads with no chunk (capacity errors)
@@ -314,8 +345,42 @@ __global__ void __launch_bounds__(256, 1)
                 if (p2 > ip) break;
                 ++hp;
             }
+            return rec;
         };
-        for (int s = 0; s < nstage && ip < c_end; ++s) issue(s);
+        // prologue: cached rows of the first stages, then the wait, then the
+        // query and appended rows of those stages with plain loads
+        int3 pro[MAX_STAGES];
+        int npro = 0;
+#pragma unroll
+        for (int s = 0; s < MAX_STAGES; ++s)
+            if (s < nstage && ip < c_end) { pro[s] = issue(s, true); npro = s + 1; }
+        if (early) ptx::grid_dep_wait();
+        ptx::grid_dep_trigger();
+        if (lane < PPR) {
+            uint4 wq[MAX_STAGES], wk[MAX_STAGES], wv[MAX_STAGES];
+#pragma unroll
+            for (int s = 0; s < MAX_STAGES; ++s) {
+                if (s >= npro) continue;
+                const size_t at = (size_t)pro[s].x * D + lane * E;
+                if (pro[s].z) wq[s] = *reinterpret_cast<const uint4*>(q_t + at);
+                if (pro[s].y >= 0) {
+                    wk[s] = *reinterpret_cast<const uint4*>(k_t + at);
+                    wv[s] = *reinterpret_cast<const uint4*>(v_t + at);
+                }
+            }
+#pragma unroll
+            for (int s = 0; s < MAX_STAGES; ++s) {
+                if (s >= npro) continue;
+                unsigned char* kd = my + (size_t)s * STAGE;
+                unsigned char* vd = kd + CHUNK * ROW;
+                if (pro[s].z) *reinterpret_cast<uint4*>(vd + CHUNK * ROW + lane * 16) = wq[s];
+                const int a = pro[s].y;
+                if (a >= 0) {
+                    *reinterpret_cast<uint4*>(kd + a * ROW + ((lane ^ (a & 7)) << 4)) = wk[s];
+                    *reinterpret_cast<uint4*>(vd + a * ROW + lane * 16) = wv[s];
+                }
+            }
+        }
 
         int hc = h_begin;
         int seg0 = c_begin;
@@ -323,7 +388,10 @@ __global__ void __launch_bounds__(256, 1)
         // j = vg (mod TPI) of its 16-byte piece vc; the groups are added up once
         // per head
         const int vg = lane / G, vc = lane % G;
-        float m = -INFINITY, l = 0.f, acc[E];
+        // m: the warp's reference maximum (log2 domain), raised only when a
+        // logit passes it by more than RESCALE; ls: this lane's share of the
+        // softmax denominator; qv: the pre-scaled query of the current head
+        float m = -INFINITY, ls = 0.f, acc[E], qv[D];
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[e] = 0.f;
         int slot, len, jn, scoring, pre, first;
@@ -347,58 +415,70 @@ __global__ void __launch_bounds__(256, 1)
             const unsigned char* kst = my + (size_t)stage * STAGE;
             const unsigned char* vst = kst + CHUNK * ROW;
             if (i == seg0) {
-                // a new head: its query, pre-scaled, in fp32 shared memory
-                const T* qs = reinterpret_cast<const T*>(vst + CHUNK * ROW);
-                Raw<T, DPL> qr;
-                qr.load_shared(qs + lane * DPL);
+                // a new head: every lane reads the whole query (broadcast reads)
+                const unsigned char* qs = vst + CHUNK * ROW;
 #pragma unroll
-                for (int e = 0; e < DPL; ++e) myq[lane * DPL + e] = qr.get(e) * qscale;
-                __syncwarp();
+                for (int c = 0; c < PPR; ++c) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(qs + c * 16);
+                    if constexpr (sizeof(T) == 2) {
+                        qv[c * 8 + 0] = bf16_lo(w.x) * qscale; qv[c * 8 + 1] = bf16_hi(w.x) * qscale;
+                        qv[c * 8 + 2] = bf16_lo(w.y) * qscale; qv[c * 8 + 3] = bf16_hi(w.y) * qscale;
+                        qv[c * 8 + 4] = bf16_lo(w.z) * qscale; qv[c * 8 + 5] = bf16_hi(w.z) * qscale;
+                        qv[c * 8 + 6] = bf16_lo(w.w) * qscale; qv[c * 8 + 7] = bf16_hi(w.w) * qscale;
+                    } else {
+                        qv[c * 4 + 0] = __uint_as_float(w.x) * qscale;
+                        qv[c * 4 + 1] = __uint_as_float(w.y) * qscale;
+                        qv[c * 4 + 2] = __uint_as_float(w.z) * qscale;
+                        qv[c * 4 + 3] = __uint_as_float(w.w) * qscale;
+                    }
+                }
             }
-            // lane j: dot product of the query with row j, reading the row's
-            // 16-byte pieces in a lane-rotated order (no bank conflicts)
+            // lane j: dot product of the query with row j; row j's pieces sit
+            // at piece ^ (j & 7), so the lanes of a quarter-warp read 8
+            // different bank groups while all reading the same query piece
             float sl = -INFINITY;
             if (lane < n) {
                 const unsigned char* krow = kst + lane * ROW;
+                const int sw = lane & 7;
                 float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-                for (int c2 = 0; c2 < PPR; ++c2) {
-                    const int c = (c2 + lane) & (PPR - 1);
-                    const uint4 kw = *reinterpret_cast<const uint4*>(krow + c * 16);
+                for (int c = 0; c < PPR; ++c) {
+                    const uint4 kw = *reinterpret_cast<const uint4*>(krow + ((c ^ sw) << 4));
                     if constexpr (sizeof(T) == 2) {
-                        const float4 qa = *reinterpret_cast<const float4*>(myq + c * 8);
-                        const float4 qb = *reinterpret_cast<const float4*>(myq + c * 8 + 4);
-                        a0 = fmaf(qa.x, bf16_lo(kw.x), a0);
-                        a1 = fmaf(qa.y, bf16_hi(kw.x), a1);
-                        a2 = fmaf(qa.z, bf16_lo(kw.y), a2);
-                        a3 = fmaf(qa.w, bf16_hi(kw.y), a3);
-                        a0 = fmaf(qb.x, bf16_lo(kw.z), a0);
-                        a1 = fmaf(qb.y, bf16_hi(kw.z), a1);
-                        a2 = fmaf(qb.z, bf16_lo(kw.w), a2);
-                        a3 = fmaf(qb.w, bf16_hi(kw.w), a3);
+                        a0 = fmaf(qv[c * 8 + 0], bf16_lo(kw.x), a0);
+                        a1 = fmaf(qv[c * 8 + 1], bf16_hi(kw.x), a1);
+                        a2 = fmaf(qv[c * 8 + 2], bf16_lo(kw.y), a2);
+                        a3 = fmaf(qv[c * 8 + 3], bf16_hi(kw.y), a3);
+                        a0 = fmaf(qv[c * 8 + 4], bf16_lo(kw.z), a0);
+                        a1 = fmaf(qv[c * 8 + 5], bf16_hi(kw.z), a1);
+                        a2 = fmaf(qv[c * 8 + 6], bf16_lo(kw.w), a2);
+                        a3 = fmaf(qv[c * 8 + 7], bf16_hi(kw.w), a3);
                     } else {
-                        const float4 qa = *reinterpret_cast<const float4*>(myq + c * 4);
-                        a0 = fmaf(qa.x, __uint_as_float(kw.x), a0);
-                        a1 = fmaf(qa.y, __uint_as_float(kw.y), a1);
-                        a2 = fmaf(qa.z, __uint_as_float(kw.z), a2);
-                        a3 = fmaf(qa.w, __uint_as_float(kw.w), a3);
+                        a0 = fmaf(qv[c * 4 + 0], __uint_as_float(kw.x), a0);
+                        a1 = fmaf(qv[c * 4 + 1], __uint_as_float(kw.y), a1);
+                        a2 = fmaf(qv[c * 4 + 2], __uint_as_float(kw.z), a2);
+                        a3 = fmaf(qv[c * 4 + 3], __uint_as_float(kw.w), a3);
                     }
                 }
                 sl = (a0 + a1) + (a2 + a3);
             }
             const size_t row0 = lrow + slot + tok0;
             if (scoring && lane < n) L.logit[(row0 + lane) * L.r + col] = sl;
-            float cm = sl;
+            // raise the reference only when some logit passes it by more than
+            // RESCALE (weights stay below 2^RESCALE); one vote otherwise
+            if (__any_sync(FULL_MASK, sl > m + RESCALE)) {
+                float cm = sl;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(FULL_MASK, cm, o));
-            const float mn = fmaxf(m, cm);
-            const float alpha = exp2f(m - mn);
-            const float p = lane < n ? exp2f(sl - mn) : 0.f;
-            float ps = p;
+                for (int o = 16; o > 0; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(FULL_MASK, cm, o));
+                const float mn = fmaxf(m, cm);
+                const float alpha = exp2f(m - mn);
+                ls *= alpha;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(FULL_MASK, ps, o);
-            l = l * alpha + ps;
-            m = mn;
+                for (int e = 0; e < E; ++e) acc[e] *= alpha;
+                m = mn;
+            }
+            const float p = lane < n ? exp2f(sl - m) : 0.f;
+            ls += p;
             // weighted V: p_j parked in shared memory; each lane group reads
             // whole 16-byte pieces of its rows; two accumulator chains
             myp[lane] = p;
@@ -429,26 +509,32 @@ __global__ void __launch_bounds__(256, 1)
                 }
             }
 #pragma unroll
-            for (int e = 0; e < E; ++e) acc[e] = acc[e] * alpha + (pa[0][e] + pa[1][e]);
+            for (int e = 0; e < E; ++e) acc[e] += pa[0][e] + pa[1][e];
             // the appended token joins the cache
             const int a = jn - tok0;
             if (append && a >= 0 && a < n) {
+                constexpr int LB = DPL * (int)sizeof(T);  // bytes per lane, within one piece
+                const int b = lane * LB;
                 Raw<T, DPL> kr, vr;
-                kr.load_shared(reinterpret_cast<const T*>(kst + a * ROW) + lane * DPL);
-                vr.load_shared(reinterpret_cast<const T*>(vst + a * ROW) + lane * DPL);
+                kr.load_shared(reinterpret_cast<const T*>(kst + a * ROW + ((((b >> 4) ^ (a & 7)) << 4) | (b & 15))));
+                vr.load_shared(reinterpret_cast<const T*>(vst + a * ROW + b));
                 kr.store(Kp + (row0 + a) * D + lane * DPL);
                 vr.store(Vp + (row0 + a) * D + lane * DPL);
                 if (lane == 0) L.pos[row0 + a] = t;
             }
             __syncwarp();
-            if (ip < c_end) issue(stage);
+            if (ip < c_end) issue(stage, false);
             if (i + 1 < c_end && pre > i + 1) continue;  // head goes on
 
             // end of this warp's segment of head hc: add up the row groups
+            // and the lanes' denominators
 #pragma unroll
             for (int o = G; o < 32; o <<= 1)
 #pragma unroll
                 for (int e = 0; e < E; ++e) acc[e] += __shfl_xor_sync(FULL_MASK, acc[e], o);
+            float l = ls;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(FULL_MASK, l, o);
             const size_t hx = hbase + hc;
             if (!(l > 0.f) || isinf(l)) latch_error(L, HKV_ERR_NUMERIC, (int)hx);
             const bool whole = seg0 == first && i + 1 == pre;
@@ -460,7 +546,7 @@ __global__ void __launch_bounds__(256, 1)
                 if (lane < G) store_row<T, E>(o_t + (size_t)hc * D + vc * E, o);
                 if (scoring && lane == 0) L.ml[hx * L.r + col] = make_float2(m, l);
             } else {
-                float* pp = L.partial + (size_t)seg0 * (D + 2);
+                float* pp = partial + (size_t)seg0 * (D + 2);
                 if (lane == 0) { pp[0] = m; pp[1] = l; }
                 if (lane < G) {
 #pragma unroll
@@ -476,19 +562,19 @@ __global__ void __launch_bounds__(256, 1)
                 if (lane == 0) {
                     // release: this warp's partial before the ticket; acquire:
                     // the other segments' partials for the last one in
-                    cuda::atomic_ref<int, cuda::thread_scope_device> tk(L.ticket[hc]);
+                    cuda::atomic_ref<int, cuda::thread_scope_device> tk(ticket[hc]);
                     prev = tk.fetch_add(1, cuda::memory_order_acq_rel);
                 }
                 prev = __shfl_sync(FULL_MASK, prev, 0);
                 __syncwarp();  // lane 0's acquire before every lane's partial loads
                 if (prev == segs - 1) {
                     // last segment in: merge (lane-parallel over segments)
-                    if (lane == 0) L.ticket[hc] = 0;
+                    if (lane == 0) ticket[hc] = 0;
                     float M = -INFINITY;
                     for (int w = w_a + lane; w <= w_b; w += 32) {
                         const int rb = range_begin(w, total, GW);
                         if (rb < range_begin(w + 1, total, GW))
-                            M = fmaxf(M, __ldcg(L.partial + (size_t)max(rb, first) * (D + 2)));
+                            M = fmaxf(M, __ldcg(partial + (size_t)max(rb, first) * (D + 2)));
                     }
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, o));
@@ -498,7 +584,7 @@ __global__ void __launch_bounds__(256, 1)
                     for (int w = w_a; w <= w_b; ++w) {
                         const int rb = range_begin(w, total, GW);
                         if (rb >= range_begin(w + 1, total, GW)) continue;
-                        const float* pi = L.partial + (size_t)max(rb, first) * (D + 2);
+                        const float* pi = partial + (size_t)max(rb, first) * (D + 2);
                         const float wt = exp2f(__ldcg(pi) - M);
                         Ls = fmaf(__ldcg(pi + 1), wt, Ls);
 #pragma unroll
@@ -514,7 +600,7 @@ __global__ void __launch_bounds__(256, 1)
             // next head holding chunk i + 1
             seg0 = i + 1;
             m = -INFINITY;
-            l = 0.f;
+            ls = 0.f;
 #pragma unroll
             for (int e = 0; e < E; ++e) acc[e] = 0.f;
             if (i + 1 < c_end) {
@@ -526,6 +612,9 @@ __global__ void __launch_bounds__(256, 1)
             }
         }
         cp_async_wait<0>();
+    } else {
+        if (early) ptx::grid_dep_wait();
+        ptx::grid_dep_trigger();
     }
     if (append) {
         __syncthreads();
@@ -594,20 +683,31 @@ DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
 template <typename T, int DPL>
 static cudaError_t launch_decode_t(const Layout& L, int layer, const void* q, const void* k,
                                    const void* v, void* o, int append, const DecodeShape& sh,
-                                   int grid, cudaStream_t st) {
-    decode_kernel<T, DPL><<<grid, 32 * sh.warps, sh.smem, st>>>(
-        L, layer, (const T*)q, (const T*)k, (const T*)v, (T*)o, append, sh.nstage);
-    return cudaGetLastError();
+                                   int grid, int early, int buf, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(32 * sh.warps);
+    cfg.dynamicSmemBytes = sh.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_kernel<T, DPL>, L, layer, (const T*)q, (const T*)k,
+                              (const T*)v, (T*)o, append, sh.nstage, early, buf);
 }
 
 cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void* k, const void* v,
-                          void* o, int append, const DecodeShape& sh, int grid, cudaStream_t st) {
+                          void* o, int append, const DecodeShape& sh, int grid, int early, int buf,
+                          cudaStream_t st) {
+    if (sh.nstage < 1 || sh.nstage > MAX_STAGES) return cudaErrorInvalidValue;
     if (L.dtype == HKV_DTYPE_BF16) {
-        if (L.d == 64) return launch_decode_t<__nv_bfloat16, 2>(L, layer, q, k, v, o, append, sh, grid, st);
-        if (L.d == 128) return launch_decode_t<__nv_bfloat16, 4>(L, layer, q, k, v, o, append, sh, grid, st);
+        if (L.d == 64) return launch_decode_t<__nv_bfloat16, 2>(L, layer, q, k, v, o, append, sh, grid, early, buf, st);
+        if (L.d == 128) return launch_decode_t<__nv_bfloat16, 4>(L, layer, q, k, v, o, append, sh, grid, early, buf, st);
     } else {
-        if (L.d == 64) return launch_decode_t<float, 2>(L, layer, q, k, v, o, append, sh, grid, st);
-        if (L.d == 128) return launch_decode_t<float, 4>(L, layer, q, k, v, o, append, sh, grid, st);
+        if (L.d == 64) return launch_decode_t<float, 2>(L, layer, q, k, v, o, append, sh, grid, early, buf, st);
+        if (L.d == 128) return launch_decode_t<float, 4>(L, layer, q, k, v, o, append, sh, grid, early, buf, st);
     }
     return cudaErrorInvalidValue;
 }

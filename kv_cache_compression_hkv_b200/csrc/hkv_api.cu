@@ -26,7 +26,35 @@ struct hkv_ctx {
     std::vector<int> classified;  // per layer
     std::vector<int> t_host;      // per layer: next position, as enqueued by API calls
     std::vector<int> prefill_len;
+    // the last kernel this context enqueued: a decode launch of layer
+    // last_decode (-1: any other kernel) on stream last_stream
+    int last_decode = -1;
+    void* last_stream = nullptr;
+    int split_buf = 0;  // split-K buffer set of the next decode launch
 };
+
+namespace {
+
+// Records a launch that is not a decode launch.
+void note_other(hkv_ctx* c, void* stream) {
+    c->last_decode = -1;
+    c->last_stream = stream;
+}
+
+// Launches the decode kernel of `layer`, overlapping its start with the
+// previous launch when that is a decode launch of another layer.
+cudaError_t decode_launch(hkv_ctx* c, int layer, const void* q, const void* k, const void* v,
+                          void* o, int append, void* stream) {
+    const int early = c->last_stream == stream && c->last_decode >= 0 && c->last_decode != layer;
+    cudaError_t e = hkv::launch_decode(c->lay, layer, q, k, v, o, append, c->decode_sh,
+                                       c->decode_grid, early, c->split_buf, (cudaStream_t)stream);
+    c->split_buf ^= 1;
+    c->last_decode = layer;
+    c->last_stream = stream;
+    return e;
+}
+
+}  // namespace
 
 namespace {
 
@@ -88,7 +116,7 @@ size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Lay
     l.status = (int32_t*)take(16);
     l.t_next = (int32_t*)take(Ly * 4);
     l.done_ctr = (int32_t*)take(Ly * 4);
-    l.ticket = (int32_t*)take(S * H * 4);
+    l.ticket = (int32_t*)take(2 * S * H * 4);  // two sets: consecutive decode launches alternate
     l.due_ctl = (int32_t*)take(16);
     const size_t ctrl_end = o;
     l.off = (int32_t*)take(nh * 4);
@@ -105,7 +133,7 @@ size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Lay
     l.logit = (float*)take(slots * r * 4);
     l.ml = (float2*)take(nh * r * 8);
     l.rows = (float*)take(S * H * r * Lmax * 4);
-    l.partial = (float*)take(max_chunks * (d + 2) * 4);
+    l.partial = (float*)take(2 * max_chunks * (d + 2) * 4);
     l.due_list = (int32_t*)take(nh * 4);
     l.plan_pre = (int32_t*)take(nh * 4);
     l.plan_head = (int4*)take(nh * 16);
@@ -126,7 +154,7 @@ size_t ctrl_bytes(const hkv_config* c) {
     o = align_up(o + 16);
     o = align_up(o + (size_t)c->num_layers * 4);
     o = align_up(o + (size_t)c->num_layers * 4);
-    o = align_up(o + (size_t)c->num_seqs * c->num_heads * 4);
+    o = align_up(o + 2 * (size_t)c->num_seqs * c->num_heads * 4);
     o = align_up(o + 16);
     return o;
 }
@@ -219,6 +247,7 @@ hkv_status hkv_prefill_classify(hkv_ctx* c, int32_t layer, const void* q, const 
         return HKV_ERR_INVALID_ARG;
     if (c->classified[layer]) return HKV_ERR_STATE;
     if (hkv::pack_smem_bytes(P) > 200 * 1024) return HKV_ERR_INVALID_ARG;
+    note_other(c, stream);
     cudaError_t e = hkv::launch_prefill(c->lay, layer, q, k, v, P, block_stride, out,
                                         (cudaStream_t)stream);
     if (e == cudaSuccess) e = hkv::launch_plan(c->lay, layer, layer + 1, 1, (cudaStream_t)stream);
@@ -242,6 +271,7 @@ hkv_status hkv_append(hkv_ctx* c, int32_t layer, const void* k_t, const void* v_
     hkv_status s = step_check(c, layer, true);
     if (s != HKV_OK) return s;
     if (!k_t || !v_t || !aligned16(k_t) || !aligned16(v_t)) return HKV_ERR_INVALID_ARG;
+    note_other(c, stream);
     cudaError_t e = hkv::launch_append(c->lay, layer, k_t, v_t, (cudaStream_t)stream);
     if (e != cudaSuccess) return HKV_ERR_CUDA;
     c->t_host[layer] += 1;
@@ -255,12 +285,11 @@ hkv_status hkv_decode_attend(hkv_ctx* c, int32_t layer, const void* q_t, void* o
     const int t = c->t_host[layer] - 1;  // newest cached position
     cudaError_t e = cudaSuccess;
     if (c->plan_for[layer] != t) {
+        note_other(c, stream);
         e = hkv::launch_plan(c->lay, layer, layer + 1, 0, (cudaStream_t)stream);
         c->plan_for[layer] = t;
     }
-    if (e == cudaSuccess)
-        e = hkv::launch_decode(c->lay, layer, q_t, nullptr, nullptr, o_t, 0, c->decode_sh,
-                               c->decode_grid, (cudaStream_t)stream);
+    if (e == cudaSuccess) e = decode_launch(c, layer, q_t, nullptr, nullptr, o_t, 0, stream);
     return cuda_status(e);
 }
 
@@ -274,12 +303,11 @@ hkv_status hkv_decode_step(hkv_ctx* c, int32_t layer, const void* q_t, const voi
     const int t = c->t_host[layer];  // position this step appends
     cudaError_t e = cudaSuccess;
     if (c->plan_for[layer] != t) {
+        note_other(c, stream);
         e = hkv::launch_plan(c->lay, layer, layer + 1, 1, (cudaStream_t)stream);
         c->plan_for[layer] = t;
     }
-    if (e == cudaSuccess)
-        e = hkv::launch_decode(c->lay, layer, q_t, k_t, v_t, o_t, 1, c->decode_sh, c->decode_grid,
-                               (cudaStream_t)stream);
+    if (e == cudaSuccess) e = decode_launch(c, layer, q_t, k_t, v_t, o_t, 1, stream);
     if (e != cudaSuccess) return HKV_ERR_CUDA;
     c->t_host[layer] += 1;
     return HKV_OK;
@@ -291,6 +319,7 @@ hkv_status hkv_ste_evict(hkv_ctx* c, int32_t layer_begin, int32_t layer_end, voi
     for (int l = layer_begin; l < layer_end; ++l)
         if (!c->classified[l]) return HKV_ERR_STATE;
     cudaError_t e = cudaSuccess;
+    note_other(c, stream);
     if (c->cfg.mode != HKV_MODE_FULL)
         e = hkv::launch_evict(c->lay, layer_begin, layer_end, c->evict_grid, (cudaStream_t)stream);
     // plans of the next step, made once for all these layers
@@ -386,6 +415,7 @@ hkv_status hkv_clear_error(hkv_ctx* c, void* stream) {
 
 hkv_status hkv_reset(hkv_ctx* c, void* stream) {
     if (!c) return HKV_ERR_INVALID_ARG;
+    note_other(c, stream);
     cudaError_t e = cudaMemsetAsync(c->lay.status, 0, ctrl_bytes(&c->cfg), (cudaStream_t)stream);
     if (e != cudaSuccess) return HKV_ERR_CUDA;
     for (int l = 0; l < c->cfg.num_layers; ++l) {

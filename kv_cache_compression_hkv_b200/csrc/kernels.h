@@ -26,8 +26,12 @@ struct DecodeShape {
     size_t smem;
 };
 DecodeShape decode_shape(const Layout& L, size_t smem_limit);
+// early: the previous launch in `st` is a decode launch of another layer (the
+// plan and cache may then be read before waiting for it); buf: which of the
+// two split-K buffer sets to use (consecutive decode launches alternate).
 cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void* k, const void* v,
-                          void* o, int append, const DecodeShape& sh, int grid, cudaStream_t st);
+                          void* o, int append, const DecodeShape& sh, int grid, int early, int buf,
+                          cudaStream_t st);
 cudaError_t launch_plan(const Layout& L, int l0, int l1, int ahead, cudaStream_t st);
 cudaError_t launch_prefill_rows_simt(int dtype, int d, int n_blocks, const void* q, const void* k,
                                      const void* v, int P, int64_t block_stride, int r, void* out,
