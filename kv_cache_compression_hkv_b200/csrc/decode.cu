@@ -235,15 +235,41 @@ struct HeadCache {
     }
 };
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                     (uint32_t)__cvta_generic_to_shared(dst)),
-                 "l"(src)
-                 : "memory");
+// d = a * b + d on two fp32 lanes at once (packed FMA; each lane rounds as a
+// scalar fmaf would).
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+    asm("{.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%0, %1};\n\t"
+        "fma.rn.f32x2 rc, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rc;}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// The elements of one 16-byte piece as floats (8 bf16 or 4 fp32).
+template <typename T>
+__device__ __forceinline__ void unpack16(const uint4& w, float (&x)[16 / sizeof(T)]) {
+    if constexpr (sizeof(T) == 2) {
+        x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+        x[4] = bf16_lo(w.z); x[5] = bf16_hi(w.z); x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
+    } else {
+        x[0] = __uint_as_float(w.x); x[1] = __uint_as_float(w.y);
+        x[2] = __uint_as_float(w.z); x[3] = __uint_as_float(w.w);
+    }
+}
+
+// Shared memory of one decode warp: its stages, one mbarrier per stage, the
+// softmax numerators of the current chunk, two split-head partial states and
+// a ticket.
+__host__ __device__ inline size_t decode_warp_bytes(int d, int es, int nstage) {
+    const size_t row = (size_t)d * es;
+    return (size_t)nstage * (2 * CHUNK + 1) * row + (size_t)nstage * 8 + CHUNK * 4 +
+           2 * (size_t)(d + 2) * 4 + 16;
+}
+
+constexpr uint64_t DECODE_WAIT_NS = 2000000000ull;  // a copy that takes 2 s has failed
 
 template <typename T, int DPL>
 __global__ void __launch_bounds__(256, 1)
@@ -257,20 +283,19 @@ __global__ void __launch_bounds__(256, 1)
     constexpr int PPR = ROW / 16;                     // 16-byte pieces per row
     constexpr int STAGE = (2 * CHUNK + 1) * ROW;      // K rows, V rows, the query
     constexpr int E = 16 / (int)sizeof(T);            // elements per 16-byte piece
-    constexpr int G = PPR;                            // lanes covering one row (PV)
-    constexpr int TPI = 32 / G;                       // rows per PV step
-    constexpr int RPI = 32 / PPR;                     // rows per copy step
-    static_assert(PPR % 8 == 0 && PPR <= 32, "rows are 8, 16 or 32 pieces");
+    constexpr int G = PPR;                            // lanes covering one row
+    constexpr int TPI = 32 / G;                       // rows per pass
+    constexpr int NPASS = CHUNK / TPI;                // passes per chunk (= G)
+    static_assert(PPR == 8 || PPR == 16 || PPR == 32, "rows are 8, 16 or 32 pieces");
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int NW = blockDim.x >> 5;
-    const int t = append ? L.t_next[layer] : L.t_next[layer] - 1;
-    const int col = t % L.r;
     const int GW = gridDim.x * NW;
     const int gw = blockIdx.x * NW + warp;
+    const int vg = lane / G, vc = lane % G;  // row group and piece of this lane
     const size_t hbase = (size_t)layer * n_heads;
     const size_t lrow = (size_t)layer * L.S * L.R;    // first slot of the layer
-    T* Kp = reinterpret_cast<T*>(L.K);
-    T* Vp = reinterpret_cast<T*>(L.V);
+    const T* Kp = reinterpret_cast<const T*>(L.K);
+    const T* Vp = reinterpret_cast<const T*>(L.V);
     const float qscale = LOG2E / sqrtf((float)D);
 
     // Launched as a programmatic dependent of the previous launch in the
@@ -282,19 +307,34 @@ __global__ void __launch_bounds__(256, 1)
     // can only ever overlap this one, whose split-K buffers (set `buf`) it
     // does not share.
     if (!early) ptx::grid_dep_wait();
+    const int t = append ? L.t_next[layer] : L.t_next[layer] - 1;
+    const int col = t % L.r;
     int* ticket = L.ticket + (size_t)buf * n_heads;
     float* partial = L.partial + (size_t)buf * L.max_chunks * (D + 2);
-    if (GW != L.plan_gw) {
+
+    // shared memory: stages of all warps, then per warp its barriers,
+    // numerators, partial states and ticket
+    unsigned char* my = dsm + (size_t)warp * nstage * STAGE;
+    unsigned char* tail = dsm + (size_t)NW * nstage * STAGE;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(tail) + warp * MAX_STAGES;
+    float* myp = reinterpret_cast<float*>(tail + (size_t)NW * MAX_STAGES * 8) + warp * CHUNK;
+    float* lpart = reinterpret_cast<float*>(tail + (size_t)NW * (MAX_STAGES * 8 + CHUNK * 4));
+    int* ltick = reinterpret_cast<int*>(lpart + (size_t)NW * 2 * (D + 2));
+
+    if (GW != L.plan_gw || nstage > MAX_STAGES) {
         if (early) ptx::grid_dep_wait();
         if (threadIdx.x == 0 && blockIdx.x == 0) latch_error(L, HKV_ERR_STATE, layer);
         return;
     }
+    if (lane == 0) {
+        for (int s = 0; s < nstage; ++s) ptx::mbar_init(&bars[s], 1);
+        ptx::fence_mbar_init();
+    }
+    if (threadIdx.x < NW) ltick[threadIdx.x] = 0;
+    __syncthreads();
+
     const int32_t* pw = L.plan_warp + (size_t)layer * (PLAN_MAX_WARPS + 1);
     const int c_begin = pw[gw], c_end = pw[gw + 1], total = pw[GW];
-
-    unsigned char* my = dsm + (size_t)warp * nstage * STAGE;
-    float* myq = reinterpret_cast<float*>(dsm + (size_t)NW * nstage * STAGE) + warp * (D + CHUNK);
-    float* myp = myq + D;  // this chunk's softmax numerators
 
     if (c_begin < c_end) {
         const int h_begin = L.plan_whead[(size_t)layer * PLAN_MAX_WARPS + gw];
@@ -302,40 +342,50 @@ __global__ void __launch_bounds__(256, 1)
         pc.load(L, hbase, n_heads, h_begin);
         cc = pc;
 
-        // producer cursor: chunk ip of head hp; lane copies piece pc_ of rows
-        // pr_, pr_ + RPI, ...
+        // Producer cursor: chunk ip of head hp.  issue() fills a stage with
+        // bulk copies from lane 0: the cached rows of the chunk, the appended
+        // row from k_t / v_t in its place, and the query for the first chunk
+        // of a head in this range.  part 1 issues only the cached rows (before
+        // the wait on the previous launch), part 2 only the rest, part 0 all.
         int ip = c_begin, hp = h_begin;
-        const int pc_ = lane % PPR, pr_ = lane / PPR;
-        // Issues the copies of chunk ip into `stage`.  With `prior` (before the
-        // wait on the previous launch) the query and the appended row are left
-        // out; the returned (head, appended row or -1, query wanted) lets the
-        // caller put them in after the wait.
-        auto issue = [&](int stage, bool prior) -> int3 {
+        int4 held = make_int4(0, -1, 0, 0);  // part 1's chunk: head, appended row, query wanted
+        auto issue = [&](int stage, int part) {
             int slot, len, jn, sc_, pre, first;
             if (hp - pc.base >= 32) pc.load(L, hbase, n_heads, hp);
             pc.get(hp, slot, len, jn, sc_, pre, first);
             const int tok0 = (ip - first) * CHUNK;
             const int n = min(CHUNK, len - tok0);
-            const int a = append ? jn - tok0 : -1;  // appended row within the chunk (or outside)
-            const size_t row0 = lrow + slot + tok0;
+            int a = append ? jn - tok0 : -1;  // appended row within the chunk
+            if (a >= n) a = -1;
+            const int needq = ip == first || ip == c_begin;
             unsigned char* kd = my + (size_t)stage * STAGE;
             unsigned char* vd = kd + CHUNK * ROW;
             unsigned char* qd = vd + CHUNK * ROW;
-            const T* kf = k_t + (size_t)hp * D + pc_ * E;
-            const T* vf = v_t + (size_t)hp * D + pc_ * E;
-            const bool needq = ip == first || ip == c_begin;  // the head's first chunk here
-            for (int row = pr_; row < n; row += RPI) {
-                const bool fresh = row == a;
-                if (prior && fresh) continue;
-                const T* ks = fresh ? kf : Kp + (row0 + row) * D + pc_ * E;
-                const T* vs = fresh ? vf : Vp + (row0 + row) * D + pc_ * E;
-                cp_async16(kd + row * ROW + ((pc_ ^ (row & 7)) << 4), ks);
-                cp_async16(vd + row * ROW + (pc_ << 4), vs);
+            uint64_t* bar = &bars[stage];
+            if (lane == 0) {
+                if (part != 2) {
+                    const uint32_t bytes = (uint32_t)(2 * n + needq) * ROW;
+                    ptx::mbar_expect_tx(bar, bytes);
+                    const size_t row0 = lrow + slot + tok0;
+                    const int lo = a < 0 ? n : a;      // cached rows [0, lo) and (a, n)
+                    if (lo > 0) {
+                        ptx::bulk_g2s(kd, Kp + row0 * D, lo * ROW, bar);
+                        ptx::bulk_g2s(vd, Vp + row0 * D, lo * ROW, bar);
+                    }
+                    if (a >= 0 && a + 1 < n) {
+                        ptx::bulk_g2s(kd + (a + 1) * ROW, Kp + (row0 + a + 1) * D, (n - a - 1) * ROW, bar);
+                        ptx::bulk_g2s(vd + (a + 1) * ROW, Vp + (row0 + a + 1) * D, (n - a - 1) * ROW, bar);
+                    }
+                }
+                if (part != 1) {
+                    if (a >= 0) {
+                        ptx::bulk_g2s(kd + a * ROW, k_t + (size_t)hp * D, ROW, bar);
+                        ptx::bulk_g2s(vd + a * ROW, v_t + (size_t)hp * D, ROW, bar);
+                    }
+                    if (needq) ptx::bulk_g2s(qd, q_t + (size_t)hp * D, ROW, bar);
+                }
             }
-            if (!prior && needq)
-                for (int c = lane; c < PPR; c += 32) cp_async16(qd + c * 16, q_t + (size_t)hp * D + c * E);
-            cp_async_commit();
-            const int3 rec = make_int3(hp, (a >= 0 && a < n) ? a : -1, needq);
+            held = make_int4(hp, a, needq, 0);
             ++ip;
             if (ip < c_end && pre <= ip) ++hp;
             while (ip < c_end) {  // skip heads with no chunk (capacity errors)
@@ -345,53 +395,40 @@ __global__ void __launch_bounds__(256, 1)
                 if (p2 > ip) break;
                 ++hp;
             }
-            return rec;
         };
-        // prologue: cached rows of the first stages, then the wait, then the
-        // query and appended rows of those stages with plain loads
-        int3 pro[MAX_STAGES];
-        int npro = 0;
-#pragma unroll
-        for (int s = 0; s < MAX_STAGES; ++s)
-            if (s < nstage && ip < c_end) { pro[s] = issue(s, true); npro = s + 1; }
-        if (early) ptx::grid_dep_wait();
-        ptx::grid_dep_trigger();
-        if (lane < PPR) {
-            uint4 wq[MAX_STAGES], wk[MAX_STAGES], wv[MAX_STAGES];
-#pragma unroll
-            for (int s = 0; s < MAX_STAGES; ++s) {
-                if (s >= npro) continue;
-                const size_t at = (size_t)pro[s].x * D + lane * E;
-                if (pro[s].z) wq[s] = *reinterpret_cast<const uint4*>(q_t + at);
-                if (pro[s].y >= 0) {
-                    wk[s] = *reinterpret_cast<const uint4*>(k_t + at);
-                    wv[s] = *reinterpret_cast<const uint4*>(v_t + at);
-                }
-            }
-#pragma unroll
-            for (int s = 0; s < MAX_STAGES; ++s) {
-                if (s >= npro) continue;
-                unsigned char* kd = my + (size_t)s * STAGE;
+        // the rest of part 1's chunk, after the wait
+        auto finish_held = [&](int stage) {
+            if (lane == 0) {
+                unsigned char* kd = my + (size_t)stage * STAGE;
                 unsigned char* vd = kd + CHUNK * ROW;
-                if (pro[s].z) *reinterpret_cast<uint4*>(vd + CHUNK * ROW + lane * 16) = wq[s];
-                const int a = pro[s].y;
-                if (a >= 0) {
-                    *reinterpret_cast<uint4*>(kd + a * ROW + ((lane ^ (a & 7)) << 4)) = wk[s];
-                    *reinterpret_cast<uint4*>(vd + a * ROW + lane * 16) = wv[s];
+                uint64_t* bar = &bars[stage];
+                if (held.y >= 0) {
+                    ptx::bulk_g2s(kd + held.y * ROW, k_t + (size_t)held.x * D, ROW, bar);
+                    ptx::bulk_g2s(vd + held.y * ROW, v_t + (size_t)held.x * D, ROW, bar);
                 }
+                if (held.z) ptx::bulk_g2s(vd + CHUNK * ROW, q_t + (size_t)held.x * D, ROW, bar);
             }
+        };
+        if (early) {
+            issue(0, 1);
+            ptx::grid_dep_wait();
+            ptx::grid_dep_trigger();
+            finish_held(0);
+        } else {
+            ptx::grid_dep_trigger();
+            issue(0, 0);
         }
+        for (int s = 1; s < nstage && ip < c_end; ++s) issue(s, 0);
 
         int hc = h_begin;
         int seg0 = c_begin;
-        // PV accumulators: lane (vg, vc) = (lane / G, lane % G) sums rows
-        // j = vg (mod TPI) of its 16-byte piece vc; the groups are added up once
-        // per head
-        const int vg = lane / G, vc = lane % G;
+        uint32_t phase = 0;  // bit s: parity of stage s's next phase
+        bool failed = false;
         // m: the warp's reference maximum (log2 domain), raised only when a
         // logit passes it by more than RESCALE; ls: this lane's share of the
-        // softmax denominator; qv: the pre-scaled query of the current head
-        float m = -INFINITY, ls = 0.f, acc[E], qv[D];
+        // softmax denominator; qv: this lane's piece of the pre-scaled query;
+        // acc: this lane's piece of the weighted V sum over its row group
+        float m = -INFINITY, ls = 0.f, acc[E], qv[E];
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[e] = 0.f;
         int slot, len, jn, scoring, pre, first;
@@ -402,68 +439,57 @@ __global__ void __launch_bounds__(256, 1)
             cc.get(hc, slot, len, jn, scoring, pre, first);
         }
 
-        for (int i = c_begin; i < c_end; ++i) {
+        int i = c_begin;
+        for (; i < c_end; ++i) {
             const int k = i - c_begin;
             const int stage = k % nstage;
-            const int pending = (ip - c_begin) - (k + 1);  // groups issued after this one
-            if (pending >= 2) cp_async_wait<2>();
-            else if (pending == 1) cp_async_wait<1>();
-            else cp_async_wait<0>();
-            __syncwarp();
+            const bool ok = ptx::mbar_wait(&bars[stage], (phase >> stage) & 1u, DECODE_WAIT_NS);
+            if (__any_sync(FULL_MASK, !ok)) {  // the whole warp stops
+                if (lane == 0) latch_error(L, HKV_ERR_TIMEOUT, (int)(hbase + hc));
+                failed = true;
+                break;
+            }
+            phase ^= 1u << stage;
             const int tok0 = (i - first) * CHUNK;
             const int n = min(CHUNK, len - tok0);
             const unsigned char* kst = my + (size_t)stage * STAGE;
             const unsigned char* vst = kst + CHUNK * ROW;
-            if (i == seg0) {
-                // a new head: every lane reads the whole query (broadcast reads)
-                const unsigned char* qs = vst + CHUNK * ROW;
+            if (i == seg0) {  // a new head: this lane's piece of its query
+                float x[E];
+                unpack16<T>(*reinterpret_cast<const uint4*>(vst + CHUNK * ROW + vc * 16), x);
 #pragma unroll
-                for (int c = 0; c < PPR; ++c) {
-                    const uint4 w = *reinterpret_cast<const uint4*>(qs + c * 16);
-                    if constexpr (sizeof(T) == 2) {
-                        qv[c * 8 + 0] = bf16_lo(w.x) * qscale; qv[c * 8 + 1] = bf16_hi(w.x) * qscale;
-                        qv[c * 8 + 2] = bf16_lo(w.y) * qscale; qv[c * 8 + 3] = bf16_hi(w.y) * qscale;
-                        qv[c * 8 + 4] = bf16_lo(w.z) * qscale; qv[c * 8 + 5] = bf16_hi(w.z) * qscale;
-                        qv[c * 8 + 6] = bf16_lo(w.w) * qscale; qv[c * 8 + 7] = bf16_hi(w.w) * qscale;
-                    } else {
-                        qv[c * 4 + 0] = __uint_as_float(w.x) * qscale;
-                        qv[c * 4 + 1] = __uint_as_float(w.y) * qscale;
-                        qv[c * 4 + 2] = __uint_as_float(w.z) * qscale;
-                        qv[c * 4 + 3] = __uint_as_float(w.w) * qscale;
-                    }
+                for (int e = 0; e < E; ++e) qv[e] = x[e] * qscale;
+            }
+            // QK: pass p, lane (vg, vc) takes piece vc of row p * TPI + vg;
+            // a butterfly over the G lanes of a group then leaves lane
+            // (vg, vc) the whole dot product of row j = vc * TPI + vg
+            float part[NPASS];
+#pragma unroll
+            for (int p = 0; p < NPASS; ++p) {
+                const int row = p * TPI + vg;
+                float a0 = 0.f, a1 = 0.f;
+                if (p * TPI < n) {
+                    float x[E];
+                    unpack16<T>(*reinterpret_cast<const uint4*>(kst + row * ROW + vc * 16), x);
+#pragma unroll
+                    for (int e = 0; e < E; e += 2) ffma2(a0, a1, qv[e], qv[e + 1], x[e], x[e + 1]);
+                }
+                part[p] = a0 + a1;
+            }
+#pragma unroll
+            for (int h = NPASS / 2; h >= 1; h >>= 1) {
+                const bool upper = (vc & h) != 0;
+#pragma unroll
+                for (int u = 0; u < h; ++u) {
+                    const float send = upper ? part[u] : part[u + h];
+                    const float keep = upper ? part[u + h] : part[u];
+                    part[u] = keep + __shfl_xor_sync(FULL_MASK, send, h);
                 }
             }
-            // lane j: dot product of the query with row j; row j's pieces sit
-            // at piece ^ (j & 7), so the lanes of a quarter-warp read 8
-            // different bank groups while all reading the same query piece
-            float sl = -INFINITY;
-            if (lane < n) {
-                const unsigned char* krow = kst + lane * ROW;
-                const int sw = lane & 7;
-                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-                for (int c = 0; c < PPR; ++c) {
-                    const uint4 kw = *reinterpret_cast<const uint4*>(krow + ((c ^ sw) << 4));
-                    if constexpr (sizeof(T) == 2) {
-                        a0 = fmaf(qv[c * 8 + 0], bf16_lo(kw.x), a0);
-                        a1 = fmaf(qv[c * 8 + 1], bf16_hi(kw.x), a1);
-                        a2 = fmaf(qv[c * 8 + 2], bf16_lo(kw.y), a2);
-                        a3 = fmaf(qv[c * 8 + 3], bf16_hi(kw.y), a3);
-                        a0 = fmaf(qv[c * 8 + 4], bf16_lo(kw.z), a0);
-                        a1 = fmaf(qv[c * 8 + 5], bf16_hi(kw.z), a1);
-                        a2 = fmaf(qv[c * 8 + 6], bf16_lo(kw.w), a2);
-                        a3 = fmaf(qv[c * 8 + 7], bf16_hi(kw.w), a3);
-                    } else {
-                        a0 = fmaf(qv[c * 4 + 0], __uint_as_float(kw.x), a0);
-                        a1 = fmaf(qv[c * 4 + 1], __uint_as_float(kw.y), a1);
-                        a2 = fmaf(qv[c * 4 + 2], __uint_as_float(kw.z), a2);
-                        a3 = fmaf(qv[c * 4 + 3], __uint_as_float(kw.w), a3);
-                    }
-                }
-                sl = (a0 + a1) + (a2 + a3);
-            }
+            const int j = vc * TPI + vg;  // this lane's row
+            const float sl = j < n ? part[0] : -INFINITY;
             const size_t row0 = lrow + slot + tok0;
-            if (scoring && lane < n) L.logit[(row0 + lane) * L.r + col] = sl;
+            if (scoring && j < n) L.logit[(row0 + j) * L.r + col] = sl;
             // raise the reference only when some logit passes it by more than
             // RESCALE (weights stay below 2^RESCALE); one vote otherwise
             if (__any_sync(FULL_MASK, sl > m + RESCALE)) {
@@ -477,35 +503,26 @@ __global__ void __launch_bounds__(256, 1)
                 for (int e = 0; e < E; ++e) acc[e] *= alpha;
                 m = mn;
             }
-            const float p = lane < n ? exp2f(sl - m) : 0.f;
-            ls += p;
-            // weighted V: p_j parked in shared memory; each lane group reads
-            // whole 16-byte pieces of its rows; two accumulator chains
-            myp[lane] = p;
+            const float pj_own = j < n ? exp2f(sl - m) : 0.f;
+            ls += pj_own;
+            myp[j] = pj_own;
             __syncwarp();
+            // PV: lane (vg, vc) adds p_j times piece vc of rows j = vg (mod TPI)
             float pa[2][E];
 #pragma unroll
             for (int u = 0; u < 2; ++u)
 #pragma unroll
                 for (int e = 0; e < E; ++e) pa[u][e] = 0.f;
 #pragma unroll
-            for (int jb = 0; jb < CHUNK; jb += TPI) {
-                const int j = jb + vg;
-                if (jb < n && j < n) {
-                    const float pj = myp[j];
-                    const uint4 vw = *reinterpret_cast<const uint4*>(vst + j * ROW + vc * 16);
-                    float* pu = pa[(jb / TPI) & 1];
-                    if constexpr (sizeof(T) == 2) {
-                        pu[0] = fmaf(pj, bf16_lo(vw.x), pu[0]); pu[1] = fmaf(pj, bf16_hi(vw.x), pu[1]);
-                        pu[2] = fmaf(pj, bf16_lo(vw.y), pu[2]); pu[3] = fmaf(pj, bf16_hi(vw.y), pu[3]);
-                        pu[4] = fmaf(pj, bf16_lo(vw.z), pu[4]); pu[5] = fmaf(pj, bf16_hi(vw.z), pu[5]);
-                        pu[6] = fmaf(pj, bf16_lo(vw.w), pu[6]); pu[7] = fmaf(pj, bf16_hi(vw.w), pu[7]);
-                    } else {
-                        pu[0] = fmaf(pj, __uint_as_float(vw.x), pu[0]);
-                        pu[1] = fmaf(pj, __uint_as_float(vw.y), pu[1]);
-                        pu[2] = fmaf(pj, __uint_as_float(vw.z), pu[2]);
-                        pu[3] = fmaf(pj, __uint_as_float(vw.w), pu[3]);
-                    }
+            for (int p = 0; p < NPASS; ++p) {
+                const int jr = p * TPI + vg;
+                if (p * TPI < n && jr < n) {
+                    const float pj = myp[jr];
+                    float x[E];
+                    unpack16<T>(*reinterpret_cast<const uint4*>(vst + jr * ROW + vc * 16), x);
+                    float* pu = pa[p & 1];
+#pragma unroll
+                    for (int e = 0; e < E; e += 2) ffma2(pu[e], pu[e + 1], pj, pj, x[e], x[e + 1]);
                 }
             }
 #pragma unroll
@@ -513,17 +530,15 @@ __global__ void __launch_bounds__(256, 1)
             // the appended token joins the cache
             const int a = jn - tok0;
             if (append && a >= 0 && a < n) {
-                constexpr int LB = DPL * (int)sizeof(T);  // bytes per lane, within one piece
-                const int b = lane * LB;
                 Raw<T, DPL> kr, vr;
-                kr.load_shared(reinterpret_cast<const T*>(kst + a * ROW + ((((b >> 4) ^ (a & 7)) << 4) | (b & 15))));
-                vr.load_shared(reinterpret_cast<const T*>(vst + a * ROW + b));
-                kr.store(Kp + (row0 + a) * D + lane * DPL);
-                vr.store(Vp + (row0 + a) * D + lane * DPL);
+                kr.load_shared(reinterpret_cast<const T*>(kst + a * ROW) + lane * DPL);
+                vr.load_shared(reinterpret_cast<const T*>(vst + a * ROW) + lane * DPL);
+                kr.store(reinterpret_cast<T*>(L.K) + (row0 + a) * D + lane * DPL);
+                vr.store(reinterpret_cast<T*>(L.V) + (row0 + a) * D + lane * DPL);
                 if (lane == 0) L.pos[row0 + a] = t;
             }
-            __syncwarp();
-            if (ip < c_end) issue(stage, false);
+            __syncwarp();  // every lane is done with this stage
+            if (ip < c_end) issue(stage, 0);
             if (i + 1 < c_end && pre > i + 1) continue;  // head goes on
 
             // end of this warp's segment of head hc: add up the row groups
@@ -546,49 +561,68 @@ __global__ void __launch_bounds__(256, 1)
                 if (lane < G) store_row<T, E>(o_t + (size_t)hc * D + vc * E, o);
                 if (scoring && lane == 0) L.ml[hx * L.r + col] = make_float2(m, l);
             } else {
-                float* pp = partial + (size_t)seg0 * (D + 2);
+                const int w_a = range_owner(first, total, GW);
+                const int w_b = range_owner(pre - 1, total, GW);
+                int segs = 0;
+                for (int w = w_a; w <= w_b; ++w)
+                    segs += range_begin(w, total, GW) < range_begin(w + 1, total, GW);
+                // segments all in this block meet in shared memory, others in
+                // global memory; the last one in merges (no waiting)
+                const bool local = w_a / NW == (int)blockIdx.x && w_b / NW == (int)blockIdx.x;
+                float* pp = local ? lpart + (size_t)(warp * 2 + (seg0 == c_begin ? 0 : 1)) * (D + 2)
+                                  : partial + (size_t)seg0 * (D + 2);
                 if (lane == 0) { pp[0] = m; pp[1] = l; }
                 if (lane < G) {
 #pragma unroll
                     for (int e = 0; e < E; ++e) pp[2 + vc * E + e] = acc[e];
                 }
                 __syncwarp();  // the lanes' partial stores precede lane 0's release
-                const int w_a = range_owner(first, total, GW);
-                const int w_b = range_owner(pre - 1, total, GW);
-                int segs = 0;
-                for (int w = w_a; w <= w_b; ++w)
-                    segs += range_begin(w, total, GW) < range_begin(w + 1, total, GW);
                 int prev = 0;
                 if (lane == 0) {
-                    // release: this warp's partial before the ticket; acquire:
-                    // the other segments' partials for the last one in
-                    cuda::atomic_ref<int, cuda::thread_scope_device> tk(ticket[hc]);
-                    prev = tk.fetch_add(1, cuda::memory_order_acq_rel);
+                    if (local) {
+                        __threadfence_block();
+                        prev = atomicAdd(&ltick[w_a % NW], 1);
+                        __threadfence_block();
+                    } else {
+                        // release: this warp's partial before the ticket;
+                        // acquire: the other segments' for the last one in
+                        cuda::atomic_ref<int, cuda::thread_scope_device> tk(ticket[hc]);
+                        prev = tk.fetch_add(1, cuda::memory_order_acq_rel);
+                    }
                 }
                 prev = __shfl_sync(FULL_MASK, prev, 0);
                 __syncwarp();  // lane 0's acquire before every lane's partial loads
                 if (prev == segs - 1) {
-                    // last segment in: merge (lane-parallel over segments)
-                    if (lane == 0) ticket[hc] = 0;
-                    float M = -INFINITY;
-                    for (int w = w_a + lane; w <= w_b; w += 32) {
+                    if (lane == 0 && !local) ticket[hc] = 0;
+                    auto part_of = [&](int w) -> const float* {
                         const int rb = range_begin(w, total, GW);
-                        if (rb < range_begin(w + 1, total, GW))
-                            M = fmaxf(M, __ldcg(partial + (size_t)max(rb, first) * (D + 2)));
-                    }
+                        if (local)
+                            return lpart + (size_t)((w % NW) * 2 + (max(rb, first) == rb ? 0 : 1)) * (D + 2);
+                        return partial + (size_t)max(rb, first) * (D + 2);
+                    };
+                    float M = -INFINITY;
+                    for (int w = w_a + lane; w <= w_b; w += 32)
+                        if (range_begin(w, total, GW) < range_begin(w + 1, total, GW))
+                            M = fmaxf(M, local ? *part_of(w) : __ldcg(part_of(w)));
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, o));
                     float Ls = 0.f, o[E];
 #pragma unroll
                     for (int e = 0; e < E; ++e) o[e] = 0.f;
                     for (int w = w_a; w <= w_b; ++w) {
-                        const int rb = range_begin(w, total, GW);
-                        if (rb >= range_begin(w + 1, total, GW)) continue;
-                        const float* pi = partial + (size_t)max(rb, first) * (D + 2);
-                        const float wt = exp2f(__ldcg(pi) - M);
-                        Ls = fmaf(__ldcg(pi + 1), wt, Ls);
+                        if (range_begin(w, total, GW) >= range_begin(w + 1, total, GW)) continue;
+                        const float* pi = part_of(w);
+                        if (local) {
+                            const float wt = exp2f(pi[0] - M);
+                            Ls = fmaf(pi[1], wt, Ls);
 #pragma unroll
-                        for (int e = 0; e < E; ++e) o[e] = fmaf(__ldcg(pi + 2 + vc * E + e), wt, o[e]);
+                            for (int e = 0; e < E; ++e) o[e] = fmaf(pi[2 + vc * E + e], wt, o[e]);
+                        } else {
+                            const float wt = exp2f(__ldcg(pi) - M);
+                            Ls = fmaf(__ldcg(pi + 1), wt, Ls);
+#pragma unroll
+                            for (int e = 0; e < E; ++e) o[e] = fmaf(__ldcg(pi + 2 + vc * E + e), wt, o[e]);
+                        }
                     }
                     const float inv = 1.0f / Ls;
 #pragma unroll
@@ -611,7 +645,15 @@ __global__ void __launch_bounds__(256, 1)
                 } while (pre <= i + 1);
             }
         }
-        cp_async_wait<0>();
+        if (failed) {
+            // copies still in flight into this warp's stages: wait for them
+            // (briefly) before the block's shared memory is given up
+            for (int k = i - c_begin; k < ip - c_begin; ++k) {
+                const int stage = k % nstage;
+                if (!ptx::mbar_wait(&bars[stage], (phase >> stage) & 1u, DECODE_WAIT_NS / 8)) break;
+                phase ^= 1u << stage;
+            }
+        }
     } else {
         if (early) ptx::grid_dep_wait();
         ptx::grid_dep_trigger();
@@ -668,14 +710,14 @@ __global__ void __launch_bounds__(256) append_kernel(Layout L, int layer, const 
 // ---------------------------------------------------------------------------
 
 DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
-    const size_t row = (size_t)L.d * (L.dtype == HKV_DTYPE_F32 ? 4 : 2);
-    const size_t stage = (2 * CHUNK + 1) * row;
+    const int es = L.dtype == HKV_DTYPE_F32 ? 4 : 2;
     DecodeShape sh{0, 0, 0};
-    for (int ns = 3; ns >= 2 && sh.warps == 0; --ns) {
-        const size_t per = ns * stage + (size_t)(L.d + CHUNK) * 4;
+    for (int ns = MAX_STAGES; ns >= 2 && sh.warps == 0; --ns) {
+        // the per-warp tail regions are laid out for MAX_STAGES barriers
+        const size_t per = decode_warp_bytes(L.d, es, ns) + (MAX_STAGES - ns) * 8;
         int w = (int)((smem_limit - 1024) / per);
         if (w > 8) w = 8;
-        if (w >= (ns == 3 ? 6 : 1)) sh = DecodeShape{w, ns, 1024 + (size_t)w * per};
+        if (w >= (ns == MAX_STAGES ? 6 : 1)) sh = DecodeShape{w, ns, 1024 + (size_t)w * per};
     }
     return sh;
 }
