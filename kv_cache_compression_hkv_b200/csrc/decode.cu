@@ -4,15 +4,15 @@
 //
 // Work decomposition: every head's cache is cut into chunks of 32 tokens.
 // A plan (plan_kernel, once per step and layer) prefix-sums the heads' chunk
-// counts and cuts the layer's chunk list into equal contiguous ranges, one
-// per warp of the persistent decode grid.  Each warp walks its range with a
-// pipeline of shared-memory stages filled by per-lane 16-byte cp.async
-// copies, keeps the online softmax of the current head in registers across
-// that head's chunks, and finishes a head it holds entirely; a head split
-// between warps leaves one partial per warp and the last to arrive (atomic
-// ticket, no spinning) merges them.  Global heads within r steps of their
-// eviction also store their exp2-domain logits per slot, which the eviction
-// normalises with the (max, sum) stored here.
+// counts, writes one descriptor per chunk and cuts the layer's chunk list
+// into equal contiguous ranges, one per warp of the persistent decode grid.
+// Each warp walks its range with a pipeline of shared-memory stages filled
+// by bulk copies (TMA engine) and keeps the online softmax of the current
+// head in registers across that head's chunks; it finishes a head it holds
+// entirely, and a head split between warps leaves one partial per warp, the
+// last to arrive (atomic ticket, no spinning) merging them.  Global heads
+// within r steps of their eviction also store their exp2-domain logits per
+// slot, which the eviction normalises with the (max, sum) stored here.
 #include <math.h>
 
 #include <cuda/atomic>
@@ -28,6 +28,8 @@ namespace hkv {
 constexpr float RESCALE = 8.f;
 // Most pipeline stages a decode warp keeps in flight.
 constexpr int MAX_STAGES = 3;
+// Most warps of one decode block (one block per SM).
+constexpr int DECODE_MAX_WARPS = 12;
 
 // Packed storage of DPL consecutive elements of one row.
 template <typename T, int DPL> struct Raw;
@@ -118,26 +120,66 @@ __device__ __forceinline__ void store_row(T* p, const float (&x)[DPL]) {
     }
 }
 
-// First chunk of warp w's range when `total` chunks go to `gw` warps.
+// First chunk of warp w's range when `total` chunks go to `gw` warps
+// (32-bit arithmetic while the products fit).
 __device__ __forceinline__ int range_begin(int w, int total, int gw) {
+    if (total < (1 << 19)) return (int)((uint32_t)w * (uint32_t)total / (uint32_t)gw);
     return (int)((int64_t)w * total / gw);
 }
 // Warp whose range holds chunk c.
 __device__ __forceinline__ int range_owner(int c, int total, int gw) {
+    if (total < (1 << 19)) return (int)(((uint32_t)(c + 1) * (uint32_t)gw - 1u) / (uint32_t)total);
     return (int)(((int64_t)(c + 1) * gw - 1) / total);
+}
+
+// ---------------------------------------------------------------------------
+// Chunk descriptors.  The plan describes every chunk of a layer in one int4:
+//   x: layer-relative row of the chunk's first token
+//   y: head (s * H + h)
+//   z: rows n (bits 0-5) | appended row + 1 (bits 6-11, 0: none) | first
+//      chunk of its head (bit 12) | last chunk (bit 13) | scoring head
+//      (bit 14) | non-empty warp ranges holding the head (bits 16-31)
+//   w: first warp range holding the head | (last - first) << 12
+// ---------------------------------------------------------------------------
+struct ChunkDesc {
+    int row, head, n, a, first, last, scoring, segs, wa, wb;
+    __device__ __forceinline__ static ChunkDesc of(const int4& v) {
+        ChunkDesc c;
+        c.row = v.x;
+        c.head = v.y;
+        c.n = v.z & 63;
+        c.a = ((v.z >> 6) & 63) - 1;
+        c.first = (v.z >> 12) & 1;
+        c.last = (v.z >> 13) & 1;
+        c.scoring = (v.z >> 14) & 1;
+        c.segs = (int)((uint32_t)v.z >> 16);
+        c.wa = v.w & 0xfff;
+        c.wb = c.wa + (v.w >> 12);
+        return c;
+    }
+};
+
+__device__ __forceinline__ int4 shfl_int4(const int4& v, int src) {
+    return make_int4(__shfl_sync(FULL_MASK, v.x, src), __shfl_sync(FULL_MASK, v.y, src),
+                     __shfl_sync(FULL_MASK, v.z, src), __shfl_sync(FULL_MASK, v.w, src));
 }
 
 // ---------------------------------------------------------------------------
 // The plan of a layer's decode launch at step t (ahead = 1: the step of the
 // next append, t_next; ahead = 0: the newest cached position, t_next - 1).
-// One block per layer: per-head facts, the chunk-count prefix, and for every
-// warp of the decode grid its first chunk and the head holding it.
+// One block per layer: per-head facts in shared memory, the chunk-count
+// prefix, every chunk's descriptor, and for every warp of the decode grid
+// its range and a copy of its first chunk's descriptor.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead) {
-    extern __shared__ int32_t cnt[];
+    extern __shared__ int32_t psm[];
     __shared__ int wsum[32];
     const int layer = l0 + blockIdx.x;
     const int n = L.S * L.H;
+    int32_t* cnt = psm;            // chunk counts, then their inclusive prefix
+    int32_t* hslot = psm + n;      // layer-relative row of the head's first token
+    int32_t* hlen = psm + 2 * n;   // len << 16 | appended slot
+    int32_t* hscore = psm + 3 * n; // scoring flag
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, NW = blockDim.x >> 5;
     const int t = L.t_next[layer] - 1 + ahead;
     if (t >= L.L) return;  // the sequence is complete: no step left to plan
@@ -152,9 +194,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
             c = 0;
         }
         const int jn = append_slot(L, hx, t, len);
-        const int scoring = L.label[hx] == 0 && L.mode != HKV_MODE_FULL && len > cap - L.r;
-        const int slot = (i / L.H) * L.R + L.off[hx];
-        L.plan_head[hbase + i] = make_int4(slot, (len << 16) | (jn & 0xffff), scoring, 0);
+        hscore[i] = L.label[hx] == 0 && L.mode != HKV_MODE_FULL && len > cap - L.r;
+        hslot[i] = (i / L.H) * L.R + L.off[hx];
+        hlen[i] = (len << 16) | (jn & 0xffff);
         cnt[i] = c;
     }
     __syncthreads();
@@ -185,55 +227,56 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
     for (int i = i0; i < i1; ++i) cnt[i] += offset;
     __syncthreads();
     const int total = cnt[n - 1];
-    for (int i = tid; i < n; i += blockDim.x) L.plan_pre[hbase + i] = cnt[i];
     const int GW = L.plan_gw;
-    int32_t* pw = L.plan_warp + (size_t)layer * (PLAN_MAX_WARPS + 1);
-    int32_t* ph = L.plan_whead + (size_t)layer * PLAN_MAX_WARPS;
-    for (int w = tid; w <= GW; w += blockDim.x) {
-        const int cb = range_begin(w, total, GW);
-        pw[w] = cb;
-        if (w < GW) {
+    if (total > L.max_chunks) {  // cannot happen for a consistent cache
+        if (tid == 0) latch_error(L, HKV_ERR_STATE, layer);
+        return;
+    }
+    // descriptor of the k-th chunk of head i (chunks c0 .. c1-1), given the
+    // head's warp-range fields hz (segments << 16) and hw
+    auto desc = [&](int i, int k, int c1mc0, int hz, int hw) -> int4 {
+        const int len = hlen[i] >> 16, jn = (int)(int16_t)(hlen[i] & 0xffff);
+        const int tok0 = k * CHUNK;
+        const int nr = min(CHUNK, len - tok0);
+        const int a = jn - tok0;
+        const int z = nr | ((a >= 0 && a < nr ? a + 1 : 0) << 6) | ((k == 0) << 12) |
+                      ((k == c1mc0 - 1) << 13) | (hscore[i] << 14) | hz;
+        return make_int4(hslot[i] + tok0, i, z, hw);
+    };
+    auto head_ranges = [&](int c0, int c1, int& hz, int& hw) {
+        const int wa = range_owner(c0, total, GW), wb = range_owner(c1 - 1, total, GW);
+        int segs = 0;
+        for (int w = wa; w <= wb; ++w) segs += range_begin(w, total, GW) < range_begin(w + 1, total, GW);
+        hz = segs << 16;
+        hw = wa | ((wb - wa) << 12);
+    };
+    int4* dsc = L.plan_desc + (size_t)layer * L.max_chunks;
+    for (int i = tid; i < n; i += blockDim.x) {
+        const int c1 = cnt[i], c0 = i ? cnt[i - 1] : 0;
+        if (c1 == c0) continue;
+        int hz, hw;
+        head_ranges(c0, c1, hz, hw);
+        for (int c = c0; c < c1; ++c) dsc[c] = desc(i, c - c0, c1 - c0, hz, hw);
+    }
+    int4* pw = L.plan_warp + (size_t)layer * PLAN_MAX_WARPS * 2;
+    for (int w = tid; w < GW; w += blockDim.x) {
+        const int cb = range_begin(w, total, GW), ce = range_begin(w + 1, total, GW);
+        int4 first = make_int4(0, 0, 0, 0);
+        if (cb < ce) {
             int lo = 0, hi = n - 1;  // head holding chunk cb
             while (lo < hi) {
                 const int mid = (lo + hi) >> 1;
                 if (cnt[mid] > cb) hi = mid; else lo = mid + 1;
             }
-            ph[w] = lo;
+            const int c0 = lo ? cnt[lo - 1] : 0;
+            int hz, hw;
+            head_ranges(c0, cnt[lo], hz, hw);
+            first = desc(lo, cb - c0, cnt[lo] - c0, hz, hw);
         }
+        pw[2 * w] = make_int4(cb, ce, total, 0);
+        pw[2 * w + 1] = first;
     }
 }
-
-// Head facts of the 32 heads [base, base + 32) of a layer, lane i holding
-// head base + i.
-struct HeadCache {
-    int base;
-    int slot, lenjn, scoring, pre, first;
-    __device__ void load(const Layout& L, size_t hbase, int n, int b) {
-        const int lane = threadIdx.x & 31;
-        base = b;
-        const int h = b + lane;
-        if (h < n) {
-            const int4 v = L.plan_head[hbase + h];
-            slot = v.x; lenjn = v.y; scoring = v.z;
-            pre = L.plan_pre[hbase + h];
-            first = h ? L.plan_pre[hbase + h - 1] : 0;
-        } else {
-            slot = 0; lenjn = 0; scoring = 0; pre = 0x7fffffff; first = 0x7fffffff;
-        }
-    }
-    // facts of head h (base <= h < base + 32), broadcast to every lane
-    __device__ void get(int h, int& o_slot, int& o_len, int& o_jn, int& o_scoring, int& o_pre,
-                        int& o_first) const {
-        const int src = h - base;
-        o_slot = __shfl_sync(FULL_MASK, slot, src);
-        const int lj = __shfl_sync(FULL_MASK, lenjn, src);
-        o_len = lj >> 16;
-        o_jn = (int)(int16_t)(lj & 0xffff);
-        o_scoring = __shfl_sync(FULL_MASK, scoring, src);
-        o_pre = __shfl_sync(FULL_MASK, pre, src);
-        o_first = __shfl_sync(FULL_MASK, first, src);
-    }
-};
 
 // d = a * b + d on two fp32 lanes at once (packed FMA; each lane rounds as a
 // scalar fmaf would).
@@ -246,6 +289,19 @@ __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, 
         "mov.b64 {%0, %1}, rc;}"
         : "+f"(d0), "+f"(d1)
         : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// d0 += lo(w) * lo(q) and d1 += hi(w) * hi(q) for two packed bf16 pairs: the
+// products of bf16 values are exact in fp32, so this equals unpacking both
+// operands and a scalar fmaf, without the unpacking.
+__device__ __forceinline__ void fma_bf16x2(float& d0, float& d1, uint32_t w, uint32_t q) {
+    asm("{.reg .b16 wl, wh, ql, qh;\n\t"
+        "mov.b32 {wl, wh}, %2;\n\t"
+        "mov.b32 {ql, qh}, %3;\n\t"
+        "fma.rn.f32.bf16 %0, wl, ql, %0;\n\t"
+        "fma.rn.f32.bf16 %1, wh, qh, %1;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "r"(w), "r"(q));
 }
 
 // The elements of one 16-byte piece as floats (8 bf16 or 4 fp32).
@@ -272,7 +328,7 @@ __host__ __device__ inline size_t decode_warp_bytes(int d, int es, int nstage) {
 constexpr uint64_t DECODE_WAIT_NS = 2000000000ull;  // a copy that takes 2 s has failed
 
 template <typename T, int DPL>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
     decode_kernel(Layout L, int layer, const T* __restrict__ q_t, const T* __restrict__ k_t,
                   const T* __restrict__ v_t, T* __restrict__ o_t, int append, int nstage,
                   int early, int buf) {
@@ -310,7 +366,7 @@ __global__ void __launch_bounds__(256, 1)
     const int t = append ? L.t_next[layer] : L.t_next[layer] - 1;
     const int col = t % L.r;
     int* ticket = L.ticket + (size_t)buf * n_heads;
-    float* partial = L.partial + (size_t)buf * L.max_chunks * (D + 2);
+    float* partial = L.partial + (size_t)buf * 2 * PLAN_MAX_WARPS * (D + 2);
 
     // shared memory: stages of all warps, then per warp its barriers,
     // numerators, partial states and ticket
@@ -333,132 +389,107 @@ __global__ void __launch_bounds__(256, 1)
     if (threadIdx.x < NW) ltick[threadIdx.x] = 0;
     __syncthreads();
 
-    const int32_t* pw = L.plan_warp + (size_t)layer * (PLAN_MAX_WARPS + 1);
-    const int c_begin = pw[gw], c_end = pw[gw + 1], total = pw[GW];
+    const int4* pw = L.plan_warp + (size_t)layer * PLAN_MAX_WARPS * 2;
+    const int4 wrec = pw[2 * gw], wfirst = pw[2 * gw + 1];
+    const int c_begin = wrec.x, c_end = wrec.y;
+    const int4* dsc = L.plan_desc + (size_t)layer * L.max_chunks;
 
     if (c_begin < c_end) {
-        const int h_begin = L.plan_whead[(size_t)layer * PLAN_MAX_WARPS + gw];
-        HeadCache pc, cc;  // producer's and consumer's view of the heads
-        pc.load(L, hbase, n_heads, h_begin);
-        cc = pc;
-
-        // Producer cursor: chunk ip of head hp.  issue() fills a stage with
-        // bulk copies from lane 0: the cached rows of the chunk, the appended
-        // row from k_t / v_t in its place, and the query for the first chunk
-        // of a head in this range.  part 1 issues only the cached rows (before
-        // the wait on the previous launch), part 2 only the rest, part 0 all.
-        int ip = c_begin, hp = h_begin;
-        int4 held = make_int4(0, -1, 0, 0);  // part 1's chunk: head, appended row, query wanted
-        auto issue = [&](int stage, int part) {
-            int slot, len, jn, sc_, pre, first;
-            if (hp - pc.base >= 32) pc.load(L, hbase, n_heads, hp);
-            pc.get(hp, slot, len, jn, sc_, pre, first);
-            const int tok0 = (ip - first) * CHUNK;
-            const int n = min(CHUNK, len - tok0);
-            int a = append ? jn - tok0 : -1;  // appended row within the chunk
-            if (a >= n) a = -1;
-            const int needq = ip == first || ip == c_begin;
+        // Lane 0's copies of one chunk into a stage: its cached rows, the
+        // appended row from k_t / v_t in its place, and the query when q is
+        // set.  part 1 issues only the cached rows (before the wait on the
+        // previous launch), part 2 only the rest, part 0 all.
+        auto copy_chunk = [&](int stage, int part, const ChunkDesc& c, int q) {
+            if (lane != 0) return;
             unsigned char* kd = my + (size_t)stage * STAGE;
             unsigned char* vd = kd + CHUNK * ROW;
-            unsigned char* qd = vd + CHUNK * ROW;
             uint64_t* bar = &bars[stage];
-            if (lane == 0) {
-                if (part != 2) {
-                    const uint32_t bytes = (uint32_t)(2 * n + needq) * ROW;
-                    ptx::mbar_expect_tx(bar, bytes);
-                    const size_t row0 = lrow + slot + tok0;
-                    const int lo = a < 0 ? n : a;      // cached rows [0, lo) and (a, n)
-                    if (lo > 0) {
-                        ptx::bulk_g2s(kd, Kp + row0 * D, lo * ROW, bar);
-                        ptx::bulk_g2s(vd, Vp + row0 * D, lo * ROW, bar);
-                    }
-                    if (a >= 0 && a + 1 < n) {
-                        ptx::bulk_g2s(kd + (a + 1) * ROW, Kp + (row0 + a + 1) * D, (n - a - 1) * ROW, bar);
-                        ptx::bulk_g2s(vd + (a + 1) * ROW, Vp + (row0 + a + 1) * D, (n - a - 1) * ROW, bar);
-                    }
+            const int a = append ? c.a : -1;
+            if (part != 2) {
+                ptx::mbar_expect_tx(bar, (uint32_t)(2 * c.n + q) * ROW);
+                const size_t row0 = lrow + c.row;
+                const int lo = a < 0 ? c.n : a;  // cached rows [0, lo) and (a, n)
+                if (lo > 0) {
+                    ptx::bulk_g2s(kd, Kp + row0 * D, lo * ROW, bar);
+                    ptx::bulk_g2s(vd, Vp + row0 * D, lo * ROW, bar);
                 }
-                if (part != 1) {
-                    if (a >= 0) {
-                        ptx::bulk_g2s(kd + a * ROW, k_t + (size_t)hp * D, ROW, bar);
-                        ptx::bulk_g2s(vd + a * ROW, v_t + (size_t)hp * D, ROW, bar);
-                    }
-                    if (needq) ptx::bulk_g2s(qd, q_t + (size_t)hp * D, ROW, bar);
+                if (a >= 0 && a + 1 < c.n) {
+                    ptx::bulk_g2s(kd + (a + 1) * ROW, Kp + (row0 + a + 1) * D, (c.n - a - 1) * ROW, bar);
+                    ptx::bulk_g2s(vd + (a + 1) * ROW, Vp + (row0 + a + 1) * D, (c.n - a - 1) * ROW, bar);
                 }
             }
-            held = make_int4(hp, a, needq, 0);
-            ++ip;
-            if (ip < c_end && pre <= ip) ++hp;
-            while (ip < c_end) {  // skip heads with no chunk (capacity errors)
-                if (hp - pc.base >= 32) pc.load(L, hbase, n_heads, hp);
-                int s2, l2, j2, c2, p2, f2;
-                pc.get(hp, s2, l2, j2, c2, p2, f2);
-                if (p2 > ip) break;
-                ++hp;
+            if (part != 1) {
+                if (a >= 0) {
+                    ptx::bulk_g2s(kd + a * ROW, k_t + (size_t)c.head * D, ROW, bar);
+                    ptx::bulk_g2s(vd + a * ROW, v_t + (size_t)c.head * D, ROW, bar);
+                }
+                if (q) ptx::bulk_g2s(vd + CHUNK * ROW, q_t + (size_t)c.head * D, ROW, bar);
             }
         };
-        // the rest of part 1's chunk, after the wait
-        auto finish_held = [&](int stage) {
-            if (lane == 0) {
-                unsigned char* kd = my + (size_t)stage * STAGE;
-                unsigned char* vd = kd + CHUNK * ROW;
-                uint64_t* bar = &bars[stage];
-                if (held.y >= 0) {
-                    ptx::bulk_g2s(kd + held.y * ROW, k_t + (size_t)held.x * D, ROW, bar);
-                    ptx::bulk_g2s(vd + held.y * ROW, v_t + (size_t)held.x * D, ROW, bar);
-                }
-                if (held.z) ptx::bulk_g2s(vd + CHUNK * ROW, q_t + (size_t)held.x * D, ROW, bar);
+        // the range's first chunk straight from the warp's plan record; with
+        // `early` its cached rows go before the wait on the previous launch
+        {
+            const ChunkDesc c0 = ChunkDesc::of(wfirst);
+            if (early) {
+                copy_chunk(0, 1, c0, 1);
+                ptx::grid_dep_wait();
+                ptx::grid_dep_trigger();
+                copy_chunk(0, 2, c0, 1);
+            } else {
+                ptx::grid_dep_trigger();
+                copy_chunk(0, 0, c0, 1);
             }
-        };
-        if (early) {
-            issue(0, 1);
-            ptx::grid_dep_wait();
-            ptx::grid_dep_trigger();
-            finish_held(0);
-        } else {
-            ptx::grid_dep_trigger();
-            issue(0, 0);
         }
-        for (int s = 1; s < nstage && ip < c_end; ++s) issue(s, 0);
+        // descriptors of the range, 32 chunks per window, lane k holding
+        // chunk base + k; the producer (ip) and the consumer (i) keep their
+        // own window
+        auto window = [&](int base) -> int4 {
+            return base + lane < c_end ? dsc[base + lane] : make_int4(0, 0, 0, 0);
+        };
+        int pbase = c_begin, cbase = c_begin;
+        int4 pwin = window(c_begin);
+        int4 cwin = pwin;
+        int ip = c_begin + 1;
+        auto issue = [&](int stage) {
+            if (ip - pbase >= 32) { pbase += 32; pwin = window(pbase); }
+            const ChunkDesc c = ChunkDesc::of(shfl_int4(pwin, ip - pbase));
+            copy_chunk(stage, 0, c, c.first || ip == c_begin);
+            ++ip;
+        };
+        for (int s = 1; s < nstage && ip < c_end; ++s) issue(s);
 
-        int hc = h_begin;
-        int seg0 = c_begin;
         uint32_t phase = 0;  // bit s: parity of stage s's next phase
         bool failed = false;
         // m: the warp's reference maximum (log2 domain), raised only when a
         // logit passes it by more than RESCALE; ls: this lane's share of the
-        // softmax denominator; qv: this lane's piece of the pre-scaled query;
+        // softmax denominator; qw: this lane's 16-byte piece of the query;
         // acc: this lane's piece of the weighted V sum over its row group
-        float m = -INFINITY, ls = 0.f, acc[E], qv[E];
+        float m = -INFINITY, ls = 0.f, acc[E];
+        uint4 qw = make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[e] = 0.f;
-        int slot, len, jn, scoring, pre, first;
-        cc.get(hc, slot, len, jn, scoring, pre, first);
-        while (pre <= c_begin) {  // heads with no chunk before the first one
-            ++hc;
-            if (hc - cc.base >= 32) cc.load(L, hbase, n_heads, hc);
-            cc.get(hc, slot, len, jn, scoring, pre, first);
-        }
+        bool seg_start = true;   // chunk i starts this warp's segment of its head
+        bool seg_whole = false;  // that segment starts at the head's first chunk
 
         int i = c_begin;
         for (; i < c_end; ++i) {
             const int k = i - c_begin;
             const int stage = k % nstage;
-            const bool ok = ptx::mbar_wait(&bars[stage], (phase >> stage) & 1u, DECODE_WAIT_NS);
+            if (i - cbase >= 32) { cbase += 32; cwin = window(cbase); }
+            const ChunkDesc c = ChunkDesc::of(shfl_int4(cwin, i - cbase));
+            const bool ok = ptx::mbar_wait_sleep(&bars[stage], (phase >> stage) & 1u, DECODE_WAIT_NS);
             if (__any_sync(FULL_MASK, !ok)) {  // the whole warp stops
-                if (lane == 0) latch_error(L, HKV_ERR_TIMEOUT, (int)(hbase + hc));
+                if (lane == 0) latch_error(L, HKV_ERR_TIMEOUT, (int)(hbase + c.head));
                 failed = true;
                 break;
             }
             phase ^= 1u << stage;
-            const int tok0 = (i - first) * CHUNK;
-            const int n = min(CHUNK, len - tok0);
+            const int n = c.n;
             const unsigned char* kst = my + (size_t)stage * STAGE;
             const unsigned char* vst = kst + CHUNK * ROW;
-            if (i == seg0) {  // a new head: this lane's piece of its query
-                float x[E];
-                unpack16<T>(*reinterpret_cast<const uint4*>(vst + CHUNK * ROW + vc * 16), x);
-#pragma unroll
-                for (int e = 0; e < E; ++e) qv[e] = x[e] * qscale;
+            if (seg_start) {  // a new head: this lane's piece of its query
+                qw = *reinterpret_cast<const uint4*>(vst + CHUNK * ROW + vc * 16);
+                seg_whole = c.first;
             }
             // QK: pass p, lane (vg, vc) takes piece vc of row p * TPI + vg;
             // a butterfly over the G lanes of a group then leaves lane
@@ -469,10 +500,18 @@ __global__ void __launch_bounds__(256, 1)
                 const int row = p * TPI + vg;
                 float a0 = 0.f, a1 = 0.f;
                 if (p * TPI < n) {
-                    float x[E];
-                    unpack16<T>(*reinterpret_cast<const uint4*>(kst + row * ROW + vc * 16), x);
-#pragma unroll
-                    for (int e = 0; e < E; e += 2) ffma2(a0, a1, qv[e], qv[e + 1], x[e], x[e + 1]);
+                    const uint4 kw = *reinterpret_cast<const uint4*>(kst + row * ROW + vc * 16);
+                    if constexpr (sizeof(T) == 2) {
+                        fma_bf16x2(a0, a1, kw.x, qw.x);
+                        fma_bf16x2(a0, a1, kw.y, qw.y);
+                        fma_bf16x2(a0, a1, kw.z, qw.z);
+                        fma_bf16x2(a0, a1, kw.w, qw.w);
+                    } else {
+                        ffma2(a0, a1, __uint_as_float(qw.x), __uint_as_float(qw.y),
+                              __uint_as_float(kw.x), __uint_as_float(kw.y));
+                        ffma2(a0, a1, __uint_as_float(qw.z), __uint_as_float(qw.w),
+                              __uint_as_float(kw.z), __uint_as_float(kw.w));
+                    }
                 }
                 part[p] = a0 + a1;
             }
@@ -487,9 +526,9 @@ __global__ void __launch_bounds__(256, 1)
                 }
             }
             const int j = vc * TPI + vg;  // this lane's row
-            const float sl = j < n ? part[0] : -INFINITY;
-            const size_t row0 = lrow + slot + tok0;
-            if (scoring && j < n) L.logit[(row0 + j) * L.r + col] = sl;
+            const float sl = j < n ? part[0] * qscale : -INFINITY;
+            const size_t row0 = lrow + c.row;
+            if (c.scoring && j < n) L.logit[(row0 + j) * L.r + col] = sl;
             // raise the reference only when some logit passes it by more than
             // RESCALE (weights stay below 2^RESCALE); one vote otherwise
             if (__any_sync(FULL_MASK, sl > m + RESCALE)) {
@@ -528,8 +567,8 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
             for (int e = 0; e < E; ++e) acc[e] += pa[0][e] + pa[1][e];
             // the appended token joins the cache
-            const int a = jn - tok0;
-            if (append && a >= 0 && a < n) {
+            if (append && c.a >= 0) {
+                const int a = c.a;
                 Raw<T, DPL> kr, vr;
                 kr.load_shared(reinterpret_cast<const T*>(kst + a * ROW) + lane * DPL);
                 vr.load_shared(reinterpret_cast<const T*>(vst + a * ROW) + lane * DPL);
@@ -538,11 +577,12 @@ __global__ void __launch_bounds__(256, 1)
                 if (lane == 0) L.pos[row0 + a] = t;
             }
             __syncwarp();  // every lane is done with this stage
-            if (ip < c_end) issue(stage, 0);
-            if (i + 1 < c_end && pre > i + 1) continue;  // head goes on
+            if (ip < c_end) issue(stage);
+            seg_start = c.last || i + 1 == c_end;
+            if (!seg_start) continue;  // the head goes on in this warp
 
-            // end of this warp's segment of head hc: add up the row groups
-            // and the lanes' denominators
+            // end of this warp's segment of head c.head: add up the row
+            // groups and the lanes' denominators
 #pragma unroll
             for (int o = G; o < 32; o <<= 1)
 #pragma unroll
@@ -550,27 +590,28 @@ __global__ void __launch_bounds__(256, 1)
             float l = ls;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(FULL_MASK, l, o);
+            const int hc = c.head;
             const size_t hx = hbase + hc;
             if (!(l > 0.f) || isinf(l)) latch_error(L, HKV_ERR_NUMERIC, (int)hx);
-            const bool whole = seg0 == first && i + 1 == pre;
-            if (whole) {
+            if (seg_whole && c.last) {
                 const float inv = 1.0f / l;
                 float o[E];
 #pragma unroll
                 for (int e = 0; e < E; ++e) o[e] = acc[e] * inv;
                 if (lane < G) store_row<T, E>(o_t + (size_t)hc * D + vc * E, o);
-                if (scoring && lane == 0) L.ml[hx * L.r + col] = make_float2(m, l);
+                if (c.scoring && lane == 0) L.ml[hx * L.r + col] = make_float2(m, l);
             } else {
-                const int w_a = range_owner(first, total, GW);
-                const int w_b = range_owner(pre - 1, total, GW);
-                int segs = 0;
-                for (int w = w_a; w <= w_b; ++w)
-                    segs += range_begin(w, total, GW) < range_begin(w + 1, total, GW);
-                // segments all in this block meet in shared memory, others in
-                // global memory; the last one in merges (no waiting)
+                const int segs = c.segs, w_a = c.wa, w_b = c.wb;
+                // A split head's segments are named by (warp, side): side 1 for
+                // the warp holding the head's first chunk (its segment ends its
+                // range), 0 for the others (theirs start their range); a warp
+                // has at most one segment of each side.  Segments all in this
+                // block meet in shared memory, the others in global memory;
+                // the last one in merges (no waiting).
                 const bool local = w_a / NW == (int)blockIdx.x && w_b / NW == (int)blockIdx.x;
-                float* pp = local ? lpart + (size_t)(warp * 2 + (seg0 == c_begin ? 0 : 1)) * (D + 2)
-                                  : partial + (size_t)seg0 * (D + 2);
+                const int side = gw == w_a ? 1 : 0;
+                float* pp = local ? lpart + (size_t)(warp * 2 + side) * (D + 2)
+                                  : partial + (size_t)(gw * 2 + side) * (D + 2);
                 if (lane == 0) { pp[0] = m; pp[1] = l; }
                 if (lane < G) {
 #pragma unroll
@@ -594,24 +635,25 @@ __global__ void __launch_bounds__(256, 1)
                 __syncwarp();  // lane 0's acquire before every lane's partial loads
                 if (prev == segs - 1) {
                     if (lane == 0 && !local) ticket[hc] = 0;
-                    auto part_of = [&](int w) -> const float* {
-                        const int rb = range_begin(w, total, GW);
-                        if (local)
-                            return lpart + (size_t)((w % NW) * 2 + (max(rb, first) == rb ? 0 : 1)) * (D + 2);
-                        return partial + (size_t)max(rb, first) * (D + 2);
+                    auto slot_of = [&](int w) -> const float* {
+                        const int sd = w == w_a ? 1 : 0;
+                        return local ? lpart + (size_t)((w % NW) * 2 + sd) * (D + 2)
+                                     : partial + (size_t)(w * 2 + sd) * (D + 2);
                     };
                     float M = -INFINITY;
-                    for (int w = w_a + lane; w <= w_b; w += 32)
-                        if (range_begin(w, total, GW) < range_begin(w + 1, total, GW))
-                            M = fmaxf(M, local ? *part_of(w) : __ldcg(part_of(w)));
+                    for (int w = w_a + lane; w <= w_b; w += 32) {
+                        const int2 r = *reinterpret_cast<const int2*>(pw + 2 * w);
+                        if (r.x < r.y) M = fmaxf(M, local ? *slot_of(w) : __ldcg(slot_of(w)));
+                    }
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, o));
                     float Ls = 0.f, o[E];
 #pragma unroll
                     for (int e = 0; e < E; ++e) o[e] = 0.f;
                     for (int w = w_a; w <= w_b; ++w) {
-                        if (range_begin(w, total, GW) >= range_begin(w + 1, total, GW)) continue;
-                        const float* pi = part_of(w);
+                        const int2 r = *reinterpret_cast<const int2*>(pw + 2 * w);
+                        if (r.x >= r.y) continue;
+                        const float* pi = slot_of(w);
                         if (local) {
                             const float wt = exp2f(pi[0] - M);
                             Ls = fmaf(pi[1], wt, Ls);
@@ -628,22 +670,14 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
                     for (int e = 0; e < E; ++e) o[e] *= inv;
                     if (lane < G) store_row<T, E>(o_t + (size_t)hc * D + vc * E, o);
-                    if (scoring && lane == 0) L.ml[hx * L.r + col] = make_float2(M, Ls);
+                    if (c.scoring && lane == 0) L.ml[hx * L.r + col] = make_float2(M, Ls);
                 }
             }
-            // next head holding chunk i + 1
-            seg0 = i + 1;
+            // the next chunk starts a new segment
             m = -INFINITY;
             ls = 0.f;
 #pragma unroll
             for (int e = 0; e < E; ++e) acc[e] = 0.f;
-            if (i + 1 < c_end) {
-                do {
-                    ++hc;
-                    if (hc - cc.base >= 32) cc.load(L, hbase, n_heads, hc);
-                    cc.get(hc, slot, len, jn, scoring, pre, first);
-                } while (pre <= i + 1);
-            }
         }
         if (failed) {
             // copies still in flight into this warp's stages: wait for them
@@ -710,16 +744,20 @@ __global__ void __launch_bounds__(256) append_kernel(Layout L, int layer, const 
 // ---------------------------------------------------------------------------
 
 DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
+    // As many warps as fit (up to DECODE_MAX_WARPS) with two stages each:
+    // the kernel is latency-bound, so warps matter more than prefetch depth
+    // (one chunk in flight per warp covers the HBM latency at the rate a
+    // warp consumes chunks); a third stage only when it costs no warp.
     const int es = L.dtype == HKV_DTYPE_F32 ? 4 : 2;
-    DecodeShape sh{0, 0, 0};
-    for (int ns = MAX_STAGES; ns >= 2 && sh.warps == 0; --ns) {
+    DecodeShape best{0, 0, 0};
+    for (int ns = 2; ns <= MAX_STAGES; ++ns) {
         // the per-warp tail regions are laid out for MAX_STAGES barriers
         const size_t per = decode_warp_bytes(L.d, es, ns) + (MAX_STAGES - ns) * 8;
         int w = (int)((smem_limit - 1024) / per);
-        if (w > 8) w = 8;
-        if (w >= (ns == MAX_STAGES ? 6 : 1)) sh = DecodeShape{w, ns, 1024 + (size_t)w * per};
+        if (w > DECODE_MAX_WARPS) w = DECODE_MAX_WARPS;
+        if (w >= 1 && w >= best.warps) best = DecodeShape{w, ns, 1024 + (size_t)w * per};
     }
-    return sh;
+    return best;
 }
 
 template <typename T, int DPL>
@@ -755,8 +793,7 @@ cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void*
 }
 
 cudaError_t launch_plan(const Layout& L, int l0, int l1, int ahead, cudaStream_t st) {
-    const size_t sm = (size_t)L.S * L.H * sizeof(int32_t);
-    plan_kernel<<<l1 - l0, 1024, sm, st>>>(L, l0, ahead);
+    plan_kernel<<<l1 - l0, 1024, plan_smem_bytes(L.S * L.H), st>>>(L, l0, ahead);
     return cudaGetLastError();
 }
 

@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(512) evict_run_kernel(Layout L, int n_max) {
         // scores: summed softmax weight of the last r queries, each
         // counting only tokens already cached at its step
         bool bad = false;
-#pragma unroll 4
+#pragma unroll 8
         for (int q = lane; q < n; q += 32) {
             const int p = L.pos[slot0 + q];
             const float* lg = L.logit + (slot0 + q) * r;

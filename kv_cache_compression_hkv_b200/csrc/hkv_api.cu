@@ -133,12 +133,10 @@ size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Lay
     l.logit = (float*)take(slots * r * 4);
     l.ml = (float2*)take(nh * r * 8);
     l.rows = (float*)take(S * H * r * Lmax * 4);
-    l.partial = (float*)take(2 * max_chunks * (d + 2) * 4);
+    l.partial = (float*)take(2 * 2 * (size_t)hkv::PLAN_MAX_WARPS * (d + 2) * 4);
     l.due_list = (int32_t*)take(nh * 4);
-    l.plan_pre = (int32_t*)take(nh * 4);
-    l.plan_head = (int4*)take(nh * 16);
-    l.plan_warp = (int32_t*)take(Ly * (hkv::PLAN_MAX_WARPS + 1) * 4);
-    l.plan_whead = (int32_t*)take(Ly * hkv::PLAN_MAX_WARPS * 4);
+    l.plan_desc = (int4*)take(Ly * max_chunks * 16);
+    l.plan_warp = (int4*)take(Ly * hkv::PLAN_MAX_WARPS * 32);
     l.S = c->num_seqs; l.Ly = c->num_layers; l.H = c->num_heads; l.d = c->head_dim;
     l.L = c->max_len; l.W = c->local_window; l.M = c->ste_m; l.D = c->near_dist;
     l.r = c->score_window; l.mode = c->mode; l.stratified = c->stratified; l.dtype = c->dtype;
@@ -218,6 +216,10 @@ hkv_status hkv_create(const hkv_config* cfg, void* pool, size_t bytes, void* str
     }
     int optin = 0;
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, c->device);
+    if (hkv::plan_smem_bytes(cfg->num_seqs * cfg->num_heads) > (size_t)optin - 1024) {
+        delete c;
+        return HKV_ERR_INVALID_ARG;  // too many heads per layer for one plan block
+    }
     c->decode_sh = hkv::decode_shape(c->lay, (size_t)optin - 256);
     c->decode_grid = c->n_sm;  // persistent: one block per SM
     if (c->decode_sh.warps == 0 || c->decode_grid * c->decode_sh.warps > hkv::PLAN_MAX_WARPS) {

@@ -14,7 +14,7 @@ constexpr unsigned FULL_MASK = 0xffffffffu;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr int CHUNK = 32;  // tokens one warp handles per decode work item
 constexpr int PLAN_MAX_WARPS = 4096;  // capacity of a decode plan's warp table
-constexpr int RANK_MAX = 256;         // strata up to this size are selected by ranking
+constexpr int RANK_MAX = 64;          // strata up to this size are selected by ranking
 
 // Everything a kernel needs to find the state of a (layer, sequence, head).
 // The pool is one caller-owned device buffer carved into these regions.
@@ -46,15 +46,15 @@ struct Layout {
     float2* ml;         // [Ly][S][H][r]   (max, sum) of those steps' softmax
     // scratch, reused by every call
     float* rows;        // [S*H][r][prefill_len] weights of the last r prefill queries
-    float* partial;     // [max_chunks][d + 2] split-K partial states
-    int32_t* ticket;    // [S*H] arrivals per head of the running decode launch
+    float* partial;     // [2][PLAN_MAX_WARPS][2][d + 2] split-K partial states
+    int32_t* ticket;    // [2][S*H] arrivals per head of the running decode launch
     int32_t* due_ctl;   // [0] due heads listed, [1] blocks of the eviction done
     int32_t* due_list;  // [Ly*S*H] heads due for eviction this step
     // decode plan per layer, for the step it was made for (see plan_kernel)
-    int32_t* plan_pre;   // [Ly][S*H] inclusive prefix of the heads' chunk counts
-    int4* plan_head;     // [Ly][S*H] {slot (layer-relative), len << 16 | jn, scoring, 0}
-    int32_t* plan_warp;  // [Ly][PLAN_MAX_WARPS + 1] first chunk of each warp's range
-    int32_t* plan_whead; // [Ly][PLAN_MAX_WARPS] head holding that chunk
+    int4* plan_desc;     // [Ly][max_chunks] one descriptor per chunk
+    // [Ly][PLAN_MAX_WARPS][2] {first chunk, end chunk, total, 0} and the
+    // descriptor of the first chunk of each warp's range
+    int4* plan_warp;
     int32_t plan_gw;     // warps of one decode launch
     int32_t max_chunks;
 };
