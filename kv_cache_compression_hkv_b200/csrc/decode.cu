@@ -258,23 +258,26 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
         head_ranges(c0, c1, hz, hw);
         for (int c = c0; c < c1; ++c) dsc[c] = desc(i, c - c0, c1 - c0, hz, hw);
     }
-    int4* pw = L.plan_warp + (size_t)layer * PLAN_MAX_WARPS * 2;
+    constexpr int PB = 1 + PLAN_WARP_DESC;
+    int4* pw = L.plan_warp + (size_t)layer * PLAN_MAX_WARPS * PB;
     for (int w = tid; w < GW; w += blockDim.x) {
         const int cb = range_begin(w, total, GW), ce = range_begin(w + 1, total, GW);
-        int4 first = make_int4(0, 0, 0, 0);
+        pw[PB * w] = make_int4(cb, ce, total, 0);
         if (cb < ce) {
             int lo = 0, hi = n - 1;  // head holding chunk cb
             while (lo < hi) {
                 const int mid = (lo + hi) >> 1;
                 if (cnt[mid] > cb) hi = mid; else lo = mid + 1;
             }
-            const int c0 = lo ? cnt[lo - 1] : 0;
-            int hz, hw;
-            head_ranges(c0, cnt[lo], hz, hw);
-            first = desc(lo, cb - c0, cnt[lo] - c0, hz, hw);
+            // the range's first descriptors, walking the heads
+            int hz = 0, hw = 0, hh = -1;
+            for (int c = cb; c < ce && c < cb + PLAN_WARP_DESC; ++c) {
+                while (cnt[lo] <= c) ++lo;
+                const int c0 = lo ? cnt[lo - 1] : 0;
+                if (hh != lo) { head_ranges(c0, cnt[lo], hz, hw); hh = lo; }
+                pw[PB * w + 1 + (c - cb)] = desc(lo, c - c0, cnt[lo] - c0, hz, hw);
+            }
         }
-        pw[2 * w] = make_int4(cb, ce, total, 0);
-        pw[2 * w + 1] = first;
     }
 }
 
@@ -382,6 +385,11 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
         if (threadIdx.x == 0 && blockIdx.x == 0) latch_error(L, HKV_ERR_STATE, layer);
         return;
     }
+    // this warp's plan block: lane 0 its range, lanes 1.. its first
+    // descriptors (loaded before the block barrier, which hides its latency)
+    constexpr int PB = 1 + PLAN_WARP_DESC;
+    const int4* pw = L.plan_warp + (size_t)layer * PLAN_MAX_WARPS * PB;
+    const int4 blk = lane < PB ? pw[(size_t)gw * PB + lane] : make_int4(0, 0, 0, 0);
     if (lane == 0) {
         for (int s = 0; s < nstage; ++s) ptx::mbar_init(&bars[s], 1);
         ptx::fence_mbar_init();
@@ -389,8 +397,7 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
     if (threadIdx.x < NW) ltick[threadIdx.x] = 0;
     __syncthreads();
 
-    const int4* pw = L.plan_warp + (size_t)layer * PLAN_MAX_WARPS * 2;
-    const int4 wrec = pw[2 * gw], wfirst = pw[2 * gw + 1];
+    const int4 wrec = shfl_int4(blk, 0);
     const int c_begin = wrec.x, c_end = wrec.y;
     const int4* dsc = L.plan_desc + (size_t)layer * L.max_chunks;
 
@@ -426,20 +433,6 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
                 if (q) ptx::bulk_g2s(vd + CHUNK * ROW, q_t + (size_t)c.head * D, ROW, bar);
             }
         };
-        // the range's first chunk straight from the warp's plan record; with
-        // `early` its cached rows go before the wait on the previous launch
-        {
-            const ChunkDesc c0 = ChunkDesc::of(wfirst);
-            if (early) {
-                copy_chunk(0, 1, c0, 1);
-                ptx::grid_dep_wait();
-                ptx::grid_dep_trigger();
-                copy_chunk(0, 2, c0, 1);
-            } else {
-                ptx::grid_dep_trigger();
-                copy_chunk(0, 0, c0, 1);
-            }
-        }
         // descriptors of the range, 32 chunks per window, lane k holding
         // chunk base + k; the producer (ip) and the consumer (i) keep their
         // own window
@@ -447,16 +440,41 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
             return base + lane < c_end ? dsc[base + lane] : make_int4(0, 0, 0, 0);
         };
         int pbase = c_begin, cbase = c_begin;
-        int4 pwin = window(c_begin);
+        // first window: the plan block's copies (lane k < PLAN_WARP_DESC
+        // holds chunk c_begin + k), the rest loaded
+        const int4 head = shfl_int4(blk, min(lane + 1, 31));
+        int4 pwin = head;
+        if (lane >= PLAN_WARP_DESC)
+            pwin = c_begin + lane < c_end ? dsc[c_begin + lane] : make_int4(0, 0, 0, 0);
         int4 cwin = pwin;
-        int ip = c_begin + 1;
+        // the first stages: with `early` their cached rows go before the
+        // wait on the previous launch, the queries and appended rows after it
+        const int npro = min(nstage, c_end - c_begin);
+        if (early) {
+            for (int s = 0; s < npro; ++s) {
+                const ChunkDesc c = ChunkDesc::of(shfl_int4(head, s));
+                copy_chunk(s, 1, c, c.first || s == 0);
+            }
+            ptx::grid_dep_wait();
+            ptx::grid_dep_trigger();
+            for (int s = 0; s < npro; ++s) {
+                const ChunkDesc c = ChunkDesc::of(shfl_int4(head, s));
+                copy_chunk(s, 2, c, c.first || s == 0);
+            }
+        } else {
+            ptx::grid_dep_trigger();
+            for (int s = 0; s < npro; ++s) {
+                const ChunkDesc c = ChunkDesc::of(shfl_int4(head, s));
+                copy_chunk(s, 0, c, c.first || s == 0);
+            }
+        }
+        int ip = c_begin + npro;
         auto issue = [&](int stage) {
             if (ip - pbase >= 32) { pbase += 32; pwin = window(pbase); }
             const ChunkDesc c = ChunkDesc::of(shfl_int4(pwin, ip - pbase));
             copy_chunk(stage, 0, c, c.first || ip == c_begin);
             ++ip;
         };
-        for (int s = 1; s < nstage && ip < c_end; ++s) issue(s);
 
         uint32_t phase = 0;  // bit s: parity of stage s's next phase
         bool failed = false;
@@ -493,25 +511,26 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
             }
             // QK: pass p, lane (vg, vc) takes piece vc of row p * TPI + vg;
             // a butterfly over the G lanes of a group then leaves lane
-            // (vg, vc) the whole dot product of row j = vc * TPI + vg
+            // (vg, vc) the whole dot product of row j = vc * TPI + vg.  All
+            // 32 rows are read (no branches between the loads): a row past n
+            // holds an earlier chunk's data, only ever added into its own
+            // row's sum, which is dropped below.
             float part[NPASS];
 #pragma unroll
             for (int p = 0; p < NPASS; ++p) {
                 const int row = p * TPI + vg;
                 float a0 = 0.f, a1 = 0.f;
-                if (p * TPI < n) {
-                    const uint4 kw = *reinterpret_cast<const uint4*>(kst + row * ROW + vc * 16);
-                    if constexpr (sizeof(T) == 2) {
-                        fma_bf16x2(a0, a1, kw.x, qw.x);
-                        fma_bf16x2(a0, a1, kw.y, qw.y);
-                        fma_bf16x2(a0, a1, kw.z, qw.z);
-                        fma_bf16x2(a0, a1, kw.w, qw.w);
-                    } else {
-                        ffma2(a0, a1, __uint_as_float(qw.x), __uint_as_float(qw.y),
-                              __uint_as_float(kw.x), __uint_as_float(kw.y));
-                        ffma2(a0, a1, __uint_as_float(qw.z), __uint_as_float(qw.w),
-                              __uint_as_float(kw.z), __uint_as_float(kw.w));
-                    }
+                const uint4 kw = *reinterpret_cast<const uint4*>(kst + row * ROW + vc * 16);
+                if constexpr (sizeof(T) == 2) {
+                    fma_bf16x2(a0, a1, kw.x, qw.x);
+                    fma_bf16x2(a0, a1, kw.y, qw.y);
+                    fma_bf16x2(a0, a1, kw.z, qw.z);
+                    fma_bf16x2(a0, a1, kw.w, qw.w);
+                } else {
+                    ffma2(a0, a1, __uint_as_float(qw.x), __uint_as_float(qw.y),
+                          __uint_as_float(kw.x), __uint_as_float(kw.y));
+                    ffma2(a0, a1, __uint_as_float(qw.z), __uint_as_float(qw.w),
+                          __uint_as_float(kw.z), __uint_as_float(kw.w));
                 }
                 part[p] = a0 + a1;
             }
@@ -547,22 +566,28 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
             myp[j] = pj_own;
             __syncwarp();
             // PV: lane (vg, vc) adds p_j times piece vc of rows j = vg (mod TPI)
+            // (rows past n are skipped: their stale V may be anything)
             float pa[2][E];
 #pragma unroll
             for (int u = 0; u < 2; ++u)
 #pragma unroll
                 for (int e = 0; e < E; ++e) pa[u][e] = 0.f;
-#pragma unroll
-            for (int p = 0; p < NPASS; ++p) {
+            auto pv_row = [&](int p) {
                 const int jr = p * TPI + vg;
-                if (p * TPI < n && jr < n) {
-                    const float pj = myp[jr];
-                    float x[E];
-                    unpack16<T>(*reinterpret_cast<const uint4*>(vst + jr * ROW + vc * 16), x);
-                    float* pu = pa[p & 1];
+                const float pj = myp[jr];
+                float x[E];
+                unpack16<T>(*reinterpret_cast<const uint4*>(vst + jr * ROW + vc * 16), x);
+                float* pu = pa[p & 1];
 #pragma unroll
-                    for (int e = 0; e < E; e += 2) ffma2(pu[e], pu[e + 1], pj, pj, x[e], x[e + 1]);
-                }
+                for (int e = 0; e < E; e += 2) ffma2(pu[e], pu[e + 1], pj, pj, x[e], x[e + 1]);
+            };
+            if (n == CHUNK) {
+#pragma unroll
+                for (int p = 0; p < NPASS; ++p) pv_row(p);
+            } else {
+#pragma unroll
+                for (int p = 0; p < NPASS; ++p)
+                    if (p * TPI + vg < n) pv_row(p);
             }
 #pragma unroll
             for (int e = 0; e < E; ++e) acc[e] += pa[0][e] + pa[1][e];
@@ -642,7 +667,7 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
                     };
                     float M = -INFINITY;
                     for (int w = w_a + lane; w <= w_b; w += 32) {
-                        const int2 r = *reinterpret_cast<const int2*>(pw + 2 * w);
+                        const int2 r = *reinterpret_cast<const int2*>(pw + (size_t)PB * w);
                         if (r.x < r.y) M = fmaxf(M, local ? *slot_of(w) : __ldcg(slot_of(w)));
                     }
 #pragma unroll
@@ -651,7 +676,7 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
 #pragma unroll
                     for (int e = 0; e < E; ++e) o[e] = 0.f;
                     for (int w = w_a; w <= w_b; ++w) {
-                        const int2 r = *reinterpret_cast<const int2*>(pw + 2 * w);
+                        const int2 r = *reinterpret_cast<const int2*>(pw + (size_t)PB * w);
                         if (r.x >= r.y) continue;
                         const float* pi = slot_of(w);
                         if (local) {

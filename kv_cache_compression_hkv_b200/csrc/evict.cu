@@ -12,14 +12,20 @@
 
 #include "hkv_internal.cuh"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace hkv {
 
-// Per-warp scratch of the eviction: the select's own scratch, then the
-// head's scores and positions, then the (max, sum) of the scoring steps.
-__host__ __device__ inline size_t evict_warp_bytes(int n_max) {
-    return select_scratch_bytes(n_max) + (size_t)round32(n_max) * 8 + 32 * 8 + 32 * 4;
+// Per-warp scratch of the eviction: the select's own scratch, the head's
+// scores and positions, the (max, sum) of the scoring steps, the step each
+// column holds, an mbarrier, then the K and V rows of the top M slots
+// (`row_bytes` each), prefetched while the head is scored.
+__host__ __device__ inline size_t evict_warp_bytes(int n_max, int m_rows, int row_bytes) {
+    return select_scratch_bytes(n_max) + (size_t)round32(n_max) * 8 + 32 * 8 + 32 * 4 + 16 +
+           2 * (size_t)m_rows * row_bytes;
 }
+
+constexpr uint64_t EVICT_WAIT_NS = 2000000000ull;  // a copy that takes 2 s has failed
 
 // Lists the Global heads of layers [l0, l1) whose cache reached budget + M
 // (one thread per head; one atomic per warp).
@@ -51,20 +57,30 @@ __global__ void __launch_bounds__(512) evict_run_kernel(Layout L, int n_max) {
     extern __shared__ __align__(16) unsigned char esm[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int NW = blockDim.x >> 5;
-    unsigned char* wbase = esm + (size_t)warp * evict_warp_bytes(n_max);
+    const int d = L.d;
+    const int r = L.r;
+    const int row_bytes = d * (int)sizeof(T);
+    const int MR = L.M;  // rows above the budget of a due head
+    unsigned char* wbase = esm + (size_t)warp * evict_warp_bytes(n_max, MR, row_bytes);
     SelectScratch sc = carve_select_scratch(wbase, n_max);
     float* sc_s = reinterpret_cast<float*>(wbase + select_scratch_bytes(n_max));
     int32_t* pos_s = reinterpret_cast<int32_t*>(sc_s + round32(n_max));
     float2* ml_s = reinterpret_cast<float2*>(pos_s + round32(n_max));
     int32_t* step_s = reinterpret_cast<int32_t*>(ml_s + 32);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(step_s + 32);
+    unsigned char* kbuf = reinterpret_cast<unsigned char*>(bar) + 16;
+    unsigned char* vbuf = kbuf + (size_t)MR * row_bytes;
     const int n_heads = L.S * L.H;
-    const int d = L.d;
-    const int r = L.r;
     T* Kp = reinterpret_cast<T*>(L.K);
     T* Vp = reinterpret_cast<T*>(L.V);
-    constexpr int PIECE = 16 / sizeof(T);  // elements per 16-byte piece
-    const int per_row = d / PIECE;
+    const int per_row = row_bytes / 16;  // 16-byte pieces per row
     const int count = L.due_ctl[0];
+    if (lane == 0) {
+        ptx::mbar_init(bar, 1);
+        ptx::fence_mbar_init();
+    }
+    __syncwarp();
+    uint32_t phase = 0;
 
     for (int e = blockIdx.x * NW + warp; e < count; e += gridDim.x * NW) {
         const size_t hx = (size_t)L.due_list[e];
@@ -74,11 +90,18 @@ __global__ void __launch_bounds__(512) evict_run_kernel(Layout L, int n_max) {
         const int t = L.t_next[l] - 1;
         const int n = len_at(L, hx, t);
         const int target = L.budget[hx];
-        if (n > n_max || n != L.cap[hx]) {
+        if (n > n_max || n != L.cap[hx] || n - target > MR || n - target < 0) {
             if (lane == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
             continue;
         }
         const size_t slot0 = region_slot0(L, l, s) + L.off[hx];
+        const int top = n - target;  // the slots a survivor may move from
+        // the K and V rows of slots target .. n-1, while the head is scored
+        if (lane == 0 && top > 0) {
+            ptx::mbar_expect_tx(bar, (uint32_t)(2 * top * row_bytes));
+            ptx::bulk_g2s(kbuf, Kp + (slot0 + target) * d, top * row_bytes, bar);
+            ptx::bulk_g2s(vbuf, Vp + (slot0 + target) * d, top * row_bytes, bar);
+        }
         // (max, 1/sum) of each scoring step, by column = step mod r, and the
         // step each column holds inside the window t-r+1 .. t
         if (lane < r) {
@@ -88,31 +111,44 @@ __global__ void __launch_bounds__(512) evict_run_kernel(Layout L, int n_max) {
         }
         __syncwarp();
         // scores: summed softmax weight of the last r queries, each
-        // counting only tokens already cached at its step
+        // counting only tokens already cached at its step.  Tokens go in
+        // batches of 8 per lane whose loads are all issued before any is used.
         bool bad = false;
-#pragma unroll 8
-        for (int q = lane; q < n; q += 32) {
-            const int p = L.pos[slot0 + q];
-            const float* lg = L.logit + (slot0 + q) * r;
-            float v[32];
-            if (r == 8) {
-                const float4 a = *reinterpret_cast<const float4*>(lg);
-                const float4 b = *reinterpret_cast<const float4*>(lg + 4);
-                v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-                v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-            } else {
+        for (int b0 = 0; b0 < n; b0 += 32 * 8) {
+            int pv[8];
+            float4 la[8], lb[8];
 #pragma unroll
-                for (int c = 0; c < 32; ++c) if (c < r) v[c] = lg[c];
+            for (int u = 0; u < 8; ++u) {
+                const int q = b0 + u * 32 + lane;
+                if (q < n) {
+                    pv[u] = L.pos[slot0 + q];
+                    if (r == 8) {
+                        const float4* lg = reinterpret_cast<const float4*>(L.logit + (slot0 + q) * 8);
+                        la[u] = lg[0];
+                        lb[u] = lg[1];
+                    }
+                }
             }
-            float acc = 0.f;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                if (c >= r) break;
-                if (p <= step_s[c]) acc += exp2f(v[c] - ml_s[c].x) * ml_s[c].y;
+            for (int u = 0; u < 8; ++u) {
+                const int q = b0 + u * 32 + lane;
+                if (q >= n) continue;
+                const int p = pv[u];
+                float acc = 0.f;
+                if (r == 8) {
+                    const float v[8] = {la[u].x, la[u].y, la[u].z, la[u].w, lb[u].x, lb[u].y, lb[u].z, lb[u].w};
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        if (p <= step_s[c]) acc += exp2f(v[c] - ml_s[c].x) * ml_s[c].y;
+                } else {
+                    const float* lg = L.logit + (slot0 + q) * r;
+                    for (int c = 0; c < r; ++c)
+                        if (p <= step_s[c]) acc += exp2f(lg[c] - ml_s[c].x) * ml_s[c].y;
+                }
+                if (isnan(acc)) bad = true;
+                sc_s[q] = acc;
+                pos_s[q] = p;
             }
-            if (isnan(acc)) bad = true;
-            sc_s[q] = acc;
-            pos_s[q] = p;
         }
         __syncwarp();
         auto key_of = [&](int q, uint32_t& sb, int32_t& p) {
@@ -138,38 +174,31 @@ __global__ void __launch_bounds__(512) evict_run_kernel(Layout L, int n_max) {
             nm += __popc(bm);
         }
         __syncwarp();
+        bool ok = true;
+        if (top > 0) {
+            ok = ptx::mbar_wait(bar, phase, EVICT_WAIT_NS);
+            ok = __all_sync(FULL_MASK, ok);
+            phase ^= 1u;
+        }
+        if (!ok) {  // the prefetch never landed: stop before reusing its buffer
+            if (lane == 0) latch_error(L, HKV_ERR_TIMEOUT, (int)hx);
+            break;
+        }
         if (nh != nm) {
             if (lane == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
             continue;
         }
-        // move rows: K and V in 16-byte pieces, eight per lane in flight
-        const int pieces = nh * per_row * 2;
-        for (int w0 = 0; w0 < pieces; w0 += 32 * 8) {
-            uint4 buf[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int w = w0 + u * 32 + lane;
-                if (w < pieces) {
-                    const int mv = w / (per_row * 2);
-                    const int rem = w % (per_row * 2);
-                    const bool isv = rem >= per_row;
-                    const int pc = (isv ? rem - per_row : rem) * PIECE;
-                    const size_t src = (slot0 + sc.moves[sc.n_max - 1 - mv]) * d + pc;
-                    buf[u] = *reinterpret_cast<const uint4*>((isv ? Vp : Kp) + src);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int w = w0 + u * 32 + lane;
-                if (w < pieces) {
-                    const int mv = w / (per_row * 2);
-                    const int rem = w % (per_row * 2);
-                    const bool isv = rem >= per_row;
-                    const int pc = (isv ? rem - per_row : rem) * PIECE;
-                    const size_t dst = (slot0 + sc.moves[mv]) * d + pc;
-                    *reinterpret_cast<uint4*>((isv ? Vp : Kp) + dst) = buf[u];
-                }
-            }
+        // move rows: each survivor's K and V rows from shared memory into a
+        // hole, in 16-byte pieces
+        const int pieces = nh * per_row;
+        for (int w = lane; w < pieces; w += 32) {
+            const int mv = w / per_row, pc = w % per_row;
+            const int src = sc.moves[sc.n_max - 1 - mv] - target;
+            const size_t dst = (slot0 + sc.moves[mv]) * row_bytes + pc * 16;
+            const uint4 kw = *reinterpret_cast<const uint4*>(kbuf + (size_t)src * row_bytes + pc * 16);
+            const uint4 vw = *reinterpret_cast<const uint4*>(vbuf + (size_t)src * row_bytes + pc * 16);
+            *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(Kp) + dst) = kw;
+            *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(Vp) + dst) = vw;
         }
         for (int mv = lane; mv < nh; mv += 32)
             L.pos[slot0 + sc.moves[mv]] = pos_s[sc.moves[sc.n_max - 1 - mv]];
@@ -229,8 +258,7 @@ __global__ void __launch_bounds__(128) select_batch_kernel(
 // launchers
 // ---------------------------------------------------------------------------
 
-static int evict_warps(int n_max) {
-    const size_t per = evict_warp_bytes(n_max);
+static int evict_warps(size_t per) {
     int w = (int)((200 * 1024) / per);
     return w < 1 ? 1 : (w > 16 ? 16 : w);
 }
@@ -241,8 +269,9 @@ cudaError_t launch_evict(const Layout& L, int l0, int l1, int grid, cudaStream_t
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int n_max = L.L;
-    const int nw = evict_warps(n_max);
-    const size_t sm = (size_t)nw * evict_warp_bytes(n_max);
+    const size_t per = evict_warp_bytes(n_max, L.M, L.d * (L.dtype == HKV_DTYPE_F32 ? 4 : 2));
+    const int nw = evict_warps(per);
+    const size_t sm = (size_t)nw * per;
     if (L.dtype == HKV_DTYPE_BF16)
         evict_run_kernel<__nv_bfloat16><<<grid, 32 * nw, sm, st>>>(L, n_max);
     else

@@ -13,8 +13,9 @@ namespace hkv {
 constexpr unsigned FULL_MASK = 0xffffffffu;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr int CHUNK = 32;  // tokens one warp handles per decode work item
-constexpr int PLAN_MAX_WARPS = 4096;  // capacity of a decode plan's warp table
-constexpr int RANK_MAX = 64;          // strata up to this size are selected by ranking
+constexpr int PLAN_MAX_WARPS = 2048;  // capacity of a decode plan's warp table
+constexpr int PLAN_WARP_DESC = 7;     // descriptors copied into each warp's plan block
+constexpr int RANK_MAX = 32;          // strata up to this size are selected by ranking
 
 // Everything a kernel needs to find the state of a (layer, sequence, head).
 // The pool is one caller-owned device buffer carved into these regions.
@@ -52,8 +53,8 @@ struct Layout {
     int32_t* due_list;  // [Ly*S*H] heads due for eviction this step
     // decode plan per layer, for the step it was made for (see plan_kernel)
     int4* plan_desc;     // [Ly][max_chunks] one descriptor per chunk
-    // [Ly][PLAN_MAX_WARPS][2] {first chunk, end chunk, total, 0} and the
-    // descriptor of the first chunk of each warp's range
+    // [Ly][PLAN_MAX_WARPS][1 + PLAN_WARP_DESC]: per warp {first chunk, end
+    // chunk, total, 0} and copies of its range's first descriptors
     int4* plan_warp;
     int32_t plan_gw;     // warps of one decode launch
     int32_t max_chunks;
@@ -136,26 +137,17 @@ template <int DPL> struct RowSlice<__nv_bfloat16, DPL> {
 // keys[i] = (bits(score) << 32) | position, score >= +0 so the bit pattern
 // orders like the value; the total order is (score, position), i.e. equal
 // scores evict the lower position first.  The k-th smallest key of a set is
-// found by a 4-ary search on the score bits (three pivots per round), then,
-// only when scores tie at the boundary, by bisection on their positions.
-// Two independent sets (the near and the far stratum) are searched in the
-// same rounds.  Every key <= the returned threshold is evicted.
+// found by an MSB-first radix select on the score bits (four 8-bit digits,
+// a shared-memory histogram per digit), then, only when scores tie at the
+// boundary, by bisection on their positions.  Every key <= the returned
+// threshold is evicted.
 // ---------------------------------------------------------------------------
 struct KthSearch {
     const uint64_t* keys;
-    int m, k;          // set size, rank wanted (1 <= k < m when active)
-    bool active;
-    uint32_t lo, hi;   // score bits of the k-th smallest lie in [lo, hi]
+    int m, k;          // set size, rank wanted (1 <= k < m)
+    uint32_t lo;       // score bits of the k-th smallest
     uint64_t thr;      // result
 };
-
-__device__ __forceinline__ void kth_round_update(KthSearch& s, uint32_t p1, uint32_t p2, uint32_t p3,
-                                                 unsigned c1, unsigned c2, unsigned c3) {
-    if ((int)c1 >= s.k) s.hi = p1;
-    else if ((int)c2 >= s.k) { s.lo = p1 + 1; s.hi = p2; }
-    else if ((int)c3 >= s.k) { s.lo = p2 + 1; s.hi = p3; }
-    else s.lo = p3 + 1;
-}
 
 // Resolves the position tie at score bits s.lo and sets s.thr.
 __device__ __forceinline__ void kth_finish(KthSearch& s) {
@@ -189,52 +181,58 @@ __device__ __forceinline__ void kth_finish(KthSearch& s) {
     s.thr = ((uint64_t)s_star << 32) | plo;
 }
 
-// Threshold keys of two sets at once.  Inactive sets are skipped.
-__device__ inline void warp_kth_pair(KthSearch& a, KthSearch& b) {
+// Score bits of the k-th smallest key (1 <= k <= m): four passes, each
+// histogramming the next 8-bit digit of the keys that match the digits
+// chosen so far (one shared-memory atomic per distinct digit per 32 keys)
+// and choosing the digit whose cumulative count reaches the wanted rank.
+__device__ inline uint32_t warp_radix_kth_score(const uint64_t* keys, int m, int k, uint32_t* hist) {
     const int lane = threadIdx.x & 31;
-    KthSearch* S[2] = {&a, &b};
+    uint32_t prefix = 0, pmask = 0;
+    int want = k;
+    for (int shift = 24; shift >= 0; shift -= 8) {
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-        KthSearch& s = *S[q];
-        uint32_t lo = 0xffffffffu, hi = 0u;
-        if (s.active)
-            for (int i = lane; i < s.m; i += 32) {
-                const uint32_t sb = (uint32_t)(s.keys[i] >> 32);
-                lo = min(lo, sb);
-                hi = max(hi, sb);
-            }
-        s.lo = __reduce_min_sync(FULL_MASK, lo);
-        s.hi = __reduce_max_sync(FULL_MASK, hi);
-        if (!s.active) s.lo = s.hi = 0;
-    }
-    const int mm = max(a.active ? a.m : 0, b.active ? b.m : 0);
-    while (a.lo < a.hi || b.lo < b.hi) {
-        const uint32_t a1 = a.lo + ((a.hi - a.lo) >> 2), a2 = a.lo + ((a.hi - a.lo) >> 1),
-                       a3 = a.lo + (uint32_t)(((uint64_t)(a.hi - a.lo) * 3) >> 2);
-        const uint32_t b1 = b.lo + ((b.hi - b.lo) >> 2), b2 = b.lo + ((b.hi - b.lo) >> 1),
-                       b3 = b.lo + (uint32_t)(((uint64_t)(b.hi - b.lo) * 3) >> 2);
-        unsigned ca1 = 0, ca2 = 0, ca3 = 0, cb1 = 0, cb2 = 0, cb3 = 0;
-        for (int i = lane; i < mm; i += 32) {
-            if (i < a.m && a.lo < a.hi) {
-                const uint32_t sb = (uint32_t)(a.keys[i] >> 32);
-                ca1 += sb <= a1; ca2 += sb <= a2; ca3 += sb <= a3;
-            }
-            if (i < b.m && b.lo < b.hi) {
-                const uint32_t sb = (uint32_t)(b.keys[i] >> 32);
-                cb1 += sb <= b1; cb2 += sb <= b2; cb3 += sb <= b3;
+        for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0u;
+        __syncwarp();
+        for (int i0 = 0; i0 < m; i0 += 32) {
+            const int i = i0 + lane;
+            const uint32_t sb = i < m ? (uint32_t)(keys[i] >> 32) : 0u;
+            const bool in = i < m && (sb & pmask) == prefix;
+            const uint32_t dg = in ? (sb >> shift) & 255u : 256u;
+            const unsigned same = __match_any_sync(FULL_MASK, dg);
+            if (in && (__ffs(same) - 1) == lane) atomicAdd(&hist[dg], (uint32_t)__popc(same));
+        }
+        __syncwarp();
+        uint32_t c[8], sum = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) { c[j] = hist[lane * 8 + j]; sum += c[j]; }
+        uint32_t incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(FULL_MASK, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const uint32_t excl = incl - sum;
+        const bool mine = excl < (uint32_t)want && (uint32_t)want <= incl;
+        const unsigned bm = __ballot_sync(FULL_MASK, mine);
+        int digit = 0, below = 0;
+        if (mine) {
+            uint32_t run = excl;
+            bool found = false;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (!found && run + c[j] >= (uint32_t)want) { digit = lane * 8 + j; below = (int)run; found = true; }
+                run += c[j];
             }
         }
-        ca1 = __reduce_add_sync(FULL_MASK, ca1);
-        ca2 = __reduce_add_sync(FULL_MASK, ca2);
-        ca3 = __reduce_add_sync(FULL_MASK, ca3);
-        cb1 = __reduce_add_sync(FULL_MASK, cb1);
-        cb2 = __reduce_add_sync(FULL_MASK, cb2);
-        cb3 = __reduce_add_sync(FULL_MASK, cb3);
-        if (a.lo < a.hi) kth_round_update(a, a1, a2, a3, ca1, ca2, ca3);
-        if (b.lo < b.hi) kth_round_update(b, b1, b2, b3, cb1, cb2, cb3);
+        const int src = bm ? __ffs(bm) - 1 : 0;
+        digit = __shfl_sync(FULL_MASK, digit, src);
+        below = __shfl_sync(FULL_MASK, below, src);
+        want -= below;
+        prefix |= (uint32_t)digit << shift;
+        pmask |= 255u << shift;
+        __syncwarp();  // every lane has read the histogram
     }
-    if (a.active) kth_finish(a);
-    if (b.active) kth_finish(b);
+    return prefix;
 }
 
 // Scratch of one warp's stratified select over up to n_max tokens.  The
@@ -242,6 +240,7 @@ __device__ inline void warp_kth_pair(KthSearch& a, KthSearch& b) {
 // same for slot[] and for the hole / mover lists of the compaction.
 struct SelectScratch {
     uint64_t* keys;        // [n_max]
+    uint32_t* hist;        // [256] digit histogram of the radix select
     uint16_t* slot;        // [n_max]
     uint32_t* evict_bits;  // [n_max / 32]
     uint16_t* moves;       // [n_max]: holes from the front, movers from the back
@@ -252,14 +251,15 @@ __host__ __device__ inline int round32(int n) { return (n + 31) / 32 * 32; }
 
 __host__ __device__ inline size_t select_scratch_bytes(int n_max) {
     size_t n = (size_t)round32(n_max);
-    return (n * 8 + n * 2 + (n / 32) * 4 + n * 2 + 15) / 16 * 16;  // 16-byte multiple
+    return (n * 8 + 1024 + n * 2 + (n / 32) * 4 + n * 2 + 15) / 16 * 16;  // 16-byte multiple
 }
 
 __device__ inline SelectScratch carve_select_scratch(unsigned char* base, int n_max) {
     const int n = round32(n_max);
     SelectScratch s;
     s.keys = reinterpret_cast<uint64_t*>(base);
-    s.slot = reinterpret_cast<uint16_t*>(s.keys + n);
+    s.hist = reinterpret_cast<uint32_t*>(s.keys + n);
+    s.slot = reinterpret_cast<uint16_t*>(s.hist + 256);
     s.evict_bits = reinterpret_cast<uint32_t*>(s.slot + n);
     s.moves = reinterpret_cast<uint16_t*>(s.evict_bits + n / 32);
     s.n_max = n;
@@ -318,23 +318,23 @@ __device__ int warp_stratified_select(const SelectScratch& sc, int n, int t, int
         kn = 0;
         if (kf > nf) kf = nf;
     }
-    // Small strata: rank every key against all keys of its stratum (keys are
-    // distinct, so rank < k is exactly the k lowest).  Large strata: thresholds
-    // by the 4-ary search; none evicted (k <= 0), all evicted (k >= m).
-    const bool rank_n = kn > 0 && kn < nn && nn <= RANK_MAX;
-    const bool rank_f = kf > 0 && kf < nf && nf <= RANK_MAX;
-    KthSearch a{sc.keys, nn, kn, kn > 0 && kn < nn && !rank_n, 0, 0, kn >= nn && kn > 0 ? ~0ull : 0ull};
-    KthSearch b{sc.keys + (n - nf), nf, kf, kf > 0 && kf < nf && !rank_f, 0, 0,
-                kf >= nf && kf > 0 ? ~0ull : 0ull};
-    if (a.active || b.active) warp_kth_pair(a, b);
+    // Strata of at most RANK_MAX keys: rank every key against all keys of
+    // its stratum (keys are distinct, so rank < k is exactly the k lowest).
+    // Larger strata: threshold by the radix select; none evicted (k <= 0),
+    // all evicted (k >= m).
     for (int which = 0; which < 2; ++which) {
         const int k = which == 0 ? kn : kf;
         const int m = which == 0 ? nn : nf;
-        const uint64_t* keys = which == 0 ? a.keys : b.keys;
+        const uint64_t* keys = which == 0 ? sc.keys : sc.keys + (n - nf);
         const uint16_t* slots = which == 0 ? sc.slot : sc.slot + (n - nf);
-        const uint64_t thr = which == 0 ? a.thr : b.thr;
-        const bool by_rank = which == 0 ? rank_n : rank_f;
         if (k <= 0) continue;
+        const bool by_rank = k < m && m <= RANK_MAX;
+        uint64_t thr = ~0ull;
+        if (k < m && !by_rank) {
+            KthSearch q{keys, m, k, warp_radix_kth_score(keys, m, k, sc.hist), 0};
+            kth_finish(q);
+            thr = q.thr;
+        }
         if (by_rank) {
             for (int i0 = 0; i0 < m; i0 += 32) {
                 const int i = i0 + lane;
