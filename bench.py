@@ -317,6 +317,7 @@ def gpu_arm(args, rank, world, dev):
     achieved = float(alg.sum() / (dec_us.sum() * 1e-6) / 1e9)
     del g_prof
 
+    traffic_ratio = decode_traffic_ratio()
     peaks = {}
     pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(pk):
@@ -331,7 +332,9 @@ def gpu_arm(args, rank, world, dev):
         "tokens_per_s": w.images * steps / (ms * 1e-3) * world,
         "clocks": clk.summary(),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": (None if traffic_ratio is None
+                                 else round(traffic_ratio * float(alg.mean()))),
                      "kernel": "decode_kernel (fused append + split-K decode attention)",
                      "peak_source": peak_src,
                      "bytes_per_launch_avg": float(alg.mean()),
@@ -443,7 +446,9 @@ def e2e_arm(args, w, cache, inp, dev, world):
 
 def profile_run(args, w):
     """Eager prefill + decode steps of a reduced copy of the workload: the
-    command ncu captures single launches of (nothing is timed here)."""
+    command ncu captures single launches of (nothing is timed here).  Prints
+    the algorithmic bytes of every decode launch, in launch order, so that
+    the DRAM bytes of a captured launch can be compared with them."""
     import kv_cache_compression_hkv_b200 as hkv
     dev = torch.device("cuda", 0)
     w = w.scaled(num_seqs=args.seqs or w.num_seqs, num_layers=args.layers or w.num_layers)
@@ -451,19 +456,43 @@ def profile_run(args, w):
     outs = [torch.empty(w.num_seqs, w.num_heads, w.head_dim, dtype=w.torch_dtype, device=dev)
             for _ in range(w.num_layers)]
     cache = hkv.HeadKVCache(hkv.config_for(w), device=dev)
+    es = 2 if w.dtype == "bf16" else 4
     for l in range(w.num_layers):
         cache.prefill_classify(l, *inp.pre[l])
+    alg = []
     for t in range(min(args.profile_steps, w.decode_steps)):
         for l in range(w.num_layers):
             q, k, v = inp.dec[l]
             cache.decode_step(l, q[t], k[t], v[t], outs[l])
+            ln, _ = cache.lens(l)
+            alg.append(int(ln.sum()) * 2 * w.head_dim * es + w.num_seqs * w.num_heads * w.head_dim * es * 4)
         cache.ste_evict()
     torch.cuda.synchronize()
     rc, detail = cache.check()
     print(json.dumps({"profile_run": w.name, "seqs": w.num_seqs, "layers": w.num_layers,
-                      "steps": min(args.profile_steps, w.decode_steps), "status": rc}))
+                      "steps": min(args.profile_steps, w.decode_steps), "status": rc,
+                      "decode_alg_bytes": alg}))
     if rc != 0:
         raise SystemExit(f"device status {rc} ({detail})")
+
+
+def decode_traffic_ratio():
+    """DRAM bytes per algorithmic byte of decode_kernel from the committed ncu
+    summary, if it was taken on the decode source as it is now (else None)."""
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", "decode_kernel_llamagen_xl.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    m_rat = re.search(r"dram_per_algorithmic_byte:\s*([0-9.]+)", text)
+    if not (m_sha and m_rat):
+        return None
+    src = os.path.join(ROOT, "kv_cache_compression_hkv_b200", "csrc", "decode.cu")
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != m_sha.group(1):
+        return None
+    return float(m_rat.group(1))
 
 
 def main():

@@ -120,18 +120,6 @@ __device__ __forceinline__ void store_row(T* p, const float (&x)[DPL]) {
     }
 }
 
-// First chunk of warp w's range when `total` chunks go to `gw` warps
-// (32-bit arithmetic while the products fit).
-__device__ __forceinline__ int range_begin(int w, int total, int gw) {
-    if (total < (1 << 19)) return (int)((uint32_t)w * (uint32_t)total / (uint32_t)gw);
-    return (int)((int64_t)w * total / gw);
-}
-// Warp whose range holds chunk c.
-__device__ __forceinline__ int range_owner(int c, int total, int gw) {
-    if (total < (1 << 19)) return (int)(((uint32_t)(c + 1) * (uint32_t)gw - 1u) / (uint32_t)total);
-    return (int)(((int64_t)(c + 1) * gw - 1) / total);
-}
-
 // ---------------------------------------------------------------------------
 // Chunk descriptors.  The plan describes every chunk of a layer in one int4:
 //   x: layer-relative row of the chunk's first token
@@ -180,6 +168,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
     int32_t* hslot = psm + n;      // layer-relative row of the head's first token
     int32_t* hlen = psm + 2 * n;   // len << 16 | appended slot
     int32_t* hscore = psm + 3 * n; // scoring flag
+    int32_t* wbeg = psm + 4 * n;   // first chunk of each warp's range, [GW + 1]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, NW = blockDim.x >> 5;
     const int t = L.t_next[layer] - 1 + ahead;
     if (t >= L.L) return;  // the sequence is complete: no step left to plan
@@ -243,42 +232,65 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
                       ((k == c1mc0 - 1) << 13) | (hscore[i] << 14) | hz;
         return make_int4(hslot[i] + tok0, i, z, hw);
     };
+    // Warp ranges of equal cost: a chunk costs CHUNK_COST units and a head
+    // one more (its end: reductions, output, a merge when split), so that
+    // warps holding many short heads get fewer chunks.  Head i's cost ends
+    // at CHUNK_COST * cnt[i] + i + 1; warp w's range starts at the first
+    // chunk whose cost starts at or after w * cost / GW.
+    constexpr int CHUNK_COST = 3;
+    const int64_t tcost = (int64_t)CHUNK_COST * total + n;
+    for (int w = tid; w <= GW; w += blockDim.x) {
+        const int64_t b = (int64_t)w * tcost / GW;
+        int lo = 0, hi = n;  // first head whose cost ends after b
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if ((int64_t)CHUNK_COST * cnt[mid] + mid + 1 > b) hi = mid; else lo = mid + 1;
+        }
+        int c = total;
+        if (lo < n) {
+            const int c0 = lo ? cnt[lo - 1] : 0;
+            const int64_t base = lo ? (int64_t)CHUNK_COST * c0 + lo : 0;
+            const int k = (int)((b - base + CHUNK_COST - 1) / CHUNK_COST);
+            c = c0 + min(max(k, 0), cnt[lo] - c0);
+        }
+        wbeg[w] = w == GW ? total : c;
+    }
+    __syncthreads();
+    // the warp whose range holds chunk c (the last w with wbeg[w] <= c)
+    auto owner = [&](int c) -> int {
+        int lo = 0, hi = GW - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (wbeg[mid] <= c) lo = mid; else hi = mid - 1;
+        }
+        return lo;
+    };
     auto head_ranges = [&](int c0, int c1, int& hz, int& hw) {
-        const int wa = range_owner(c0, total, GW), wb = range_owner(c1 - 1, total, GW);
+        const int wa = owner(c0), wb = owner(c1 - 1);
         int segs = 0;
-        for (int w = wa; w <= wb; ++w) segs += range_begin(w, total, GW) < range_begin(w + 1, total, GW);
+        for (int w = wa; w <= wb; ++w) segs += wbeg[w] < wbeg[w + 1];
         hz = segs << 16;
         hw = wa | ((wb - wa) << 12);
     };
+    // every chunk's descriptor, and a copy of the first PLAN_WARP_DESC
+    // descriptors of each warp's range in that warp's plan block
+    constexpr int PB = 1 + PLAN_WARP_DESC;
     int4* dsc = L.plan_desc + (size_t)layer * L.max_chunks;
+    int4* pw = L.plan_warp + (size_t)layer * PLAN_MAX_WARPS * PB;
     for (int i = tid; i < n; i += blockDim.x) {
         const int c1 = cnt[i], c0 = i ? cnt[i - 1] : 0;
         if (c1 == c0) continue;
         int hz, hw;
         head_ranges(c0, c1, hz, hw);
-        for (int c = c0; c < c1; ++c) dsc[c] = desc(i, c - c0, c1 - c0, hz, hw);
-    }
-    constexpr int PB = 1 + PLAN_WARP_DESC;
-    int4* pw = L.plan_warp + (size_t)layer * PLAN_MAX_WARPS * PB;
-    for (int w = tid; w < GW; w += blockDim.x) {
-        const int cb = range_begin(w, total, GW), ce = range_begin(w + 1, total, GW);
-        pw[PB * w] = make_int4(cb, ce, total, 0);
-        if (cb < ce) {
-            int lo = 0, hi = n - 1;  // head holding chunk cb
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if (cnt[mid] > cb) hi = mid; else lo = mid + 1;
-            }
-            // the range's first descriptors, walking the heads
-            int hz = 0, hw = 0, hh = -1;
-            for (int c = cb; c < ce && c < cb + PLAN_WARP_DESC; ++c) {
-                while (cnt[lo] <= c) ++lo;
-                const int c0 = lo ? cnt[lo - 1] : 0;
-                if (hh != lo) { head_ranges(c0, cnt[lo], hz, hw); hh = lo; }
-                pw[PB * w + 1 + (c - cb)] = desc(lo, c - c0, cnt[lo] - c0, hz, hw);
-            }
+        int w = hw & 0xfff;  // the warp holding chunk c
+        for (int c = c0; c < c1; ++c) {
+            while (wbeg[w + 1] <= c) ++w;
+            const int4 d = desc(i, c - c0, c1 - c0, hz, hw);
+            dsc[c] = d;
+            if (c - wbeg[w] < PLAN_WARP_DESC) pw[PB * w + 1 + (c - wbeg[w])] = d;
         }
     }
+    for (int w = tid; w < GW; w += blockDim.x) pw[PB * w] = make_int4(wbeg[w], wbeg[w + 1], total, 0);
 }
 
 // d = a * b + d on two fp32 lanes at once (packed FMA; each lane rounds as a
@@ -665,30 +677,52 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
                         return local ? lpart + (size_t)((w % NW) * 2 + sd) * (D + 2)
                                      : partial + (size_t)(w * 2 + sd) * (D + 2);
                     };
-                    float M = -INFINITY;
-                    for (int w = w_a + lane; w <= w_b; w += 32) {
-                        const int2 r = *reinterpret_cast<const int2*>(pw + (size_t)PB * w);
-                        if (r.x < r.y) M = fmaxf(M, local ? *slot_of(w) : __ldcg(slot_of(w)));
-                    }
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, o));
-                    float Ls = 0.f, o[E];
+                    // online merge of the segments, four at a time with all
+                    // their loads issued first; warp ranges between w_a and
+                    // w_b are all non-empty unless segs says otherwise
+                    const bool dense = segs == w_b - w_a + 1;
+                    float M = -INFINITY, Ls = 0.f, o[E];
 #pragma unroll
                     for (int e = 0; e < E; ++e) o[e] = 0.f;
-                    for (int w = w_a; w <= w_b; ++w) {
-                        const int2 r = *reinterpret_cast<const int2*>(pw + (size_t)PB * w);
-                        if (r.x >= r.y) continue;
-                        const float* pi = slot_of(w);
-                        if (local) {
-                            const float wt = exp2f(pi[0] - M);
-                            Ls = fmaf(pi[1], wt, Ls);
+                    for (int w0 = w_a; w0 <= w_b; w0 += 4) {
+                        float pm[4], pl[4], px[4][E];
+                        bool ok[4];
 #pragma unroll
-                            for (int e = 0; e < E; ++e) o[e] = fmaf(pi[2 + vc * E + e], wt, o[e]);
-                        } else {
-                            const float wt = exp2f(__ldcg(pi) - M);
-                            Ls = fmaf(__ldcg(pi + 1), wt, Ls);
+                        for (int u = 0; u < 4; ++u) {
+                            const int w = w0 + u;
+                            ok[u] = w <= w_b;
+                            if (ok[u] && !dense) {
+                                const int2 r = *reinterpret_cast<const int2*>(pw + (size_t)PB * w);
+                                ok[u] = r.x < r.y;
+                            }
+                            pm[u] = -INFINITY;
+                            pl[u] = 0.f;
 #pragma unroll
-                            for (int e = 0; e < E; ++e) o[e] = fmaf(__ldcg(pi + 2 + vc * E + e), wt, o[e]);
+                            for (int e = 0; e < E; ++e) px[u][e] = 0.f;
+                            if (ok[u]) {
+                                const float* pi = slot_of(w);
+                                if (local) {
+                                    pm[u] = pi[0];
+                                    pl[u] = pi[1];
+#pragma unroll
+                                    for (int e = 0; e < E; ++e) px[u][e] = pi[2 + vc * E + e];
+                                } else {
+                                    pm[u] = __ldcg(pi);
+                                    pl[u] = __ldcg(pi + 1);
+#pragma unroll
+                                    for (int e = 0; e < E; ++e) px[u][e] = __ldcg(pi + 2 + vc * E + e);
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            if (!ok[u]) continue;
+                            const float mn = fmaxf(M, pm[u]);
+                            const float fa = exp2f(M - mn), fb = exp2f(pm[u] - mn);
+                            Ls = Ls * fa + pl[u] * fb;
+#pragma unroll
+                            for (int e = 0; e < E; ++e) o[e] = o[e] * fa + px[u][e] * fb;
+                            M = mn;
                         }
                     }
                     const float inv = 1.0f / Ls;
@@ -774,13 +808,13 @@ DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
     // (one chunk in flight per warp covers the HBM latency at the rate a
     // warp consumes chunks); a third stage only when it costs no warp.
     const int es = L.dtype == HKV_DTYPE_F32 ? 4 : 2;
-    DecodeShape best{0, 0, 0};
+    DecodeShape best{0, 0, 0, 1};
     for (int ns = 2; ns <= MAX_STAGES; ++ns) {
         // the per-warp tail regions are laid out for MAX_STAGES barriers
         const size_t per = decode_warp_bytes(L.d, es, ns) + (MAX_STAGES - ns) * 8;
         int w = (int)((smem_limit - 1024) / per);
         if (w > DECODE_MAX_WARPS) w = DECODE_MAX_WARPS;
-        if (w >= 1 && w >= best.warps) best = DecodeShape{w, ns, 1024 + (size_t)w * per};
+        if (w >= 1 && w >= best.warps) best = DecodeShape{w, ns, 1024 + (size_t)w * per, 1};
     }
     return best;
 }

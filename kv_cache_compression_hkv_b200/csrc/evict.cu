@@ -52,8 +52,10 @@ __global__ void __launch_bounds__(256) evict_scan_kernel(Layout L, int l0, int l
 
 // Evicts every listed head, one warp per head: scores from the stored
 // logits, stratified select, compaction.  The last block clears the list.
+constexpr int EVICT_MAX_WARPS = 12;
+
 template <typename T>
-__global__ void __launch_bounds__(512) evict_run_kernel(Layout L, int n_max) {
+__global__ void __launch_bounds__(EVICT_MAX_WARPS * 32) evict_run_kernel(Layout L, int n_max) {
     extern __shared__ __align__(16) unsigned char esm[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int NW = blockDim.x >> 5;
@@ -260,7 +262,7 @@ __global__ void __launch_bounds__(128) select_batch_kernel(
 
 static int evict_warps(size_t per) {
     int w = (int)((200 * 1024) / per);
-    return w < 1 ? 1 : (w > 16 ? 16 : w);
+    return w < 1 ? 1 : (w > EVICT_MAX_WARPS ? EVICT_MAX_WARPS : w);
 }
 
 cudaError_t launch_evict(const Layout& L, int l0, int l1, int grid, cudaStream_t st) {

@@ -221,7 +221,7 @@ hkv_status hkv_create(const hkv_config* cfg, void* pool, size_t bytes, void* str
         return HKV_ERR_INVALID_ARG;  // too many heads per layer for one plan block
     }
     c->decode_sh = hkv::decode_shape(c->lay, (size_t)optin - 256);
-    c->decode_grid = c->n_sm;  // persistent: one block per SM
+    c->decode_grid = c->n_sm * c->decode_sh.per_sm;  // persistent: every block resident
     if (c->decode_sh.warps == 0 || c->decode_grid * c->decode_sh.warps > hkv::PLAN_MAX_WARPS) {
         delete c;
         return HKV_ERR_INVALID_ARG;

@@ -15,7 +15,7 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr int CHUNK = 32;  // tokens one warp handles per decode work item
 constexpr int PLAN_MAX_WARPS = 2048;  // capacity of a decode plan's warp table
 constexpr int PLAN_WARP_DESC = 7;     // descriptors copied into each warp's plan block
-constexpr int RANK_MAX = 32;          // strata up to this size are selected by ranking
+constexpr int RANK_MAX = 256;         // strata up to this size are selected by ranking
 
 // Everything a kernel needs to find the state of a (layer, sequence, head).
 // The pool is one caller-owned device buffer carved into these regions.
@@ -235,6 +235,33 @@ __device__ inline uint32_t warp_radix_kth_score(const uint64_t* keys, int m, int
     return prefix;
 }
 
+// Marks the k lowest of m <= 32 * U distinct keys: lane l ranks keys
+// l, l + 32, ... (held in registers) against every key in one pass of
+// shared-memory broadcast reads; rank < k is exactly the k lowest.
+template <int U>
+__device__ inline void warp_rank_evict(const uint64_t* keys, const uint16_t* slots, int m, int k,
+                                       uint32_t* evict_bits) {
+    const int lane = threadIdx.x & 31;
+    uint64_t mine[U];
+    int rk[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int i = lane + 32 * u;
+        mine[u] = i < m ? keys[i] : ~0ull;
+        rk[u] = 0;
+    }
+    for (int j = 0; j < m; ++j) {
+        const uint64_t kj = keys[j];
+#pragma unroll
+        for (int u = 0; u < U; ++u) rk[u] += kj < mine[u];
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int i = lane + 32 * u;
+        if (i < m && rk[u] < k) atomicOr(&evict_bits[slots[i] >> 5], 1u << (slots[i] & 31));
+    }
+}
+
 // Scratch of one warp's stratified select over up to n_max tokens.  The
 // near keys fill keys[] from the front and the far keys from the back; the
 // same for slot[] and for the hole / mover lists of the compaction.
@@ -336,13 +363,9 @@ __device__ int warp_stratified_select(const SelectScratch& sc, int n, int t, int
             thr = q.thr;
         }
         if (by_rank) {
-            for (int i0 = 0; i0 < m; i0 += 32) {
-                const int i = i0 + lane;
-                const uint64_t ki = i < m ? keys[i] : ~0ull;
-                int rank = 0;
-                for (int j = 0; j < m; ++j) rank += keys[j] < ki;  // broadcast reads
-                if (i < m && rank < k) atomicOr(&sc.evict_bits[slots[i] >> 5], 1u << (slots[i] & 31));
-            }
+            if (m <= 64) warp_rank_evict<2>(keys, slots, m, k, sc.evict_bits);
+            else if (m <= 128) warp_rank_evict<4>(keys, slots, m, k, sc.evict_bits);
+            else warp_rank_evict<8>(keys, slots, m, k, sc.evict_bits);
         } else {
             for (int i = lane; i < m; i += 32)
                 if (keys[i] <= thr) atomicOr(&sc.evict_bits[slots[i] >> 5], 1u << (slots[i] & 31));
