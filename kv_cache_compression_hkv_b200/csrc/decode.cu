@@ -30,6 +30,9 @@ constexpr float RESCALE = 8.f;
 constexpr int MAX_STAGES = 3;
 // Most warps of one decode block (one block per SM).
 constexpr int DECODE_MAX_WARPS = 12;
+// Cost of a chunk, in units of the cost of a head's end, in the plan's
+// balancing of the warp ranges.
+constexpr int CHUNK_COST = 3;
 
 // Packed storage of DPL consecutive elements of one row.
 template <typename T, int DPL> struct Raw;
@@ -168,7 +171,6 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
     int32_t* hslot = psm + n;      // layer-relative row of the head's first token
     int32_t* hlen = psm + 2 * n;   // len << 16 | appended slot
     int32_t* hscore = psm + 3 * n; // scoring flag
-    int32_t* wbeg = psm + 4 * n;   // first chunk of each warp's range, [GW + 1]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, NW = blockDim.x >> 5;
     const int t = L.t_next[layer] - 1 + ahead;
     if (t >= L.L) return;  // the sequence is complete: no step left to plan
@@ -221,30 +223,28 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
         if (tid == 0) latch_error(L, HKV_ERR_STATE, layer);
         return;
     }
-    // descriptor of the k-th chunk of head i (chunks c0 .. c1-1), given the
-    // head's warp-range fields hz (segments << 16) and hw
-    auto desc = [&](int i, int k, int c1mc0, int hz, int hw) -> int4 {
-        const int len = hlen[i] >> 16, jn = (int)(int16_t)(hlen[i] & 0xffff);
-        const int tok0 = k * CHUNK;
-        const int nr = min(CHUNK, len - tok0);
-        const int a = jn - tok0;
-        const int z = nr | ((a >= 0 && a < nr ? a + 1 : 0) << 6) | ((k == 0) << 12) |
-                      ((k == c1mc0 - 1) << 13) | (hscore[i] << 14) | hz;
-        return make_int4(hslot[i] + tok0, i, z, hw);
-    };
     // Warp ranges of equal cost: a chunk costs CHUNK_COST units and a head
     // one more (its end: reductions, output, a merge when split), so that
     // warps holding many short heads get fewer chunks.  Head i's cost ends
     // at CHUNK_COST * cnt[i] + i + 1; warp w's range starts at the first
     // chunk whose cost starts at or after w * cost / GW.
-    constexpr int CHUNK_COST = 3;
     const int64_t tcost = (int64_t)CHUNK_COST * total + n;
+    const bool narrow = tcost * GW < ((int64_t)1 << 31);  // 32-bit arithmetic suffices
+    int32_t* gw_beg = L.plan_wbeg + (size_t)layer * (PLAN_MAX_WARPS + 1);
     for (int w = tid; w <= GW; w += blockDim.x) {
-        const int64_t b = (int64_t)w * tcost / GW;
+        const int64_t b = narrow ? (int64_t)((uint32_t)w * (uint32_t)tcost / (uint32_t)GW)
+                                 : (int64_t)w * tcost / GW;
         int lo = 0, hi = n;  // first head whose cost ends after b
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if ((int64_t)CHUNK_COST * cnt[mid] + mid + 1 > b) hi = mid; else lo = mid + 1;
+        if (narrow) {
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (CHUNK_COST * cnt[mid] + mid + 1 > (int)b) hi = mid; else lo = mid + 1;
+            }
+        } else {
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if ((int64_t)CHUNK_COST * cnt[mid] + mid + 1 > b) hi = mid; else lo = mid + 1;
+            }
         }
         int c = total;
         if (lo < n) {
@@ -253,9 +253,38 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
             const int k = (int)((b - base + CHUNK_COST - 1) / CHUNK_COST);
             c = c0 + min(max(k, 0), cnt[lo] - c0);
         }
-        wbeg[w] = w == GW ? total : c;
+        gw_beg[w] = w == GW ? total : c;
     }
+    // the head facts and chunk prefix for the descriptor kernel
+    int32_t* gcnt = L.plan_cnt + hbase;
+    int4* gfact = L.plan_hfact + hbase;
+    for (int i = tid; i < n; i += blockDim.x) {
+        gcnt[i] = cnt[i];
+        gfact[i] = make_int4(hslot[i], hlen[i], hscore[i], 0);
+    }
+}
+
+// Second half of the plan: every chunk's descriptor, each warp's record
+// and a copy of the first PLAN_WARP_DESC descriptors of its range in its
+// plan block.  Blocks (layer, part): part p takes the p-th slice of the
+// layer's heads and of its warps.
+__global__ void __launch_bounds__(1024) plan_desc_kernel(Layout L, int l0, int ahead) {
+    extern __shared__ int32_t dsm32[];
+    const int layer = l0 + blockIdx.x;
+    const int n = L.S * L.H;
+    const int GW = L.plan_gw;
+    const int t = L.t_next[layer] - 1 + ahead;
+    if (t >= L.L) return;
+    const size_t hbase = (size_t)layer * n;
+    int32_t* cnt = dsm32;            // inclusive prefix of the chunk counts
+    int32_t* wbeg = dsm32 + n;       // [GW + 1]
+    const int32_t* gcnt = L.plan_cnt + hbase;
+    const int32_t* gw_beg = L.plan_wbeg + (size_t)layer * (PLAN_MAX_WARPS + 1);
+    for (int i = threadIdx.x; i < n; i += blockDim.x) cnt[i] = gcnt[i];
+    for (int w = threadIdx.x; w <= GW; w += blockDim.x) wbeg[w] = gw_beg[w];
     __syncthreads();
+    const int total = cnt[n - 1];
+    if (total > L.max_chunks) return;  // the first half latched the error
     // the warp whose range holds chunk c (the last w with wbeg[w] <= c)
     auto owner = [&](int c) -> int {
         int lo = 0, hi = GW - 1;
@@ -265,32 +294,37 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
         }
         return lo;
     };
-    auto head_ranges = [&](int c0, int c1, int& hz, int& hw) {
-        const int wa = owner(c0), wb = owner(c1 - 1);
-        int segs = 0;
-        for (int w = wa; w <= wb; ++w) segs += wbeg[w] < wbeg[w + 1];
-        hz = segs << 16;
-        hw = wa | ((wb - wa) << 12);
-    };
-    // every chunk's descriptor, and a copy of the first PLAN_WARP_DESC
-    // descriptors of each warp's range in that warp's plan block
     constexpr int PB = 1 + PLAN_WARP_DESC;
     int4* dsc = L.plan_desc + (size_t)layer * L.max_chunks;
     int4* pw = L.plan_warp + (size_t)layer * PLAN_MAX_WARPS * PB;
-    for (int i = tid; i < n; i += blockDim.x) {
+    const int parts = gridDim.y, part = blockIdx.y;
+    const int h0 = (int)((int64_t)part * n / parts), h1 = (int)((int64_t)(part + 1) * n / parts);
+    for (int i = h0 + threadIdx.x; i < h1; i += blockDim.x) {
         const int c1 = cnt[i], c0 = i ? cnt[i - 1] : 0;
         if (c1 == c0) continue;
-        int hz, hw;
-        head_ranges(c0, c1, hz, hw);
-        int w = hw & 0xfff;  // the warp holding chunk c
+        const int4 f = L.plan_hfact[hbase + i];
+        const int wa = owner(c0), wb = owner(c1 - 1);
+        int segs = 0;
+        for (int w = wa; w <= wb; ++w) segs += wbeg[w] < wbeg[w + 1];
+        const int hw = wa | ((wb - wa) << 12);
+        const int len = f.y >> 16, jn = (int)(int16_t)(f.y & 0xffff);
+        int w = wa;  // the warp holding chunk c
         for (int c = c0; c < c1; ++c) {
             while (wbeg[w + 1] <= c) ++w;
-            const int4 d = desc(i, c - c0, c1 - c0, hz, hw);
+            const int k = c - c0;
+            const int tok0 = k * CHUNK;
+            const int nr = min(CHUNK, len - tok0);
+            const int a = jn - tok0;
+            const int z = nr | ((a >= 0 && a < nr ? a + 1 : 0) << 6) | ((k == 0) << 12) |
+                          ((c == c1 - 1) << 13) | (f.z << 14) | (segs << 16);
+            const int4 d = make_int4(f.x + tok0, i, z, hw);
             dsc[c] = d;
             if (c - wbeg[w] < PLAN_WARP_DESC) pw[PB * w + 1 + (c - wbeg[w])] = d;
         }
     }
-    for (int w = tid; w < GW; w += blockDim.x) pw[PB * w] = make_int4(wbeg[w], wbeg[w + 1], total, 0);
+    const int w0 = (int)((int64_t)part * GW / parts), w1 = (int)((int64_t)(part + 1) * GW / parts);
+    for (int w = w0 + threadIdx.x; w < w1; w += blockDim.x)
+        pw[PB * w] = make_int4(wbeg[w], wbeg[w + 1], total, 0);
 }
 
 // d = a * b + d on two fp32 lanes at once (packed FMA; each lane rounds as a
@@ -853,6 +887,10 @@ cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void*
 
 cudaError_t launch_plan(const Layout& L, int l0, int l1, int ahead, cudaStream_t st) {
     plan_kernel<<<l1 - l0, 1024, plan_smem_bytes(L.S * L.H), st>>>(L, l0, ahead);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t sm = ((size_t)L.S * L.H + PLAN_MAX_WARPS + 1) * 4;
+    plan_desc_kernel<<<dim3(l1 - l0, PLAN_DESC_PARTS), 1024, sm, st>>>(L, l0, ahead);
     return cudaGetLastError();
 }
 
@@ -875,6 +913,7 @@ cudaError_t prepare_decode(int smem) {
     if (e == cudaSuccess) e = allow_max_dynamic_smem(decode_kernel<float, 2>, smem);
     if (e == cudaSuccess) e = allow_max_dynamic_smem(decode_kernel<float, 4>, smem);
     if (e == cudaSuccess) e = allow_max_dynamic_smem(plan_kernel, smem);
+    if (e == cudaSuccess) e = allow_max_dynamic_smem(plan_desc_kernel, smem);
     return e;
 }
 
