@@ -131,6 +131,13 @@ def test_lockstep_scaled_stacks(name):
     _lockstep(w, units, seed=11)
 
 
+@pytest.mark.parametrize("name", ["llamagen_xl", "janus_pro_1b"])
+def test_lockstep_fp32_caches(name):
+    """fp32 caches at d = 64 and d = 128 (chunks of 16 and 8 rows)."""
+    w = WORKLOADS[name].scaled(num_seqs=2, num_layers=1, dtype="f32")
+    _lockstep(w, [(0, 0), (1, 0)], seed=12)
+
+
 def test_unfused_append_attend_matches_oracle():
     w = WORKLOADS["janus_pro_1b"].scaled(num_seqs=2, num_layers=1)
     _lockstep(w, [(0, 0), (1, 0)], seed=5, fused=False)
