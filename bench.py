@@ -342,7 +342,9 @@ def gpu_arm(args, rank, world, dev):
         "evict_us_avg": float(evict_us.mean()),
         "evict_us_max": float(evict_us.max()),
         "labels_local_frac": float((labels == 1).mean()),
-        "gpu_launches": args.steps * (3 * Ly + steps * (Ly + 1)),
+        # per layer at prefill: attention, grouping, packing, plan (2); per
+        # step: one decode launch per layer, eviction scan and run, plan (2)
+        "gpu_launches": args.steps * (5 * Ly + steps * (Ly + 4)),
         "kv_pool_bytes": cache.nbytes,
     }
     del g_main

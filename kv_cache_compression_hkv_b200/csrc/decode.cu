@@ -33,6 +33,8 @@ constexpr int DECODE_MAX_WARPS = 12;
 // Cost of a chunk, in units of the cost of a head's end, in the plan's
 // balancing of the warp ranges.
 constexpr int CHUNK_COST = 3;
+// Most chunks a range starting a decode block moves to avoid cutting a head.
+constexpr int SNAP_MAX = 2;
 
 // Packed storage of DPL consecutive elements of one row.
 template <typename T, int DPL> struct Raw;
@@ -231,7 +233,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
     const int64_t tcost = (int64_t)CHUNK_COST * total + n;
     const bool narrow = tcost * GW < ((int64_t)1 << 31);  // 32-bit arithmetic suffices
     int32_t* gw_beg = L.plan_wbeg + (size_t)layer * (PLAN_MAX_WARPS + 1);
-    for (int w = tid; w <= GW; w += blockDim.x) {
+    // first chunk of warp w's range by cost; *head: the head holding it
+    auto begin_of = [&](int w, int* head) -> int {
+        if (w >= GW) { *head = n; return total; }
         const int64_t b = narrow ? (int64_t)((uint32_t)w * (uint32_t)tcost / (uint32_t)GW)
                                  : (int64_t)w * tcost / GW;
         int lo = 0, hi = n;  // first head whose cost ends after b
@@ -246,14 +250,33 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
                 if ((int64_t)CHUNK_COST * cnt[mid] + mid + 1 > b) hi = mid; else lo = mid + 1;
             }
         }
-        int c = total;
-        if (lo < n) {
-            const int c0 = lo ? cnt[lo - 1] : 0;
-            const int64_t base = lo ? (int64_t)CHUNK_COST * c0 + lo : 0;
-            const int k = (int)((b - base + CHUNK_COST - 1) / CHUNK_COST);
-            c = c0 + min(max(k, 0), cnt[lo] - c0);
+        *head = lo;
+        if (lo >= n) return total;
+        const int c0 = lo ? cnt[lo - 1] : 0;
+        const int64_t base = lo ? (int64_t)CHUNK_COST * c0 + lo : 0;
+        const int k = (int)((b - base + CHUNK_COST - 1) / CHUNK_COST);
+        return c0 + min(max(k, 0), cnt[lo] - c0);
+    };
+    // A range starting a decode block moves to the nearer end of the head
+    // it would cut (at most SNAP_MAX chunks, staying between its neighbours'
+    // starts), so that heads seldom span two blocks and their split
+    // segments meet in shared memory.
+    const int NWB = L.plan_nw;
+    for (int w = tid; w <= GW; w += blockDim.x) {
+        int lo;
+        int c = begin_of(w, &lo);
+        if (w > 0 && w < GW && NWB > 1 && w % NWB == 0 && lo < n) {
+            const int c0 = lo ? cnt[lo - 1] : 0, c1 = cnt[lo];
+            if (c > c0 && c < c1) {
+                int dummy;
+                const int prev = begin_of(w - 1, &dummy), next = begin_of(w + 1, &dummy);
+                const int down = c - c0, up = c1 - c;
+                if (down <= up && down <= SNAP_MAX && c0 >= prev) c = c0;
+                else if (up <= SNAP_MAX && c1 <= next) c = c1;
+                else if (down <= SNAP_MAX && c0 >= prev) c = c0;
+            }
         }
-        gw_beg[w] = w == GW ? total : c;
+        gw_beg[w] = c;
     }
     // the head facts and chunk prefix for the descriptor kernel
     int32_t* gcnt = L.plan_cnt + hbase;

@@ -16,12 +16,12 @@
 
 namespace hkv {
 
-// Per-warp scratch of the eviction: the select's own scratch, the head's
-// scores and positions, the (max, sum) of the scoring steps, the step each
-// column holds, an mbarrier, then the K and V rows of the top M slots
-// (`row_bytes` each), prefetched while the head is scored.
+// Per-warp scratch of the eviction: the select's own scratch, the (max, sum)
+// of the scoring steps, the step each column holds, an mbarrier, the
+// positions of the top M slots, then their K and V rows (`row_bytes` each),
+// prefetched while the head is scored.
 __host__ __device__ inline size_t evict_warp_bytes(int n_max, int m_rows, int row_bytes) {
-    return select_scratch_bytes(n_max) + (size_t)round32(n_max) * 8 + 32 * 8 + 32 * 4 + 16 +
+    return select_scratch_bytes(n_max) + 32 * 8 + 32 * 4 + 16 + (size_t)round32(m_rows) * 4 +
            2 * (size_t)m_rows * row_bytes;
 }
 
@@ -65,12 +65,11 @@ __global__ void __launch_bounds__(EVICT_MAX_WARPS * 32) evict_run_kernel(Layout 
     const int MR = L.M;  // rows above the budget of a due head
     unsigned char* wbase = esm + (size_t)warp * evict_warp_bytes(n_max, MR, row_bytes);
     SelectScratch sc = carve_select_scratch(wbase, n_max);
-    float* sc_s = reinterpret_cast<float*>(wbase + select_scratch_bytes(n_max));
-    int32_t* pos_s = reinterpret_cast<int32_t*>(sc_s + round32(n_max));
-    float2* ml_s = reinterpret_cast<float2*>(pos_s + round32(n_max));
+    float2* ml_s = reinterpret_cast<float2*>(wbase + select_scratch_bytes(n_max));
     int32_t* step_s = reinterpret_cast<int32_t*>(ml_s + 32);
     uint64_t* bar = reinterpret_cast<uint64_t*>(step_s + 32);
-    unsigned char* kbuf = reinterpret_cast<unsigned char*>(bar) + 16;
+    int32_t* top_pos = reinterpret_cast<int32_t*>(bar + 2);
+    unsigned char* kbuf = reinterpret_cast<unsigned char*>(top_pos + round32(MR));
     unsigned char* vbuf = kbuf + (size_t)MR * row_bytes;
     const int n_heads = L.S * L.H;
     T* Kp = reinterpret_cast<T*>(L.K);
@@ -114,8 +113,10 @@ __global__ void __launch_bounds__(EVICT_MAX_WARPS * 32) evict_run_kernel(Layout 
         __syncwarp();
         // scores: summed softmax weight of the last r queries, each
         // counting only tokens already cached at its step.  Tokens go in
-        // batches of 8 per lane whose loads are all issued before any is used.
+        // batches of 8 per lane whose loads are all issued before any is
+        // used; every 32 of them are sorted into the strata right away.
         bool bad = false;
+        int nn = 0, nf = 0;
         for (int b0 = 0; b0 < n; b0 += 32 * 8) {
             int pv[8];
             float4 la[8], lb[8];
@@ -133,32 +134,32 @@ __global__ void __launch_bounds__(EVICT_MAX_WARPS * 32) evict_run_kernel(Layout 
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int q = b0 + u * 32 + lane;
-                if (q >= n) continue;
-                const int p = pv[u];
+                const int base = b0 + u * 32;
+                if (base >= n) break;  // warp-uniform
+                const int q = base + lane;
+                const bool valid = q < n;
+                const int p = valid ? pv[u] : 0;
                 float acc = 0.f;
-                if (r == 8) {
-                    const float v[8] = {la[u].x, la[u].y, la[u].z, la[u].w, lb[u].x, lb[u].y, lb[u].z, lb[u].w};
+                if (valid) {
+                    if (r == 8) {
+                        const float v[8] = {la[u].x, la[u].y, la[u].z, la[u].w, lb[u].x, lb[u].y, lb[u].z, lb[u].w};
 #pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        if (p <= step_s[c]) acc += exp2f(v[c] - ml_s[c].x) * ml_s[c].y;
-                } else {
-                    const float* lg = L.logit + (slot0 + q) * r;
-                    for (int c = 0; c < r; ++c)
-                        if (p <= step_s[c]) acc += exp2f(lg[c] - ml_s[c].x) * ml_s[c].y;
+                        for (int c = 0; c < 8; ++c)
+                            if (p <= step_s[c]) acc += exp2f(v[c] - ml_s[c].x) * ml_s[c].y;
+                    } else {
+                        const float* lg = L.logit + (slot0 + q) * r;
+                        for (int c = 0; c < r; ++c)
+                            if (p <= step_s[c]) acc += exp2f(lg[c] - ml_s[c].x) * ml_s[c].y;
+                    }
+                    if (isnan(acc)) bad = true;
+                    if (q >= target) top_pos[q - target] = p;
                 }
-                if (isnan(acc)) bad = true;
-                sc_s[q] = acc;
-                pos_s[q] = p;
+                warp_partition_batch(sc, n, t, L.D, L.stratified, base, valid, __float_as_uint(acc), p, nn, nf);
             }
         }
         __syncwarp();
-        auto key_of = [&](int q, uint32_t& sb, int32_t& p) {
-            sb = __float_as_uint(sc_s[q]);
-            p = pos_s[q];
-        };
         const int E = n - target;
-        warp_stratified_select(sc, n, t, L.D, E / 2, E - E / 2, L.stratified, key_of);
+        warp_select_partitioned(sc, n, nn, nf, E / 2, E - E / 2, L.stratified);
         if (__any_sync(FULL_MASK, bad) && lane == 0) latch_error(L, HKV_ERR_NUMERIC, (int)hx);
         // holes: evicted slots below the budget; movers: survivors above it
         int nh = 0, nm = 0;
@@ -203,7 +204,7 @@ __global__ void __launch_bounds__(EVICT_MAX_WARPS * 32) evict_run_kernel(Layout 
             *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(Vp) + dst) = vw;
         }
         for (int mv = lane; mv < nh; mv += 32)
-            L.pos[slot0 + sc.moves[mv]] = pos_s[sc.moves[sc.n_max - 1 - mv]];
+            L.pos[slot0 + sc.moves[mv]] = top_pos[sc.moves[sc.n_max - 1 - mv] - target];
         __syncwarp();
         if (lane == 0) {
             L.base_len[hx] = target;

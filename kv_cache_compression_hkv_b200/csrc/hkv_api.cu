@@ -230,6 +230,7 @@ hkv_status hkv_create(const hkv_config* cfg, void* pool, size_t bytes, void* str
         return HKV_ERR_INVALID_ARG;
     }
     c->lay.plan_gw = c->decode_grid * c->decode_sh.warps;
+    c->lay.plan_nw = c->decode_sh.warps;
     c->plan_for.assign(cfg->num_layers, -1);
     c->evict_grid = c->n_sm;
     *out = c;

@@ -61,6 +61,7 @@ struct Layout {
     // chunk, total, 0} and copies of its range's first descriptors
     int4* plan_warp;
     int32_t plan_gw;     // warps of one decode launch
+    int32_t plan_nw;     // warps of one decode block
     int32_t max_chunks;
 };
 
@@ -242,20 +243,37 @@ __device__ inline uint32_t warp_radix_kth_score(const uint64_t* keys, int m, int
 // Marks the k lowest of m <= 32 * U distinct keys: lane l ranks keys
 // l, l + 32, ... (held in registers) against every key in one pass of
 // shared-memory broadcast reads; rank < k is exactly the k lowest.
+__device__ __forceinline__ uint64_t lds_u64(uint32_t addr) {
+    uint64_t v;
+    asm volatile("ld.shared.u64 %0, [%1];" : "=l"(v) : "r"(addr));
+    return v;
+}
+
 template <int U>
 __device__ inline void warp_rank_evict(const uint64_t* keys, const uint16_t* slots, int m, int k,
                                        uint32_t* evict_bits) {
     const int lane = threadIdx.x & 31;
+    const uint32_t kbase = (uint32_t)__cvta_generic_to_shared(keys);  // keys live in shared memory
     uint64_t mine[U];
     int rk[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
         const int i = lane + 32 * u;
-        mine[u] = i < m ? keys[i] : ~0ull;
+        mine[u] = i < m ? lds_u64(kbase + 8 * i) : ~0ull;
         rk[u] = 0;
     }
-    for (int j = 0; j < m; ++j) {
-        const uint64_t kj = keys[j];
+    int j = 0;
+    for (; j + 8 <= m; j += 8) {  // eight broadcast reads in flight
+        uint64_t kj[8];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) kj[v] = lds_u64(kbase + 8 * (j + v));
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+#pragma unroll
+            for (int u = 0; u < U; ++u) rk[u] += kj[v] < mine[u];
+    }
+    for (; j < m; ++j) {
+        const uint64_t kj = lds_u64(kbase + 8 * j);
 #pragma unroll
         for (int u = 0; u < U; ++u) rk[u] += kj < mine[u];
     }
@@ -297,6 +315,43 @@ __device__ inline SelectScratch carve_select_scratch(unsigned char* base, int n_
     return s;
 }
 
+// One batch of 32 tokens (token base + lane) into the strata: near keys
+// fill keys[] from the front, far keys from the back (nn, nf: counts so far,
+// updated); the batch's evict-bit word is cleared.  All lanes call it.
+__device__ __forceinline__ void warp_partition_batch(const SelectScratch& sc, int n, int t, int D,
+                                                     int stratified, int base, bool valid,
+                                                     uint32_t sb, int32_t p, int& nn, int& nf) {
+    const int lane = threadIdx.x & 31;
+    const int i = base + lane;
+    bool is_near = false, is_far = false;
+    const uint64_t key = ((uint64_t)sb << 32) | (uint32_t)p;
+    if (valid) {
+        const int delta = t - p;
+        if (delta >= 1) {
+            if (stratified && delta <= D) is_near = true; else is_far = true;
+        }
+    }
+    const unsigned bn = __ballot_sync(FULL_MASK, is_near);
+    const unsigned bf = __ballot_sync(FULL_MASK, is_far);
+    const unsigned lt = (1u << lane) - 1u;
+    if (is_near) {
+        const int o = nn + __popc(bn & lt);
+        sc.keys[o] = key;
+        sc.slot[o] = (uint16_t)i;
+    }
+    if (is_far) {
+        const int o = n - 1 - (nf + __popc(bf & lt));
+        sc.keys[o] = key;
+        sc.slot[o] = (uint16_t)i;
+    }
+    nn += __popc(bn);
+    nf += __popc(bf);
+    if (lane == 0) sc.evict_bits[base >> 5] = 0u;
+}
+
+__device__ int warp_select_partitioned(const SelectScratch& sc, int n, int nn, int nf, int k_near,
+                                       int k_far, int stratified);
+
 // Stratified select over tokens 0..n) whose keys a functor provides:
 // key_of(i, score_bits, pos).  Candidates: t - pos >= 1; near: t - pos <= D
 // (every candidate is "far" when !stratified).  k_near / k_far lowest keys
@@ -310,36 +365,20 @@ __device__ int warp_stratified_select(const SelectScratch& sc, int n, int t, int
     int nn = 0, nf = 0;
     for (int base = 0; base < n; base += 32) {
         const int i = base + lane;
-        bool is_near = false, is_far = false;
-        uint64_t key = 0;
-        if (i < n) {
-            uint32_t sb;
-            int32_t p;
-            key_of(i, sb, p);
-            key = ((uint64_t)sb << 32) | (uint32_t)p;
-            const int delta = t - p;
-            if (delta >= 1) {
-                if (stratified && delta <= D) is_near = true; else is_far = true;
-            }
-        }
-        const unsigned bn = __ballot_sync(FULL_MASK, is_near);
-        const unsigned bf = __ballot_sync(FULL_MASK, is_far);
-        const unsigned lt = (1u << lane) - 1u;
-        if (is_near) {
-            const int o = nn + __popc(bn & lt);
-            sc.keys[o] = key;
-            sc.slot[o] = (uint16_t)i;
-        }
-        if (is_far) {
-            const int o = n - 1 - (nf + __popc(bf & lt));
-            sc.keys[o] = key;
-            sc.slot[o] = (uint16_t)i;
-        }
-        nn += __popc(bn);
-        nf += __popc(bf);
-        if (lane == 0) sc.evict_bits[base >> 5] = 0u;
+        uint32_t sb = 0;
+        int32_t p = 0;
+        if (i < n) key_of(i, sb, p);
+        warp_partition_batch(sc, n, t, D, stratified, base, i < n, sb, p, nn, nf);
     }
     __syncwarp();
+    return warp_select_partitioned(sc, n, nn, nf, k_near, k_far, stratified);
+}
+
+// The selection once the strata are partitioned (nn near keys at the
+// front of keys[], nf far keys at the back, evict bits cleared).
+__device__ inline int warp_select_partitioned(const SelectScratch& sc, int n, int nn, int nf, int k_near,
+                                              int k_far, int stratified) {
+    const int lane = threadIdx.x & 31;
     int kn = k_near, kf = k_far;
     if (stratified) {
         if (kn > nn) { kf += kn - nn; kn = nn; }

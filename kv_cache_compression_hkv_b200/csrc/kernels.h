@@ -7,6 +7,7 @@
 
 namespace hkv {
 
+
 // Raises the dynamic shared-memory limits the kernels of this layout need
 // (a host call that must not run inside a stream capture; hkv_create makes it).
 cudaError_t prepare_kernels();
