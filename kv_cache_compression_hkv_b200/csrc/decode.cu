@@ -220,11 +220,39 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
     for (int i = i0; i < i1; ++i) cnt[i] += offset;
     __syncthreads();
     const int total = cnt[n - 1];
-    const int GW = L.plan_gw;
     if (total > L.max_chunks) {  // cannot happen for a consistent cache
         if (tid == 0) latch_error(L, HKV_ERR_STATE, layer);
         return;
     }
+    // the head facts and chunk prefix for the descriptor kernel
+    int32_t* gcnt = L.plan_cnt + hbase;
+    int4* gfact = L.plan_hfact + hbase;
+    for (int i = tid; i < n; i += blockDim.x) {
+        gcnt[i] = cnt[i];
+        gfact[i] = make_int4(hslot[i], hlen[i], hscore[i], 0);
+    }
+}
+
+// Second half of the plan: the warp ranges (every block of a layer
+// computes them all), every chunk's descriptor, each warp's record and a
+// copy of the first PLAN_WARP_DESC descriptors of its range in its plan
+// block.  Blocks (layer, part): part p takes the p-th slice of the layer's
+// heads and of its warps.
+__global__ void __launch_bounds__(1024) plan_desc_kernel(Layout L, int l0, int ahead) {
+    extern __shared__ int32_t dsm32[];
+    const int layer = l0 + blockIdx.x;
+    const int n = L.S * L.H;
+    const int GW = L.plan_gw;
+    const int t = L.t_next[layer] - 1 + ahead;
+    if (t >= L.L) return;
+    const size_t hbase = (size_t)layer * n;
+    int32_t* cnt = dsm32;            // inclusive prefix of the chunk counts
+    int32_t* wbeg = dsm32 + n;       // [GW + 1] first chunk of each warp's range
+    const int32_t* gcnt = L.plan_cnt + hbase;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) cnt[i] = gcnt[i];
+    __syncthreads();
+    const int total = cnt[n - 1];
+    if (total > L.max_chunks) return;  // the first half latched the error
     // Warp ranges of equal cost: a chunk costs CHUNK_COST units and a head
     // one more (its end: reductions, output, a merge when split), so that
     // warps holding many short heads get fewer chunks.  Head i's cost ends
@@ -232,7 +260,6 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
     // chunk whose cost starts at or after w * cost / GW.
     const int64_t tcost = (int64_t)CHUNK_COST * total + n;
     const bool narrow = tcost * GW < ((int64_t)1 << 31);  // 32-bit arithmetic suffices
-    int32_t* gw_beg = L.plan_wbeg + (size_t)layer * (PLAN_MAX_WARPS + 1);
     // first chunk of warp w's range by cost; *head: the head holding it
     auto begin_of = [&](int w, int* head) -> int {
         if (w >= GW) { *head = n; return total; }
@@ -262,7 +289,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
     // starts), so that heads seldom span two blocks and their split
     // segments meet in shared memory.
     const int NWB = L.plan_nw;
-    for (int w = tid; w <= GW; w += blockDim.x) {
+    for (int w = threadIdx.x; w <= GW; w += blockDim.x) {
         int lo;
         int c = begin_of(w, &lo);
         if (w > 0 && w < GW && NWB > 1 && w % NWB == 0 && lo < n) {
@@ -276,38 +303,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
                 else if (down <= SNAP_MAX && c0 >= prev) c = c0;
             }
         }
-        gw_beg[w] = c;
+        wbeg[w] = c;
     }
-    // the head facts and chunk prefix for the descriptor kernel
-    int32_t* gcnt = L.plan_cnt + hbase;
-    int4* gfact = L.plan_hfact + hbase;
-    for (int i = tid; i < n; i += blockDim.x) {
-        gcnt[i] = cnt[i];
-        gfact[i] = make_int4(hslot[i], hlen[i], hscore[i], 0);
-    }
-}
-
-// Second half of the plan: every chunk's descriptor, each warp's record
-// and a copy of the first PLAN_WARP_DESC descriptors of its range in its
-// plan block.  Blocks (layer, part): part p takes the p-th slice of the
-// layer's heads and of its warps.
-__global__ void __launch_bounds__(1024) plan_desc_kernel(Layout L, int l0, int ahead) {
-    extern __shared__ int32_t dsm32[];
-    const int layer = l0 + blockIdx.x;
-    const int n = L.S * L.H;
-    const int GW = L.plan_gw;
-    const int t = L.t_next[layer] - 1 + ahead;
-    if (t >= L.L) return;
-    const size_t hbase = (size_t)layer * n;
-    int32_t* cnt = dsm32;            // inclusive prefix of the chunk counts
-    int32_t* wbeg = dsm32 + n;       // [GW + 1]
-    const int32_t* gcnt = L.plan_cnt + hbase;
-    const int32_t* gw_beg = L.plan_wbeg + (size_t)layer * (PLAN_MAX_WARPS + 1);
-    for (int i = threadIdx.x; i < n; i += blockDim.x) cnt[i] = gcnt[i];
-    for (int w = threadIdx.x; w <= GW; w += blockDim.x) wbeg[w] = gw_beg[w];
     __syncthreads();
-    const int total = cnt[n - 1];
-    if (total > L.max_chunks) return;  // the first half latched the error
     // the warp whose range holds chunk c (the last w with wbeg[w] <= c)
     auto owner = [&](int c) -> int {
         int lo = 0, hi = GW - 1;
@@ -409,7 +407,8 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
     constexpr int D = DPL * 32;
     constexpr int ROW = D * (int)sizeof(T);           // bytes of one cache row
     constexpr int PPR = ROW / 16;                     // 16-byte pieces per row
-    constexpr int STAGE = (2 * CHUNK + 1) * ROW;      // K rows, V rows, the query
+    constexpr int KVR = 2 * ROW;                      // bytes of one K|V row pair
+    constexpr int STAGE = CHUNK * KVR + ROW;          // K|V row pairs, the query
     constexpr int E = 16 / (int)sizeof(T);            // elements per 16-byte piece
     constexpr int G = PPR;                            // lanes covering one row
     constexpr int TPI = 32 / G;                       // rows per pass
@@ -422,8 +421,7 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
     const int vg = lane / G, vc = lane % G;  // row group and piece of this lane
     const size_t hbase = (size_t)layer * n_heads;
     const size_t lrow = (size_t)layer * L.S * L.R;    // first slot of the layer
-    const T* Kp = reinterpret_cast<const T*>(L.K);
-    const T* Vp = reinterpret_cast<const T*>(L.V);
+    const T* KVp = reinterpret_cast<const T*>(L.K);  // slot s: K at 2 D s, V at 2 D s + D
     const float qscale = LOG2E / sqrtf((float)D);
 
     // Launched as a programmatic dependent of the previous launch in the
@@ -478,7 +476,6 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
         auto copy_chunk = [&](int stage, int part, const ChunkDesc& c, int q) {
             if (lane != 0) return;
             unsigned char* kd = my + (size_t)stage * STAGE;
-            unsigned char* vd = kd + CHUNK * ROW;
             uint64_t* bar = &bars[stage];
             const int a = append ? c.a : -1;
             if (part != 2) {
@@ -486,20 +483,18 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
                 const size_t row0 = lrow + c.row;
                 const int lo = a < 0 ? c.n : a;  // cached rows [0, lo) and (a, n)
                 if (lo > 0) {
-                    ptx::bulk_g2s(kd, Kp + row0 * D, lo * ROW, bar);
-                    ptx::bulk_g2s(vd, Vp + row0 * D, lo * ROW, bar);
+                    ptx::bulk_g2s(kd, KVp + row0 * 2 * D, lo * KVR, bar);
                 }
                 if (a >= 0 && a + 1 < c.n) {
-                    ptx::bulk_g2s(kd + (a + 1) * ROW, Kp + (row0 + a + 1) * D, (c.n - a - 1) * ROW, bar);
-                    ptx::bulk_g2s(vd + (a + 1) * ROW, Vp + (row0 + a + 1) * D, (c.n - a - 1) * ROW, bar);
+                    ptx::bulk_g2s(kd + (a + 1) * KVR, KVp + (row0 + a + 1) * 2 * D, (c.n - a - 1) * KVR, bar);
                 }
             }
             if (part != 1) {
                 if (a >= 0) {
-                    ptx::bulk_g2s(kd + a * ROW, k_t + (size_t)c.head * D, ROW, bar);
-                    ptx::bulk_g2s(vd + a * ROW, v_t + (size_t)c.head * D, ROW, bar);
+                    ptx::bulk_g2s(kd + a * KVR, k_t + (size_t)c.head * D, ROW, bar);
+                    ptx::bulk_g2s(kd + a * KVR + ROW, v_t + (size_t)c.head * D, ROW, bar);
                 }
-                if (q) ptx::bulk_g2s(vd + CHUNK * ROW, q_t + (size_t)c.head * D, ROW, bar);
+                if (q) ptx::bulk_g2s(kd + CHUNK * KVR, q_t + (size_t)c.head * D, ROW, bar);
             }
         };
         // descriptors of the range, 32 chunks per window, lane k holding
@@ -573,9 +568,9 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
             phase ^= 1u << stage;
             const int n = c.n;
             const unsigned char* kst = my + (size_t)stage * STAGE;
-            const unsigned char* vst = kst + CHUNK * ROW;
+            const unsigned char* vst = kst + ROW;  // V half of each row pair
             if (seg_start) {  // a new head: this lane's piece of its query
-                qw = *reinterpret_cast<const uint4*>(vst + CHUNK * ROW + vc * 16);
+                qw = *reinterpret_cast<const uint4*>(kst + CHUNK * KVR + vc * 16);
                 seg_whole = c.first;
             }
             // QK: pass p, lane (vg, vc) takes piece vc of row p * TPI + vg;
@@ -589,7 +584,7 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
             for (int p = 0; p < NPASS; ++p) {
                 const int row = p * TPI + vg;
                 float a0 = 0.f, a1 = 0.f;
-                const uint4 kw = *reinterpret_cast<const uint4*>(kst + row * ROW + vc * 16);
+                const uint4 kw = *reinterpret_cast<const uint4*>(kst + row * KVR + vc * 16);
                 if constexpr (sizeof(T) == 2) {
                     fma_bf16x2(a0, a1, kw.x, qw.x);
                     fma_bf16x2(a0, a1, kw.y, qw.y);
@@ -645,7 +640,7 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
                 const int jr = p * TPI + vg;
                 const float pj = myp[jr];
                 float x[E];
-                unpack16<T>(*reinterpret_cast<const uint4*>(vst + jr * ROW + vc * 16), x);
+                unpack16<T>(*reinterpret_cast<const uint4*>(vst + jr * KVR + vc * 16), x);
                 float* pu = pa[p & 1];
 #pragma unroll
                 for (int e = 0; e < E; e += 2) ffma2(pu[e], pu[e + 1], pj, pj, x[e], x[e + 1]);
@@ -664,10 +659,10 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
             if (append && c.a >= 0) {
                 const int a = c.a;
                 Raw<T, DPL> kr, vr;
-                kr.load_shared(reinterpret_cast<const T*>(kst + a * ROW) + lane * DPL);
-                vr.load_shared(reinterpret_cast<const T*>(vst + a * ROW) + lane * DPL);
-                kr.store(reinterpret_cast<T*>(L.K) + (row0 + a) * D + lane * DPL);
-                vr.store(reinterpret_cast<T*>(L.V) + (row0 + a) * D + lane * DPL);
+                kr.load_shared(reinterpret_cast<const T*>(kst + a * KVR) + lane * DPL);
+                vr.load_shared(reinterpret_cast<const T*>(vst + a * KVR) + lane * DPL);
+                kr.store(reinterpret_cast<T*>(L.K) + (row0 + a) * 2 * D + lane * DPL);
+                vr.store(reinterpret_cast<T*>(L.K) + (row0 + a) * 2 * D + D + lane * DPL);
                 if (lane == 0) L.pos[row0 + a] = t;
             }
             __syncwarp();  // every lane is done with this stage
@@ -840,8 +835,8 @@ __global__ void __launch_bounds__(256) append_kernel(Layout L, int layer, const 
             Raw<T, DPL> kr, vr;
             kr.load(k_t + (size_t)h * L.d + lane * DPL);
             vr.load(v_t + (size_t)h * L.d + lane * DPL);
-            kr.store(reinterpret_cast<T*>(L.K) + slot * L.d + lane * DPL);
-            vr.store(reinterpret_cast<T*>(L.V) + slot * L.d + lane * DPL);
+            kr.store(reinterpret_cast<T*>(L.K) + slot * 2 * L.d + lane * DPL);
+            vr.store(reinterpret_cast<T*>(L.K) + slot * 2 * L.d + L.d + lane * DPL);
             if (lane == 0) L.pos[slot] = t;
         }
     }

@@ -69,12 +69,11 @@ __global__ void __launch_bounds__(EVICT_MAX_WARPS * 32) evict_run_kernel(Layout 
     int32_t* step_s = reinterpret_cast<int32_t*>(ml_s + 32);
     uint64_t* bar = reinterpret_cast<uint64_t*>(step_s + 32);
     int32_t* top_pos = reinterpret_cast<int32_t*>(bar + 2);
-    unsigned char* kbuf = reinterpret_cast<unsigned char*>(top_pos + round32(MR));
-    unsigned char* vbuf = kbuf + (size_t)MR * row_bytes;
+    unsigned char* kvbuf = reinterpret_cast<unsigned char*>(top_pos + round32(MR));  // K|V row pairs
     const int n_heads = L.S * L.H;
-    T* Kp = reinterpret_cast<T*>(L.K);
-    T* Vp = reinterpret_cast<T*>(L.V);
-    const int per_row = row_bytes / 16;  // 16-byte pieces per row
+    unsigned char* KVb = reinterpret_cast<unsigned char*>(L.K);  // slot s: K|V pair at 2 row_bytes s
+    const int pair = 2 * row_bytes;
+    const int per_pair = pair / 16;  // 16-byte pieces per K|V pair
     const int count = L.due_ctl[0];
     if (lane == 0) {
         ptx::mbar_init(bar, 1);
@@ -99,9 +98,8 @@ __global__ void __launch_bounds__(EVICT_MAX_WARPS * 32) evict_run_kernel(Layout 
         const int top = n - target;  // the slots a survivor may move from
         // the K and V rows of slots target .. n-1, while the head is scored
         if (lane == 0 && top > 0) {
-            ptx::mbar_expect_tx(bar, (uint32_t)(2 * top * row_bytes));
-            ptx::bulk_g2s(kbuf, Kp + (slot0 + target) * d, top * row_bytes, bar);
-            ptx::bulk_g2s(vbuf, Vp + (slot0 + target) * d, top * row_bytes, bar);
+            ptx::mbar_expect_tx(bar, (uint32_t)(top * pair));
+            ptx::bulk_g2s(kvbuf, KVb + (slot0 + target) * pair, top * pair, bar);
         }
         // (max, 1/sum) of each scoring step, by column = step mod r, and the
         // step each column holds inside the window t-r+1 .. t
@@ -193,15 +191,13 @@ __global__ void __launch_bounds__(EVICT_MAX_WARPS * 32) evict_run_kernel(Layout 
         }
         // move rows: each survivor's K and V rows from shared memory into a
         // hole, in 16-byte pieces
-        const int pieces = nh * per_row;
+        const int pieces = nh * per_pair;
         for (int w = lane; w < pieces; w += 32) {
-            const int mv = w / per_row, pc = w % per_row;
+            const int mv = w / per_pair, pc = w % per_pair;
             const int src = sc.moves[sc.n_max - 1 - mv] - target;
-            const size_t dst = (slot0 + sc.moves[mv]) * row_bytes + pc * 16;
-            const uint4 kw = *reinterpret_cast<const uint4*>(kbuf + (size_t)src * row_bytes + pc * 16);
-            const uint4 vw = *reinterpret_cast<const uint4*>(vbuf + (size_t)src * row_bytes + pc * 16);
-            *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(Kp) + dst) = kw;
-            *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(Vp) + dst) = vw;
+            const size_t dst = (slot0 + sc.moves[mv]) * pair + pc * 16;
+            *reinterpret_cast<uint4*>(KVb + dst) =
+                *reinterpret_cast<const uint4*>(kvbuf + (size_t)src * pair + pc * 16);
         }
         for (int mv = lane; mv < nh; mv += 32)
             L.pos[slot0 + sc.moves[mv]] = top_pos[sc.moves[sc.n_max - 1 - mv] - target];

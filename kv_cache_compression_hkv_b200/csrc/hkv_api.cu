@@ -127,8 +127,8 @@ size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Lay
     l.n_tau = (int32_t*)take(nh * 4);
     l.label = (uint8_t*)take(nh);
     l.due_t = (int32_t*)take(Ly * S * 4);
-    l.K = take(slots * d * es);
-    l.V = take(slots * d * es);
+    l.K = take(slots * 2 * d * es);  // K and V rows interleaved per slot
+    l.V = l.K ? (unsigned char*)l.K + d * es : nullptr;
     l.pos = (int32_t*)take(slots * 4);
     l.logit = (float*)take(slots * r * 4);
     l.ml = (float2*)take(nh * r * 8);
@@ -138,7 +138,6 @@ size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Lay
     l.plan_desc = (int4*)take(Ly * max_chunks * 16);
     l.plan_cnt = (int32_t*)take(nh * 4);
     l.plan_hfact = (int4*)take(nh * 16);
-    l.plan_wbeg = (int32_t*)take(Ly * (hkv::PLAN_MAX_WARPS + 1) * 4);
     l.plan_warp = (int4*)take(Ly * hkv::PLAN_MAX_WARPS * (1 + hkv::PLAN_WARP_DESC) * 16);
     l.S = c->num_seqs; l.Ly = c->num_layers; l.H = c->num_heads; l.d = c->head_dim;
     l.L = c->max_len; l.W = c->local_window; l.M = c->ste_m; l.D = c->near_dist;

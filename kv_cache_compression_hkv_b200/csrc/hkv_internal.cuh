@@ -41,8 +41,8 @@ struct Layout {
     // per (layer, sequence): step at which its Global heads reach their cap
     int32_t* due_t;
     // cache rows, slot index (l*S + s)*R + slot
-    void* K;            // [Ly][S][R][d]
-    void* V;
+    void* K;            // [Ly][S][R][2][d]: per slot its K row, then its V row
+    void* V;            // K + d elements (same row stride 2 d)
     int32_t* pos;       // [Ly][S][R]
     float* logit;       // [Ly][S][R][r]   exp2-domain logits of scoring steps
     float2* ml;         // [Ly][S][H][r]   (max, sum) of those steps' softmax
@@ -56,7 +56,6 @@ struct Layout {
     int4* plan_desc;     // [Ly][max_chunks] one descriptor per chunk
     int32_t* plan_cnt;   // [Ly][S*H] inclusive prefix of the heads' chunk counts
     int4* plan_hfact;    // [Ly][S*H] {first row, len << 16 | appended slot, scoring, 0}
-    int32_t* plan_wbeg;  // [Ly][PLAN_MAX_WARPS + 1] first chunk of each warp's range
     // [Ly][PLAN_MAX_WARPS][1 + PLAN_WARP_DESC]: per warp {first chunk, end
     // chunk, total, 0} and copies of its range's first descriptors
     int4* plan_warp;

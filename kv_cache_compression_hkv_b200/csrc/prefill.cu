@@ -202,16 +202,15 @@ __global__ void __launch_bounds__(128) pack_kernel(Layout L, int layer, const T*
     const int per_row = d / piece;
     const size_t slot0 = region_slot0(L, layer, s) + L.off[hi];
     const int n_slots = lab == 1 ? (n_keep < L.W ? n_keep : L.W) : n_keep;
-    T* Kp = reinterpret_cast<T*>(L.K);
-    T* Vp = reinterpret_cast<T*>(L.V);
+    T* KVp = reinterpret_cast<T*>(L.K);  // slot s: K at 2 d s, V at 2 d s + d
     const T* kb = k + (size_t)b * block_stride;
     const T* vb = v + (size_t)b * block_stride;
     for (int w = threadIdx.x; w < n_slots * per_row; w += blockDim.x) {
         const int slot = w / per_row, c = (w % per_row) * piece;
         const int p = kept[slot];
-        *reinterpret_cast<uint4*>(Kp + (slot0 + slot) * d + c) =
+        *reinterpret_cast<uint4*>(KVp + (slot0 + slot) * 2 * d + c) =
             *reinterpret_cast<const uint4*>(kb + (size_t)p * d + c);
-        *reinterpret_cast<uint4*>(Vp + (slot0 + slot) * d + c) =
+        *reinterpret_cast<uint4*>(KVp + (slot0 + slot) * 2 * d + d + c) =
             *reinterpret_cast<const uint4*>(vb + (size_t)p * d + c);
     }
     for (int i = threadIdx.x; i < n_slots; i += blockDim.x) L.pos[slot0 + i] = kept[i];
