@@ -342,9 +342,9 @@ def gpu_arm(args, rank, world, dev):
         "evict_us_avg": float(evict_us.mean()),
         "evict_us_max": float(evict_us.max()),
         "labels_local_frac": float((labels == 1).mean()),
-        # per layer at prefill: attention, grouping, packing, plan (2); per
-        # step: one decode launch per layer, eviction scan and run, plan (2)
-        "gpu_launches": args.steps * (5 * Ly + steps * (Ly + 4)),
+        # per layer at prefill: attention, grouping, packing, plan; per
+        # step: one decode launch per layer, eviction scan and run, plan
+        "gpu_launches": args.steps * (4 * Ly + steps * (Ly + 3)),
         "kv_pool_bytes": cache.nbytes,
     }
     del g_main

@@ -160,9 +160,11 @@ __device__ __forceinline__ int4 shfl_int4(const int4& v, int src) {
 // ---------------------------------------------------------------------------
 // The plan of a layer's decode launch at step t (ahead = 1: the step of the
 // next append, t_next; ahead = 0: the newest cached position, t_next - 1).
-// One block per layer: per-head facts in shared memory, the chunk-count
-// prefix, every chunk's descriptor, and for every warp of the decode grid
-// its range and a copy of its first chunk's descriptor.
+// Blocks (layer, part): every block computes the layer's per-head facts,
+// the chunk-count prefix and the warp ranges in shared memory; part p then
+// writes the descriptors of the p-th slice of the heads and the records of
+// the p-th slice of the warps (each warp: its range and copies of the first
+// PLAN_WARP_DESC descriptors of its range).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead) {
     extern __shared__ int32_t psm[];
@@ -173,6 +175,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
     int32_t* hslot = psm + n;      // layer-relative row of the head's first token
     int32_t* hlen = psm + 2 * n;   // len << 16 | appended slot
     int32_t* hscore = psm + 3 * n; // scoring flag
+    int32_t* wbeg = psm + 4 * n;   // [GW + 1] first chunk of each warp's range
+    const int GW = L.plan_gw;
+    const int parts = gridDim.y, part = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, NW = blockDim.x >> 5;
     const int t = L.t_next[layer] - 1 + ahead;
     if (t >= L.L) return;  // the sequence is complete: no step left to plan
@@ -183,7 +188,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
         const int cap = L.cap[hx];
         int c = (len + CHUNK - 1) / CHUNK;
         if (len > cap || len < 1) {
-            latch_error(L, HKV_ERR_CAPACITY, (int)hx);
+            if (part == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
             c = 0;
         }
         const int jn = append_slot(L, hx, t, len);
@@ -221,38 +226,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
     __syncthreads();
     const int total = cnt[n - 1];
     if (total > L.max_chunks) {  // cannot happen for a consistent cache
-        if (tid == 0) latch_error(L, HKV_ERR_STATE, layer);
+        if (tid == 0 && part == 0) latch_error(L, HKV_ERR_STATE, layer);
         return;
     }
-    // the head facts and chunk prefix for the descriptor kernel
-    int32_t* gcnt = L.plan_cnt + hbase;
-    int4* gfact = L.plan_hfact + hbase;
-    for (int i = tid; i < n; i += blockDim.x) {
-        gcnt[i] = cnt[i];
-        gfact[i] = make_int4(hslot[i], hlen[i], hscore[i], 0);
-    }
-}
-
-// Second half of the plan: the warp ranges (every block of a layer
-// computes them all), every chunk's descriptor, each warp's record and a
-// copy of the first PLAN_WARP_DESC descriptors of its range in its plan
-// block.  Blocks (layer, part): part p takes the p-th slice of the layer's
-// heads and of its warps.
-__global__ void __launch_bounds__(1024) plan_desc_kernel(Layout L, int l0, int ahead) {
-    extern __shared__ int32_t dsm32[];
-    const int layer = l0 + blockIdx.x;
-    const int n = L.S * L.H;
-    const int GW = L.plan_gw;
-    const int t = L.t_next[layer] - 1 + ahead;
-    if (t >= L.L) return;
-    const size_t hbase = (size_t)layer * n;
-    int32_t* cnt = dsm32;            // inclusive prefix of the chunk counts
-    int32_t* wbeg = dsm32 + n;       // [GW + 1] first chunk of each warp's range
-    const int32_t* gcnt = L.plan_cnt + hbase;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) cnt[i] = gcnt[i];
-    __syncthreads();
-    const int total = cnt[n - 1];
-    if (total > L.max_chunks) return;  // the first half latched the error
     // Warp ranges of equal cost: a chunk costs CHUNK_COST units and a head
     // one more (its end: reductions, output, a merge when split), so that
     // warps holding many short heads get fewer chunks.  Head i's cost ends
@@ -318,12 +294,11 @@ __global__ void __launch_bounds__(1024) plan_desc_kernel(Layout L, int l0, int a
     constexpr int PB = 1 + PLAN_WARP_DESC;
     int4* dsc = L.plan_desc + (size_t)layer * L.max_chunks;
     int4* pw = L.plan_warp + (size_t)layer * PLAN_MAX_WARPS * PB;
-    const int parts = gridDim.y, part = blockIdx.y;
     const int h0 = (int)((int64_t)part * n / parts), h1 = (int)((int64_t)(part + 1) * n / parts);
     for (int i = h0 + threadIdx.x; i < h1; i += blockDim.x) {
         const int c1 = cnt[i], c0 = i ? cnt[i - 1] : 0;
         if (c1 == c0) continue;
-        const int4 f = L.plan_hfact[hbase + i];
+        const int4 f = make_int4(hslot[i], hlen[i], hscore[i], 0);
         const int wa = owner(c0), wb = owner(c1 - 1);
         int segs = 0;
         for (int w = wa; w <= wb; ++w) segs += wbeg[w] < wbeg[w + 1];
@@ -904,11 +879,7 @@ cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void*
 }
 
 cudaError_t launch_plan(const Layout& L, int l0, int l1, int ahead, cudaStream_t st) {
-    plan_kernel<<<l1 - l0, 1024, plan_smem_bytes(L.S * L.H), st>>>(L, l0, ahead);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    const size_t sm = ((size_t)L.S * L.H + PLAN_MAX_WARPS + 1) * 4;
-    plan_desc_kernel<<<dim3(l1 - l0, PLAN_DESC_PARTS), 1024, sm, st>>>(L, l0, ahead);
+    plan_kernel<<<dim3(l1 - l0, PLAN_DESC_PARTS), 1024, plan_smem_bytes(L.S * L.H), st>>>(L, l0, ahead);
     return cudaGetLastError();
 }
 
@@ -931,7 +902,6 @@ cudaError_t prepare_decode(int smem) {
     if (e == cudaSuccess) e = allow_max_dynamic_smem(decode_kernel<float, 2>, smem);
     if (e == cudaSuccess) e = allow_max_dynamic_smem(decode_kernel<float, 4>, smem);
     if (e == cudaSuccess) e = allow_max_dynamic_smem(plan_kernel, smem);
-    if (e == cudaSuccess) e = allow_max_dynamic_smem(plan_desc_kernel, smem);
     return e;
 }
 

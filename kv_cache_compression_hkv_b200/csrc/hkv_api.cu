@@ -136,8 +136,6 @@ size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Lay
     l.partial = (float*)take(2 * 2 * (size_t)hkv::PLAN_MAX_WARPS * (d + 2) * 4);
     l.due_list = (int32_t*)take(nh * 4);
     l.plan_desc = (int4*)take(Ly * max_chunks * 16);
-    l.plan_cnt = (int32_t*)take(nh * 4);
-    l.plan_hfact = (int4*)take(nh * 16);
     l.plan_warp = (int4*)take(Ly * hkv::PLAN_MAX_WARPS * (1 + hkv::PLAN_WARP_DESC) * 16);
     l.S = c->num_seqs; l.Ly = c->num_layers; l.H = c->num_heads; l.d = c->head_dim;
     l.L = c->max_len; l.W = c->local_window; l.M = c->ste_m; l.D = c->near_dist;

@@ -15,7 +15,7 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr int CHUNK = 32;  // tokens one warp handles per decode work item
 constexpr int PLAN_MAX_WARPS = 2048;  // capacity of a decode plan's warp table
 constexpr int PLAN_WARP_DESC = 7;     // descriptors copied into each warp's plan block
-constexpr int PLAN_DESC_PARTS = 4;    // blocks per layer writing a plan's descriptors
+constexpr int PLAN_DESC_PARTS = 4;    // blocks per layer of the plan kernel
 constexpr int RANK_MAX = 256;         // strata up to this size are selected by ranking
 
 // Everything a kernel needs to find the state of a (layer, sequence, head).
@@ -54,8 +54,6 @@ struct Layout {
     int32_t* due_list;  // [Ly*S*H] heads due for eviction this step
     // decode plan per layer, for the step it was made for (see plan_kernel)
     int4* plan_desc;     // [Ly][max_chunks] one descriptor per chunk
-    int32_t* plan_cnt;   // [Ly][S*H] inclusive prefix of the heads' chunk counts
-    int4* plan_hfact;    // [Ly][S*H] {first row, len << 16 | appended slot, scoring, 0}
     // [Ly][PLAN_MAX_WARPS][1 + PLAN_WARP_DESC]: per warp {first chunk, end
     // chunk, total, 0} and copies of its range's first descriptors
     int4* plan_warp;
