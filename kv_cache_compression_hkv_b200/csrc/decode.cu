@@ -486,9 +486,12 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
         if (lane >= PLAN_WARP_DESC)
             pwin = c_begin + lane < c_end ? dsc[c_begin + lane] : make_int4(0, 0, 0, 0);
         int4 cwin = pwin;
-        // the first stages: with `early` their cached rows go before the
-        // wait on the previous launch, the queries and appended rows after it
-        const int npro = min(nstage, c_end - c_begin);
+        // The first stage only (the others once it has landed: with every
+        // warp of the GPU asking at once, a single stage each reaches the
+        // warps sooner and the queue stays short).  With `early` its cached
+        // rows go before the wait on the previous launch, the query and
+        // appended row after it.
+        const int npro = 1;
         if (early) {
             for (int s = 0; s < npro; ++s) {
                 const ChunkDesc c = ChunkDesc::of(shfl_int4(head, s));
@@ -541,6 +544,8 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
                 break;
             }
             phase ^= 1u << stage;
+            if (k == 0)  // the first chunk has landed: fill the other stages
+                for (int s2 = 1; s2 < nstage && ip < c_end; ++s2) issue(s2);
             const int n = c.n;
             const unsigned char* kst = my + (size_t)stage * STAGE;
             const unsigned char* vst = kst + ROW;  // V half of each row pair
