@@ -525,7 +525,9 @@ def main():
         sample = f"whole (sequence, layer) units of {w.name} through the oracle, ~{per:.0f} s per step"
         print(json.dumps({
             "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+            "steps": args.steps, "warmup": args.warmup,
+            # a whole pass (every image token of the workload) at the sampled rate
+            "ms_per_step": 1e3 * w.images * w.decode_steps / val,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": config,
             "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle",
