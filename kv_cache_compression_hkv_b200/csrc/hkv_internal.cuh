@@ -16,7 +16,7 @@ constexpr int CHUNK = 32;  // tokens one warp handles per decode work item
 constexpr int PLAN_MAX_WARPS = 2048;  // capacity of a decode plan's warp table
 constexpr int PLAN_WARP_DESC = 7;     // descriptors copied into each warp's plan block
 constexpr int PLAN_DESC_PARTS = 4;    // blocks per layer of the plan kernel
-constexpr int RANK_MAX = 256;         // strata up to this size are selected by ranking
+constexpr int RANK_MAX = 32;          // strata up to this size are selected by ranking
 
 // Everything a kernel needs to find the state of a (layer, sequence, head).
 // The pool is one caller-owned device buffer carved into these regions.
@@ -281,6 +281,123 @@ __device__ inline void warp_rank_evict(const uint64_t* keys, const uint16_t* slo
     }
 }
 
+// Thresholds of two strata at once, with each lane's keys in registers
+// (stratum a: keys l, l + 32, ... of a set of ma; likewise b), for 1 <= k < m
+// in each active stratum: a 4-ary search on the score bits (three pivots
+// per round, counts by warp reductions), then the position tie at the
+// boundary.  Every key <= the returned threshold is evicted.  Lanes hold
+// ~0 for absent keys (scores are >= +0, so their bits stay below 2^31).
+template <int U>
+__device__ inline void warp_kth_regs2(const uint64_t (&ka)[U], int ka_k, bool a_on,
+                                      const uint64_t (&kb)[U], int kb_k, bool b_on,
+                                      uint64_t& thr_a, uint64_t& thr_b) {
+    uint32_t alo = 0xffffffffu, ahi = 0u, blo = 0xffffffffu, bhi = 0u;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const uint32_t sa = (uint32_t)(ka[u] >> 32), sb = (uint32_t)(kb[u] >> 32);
+        if (ka[u] != ~0ull) { alo = min(alo, sa); ahi = max(ahi, sa); }
+        if (kb[u] != ~0ull) { blo = min(blo, sb); bhi = max(bhi, sb); }
+    }
+    alo = __reduce_min_sync(FULL_MASK, alo);
+    ahi = __reduce_max_sync(FULL_MASK, ahi);
+    blo = __reduce_min_sync(FULL_MASK, blo);
+    bhi = __reduce_max_sync(FULL_MASK, bhi);
+    if (!a_on) alo = ahi = 0;
+    if (!b_on) blo = bhi = 0;
+    while (alo < ahi || blo < bhi) {
+        const uint32_t a1 = alo + ((ahi - alo) >> 2), a2 = alo + ((ahi - alo) >> 1),
+                       a3 = alo + (uint32_t)(((uint64_t)(ahi - alo) * 3) >> 2);
+        const uint32_t b1 = blo + ((bhi - blo) >> 2), b2 = blo + ((bhi - blo) >> 1),
+                       b3 = blo + (uint32_t)(((uint64_t)(bhi - blo) * 3) >> 2);
+        unsigned ca1 = 0, ca2 = 0, ca3 = 0, cb1 = 0, cb2 = 0, cb3 = 0;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint32_t sa = (uint32_t)(ka[u] >> 32), sb = (uint32_t)(kb[u] >> 32);
+            ca1 += sa <= a1; ca2 += sa <= a2; ca3 += sa <= a3;
+            cb1 += sb <= b1; cb2 += sb <= b2; cb3 += sb <= b3;
+        }
+        ca1 = __reduce_add_sync(FULL_MASK, ca1);
+        ca2 = __reduce_add_sync(FULL_MASK, ca2);
+        ca3 = __reduce_add_sync(FULL_MASK, ca3);
+        cb1 = __reduce_add_sync(FULL_MASK, cb1);
+        cb2 = __reduce_add_sync(FULL_MASK, cb2);
+        cb3 = __reduce_add_sync(FULL_MASK, cb3);
+        if (alo < ahi) {
+            if ((int)ca1 >= ka_k) ahi = a1;
+            else if ((int)ca2 >= ka_k) { alo = a1 + 1; ahi = a2; }
+            else if ((int)ca3 >= ka_k) { alo = a2 + 1; ahi = a3; }
+            else alo = a3 + 1;
+        }
+        if (blo < bhi) {
+            if ((int)cb1 >= kb_k) bhi = b1;
+            else if ((int)cb2 >= kb_k) { blo = b1 + 1; bhi = b2; }
+            else if ((int)cb3 >= kb_k) { blo = b2 + 1; bhi = b3; }
+            else blo = b3 + 1;
+        }
+    }
+    // the position tie at the boundary score s* of each stratum: need =
+    // k - (keys below s*) of the tied keys go, lowest positions first
+    auto finish = [&](const uint64_t (&kk)[U], int k, uint32_t sstar) -> uint64_t {
+        unsigned c_lt = 0, c_eq = 0;
+        uint32_t plo = 0xffffffffu, phi = 0u;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint32_t sc = (uint32_t)(kk[u] >> 32), p = (uint32_t)kk[u];
+            if (kk[u] == ~0ull) continue;
+            c_lt += sc < sstar;
+            if (sc == sstar) { ++c_eq; plo = min(plo, p); phi = max(phi, p); }
+        }
+        c_lt = __reduce_add_sync(FULL_MASK, c_lt);
+        c_eq = __reduce_add_sync(FULL_MASK, c_eq);
+        plo = __reduce_min_sync(FULL_MASK, plo);
+        phi = __reduce_max_sync(FULL_MASK, phi);
+        const int need = k - (int)c_lt;  // 1 <= need <= c_eq
+        if (need < (int)c_eq) {
+            while (plo < phi) {
+                const uint32_t mid = plo + ((phi - plo) >> 1);
+                unsigned c = 0;
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    c += kk[u] != ~0ull && (uint32_t)(kk[u] >> 32) == sstar && (uint32_t)kk[u] <= mid;
+                c = __reduce_add_sync(FULL_MASK, c);
+                if ((int)c >= need) phi = mid; else plo = mid + 1;
+            }
+        } else {
+            plo = phi;  // every tied key goes
+        }
+        return ((uint64_t)sstar << 32) | plo;
+    };
+    thr_a = a_on ? finish(ka, ka_k, alo) : 0ull;
+    thr_b = b_on ? finish(kb, kb_k, blo) : 0ull;
+}
+
+// Both strata (at most 32 * U keys each) selected by warp_kth_regs2: keys
+// read once into registers, evict bits set from the thresholds.
+template <int U>
+__device__ inline void warp_select_regs(const uint64_t* keys_a, const uint16_t* slots_a, int ma, int ka_k,
+                                        const uint64_t* keys_b, const uint16_t* slots_b, int mb, int kb_k,
+                                        uint32_t* evict_bits) {
+    const int lane = threadIdx.x & 31;
+    uint64_t ka[U], kb[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int i = lane + 32 * u;
+        ka[u] = i < ma ? keys_a[i] : ~0ull;
+        kb[u] = i < mb ? keys_b[i] : ~0ull;
+    }
+    const bool a_on = ka_k > 0 && ka_k < ma, b_on = kb_k > 0 && kb_k < mb;
+    uint64_t ta = 0, tb = 0;
+    warp_kth_regs2<U>(ka, ka_k, a_on, kb, kb_k, b_on, ta, tb);
+    if (ka_k >= ma) ta = ~0ull;  // the whole stratum goes
+    if (kb_k >= mb) tb = ~0ull;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int i = lane + 32 * u;
+        if (i < ma && ka_k > 0 && ka[u] <= ta) atomicOr(&evict_bits[slots_a[i] >> 5], 1u << (slots_a[i] & 31));
+        if (i < mb && kb_k > 0 && kb[u] <= tb) atomicOr(&evict_bits[slots_b[i] >> 5], 1u << (slots_b[i] & 31));
+    }
+}
+
 // Scratch of one warp's stratified select over up to n_max tokens.  The
 // near keys fill keys[] from the front and the far keys from the back; the
 // same for slot[] and for the hole / mover lists of the compaction.
@@ -385,10 +502,22 @@ __device__ inline int warp_select_partitioned(const SelectScratch& sc, int n, in
         kn = 0;
         if (kf > nf) kf = nf;
     }
-    // Strata of at most RANK_MAX keys: rank every key against all keys of
-    // its stratum (keys are distinct, so rank < k is exactly the k lowest).
-    // Larger strata: threshold by the radix select; none evicted (k <= 0),
-    // all evicted (k >= m).
+    // Both strata of at most 256 keys, one of them over RANK_MAX: keys in
+    // registers, thresholds by a joint 4-ary search.
+    const int mm = max(nn, nf);
+    if (mm > RANK_MAX && mm <= 256) {
+        const uint64_t* kf_keys = sc.keys + (n - nf);
+        const uint16_t* kf_slots = sc.slot + (n - nf);
+        if (mm <= 64) warp_select_regs<2>(sc.keys, sc.slot, nn, kn, kf_keys, kf_slots, nf, kf, sc.evict_bits);
+        else if (mm <= 128) warp_select_regs<4>(sc.keys, sc.slot, nn, kn, kf_keys, kf_slots, nf, kf, sc.evict_bits);
+        else warp_select_regs<8>(sc.keys, sc.slot, nn, kn, kf_keys, kf_slots, nf, kf, sc.evict_bits);
+        __syncwarp();
+        return kn + kf;
+    }
+    // Otherwise each stratum alone: at most RANK_MAX keys by ranking every
+    // key against all keys of its stratum (keys are distinct, so rank < k is
+    // exactly the k lowest); larger by the radix select; none evicted
+    // (k <= 0), all evicted (k >= m).
     for (int which = 0; which < 2; ++which) {
         const int k = which == 0 ? kn : kf;
         const int m = which == 0 ? nn : nf;
