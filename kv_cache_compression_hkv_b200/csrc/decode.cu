@@ -175,8 +175,10 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
     int32_t* hslot = psm + n;      // layer-relative row of the head's first token
     int32_t* hlen = psm + 2 * n;   // len << 16 | appended slot
     int32_t* hscore = psm + 3 * n; // scoring flag
-    int32_t* wbeg = psm + 4 * n;   // [GW + 1] first chunk of each warp's range
     const int GW = L.plan_gw;
+    int32_t* wbeg = psm + 4 * n;   // [GW + 1] first chunk of each warp's range
+    int32_t* whead = wbeg + PLAN_MAX_WARPS + 1;  // [GW] the head holding that chunk
+    uint16_t* own = reinterpret_cast<uint16_t*>(whead + PLAN_MAX_WARPS);  // [total] warp of each chunk
     const int parts = gridDim.y, part = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, NW = blockDim.x >> 5;
     const int t = L.t_next[layer] - 1 + ahead;
@@ -234,63 +236,49 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
     // warps holding many short heads get fewer chunks.  Head i's cost ends
     // at CHUNK_COST * cnt[i] + i + 1; warp w's range starts at the first
     // chunk whose cost starts at or after w * cost / GW.
+    // Head i's cost interval is [E(i-1), E(i)), E(i) = CHUNK_COST * cnt[i] +
+    // i + 1; the warps w whose boundary w * cost / GW falls in it start in
+    // head i, at the first of its chunks whose cost starts at or after the
+    // boundary.  (Every warp start found by arithmetic, no search.)
     const int64_t tcost = (int64_t)CHUNK_COST * total + n;
-    const bool narrow = tcost * GW < ((int64_t)1 << 31);  // 32-bit arithmetic suffices
-    // first chunk of warp w's range by cost; *head: the head holding it
-    auto begin_of = [&](int w, int* head) -> int {
-        if (w >= GW) { *head = n; return total; }
-        const int64_t b = narrow ? (int64_t)((uint32_t)w * (uint32_t)tcost / (uint32_t)GW)
-                                 : (int64_t)w * tcost / GW;
-        int lo = 0, hi = n;  // first head whose cost ends after b
-        if (narrow) {
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if (CHUNK_COST * cnt[mid] + mid + 1 > (int)b) hi = mid; else lo = mid + 1;
-            }
-        } else {
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if ((int64_t)CHUNK_COST * cnt[mid] + mid + 1 > b) hi = mid; else lo = mid + 1;
-            }
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int c0 = i ? cnt[i - 1] : 0, c1 = cnt[i];
+        const int64_t e0 = i ? (int64_t)CHUNK_COST * c0 + i : 0;
+        const int64_t e1 = (int64_t)CHUNK_COST * c1 + i + 1;
+        const int w_lo = (int)((e0 * GW + tcost - 1) / tcost);
+        const int w_hi = min((int)((e1 * GW + tcost - 1) / tcost), GW);  // exclusive
+        for (int w = w_lo; w < w_hi; ++w) {
+            const int64_t bnd = (int64_t)w * tcost / GW;
+            const int k = (int)((bnd - e0 + CHUNK_COST - 1) / CHUNK_COST);
+            wbeg[w] = c0 + min(max(k, 0), c1 - c0);
+            whead[w] = i;
         }
-        *head = lo;
-        if (lo >= n) return total;
-        const int c0 = lo ? cnt[lo - 1] : 0;
-        const int64_t base = lo ? (int64_t)CHUNK_COST * c0 + lo : 0;
-        const int k = (int)((b - base + CHUNK_COST - 1) / CHUNK_COST);
-        return c0 + min(max(k, 0), cnt[lo] - c0);
-    };
+    }
+    if (threadIdx.x == 0) wbeg[GW] = total;
+    __syncthreads();
     // A range starting a decode block moves to the nearer end of the head
     // it would cut (at most SNAP_MAX chunks, staying between its neighbours'
     // starts), so that heads seldom span two blocks and their split
-    // segments meet in shared memory.
+    // segments meet in shared memory.  Neighbours of a block start are not
+    // block starts, so the entries read here are not being written.
     const int NWB = L.plan_nw;
-    for (int w = threadIdx.x; w <= GW; w += blockDim.x) {
-        int lo;
-        int c = begin_of(w, &lo);
-        if (w > 0 && w < GW && NWB > 1 && w % NWB == 0 && lo < n) {
+    if (NWB > 1)
+        for (int w = NWB * (threadIdx.x + 1); w < GW; w += NWB * blockDim.x) {
+            const int lo = whead[w], c = wbeg[w];
             const int c0 = lo ? cnt[lo - 1] : 0, c1 = cnt[lo];
             if (c > c0 && c < c1) {
-                int dummy;
-                const int prev = begin_of(w - 1, &dummy), next = begin_of(w + 1, &dummy);
+                const int prev = wbeg[w - 1], next = wbeg[w + 1];
                 const int down = c - c0, up = c1 - c;
-                if (down <= up && down <= SNAP_MAX && c0 >= prev) c = c0;
-                else if (up <= SNAP_MAX && c1 <= next) c = c1;
-                else if (down <= SNAP_MAX && c0 >= prev) c = c0;
+                if (down <= up && down <= SNAP_MAX && c0 >= prev) wbeg[w] = c0;
+                else if (up <= SNAP_MAX && c1 <= next) wbeg[w] = c1;
+                else if (down <= SNAP_MAX && c0 >= prev) wbeg[w] = c0;
             }
         }
-        wbeg[w] = c;
-    }
     __syncthreads();
-    // the warp whose range holds chunk c (the last w with wbeg[w] <= c)
-    auto owner = [&](int c) -> int {
-        int lo = 0, hi = GW - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (wbeg[mid] <= c) lo = mid; else hi = mid - 1;
-        }
-        return lo;
-    };
+    // the warp whose range holds each chunk
+    for (int w = threadIdx.x; w < GW; w += blockDim.x)
+        for (int c = wbeg[w]; c < wbeg[w + 1]; ++c) own[c] = (uint16_t)w;
+    __syncthreads();
     constexpr int PB = 1 + PLAN_WARP_DESC;
     int4* dsc = L.plan_desc + (size_t)layer * L.max_chunks;
     int4* pw = L.plan_warp + (size_t)layer * PLAN_MAX_WARPS * PB;
@@ -299,7 +287,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
         const int c1 = cnt[i], c0 = i ? cnt[i - 1] : 0;
         if (c1 == c0) continue;
         const int4 f = make_int4(hslot[i], hlen[i], hscore[i], 0);
-        const int wa = owner(c0), wb = owner(c1 - 1);
+        const int wa = own[c0], wb = own[c1 - 1];
         int segs = 0;
         for (int w = wa; w <= wb; ++w) segs += wbeg[w] < wbeg[w + 1];
         const int hw = wa | ((wb - wa) << 12);
@@ -884,7 +872,8 @@ cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void*
 }
 
 cudaError_t launch_plan(const Layout& L, int l0, int l1, int ahead, cudaStream_t st) {
-    plan_kernel<<<dim3(l1 - l0, PLAN_DESC_PARTS), 1024, plan_smem_bytes(L.S * L.H), st>>>(L, l0, ahead);
+    plan_kernel<<<dim3(l1 - l0, PLAN_DESC_PARTS), 1024, plan_smem_bytes(L.S * L.H, L.max_chunks), st>>>(
+        L, l0, ahead);
     return cudaGetLastError();
 }
 

@@ -216,7 +216,7 @@ hkv_status hkv_create(const hkv_config* cfg, void* pool, size_t bytes, void* str
     }
     int optin = 0;
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, c->device);
-    if (hkv::plan_smem_bytes(cfg->num_seqs * cfg->num_heads) > (size_t)optin - 1024) {
+    if (hkv::plan_smem_bytes(cfg->num_seqs * cfg->num_heads, c->lay.max_chunks) > (size_t)optin - 1024) {
         delete c;
         return HKV_ERR_INVALID_ARG;  // too many heads per layer for one plan block
     }

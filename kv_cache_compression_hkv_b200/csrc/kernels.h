@@ -35,10 +35,10 @@ cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void*
                           void* o, int append, const DecodeShape& sh, int grid, int early, int buf,
                           cudaStream_t st);
 cudaError_t launch_plan(const Layout& L, int l0, int l1, int ahead, cudaStream_t st);
-// Shared memory of the plan kernel: four words per head of a layer and one
-// per warp of the decode grid (and one more).
-inline size_t plan_smem_bytes(int heads_per_layer) {
-    return (size_t)heads_per_layer * 16 + (PLAN_MAX_WARPS + 1) * 4;
+// Shared memory of the plan kernel: four words per head of a layer, two per
+// warp of the decode grid (and one more), two bytes per chunk.
+inline size_t plan_smem_bytes(int heads_per_layer, int max_chunks) {
+    return (size_t)heads_per_layer * 16 + (2 * PLAN_MAX_WARPS + 1) * 4 + ((size_t)max_chunks * 2 + 15) / 16 * 16;
 }
 cudaError_t launch_prefill_rows_simt(int dtype, int d, int n_blocks, const void* q, const void* k,
                                      const void* v, int P, int64_t block_stride, int r, void* out,
