@@ -474,12 +474,13 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
         if (lane >= PLAN_WARP_DESC)
             pwin = c_begin + lane < c_end ? dsc[c_begin + lane] : make_int4(0, 0, 0, 0);
         int4 cwin = pwin;
-        // The first stage only (the others once it has landed: with every
-        // warp of the GPU asking at once, a single stage each reaches the
-        // warps sooner and the queue stays short).  With `early` its cached
-        // rows go before the wait on the previous launch, the query and
-        // appended row after it.
-        const int npro = 1;
+        // With many warps per SM the first stage only (the others once it
+        // has landed: with every warp of the GPU asking at once, a single
+        // stage each reaches the warps sooner and the queue stays short);
+        // with few, every stage (fewer bytes would be in flight otherwise).
+        // With `early` their cached rows go before the wait on the previous
+        // launch, queries and appended rows after it.
+        const int npro = NW >= 8 ? 1 : min(nstage, c_end - c_begin);
         if (early) {
             for (int s = 0; s < npro; ++s) {
                 const ChunkDesc c = ChunkDesc::of(shfl_int4(head, s));
@@ -532,7 +533,7 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
                 break;
             }
             phase ^= 1u << stage;
-            if (k == 0)  // the first chunk has landed: fill the other stages
+            if (k == 0 && npro == 1)  // the first chunk has landed: fill the other stages
                 for (int s2 = 1; s2 < nstage && ip < c_end; ++s2) issue(s2);
             const int n = c.n;
             const unsigned char* kst = my + (size_t)stage * STAGE;
