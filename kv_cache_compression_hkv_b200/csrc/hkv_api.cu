@@ -126,7 +126,6 @@ size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Lay
     l.base_t = (int32_t*)take(nh * 4);
     l.n_tau = (int32_t*)take(nh * 4);
     l.label = (uint8_t*)take(nh);
-    l.due_t = (int32_t*)take(Ly * S * 4);
     l.K = take(slots * 2 * d * es);  // K and V rows interleaved per slot
     l.V = l.K ? (unsigned char*)l.K + d * es : nullptr;
     l.pos = (int32_t*)take(slots * 4);

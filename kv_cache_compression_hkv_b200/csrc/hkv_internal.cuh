@@ -39,7 +39,6 @@ struct Layout {
     uint8_t* label;     // 1 Local, 0 Global, 2 full cache
     int32_t* n_tau;
     // per (layer, sequence): step at which its Global heads reach their cap
-    int32_t* due_t;
     // cache rows, slot index (l*S + s)*R + slot
     void* K;            // [Ly][S][R][2][d]: per slot its K row, then its V row
     void* V;            // K + d elements (same row stride 2 d)

@@ -130,9 +130,6 @@ __global__ void classify_kernel(Layout L, int layer, int P) {
         o += cap;
     }
     if (o > L.R) latch_error(L, HKV_ERR_CAPACITY, layer * L.S + s);
-    const int g0 = P < bg ? P : bg;
-    L.due_t[(size_t)layer * L.S + s] =
-        (ng > 0 && L.mode != HKV_MODE_FULL) ? (P - 1) + (bg + L.M - g0) : 0x7fffffff;
     if (s == 0) L.t_next[layer] = P;
 }
 
