@@ -137,11 +137,13 @@ template <int DPL> struct RowSlice<__nv_bfloat16, DPL> {
 //
 // keys[i] = (bits(score) << 32) | position, score >= +0 so the bit pattern
 // orders like the value; the total order is (score, position), i.e. equal
-// scores evict the lower position first.  The k-th smallest key of a set is
-// found by an MSB-first radix select on the score bits (four 8-bit digits,
-// a shared-memory histogram per digit), then, only when scores tie at the
-// boundary, by bisection on their positions.  Every key <= the returned
-// threshold is evicted.
+// scores evict the lower position first.  The k lowest keys of a stratum
+// are found by ranking (at most RANK_MAX keys), by a register-resident
+// 4-ary search on the score bits (at most 256 keys), or by an MSB-first
+// radix select on the score bits (four 8-bit digits, a shared-memory
+// histogram per digit); the two searches resolve a score tie at the
+// boundary by bisection on positions.  Every key <= the threshold found is
+// evicted.
 // ---------------------------------------------------------------------------
 struct KthSearch {
     const uint64_t* keys;
@@ -236,14 +238,16 @@ __device__ inline uint32_t warp_radix_kth_score(const uint64_t* keys, int m, int
     return prefix;
 }
 
-// Marks the k lowest of m <= 32 * U distinct keys: lane l ranks keys
-// l, l + 32, ... (held in registers) against every key in one pass of
-// shared-memory broadcast reads; rank < k is exactly the k lowest.
+// 64-bit load from a shared-memory address.
 __device__ __forceinline__ uint64_t lds_u64(uint32_t addr) {
     uint64_t v;
     asm volatile("ld.shared.u64 %0, [%1];" : "=l"(v) : "r"(addr));
     return v;
 }
+
+// Marks the k lowest of m <= 32 * U distinct keys: lane l ranks keys
+// l, l + 32, ... (held in registers) against every key in one pass of
+// shared-memory broadcast reads; rank < k is exactly the k lowest.
 
 template <int U>
 __device__ inline void warp_rank_evict(const uint64_t* keys, const uint16_t* slots, int m, int k,
