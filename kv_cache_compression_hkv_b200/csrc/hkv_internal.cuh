@@ -93,45 +93,6 @@ __device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162f
 __device__ __forceinline__ void from_float(float& dst, float x) { dst = x; }
 __device__ __forceinline__ void from_float(__nv_bfloat16& dst, float x) { dst = __float2bfloat16_rn(x); }
 
-// Loads DPL consecutive elements starting at p (aligned to DPL elements) as floats.
-template <typename T, int DPL> struct RowSlice;
-template <int DPL> struct RowSlice<float, DPL> {
-    __device__ static __forceinline__ void load(const float* p, float (&x)[DPL]) {
-        if constexpr (DPL == 4) {
-            float4 v = *reinterpret_cast<const float4*>(p);
-            x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-        } else if constexpr (DPL == 2) {
-            float2 v = *reinterpret_cast<const float2*>(p);
-            x[0] = v.x; x[1] = v.y;
-        } else {
-#pragma unroll
-            for (int i = 0; i < DPL; ++i) x[i] = p[i];
-        }
-    }
-    __device__ static __forceinline__ void store(float* p, const float (&x)[DPL]) {
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) p[i] = x[i];
-    }
-};
-template <int DPL> struct RowSlice<__nv_bfloat16, DPL> {
-    __device__ static __forceinline__ void load(const __nv_bfloat16* p, float (&x)[DPL]) {
-        if constexpr (DPL == 4) {
-            uint2 v = *reinterpret_cast<const uint2*>(p);
-            x[0] = bf16_lo(v.x); x[1] = bf16_hi(v.x); x[2] = bf16_lo(v.y); x[3] = bf16_hi(v.y);
-        } else if constexpr (DPL == 2) {
-            uint32_t v = *reinterpret_cast<const uint32_t*>(p);
-            x[0] = bf16_lo(v); x[1] = bf16_hi(v);
-        } else {
-#pragma unroll
-            for (int i = 0; i < DPL; ++i) x[i] = __bfloat162float(p[i]);
-        }
-    }
-    __device__ static __forceinline__ void store(__nv_bfloat16* p, const float (&x)[DPL]) {
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) p[i] = __float2bfloat16_rn(x[i]);
-    }
-};
-
 // ---------------------------------------------------------------------------
 // Warp-level bottom-k selection (Stratified Token Eviction).
 //
