@@ -45,6 +45,10 @@ def parse_args():
     ap.add_argument("--no-full", action="store_true", help="skip the full-cache comparator")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end arm")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--mode", default="headkv", choices=["headkv", "uniform"],
+                    help="uniform: the same per-head budget for every head (a comparator)")
+    ap.add_argument("--unstratified", action="store_true",
+                    help="eviction over one pool instead of near/far strata (a comparator)")
     ap.add_argument("--profile", action="store_true",
                     help="eager run of a reduced workload for ncu captures (no timing line)")
     ap.add_argument("--seqs", type=int, default=None, help="override the workload's sequences")
@@ -253,7 +257,8 @@ def gpu_arm(args, rank, world, dev):
     inp = Inputs(w, dist.rank_seed(args.seed, rank), dev)
     outs = [torch.empty(S, H, d, dtype=w.torch_dtype, device=dev) for _ in range(Ly)]
     pre_out = [torch.empty(S, H, w.prefill_len, d, dtype=w.torch_dtype, device=dev) for _ in range(Ly)]
-    cfg = hkv.config_for(w)
+    cfg = hkv.config_for(w, mode=hkv.MODE_UNIFORM if args.mode == "uniform" else hkv.MODE_HEADKV,
+                         stratified=not args.unstratified)
     cache = hkv.HeadKVCache(cfg, device=dev)
 
     # one eager pass: warms every kernel and yields the bytes each decode launch reads
@@ -509,6 +514,9 @@ def main():
               "max_len": w.max_len, "prefill_len": w.prefill_len, "decode_steps": w.decode_steps,
               "rho": f"{w.rho[0]}/{w.rho[1]}", "local_window": w.local_window, "ste_m": w.ste_m,
               "near_dist": w.near_dist, "l2": "inputs and cache larger than L2 (no flush needed)"}
+    if args.mode != "headkv" or args.unstratified:
+        config["budgets"] = args.mode
+        config["strata"] = "pooled" if args.unstratified else "near/far"
 
     if args.impl == "reference":
         # the reference arm is the CPU oracle, on rank 0 only
