@@ -110,6 +110,24 @@ int hkvo_classify(const double* p_row, int32_t n, int32_t W, double tau,
     return 0;
 }
 
+int hkvo_class_row(const double* qh, const double* kh, const double* vh,
+                   int32_t P, int32_t d, int32_t nq, double* row)
+{
+    if (!qh || !kh || !vh || !row || P <= 0 || d <= 0 || nq < 1 || nq > P) return -1;
+    double* w = (double*)malloc(sizeof(double) * (size_t)P);
+    for (int32_t j = 0; j < P; ++j) row[j] = 0.0;
+    for (int32_t i = P - nq; i < P; ++i) {
+        /* weights of the query at position i over positions 0..i */
+        hkvo_causal_attention(qh + (size_t)i * d, kh, vh, 1, P, d, i, NULL, w);
+        /* its weight at distance delta lands where the last query's row
+         * holds distance delta */
+        for (int32_t delta = 0; delta <= i; ++delta) row[P - 1 - delta] += w[i - delta];
+    }
+    for (int32_t j = 0; j < P; ++j) row[j] /= (double)nq;
+    free(w);
+    return 0;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Budgets [Contrib/Budgets]                                                */
 /* ------------------------------------------------------------------------ */
@@ -316,9 +334,12 @@ int hkvo_run_unit(const hkvo_unit_params* prm, const double* q,
     out->n_events = 0;
     out->first_hard_step = -1;
 
+    const int32_t nq = prm->cls_queries;
+    if (nq < 1 || nq > r) return -1;
+
     /* Step 1, cache prefilling [Method/Prefill]: uncompressed causal attention
-     * over the first P tokens; the weights of the last query are kept for
-     * classification. */
+     * over the first P tokens; the weights of the last query (the last nq
+     * queries, averaged by distance) are kept for classification. */
     double* prow = (double*)malloc(sizeof(double) * (size_t)P);
     for (int32_t h = 0; h < H; ++h) {
         const double* qh = q + h * HL;
@@ -329,11 +350,11 @@ int hkvo_run_unit(const hkvo_unit_params* prm, const double* q,
             hkvo_causal_attention(qh, kh, vh, P, P, d, 0,
                                   out->o_prefill + (size_t)h * P * d, NULL);
         }
-        /* weights of the query at position P-1 over positions 0..P-1 */
-        hkvo_causal_attention(qh + (size_t)(P - 1) * d, kh, vh, 1, P, d, P - 1,
-                              NULL, prow);
+        const double* crow = prow;
+        if (prm->cls_rows) crow = prm->cls_rows + (size_t)h * P;
+        else hkvo_class_row(qh, kh, vh, P, d, nq, prow);
         /* Step 2, head grouping [Method/Grouping], once, at this length. */
-        hkvo_classify(prow, P, W, prm->tau, &out->n_tau[h], &out->labels[h],
+        hkvo_classify(crow, P, W, prm->tau, &out->n_tau[h], &out->labels[h],
                       &out->c_window[h]);
         if (prm->mode == HKVO_MODE_FULL) out->labels[h] = 2;
         if (prm->mode == HKVO_MODE_UNIFORM) out->labels[h] = 0;

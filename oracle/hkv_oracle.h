@@ -50,6 +50,16 @@ int hkvo_causal_attention(const double* q, const double* k, const double* v,
 int hkvo_classify(const double* p_row, int32_t n, int32_t W, double tau,
                   int32_t* n_tau, uint8_t* label, double* c_window);
 
+/* Classification row of one head from its last nq prefill queries
+ * [Method/Grouping], the distance-averaged variant of the grouping rule.
+ * The query at position i puts weight w_i(j) on position j <= i; its weight
+ * at distance delta is w_i(i - delta) (0 when delta > i).  The row is the
+ * mean over i = P-nq .. P-1 of those per-distance weights, written in the
+ * position order hkvo_classify reads: row[P-1-delta].  nq = 1 gives the last
+ * query's own weights.  qh, kh, vh: [>= P][d] rows of one head; row: [P]. */
+int hkvo_class_row(const double* qh, const double* kh, const double* vh,
+                   int32_t P, int32_t d, int32_t nq, double* row);
+
 /* Asymmetric budgets [Contrib/Budgets]: total T = floor(H * L * rho_num /
  * rho_den) tokens per (sequence, layer); Local heads keep W, the Global heads
  * split the rest evenly, rounded down.  budget_g = 0 when there is no Global
@@ -90,10 +100,16 @@ typedef struct {
     int32_t rho_num, rho_den;
     int32_t mode;        /* HKVO_MODE_* */
     int32_t stratified;  /* 1: near/far strata (STE); 0: one pool */
+    int32_t cls_queries; /* prefill queries whose per-distance weights are
+                            averaged for grouping (1: the last one alone) */
     double tau;
     double label_band;   /* |c_window - tau| <= band: either label is valid */
     double select_band;  /* boundary scores within this relative gap: either
                             order is valid */
+    const double* cls_rows; /* [H][P] classification rows to group by instead
+                               of the unit's own (labels tied across a CFG
+                               pair: the mean of both sequences' rows), or
+                               NULL */
 } hkvo_unit_params;
 
 /* Decisions another implementation took for the same unit.  When the

@@ -36,8 +36,10 @@ def build(force: bool = False) -> str:
 class _UnitParams(C.Structure):
     _fields_ = [(n, C.c_int32) for n in (
         "num_heads", "head_dim", "max_len", "prefill_len", "local_window", "ste_m",
-        "near_dist", "score_window", "rho_num", "rho_den", "mode", "stratified")] + [
-        ("tau", C.c_double), ("label_band", C.c_double), ("select_band", C.c_double)]
+        "near_dist", "score_window", "rho_num", "rho_den", "mode", "stratified",
+        "cls_queries")] + [
+        ("tau", C.c_double), ("label_band", C.c_double), ("select_band", C.c_double),
+        ("cls_rows", C.c_void_p)]
 
 
 class _Hints(C.Structure):
@@ -66,11 +68,12 @@ def lib():
         P, I, D = C.c_void_p, C.c_int32, C.c_double
         _lib.hkvo_causal_attention.argtypes = [P, P, P, I, I, I, I, P, P]
         _lib.hkvo_classify.argtypes = [P, I, I, D, P, P, P]
+        _lib.hkvo_class_row.argtypes = [P, P, P, I, I, I, P]
         _lib.hkvo_budgets.argtypes = [P, I, I, I, I, I, P, P, P]
         _lib.hkvo_ste_select.argtypes = [P, P, I, I, I, I, I, I, P, P, P]
         _lib.hkvo_ste_scores.argtypes = [P, P, I, P, I, I, I, P]
         _lib.hkvo_run_unit.argtypes = [P, P, P, P, P, P]
-        for f in ("hkvo_causal_attention", "hkvo_classify", "hkvo_budgets",
+        for f in ("hkvo_causal_attention", "hkvo_classify", "hkvo_class_row", "hkvo_budgets",
                   "hkvo_ste_select", "hkvo_ste_scores", "hkvo_run_unit"):
             getattr(_lib, f).restype = C.c_int
     return _lib
@@ -116,6 +119,17 @@ def classify(p_row, W: int, tau: float = 0.9):
     return nt.value, lab.value, cw.value
 
 
+def class_row(q, k, v, nq: int = 1):
+    """Classification row [P] of one head from its last nq queries (mean of
+    the per-distance weights, in the last query's position order).
+    q, k, v: [P, d]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    P, d = q.shape
+    row = np.zeros(P)
+    _check(lib().hkvo_class_row(_p(q), _p(k), _p(v), P, d, nq, _p(row)), "class_row")
+    return row
+
+
 def budgets(labels, L: int, W: int, rho_num: int, rho_den: int):
     """(n_local, budget_g, total) or ValueError when T < H * W."""
     labels = np.ascontiguousarray(np.asarray(labels, dtype=np.uint8))
@@ -158,6 +172,7 @@ class UnitParams:
     rho_den: int = 4
     mode: int = MODE_HEADKV
     stratified: bool = True
+    cls_queries: int = 1
     tau: float = 0.9
     label_band: float = 0.0
     select_band: float = 0.0
@@ -181,8 +196,11 @@ class UnitResult:
 
 def run_unit(prm: UnitParams, q, k, v, hints: dict | None = None,
              want_prefill: bool = False, want_decode: bool = True,
-             max_events: int | None = None) -> UnitResult:
+             max_events: int | None = None, cls_rows=None) -> UnitResult:
     """Run one (sequence, layer) unit.  q, k, v: [H, L, d].
+
+    cls_rows (optional): [H, P] classification rows to group by instead of
+    the unit's own (labels tied across a CFG pair).
 
     hints (optional): {"labels": uint8[H], "event_step": int32[E],
     "kept": int32[E, H, stride]} -- another implementation's decisions,
@@ -193,7 +211,13 @@ def run_unit(prm: UnitParams, q, k, v, hints: dict | None = None,
     P = prm.prefill_len
     cp = _UnitParams(H, d, L, P, prm.local_window, prm.ste_m, prm.near_dist,
                      prm.score_window, prm.rho_num, prm.rho_den, prm.mode,
-                     int(prm.stratified), prm.tau, prm.label_band, prm.select_band)
+                     int(prm.stratified), prm.cls_queries, prm.tau, prm.label_band,
+                     prm.select_band)
+    if cls_rows is not None:
+        cls_rows = _f64(cls_rows)
+        if cls_rows.shape != (H, P):
+            raise ValueError("cls_rows must be [H, P]")
+        cp.cls_rows = _p(cls_rows).value
     labels = np.zeros(H, np.uint8)
     n_tau = np.zeros(H, np.int32)
     cw = np.zeros(H)
@@ -236,3 +260,30 @@ def run_unit(prm: UnitParams, q, k, v, hints: dict | None = None,
         stats=dict(n_events=ne, n_label_ties=out.n_label_ties, n_label_hard=out.n_label_hard,
                    n_select=out.n_select, n_select_ties=out.n_select_ties,
                    n_select_hard=out.n_select_hard, first_hard_step=out.first_hard_step))
+
+
+CFG_UNTIED, CFG_HALVES, CFG_ADJACENT = 0, 1, 2
+
+
+def cfg_partner(s: int, num_seqs: int, pairing: int) -> int:
+    """The other sequence of s's classifier-free-guidance pair: the same
+    image's conditional and unconditional streams.  CFG_HALVES: the batch
+    is [conditional | unconditional], s pairs with s +- S/2; CFG_ADJACENT:
+    the two streams alternate, s pairs with s xor 1; CFG_UNTIED: s alone."""
+    if pairing == CFG_UNTIED:
+        return s
+    if num_seqs % 2:
+        raise ValueError("CFG pairs need an even number of sequences")
+    if pairing == CFG_HALVES:
+        half = num_seqs // 2
+        return s + half if s < half else s - half
+    if pairing == CFG_ADJACENT:
+        return s ^ 1
+    raise ValueError(f"unknown CFG pairing {pairing}")
+
+
+def tied_rows(rows_a, rows_b):
+    """Classification rows shared by a CFG pair: the plain mean of the two
+    sequences' rows, so that both streams of an image get one label per
+    (layer, head) and hence the same budgets."""
+    return 0.5 * (_f64(rows_a) + _f64(rows_b))

@@ -384,3 +384,120 @@ def test_hints_adopt_only_near_ties():
     lab[far] ^= 1
     res = O.run_unit(prm, q, k, v, hints={"labels": lab})
     assert res.stats["n_label_hard"] == 1
+
+
+# --------------------------------------------------------------------------
+# classifier variants: distance-averaged rows, CFG-tied rows
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("P,nq", [(9, 1), (9, 4), (30, 8), (97, 8), (12, 12)])
+def test_class_row_uniform_closed_form(P, nq):
+    """q = 0: query i spreads 1/(i+1) over positions 0..i, so the weight at
+    distance delta averaged over i = P-nq..P-1 is
+    (H_P - H_max(delta, P-nq)) / nq with H_n the n-th harmonic number."""
+    d = 8
+    q = np.zeros((P, d)); k = rng.standard_normal((P, d)); v = rng.standard_normal((P, d))
+    row = O.class_row(q, k, v, nq)
+    harm = np.concatenate([[0.0], np.cumsum(1.0 / np.arange(1, P + 1))])
+    for delta in range(P):
+        expect = (harm[P] - harm[max(delta, P - nq)]) / nq
+        assert row[P - 1 - delta] == pytest.approx(expect, rel=1e-12, abs=1e-15), delta
+    assert row.sum() == pytest.approx(1.0, abs=1e-12)
+
+
+def test_class_row_aligns_by_distance():
+    """Every query aimed at one fixed position j0 puts its weight at a
+    different distance; the averaged row holds 1/nq at each distance
+    i - j0, i = P-nq..P-1.  The last query alone holds it all at P-1-j0."""
+    P, d, nq, j0 = 40, 16, 8, 10
+    k = 0.01 * rng.standard_normal((P, d))
+    e = np.zeros(d); e[3] = 1.0
+    k[j0] = e * 40.0
+    q = np.tile(e * 40.0, (P, 1))
+    v = rng.standard_normal((P, d))
+    row = O.class_row(q, k, v, nq)
+    for i in range(P - nq, P):
+        assert row[P - 1 - (i - j0)] == pytest.approx(1.0 / nq, abs=1e-9)
+    one = O.class_row(q, k, v, 1)
+    assert one[j0] == pytest.approx(1.0, abs=1e-9)
+    # grouping follows: the neighbour-aimed head stays Local under averaging
+    W = 28
+    kk = rng.standard_normal((P, d))
+    qq = np.zeros((P, d))
+    for i in range(1, P):
+        qq[i] = 60.0 * math.sqrt(d) * kk[i - 1] / np.linalg.norm(kk[i - 1])
+    for n in (1, nq):
+        assert O.classify(O.class_row(qq, kk, kk, n), W=W, tau=0.9)[:2] == (2, 1)
+
+
+def test_class_row_one_query_is_last_weight_row():
+    P, d = 33, 16
+    q, k, v = (rng.standard_normal((P, d)) for _ in range(3))
+    _, p = O.causal_attention(q[P - 1:], k, v, q_pos0=P - 1)
+    np.testing.assert_array_equal(O.class_row(q, k, v, 1), p[0])
+
+
+def test_cfg_partner_pairs():
+    for S in (2, 4, 64):
+        for pairing in (O.CFG_HALVES, O.CFG_ADJACENT):
+            part = [O.cfg_partner(s, S, pairing) for s in range(S)]
+            assert sorted(part) == list(range(S))
+            assert all(part[p] == s and p != s for s, p in enumerate(part))
+        assert [O.cfg_partner(s, S, O.CFG_HALVES) for s in range(S)][: S // 2] == \
+            list(range(S // 2, S))
+        assert all(O.cfg_partner(s, S, O.CFG_UNTIED) == s for s in range(S))
+    with pytest.raises(ValueError):
+        O.cfg_partner(0, 3, O.CFG_HALVES)
+
+
+def test_tied_rows_decide_one_label_for_the_pair():
+    """Two rows whose own windows hold 0.95 and 0.80 of the mass: alone one
+    is Local and one Global; tied (mean 0.875 < 0.9) both are Global."""
+    P, W = 20, 5
+
+    def row_with(c_window):
+        r = np.zeros(P)
+        r[P - (W - 1):] = c_window / (W - 1)   # the W-1 newest tokens
+        r[: P - (W - 1)] = (1 - c_window) / (P - (W - 1))
+        return r
+
+    a, b = row_with(0.95), row_with(0.80)
+    assert O.classify(a, W, 0.9)[1] == 1 and O.classify(b, W, 0.9)[1] == 0
+    t = O.tied_rows(a, b)
+    assert O.classify(t, W, 0.9)[1] == 0
+    assert O.classify(t, W, 0.9)[2] == pytest.approx(0.875, abs=1e-12)
+    np.testing.assert_array_equal(O.tied_rows(a, b), O.tied_rows(b, a))
+
+
+def test_unit_classifier_variants():
+    """cls_queries = r runs the whole unit with both labels present and the
+    budget invariants intact; a unit given its own one-query rows as
+    cls_rows reproduces the default run exactly; a unit given a tied row
+    takes its labels from that row."""
+    prm, q, k, v = _small_unit(seed=5)
+    base = O.run_unit(prm, q, k, v)
+    H, P = prm.num_heads, prm.prefill_len
+    own = np.stack([O.class_row(q[h, :P], k[h, :P], v[h, :P], 1) for h in range(H)])
+    same = O.run_unit(prm, q, k, v, cls_rows=own)
+    np.testing.assert_array_equal(same.labels, base.labels)
+    np.testing.assert_array_equal(same.o_decode, base.o_decode)
+    prm_r = O.UnitParams(**{**prm.__dict__, "cls_queries": prm.score_window})
+    res_r = O.run_unit(prm_r, q, k, v)
+    avg = np.stack([O.class_row(q[h, :P], k[h, :P], v[h, :P], prm.score_window)
+                    for h in range(H)])
+    for h in range(H):
+        assert res_r.labels[h] == O.classify(avg[h], prm.local_window, 0.9)[1]
+    nl, bg, _ = O.budgets(res_r.labels, prm.max_len, prm.local_window, prm.rho_num, prm.rho_den)
+    assert res_r.n_local == nl and res_r.budget_g == bg
+    assert all(len(x) <= (bg + prm.ste_m if res_r.labels[h] == 0 else prm.local_window)
+               for h, x in enumerate(res_r.kept_final))
+    g = np.random.default_rng(3)
+    q2, k2 = q + 0.5 * g.standard_normal(q.shape), k + 0.5 * g.standard_normal(k.shape)
+    other = np.stack([O.class_row(q2[h, :P], k2[h, :P], v[h, :P], 1) for h in range(H)])
+    tied = O.tied_rows(own, other)
+    res_t = O.run_unit(prm, q, k, v, cls_rows=tied)
+    for h in range(H):
+        assert res_t.labels[h] == O.classify(tied[h], prm.local_window, 0.9)[1]
+    with pytest.raises(ValueError):
+        O.run_unit(O.UnitParams(**{**prm.__dict__, "cls_queries": prm.score_window + 1}),
+                   q, k, v)
