@@ -32,6 +32,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "compressed decode image tokens/s and step µs; achieved HBM GB/s vs B200 peak"
 UNIT = "image tokens/s"
+# which sequences form a classifier-free-guidance pair (values of hkv_cfg_pairing)
+PAIRINGS = {"untied": 0, "halves": 1, "adjacent": 2}
 
 
 def parse_args():
@@ -49,6 +51,10 @@ def parse_args():
                     help="uniform: the same per-head budget for every head (a comparator)")
     ap.add_argument("--unstratified", action="store_true",
                     help="eviction over one pool instead of near/far strata (a comparator)")
+    ap.add_argument("--cls-queries", type=int, default=1,
+                    help="group heads by the last n prefill queries' per-distance weights")
+    ap.add_argument("--cfg-pairing", default="untied", choices=list(PAIRINGS),
+                    help="group the two streams of a CFG pair by their mean row")
     ap.add_argument("--profile", action="store_true",
                     help="eager run of a reduced workload for ncu captures (no timing line)")
     ap.add_argument("--seqs", type=int, default=None, help="override the workload's sequences")
@@ -61,31 +67,51 @@ def parse_args():
 # CPU oracle timing (the reported CPU baseline and the reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(w, seed, seconds, threads=None):
+def oracle_sample(w, seed, seconds, threads=None, opts=None):
     """Runs whole (sequence, layer) units of the workload through the CPU
     oracle on host threads for about `seconds`; returns (image tokens/s,
-    threads, units done)."""
+    threads, units done).  opts: the variant flags (mode, stratified,
+    cls_queries, cfg_pairing)."""
     from concurrent.futures import ThreadPoolExecutor
 
     from kv_cache_compression_hkv_b200.inputs import generate_layer
     from oracle import hkv_oracle as O
 
     threads = threads or os.cpu_count() or 1
+    opts = opts or {}
+    pairing = opts.get("cfg_pairing", O.CFG_UNTIED)
+    nq = opts.get("cls_queries", 1)
     prm = O.UnitParams(num_heads=w.num_heads, head_dim=w.head_dim, max_len=w.max_len,
                        prefill_len=w.prefill_len, local_window=w.local_window, ste_m=w.ste_m,
                        near_dist=w.near_dist, score_window=w.score_window, rho_num=w.rho[0],
-                       rho_den=w.rho[1])
-    q, k, v = generate_layer(w, 0, seed, "cpu", num_seqs=min(w.num_seqs, threads))
-    units = [tuple(x[s].double().numpy() for x in (q, k, v)) for s in range(q.shape[0])]
+                       rho_den=w.rho[1], mode=opts.get("mode", O.MODE_HEADKV),
+                       stratified=opts.get("stratified", True), cls_queries=nq)
+    n_seq = min(w.num_seqs, threads)
+    if pairing != O.CFG_UNTIED:
+        n_seq = max(2, n_seq - n_seq % 2)
+    q, k, v = generate_layer(w, 0, seed, "cpu", num_seqs=n_seq)
+    units = [tuple(x[s].double().numpy() for x in (q, k, v)) for s in range(n_seq)]
     O.build()
     done = [0]
     deadline = time.perf_counter() + seconds
     lock = threading.Lock()
+    P = w.prefill_len
+
+    def rows(s):
+        qs, ks, vs = units[s]
+        return np.stack([O.class_row(qs[h, :P], ks[h, :P], vs[h, :P], nq)
+                         for h in range(w.num_heads)])
 
     def worker(i):
         n = 0
         while True:
-            O.run_unit(prm, *units[i % len(units)], want_decode=True)
+            s = i % len(units)
+            cls = None
+            if pairing != O.CFG_UNTIED:
+                # the sample pairs its own sequences: the same work as the
+                # true partner's row
+                cls = O.tied_rows(rows(s), rows(O.cfg_partner(s, n_seq, pairing)))
+            O.run_unit(prm, *units[s], want_decode=True, cls_rows=cls)
             n += 1
             if time.perf_counter() > deadline:
                 break
@@ -98,6 +124,24 @@ def oracle_sample(w, seed, seconds, threads=None):
     el = time.perf_counter() - t0
     tokens_per_unit = w.images * w.decode_steps / (w.num_seqs * w.num_layers)
     return done[0] * tokens_per_unit / el, threads, done[0], el
+
+
+def oracle_opts(args) -> dict:
+    """The variant flags as oracle unit parameters."""
+    return {"mode": 2 if args.mode == "uniform" else 0, "stratified": not args.unstratified,
+            "cls_queries": args.cls_queries, "cfg_pairing": PAIRINGS[args.cfg_pairing]}
+
+
+def planted_recovery(w, labels, seed) -> dict:
+    """How the computed labels ([layers, S, H], 1 = Local) meet the heads
+    the synthetic inputs planted Local: the share of planted Local heads
+    labelled Local, and of planted Global heads labelled Local."""
+    from kv_cache_compression_hkv_b200.inputs import planted_local_heads
+    planted = np.stack([planted_local_heads(w, l, seed).numpy() for l in range(w.num_layers)])
+    planted = np.broadcast_to(planted[:, None, :], labels.shape)
+    local = labels == 1
+    return {"local_as_local": float(local[planted].mean()) if planted.any() else None,
+            "global_as_local": float(local[~planted].mean()) if (~planted).any() else None}
 
 
 # ---------------------------------------------------------------------------
@@ -258,7 +302,8 @@ def gpu_arm(args, rank, world, dev):
     outs = [torch.empty(S, H, d, dtype=w.torch_dtype, device=dev) for _ in range(Ly)]
     pre_out = [torch.empty(S, H, w.prefill_len, d, dtype=w.torch_dtype, device=dev) for _ in range(Ly)]
     cfg = hkv.config_for(w, mode=hkv.MODE_UNIFORM if args.mode == "uniform" else hkv.MODE_HEADKV,
-                         stratified=not args.unstratified)
+                         stratified=not args.unstratified, cls_queries=args.cls_queries,
+                         cfg_pairing=PAIRINGS[args.cfg_pairing])
     cache = hkv.HeadKVCache(cfg, device=dev)
 
     # one eager pass: warms every kernel and yields the bytes each decode launch reads
@@ -347,6 +392,7 @@ def gpu_arm(args, rank, world, dev):
         "evict_us_avg": float(evict_us.mean()),
         "evict_us_max": float(evict_us.max()),
         "labels_local_frac": float((labels == 1).mean()),
+        "labels_planted": planted_recovery(w, labels, dist.rank_seed(args.seed, rank)),
         # per layer at prefill: attention, grouping, packing, plan; per
         # step: one decode launch per layer, eviction scan and run, plan
         "gpu_launches": args.steps * (4 * Ly + steps * (Ly + 3)),
@@ -517,6 +563,9 @@ def main():
     if args.mode != "headkv" or args.unstratified:
         config["budgets"] = args.mode
         config["strata"] = "pooled" if args.unstratified else "near/far"
+    if args.cls_queries != 1 or args.cfg_pairing != "untied":
+        config["grouping_queries"] = args.cls_queries
+        config["cfg_pairing"] = args.cfg_pairing
 
     if args.impl == "reference":
         # the reference arm is the CPU oracle, on rank 0 only
@@ -526,7 +575,8 @@ def main():
         cores = 0
         per = max(2.0, min(args.cpu_seconds, 20.0))
         for i in range(args.warmup + args.steps):
-            v, cores, n, el = oracle_sample(w, args.seed, per if i >= args.warmup else 1.0)
+            v, cores, n, el = oracle_sample(w, args.seed, per if i >= args.warmup else 1.0,
+                                            opts=oracle_opts(args))
             if i >= args.warmup:
                 vals.append(v)
         val = float(np.mean(vals))
@@ -556,7 +606,7 @@ def main():
     res = gpu_arm(args, rank, world, dev)
     cpu = None
     if rank == 0 and world == 1:
-        v, cores, n, el = oracle_sample(w, args.seed, args.cpu_seconds)
+        v, cores, n, el = oracle_sample(w, args.seed, args.cpu_seconds, opts=oracle_opts(args))
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{n} whole (sequence, layer) units of {w.name} in {el:.1f} s "
                          f"(one unit = 1/{w.num_seqs * w.num_layers} of a pass)"}
@@ -575,6 +625,7 @@ def main():
             "speedup_decode_vs_full": res.get("speedup_decode_vs_full"),
             "speedup_pass_vs_full": res.get("speedup_pass_vs_full"),
             "kv_pool_bytes": res["kv_pool_bytes"], "labels_local_frac": res["labels_local_frac"],
+            "labels_planted": res["labels_planted"],
         }
         print(json.dumps(line))
     if world > 1:

@@ -60,6 +60,14 @@ typedef enum {
     HKV_MODE_UNIFORM = 2  /* one uniform budget for every head, STE eviction */
 } hkv_mode;
 
+/* Which sequences form a classifier-free-guidance pair (the conditional and
+ * the unconditional stream of one image) when grouping is tied across it. */
+typedef enum {
+    HKV_CFG_UNTIED = 0,   /* every sequence is grouped on its own */
+    HKV_CFG_HALVES = 1,   /* batch = [conditional | unconditional]: s, s + S/2 */
+    HKV_CFG_ADJACENT = 2  /* streams alternate: 2i, 2i + 1 */
+} hkv_cfg_pairing;
+
 typedef struct {
     int32_t num_seqs;     /* S: independent sequences (CFG halves included) */
     int32_t num_layers;   /* layers; each keeps its own cache */
@@ -75,6 +83,12 @@ typedef struct {
     int32_t rho_den;
     int32_t mode;         /* hkv_mode */
     int32_t stratified;   /* 1: near/far strata (STE); 0: one pool */
+    int32_t cls_queries;  /* grouping reads the per-distance weights of the
+                             last cls_queries prefill queries, averaged
+                             (1..r; 0 means 1 = the last query alone) */
+    int32_t cfg_pairing;  /* hkv_cfg_pairing: grouping of a CFG pair by the
+                             mean of both streams' rows (one label per pair);
+                             S must be even unless HKV_CFG_UNTIED */
     double tau;           /* grouping threshold, 0.9 on the pages */
 } hkv_config;
 
@@ -106,7 +120,11 @@ HKV_API hkv_status hkv_create(const hkv_config* cfg, void* pool, size_t bytes, v
  *  out:     [S][H][prefill_len][d] causal attention outputs, or NULL.
  * Causal softmax(q k^T / sqrt(d)) v over the prefill tokens.  Each head is
  * then labelled from the weights of the last prefill query: Local iff the
- * newest tokens reach tau in fewer than W tokens.  Budgets follow: Local
+ * newest tokens reach tau in fewer than W tokens.  With cls_queries = n > 1
+ * the weight at each distance is the mean over the last n queries; with a
+ * cfg_pairing the row is also averaged over the pair's two streams, which
+ * then share their labels and budgets (the pair's two layers must be
+ * classified by the same call: they are, as one call covers all S).  Budgets follow: Local
  * heads keep W, Global heads split floor(H*L*rho) - nL*W evenly (rounded
  * down) per (sequence, layer).  Local heads keep their last W prefill
  * tokens; Global heads keep all, or, beyond their budget, run one

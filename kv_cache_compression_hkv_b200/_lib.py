@@ -21,6 +21,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "hkv.h")
 
 DTYPE_F32, DTYPE_BF16 = 0, 1
 MODE_HEADKV, MODE_FULL, MODE_UNIFORM = 0, 1, 2
+CFG_UNTIED, CFG_HALVES, CFG_ADJACENT = 0, 1, 2
 STATUS = {0: "HKV_OK", 1: "HKV_ERR_INVALID_ARG", 2: "HKV_ERR_STATE", 3: "HKV_ERR_CAPACITY",
           4: "HKV_ERR_NUMERIC", 5: "HKV_ERR_CUDA", 6: "HKV_ERR_TIMEOUT"}
 
@@ -34,8 +35,8 @@ class HkvError(RuntimeError):
 class _Config(C.Structure):
     _fields_ = [(n, C.c_int32) for n in (
         "num_seqs", "num_layers", "num_heads", "head_dim", "dtype", "max_len", "local_window",
-        "ste_m", "near_dist", "score_window", "rho_num", "rho_den", "mode", "stratified")] + [
-        ("tau", C.c_double)]
+        "ste_m", "near_dist", "score_window", "rho_num", "rho_den", "mode", "stratified",
+        "cls_queries", "cfg_pairing")] + [("tau", C.c_double)]
 
 
 _lib = None
@@ -114,13 +115,16 @@ class Config:
     dtype: int = DTYPE_BF16
     mode: int = MODE_HEADKV
     stratified: int = 1
+    cls_queries: int = 1   # grouping by the last n prefill queries' per-distance weights
+    cfg_pairing: int = CFG_UNTIED
     tau: float = 0.9
 
     def c(self) -> _Config:
         return _Config(self.num_seqs, self.num_layers, self.num_heads, self.head_dim, self.dtype,
                        self.max_len, self.local_window, self.ste_m, self.near_dist,
                        self.score_window, self.rho_num, self.rho_den, self.mode,
-                       int(self.stratified), float(self.tau))
+                       int(self.stratified), int(self.cls_queries), int(self.cfg_pairing),
+                       float(self.tau))
 
     @property
     def torch_dtype(self):

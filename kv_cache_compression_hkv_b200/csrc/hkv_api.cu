@@ -77,6 +77,9 @@ bool config_ok(const hkv_config* c, int64_t* T_out, int32_t* R_out) {
     if (c->rho_num < 1 || c->rho_den < c->rho_num) return false;
     if (c->mode < HKV_MODE_HEADKV || c->mode > HKV_MODE_UNIFORM) return false;
     if (c->stratified != 0 && c->stratified != 1) return false;
+    if (c->cls_queries < 0 || c->cls_queries > c->score_window) return false;
+    if (c->cfg_pairing < HKV_CFG_UNTIED || c->cfg_pairing > HKV_CFG_ADJACENT) return false;
+    if (c->cfg_pairing != HKV_CFG_UNTIED && (c->num_seqs & 1)) return false;
     if (!(c->tau > 0.0 && c->tau <= 1.0)) return false;
     if ((int64_t)c->num_seqs * c->num_heads > 12288) return false;
     const int64_t H = c->num_heads, L = c->max_len;
@@ -139,6 +142,7 @@ size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Lay
     l.S = c->num_seqs; l.Ly = c->num_layers; l.H = c->num_heads; l.d = c->head_dim;
     l.L = c->max_len; l.W = c->local_window; l.M = c->ste_m; l.D = c->near_dist;
     l.r = c->score_window; l.mode = c->mode; l.stratified = c->stratified; l.dtype = c->dtype;
+    l.nq = c->cls_queries > 0 ? c->cls_queries : 1; l.pairing = c->cfg_pairing;
     l.R = R; l.T_total = T; l.tau = c->tau; l.max_chunks = (int32_t)max_chunks;
     if (L) *L = l;
     (void)ctrl_end;

@@ -23,6 +23,8 @@ constexpr int RANK_MAX = 32;          // strata up to this size are selected by 
 struct Layout {
     int32_t S, Ly, H, d, L, W, M, D, r;
     int32_t mode, stratified, dtype;
+    int32_t nq;         // prefill queries whose per-distance weights group a head
+    int32_t pairing;    // hkv_cfg_pairing: grouping tied across a CFG pair
     int32_t R;          // slots per (sequence, layer) region
     int64_t T_total;    // floor(H * L * rho): tokens one (sequence, layer) keeps
     double tau;

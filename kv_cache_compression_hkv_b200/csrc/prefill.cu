@@ -84,6 +84,54 @@ __global__ void __launch_bounds__(128) prefill_attn_simt(const T* __restrict__ q
     }
 }
 
+// The other stream of sequence s's classifier-free-guidance pair (s itself
+// when grouping is not tied).
+__device__ __forceinline__ int cfg_partner(const Layout& L, int s) {
+    if (L.pairing == HKV_CFG_HALVES) return s < L.S / 2 ? s + L.S / 2 : s - L.S / 2;
+    if (L.pairing == HKV_CFG_ADJACENT) return s ^ 1;
+    return s;
+}
+
+// Grouping row of head h (Methodology step 2): the weight at distance delta
+// is the mean, over the last nq prefill queries i of sequence sa and, when
+// sb != sa, of sequence sb, of query i's weight on position i - delta (none
+// when delta > i).  The kept weight rows are [s*H + h][r][P], row q holding
+// the query at position P - r + q.  Each lane owns one distance per pass;
+// the mean weights are summed newest first in double until they reach tau.
+// sa < sb fixes the order of the sums, so both streams of a pair get the
+// same count.  Returns the number of tokens that took (P if never).
+__device__ int warp_group_need(const Layout& L, int sa, int sb, int h, int P) {
+    const int lane = threadIdx.x & 31;
+    const int r = L.r, nq = L.nq;
+    const double inv = 1.0 / (double)(nq * (sb != sa ? 2 : 1));
+    double carry = 0.0;
+    for (int base = 0; base < P; base += 32) {
+        const int delta = base + lane;
+        double x = 0.0;
+        if (delta < P) {
+            for (int s = sa;; s = sb) {
+                const float* rows = L.rows + (size_t)(s * L.H + h) * r * P;
+                for (int q = r - nq; q < r; ++q) {
+                    const int i = P - r + q;
+                    if (delta <= i) x += (double)rows[(size_t)q * P + (i - delta)];
+                }
+                if (s == sb) break;
+            }
+            x *= inv;
+        }
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double y = __shfl_up_sync(FULL_MASK, x, o);
+            if (lane >= o) x += y;
+        }
+        const double c = carry + x;
+        const unsigned hit = __ballot_sync(FULL_MASK, delta < P && c >= L.tau);
+        if (hit) return base + __ffs(hit);  // delta = 0 .. first hit
+        carry += __shfl_sync(FULL_MASK, x, 31);
+    }
+    return P;
+}
+
 // Head grouping (Methodology step 2) for one (layer, sequence) per block,
 // one warp per head, then budgets (Main contributions: asymmetric budgets)
 // and the layout of the heads' slots.  The backward accumulation runs in
@@ -96,8 +144,8 @@ __global__ void classify_kernel(Layout L, int layer, int P) {
     int need = P;
     uint8_t label = 0;
     if (L.mode == HKV_MODE_HEADKV) {
-        const float* row = L.rows + ((size_t)(s * L.H + h) * L.r + (L.r - 1)) * P;
-        need = warp_tokens_to_tau(row, P, L.tau);
+        const int sp = cfg_partner(L, s);
+        need = warp_group_need(L, min(s, sp), max(s, sp), h, P);
         label = need < L.W ? 1 : 0;  // fewer tokens than the window: Local
     } else if (L.mode == HKV_MODE_FULL) {
         label = 2;

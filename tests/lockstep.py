@@ -27,11 +27,12 @@ LABEL_BAND = 1e-3
 SELECT_BAND = 1e-3
 
 
-def oracle_params(w, mode=O.MODE_HEADKV, stratified=True) -> O.UnitParams:
+def oracle_params(w, mode=O.MODE_HEADKV, stratified=True, cls_queries=1) -> O.UnitParams:
     return O.UnitParams(num_heads=w.num_heads, head_dim=w.head_dim, max_len=w.max_len,
                         prefill_len=w.prefill_len, local_window=w.local_window, ste_m=w.ste_m,
                         near_dist=w.near_dist, score_window=w.score_window, rho_num=w.rho[0],
                         rho_den=w.rho[1], mode=mode, stratified=stratified,
+                        cls_queries=cls_queries,
                         label_band=LABEL_BAND, select_band=SELECT_BAND)
 
 
@@ -91,13 +92,26 @@ def run_gpu(w, cfg, data, units, fused=True, with_prefill_out=False):
     return cache, rec, pre_out
 
 
-def compare_unit(w, data, unit, r, mode=O.MODE_HEADKV, stratified=True):
+def class_rows(w, data, s, l, nq):
+    """[H, P] oracle grouping rows of sequence s in layer l."""
+    P = w.prefill_len
+    q, k, v = (x[s, :, :P].double().cpu().numpy() for x in data[l])
+    return np.stack([O.class_row(q[h], k[h], v[h], nq) for h in range(w.num_heads)])
+
+
+def compare_unit(w, data, unit, r, mode=O.MODE_HEADKV, stratified=True, cls_queries=1,
+                 pairing=O.CFG_UNTIED):
     """Replays one unit through the oracle with the GPU's decisions as hints.
     Returns (oracle result, max relative output error per decode call)."""
     s, l = unit
     q, k, v = (x[s].double().cpu().numpy() for x in data[l])
     H = w.num_heads
-    prm = oracle_params(w, mode, stratified)
+    prm = oracle_params(w, mode, stratified, cls_queries)
+    cls = None
+    if pairing != O.CFG_UNTIED:
+        sp = O.cfg_partner(s, data[l][0].shape[0], pairing)
+        cls = O.tied_rows(class_rows(w, data, s, l, cls_queries),
+                          class_rows(w, data, sp, l, cls_queries))
     hints = None
     if mode != O.MODE_FULL:
         ev = r["events"]
@@ -110,7 +124,7 @@ def compare_unit(w, data, unit, r, mode=O.MODE_HEADKV, stratified=True):
                  "kept": kept[: len(ev)] if ev else None}
         if not ev:
             hints.pop("kept")
-    res = O.run_unit(prm, q, k, v, hints=hints)
+    res = O.run_unit(prm, q, k, v, hints=hints, cls_rows=cls)
     got = r["o"].double().cpu().numpy()
     ref = res.o_decode
     err = np.abs(got - ref).max(axis=(1, 2)) / np.abs(ref).max(axis=(1, 2))

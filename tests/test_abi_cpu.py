@@ -53,12 +53,25 @@ def test_config_validation():
     bad = [dict(num_heads=0), dict(num_heads=33), dict(head_dim=96), dict(ste_m=31), dict(ste_m=0),
            dict(score_window=0), dict(score_window=40), dict(rho_num=2, rho_den=1), dict(tau=0.0),
            dict(tau=1.5), dict(mode=7), dict(stratified=2), dict(max_len=1), dict(max_len=9000),
-           dict(local_window=0), dict(rho_num=1, rho_den=64)]  # last: budget below H*W
+           dict(local_window=0), dict(cls_queries=-1), dict(cls_queries=9),
+           dict(cfg_pairing=3), dict(cfg_pairing=-1), dict(num_seqs=63, cfg_pairing=1),
+           dict(num_seqs=63, cfg_pairing=2),
+           dict(rho_num=1, rho_den=64)]  # last: budget below H*W
     for kw in bad:
         cfg = hkv.Config(**{**base.__dict__, **kw})
         with pytest.raises(hkv.HkvError) as e:
             hkv.pool_bytes(cfg)
         assert e.value.code == 1, kw
+
+
+def test_classifier_variants_accepted():
+    base = hkv.config_for(WORKLOADS["llamagen_xl"])
+    n = hkv.pool_bytes(base)
+    for kw in (dict(cls_queries=0), dict(cls_queries=8), dict(cfg_pairing=hkv.CFG_HALVES),
+               dict(cfg_pairing=hkv.CFG_ADJACENT, cls_queries=8), dict(num_seqs=63)):
+        assert hkv.pool_bytes(hkv.Config(**{**base.__dict__, **kw})) > 0, kw
+    # the variants change no buffer
+    assert hkv.pool_bytes(hkv.Config(**{**base.__dict__, "cls_queries": 8, "cfg_pairing": 1})) == n
 
 
 def test_create_rejects_bad_pool_without_touching_the_device():

@@ -95,8 +95,10 @@ def test_select_batch_bitexact(n, stratified):
 # whole hot path, lock-step with the oracle
 # ---------------------------------------------------------------------------
 
-def _lockstep(w, units, seed=0, fused=True, mode=hkv.MODE_HEADKV, stratified=True):
-    cfg = hkv.config_for(w, mode=mode, stratified=stratified)
+def _lockstep(w, units, seed=0, fused=True, mode=hkv.MODE_HEADKV, stratified=True,
+              cls_queries=1, pairing=hkv.CFG_UNTIED):
+    cfg = hkv.config_for(w, mode=mode, stratified=stratified, cls_queries=cls_queries,
+                         cfg_pairing=pairing)
     data = generate(w, seed, DEV)
     cache, rec, _ = run_gpu(w, cfg, data, units, fused=fused)
     rc, detail = cache.check()
@@ -105,7 +107,7 @@ def _lockstep(w, units, seed=0, fused=True, mode=hkv.MODE_HEADKV, stratified=Tru
              hkv.MODE_UNIFORM: O.MODE_UNIFORM}[mode]
     stats = []
     for u in units:
-        res, err = compare_unit(w, data, u, rec[u], omode, stratified)
+        res, err = compare_unit(w, data, u, rec[u], omode, stratified, cls_queries, pairing)
         assert_lockstep(res, err, TOL[w.dtype], len(rec[u]["events"]))
         if mode == hkv.MODE_HEADKV:
             np.testing.assert_array_equal(res.labels, rec[u]["labels"])
@@ -152,6 +154,26 @@ def test_unstratified_and_uniform_variants():
     w = WORKLOADS["llamagen_xl"].scaled(num_seqs=2, num_layers=1)
     _lockstep(w, [(0, 0), (1, 0)], seed=7, stratified=False)
     _lockstep(w, [(0, 0)], seed=8, mode=hkv.MODE_UNIFORM)
+
+
+@pytest.mark.parametrize("nq,pairing", [(8, hkv.CFG_UNTIED), (1, hkv.CFG_HALVES),
+                                         (8, hkv.CFG_ADJACENT)])
+def test_classifier_variants(nq, pairing):
+    """Grouping by the last nq queries' per-distance weights, and tied
+    across CFG pairs: labels and the whole unit in lock step with the
+    oracle; a tied pair's two streams carry identical labels."""
+    w = WORKLOADS["llamagen_xl"].scaled(num_seqs=4, num_layers=1)
+    units = [(s, 0) for s in range(4)]
+    cfg = hkv.config_for(w, cls_queries=nq, cfg_pairing=pairing)
+    _lockstep(w, units, seed=13, cls_queries=nq, pairing=pairing)
+    if pairing != hkv.CFG_UNTIED:
+        data = generate(w, 13, DEV)
+        cache, _, _ = run_gpu(w.scaled(image_tokens=w.prefill_image + 1), cfg, data, [])
+        lab, ntau = cache.labels(0)
+        for s in range(4):
+            sp = O.cfg_partner(s, 4, pairing)
+            np.testing.assert_array_equal(lab[s], lab[sp])
+            np.testing.assert_array_equal(ntau[s], ntau[sp])
 
 
 def test_prefill_outputs_match_oracle():
