@@ -89,6 +89,12 @@ typedef struct {
     int32_t cfg_pairing;  /* hkv_cfg_pairing: grouping of a CFG pair by the
                              mean of both streams' rows (one label per pair);
                              S must be even unless HKV_CFG_UNTIED */
+    int32_t heads_total;  /* heads of a whole (sequence, layer) when this
+                             context holds only num_heads of them (heads
+                             sharded over GPUs); 0 means num_heads.  Budgets
+                             count all heads_total heads: T = floor(heads_total
+                             * L * rho).  A sharded context prefills with
+                             hkv_prefill_label + hkv_prefill_compress */
     double tau;           /* grouping threshold, 0.9 on the pages */
 } hkv_config;
 
@@ -135,6 +141,33 @@ HKV_API hkv_status hkv_create(const hkv_config* cfg, void* pool, size_t bytes, v
 HKV_API hkv_status hkv_prefill_classify(hkv_ctx* ctx, int32_t layer, const void* q, const void* k,
                                 const void* v, int32_t prefill_len, int64_t block_stride,
                                 void* out, void* stream);
+
+/* The same, in two phases, for heads sharded over several contexts (one per
+ * GPU), whose budgets need the Local count of every shard [Main
+ * contributions: asymmetric budgets count all heads of a sequence and
+ * layer].  hkv_prefill_label runs the prefill attention and the grouping of
+ * the heads held here and writes, per sequence, their Local count:
+ *  n_local: int32[S] device output (4-byte aligned), stream-ordered.
+ * The caller sums n_local over the shards (an all-reduce; NCCL over NVLink
+ * on GPUs) into n_local_total and calls hkv_prefill_compress with the same
+ * layer, prefill_len, k, v and block_stride (k and v must still hold the
+ * prefill tokens): budgets from the total, then the compression at
+ * classification.  Between the two calls no other layer may be labelled
+ * (the weight rows of the last r queries live in one shared scratch).
+ * A total outside [Local count here, Local count here + heads_total -
+ * num_heads] latches HKV_ERR_INVALID_ARG in the status word and is clamped
+ * into that range.  With heads_total == num_heads and n_local_total =
+ * n_local the pair computes exactly what hkv_prefill_classify computes;
+ * hkv_prefill_classify on a context with heads_total > num_heads returns
+ * INVALID_ARG.  Errors: INVALID_ARG, STATE (label: layer classified or
+ * another layer labelled and not compressed; compress: layer not the one
+ * labelled, or another prefill_len), CUDA. */
+HKV_API hkv_status hkv_prefill_label(hkv_ctx* ctx, int32_t layer, const void* q, const void* k,
+                                     const void* v, int32_t prefill_len, int64_t block_stride,
+                                     void* out, int32_t* n_local, void* stream);
+HKV_API hkv_status hkv_prefill_compress(hkv_ctx* ctx, int32_t layer, const void* k, const void* v,
+                                        int32_t prefill_len, int64_t block_stride,
+                                        const int32_t* n_local_total, void* stream);
 
 /* Appends the next token's key and value ([S][H][d] each) to every head of
  * `layer` [step 3]: Local heads overwrite their oldest token (sliding

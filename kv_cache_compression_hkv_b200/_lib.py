@@ -36,7 +36,7 @@ class _Config(C.Structure):
     _fields_ = [(n, C.c_int32) for n in (
         "num_seqs", "num_layers", "num_heads", "head_dim", "dtype", "max_len", "local_window",
         "ste_m", "near_dist", "score_window", "rho_num", "rho_den", "mode", "stratified",
-        "cls_queries", "cfg_pairing")] + [("tau", C.c_double)]
+        "cls_queries", "cfg_pairing", "heads_total")] + [("tau", C.c_double)]
 
 
 _lib = None
@@ -56,6 +56,8 @@ def lib():
             "hkv_pool_bytes": [P, P],
             "hkv_create": [P, P, Z, P, P],
             "hkv_prefill_classify": [P, I, P, P, P, I, I64, P, P],
+            "hkv_prefill_label": [P, I, P, P, P, I, I64, P, P, P],
+            "hkv_prefill_compress": [P, I, P, P, I, I64, P, P],
             "hkv_append": [P, I, P, P, P],
             "hkv_decode_attend": [P, I, P, P, P],
             "hkv_decode_step": [P, I, P, P, P, P, P],
@@ -117,6 +119,7 @@ class Config:
     stratified: int = 1
     cls_queries: int = 1   # grouping by the last n prefill queries' per-distance weights
     cfg_pairing: int = CFG_UNTIED
+    heads_total: int = 0   # heads of a whole (sequence, layer) when heads are sharded
     tau: float = 0.9
 
     def c(self) -> _Config:
@@ -124,7 +127,7 @@ class Config:
                        self.max_len, self.local_window, self.ste_m, self.near_dist,
                        self.score_window, self.rho_num, self.rho_den, self.mode,
                        int(self.stratified), int(self.cls_queries), int(self.cfg_pairing),
-                       float(self.tau))
+                       int(self.heads_total), float(self.tau))
 
     @property
     def torch_dtype(self):
@@ -186,9 +189,7 @@ class HeadKVCache:
         if tuple(x.shape) != (c.num_seqs, c.num_heads, c.head_dim) or not x.is_contiguous():
             raise ValueError(f"{name}: expected a contiguous [S, H, d] tensor")
 
-    def prefill_classify(self, layer: int, q, k, v, out=None, stream=None):
-        """q, k, v: [S, H, P, d] with unit stride in d, stride d in P and the
-        (s, h) blocks evenly spaced (a [S, H, L, d] tensor sliced to P works)."""
+    def _prefill_inputs(self, q, k, v, out):
         c = self.cfg
         for x, nm in ((q, "q"), (k, "k"), (v, "v")):
             self._tensor(x, nm)
@@ -205,9 +206,43 @@ class HeadKVCache:
             self._tensor(out, "out")
             if tuple(out.shape) != tuple(q.shape) or not out.is_contiguous():
                 raise ValueError("out: expected a contiguous [S, H, P, d] tensor")
+        return P
+
+    def prefill_classify(self, layer: int, q, k, v, out=None, stream=None):
+        """q, k, v: [S, H, P, d] with unit stride in d, stride d in P and the
+        (s, h) blocks evenly spaced (a [S, H, L, d] tensor sliced to P works)."""
+        P = self._prefill_inputs(q, k, v, out)
         _check(lib().hkv_prefill_classify(self.ctx, layer, q.data_ptr(), k.data_ptr(),
                                           v.data_ptr(), P, q.stride(1), _ptr(out),
                                           _stream(stream)), "hkv_prefill_classify")
+
+    def prefill_label(self, layer: int, q, k, v, out=None, n_local=None, stream=None):
+        """Sharded heads, phase 1: prefill attention and grouping of the
+        heads held here.  Returns n_local (int32 [S] on the device): each
+        sequence's Local count here, to be summed over the shards."""
+        P = self._prefill_inputs(q, k, v, out)
+        if n_local is None:
+            n_local = torch.empty(self.cfg.num_seqs, dtype=torch.int32, device=self.device)
+        elif n_local.dtype != torch.int32 or n_local.device != self.device or \
+                n_local.numel() != self.cfg.num_seqs or not n_local.is_contiguous():
+            raise ValueError("n_local: expected a contiguous int32 [S] tensor on the device")
+        _check(lib().hkv_prefill_label(self.ctx, layer, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                       P, q.stride(1), _ptr(out), n_local.data_ptr(),
+                                       _stream(stream)), "hkv_prefill_label")
+        return n_local
+
+    def prefill_compress(self, layer: int, k, v, n_local_total, stream=None):
+        """Sharded heads, phase 2: budgets from the all-shards Local counts
+        (int32 [S] on the device), then compression at classification.  k, v:
+        the same prefill tensors prefill_label got."""
+        P = self._prefill_inputs(k, k, v, None)
+        t = n_local_total
+        if t.dtype != torch.int32 or t.device != self.device or t.numel() != self.cfg.num_seqs \
+                or not t.is_contiguous():
+            raise ValueError("n_local_total: expected a contiguous int32 [S] tensor on the device")
+        _check(lib().hkv_prefill_compress(self.ctx, layer, k.data_ptr(), v.data_ptr(), P,
+                                          k.stride(1), t.data_ptr(), _stream(stream)),
+               "hkv_prefill_compress")
 
     def append(self, layer: int, k_t, v_t, stream=None):
         self._step_tensor(k_t, "k_t")

@@ -31,6 +31,10 @@ struct hkv_ctx {
     int last_decode = -1;
     void* last_stream = nullptr;
     int split_buf = 0;  // split-K buffer set of the next decode launch
+    // a layer labelled by hkv_prefill_label and not yet compressed (-1: none),
+    // and its prefill length; its weight rows occupy the shared row scratch
+    int labelled_layer = -1;
+    int labelled_len = 0;
 };
 
 namespace {
@@ -64,6 +68,8 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 size_t elem_size(int dtype) { return dtype == HKV_DTYPE_F32 ? 4 : 2; }
 
+int64_t total_heads(const hkv_config* c) { return c->heads_total > 0 ? c->heads_total : c->num_heads; }
+
 bool config_ok(const hkv_config* c, int64_t* T_out, int32_t* R_out) {
     if (!c) return false;
     if (c->num_seqs < 1 || c->num_layers < 1 || c->num_heads < 1 || c->num_heads > 32) return false;
@@ -82,15 +88,19 @@ bool config_ok(const hkv_config* c, int64_t* T_out, int32_t* R_out) {
     if (c->cfg_pairing != HKV_CFG_UNTIED && (c->num_seqs & 1)) return false;
     if (!(c->tau > 0.0 && c->tau <= 1.0)) return false;
     if ((int64_t)c->num_seqs * c->num_heads > 12288) return false;
+    if (c->heads_total != 0 && (c->heads_total < c->num_heads || c->heads_total > 4096)) return false;
     const int64_t H = c->num_heads, L = c->max_len;
-    const int64_t T = H * L * c->rho_num / c->rho_den;
+    const int64_t Ht = total_heads(c);
+    // the budget of a (sequence, layer) counts all its heads, sharded or not
+    const int64_t T = Ht * L * c->rho_num / c->rho_den;
     int64_t R;
     if (c->mode == HKV_MODE_HEADKV) {
-        if (T < H * c->local_window) return false;
+        if (T < Ht * c->local_window) return false;
+        // this shard's caps: nL_here*W + nG_here*(B_g + M) <= T + H*M
         R = T + H * c->ste_m;
     } else if (c->mode == HKV_MODE_UNIFORM) {
-        if (T / H < 1) return false;
-        R = (T / H + c->ste_m) * H;
+        if (T / Ht < 1) return false;
+        R = (T / Ht + c->ste_m) * H;
     } else {
         R = H * L;
     }
@@ -140,6 +150,7 @@ size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Lay
     l.plan_desc = (int4*)take(Ly * max_chunks * 16);
     l.plan_warp = (int4*)take(Ly * hkv::PLAN_MAX_WARPS * (1 + hkv::PLAN_WARP_DESC) * 16);
     l.S = c->num_seqs; l.Ly = c->num_layers; l.H = c->num_heads; l.d = c->head_dim;
+    l.H_total = (int32_t)total_heads(c);
     l.L = c->max_len; l.W = c->local_window; l.M = c->ste_m; l.D = c->near_dist;
     l.r = c->score_window; l.mode = c->mode; l.stratified = c->stratified; l.dtype = c->dtype;
     l.nq = c->cls_queries > 0 ? c->cls_queries : 1; l.pairing = c->cfg_pairing;
@@ -237,32 +248,81 @@ hkv_status hkv_create(const hkv_config* cfg, void* pool, size_t bytes, void* str
     return HKV_OK;
 }
 
-hkv_status hkv_prefill_classify(hkv_ctx* c, int32_t layer, const void* q, const void* k,
-                                const void* v, int32_t prefill_len, int64_t block_stride,
-                                void* out, void* stream) {
-    if (!c || !q || !k || !v) return HKV_ERR_INVALID_ARG;
+// Argument checks shared by the prefill entry points (q may be null for the
+// compression phase, which reads only k and v).
+static hkv_status prefill_args(const hkv_ctx* c, int32_t layer, const void* q, const void* k,
+                               const void* v, int32_t P, int64_t block_stride, const void* out,
+                               bool need_q) {
+    if (!c || (need_q && !q) || !k || !v) return HKV_ERR_INVALID_ARG;
     const hkv_config& g = c->cfg;
     if (layer < 0 || layer >= g.num_layers) return HKV_ERR_INVALID_ARG;
-    const int P = prefill_len;
     if (P < g.local_window || P >= g.max_len || P < g.score_window || P < 2)
         return HKV_ERR_INVALID_ARG;
     const size_t es = elem_size(g.dtype);
     if (block_stride < (int64_t)P * g.head_dim || (block_stride * (int64_t)es) % 16 != 0)
         return HKV_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || (out && !aligned16(out)))
+    if ((q && !aligned16(q)) || !aligned16(k) || !aligned16(v) || (out && !aligned16(out)))
         return HKV_ERR_INVALID_ARG;
-    if (c->classified[layer]) return HKV_ERR_STATE;
     if (hkv::pack_smem_bytes(P) > 200 * 1024) return HKV_ERR_INVALID_ARG;
-    note_other(c, stream);
-    cudaError_t e = hkv::launch_prefill(c->lay, layer, q, k, v, P, block_stride, out,
-                                        (cudaStream_t)stream);
-    if (e == cudaSuccess) e = hkv::launch_plan(c->lay, layer, layer + 1, 1, (cudaStream_t)stream);
-    if (e != cudaSuccess) return HKV_ERR_CUDA;
+    return HKV_OK;
+}
+
+// Marks `layer` ready for appends and decodes at length P and enqueues its
+// first decode plan.
+static hkv_status prefill_done(hkv_ctx* c, int32_t layer, int P, void* stream) {
+    if (hkv::launch_plan(c->lay, layer, layer + 1, 1, (cudaStream_t)stream) != cudaSuccess)
+        return HKV_ERR_CUDA;
     c->plan_for[layer] = P;
     c->classified[layer] = 1;
     c->t_host[layer] = P;
     c->prefill_len[layer] = P;
     return HKV_OK;
+}
+
+hkv_status hkv_prefill_classify(hkv_ctx* c, int32_t layer, const void* q, const void* k,
+                                const void* v, int32_t prefill_len, int64_t block_stride,
+                                void* out, void* stream) {
+    hkv_status st = prefill_args(c, layer, q, k, v, prefill_len, block_stride, out, true);
+    if (st != HKV_OK) return st;
+    // sharded heads need every shard's Local count: hkv_prefill_label + _compress
+    if (total_heads(&c->cfg) != c->cfg.num_heads) return HKV_ERR_INVALID_ARG;
+    if (c->classified[layer] || c->labelled_layer >= 0) return HKV_ERR_STATE;
+    note_other(c, stream);
+    if (hkv::launch_prefill(c->lay, layer, q, k, v, prefill_len, block_stride, out,
+                            (cudaStream_t)stream) != cudaSuccess)
+        return HKV_ERR_CUDA;
+    return prefill_done(c, layer, prefill_len, stream);
+}
+
+hkv_status hkv_prefill_label(hkv_ctx* c, int32_t layer, const void* q, const void* k,
+                             const void* v, int32_t prefill_len, int64_t block_stride, void* out,
+                             int32_t* n_local, void* stream) {
+    hkv_status st = prefill_args(c, layer, q, k, v, prefill_len, block_stride, out, true);
+    if (st != HKV_OK) return st;
+    if (!n_local || ((uintptr_t)n_local & 3)) return HKV_ERR_INVALID_ARG;
+    if (c->classified[layer] || c->labelled_layer >= 0) return HKV_ERR_STATE;
+    note_other(c, stream);
+    if (hkv::launch_prefill_label(c->lay, layer, q, k, v, prefill_len, block_stride, out, n_local,
+                                  (cudaStream_t)stream) != cudaSuccess)
+        return HKV_ERR_CUDA;
+    c->labelled_layer = layer;
+    c->labelled_len = prefill_len;
+    return HKV_OK;
+}
+
+hkv_status hkv_prefill_compress(hkv_ctx* c, int32_t layer, const void* k, const void* v,
+                                int32_t prefill_len, int64_t block_stride,
+                                const int32_t* n_local_total, void* stream) {
+    hkv_status st = prefill_args(c, layer, nullptr, k, v, prefill_len, block_stride, nullptr, false);
+    if (st != HKV_OK) return st;
+    if (!n_local_total || ((uintptr_t)n_local_total & 3)) return HKV_ERR_INVALID_ARG;
+    if (c->labelled_layer != layer || c->labelled_len != prefill_len) return HKV_ERR_STATE;
+    note_other(c, stream);
+    if (hkv::launch_prefill_compress(c->lay, layer, k, v, prefill_len, block_stride, n_local_total,
+                                     (cudaStream_t)stream) != cudaSuccess)
+        return HKV_ERR_CUDA;
+    c->labelled_layer = -1;
+    return prefill_done(c, layer, prefill_len, stream);
 }
 
 static hkv_status step_check(hkv_ctx* c, int32_t layer, bool appends) {
@@ -430,6 +490,7 @@ hkv_status hkv_reset(hkv_ctx* c, void* stream) {
         c->prefill_len[l] = 0;
         c->plan_for[l] = -1;
     }
+    c->labelled_layer = -1;
     return HKV_OK;
 }
 

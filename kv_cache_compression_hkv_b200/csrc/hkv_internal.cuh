@@ -22,6 +22,7 @@ constexpr int RANK_MAX = 32;          // strata up to this size are selected by 
 // The pool is one caller-owned device buffer carved into these regions.
 struct Layout {
     int32_t S, Ly, H, d, L, W, M, D, r;
+    int32_t H_total;    // heads of a whole (sequence, layer): H, or more when heads are sharded
     int32_t mode, stratified, dtype;
     int32_t nq;         // prefill queries whose per-distance weights group a head
     int32_t pairing;    // hkv_cfg_pairing: grouping tied across a CFG pair

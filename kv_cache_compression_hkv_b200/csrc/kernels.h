@@ -20,6 +20,15 @@ cudaError_t launch_prefill_umma(const Layout& L, const void* q, const void* k, c
                                 int64_t block_stride, void* out, cudaStream_t st);
 cudaError_t launch_prefill(const Layout& L, int layer, const void* q, const void* k, const void* v,
                            int P, int64_t block_stride, void* out, cudaStream_t st);
+// Sharded heads: attention and labels, with each sequence's Local count of
+// the heads held here in n_local[S]; then budgets from the all-shards count
+// n_local_total[S] and the compression at classification.
+cudaError_t launch_prefill_label(const Layout& L, int layer, const void* q, const void* k,
+                                 const void* v, int P, int64_t block_stride, void* out,
+                                 int32_t* n_local, cudaStream_t st);
+cudaError_t launch_prefill_compress(const Layout& L, int layer, const void* k, const void* v, int P,
+                                    int64_t block_stride, const int32_t* n_local_total,
+                                    cudaStream_t st);
 // Launch shape of the decode kernel: warps per block, pipeline stages per
 // warp, dynamic shared memory.
 struct DecodeShape {

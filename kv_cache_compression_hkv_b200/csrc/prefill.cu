@@ -132,37 +132,20 @@ __device__ int warp_group_need(const Layout& L, int sa, int sb, int h, int P) {
     return P;
 }
 
-// Head grouping (Methodology step 2) for one (layer, sequence) per block,
-// one warp per head, then budgets (Main contributions: asymmetric budgets)
-// and the layout of the heads' slots.  The backward accumulation runs in
-// double.
-__global__ void classify_kernel(Layout L, int layer, int P) {
-    __shared__ uint8_t lab[32];
-    __shared__ int32_t ntau[32];
-    const int s = blockIdx.x;
-    const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int need = P;
-    uint8_t label = 0;
-    if (L.mode == HKV_MODE_HEADKV) {
-        const int sp = cfg_partner(L, s);
-        need = warp_group_need(L, min(s, sp), max(s, sp), h, P);
-        label = need < L.W ? 1 : 0;  // fewer tokens than the window: Local
-    } else if (L.mode == HKV_MODE_FULL) {
-        label = 2;
-    }
-    if (lane == 0) { lab[h] = label; ntau[h] = need; }
-    __syncthreads();
-    if (threadIdx.x != 0) return;
-    const int H = L.H;
-    int nl = 0;
-    for (int j = 0; j < H; ++j) nl += lab[j] == 1;
-    const int ng = H - nl;
+// Budgets (Main contributions: asymmetric budgets) and the slot layout of
+// the heads of (layer, s) held here, from their labels lab[] and the Local
+// count nl of the whole (sequence, layer): every shard of its heads.
+// Local heads keep W; Global heads split T - nl*W evenly over the
+// H_total - nl Global heads, rounded down.  One thread.
+__device__ void lay_out_heads(const Layout& L, int layer, int s, int P, const uint8_t* lab,
+                              const int32_t* ntau, int nl) {
+    const int ng = L.H_total - nl;
     int bg;
     if (L.mode == HKV_MODE_HEADKV) bg = ng > 0 ? (int)((L.T_total - (int64_t)nl * L.W) / ng) : 0;
-    else if (L.mode == HKV_MODE_UNIFORM) bg = (int)(L.T_total / H);
+    else if (L.mode == HKV_MODE_UNIFORM) bg = (int)(L.T_total / L.H_total);
     else bg = L.L;
     int o = 0;
-    for (int j = 0; j < H; ++j) {
+    for (int j = 0; j < L.H; ++j) {
         const size_t hi = head_index(L, layer, s, j);
         int cap, budget, len0;
         if (lab[j] == 1) { cap = L.W; budget = L.W; len0 = P < L.W ? P : L.W; }
@@ -179,6 +162,69 @@ __global__ void classify_kernel(Layout L, int layer, int P) {
     }
     if (o > L.R) latch_error(L, HKV_ERR_CAPACITY, layer * L.S + s);
     if (s == 0) L.t_next[layer] = P;
+}
+
+// Head grouping (Methodology step 2) for one (layer, sequence) per block,
+// one warp per head; the backward accumulation runs in double.  With
+// n_local == nullptr the budgets and slot layout follow at once from this
+// block's own Local count (every head of the sequence is here).  Otherwise
+// the labels are stored and n_local[s] receives the Local count of the
+// heads held here, for the caller to sum over the shards of the heads.
+__global__ void classify_kernel(Layout L, int layer, int P, int32_t* n_local) {
+    __shared__ uint8_t lab[32];
+    __shared__ int32_t ntau[32];
+    const int s = blockIdx.x;
+    const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int need = P;
+    uint8_t label = 0;
+    if (L.mode == HKV_MODE_HEADKV) {
+        const int sp = cfg_partner(L, s);
+        need = warp_group_need(L, min(s, sp), max(s, sp), h, P);
+        label = need < L.W ? 1 : 0;  // fewer tokens than the window: Local
+    } else if (L.mode == HKV_MODE_FULL) {
+        label = 2;
+    }
+    if (lane == 0) { lab[h] = label; ntau[h] = need; }
+    __syncthreads();
+    if (threadIdx.x != 0) return;
+    int nl = 0;
+    for (int j = 0; j < L.H; ++j) nl += lab[j] == 1;
+    if (n_local) {
+        for (int j = 0; j < L.H; ++j) {
+            const size_t hi = head_index(L, layer, s, j);
+            L.label[hi] = lab[j];
+            L.n_tau[hi] = ntau[j];
+        }
+        n_local[s] = nl;
+        return;
+    }
+    lay_out_heads(L, layer, s, P, lab, ntau, nl);
+}
+
+// Budgets and slot layout of sharded heads (one block per sequence), once
+// the caller has summed the shards' Local counts into n_local_total.  A
+// count outside what the labels held here allow latches
+// HKV_ERR_INVALID_ARG and is clamped into that range.
+__global__ void layout_kernel(Layout L, int layer, int P, const int32_t* __restrict__ n_local_total) {
+    __shared__ uint8_t lab[32];
+    __shared__ int32_t ntau[32];
+    const int s = blockIdx.x;
+    if (threadIdx.x < L.H) {
+        const size_t hi = head_index(L, layer, s, threadIdx.x);
+        lab[threadIdx.x] = L.label[hi];
+        ntau[threadIdx.x] = L.n_tau[hi];
+    }
+    __syncthreads();
+    if (threadIdx.x != 0) return;
+    int here = 0;
+    for (int j = 0; j < L.H; ++j) here += lab[j] == 1;
+    int nl = n_local_total[s];
+    const int hi_bound = here + (L.H_total - L.H);  // every other shard's heads Local
+    if (nl < here || nl > hi_bound) {
+        latch_error(L, HKV_ERR_INVALID_ARG, layer * L.S + s);
+        nl = nl < here ? here : hi_bound;
+    }
+    lay_out_heads(L, layer, s, P, lab, ntau, nl);
 }
 
 // Bytes of the pack kernel's kept-position list, rounded so that the select
@@ -267,26 +313,29 @@ __global__ void __launch_bounds__(128) pack_kernel(Layout L, int layer, const T*
 
 size_t pack_smem_bytes(int P) { return pack_kept_bytes(P) + select_scratch_bytes(P); }
 
-cudaError_t launch_prefill(const Layout& L, int layer, const void* q, const void* k, const void* v,
-                           int P, int64_t block_stride, void* out, cudaStream_t st) {
+// Causal prefill attention of every (sequence, head) block; the weights of
+// the last r queries land in L.rows.
+static cudaError_t launch_attention(const Layout& L, const void* q, const void* k, const void* v,
+                                    int P, int64_t block_stride, void* out, cudaStream_t st) {
     const int nb = L.S * L.H;
     dim3 grid(nb, (P + 3) / 4);
     size_t sm = (size_t)4 * (L.d + P) * sizeof(float);
-    cudaError_t e;
     if (L.dtype == HKV_DTYPE_F32) {
         // fp32 caches keep fp32 products: CUDA cores
         prefill_attn_simt<float><<<grid, 128, sm, st>>>(
             (const float*)q, (const float*)k, (const float*)v, P, L.d, block_stride, L.r,
             (float*)out, L.rows);
-        e = cudaGetLastError();
-    } else {
-        // bf16 caches: tcgen05 tensor cores
-        e = launch_prefill_umma(L, q, k, v, P, block_stride, out, st);
+        return cudaGetLastError();
     }
-    if (e != cudaSuccess) return e;
-    classify_kernel<<<L.S, 32 * L.H, 0, st>>>(L, layer, P);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    // bf16 caches: tcgen05 tensor cores
+    return launch_prefill_umma(L, q, k, v, P, block_stride, out, st);
+}
+
+// Compression at classification time: each head's kept prefill tokens into
+// its slots.
+static cudaError_t launch_pack(const Layout& L, int layer, const void* k, const void* v, int P,
+                               int64_t block_stride, cudaStream_t st) {
+    const int nb = L.S * L.H;
     size_t psm = pack_smem_bytes(P);
     if (L.dtype == HKV_DTYPE_F32)
         pack_kernel<float><<<nb, 128, psm, st>>>(L, layer, (const float*)k, (const float*)v, P,
@@ -295,6 +344,34 @@ cudaError_t launch_prefill(const Layout& L, int layer, const void* q, const void
         pack_kernel<__nv_bfloat16><<<nb, 128, psm, st>>>(
             L, layer, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, P, block_stride);
     return cudaGetLastError();
+}
+
+cudaError_t launch_prefill(const Layout& L, int layer, const void* q, const void* k, const void* v,
+                           int P, int64_t block_stride, void* out, cudaStream_t st) {
+    cudaError_t e = launch_attention(L, q, k, v, P, block_stride, out, st);
+    if (e != cudaSuccess) return e;
+    classify_kernel<<<L.S, 32 * L.H, 0, st>>>(L, layer, P, nullptr);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_pack(L, layer, k, v, P, block_stride, st);
+}
+
+cudaError_t launch_prefill_label(const Layout& L, int layer, const void* q, const void* k,
+                                 const void* v, int P, int64_t block_stride, void* out,
+                                 int32_t* n_local, cudaStream_t st) {
+    cudaError_t e = launch_attention(L, q, k, v, P, block_stride, out, st);
+    if (e != cudaSuccess) return e;
+    classify_kernel<<<L.S, 32 * L.H, 0, st>>>(L, layer, P, n_local);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_compress(const Layout& L, int layer, const void* k, const void* v, int P,
+                                    int64_t block_stride, const int32_t* n_local_total,
+                                    cudaStream_t st) {
+    layout_kernel<<<L.S, 32, 0, st>>>(L, layer, P, n_local_total);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_pack(L, layer, k, v, P, block_stride, st);
 }
 
 // CUDA-core causal prefill of n_blocks caller blocks writing the weights of

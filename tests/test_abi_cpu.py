@@ -55,7 +55,8 @@ def test_config_validation():
            dict(tau=1.5), dict(mode=7), dict(stratified=2), dict(max_len=1), dict(max_len=9000),
            dict(local_window=0), dict(cls_queries=-1), dict(cls_queries=9),
            dict(cfg_pairing=3), dict(cfg_pairing=-1), dict(num_seqs=63, cfg_pairing=1),
-           dict(num_seqs=63, cfg_pairing=2),
+           dict(num_seqs=63, cfg_pairing=2), dict(heads_total=19), dict(heads_total=5000),
+           dict(heads_total=-1),
            dict(rho_num=1, rho_den=64)]  # last: budget below H*W
     for kw in bad:
         cfg = hkv.Config(**{**base.__dict__, **kw})
@@ -72,6 +73,19 @@ def test_classifier_variants_accepted():
         assert hkv.pool_bytes(hkv.Config(**{**base.__dict__, **kw})) > 0, kw
     # the variants change no buffer
     assert hkv.pool_bytes(hkv.Config(**{**base.__dict__, "cls_queries": 8, "cfg_pairing": 1})) == n
+
+
+def test_sharded_heads_pool():
+    """A context holding 7 of 20 heads: the budget counts all 20 heads, the
+    pool only this shard's slots (T + 7 * M per (sequence, layer))."""
+    w = WORKLOADS["llamagen_xl"]
+    base = hkv.config_for(w)
+    part = hkv.Config(**{**base.__dict__, "num_heads": 7, "heads_total": 20})
+    assert hkv.pool_bytes(part) < hkv.pool_bytes(base)
+    same = hkv.Config(**{**base.__dict__, "heads_total": 20})
+    assert hkv.pool_bytes(same) == hkv.pool_bytes(base)
+    for name in ("hkv_prefill_label", "hkv_prefill_compress"):
+        assert name in hkv.declared_symbols()
 
 
 def test_create_rejects_bad_pool_without_touching_the_device():
