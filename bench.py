@@ -55,6 +55,9 @@ def parse_args():
                     help="group heads by the last n prefill queries' per-distance weights")
     ap.add_argument("--cfg-pairing", default="untied", choices=list(PAIRINGS),
                     help="group the two streams of a CFG pair by their mean row")
+    ap.add_argument("--decoder-layer", action="store_true",
+                    help="also time whole decoder layers (projections + MLP on random "
+                         "weights around each attention call), compressed and full cache")
     ap.add_argument("--profile", action="store_true",
                     help="eager run of a reduced workload for ncu captures (no timing line)")
     ap.add_argument("--seqs", type=int, default=None, help="override the workload's sequences")
@@ -416,10 +419,111 @@ def gpu_arm(args, rank, world, dev):
         del g_full, cache_f
         torch.cuda.empty_cache()
 
+    if args.decoder_layer:
+        res["decoder_layer"] = decoder_layer_arm(args, w, cache, inp, outs, pre_out, dev)
+
     # end to end through the C ABI from pinned host buffers
     if not args.no_e2e:
         res["e2e"] = e2e_arm(args, w, cache, inp, dev, world)
     return res
+
+
+# ---------------------------------------------------------------------------
+# dense work of a decoder layer around each attention call (comparison harness)
+# ---------------------------------------------------------------------------
+
+class DecoderLayers:
+    """The dense work of a LLaMA-style decoder layer around every attention
+    call, on random weights: a QKV projection before it, the output
+    projection, a SwiGLU MLP and the residual adds after it.  hidden = H * d;
+    the MLP width is the LLaMA rule (the multiple of 256 at or above
+    8/3 * hidden), which gives 3584 / 5632 / 11008 for hidden 1280 / 2048 /
+    4096.  The projections run on cuBLAS (torch.matmul): a harness for
+    whole-layer step times, not part of the compressed path.  The cache is
+    still fed the workload's planted q, k, v, so that compression behaves as
+    in the headline runs; the QKV projection's output is computed and left
+    in a scratch buffer."""
+
+    def __init__(self, w, dev, seed):
+        S, Ly = w.num_seqs, w.num_layers
+        self.hid = hid = w.num_heads * w.head_dim
+        self.ffn = ffn = -(-(8 * hid) // (3 * 256)) * 256
+        dt = w.torch_dtype
+        g = torch.Generator(device=dev).manual_seed(seed * 31 + 5)
+
+        def rnd(n_in, n_out):
+            # small branch gain so 2 x layers residual adds stay finite
+            return (torch.randn(n_in, n_out, generator=g, device=dev) * (0.1 / n_in ** 0.5)).to(dt)
+
+        self.wqkv = [rnd(hid, 3 * hid) for _ in range(Ly)]
+        self.wo = [rnd(hid, hid) for _ in range(Ly)]
+        self.w13 = [rnd(hid, 2 * ffn) for _ in range(Ly)]
+        self.w2 = [rnd(ffn, hid) for _ in range(Ly)]
+        self.x0 = torch.randn(S, hid, generator=g, device=dev).to(dt)
+        self.x = torch.empty_like(self.x0)
+        self.qkv = torch.empty(S, 3 * hid, dtype=dt, device=dev)
+        self.gu = torch.empty(S, 2 * ffn, dtype=dt, device=dev)
+        self.act = torch.empty(S, ffn, dtype=dt, device=dev)
+        self.y = torch.empty(S, hid, dtype=dt, device=dev)
+        self.weight_bytes = sum(t.numel() * t.element_size()
+                                for ts in (self.wqkv, self.wo, self.w13, self.w2) for t in ts)
+
+    def flops_per_step(self, S, Ly):
+        return 2 * S * Ly * self.hid * (3 * self.hid + self.hid + 3 * self.ffn)
+
+    def pre(self, l):
+        if l == 0:
+            self.x.copy_(self.x0)  # the new token's embedding
+        torch.matmul(self.x, self.wqkv[l], out=self.qkv)
+
+    def post(self, l, o):
+        torch.matmul(o.view(o.shape[0], -1), self.wo[l], out=self.y)
+        self.x.add_(self.y)
+        torch.matmul(self.x, self.w13[l], out=self.gu)
+        gate, up = self.gu[:, : self.ffn], self.gu[:, self.ffn:]
+        torch.mul(torch.nn.functional.silu(gate), up, out=self.act)
+        torch.matmul(self.act, self.w2[l], out=self.y)
+        self.x.add_(self.y)
+
+
+def decoder_layer_arm(args, w, cache, inp, outs, pre_out, dev):
+    """Whole-layer step times, compressed and full cache, with the dense
+    work of DecoderLayers around every attention call."""
+    import kv_cache_compression_hkv_b200 as hkv
+    dense = DecoderLayers(w, dev, args.seed)
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+
+    def hooks(what, t, l):
+        if what == "decode_begin":
+            ev[0].record()
+        elif what == "decode_end":
+            ev[1].record()
+        elif what == "pre_decode":
+            dense.pre(l)
+        elif what == "post_decode":
+            dense.post(l, outs[l])
+
+    def step_us(c):
+        g = capture(lambda: run_pass(c, w, inp, outs, pre_out=pre_out, hooks=hooks))
+        for _ in range(2):
+            g.replay()
+        timed_replays(g, max(1, min(args.steps, 3)))
+        us = ev[0].elapsed_time(ev[1]) * 1e3 / w.decode_steps
+        del g
+        return us
+
+    us = step_us(cache)
+    cache_f = hkv.HeadKVCache(hkv.config_for(w, mode=hkv.MODE_FULL), device=dev)
+    us_f = step_us(cache_f)
+    out = {"hidden": dense.hid, "ffn": dense.ffn, "step_us": us, "full_step_us": us_f,
+           "speedup": us_f / us, "weight_bytes": dense.weight_bytes,
+           "kv_pool_bytes": cache.nbytes, "full_kv_pool_bytes": cache_f.nbytes,
+           "memory_saving": 1.0 - (cache.nbytes + dense.weight_bytes)
+                                  / (cache_f.nbytes + dense.weight_bytes),
+           "dense_gflop_per_step": dense.flops_per_step(w.num_seqs, w.num_layers) / 1e9}
+    del cache_f, dense
+    torch.cuda.empty_cache()
+    return out
 
 
 def e2e_arm(args, w, cache, inp, dev, world):
@@ -626,6 +730,7 @@ def main():
             "speedup_pass_vs_full": res.get("speedup_pass_vs_full"),
             "kv_pool_bytes": res["kv_pool_bytes"], "labels_local_frac": res["labels_local_frac"],
             "labels_planted": res["labels_planted"],
+            "decoder_layer": res.get("decoder_layer"),
         }
         print(json.dumps(line))
     if world > 1:
