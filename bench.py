@@ -491,6 +491,12 @@ def decoder_layer_arm(args, w, cache, inp, outs, pre_out, dev):
     work of DecoderLayers around every attention call."""
     import kv_cache_compression_hkv_b200 as hkv
     dense = DecoderLayers(w, dev, args.seed)
+    # one eager round first: cuBLAS makes its handle and workspace on first
+    # use, which a stream capture does not allow
+    for l in range(w.num_layers):
+        dense.pre(l)
+        dense.post(l, outs[l])
+    torch.cuda.synchronize()
     ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
 
     def hooks(what, t, l):
