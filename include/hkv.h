@@ -185,7 +185,13 @@ HKV_API hkv_status hkv_append(hkv_ctx* ctx, int32_t layer, const void* k_t, cons
 HKV_API hkv_status hkv_decode_attend(hkv_ctx* ctx, int32_t layer, const void* q_t, void* o_t,
                              void* stream);
 
-/* hkv_append followed by hkv_decode_attend in one kernel. */
+/* hkv_append followed by hkv_decode_attend in one kernel.
+ * Launch overlap: when the previous launch this context made on `stream`
+ * was a decode of another layer, this launch may start before the kernel
+ * in front of it has finished (programmatic dependent launch).  Before
+ * that kernel finishes it reads only this layer's cache and plan in the
+ * pool; q_t, k_t, v_t and o_t are touched after it, so a caller's kernel
+ * may produce q_t, k_t, v_t (a projection) right before the call. */
 HKV_API hkv_status hkv_decode_step(hkv_ctx* ctx, int32_t layer, const void* q_t, const void* k_t,
                            const void* v_t, void* o_t, void* stream);
 
