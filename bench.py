@@ -720,6 +720,11 @@ def main():
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{n} whole (sequence, layer) units of {w.name} in {el:.1f} s "
                          f"(one unit = 1/{w.num_seqs * w.num_layers} of a pass)"}
+        if cores > 1:
+            v1, _, n1, el1 = oracle_sample(w, args.seed, max(1.0, args.cpu_seconds / 3),
+                                           threads=1, opts=oracle_opts(args))
+            cpu["single_core"] = {"value": v1, "unit": UNIT, "cores": 1,
+                                  "sample": f"{n1} units in {el1:.1f} s"}
     if rank == 0:
         line = {
             "metric": METRIC, "value": res["tokens_per_s"], "unit": UNIT, "n_gpus": world,
