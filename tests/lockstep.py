@@ -27,12 +27,13 @@ LABEL_BAND = 1e-3
 SELECT_BAND = 1e-3
 
 
-def oracle_params(w, mode=O.MODE_HEADKV, stratified=True, cls_queries=1) -> O.UnitParams:
+def oracle_params(w, mode=O.MODE_HEADKV, stratified=True, cls_queries=1,
+                  tau=0.9) -> O.UnitParams:
     return O.UnitParams(num_heads=w.num_heads, head_dim=w.head_dim, max_len=w.max_len,
                         prefill_len=w.prefill_len, local_window=w.local_window, ste_m=w.ste_m,
                         near_dist=w.near_dist, score_window=w.score_window, rho_num=w.rho[0],
                         rho_den=w.rho[1], mode=mode, stratified=stratified,
-                        cls_queries=cls_queries,
+                        cls_queries=cls_queries, tau=tau,
                         label_band=LABEL_BAND, select_band=SELECT_BAND)
 
 
@@ -100,13 +101,13 @@ def class_rows(w, data, s, l, nq):
 
 
 def compare_unit(w, data, unit, r, mode=O.MODE_HEADKV, stratified=True, cls_queries=1,
-                 pairing=O.CFG_UNTIED):
+                 pairing=O.CFG_UNTIED, tau=0.9):
     """Replays one unit through the oracle with the GPU's decisions as hints.
     Returns (oracle result, max relative output error per decode call)."""
     s, l = unit
     q, k, v = (x[s].double().cpu().numpy() for x in data[l])
     H = w.num_heads
-    prm = oracle_params(w, mode, stratified, cls_queries)
+    prm = oracle_params(w, mode, stratified, cls_queries, tau)
     cls = None
     if pairing != O.CFG_UNTIED:
         sp = O.cfg_partner(s, data[l][0].shape[0], pairing)

@@ -96,9 +96,10 @@ def test_select_batch_bitexact(n, stratified):
 # ---------------------------------------------------------------------------
 
 def _lockstep(w, units, seed=0, fused=True, mode=hkv.MODE_HEADKV, stratified=True,
-              cls_queries=1, pairing=hkv.CFG_UNTIED):
+              cls_queries=1, pairing=hkv.CFG_UNTIED, tau=0.9, expect_label=None):
     cfg = hkv.config_for(w, mode=mode, stratified=stratified, cls_queries=cls_queries,
                          cfg_pairing=pairing)
+    cfg.tau = tau
     data = generate(w, seed, DEV)
     cache, rec, _ = run_gpu(w, cfg, data, units, fused=fused)
     rc, detail = cache.check()
@@ -107,10 +108,13 @@ def _lockstep(w, units, seed=0, fused=True, mode=hkv.MODE_HEADKV, stratified=Tru
              hkv.MODE_UNIFORM: O.MODE_UNIFORM}[mode]
     stats = []
     for u in units:
-        res, err = compare_unit(w, data, u, rec[u], omode, stratified, cls_queries, pairing)
+        res, err = compare_unit(w, data, u, rec[u], omode, stratified, cls_queries, pairing,
+                                tau)
         assert_lockstep(res, err, TOL[w.dtype], len(rec[u]["events"]))
         if mode == hkv.MODE_HEADKV:
             np.testing.assert_array_equal(res.labels, rec[u]["labels"])
+        if expect_label is not None:
+            assert (rec[u]["labels"] == expect_label).all(), rec[u]["labels"]
         stats.append(res.stats)
     return stats
 
@@ -245,6 +249,20 @@ def test_head_sharded_contexts_match_unsharded():
     n = c.prefill_label(0, q, k, v)
     c.prefill_compress(0, k, v, n + (H - len(shards[0])) + 1)
     assert c.check()[0] == 1  # HKV_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("tau,kind", [(1e-6, 1), (0.999, 0)])
+def test_every_head_one_kind(tau, kind):
+    """tau so low that every head is Local (no Global head: nG = 0, windows
+    only), or so high that every head is Global (T / H each, below the
+    prefill length: an initial eviction of E > M tokens on every head, then
+    the regular ones); the whole unit in lock step with the oracle."""
+    w = WORKLOADS["janus_pro_1b"].scaled(num_seqs=2, num_layers=1)
+    stats = _lockstep(w, [(0, 0), (1, 0)], seed=15, tau=tau, expect_label=kind)
+    if kind == 0:
+        assert all(st["n_events"] >= 2 for st in stats)
+    else:
+        assert all(st["n_events"] == 0 for st in stats)
 
 
 def test_prefill_outputs_match_oracle():
