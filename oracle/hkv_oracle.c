@@ -110,20 +110,30 @@ int hkvo_classify(const double* p_row, int32_t n, int32_t W, double tau,
     return 0;
 }
 
+int hkvo_class_row_from_weights(const double* w, int32_t P, int32_t nq, double* row)
+{
+    if (!w || !row || P <= 0 || nq < 1 || nq > P) return -1;
+    for (int32_t j = 0; j < P; ++j) row[j] = 0.0;
+    for (int32_t k = 0; k < nq; ++k) {
+        const int32_t i = P - nq + k;  /* position of the k-th query */
+        const double* wi = w + (size_t)k * P;
+        /* its weight at distance delta lands where the last query's row
+         * holds distance delta */
+        for (int32_t delta = 0; delta <= i; ++delta) row[P - 1 - delta] += wi[i - delta];
+    }
+    for (int32_t j = 0; j < P; ++j) row[j] /= (double)nq;
+    return 0;
+}
+
 int hkvo_class_row(const double* qh, const double* kh, const double* vh,
                    int32_t P, int32_t d, int32_t nq, double* row)
 {
     if (!qh || !kh || !vh || !row || P <= 0 || d <= 0 || nq < 1 || nq > P) return -1;
-    double* w = (double*)malloc(sizeof(double) * (size_t)P);
-    for (int32_t j = 0; j < P; ++j) row[j] = 0.0;
-    for (int32_t i = P - nq; i < P; ++i) {
-        /* weights of the query at position i over positions 0..i */
-        hkvo_causal_attention(qh + (size_t)i * d, kh, vh, 1, P, d, i, NULL, w);
-        /* its weight at distance delta lands where the last query's row
-         * holds distance delta */
-        for (int32_t delta = 0; delta <= i; ++delta) row[P - 1 - delta] += w[i - delta];
-    }
-    for (int32_t j = 0; j < P; ++j) row[j] /= (double)nq;
+    double* w = (double*)malloc(sizeof(double) * (size_t)P * (size_t)nq);
+    /* weights of the queries at positions P-nq .. P-1 over positions 0..P-1
+     * (0 past each query's own position) */
+    hkvo_causal_attention(qh + (size_t)(P - nq) * d, kh, vh, nq, P, d, P - nq, NULL, w);
+    hkvo_class_row_from_weights(w, P, nq, row);
     free(w);
     return 0;
 }

@@ -60,6 +60,11 @@ int hkvo_classify(const double* p_row, int32_t n, int32_t W, double tau,
 int hkvo_class_row(const double* qh, const double* kh, const double* vh,
                    int32_t P, int32_t d, int32_t nq, double* row);
 
+/* The same from given weights: w [nq][P], row k holding the weights of the
+ * query at position P-nq+k over positions 0..P-1 (only positions up to the
+ * query's own are read). */
+int hkvo_class_row_from_weights(const double* w, int32_t P, int32_t nq, double* row);
+
 /* Asymmetric budgets [Contrib/Budgets]: total T = floor(H * L * rho_num /
  * rho_den) tokens per (sequence, layer); Local heads keep W, the Global heads
  * split the rest evenly, rounded down.  budget_g = 0 when there is no Global

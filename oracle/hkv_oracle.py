@@ -69,11 +69,13 @@ def lib():
         _lib.hkvo_causal_attention.argtypes = [P, P, P, I, I, I, I, P, P]
         _lib.hkvo_classify.argtypes = [P, I, I, D, P, P, P]
         _lib.hkvo_class_row.argtypes = [P, P, P, I, I, I, P]
+        _lib.hkvo_class_row_from_weights.argtypes = [P, I, I, P]
         _lib.hkvo_budgets.argtypes = [P, I, I, I, I, I, P, P, P]
         _lib.hkvo_ste_select.argtypes = [P, P, I, I, I, I, I, I, P, P, P]
         _lib.hkvo_ste_scores.argtypes = [P, P, I, P, I, I, I, P]
         _lib.hkvo_run_unit.argtypes = [P, P, P, P, P, P]
-        for f in ("hkvo_causal_attention", "hkvo_classify", "hkvo_class_row", "hkvo_budgets",
+        for f in ("hkvo_causal_attention", "hkvo_classify", "hkvo_class_row",
+                  "hkvo_class_row_from_weights", "hkvo_budgets",
                   "hkvo_ste_select", "hkvo_ste_scores", "hkvo_run_unit"):
             getattr(_lib, f).restype = C.c_int
     return _lib
@@ -127,6 +129,16 @@ def class_row(q, k, v, nq: int = 1):
     P, d = q.shape
     row = np.zeros(P)
     _check(lib().hkvo_class_row(_p(q), _p(k), _p(v), P, d, nq, _p(row)), "class_row")
+    return row
+
+
+def class_row_from_weights(w):
+    """Classification row [P] from the weights [nq, P] of the last nq
+    queries (row k: the query at position P-nq+k)."""
+    w = _f64(w)
+    nq, P = w.shape
+    row = np.zeros(P)
+    _check(lib().hkvo_class_row_from_weights(_p(w), P, nq, _p(row)), "class_row_from_weights")
     return row
 
 

@@ -36,8 +36,8 @@ MUTANTS = {
                       "if (x->s < y->s) return 1;\n    if (x->s > y->s) return -1;"),
     "no_causal_mask": ("int32_t nvis = pos + 1 < n_k ? pos + 1 : n_k;",
                        "int32_t nvis = n_k;"),
-    "class_row_by_position": ("for (int32_t delta = 0; delta <= i; ++delta) row[P - 1 - delta] += w[i - delta];",
-                              "for (int32_t delta = 0; delta <= i; ++delta) row[i - delta] += w[i - delta];"),
+    "class_row_by_position": ("for (int32_t delta = 0; delta <= i; ++delta) row[P - 1 - delta] += wi[i - delta];",
+                              "for (int32_t delta = 0; delta <= i; ++delta) row[i - delta] += wi[i - delta];"),
     "class_row_mean_over_P": ("for (int32_t j = 0; j < P; ++j) row[j] /= (double)nq;",
                               "for (int32_t j = 0; j < P; ++j) row[j] /= (double)P;"),
     "ste_scores_ignore_step_cache": ("if (kept[i] <= step) { rows[nv] = kept[i]; where[nv] = i; ++nv; }",

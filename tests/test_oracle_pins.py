@@ -501,3 +501,22 @@ def test_unit_classifier_variants():
     with pytest.raises(ValueError):
         O.run_unit(O.UnitParams(**{**prm.__dict__, "cls_queries": prm.score_window + 1}),
                    q, k, v)
+
+
+def test_class_row_from_weights_worked_example():
+    """P = 3, the last two queries.  Query at position 1 puts 0.3, 0.7 on
+    positions 0, 1 (distances 1, 0); query at position 2 puts 0.2, 0.3, 0.5
+    on positions 0, 1, 2 (distances 2, 1, 0).  Per distance, averaged:
+    delta 0: (0.7 + 0.5) / 2 = 0.6; delta 1: (0.3 + 0.3) / 2 = 0.3;
+    delta 2: (0 + 0.2) / 2 = 0.1 (the query at 1 cannot reach distance 2).
+    In the last query's position order: [0.1, 0.3, 0.6]."""
+    w = np.array([[0.3, 0.7, 0.0], [0.2, 0.3, 0.5]])
+    np.testing.assert_allclose(O.class_row_from_weights(w), [0.1, 0.3, 0.6], atol=1e-15)
+    # the entries past a query's own position are never read
+    w2 = w.copy(); w2[0, 2] = 123.0
+    np.testing.assert_array_equal(O.class_row_from_weights(w2), O.class_row_from_weights(w))
+    # from q, k, v: the same as averaging the causal weights of those queries
+    P, d, nq = 25, 8, 6
+    q, k, v = (rng.standard_normal((P, d)) for _ in range(3))
+    _, p = O.causal_attention(q[P - nq:], k, v, q_pos0=P - nq)
+    np.testing.assert_array_equal(O.class_row(q, k, v, nq), O.class_row_from_weights(p))
