@@ -249,6 +249,23 @@ HKV_API void hkv_destroy(hkv_ctx* ctx);
 HKV_API hkv_status hkv_classify_rows(const float* rows, int32_t n_rows, int32_t n, int32_t W,
                              double tau, int32_t* n_tau, uint8_t* label, void* stream);
 
+/* Head grouping [step 2] with the averaged and tied variants, on n_units
+ * blocks of kept weight rows (fp32, [n_units][r][n]): row q of a block
+ * holds the weights of the query at position n - r + q over positions
+ * 0..n-1 (entries past that position are not read).  The weight at
+ * distance delta is the mean over the last nq queries of each query's
+ * weight on the position delta back from its own; with partner (int32
+ * [n_units], nullable) and partner[u] = p != u, unit u is grouped on the
+ * mean of its and p's values (the lower index summed first, so u and p get
+ * the same answer).  Each unit's sum over its queries runs in position
+ * order in double and is divided by nq; the pair mean is taken after.
+ * Outputs as hkv_classify_rows; a partner outside [0, n_units) gives
+ * n_tau -1 and label 255.  Requirements: 1 <= nq <= r <= n.
+ * Errors: INVALID_ARG. */
+HKV_API hkv_status hkv_classify_groups(const float* rows, int32_t n_units, int32_t r, int32_t nq,
+                                       int32_t n, const int32_t* partner, int32_t W, double tau,
+                                       int32_t* n_tau, uint8_t* label, void* stream);
+
 /* Stratified selection [step 3, STE] on n_probs independent problems.
  * Problem i has count[i] <= n tokens: score[i*n + j] (fp32, >= 0) and
  * pos[i*n + j] (int32, distinct); the newest position is t[i].  Evicts

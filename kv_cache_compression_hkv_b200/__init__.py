@@ -9,7 +9,8 @@ arguments.
 from ._lib import (  # noqa: F401
     CFG_ADJACENT, CFG_HALVES, CFG_UNTIED, DTYPE_BF16, DTYPE_F32, MODE_FULL, MODE_HEADKV,
     MODE_UNIFORM, Config, HeadKVCache, HkvError,
-    LIB_PATH, classify_rows, declared_symbols, lib, pool_bytes, ste_select_batch)
+    LIB_PATH, classify_groups, classify_rows, declared_symbols, lib, pool_bytes,
+    ste_select_batch)
 
 
 def config_for(w, mode: int = MODE_HEADKV, stratified: bool = True, num_seqs: int | None = None,

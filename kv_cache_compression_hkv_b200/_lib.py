@@ -69,6 +69,7 @@ def lib():
             "hkv_clear_error": [P, P],
             "hkv_reset": [P, P],
             "hkv_classify_rows": [P, I, I, I, D, P, P, P],
+            "hkv_classify_groups": [P, I, I, I, I, P, I, D, P, P, P],
             "hkv_ste_select_batch": [P, P, P, P, I, I, I, I, I, I, P, P],
             "hkv_prefill_classify_noalloc": [I, I, I, P, P, P, I, I64, I, D, P, P, P, P, P],
         }
@@ -299,6 +300,27 @@ class HeadKVCache:
 
     def clear_error(self, stream=None):
         _check(lib().hkv_clear_error(self.ctx, _stream(stream)), "hkv_clear_error")
+
+
+def classify_groups(rows: torch.Tensor, nq: int, W: int, tau: float = 0.9, partner=None,
+                    stream=None):
+    """Grouping of [U, r, n] fp32 kept weight rows (row q: the query at
+    position n - r + q) by the mean of the last nq queries' per-distance
+    weights, units u and partner[u] (int32 [U], optional) tied.  Returns
+    (n_tau int32 [U], label uint8 [U]) on the rows' device."""
+    if rows.dtype != torch.float32 or rows.dim() != 3 or not rows.is_cuda or \
+            not rows.is_contiguous():
+        raise ValueError("rows: expected a contiguous float32 [U, r, n] CUDA tensor")
+    U, r, n = rows.shape
+    if partner is not None and (partner.dtype != torch.int32 or partner.numel() != U or
+                                partner.device != rows.device or not partner.is_contiguous()):
+        raise ValueError("partner: expected a contiguous int32 [U] tensor on the rows' device")
+    n_tau = torch.empty(U, dtype=torch.int32, device=rows.device)
+    label = torch.empty(U, dtype=torch.uint8, device=rows.device)
+    _check(lib().hkv_classify_groups(rows.data_ptr(), U, r, nq, n, _ptr(partner), W, float(tau),
+                                     n_tau.data_ptr(), label.data_ptr(), _stream(stream)),
+           "hkv_classify_groups")
+    return n_tau, label
 
 
 def classify_rows(rows: torch.Tensor, W: int, tau: float = 0.9, stream=None):

@@ -231,6 +231,31 @@ __global__ void classify_rows_kernel(const float* __restrict__ rows, int n_rows,
     }
 }
 
+// Standalone grouping of caller weight rows, one warp per unit: unit u is
+// grouped alone or, with partner[u] = p != u, with p (the lower of the two
+// first).  A partner outside [0, n_units) marks the unit: n_tau -1, label
+// 255.
+__global__ void classify_groups_kernel(const float* __restrict__ rows, int n_units, int r, int nq,
+                                       int n, const int32_t* __restrict__ partner, int W,
+                                       double tau, int32_t* __restrict__ n_tau,
+                                       uint8_t* __restrict__ label) {
+    const int u = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (u >= n_units) return;
+    const int p = partner ? partner[u] : u;
+    if (p < 0 || p >= n_units) {
+        if ((threadIdx.x & 31) == 0) { n_tau[u] = -1; label[u] = 255; }
+        return;
+    }
+    const int a = min(u, p), b = max(u, p);
+    const size_t blk = (size_t)r * n;
+    const int need = warp_group_need_rows(rows + (size_t)a * blk,
+                                          b != a ? rows + (size_t)b * blk : nullptr, r, nq, n, tau);
+    if ((threadIdx.x & 31) == 0) {
+        n_tau[u] = need;
+        label[u] = need < W ? 1 : 0;
+    }
+}
+
 // Standalone stratified select, one warp per problem.
 __global__ void __launch_bounds__(128) select_batch_kernel(
     const float* __restrict__ score, const int32_t* __restrict__ pos, const int32_t* __restrict__ count,
@@ -283,6 +308,15 @@ cudaError_t prepare_evict(int smem) {
     if (e == cudaSuccess) e = allow_max_dynamic_smem(evict_run_kernel<float>, smem);
     if (e == cudaSuccess) e = allow_max_dynamic_smem(select_batch_kernel, smem);
     return e;
+}
+
+cudaError_t launch_classify_groups(const float* rows, int n_units, int r, int nq, int n,
+                                   const int32_t* partner, int W, double tau, int32_t* n_tau,
+                                   uint8_t* label, cudaStream_t st) {
+    const int grid = (n_units + 7) / 8;  // 8 warps per block
+    classify_groups_kernel<<<grid, 256, 0, st>>>(rows, n_units, r, nq, n, partner, W, tau, n_tau,
+                                                 label);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_classify_rows(const float* rows, int n_rows, int n, int W, double tau,

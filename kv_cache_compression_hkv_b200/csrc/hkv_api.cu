@@ -496,6 +496,17 @@ hkv_status hkv_reset(hkv_ctx* c, void* stream) {
 
 void hkv_destroy(hkv_ctx* c) { delete c; }
 
+hkv_status hkv_classify_groups(const float* rows, int32_t n_units, int32_t r, int32_t nq,
+                               int32_t n, const int32_t* partner, int32_t W, double tau,
+                               int32_t* n_tau, uint8_t* label, void* stream) {
+    if (!rows || !n_tau || !label || n_units < 0 || r < 1 || nq < 1 || nq > r || n < r || W < 1 ||
+        !(tau > 0.0 && tau <= 1.0))
+        return HKV_ERR_INVALID_ARG;
+    if (n_units == 0) return HKV_OK;
+    return cuda_status(hkv::launch_classify_groups(rows, n_units, r, nq, n, partner, W, tau, n_tau,
+                                                   label, (cudaStream_t)stream));
+}
+
 hkv_status hkv_classify_rows(const float* rows, int32_t n_rows, int32_t n, int32_t W, double tau,
                              int32_t* n_tau, uint8_t* label, void* stream) {
     if (!rows || !n_tau || !label || n_rows < 0 || n < 1 || W < 1 || !(tau > 0.0 && tau <= 1.0))

@@ -534,6 +534,47 @@ __device__ __forceinline__ int warp_tokens_to_tau(const float* row, int n, doubl
     return n;
 }
 
+// Head grouping over kept weight rows (Methodology step 2, with the
+// averaged and tied variants).  ra and rb (nullable) are [r][n] blocks of
+// fp32 weights, row q holding the query at position n - r + q over
+// positions 0..n-1.  The weight at distance delta is the mean over the last
+// nq queries i of row i's weight on position i - delta (none when
+// delta > i), per block; with rb, the mean of the two blocks' values.  Each
+// block's sum runs over the queries in position order and is divided by
+// nq, the pair's mean is halved after, all in double.  Summed newest first
+// until the total reaches tau.  All lanes of the warp call it and get the
+// number of tokens that took (n if never).
+__device__ __forceinline__ int warp_group_need_rows(const float* ra, const float* rb, int r,
+                                                    int nq, int n, double tau) {
+    const int lane = threadIdx.x & 31;
+    double carry = 0.0;
+    for (int base = 0; base < n; base += 32) {
+        const int delta = base + lane;
+        double x = 0.0;
+        if (delta < n) {
+            double xa = 0.0, xb = 0.0;
+            for (int q = r - nq; q < r; ++q) {
+                const int i = n - r + q;
+                if (delta <= i) {
+                    xa += (double)ra[(size_t)q * n + (i - delta)];
+                    if (rb) xb += (double)rb[(size_t)q * n + (i - delta)];
+                }
+            }
+            x = rb ? (xa / nq + xb / nq) * 0.5 : xa / nq;
+        }
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double y = __shfl_up_sync(FULL_MASK, x, o);
+            if (lane >= o) x += y;
+        }
+        const double c = carry + x;
+        const unsigned hit = __ballot_sync(FULL_MASK, delta < n && c >= tau);
+        if (hit) return base + __ffs(hit);  // delta = 0 .. first hit
+        carry += __shfl_sync(FULL_MASK, x, 31);
+    }
+    return n;
+}
+
 // Allows `func` as much dynamic shared memory as the device's opt-in limit
 // leaves next to its static shared memory.
 template <typename F>

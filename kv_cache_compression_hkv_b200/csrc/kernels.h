@@ -54,6 +54,9 @@ cudaError_t launch_prefill_rows_simt(int dtype, int d, int n_blocks, const void*
                                      float* rows, cudaStream_t st);
 cudaError_t launch_append(const Layout& L, int layer, const void* k, const void* v, cudaStream_t st);
 cudaError_t launch_evict(const Layout& L, int l0, int l1, int grid, cudaStream_t st);
+cudaError_t launch_classify_groups(const float* rows, int n_units, int r, int nq, int n,
+                                   const int32_t* partner, int W, double tau, int32_t* n_tau,
+                                   uint8_t* label, cudaStream_t st);
 cudaError_t launch_classify_rows(const float* rows, int n_rows, int n, int W, double tau,
                                  int32_t* n_tau, uint8_t* label, cudaStream_t st);
 cudaError_t launch_select_batch(const float* score, const int32_t* pos, const int32_t* count,

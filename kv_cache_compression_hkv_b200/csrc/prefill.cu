@@ -92,46 +92,6 @@ __device__ __forceinline__ int cfg_partner(const Layout& L, int s) {
     return s;
 }
 
-// Grouping row of head h (Methodology step 2): the weight at distance delta
-// is the mean, over the last nq prefill queries i of sequence sa and, when
-// sb != sa, of sequence sb, of query i's weight on position i - delta (none
-// when delta > i).  The kept weight rows are [s*H + h][r][P], row q holding
-// the query at position P - r + q.  Each lane owns one distance per pass;
-// the mean weights are summed newest first in double until they reach tau.
-// sa < sb fixes the order of the sums, so both streams of a pair get the
-// same count.  Returns the number of tokens that took (P if never).
-__device__ int warp_group_need(const Layout& L, int sa, int sb, int h, int P) {
-    const int lane = threadIdx.x & 31;
-    const int r = L.r, nq = L.nq;
-    const double inv = 1.0 / (double)(nq * (sb != sa ? 2 : 1));
-    double carry = 0.0;
-    for (int base = 0; base < P; base += 32) {
-        const int delta = base + lane;
-        double x = 0.0;
-        if (delta < P) {
-            for (int s = sa;; s = sb) {
-                const float* rows = L.rows + (size_t)(s * L.H + h) * r * P;
-                for (int q = r - nq; q < r; ++q) {
-                    const int i = P - r + q;
-                    if (delta <= i) x += (double)rows[(size_t)q * P + (i - delta)];
-                }
-                if (s == sb) break;
-            }
-            x *= inv;
-        }
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const double y = __shfl_up_sync(FULL_MASK, x, o);
-            if (lane >= o) x += y;
-        }
-        const double c = carry + x;
-        const unsigned hit = __ballot_sync(FULL_MASK, delta < P && c >= L.tau);
-        if (hit) return base + __ffs(hit);  // delta = 0 .. first hit
-        carry += __shfl_sync(FULL_MASK, x, 31);
-    }
-    return P;
-}
-
 // Budgets (Main contributions: asymmetric budgets) and the slot layout of
 // the heads of (layer, s) held here, from their labels lab[] and the Local
 // count nl of the whole (sequence, layer): every shard of its heads.
@@ -178,8 +138,12 @@ __global__ void classify_kernel(Layout L, int layer, int P, int32_t* n_local) {
     int need = P;
     uint8_t label = 0;
     if (L.mode == HKV_MODE_HEADKV) {
-        const int sp = cfg_partner(L, s);
-        need = warp_group_need(L, min(s, sp), max(s, sp), h, P);
+        // the pair's lower sequence first, so both streams sum alike
+        const int sp = cfg_partner(L, s), sa = min(s, sp), sb = max(s, sp);
+        const size_t blk = (size_t)L.r * P;
+        need = warp_group_need_rows(L.rows + (size_t)(sa * L.H + h) * blk,
+                                    sb != sa ? L.rows + (size_t)(sb * L.H + h) * blk : nullptr,
+                                    L.r, L.nq, P, L.tau);
         label = need < L.W ? 1 : 0;  // fewer tokens than the window: Local
     } else if (L.mode == HKV_MODE_FULL) {
         label = 2;

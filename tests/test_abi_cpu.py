@@ -99,3 +99,10 @@ def test_create_rejects_bad_pool_without_touching_the_device():
     assert L.hkv_prefill_classify(None, 0, None, None, None, 10, 640, None, None) == 1
     assert L.hkv_ste_evict(None, 0, 1, None) == 1
     assert L.hkv_ste_select_batch(None, None, None, None, 1, 8, 4, 1, 1, 1, None, None) == 1
+    assert L.hkv_prefill_label(None, 0, None, None, None, 10, 640, None, None, None) == 1
+    assert L.hkv_prefill_compress(None, 0, None, None, 10, 640, None, None) == 1
+    assert L.hkv_classify_groups(None, 4, 8, 1, 40, None, 28, 0.9, None, None, None) == 1
+    # nq above r, r above n: rejected before anything is read
+    assert L.hkv_classify_groups(0x1000, 4, 8, 9, 40, None, 28, 0.9, 0x2000, 0x3000, None) == 1
+    assert L.hkv_classify_groups(0x1000, 4, 8, 8, 7, None, 28, 0.9, 0x2000, 0x3000, None) == 1
+    assert L.hkv_classify_groups(0x1000, 0, 8, 8, 40, None, 28, 0.9, 0x2000, 0x3000, None) == 0

@@ -58,6 +58,52 @@ def test_classify_rows_bitexact():
     assert n_max < 1000
 
 
+def _weight_blocks(g, U, r, n):
+    """[U, r, n] fp32 kept weight rows: row q is a softmax over positions
+    0..n-r+q (zero after), with a per-unit mix of recency and spread so
+    that the grouping lands on both sides of tau."""
+    blocks = np.zeros((U, r, n), np.float32)
+    for u in range(U):
+        gamma = float(g.choice([0.02, 0.1, 0.3, 1.0, 3.0]))
+        for q in range(r):
+            i = n - r + q
+            logits = gamma * (np.arange(i + 1) - i) + g.standard_normal(i + 1)
+            w = np.exp(logits - logits.max())
+            blocks[u, q, : i + 1] = w / w.sum()
+    return blocks
+
+
+@pytest.mark.parametrize("n,nq", [(40, 1), (97, 4), (97, 8), (384, 8), (130, 3), (9, 8)])
+def test_classify_groups_bitexact(n, nq):
+    """Grouping by the last nq queries' per-distance weights, alone and tied
+    in pairs, on identical fp32 rows: n_tau and labels equal the oracle's
+    (averaging in the same order; only the running sum's order differs,
+    which decides nothing unless a sum lands within a few ulps of tau)."""
+    g = np.random.default_rng(n * 10 + nq)
+    U, r, W = 96, 8, 28 if n > 28 else 4
+    blocks = _weight_blocks(g, U, r, n)
+    partner = np.arange(U, dtype=np.int32)
+    partner[: U // 2] ^= 1                                   # adjacent pairs
+    partner[48:88] = 48 + (np.arange(40) + 20) % 40         # halves of the next 40
+    # the last 8 stay alone
+    for part in (None, partner):
+        nt, lab = hkv.classify_groups(torch.tensor(blocks, device=DEV), nq, W,
+                                      partner=None if part is None else torch.tensor(part, device=DEV))
+        nt, lab = nt.cpu().numpy(), lab.cpu().numpy()
+        rows = [O.class_row_from_weights(blocks[u, r - nq:].astype(np.float64)) for u in range(U)]
+        for u in range(U):
+            p = u if part is None else int(part[u])
+            row = rows[u] if p == u else O.tied_rows(rows[min(u, p)], rows[max(u, p)])
+            e_nt, e_lab, _ = O.classify(row, W, 0.9)
+            assert (nt[u], lab[u]) == (e_nt, e_lab), (u, p)
+        assert 0 < lab.sum() < U  # both kinds present
+        if part is not None:
+            assert all(nt[u] == nt[int(part[u])] for u in range(U))
+    bad = torch.tensor(np.full(U, U, np.int32), device=DEV)
+    nt, lab = hkv.classify_groups(torch.tensor(blocks, device=DEV), nq, W, partner=bad)
+    assert (nt.cpu().numpy() == -1).all() and (lab.cpu().numpy() == 255).all()
+
+
 @pytest.mark.parametrize("n,stratified", [(40, True), (230, True), (834, True), (2480, True),
                                           (230, False), (33, True), (1, True)])
 def test_select_batch_bitexact(n, stratified):
