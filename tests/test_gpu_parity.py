@@ -311,6 +311,31 @@ def test_every_head_one_kind(tau, kind):
         assert all(st["n_events"] == 0 for st in stats)
 
 
+def test_prefill_sharded_one_rank_equals_prefill_classify():
+    """dist.prefill_sharded with no process group (one rank holding every
+    head): label, its own counts, compress; the same labels, lengths and
+    kept sets as hkv_prefill_classify."""
+    from kv_cache_compression_hkv_b200 import dist
+    w = WORKLOADS["janus_pro_1b"].scaled(num_seqs=2, num_layers=1)
+    P = w.prefill_len
+    q, k, v = (x[:, :, :P] for x in generate(w, 23, DEV)[0])
+    a = hkv.HeadKVCache(hkv.config_for(w), device=DEV)
+    b = hkv.HeadKVCache(hkv.config_for(w), device=DEV)
+    a.prefill_classify(0, q, k, v)
+    n = dist.prefill_sharded(b, 0, q, k, v)
+    la, ta = a.labels(0)
+    lb, tb = b.labels(0)
+    np.testing.assert_array_equal(la, lb)
+    np.testing.assert_array_equal(ta, tb)
+    np.testing.assert_array_equal(n.cpu().numpy(), (la == 1).sum(1))
+    for x, y in zip(a.lens(0), b.lens(0)):
+        np.testing.assert_array_equal(x, y)
+    for s in range(2):
+        for h in range(w.num_heads):
+            np.testing.assert_array_equal(a.kept(s, 0, h), b.kept(s, 0, h))
+    assert a.check()[0] == 0 and b.check()[0] == 0
+
+
 def test_prefill_outputs_match_oracle():
     w = WORKLOADS["janus_pro_7b_rho6"].scaled(num_seqs=2, num_layers=1)
     cfg = hkv.config_for(w)
