@@ -4,6 +4,7 @@ import ctypes as C
 import subprocess
 
 import pytest
+import torch
 
 import kv_cache_compression_hkv_b200 as hkv
 from kv_cache_compression_hkv_b200 import build
@@ -106,3 +107,18 @@ def test_create_rejects_bad_pool_without_touching_the_device():
     assert L.hkv_classify_groups(0x1000, 4, 8, 9, 40, None, 28, 0.9, 0x2000, 0x3000, None) == 1
     assert L.hkv_classify_groups(0x1000, 4, 8, 8, 7, None, 28, 0.9, 0x2000, 0x3000, None) == 1
     assert L.hkv_classify_groups(0x1000, 0, 8, 8, 40, None, 28, 0.9, 0x2000, 0x3000, None) == 0
+
+
+def test_create_reports_a_failed_cuda_call():
+    """With no CUDA device (this host) a create whose arguments are all
+    valid fails in its first runtime call: HKV_ERR_CUDA, no context, and
+    nothing written through the pool pointer.  Only where no GPU is visible:
+    on a GPU the fake pool address would be handed to the device."""
+    if torch.cuda.is_available():
+        pytest.skip("needs a host without a visible CUDA device")
+    cfg = hkv.config_for(WORKLOADS["llamagen_1layer_f32"])
+    cc = cfg.c()
+    ctx = C.c_void_p()
+    n = hkv.pool_bytes(cfg)
+    assert hkv.lib().hkv_create(C.byref(cc), 0x100000, n, None, C.byref(ctx)) == 5
+    assert not ctx.value
