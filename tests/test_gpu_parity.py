@@ -311,6 +311,17 @@ def test_every_head_one_kind(tau, kind):
         assert all(st["n_events"] == 0 for st in stats)
 
 
+@pytest.mark.parametrize("name,W", [("llamagen_xl", 2), ("llamagen_xl", 31), ("llamagen_xl", 33),
+                                    ("janus_pro_1b", 32), ("janus_pro_1b", 33)])
+def test_local_windows_around_a_chunk(name, W):
+    """Every head Local (tau = 1e-9: with W = 2 the newest token's own
+    weight, at least ~1e-6 here, decides) with windows of 2 tokens and of
+    one 32-token chunk minus, exactly, and plus one: ring wrap-around and a
+    one-row last chunk, at d = 64 and d = 128, in lock step."""
+    w = WORKLOADS[name].scaled(num_seqs=2, num_layers=1, local_window=W)
+    _lockstep(w, [(0, 0), (1, 0)], seed=16 + W, tau=1e-9, expect_label=1)
+
+
 def test_prefill_sharded_one_rank_equals_prefill_classify():
     """dist.prefill_sharded with no process group (one rank holding every
     head): label, its own counts, compress; the same labels, lengths and
