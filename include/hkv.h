@@ -232,7 +232,8 @@ HKV_API hkv_status hkv_clear_error(hkv_ctx* ctx, void* stream);
 
 /* Starts a new generation on the same pool: enqueues the clearing of the
  * control words (positions, counters, status) on `stream` and forgets every
- * layer's classification, so prefill_classify must run again per layer.
+ * layer's classification (and a labelled layer awaiting
+ * hkv_prefill_compress), so prefill_classify must run again per layer.
  * Cache contents are not cleared (they are rewritten by the next prefill). */
 HKV_API hkv_status hkv_reset(hkv_ctx* ctx, void* stream);
 
