@@ -8,7 +8,7 @@ unit through the oracle with those decisions as hints: the oracle adopts a
 GPU decision only where its own differs by a near-tie inside the stated band,
 and counts every other difference as a hard mismatch.
 
-Bands (derivation in the design doc): fp32 logits carry an absolute error of at
+Bands: fp32 logits carry an absolute error of at
 most ~1e-4 on these inputs (sequential fp32 dot products of length <= 128),
 so softmax weights carry a relative error <= ~1e-4; labels compare
 sum-of-weights with tau (band 1e-3 absolute) and selections compare two
