@@ -122,3 +122,14 @@ def test_create_reports_a_failed_cuda_call():
     n = hkv.pool_bytes(cfg)
     assert hkv.lib().hkv_create(C.byref(cc), 0x100000, n, None, C.byref(ctx)) == 5
     assert not ctx.value
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    """No silent fallback: without libhkv.so every entry point raises."""
+    from kv_cache_compression_hkv_b200 import _lib
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", "/nonexistent/libhkv.so")
+    with pytest.raises(RuntimeError, match="libhkv.so not found"):
+        _lib.lib()
+    with pytest.raises(RuntimeError, match="libhkv.so not found"):
+        hkv.pool_bytes(hkv.config_for(WORKLOADS["llamagen_xl"]))
