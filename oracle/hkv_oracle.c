@@ -280,12 +280,15 @@ static int cmp_i32(const void* a, const void* b)
 
 /* Is the hinted eviction a valid answer once scores within `band` of each
  * other are treated as tied?  before[0..n) are the cached positions (with
- * their scores), after[0..keep) the hinted survivors. */
+ * their scores), after[0..keep) the hinted survivors.  *excess gets the
+ * largest relative amount by which an evicted score exceeds a kept score of
+ * its stratum (0 when the hint orders every stratum exactly). */
 static int hint_valid_in_band(const int32_t* before, const double* score, int32_t n,
                               const int32_t* after, int32_t keep, int32_t t,
                               int32_t D, int32_t k_near, int32_t k_far,
-                              int32_t stratified, double band)
+                              int32_t stratified, double band, double* excess)
 {
+    *excess = 0.0;
     uint8_t* gone = (uint8_t*)malloc((size_t)(n > 0 ? n : 1));
     memset(gone, 1, (size_t)n);
     int32_t found = 0;
@@ -320,6 +323,10 @@ static int hint_valid_in_band(const int32_t* before, const double* score, int32_
         }
         if (cnt != (s == 0 ? kn : kf)) ok = 0;
         else if (max_gone > min_kept * (1.0 + band)) ok = 0;
+        else if (max_gone > min_kept) {
+            const double x = (max_gone - min_kept) / min_kept;
+            if (x > *excess) *excess = x;
+        }
     }
     free(gone);
     return ok;
@@ -343,6 +350,8 @@ int hkvo_run_unit(const hkvo_unit_params* prm, const double* q,
     out->n_select = out->n_select_ties = out->n_select_hard = 0;
     out->n_events = 0;
     out->first_hard_step = -1;
+    out->max_label_tie_gap = 0.0;
+    out->max_select_tie_gap = 0.0;
 
     const int32_t nq = prm->cls_queries;
     if (nq < 1 || nq > r) return -1;
@@ -370,8 +379,11 @@ int hkvo_run_unit(const hkvo_unit_params* prm, const double* q,
         if (prm->mode == HKVO_MODE_UNIFORM) out->labels[h] = 0;
         if (prm->mode == HKVO_MODE_HEADKV && hints && hints->labels &&
             hints->labels[h] != out->labels[h]) {
-            if (fabs(out->c_window[h] - prm->tau) <= prm->label_band) ++out->n_label_ties;
-            else { ++out->n_label_hard; if (out->first_hard_step < 0) out->first_hard_step = P - 1; }
+            if (fabs(out->c_window[h] - prm->tau) <= prm->label_band) {
+                ++out->n_label_ties;
+                if (fabs(out->c_window[h] - prm->tau) > out->max_label_tie_gap)
+                    out->max_label_tie_gap = fabs(out->c_window[h] - prm->tau);
+            } else { ++out->n_label_hard; if (out->first_hard_step < 0) out->first_hard_step = P - 1; }
             out->labels[h] = hints->labels[h];
         }
     }
@@ -444,11 +456,13 @@ int hkvo_run_unit(const hkvo_unit_params* prm, const double* q,
                 int same = nk == (target_);                                     \
                 for (int32_t i = 0; same && i < nk; ++i) same = tmp[i] == g[i]; \
                 if (!same) {                                                    \
+                    double xs = 0.0;                                            \
                     if (hint_valid_in_band(S->kept, sc, S->len, g, (target_), et, D, \
                                            (kn_), (kf_), prm->stratified,       \
-                                           prm->select_band))                   \
+                                           prm->select_band, &xs)) {            \
                         ++out->n_select_ties;                                   \
-                    else {                                                      \
+                        if (xs > out->max_select_tie_gap) out->max_select_tie_gap = xs; \
+                    } else {                                                    \
                         ++out->n_select_hard;                                   \
                         if (out->first_hard_step < 0) out->first_hard_step = et; \
                     }                                                           \

@@ -147,6 +147,10 @@ typedef struct {
     int32_t n_label_ties, n_label_hard;
     int32_t n_select, n_select_ties, n_select_hard;
     int32_t first_hard_step;  /* -1 if none */
+    double max_label_tie_gap;  /* largest |c_window - tau| of an adopted label */
+    double max_select_tie_gap; /* largest relative excess of an evicted score
+                                  over a kept one of its stratum in an
+                                  adopted selection */
 } hkvo_unit_out;
 
 /* Whole hot path for one (sequence, layer) unit [Method/Prefill] ..

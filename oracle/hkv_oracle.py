@@ -56,7 +56,8 @@ class _UnitOut(C.Structure):
                 ("evicted", C.c_void_p), ("evicted_stride", C.c_int32)] + [
         (n, C.c_int32) for n in (
             "n_local", "budget_g", "cap_g", "n_events", "n_label_ties", "n_label_hard",
-            "n_select", "n_select_ties", "n_select_hard", "first_hard_step")]
+            "n_select", "n_select_ties", "n_select_hard", "first_hard_step")] + [
+        ("max_label_tie_gap", C.c_double), ("max_select_tie_gap", C.c_double)]
 
 
 def lib():
@@ -271,7 +272,9 @@ def run_unit(prm: UnitParams, q, k, v, hints: dict | None = None,
         n_local=out.n_local, budget_g=out.budget_g, cap_g=out.cap_g,
         stats=dict(n_events=ne, n_label_ties=out.n_label_ties, n_label_hard=out.n_label_hard,
                    n_select=out.n_select, n_select_ties=out.n_select_ties,
-                   n_select_hard=out.n_select_hard, first_hard_step=out.first_hard_step))
+                   n_select_hard=out.n_select_hard, first_hard_step=out.first_hard_step,
+                   max_label_tie_gap=out.max_label_tie_gap,
+                   max_select_tie_gap=out.max_select_tie_gap))
 
 
 CFG_UNTIED, CFG_HALVES, CFG_ADJACENT = 0, 1, 2

@@ -16,6 +16,8 @@ scores (band 1e-3 relative).
 """
 from __future__ import annotations
 
+import json
+
 import numpy as np
 import torch
 
@@ -132,8 +134,22 @@ def compare_unit(w, data, unit, r, mode=O.MODE_HEADKV, stratified=True, cls_quer
     return res, err
 
 
-def assert_lockstep(res, err, tol, n_events_gpu):
+def tie_report(res, err, unit=None) -> dict:
+    """How many GPU decisions the oracle took inside a band, and how close
+    the closest call was: the adoption counts, the largest |C(W-1) - tau| of
+    an adopted label and the largest relative score excess of an adopted
+    selection (0 when every adopted answer ordered its strata exactly)."""
     st = res.stats
+    return {"unit": list(unit) if unit is not None else None,
+            "labels": int(len(res.labels)), "label_ties": st["n_label_ties"],
+            "selects": st["n_select"], "select_ties": st["n_select_ties"],
+            "max_label_gap": st["max_label_tie_gap"], "max_select_gap": st["max_select_tie_gap"],
+            "events": st["n_events"], "max_err": float(err.max()) if len(err) else 0.0}
+
+
+def assert_lockstep(res, err, tol, n_events_gpu, unit=None):
+    st = res.stats
+    print("lockstep", json.dumps(tie_report(res, err, unit)))
     assert st["n_label_hard"] == 0, st
     assert st["n_select_hard"] == 0, st
     assert st["n_events"] == n_events_gpu, (st, n_events_gpu)

@@ -156,7 +156,7 @@ def _lockstep(w, units, seed=0, fused=True, mode=hkv.MODE_HEADKV, stratified=Tru
     for u in units:
         res, err = compare_unit(w, data, u, rec[u], omode, stratified, cls_queries, pairing,
                                 tau)
-        assert_lockstep(res, err, TOL[w.dtype], len(rec[u]["events"]))
+        assert_lockstep(res, err, TOL[w.dtype], len(rec[u]["events"]), unit=(w.name,) + u)
         if mode == hkv.MODE_HEADKV:
             np.testing.assert_array_equal(res.labels, rec[u]["labels"])
         if expect_label is not None:
@@ -171,8 +171,8 @@ def test_llamagen_1layer_f32_full_config():
     assert stats[0]["n_events"] >= 1 and stats[0]["n_select"] > 0
 
 
-@pytest.mark.parametrize("name", ["llamagen_xl", "janus_pro_1b", "janus_pro_7b_rho6",
-                                  "janus_pro_7b_rho8", "lumina_mgpt_768"])
+@pytest.mark.parametrize("name", ["llamagen_xl", "janus_pro_1b", "janus_pro_7b_rho4",
+                                  "janus_pro_7b_rho6", "janus_pro_7b_rho8", "lumina_mgpt_768"])
 def test_lockstep_scaled_stacks(name):
     """Every shape of the stacks, full sequence length, few sequences/layers."""
     w = WORKLOADS[name]

@@ -40,6 +40,12 @@ MUTANTS = {
                               "for (int32_t delta = 0; delta <= i; ++delta) row[i - delta] += wi[i - delta];"),
     "class_row_mean_over_P": ("for (int32_t j = 0; j < P; ++j) row[j] /= (double)nq;",
                               "for (int32_t j = 0; j < P; ++j) row[j] /= (double)P;"),
+    "select_band_absolute": ("else if (max_gone > min_kept * (1.0 + band)) ok = 0;",
+                             "else if (max_gone - min_kept > band) ok = 0;"),
+    "select_band_wrong_side": ("else if (max_gone > min_kept * (1.0 + band)) ok = 0;",
+                               "else if (max_gone > min_kept * (1.0 - band)) ok = 0;"),
+    "label_band_one_sided": ("if (fabs(out->c_window[h] - prm->tau) <= prm->label_band) {",
+                             "if (out->c_window[h] - prm->tau <= prm->label_band) {"),
     "ste_scores_ignore_step_cache": ("if (kept[i] <= step) { rows[nv] = kept[i]; where[nv] = i; ++nv; }",
                                      "{ rows[nv] = kept[i]; where[nv] = i; ++nv; }"),
 }

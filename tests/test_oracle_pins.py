@@ -386,6 +386,99 @@ def test_hints_adopt_only_near_ties():
     assert res.stats["n_label_hard"] == 1
 
 
+def _event_states(prm, res):
+    """Cached positions of every Global head just before each event of an
+    oracle run (from its labels, event steps and evicted logs)."""
+    H, P = prm.num_heads, prm.prefill_len
+    state = {h: set(range(P)) for h in range(H) if res.labels[h] == 0}
+    last, before = P - 1, []
+    for e, t in enumerate(res.event_step.tolist()):
+        for h in state:
+            state[h] |= set(range(last + 1, t + 1))
+        before.append({h: sorted(x) for h, x in state.items()})
+        for h in state:
+            state[h] -= {x for x in res.evicted[e, h] if x >= 0}
+        last = t
+    return before
+
+
+def _scores_numpy(q, k, kept, t, r):
+    """STE scores written out with numpy: for each of the last r steps, the
+    softmax (scale 1/sqrt(d)) of that step's query over the cached keys not
+    newer than the step, summed per key."""
+    kept = np.asarray(kept)
+    s = np.zeros(kept.size)
+    for step in range(t - r + 1, t + 1):
+        vis = kept <= step
+        x = k[kept[vis]] @ q[step] / np.sqrt(q.shape[1])
+        w = np.exp(x - x.max())
+        s[vis] += w / w.sum()
+    return s
+
+
+def test_hints_adopt_inside_the_band_and_only_there():
+    """The near-tie band is relative and two-sided in the right direction:
+    a hint that keeps the highest-scored evicted token g of a stratum and
+    evicts the lowest-scored kept token c in its place exceeds the exact
+    answer by x = (s_c - s_g) / s_g; with band 1.01 x it is
+    adopted as a tie, with band 0.99 x it is a hard mismatch.  Scores are
+    well below 1, so an absolute band (s_c - s_g <= band) would adopt the
+    second one, and a band on the wrong side (s_c <= s_g (1 - band)) would
+    reject the first.  A flipped label is adopted exactly when
+    |C(W-1) - tau| is inside its band, on either side of tau."""
+    prm, q, k, v = _small_unit(seed=11)
+    base = O.run_unit(prm, q, k, v)
+    H, E = prm.num_heads, len(base.event_step)
+    assert E >= 2
+    before = _event_states(prm, base)
+    kept_log = np.full((E, H, base.budget_g), -1, np.int32)
+    for e in range(E):
+        for h in before[e]:
+            gone = {x for x in base.evicted[e, h] if x >= 0}
+            kept_log[e, h] = sorted(set(before[e][h]) - gone)
+    hints = {"labels": base.labels, "event_step": base.event_step, "kept": kept_log}
+    # the swap goes into the last event, so no later event sees its effect
+    e, t = E - 1, int(base.event_step[-1])
+    cases = []
+    for h in before[e]:
+        cached = np.array(before[e][h])
+        sc = _scores_numpy(q[h], k[h], cached, t, prm.score_window)
+        gone = {x for x in base.evicted[e, h] if x >= 0}
+        far = (t - cached) > prm.near_dist
+        ev = np.array([p in gone for p in cached])
+        if not (far & ev).any() or not (far & ~ev).any():
+            continue
+        ig = np.flatnonzero(far & ev)[np.argmax(sc[far & ev])]
+        ic = np.flatnonzero(far & ~ev)[np.argmin(sc[far & ~ev])]
+        x = (sc[ic] - sc[ig]) / sc[ig]
+        if x > 1e-9:
+            cases.append((x, h, int(cached[ig]), int(cached[ic]), sc[ig]))
+    assert cases
+    x, h, pg, pc, sg = min(cases)
+    assert sg < 0.5  # an absolute band would differ from the relative one here
+    swapped = kept_log.copy()
+    row = [p for p in swapped[e, h] if p != pc] + [pg]
+    swapped[e, h] = np.sort(row)
+    for factor, ties, hard in ((1.01, 1, 0), (0.99, 0, 1)):
+        prm_b = O.UnitParams(**{**prm.__dict__, "select_band": x * factor})
+        res = O.run_unit(prm_b, q, k, v, hints={**hints, "kept": swapped})
+        assert (res.stats["n_select_ties"], res.stats["n_select_hard"]) == (ties, hard), factor
+        if ties:
+            assert res.stats["max_select_tie_gap"] == pytest.approx(x, rel=1e-9)
+            assert sorted(res.kept_final[h]) == sorted(set(swapped[e, h]) | set(range(t + 1, prm.max_len)))
+    # labels: the head closest to tau above it and below it
+    gap = base.c_window - prm.tau
+    for side in (gap > 0, gap < 0):
+        hh = int(np.flatnonzero(side)[np.argmin(np.abs(gap[side]))])
+        lab = base.labels.copy()
+        lab[hh] ^= 1
+        for factor, ties, hard in ((1.01, 1, 0), (0.99, 0, 1)):
+            prm_b = O.UnitParams(**{**prm.__dict__, "label_band": abs(gap[hh]) * factor})
+            res = O.run_unit(prm_b, q, k, v, hints={"labels": lab})
+            assert (res.stats["n_label_ties"], res.stats["n_label_hard"]) == (ties, hard), (hh, factor)
+            assert res.labels[hh] == lab[hh]
+
+
 # --------------------------------------------------------------------------
 # classifier variants: distance-averaged rows, CFG-tied rows
 # --------------------------------------------------------------------------
