@@ -19,19 +19,35 @@ def rank_seed(seed: int, rank: int) -> int:
     return seed + 1000 * rank
 
 
-def shard_sequences(num_seqs: int, world: int, rank: int, cfg_pairs: bool = True) -> range:
-    """Contiguous range of the sequences a rank owns.  With cfg_pairs the
-    conditional and unconditional halves of an image (sequences 2i, 2i+1)
-    stay on one rank."""
+def shard_sequences(num_seqs: int, world: int, rank: int, pairing: int = 2) -> list[int]:
+    """The sequences a rank owns, in the order its own batch should hold
+    them.  The images are split into contiguous, balanced ranges, and both
+    streams of an image (its conditional and unconditional sequence under
+    classifier-free guidance) stay on one rank, laid out as the pairing
+    says (the values of hkv_cfg_pairing):
+      0 untied:   no pairs; a contiguous range of sequences;
+      1 halves:   the batch is [conditional | unconditional], s pairs with
+                  s + S/2; the rank gets images [lo, hi) as
+                  [lo..hi) + [lo+S/2..hi+S/2), so its own batch is again
+                  [conditional | unconditional] (pairing halves locally);
+      2 adjacent: streams alternate, 2i pairs with 2i+1; the rank gets the
+                  contiguous sequences [2 lo, 2 hi) (pairing adjacent
+                  locally)."""
     if world < 1 or not 0 <= rank < world:
         raise ValueError("bad rank/world")
-    unit = 2 if cfg_pairs else 1
-    if num_seqs % unit:
+    if pairing not in (0, 1, 2):
+        raise ValueError(f"unknown CFG pairing {pairing}")
+    if pairing and num_seqs % 2:
         raise ValueError("CFG pairs need an even number of sequences")
-    n_units = num_seqs // unit
+    n_units = num_seqs // 2 if pairing else num_seqs
     lo = n_units * rank // world
     hi = n_units * (rank + 1) // world
-    return range(lo * unit, hi * unit)
+    if pairing == 0:
+        return list(range(lo, hi))
+    if pairing == 2:
+        return list(range(2 * lo, 2 * hi))
+    half = num_seqs // 2
+    return list(range(lo, hi)) + list(range(lo + half, hi + half))
 
 
 def max_over_ranks(x: float, device=None) -> float:

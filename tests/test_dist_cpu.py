@@ -20,9 +20,10 @@ def _worker(rank, world, port, q):
     torch.distributed.init_process_group("gloo", rank=rank, world_size=world)
     try:
         mx = dist.max_over_ranks(10.0 + rank * 3.5)
-        mine = list(dist.shard_sequences(64, world, rank))
+        mine = dist.shard_sequences(64, world, rank)
+        halves = dist.shard_sequences(64, world, rank, pairing=1)
         got = [None] * world
-        torch.distributed.all_gather_object(got, mine)
+        torch.distributed.all_gather_object(got, (mine, halves))
         q.put((rank, mx, got, dist.rank_seed(7, rank)))
     finally:
         torch.distributed.destroy_process_group()
@@ -42,23 +43,52 @@ def test_two_gloo_ranks():
     seeds = set()
     for rank, mx, shards, seed in res:
         assert mx == 13.5  # max over both ranks
-        flat = sorted(x for s in shards for x in s)
-        assert flat == list(range(64))  # every sequence exactly once
-        for s in shards:
-            assert all(x % 2 == 0 for x in s[::2]) and len(s) % 2 == 0  # CFG pairs intact
+        for which in range(2):
+            flat = sorted(x for s in shards for x in s[which])
+            assert flat == list(range(64))  # every sequence exactly once
+        for adj, halves in shards:
+            assert all(x % 2 == 0 for x in adj[::2]) and len(adj) % 2 == 0  # pairs intact
+            n = len(halves) // 2
+            assert all(halves[j] + 32 == halves[j + n] for j in range(n))
         seeds.add(seed)
     assert len(seeds) == 2
 
 
 def test_shard_sequences_edges():
-    assert list(dist.shard_sequences(2, 1, 0)) == [0, 1]
+    assert dist.shard_sequences(2, 1, 0) == [0, 1]
     assert [len(dist.shard_sequences(16, 3, r)) for r in range(3)] == [4, 6, 6]
-    assert list(dist.shard_sequences(5, 2, 1, cfg_pairs=False)) == [2, 3, 4]
+    assert dist.shard_sequences(5, 2, 1, pairing=0) == [2, 3, 4]
     with pytest.raises(ValueError):
         dist.shard_sequences(5, 2, 0)
     with pytest.raises(ValueError):
         dist.shard_sequences(8, 2, 2)
+    with pytest.raises(ValueError):
+        dist.shard_sequences(8, 2, 0, pairing=3)
     assert dist.max_over_ranks(3.0) == 3.0  # no process group
+
+
+@pytest.mark.parametrize("S,world", [(16, 3), (64, 2), (2, 1), (32, 8), (10, 4)])
+def test_shard_sequences_keep_cfg_halves_together(S, world):
+    """A [conditional | unconditional] batch (s pairs with s + S/2, the
+    library's HKV_CFG_HALVES): every pair lands on one rank, and the rank's
+    own batch is again [conditional | unconditional], so a context made
+    for it with the same pairing ties the same two streams."""
+    from oracle import hkv_oracle as O
+    owner = {}
+    for r in range(world):
+        mine = dist.shard_sequences(S, world, r, pairing=1)
+        n = len(mine)
+        assert n % 2 == 0
+        for j, s in enumerate(mine):
+            owner[s] = r
+            # local partner under the same pairing is the global partner
+            jp = O.cfg_partner(j, n, O.CFG_HALVES)
+            assert mine[jp] == O.cfg_partner(s, S, O.CFG_HALVES)
+    assert sorted(owner) == list(range(S))
+    assert all(owner[s] == owner[O.cfg_partner(s, S, O.CFG_HALVES)] for s in range(S))
+    for r in range(world):  # adjacent pairing: 2i and 2i+1 together, locally adjacent
+        mine = dist.shard_sequences(S, world, r, pairing=2)
+        assert all(mine[j] ^ 1 == mine[j ^ 1] for j in range(len(mine)))
 
 
 class _ShardCache:
