@@ -298,10 +298,17 @@ HKV_API hkv_status hkv_ste_select_batch(const float* score, const int32_t* pos, 
  *            of the last query's weights needs to reach tau.
  *  label:    uint8[n_blocks] device output: 1 (Local) iff n_tau < local_window.
  *  status:   int32[2] device output (nullable): zeroed, then a device-side
- *            fault (HKV_ERR_TIMEOUT, block index) if one occurs.
+ *            fault (HKV_ERR_TIMEOUT, block index) if one occurs.  A block
+ *            whose bounded wait gave up leaves its n_tau and label computed
+ *            from stale scratch, so a caller that passes NULL here cannot
+ *            tell a timed-out call from a good one: pass a status buffer
+ *            and read it.
  * Scratch: a fixed 8 MiB array inside the library, present on every GPU that
  * loads it until the process exits.  Limit: n_blocks * prefill_len <=
  * 2,097,088; larger calls return HKV_ERR_CAPACITY and enqueue nothing.  The
+ * fp32 path also needs prefill_len <= 12,288 (its attention kernel stages
+ * 16 * (head_dim + prefill_len) bytes of shared memory); longer fp32 calls
+ * return HKV_ERR_INVALID_ARG and enqueue nothing.  The
  * first call on a device looks the array's address up and sets kernel
  * attributes (host-side work): make it before any stream capture.  Every
  * call reuses the same array, so calls that overlap on the GPU (other

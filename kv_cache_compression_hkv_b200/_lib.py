@@ -358,11 +358,18 @@ def prefill_classify_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, 
     with unit stride in d, stride d in P and evenly spaced blocks.  Returns
     (n_tau int32, label uint8, status int32[2]) device tensors; the caller's
     tensors here are the outputs it passes."""
+    if q.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("q, k, v: float32 or bfloat16 only")
     d, P = q.shape[-1], q.shape[-2]
     nb = q.numel() // (P * d) if q.is_contiguous() else int(np.prod(q.shape[:-2]))
     for x in (q, k, v):
+        if not x.is_cuda or x.device != q.device or x.dtype != q.dtype:
+            raise ValueError("q, k, v: CUDA tensors of one dtype on one device")
         if x.stride(-1) != 1 or x.stride(-2) != d or x.shape != q.shape or x.stride() != q.stride():
             raise ValueError("q, k, v: unsupported layout")
+    if out is not None and (out.dtype != q.dtype or out.device != q.device or
+                            not out.is_contiguous() or out.numel() != nb * P * d):
+        raise ValueError("out: a contiguous tensor of q's dtype and device with n_blocks*P*d elements")
     bs = q.stride(-3) if q.dim() >= 3 else P * d
     if q.dim() == 4 and q.stride(0) != q.shape[1] * q.stride(1):
         raise ValueError("q, k, v: blocks must be evenly spaced")

@@ -10,6 +10,8 @@
 // the surviving tail tokens into the holes below the budget.
 #include <math.h>
 
+#include <mutex>
+
 #include "hkv_internal.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
@@ -339,18 +341,24 @@ cudaError_t launch_select_batch(const float* score, const int32_t* pos, const in
 }
 
 cudaError_t prepare_kernels() {
-    // Every kernel may use up to the device's opt-in shared memory; set once
-    // per process (a host-side attribute call, kept out of stream captures).
-    static cudaError_t done = cudaErrorNotReady;
-    if (done == cudaSuccess) return done;
+    // Every kernel may use up to the device's opt-in shared memory.  The
+    // attribute belongs to the current device, so the latch is kept per
+    // device (a host-side attribute call, kept out of stream captures).
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static bool done[kMaxDevices] = {};
     int dev = 0, optin = 0;
     cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done[dev]) return cudaSuccess;
+    e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e == cudaSuccess) e = prepare_prefill(optin);
     if (e == cudaSuccess) e = prepare_prefill_umma(optin);
     if (e == cudaSuccess) e = prepare_decode(optin);
     if (e == cudaSuccess) e = prepare_evict(optin);
-    done = e;
+    if (e == cudaSuccess) done[dev] = true;
     return e;
 }
 

@@ -23,6 +23,9 @@ namespace {
 constexpr size_t kScratchBytes = size_t(8) << 20;
 constexpr size_t kStatusBytes = 256;
 constexpr size_t kMaxWeights = (kScratchBytes - kStatusBytes) / sizeof(float);
+// Longest prefill of the fp32 path: its attention kernel stages 16 (d + P)
+// bytes of shared memory per block (198,656 bytes at d = 128).
+constexpr int kMaxPrefillF32 = 12288;
 
 static __device__ __align__(256) unsigned char hkv_noalloc_scratch[kScratchBytes];
 
@@ -62,6 +65,7 @@ extern "C" hkv_status hkv_prefill_classify_noalloc(int32_t dtype, int32_t head_d
     const int64_t es = dtype == HKV_DTYPE_F32 ? 4 : 2;
     if (block_stride < (int64_t)P * head_dim || (block_stride * es) % 16 != 0) return HKV_ERR_INVALID_ARG;
     if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)out) & 15) return HKV_ERR_INVALID_ARG;
+    if (dtype == HKV_DTYPE_F32 && P > kMaxPrefillF32) return HKV_ERR_INVALID_ARG;
     if ((size_t)n_blocks * (size_t)P > kMaxWeights) return HKV_ERR_CAPACITY;  // beyond the array
     void* base = nullptr;
     hkv_status s = scratch_address(&base);

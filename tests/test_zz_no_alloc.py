@@ -1,4 +1,5 @@
-"""The allocation-free entry point against the context-based one.
+"""The allocation-free entry point against the context-based one and the
+oracle.
 
 hkv_prefill_classify_noalloc serves callers that cannot allocate device
 memory (not even the pool hkv_create needs): during a global-mode graph
@@ -15,6 +16,7 @@ import torch
 import kv_cache_compression_hkv_b200 as hkv
 from kv_cache_compression_hkv_b200 import _lib
 from kv_cache_compression_hkv_b200.inputs import WORKLOADS, generate_layer
+from oracle import hkv_oracle as O
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
@@ -57,6 +59,31 @@ def test_noalloc_matches_context_path_two_calls(name):
         np.testing.assert_array_equal(n_tau.cpu().numpy(), ref_ntau, err_msg=f"call {call}")
         err = (out.double() - ref_out.double()).abs().max() / ref_out.double().abs().max()
         assert float(err) <= tol, (call, float(err))
+        _check_against_oracle(w, q, k, v, out, n_tau, label, tol)
+
+
+def _check_against_oracle(w, q, k, v, out, n_tau, label, tol):
+    """Every block against the oracle's causal attention and grouping of
+    the last query's weights on the same bits: outputs within tol, labels
+    equal unless the sum of the W-1 newest weights lies within 1e-3 of tau,
+    n_tau equal unless a running sum next to the boundary does."""
+    P, W = w.prefill_len, w.local_window
+    S, H = q.shape[0], q.shape[1]
+    got_out = out.double().cpu().numpy().reshape(S, H, P, -1)
+    nt, lab = n_tau.cpu().numpy().reshape(S, H), label.cpu().numpy().reshape(S, H)
+    for s in range(S):
+        for h in range(H):
+            qq, kk, vv = (x[s, h, :P].double().cpu().numpy() for x in (q, k, v))
+            o, p = O.causal_attention(qq, kk, vv)
+            err = np.abs(got_out[s, h] - o).max() / np.abs(o).max()
+            assert err <= tol, (s, h, err)
+            e_nt, e_lab, cw = O.classify(p[-1], W, 0.9)
+            if abs(cw - 0.9) > 1e-3:
+                assert lab[s, h] == e_lab, (s, h, cw)
+            c = np.cumsum(p[-1][::-1])
+            near = [abs(c[i] - 0.9) <= 1e-3 for i in (e_nt - 2, e_nt - 1) if 0 <= i < P]
+            if not any(near):
+                assert nt[s, h] == e_nt, (s, h)
 
 
 def test_noalloc_rejects_sizes_beyond_its_array():
@@ -68,3 +95,10 @@ def test_noalloc_rejects_sizes_beyond_its_array():
         hkv.DTYPE_BF16, 64, too_many_blocks, x.data_ptr(), x.data_ptr(), x.data_ptr(), 16, 16 * 64,
         8, 0.9, None, n_tau.data_ptr(), label.data_ptr(), None, None)
     assert rc == 3  # HKV_ERR_CAPACITY, nothing enqueued
+    # the fp32 path's shared memory bounds its prefill length
+    xf = torch.zeros(1, 16, 64, dtype=torch.float32, device=DEV)
+    P = 12289
+    rc = _lib.lib().hkv_prefill_classify_noalloc(
+        hkv.DTYPE_F32, 64, 1, xf.data_ptr(), xf.data_ptr(), xf.data_ptr(), P, P * 64,
+        8, 0.9, None, n_tau.data_ptr(), label.data_ptr(), None, None)
+    assert rc == 1  # HKV_ERR_INVALID_ARG, nothing enqueued
