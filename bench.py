@@ -42,7 +42,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="llamagen_xl")
+    ap.add_argument("--workload", default="lumina_mgpt_768",
+                    help="the headline workload (default: the largest single-GPU shape)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-full", action="store_true", help="skip the full-cache comparator")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end arm")
@@ -55,9 +56,11 @@ def parse_args():
                     help="group heads by the last n prefill queries' per-distance weights")
     ap.add_argument("--cfg-pairing", default="untied", choices=list(PAIRINGS),
                     help="group the two streams of a CFG pair by their mean row")
-    ap.add_argument("--decoder-layer", action="store_true",
-                    help="also time whole decoder layers (projections + MLP on random "
-                         "weights around each attention call), compressed and full cache")
+    ap.add_argument("--no-decoder-layer", action="store_true",
+                    help="skip whole decoder layers (projections + MLP on random weights "
+                         "around each attention call), compressed and full cache")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the shorter runs of every other workload (all_configs)")
     ap.add_argument("--profile", action="store_true",
                     help="eager run of a reduced workload for ncu captures (no timing line)")
     ap.add_argument("--seqs", type=int, default=None, help="override the workload's sequences")
@@ -170,6 +173,8 @@ class ClockSampler:
         self.proc = None
 
     def __enter__(self):
+        if self.index is None:  # not sampled
+            return self
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
@@ -292,11 +297,12 @@ def timed_replays(g, n):
     return e0.elapsed_time(e1) / n  # ms per replay
 
 
-def gpu_arm(args, rank, world, dev):
+def gpu_arm(args, rank, world, dev, w, lite=False):
+    """The timed GPU arm on workload w.  lite: the shorter run of the sweep
+    (one warm-up and two timed passes, the full-cache comparator on one
+    timed pass, no end-to-end or decoder-layer arm, no clock sampling)."""
     import kv_cache_compression_hkv_b200 as hkv
-    from kv_cache_compression_hkv_b200.inputs import WORKLOADS
 
-    w = WORKLOADS[args.workload]
     S, H, d, Ly = w.num_seqs, w.num_heads, w.head_dim, w.num_layers
     es = 2 if w.dtype == "bf16" else 4
     steps = w.decode_steps
@@ -326,14 +332,14 @@ def gpu_arm(args, rank, world, dev):
             ev_dec[1].record()
 
     g_main = capture(lambda: run_pass(cache, w, inp, outs, pre_out=pre_out, hooks=hooks_main))
-    for _ in range(args.warmup):
+    for _ in range(1 if lite else args.warmup):
         g_main.replay()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(gpu_id(dev)) as clk:
-        ms = timed_replays(g_main, args.steps)
+    with ClockSampler(None if lite else gpu_id(dev)) as clk:
+        ms = timed_replays(g_main, 2 if lite else args.steps)
         decode_ms = ev_dec[0].elapsed_time(ev_dec[1])
     if world > 1:
         ms = dist.max_over_ranks(ms, dev)
@@ -370,7 +376,7 @@ def gpu_arm(args, rank, world, dev):
     achieved = float(alg.sum() / (dec_us.sum() * 1e-6) / 1e9)
     del g_prof
 
-    traffic_ratio = decode_traffic_ratio()
+    traffic_ratio = decode_traffic_ratio(w.name)
     peaks = {}
     pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(pk):
@@ -408,9 +414,9 @@ def gpu_arm(args, rank, world, dev):
         cache_f = hkv.HeadKVCache(hkv.config_for(w, mode=hkv.MODE_FULL), device=dev)
         g_full = capture(lambda: run_pass(cache_f, w, inp, outs, pre_out=pre_out,
                                           hooks=hooks_main))
-        for _ in range(2):
+        for _ in range(1 if lite else 2):
             g_full.replay()
-        ms_f = timed_replays(g_full, max(1, min(args.steps, 3)))
+        ms_f = timed_replays(g_full, 1 if lite else max(1, min(args.steps, 3)))
         dec_f = ev_dec[0].elapsed_time(ev_dec[1])
         res["full"] = {"ms_per_step": ms_f, "decode_step_us": dec_f * 1e3 / steps,
                        "kv_pool_bytes": cache_f.nbytes}
@@ -419,13 +425,38 @@ def gpu_arm(args, rank, world, dev):
         del g_full, cache_f
         torch.cuda.empty_cache()
 
-    if args.decoder_layer:
+    if not lite and not args.no_decoder_layer:
         res["decoder_layer"] = decoder_layer_arm(args, w, cache, inp, outs, pre_out, dev)
 
     # end to end through the C ABI from pinned host buffers
-    if not args.no_e2e:
+    if not lite and not args.no_e2e:
         res["e2e"] = e2e_arm(args, w, cache, inp, dev, world)
     return res
+
+
+def sweep_arm(args, dev, skip):
+    """Shorter runs of every workload but `skip` (one warm-up, two timed
+    passes each, with the full-cache comparator): image tokens/s, decode
+    step and launch, roofline fraction and speedup over full per workload."""
+    from kv_cache_compression_hkv_b200.inputs import WORKLOADS
+    out = {}
+    for name, w in WORKLOADS.items():
+        if name == skip:
+            continue
+        r = gpu_arm(args, 0, 1, dev, w, lite=True)
+        out[name] = {
+            "value": r["tokens_per_s"], "ms_per_step": r["ms_per_step"],
+            "decode_step_us": r["decode_step_us"],
+            "launch_us_avg": r["roofline"]["launch_us_avg"],
+            "roofline_frac": r["roofline"]["frac"],
+            "evict_us_avg": r["evict_us_avg"], "evict_us_max": r["evict_us_max"],
+            "full_decode_step_us": (r.get("full") or {}).get("decode_step_us"),
+            "speedup_decode_vs_full": r.get("speedup_decode_vs_full"),
+            "kv_pool_bytes": r["kv_pool_bytes"],
+            "full_kv_pool_bytes": (r.get("full") or {}).get("kv_pool_bytes"),
+            "labels_local_frac": r["labels_local_frac"]}
+        torch.cuda.empty_cache()
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -511,9 +542,8 @@ def decoder_layer_arm(args, w, cache, inp, outs, pre_out, dev):
 
     def step_us(c):
         g = capture(lambda: run_pass(c, w, inp, outs, pre_out=pre_out, hooks=hooks))
-        for _ in range(2):
-            g.replay()
-        timed_replays(g, max(1, min(args.steps, 3)))
+        g.replay()
+        timed_replays(g, max(1, min(args.steps, 2)))
         us = ev[0].elapsed_time(ev[1]) * 1e3 / w.decode_steps
         del g
         return us
@@ -639,12 +669,13 @@ def profile_run(args, w):
         raise SystemExit(f"device status {rc} ({detail})")
 
 
-def decode_traffic_ratio():
-    """DRAM bytes per algorithmic byte of decode_kernel from the committed ncu
-    summary, if it was taken on the decode source as it is now (else None)."""
+def decode_traffic_ratio(workload: str):
+    """DRAM bytes per algorithmic byte of decode_kernel on this workload from
+    the committed ncu summary, if it was taken on the decode source as it is
+    now (else None)."""
     import hashlib
     import re
-    path = os.path.join(ROOT, "profiles", "decode_kernel_llamagen_xl.md")
+    path = os.path.join(ROOT, "profiles", f"decode_kernel_{workload}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
@@ -713,7 +744,11 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    res = gpu_arm(args, rank, world, dev)
+    res = gpu_arm(args, rank, world, dev, w)
+    torch.cuda.empty_cache()
+    sweep = None
+    if world == 1 and not args.no_sweep:
+        sweep = sweep_arm(args, dev, w.name)
     cpu = None
     if rank == 0 and world == 1:
         v, cores, n, el = oracle_sample(w, args.seed, args.cpu_seconds, opts=oracle_opts(args))
@@ -742,6 +777,7 @@ def main():
             "kv_pool_bytes": res["kv_pool_bytes"], "labels_local_frac": res["labels_local_frac"],
             "labels_planted": res["labels_planted"],
             "decoder_layer": res.get("decoder_layer"),
+            "all_configs": sweep,
         }
         print(json.dumps(line))
     if world > 1:

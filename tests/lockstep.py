@@ -43,12 +43,73 @@ def generate(w, seed, device, num_seqs=None):
     return [generate_layer(w, l, seed, device, num_seqs=num_seqs) for l in range(w.num_layers)]
 
 
-def run_gpu(w, cfg, data, units, fused=True, with_prefill_out=False):
+class HeadShardedView:
+    """Several contexts that each hold a contiguous range of the heads of
+    every (sequence, layer), seen as one cache of all heads: the two-phase
+    prefill (label on every shard, the sum of their Local counts standing in
+    for the all-reduce, compress on every shard), per-step calls on each
+    shard's slice of the heads, and read-backs concatenated over the heads
+    (a head index here is the unsharded one)."""
+
+    def __init__(self, cfg, shards, device):
+        self.shards = shards
+        self.parts = [hkv.HeadKVCache(hkv.Config(**{**cfg.__dict__, "num_heads": len(r),
+                                                     "heads_total": cfg.num_heads}), device=device)
+                      for r in shards]
+
+    @staticmethod
+    def _sl(x, r):
+        return x[:, r.start:r.stop].contiguous()
+
+    def prefill_classify(self, layer, q, k, v, out=None):
+        pre = [tuple(self._sl(x, r) for x in (q, k, v)) for r in self.shards]
+        ns = [c.prefill_label(layer, *p) for c, p in zip(self.parts, pre)]
+        tot = sum(ns[1:], ns[0].clone())
+        for c, p in zip(self.parts, pre):
+            c.prefill_compress(layer, p[1], p[2], tot)
+        return tot
+
+    def decode_step(self, layer, q_t, k_t, v_t, o_t):
+        for c, r in zip(self.parts, self.shards):
+            o = torch.empty_like(o_t[:, r.start:r.stop])
+            c.decode_step(layer, self._sl(q_t, r), self._sl(k_t, r), self._sl(v_t, r), o)
+            o_t[:, r.start:r.stop] = o
+
+    def ste_evict(self):
+        for c in self.parts:
+            c.ste_evict()
+
+    def labels(self, layer):
+        got = [c.labels(layer) for c in self.parts]
+        return np.concatenate([g[0] for g in got], 1), np.concatenate([g[1] for g in got], 1)
+
+    def lens(self, layer):
+        got = [c.lens(layer) for c in self.parts]
+        return np.concatenate([g[0] for g in got], 1), np.concatenate([g[1] for g in got], 1)
+
+    def kept(self, s, layer, h):
+        for c, r in zip(self.parts, self.shards):
+            if r.start <= h < r.stop:
+                return c.kept(s, layer, h - r.start)
+        raise IndexError(h)
+
+    def check(self):
+        for c in self.parts:
+            rc, detail = c.check()
+            if rc:
+                return rc, detail
+        return 0, 0
+
+
+def run_gpu(w, cfg, data, units, fused=True, with_prefill_out=False, cache=None):
     """Runs the pipeline; returns the cache and, per sampled unit (s, l),
-    {"labels", "o" [steps, H, d], "events" [(t, {h: kept positions})]}."""
+    {"labels", "o" [steps, H, d], "events" [(t, {h: kept positions})]}.
+    cache: a prebuilt cache object (e.g. a HeadShardedView) instead of a
+    new context of cfg."""
     dev = data[0][0].device
     S, H, P, L, d = cfg.num_seqs, cfg.num_heads, w.prefill_len, w.max_len, cfg.head_dim
-    cache = hkv.HeadKVCache(cfg, device=dev)
+    if cache is None:
+        cache = hkv.HeadKVCache(cfg, device=dev)
     rec = {u: {"o": torch.empty(L - P, H, d, dtype=cfg.torch_dtype, device=dev), "events": []}
            for u in units}
     pre_out = []

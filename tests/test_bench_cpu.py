@@ -23,7 +23,7 @@ def test_reference_arm_json_line():
         assert key in d, key
     assert d["impl"] == "reference"
     assert d["value"] > 0 and d["ms_per_step"] > 0
-    assert d["config"]["workload"] == "llamagen_xl"
+    assert d["config"]["workload"] == "lumina_mgpt_768"  # the default headline workload
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["e2e"]["value"] == d["value"]
@@ -32,7 +32,8 @@ def test_reference_arm_json_line():
 def test_reference_arm_takes_the_variant_flags():
     out = subprocess.run(
         [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
-         "--warmup", "0", "--cpu-seconds", "1", "--cls-queries", "8", "--cfg-pairing", "halves",
+         "--warmup", "0", "--cpu-seconds", "1", "--workload", "llamagen_xl",
+         "--cls-queries", "8", "--cfg-pairing", "halves",
          "--mode", "uniform", "--unstratified"],
         cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert out.returncode == 0, out.stderr[-2000:]

@@ -226,68 +226,53 @@ def test_classifier_variants(nq, pairing):
             np.testing.assert_array_equal(ntau[s], ntau[sp])
 
 
-def test_head_sharded_contexts_match_unsharded():
+def test_head_sharded_contexts_match_unsharded_and_oracle():
     """Heads split over two contexts (as over two GPUs; the sum of their
-    Local counts stands for the all-reduce): every label, length and kept
-    set equals the unsharded context's and the outputs agree within the
-    bf16 tolerance; a total no shard split allows latches INVALID_ARG."""
+    Local counts stands for the all-reduce): sampled units of the sharded
+    run, concatenated over the shards, are in lock step with the oracle;
+    every label, length and kept set equals the unsharded context's and the
+    outputs agree within the bf16 tolerance; a total no shard split allows
+    latches INVALID_ARG."""
+    from lockstep import HeadShardedView
     w = WORKLOADS["llamagen_xl"].scaled(num_seqs=2, num_layers=2)
-    S, H, P, L, d = w.num_seqs, w.num_heads, w.prefill_len, w.max_len, w.head_dim
+    S, H, P = w.num_seqs, w.num_heads, w.prefill_len
     data = generate(w, 21, DEV)
     base = hkv.config_for(w)
-    full = hkv.HeadKVCache(base, device=DEV)
     shards = [range(0, 7), range(7, H)]  # unequal on purpose
-    parts = [hkv.HeadKVCache(hkv.Config(**{**base.__dict__, "num_heads": len(r),
-                                            "heads_total": H}), device=DEV) for r in shards]
-
-    def sl(x, r):
-        return x[:, r.start:r.stop].contiguous()
-
+    view = HeadShardedView(base, shards, DEV)
+    parts = view.parts
+    sl = HeadShardedView._sl
     with pytest.raises(hkv.HkvError):  # a sharded context cannot group alone
         parts[0].prefill_classify(0, *(sl(x[:, :, :P], shards[0]) for x in data[0]))
-    for l, (q, k, v) in enumerate(data):
-        full.prefill_classify(l, q[:, :, :P], k[:, :, :P], v[:, :, :P])
-        pre = [tuple(sl(x[:, :, :P], r) for x in (q, k, v)) for r in shards]
-        with pytest.raises(hkv.HkvError):  # compress before label
-            parts[0].prefill_compress(l, pre[0][1], pre[0][2],
-                                      torch.zeros(S, dtype=torch.int32, device=DEV))
-        ns = [c.prefill_label(l, *p) for c, p in zip(parts, pre)]
-        tot = ns[0] + ns[1]
-        for c, p in zip(parts, pre):
-            c.prefill_compress(l, p[1], p[2], tot)
-        lab, ntau = full.labels(l)
-        np.testing.assert_array_equal(tot.cpu().numpy(), (lab == 1).sum(1))
-        got = [c.labels(l) for c in parts]
-        np.testing.assert_array_equal(np.concatenate([g[0] for g in got], 1), lab)
-        np.testing.assert_array_equal(np.concatenate([g[1] for g in got], 1), ntau)
-    o_full = torch.empty(S, H, d, dtype=w.torch_dtype, device=DEV)
-    o_part = [torch.empty(S, len(r), d, dtype=w.torch_dtype, device=DEV) for r in shards]
-    worst = 0.0
-    for t in range(P, L):
-        for l, (q, k, v) in enumerate(data):
-            qt, kt, vt = (x[:, :, t].contiguous() for x in (q, k, v))
-            full.decode_step(l, qt, kt, vt, o_full)
-            for c, r, o in zip(parts, shards, o_part):
-                c.decode_step(l, sl(qt, r), sl(kt, r), sl(vt, r), o)
-            ref = o_full.float()
-            got = torch.cat(o_part, 1).float()
-            worst = max(worst, float((got - ref).abs().max() / ref.abs().max()))
-        full.ste_evict()
-        for c in parts:
-            c.ste_evict()
-    assert worst <= TOL["bf16"], worst
+    with pytest.raises(hkv.HkvError):  # compress before label
+        k0, v0 = (sl(x[:, :, :P], shards[0]) for x in data[0][1:])
+        parts[0].prefill_compress(0, k0, v0, torch.zeros(S, dtype=torch.int32, device=DEV))
+    units = [(s, l) for s in range(S) for l in range(w.num_layers)]
+    _, rec_v, _ = run_gpu(w, base, data, units, cache=view)
+    full, rec_f, _ = run_gpu(w, base, data, units)
+    assert view.check()[0] == 0 and full.check()[0] == 0
+    for u in units:
+        # the sharded run against the oracle (budgets over all heads)
+        res, err = compare_unit(w, data, u, rec_v[u])
+        assert_lockstep(res, err, TOL["bf16"], len(rec_v[u]["events"]), unit=("sharded",) + u)
+        np.testing.assert_array_equal(res.labels, rec_v[u]["labels"])
+        # and against the unsharded context
+        np.testing.assert_array_equal(rec_v[u]["labels"], rec_f[u]["labels"])
+        assert [t for t, _ in rec_v[u]["events"]] == [t for t, _ in rec_f[u]["events"]]
+        for (_, kv), (_, kf) in zip(rec_v[u]["events"], rec_f[u]["events"]):
+            assert kv.keys() == kf.keys()
+            for h in kv:
+                np.testing.assert_array_equal(kv[h], kf[h])
+        a, b = rec_v[u]["o"].double(), rec_f[u]["o"].double()
+        assert float((a - b).abs().max() / b.abs().max()) <= TOL["bf16"]
     for l in range(w.num_layers):
-        ln, bd = full.lens(l)
-        got = [c.lens(l) for c in parts]
-        np.testing.assert_array_equal(np.concatenate([g[0] for g in got], 1), ln)
-        np.testing.assert_array_equal(np.concatenate([g[1] for g in got], 1), bd)
+        for x, y in zip(view.labels(l), full.labels(l)):
+            np.testing.assert_array_equal(x, y)
+        for x, y in zip(view.lens(l), full.lens(l)):
+            np.testing.assert_array_equal(x, y)
         for s in range(S):
             for h in (0, 6, 7, H - 1):
-                i = 0 if h < 7 else 1
-                np.testing.assert_array_equal(parts[i].kept(s, l, h - shards[i].start),
-                                              full.kept(s, l, h))
-    for c in [full] + parts:
-        assert c.check()[0] == 0
+                np.testing.assert_array_equal(view.kept(s, l, h), full.kept(s, l, h))
     # a Local total no split of the heads allows
     c = parts[0]
     c.reset()
