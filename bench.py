@@ -63,8 +63,11 @@ def parse_args():
                     help="skip the shorter runs of every other workload (all_configs)")
     ap.add_argument("--profile", action="store_true",
                     help="eager run of a reduced workload for ncu captures (no timing line)")
-    ap.add_argument("--seqs", type=int, default=None, help="override the workload's sequences")
-    ap.add_argument("--layers", type=int, default=None, help="override the workload's layers")
+    ap.add_argument("--seqs", type=int, default=None,
+                    help="override the workload's sequences (profile runs and reduced timings)")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="override the workload's layers (profile runs and reduced timings)")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
     ap.add_argument("--profile-steps", type=int, default=64)
     return ap.parse_args()
 
@@ -367,6 +370,7 @@ def gpu_arm(args, rank, world, dev, w, lite=False):
     g_prof = capture(lambda: run_pass(cache, w, inp, outs, pre_out=pre_out, hooks=hooks_prof))
     g_prof.replay()
     torch.cuda.synchronize()
+    ev = cache.evict_stats()  # this pass's evictions (reset clears the counters)
     dur = np.array([evs[2 * i].elapsed_time(evs[2 * i + 1]) for i in range(n_ev)]).reshape(steps, 2)
     dec_us = np.repeat(dur[:, :1] * 1e3 / Ly, Ly, axis=1)  # average launch of each step
     evict_us = dur[:, 1] * 1e3
@@ -400,6 +404,12 @@ def gpu_arm(args, rank, world, dev, w, lite=False):
                      "launch_us_avg": float(dec_us.mean())},
         "evict_us_avg": float(evict_us.mean()),
         "evict_us_max": float(evict_us.max()),
+        # eviction over the pass: positions + r logits of every scored token,
+        # K|V pairs of the moved rows read and written; time = the spans of
+        # the steps' eviction calls (eviction kernel + next-step plan)
+        "evict": {"heads": ev["heads"], "rows_moved": ev["rows_moved"],
+                  "bytes": ev["tokens"] * (4 + 4 * w.score_window) + ev["rows_moved"] * 4 * d * es,
+                  "call_us_total": float(evict_us.sum())},
         "labels_local_frac": float((labels == 1).mean()),
         "labels_planted": planted_recovery(w, labels, dist.rank_seed(args.seed, rank)),
         # per layer at prefill: attention, grouping, packing, plan; per
@@ -652,19 +662,28 @@ def profile_run(args, w):
     es = 2 if w.dtype == "bf16" else 4
     for l in range(w.num_layers):
         cache.prefill_classify(l, *inp.pre[l])
-    alg = []
-    for t in range(min(args.profile_steps, w.decode_steps)):
+    alg, evict_steps, evict_alg = [], [], []
+    steps = min(args.profile_steps, w.decode_steps)
+    for t in range(steps):
         for l in range(w.num_layers):
             q, k, v = inp.dec[l]
             cache.decode_step(l, q[t], k[t], v[t], outs[l])
             ln, _ = cache.lens(l)
             alg.append(int(ln.sum()) * 2 * w.head_dim * es + w.num_seqs * w.num_heads * w.head_dim * es * 4)
+        st0 = cache.evict_stats()
         cache.ste_evict()
+        st1 = cache.evict_stats()
+        # algorithmic bytes of this step's eviction: per evicted head its
+        # positions and r logits, and the rows it moved (K|V pair read + written)
+        if st1["heads"] > st0["heads"]:
+            evict_steps.append(t)
+            evict_alg.append((st1["tokens"] - st0["tokens"]) * (4 + 4 * w.score_window) +
+                             (st1["rows_moved"] - st0["rows_moved"]) * 2 * 2 * w.head_dim * es)
     torch.cuda.synchronize()
     rc, detail = cache.check()
     print(json.dumps({"profile_run": w.name, "seqs": w.num_seqs, "layers": w.num_layers,
-                      "steps": min(args.profile_steps, w.decode_steps), "status": rc,
-                      "decode_alg_bytes": alg}))
+                      "steps": steps, "status": rc, "decode_alg_bytes": alg,
+                      "evict_steps": evict_steps, "evict_alg_bytes": evict_alg}))
     if rc != 0:
         raise SystemExit(f"device status {rc} ({detail})")
 
@@ -696,6 +715,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     from kv_cache_compression_hkv_b200.inputs import WORKLOADS
     w = WORKLOADS[args.workload]
+    if not args.profile and (args.seqs or args.layers):
+        w = w.scaled(num_seqs=args.seqs or w.num_seqs, num_layers=args.layers or w.num_layers,
+                     images=(args.seqs or w.num_seqs) * w.images // w.num_seqs)
     config = {"workload": w.name, "num_seqs": w.num_seqs, "images": w.images,
               "num_layers": w.num_layers, "num_heads": w.num_heads, "head_dim": w.head_dim,
               "max_len": w.max_len, "prefill_len": w.prefill_len, "decode_steps": w.decode_steps,
@@ -750,7 +772,7 @@ def main():
     if world == 1 and not args.no_sweep:
         sweep = sweep_arm(args, dev, w.name)
     cpu = None
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and not args.no_cpu:
         v, cores, n, el = oracle_sample(w, args.seed, args.cpu_seconds, opts=oracle_opts(args))
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{n} whole (sequence, layer) units of {w.name} in {el:.1f} s "
@@ -769,7 +791,7 @@ def main():
             "config": config,
             "decode_step_us": res["decode_step_us"], "prefill_ms": res["prefill_ms"],
             "roofline": res["roofline"], "evict_us_avg": res["evict_us_avg"],
-            "evict_us_max": res["evict_us_max"],
+            "evict_us_max": res["evict_us_max"], "evict": res["evict"],
             "cpu_baseline": cpu, "e2e": res.get("e2e"), "gpu_launches": res["gpu_launches"],
             "clocks": res["clocks"], "full": res.get("full"),
             "speedup_decode_vs_full": res.get("speedup_decode_vs_full"),

@@ -222,6 +222,14 @@ HKV_API hkv_status hkv_get_lens(hkv_ctx* ctx, int32_t layer, int32_t* len_host, 
 HKV_API hkv_status hkv_get_kept(hkv_ctx* ctx, int32_t seq, int32_t layer, int32_t head,
                         int32_t* pos_host, int32_t capacity, int32_t* len_out, void* stream);
 
+/* Counters of the evictions run since hkv_create or hkv_reset, into
+ * stats_host[3] (int64): Global heads evicted, cached tokens they scored
+ * (their lengths at eviction), rows moved by the compaction (one K row, one
+ * V row and a position each).  A head's eviction reads its positions and r
+ * logits per token and each moved row's K|V pair once, and writes it once:
+ * these counts give the eviction's bytes.  Waits for `stream`. */
+HKV_API hkv_status hkv_get_evict_stats(hkv_ctx* ctx, int64_t* stats_host, void* stream);
+
 /* Reads the device status word (waits for `stream`) and returns the first
  * error latched on the device, or HKV_OK.  *detail_host (nullable) gets a
  * code-specific detail (e.g. the head index). */

@@ -66,6 +66,7 @@ def lib():
             "hkv_get_lens": [P, I, P, P, P],
             "hkv_get_kept": [P, I, I, I, P, I, P, P],
             "hkv_check": [P, P, P],
+            "hkv_get_evict_stats": [P, P, P],
             "hkv_clear_error": [P, P],
             "hkv_reset": [P, P],
             "hkv_classify_rows": [P, I, I, I, D, P, P, P],
@@ -292,6 +293,13 @@ class HeadKVCache:
         _check(lib().hkv_get_kept(self.ctx, seq, layer, head, buf.ctypes.data, cap, C.byref(n),
                                   _stream(stream)), "hkv_get_kept")
         return buf[: n.value].copy()
+
+    def evict_stats(self, stream=None) -> dict:
+        """Evictions since create/reset: heads, tokens scored, rows moved."""
+        out = np.zeros(3, dtype=np.int64)
+        _check(lib().hkv_get_evict_stats(self.ctx, out.ctypes.data, _stream(stream)),
+               "hkv_get_evict_stats")
+        return {"heads": int(out[0]), "tokens": int(out[1]), "rows_moved": int(out[2])}
 
     def check(self, stream=None):
         detail = C.c_int32()

@@ -14,6 +14,7 @@
 // within r steps of their eviction also store their exp2-domain logits per
 // slot, which the eviction normalises with the (max, sum) stored here.
 #include <math.h>
+#include <stdlib.h>
 
 #include <cuda/atomic>
 
@@ -27,7 +28,7 @@ namespace hkv {
 // before the reference is raised: weights stay below 2^8, far from fp32 range.
 constexpr float RESCALE = 8.f;
 // Most pipeline stages a decode warp keeps in flight.
-constexpr int MAX_STAGES = 3;
+constexpr int MAX_STAGES = 4;
 // Most warps of one decode block (one block per SM).
 constexpr int DECODE_MAX_WARPS = 12;
 // Cost of a chunk, in units of the cost of a head's end, in the plan's
@@ -166,7 +167,11 @@ __device__ __forceinline__ int4 shfl_int4(const int4& v, int src) {
 // the p-th slice of the warps (each warp: its range and copies of the first
 // PLAN_WARP_DESC descriptors of its range).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead) {
+// With commit (the launch right after an eviction at step t_next - 1), the
+// Global heads that were due at that step get their new length first (the
+// budget, from that step on) and each unit its next due step; part 0 writes
+// them, every part plans with them.
+__global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead, int commit) {
     extern __shared__ int32_t psm[];
     __shared__ int wsum[32];
     const int layer = l0 + blockIdx.x;
@@ -181,13 +186,44 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead)
     uint16_t* own = reinterpret_cast<uint16_t*>(whead + PLAN_MAX_WARPS);  // [total] warp of each chunk
     const int parts = gridDim.y, part = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, NW = blockDim.x >> 5;
-    const int t = L.t_next[layer] - 1 + ahead;
-    if (t >= L.L) return;  // the sequence is complete: no step left to plan
+    const int te = L.t_next[layer] - 1;  // newest cached position
+    const int t = te + ahead;
     const size_t hbase = (size_t)layer * n;
+    if (commit) {
+        // heads evicted at te: length = budget from te on; due again M steps later
+        for (int i = tid; i < n; i += blockDim.x) {
+            const size_t hx = hbase + i;
+            const int cap = L.cap[hx];
+            int bl = L.base_len[hx], bt = L.base_t[hx];
+            if (L.label[hx] != 0 || L.mode == HKV_MODE_FULL) continue;
+            if (bl + (te - bt) >= cap) {
+                bl = L.budget[hx];
+                bt = te;
+                if (part == 0) { L.base_len[hx] = bl; L.base_t[hx] = bt; }
+            }
+            const int s = i / L.H;
+            const uint32_t gm = L.unit_gmask[(size_t)layer * L.S + s];
+            if (part == 0 && gm && (i % L.H) == __ffs(gm) - 1)
+                L.unit_due[(size_t)layer * L.S + s] = bt + (cap - bl);
+        }
+        __syncthreads();
+    }
+    if (t >= L.L) return;  // the sequence is complete: no step left to plan
     for (int i = tid; i < n; i += blockDim.x) {
         const size_t hx = hbase + i;
-        const int len = len_at(L, hx, t);
         const int cap = L.cap[hx];
+        int len;
+        {
+            int bl = L.base_len[hx], bt = L.base_t[hx];
+            // part 0 may already have written the committed values: either
+            // reading gives the same length
+            if (commit && L.label[hx] == 0 && L.mode != HKV_MODE_FULL && bl + (te - bt) >= cap) {
+                bl = L.budget[hx];
+                bt = te;
+            }
+            len = bl + (t - bt);
+            if (L.label[hx] == 1 && len > cap) len = cap;
+        }
         int c = (len + CHUNK - 1) / CHUNK;
         if (len > cap || len < 1) {
             if (part == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
@@ -364,7 +400,7 @@ template <typename T, int DPL>
 __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
     decode_kernel(Layout L, int layer, const T* __restrict__ q_t, const T* __restrict__ k_t,
                   const T* __restrict__ v_t, T* __restrict__ o_t, int append, int nstage,
-                  int early, int buf) {
+                  int early, int buf, int prologue) {
     extern __shared__ __align__(128) unsigned char dsm[];
     const int n_heads = L.S * L.H;
     constexpr int D = DPL * 32;
@@ -480,7 +516,7 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
         // with few, every stage (fewer bytes would be in flight otherwise).
         // With `early` their cached rows go before the wait on the previous
         // launch, queries and appended rows after it.
-        const int npro = NW >= 8 ? 1 : min(nstage, c_end - c_begin);
+        const int npro = (prologue == 1 || (prologue == 0 && NW >= 8)) ? 1 : min(nstage, c_end - c_begin);
         if (early) {
             for (int s = 0; s < npro; ++s) {
                 const ChunkDesc c = ChunkDesc::of(shfl_int4(head, s));
@@ -823,19 +859,36 @@ __global__ void __launch_bounds__(256) append_kernel(Layout L, int layer, const 
 // launchers
 // ---------------------------------------------------------------------------
 
+// Positive integer from the environment, or 0 when unset or invalid.
+static int env_int(const char* name) {
+    const char* v = getenv(name);
+    if (!v) return 0;
+    const int x = atoi(v);
+    return x > 0 ? x : 0;
+}
+
 DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
     // As many warps as fit (up to DECODE_MAX_WARPS) with two stages each:
     // the kernel is latency-bound, so warps matter more than prefetch depth
     // (one chunk in flight per warp covers the HBM latency at the rate a
     // warp consumes chunks); a third stage only when it costs no warp.
+    // Tuning overrides (read once per context): HKV_DECODE_WARPS caps the
+    // warps per block, HKV_DECODE_STAGES fixes the stages per warp (2 ..
+    // MAX_STAGES), HKV_DECODE_PROLOGUE sets DecodeShape::prologue (1 or 2).
     const int es = L.dtype == HKV_DTYPE_F32 ? 4 : 2;
-    DecodeShape best{0, 0, 0, 1};
+    const int max_w = env_int("HKV_DECODE_WARPS");
+    const int fix_s = env_int("HKV_DECODE_STAGES");
+    const int pro = env_int("HKV_DECODE_PROLOGUE");
+    DecodeShape best{0, 0, 0, 1, pro <= 2 ? pro : 0};
     for (int ns = 2; ns <= MAX_STAGES; ++ns) {
+        if (fix_s && ns != fix_s) continue;
         // the per-warp tail regions are laid out for MAX_STAGES barriers
         const size_t per = decode_warp_bytes(L.d, es, ns) + (MAX_STAGES - ns) * 8;
         int w = (int)((smem_limit - 1024) / per);
         if (w > DECODE_MAX_WARPS) w = DECODE_MAX_WARPS;
-        if (w >= 1 && w >= best.warps) best = DecodeShape{w, ns, 1024 + (size_t)w * per, 1};
+        if (max_w && w > max_w) w = max_w;
+        if (w >= 1 && w >= best.warps)
+            best = DecodeShape{w, ns, 1024 + (size_t)w * per, 1, best.prologue};
     }
     return best;
 }
@@ -855,7 +908,7 @@ static cudaError_t launch_decode_t(const Layout& L, int layer, const void* q, co
     cfg.attrs = at;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, decode_kernel<T, DPL>, L, layer, (const T*)q, (const T*)k,
-                              (const T*)v, (T*)o, append, sh.nstage, early, buf);
+                              (const T*)v, (T*)o, append, sh.nstage, early, buf, sh.prologue);
 }
 
 cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void* k, const void* v,
@@ -872,9 +925,9 @@ cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void*
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_plan(const Layout& L, int l0, int l1, int ahead, cudaStream_t st) {
+cudaError_t launch_plan(const Layout& L, int l0, int l1, int ahead, int commit, cudaStream_t st) {
     plan_kernel<<<dim3(l1 - l0, PLAN_DESC_PARTS), 1024, plan_smem_bytes(L.S * L.H, L.max_chunks), st>>>(
-        L, l0, ahead);
+        L, l0, ahead, commit);
     return cudaGetLastError();
 }
 

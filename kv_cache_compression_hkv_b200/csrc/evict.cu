@@ -18,204 +18,433 @@
 
 namespace hkv {
 
-// Per-warp scratch of the eviction: the select's own scratch, the (max, sum)
-// of the scoring steps, the step each column holds, an mbarrier, the
-// positions of the top M slots, then their K and V rows (`row_bytes` each),
-// prefetched while the head is scored.
-__host__ __device__ inline size_t evict_warp_bytes(int n_max, int m_rows, int row_bytes) {
-    return select_scratch_bytes(n_max) + 32 * 8 + 32 * 4 + 16 + (size_t)round32(m_rows) * 4 +
-           2 * (size_t)m_rows * row_bytes;
-}
+// ---------------------------------------------------------------------------
+// Eviction of the due heads of layers [l0, l1), one block per head.  A
+// head's unit (layer, sequence) is due at step t when its due step (kept
+// by the plan kernel; all Global heads of a unit share capacity and length)
+// is t, the layer's newest position.  Block c looks at the items (unit,
+// head) numbered c, c + G, c + 2G, ... (G blocks), lists the due ones among
+// them in shared memory and evicts them one after the other: a unit's heads
+// land on consecutive blocks.  Nothing here changes what the due test
+// reads, so every block sees the same due set; the plan kernel that follows
+// the eviction records the heads' new lengths.  Per head:
+//  1. the rows a survivor may move from (slots budget .. len-1) are
+//     prefetched into L2 while the head is scored;
+//  2. every thread loads the position and the r stored logits of its tokens
+//     (all loads of up to 4 tokens issued before any is used) and turns them
+//     into the token's score: the summed softmax weight of the last r steps,
+//     each step's weight exp2(logit - max) / sum, only for tokens already
+//     cached at that step; key = (score bits, position) in shared memory;
+//  3. the threshold of each stratum (near: distance 1..D; far: beyond) is
+//     found by a 16-ary search on the score bits, both strata per round
+//     (15 pivots each, counts reduced over the block), then the position tie
+//     at the boundary; every key <= the threshold is evicted, so each
+//     stratum loses exactly its share, lowest (score, position) first;
+//  4. holes (evicted slots below the budget) and movers (survivors above it)
+//     are listed in (thread, token) order and the i-th mover's K|V row pair
+//     and position are copied into the i-th hole.
+// ---------------------------------------------------------------------------
+constexpr int EVB_THREADS = 256;  // threads of an eviction block
+constexpr int EVB_WARPS = EVB_THREADS / 32;
 
-constexpr uint64_t EVICT_WAIT_NS = 2000000000ull;  // a copy that takes 2 s has failed
-
-// Lists the Global heads of layers [l0, l1) whose cache reached budget + M
-// (one thread per head; one atomic per warp).
-__global__ void __launch_bounds__(256) evict_scan_kernel(Layout L, int l0, int l1) {
-    const int n_heads = L.S * L.H;
-    const int total = (l1 - l0) * n_heads;
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    const int lane = threadIdx.x & 31;
-    bool due = false;
-    size_t hx = 0;
-    if (i < total && L.mode != HKV_MODE_FULL) {
-        const int l = l0 + i / n_heads;
-        hx = (size_t)l * n_heads + (i % n_heads);
-        due = L.label[hx] == 0 && len_at(L, hx, L.t_next[l] - 1) >= L.cap[hx];
+// One round of the threshold search of both strata: every thread adds its
+// candidate keys with score bits in [lo, hi] of their stratum to 16 bins of
+// width 2^sh above lo (16-bit counters packed two to a word: a warp holds
+// far fewer than 65536 keys) and counts those below lo; the block's totals
+// are reduced through `red` (this round's buffer; rounds alternate between
+// two, so one barrier per round suffices).  Lane i of every warp returns the
+// number of keys at or below the top of bin i (i < 16: near stratum, else
+// bin i - 16 of the far stratum).
+__device__ __forceinline__ int block_bin_counts(const uint32_t (&ha)[8], const uint32_t (&hb)[8],
+                                                int below_a, int below_b, int (*red)[32], int NW) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t w[16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        w[j] = __reduce_add_sync(FULL_MASK, ha[j]);
+        w[8 + j] = __reduce_add_sync(FULL_MASK, hb[j]);
     }
-    const unsigned b = __ballot_sync(FULL_MASK, due);
-    if (!b) return;
-    const int leader = __ffs(b) - 1;  // every lane of the warp reaches here
-    int base = 0;
-    if (lane == leader) base = atomicAdd(L.due_ctl, __popc(b));
-    base = __shfl_sync(FULL_MASK, base, leader);
-    if (due) L.due_list[base + __popc(b & ((1u << lane) - 1u))] = (int)hx;
+    below_a = __reduce_add_sync(FULL_MASK, below_a);
+    below_b = __reduce_add_sync(FULL_MASK, below_b);
+    if (lane == 0) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) red[warp][j] = (int)w[j];
+        red[warp][16] = below_a;
+        red[warp][17] = below_b;
+    }
+    __syncthreads();
+    // lane i: bin i & 15 of stratum i >> 4, summed over the warps
+    int tot = 0, below = 0;
+    const int word = lane >> 1, sh = 16 * (lane & 1);
+    for (int v = 0; v < NW; ++v) {
+        tot += ((uint32_t)red[v][word] >> sh) & 0xffffu;
+        below += red[v][16 + (lane >> 4)];
+    }
+    // inclusive prefix over the 16 bins of each stratum
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) {
+        const int y = __shfl_up_sync(FULL_MASK, tot, o);
+        if ((lane & 15) >= o) tot += y;
+    }
+    return tot + below;
 }
 
-// Evicts every listed head, one warp per head: scores from the stored
-// logits, stratified select, compaction.  The last block clears the list.
-constexpr int EVICT_MAX_WARPS = 12;
+// Adds one candidate key to its stratum's packed bins.
+__device__ __forceinline__ void bin_add(uint32_t (&h)[8], int& below, uint32_t sb, uint32_t lo,
+                                        uint32_t hi, int sh) {
+    if (sb < lo) { ++below; return; }
+    if (sb > hi) return;
+    const uint32_t b = (sb - lo) >> sh;  // 0 .. 15
+    const uint32_t inc = 1u << (16 * (b & 1));
+    const uint32_t wi = b >> 1;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) h[j] += wi == (uint32_t)j ? inc : 0u;
+}
+
+// Bin width (log2) that splits [lo, hi] into at most 16 bins.
+__device__ __forceinline__ int bin_shift(uint32_t lo, uint32_t hi) {
+    const uint32_t w = hi - lo;
+    const int bits = w ? 32 - __clz(w) : 0;
+    return bits > 4 ? bits - 4 : 0;
+}
 
 template <typename T>
-__global__ void __launch_bounds__(EVICT_MAX_WARPS * 32) evict_run_kernel(Layout L, int n_max) {
-    extern __shared__ __align__(16) unsigned char esm[];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int NW = blockDim.x >> 5;
-    const int d = L.d;
-    const int r = L.r;
-    const int row_bytes = d * (int)sizeof(T);
-    const int MR = L.M;  // rows above the budget of a due head
-    unsigned char* wbase = esm + (size_t)warp * evict_warp_bytes(n_max, MR, row_bytes);
-    SelectScratch sc = carve_select_scratch(wbase, n_max);
-    float2* ml_s = reinterpret_cast<float2*>(wbase + select_scratch_bytes(n_max));
-    int32_t* step_s = reinterpret_cast<int32_t*>(ml_s + 32);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(step_s + 32);
-    int32_t* top_pos = reinterpret_cast<int32_t*>(bar + 2);
-    unsigned char* kvbuf = reinterpret_cast<unsigned char*>(top_pos + round32(MR));  // K|V row pairs
+__global__ void __launch_bounds__(EVB_THREADS, 3) evict_block_kernel(Layout L, int l0, int l1, int n_max) {
+    extern __shared__ __align__(16) unsigned char ebs[];
+    __shared__ float2 ml_s[32];
+    __shared__ int step_s[32];
+    __shared__ int red[2][EVB_WARPS][32];
+    __shared__ int lists[2][EVB_WARPS];
+    __shared__ int due_items[EVB_THREADS];
+    __shared__ int n_due;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int BT = blockDim.x, NW = BT >> 5;
+    const int r = L.r, M = L.M;
+    uint64_t* keys = reinterpret_cast<uint64_t*>(ebs);            // [n_max]
+    int32_t* holes = reinterpret_cast<int32_t*>(keys + n_max);    // [M]
+    int32_t* movers = holes + M;                                  // [M]
+    int32_t* mpos = movers + M;                                   // [M]
     const int n_heads = L.S * L.H;
-    unsigned char* KVb = reinterpret_cast<unsigned char*>(L.K);  // slot s: K|V pair at 2 row_bytes s
-    const int pair = 2 * row_bytes;
-    const int per_pair = pair / 16;  // 16-byte pieces per K|V pair
-    const int count = L.due_ctl[0];
-    if (lane == 0) {
-        ptx::mbar_init(bar, 1);
-        ptx::fence_mbar_init();
-    }
-    __syncwarp();
-    uint32_t phase = 0;
+    const int pair = 2 * L.d * (int)sizeof(T);                    // bytes of a K|V row pair
+    const int per_pair = pair / 16;
+    unsigned char* KVb = reinterpret_cast<unsigned char*>(L.K);
+    int par = 0;  // reduction buffer of the next round
+    const int64_t items = (int64_t)(l1 - l0) * L.S * L.H;
+    const int64_t G = gridDim.x;
 
-    for (int e = blockIdx.x * NW + warp; e < count; e += gridDim.x * NW) {
-        const size_t hx = (size_t)L.due_list[e];
-        const int l = (int)(hx / n_heads);
-        const int hs = (int)(hx % n_heads);
-        const int s = hs / L.H;
-        const int t = L.t_next[l] - 1;
-        const int n = len_at(L, hx, t);
-        const int target = L.budget[hx];
-        if (n > n_max || n != L.cap[hx] || n - target > MR || n - target < 0) {
-            if (lane == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
-            continue;
+    for (int64_t k0 = 0; (int64_t)blockIdx.x + k0 * G < items; k0 += BT) {
+        // this block's next BT items: the due ones, in item order
+        {
+            const int64_t i = (int64_t)blockIdx.x + (k0 + tid) * G;
+            bool due = false;
+            int hxi = 0;
+            if (i < items) {
+                const int64_t u = i / L.H;  // unit within the range
+                const int h = (int)(i % L.H);
+                const int l = l0 + (int)(u / L.S), s = (int)(u % L.S);
+                const size_t uu = (size_t)l * L.S + s;
+                due = L.unit_due[uu] == L.t_next[l] - 1 && ((L.unit_gmask[uu] >> h) & 1u);
+                hxi = (int)(uu * L.H + h);
+            }
+            const unsigned b = __ballot_sync(FULL_MASK, due);
+            __syncthreads();  // the previous round's list is no longer read
+            if (lane == 0) lists[0][warp] = __popc(b);
+            __syncthreads();
+            int o = __popc(b & ((1u << lane) - 1u)), tot = 0;
+            for (int w = 0; w < NW; ++w) {
+                if (w < warp) o += lists[0][w];
+                tot += lists[0][w];
+            }
+            if (due) due_items[o] = hxi;
+            if (tid == 0) n_due = tot;
+            __syncthreads();
         }
-        const size_t slot0 = region_slot0(L, l, s) + L.off[hx];
-        const int top = n - target;  // the slots a survivor may move from
-        // the K and V rows of slots target .. n-1, while the head is scored
-        if (lane == 0 && top > 0) {
-            ptx::mbar_expect_tx(bar, (uint32_t)(top * pair));
-            ptx::bulk_g2s(kvbuf, KVb + (slot0 + target) * pair, top * pair, bar);
-        }
-        // (max, 1/sum) of each scoring step, by column = step mod r, and the
-        // step each column holds inside the window t-r+1 .. t
-        if (lane < r) {
-            const float2 ml = L.ml[hx * r + lane];
-            ml_s[lane] = make_float2(ml.x, 1.0f / ml.y);
-            step_s[lane] = t - (((t - lane) % r) + r) % r;
-        }
-        __syncwarp();
-        // scores: summed softmax weight of the last r queries, each
-        // counting only tokens already cached at its step.  Tokens go in
-        // batches of 8 per lane whose loads are all issued before any is
-        // used; every 32 of them are sorted into the strata right away.
-        bool bad = false;
-        int nn = 0, nf = 0;
-        for (int b0 = 0; b0 < n; b0 += 32 * 8) {
-            int pv[8];
-            float4 la[8], lb[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int q = b0 + u * 32 + lane;
-                if (q < n) {
-                    pv[u] = L.pos[slot0 + q];
-                    if (r == 8) {
-                        const float4* lg = reinterpret_cast<const float4*>(L.logit + (slot0 + q) * 8);
-                        la[u] = lg[0];
-                        lb[u] = lg[1];
+        const int nd = n_due;
+        for (int e = 0; e < nd; ++e) {
+            const size_t hx = (size_t)due_items[e];
+            const int l = (int)(hx / n_heads);
+            const int s = (int)(hx % n_heads) / L.H;
+            const int t = L.t_next[l] - 1;
+            const int n = len_at(L, hx, t);
+            const int target = L.budget[hx];
+            __syncthreads();  // the previous head's lists and keys are no longer read
+            if (n > n_max || n != L.cap[hx] || n - target > M || n - target < 0) {
+                if (tid == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
+                continue;
+            }
+            const size_t slot0 = region_slot0(L, l, s) + L.off[hx];
+            const int top = n - target;
+            if (tid == 0 && top > 0) ptx::bulk_prefetch_l2(KVb + (slot0 + target) * pair, (uint32_t)(top * pair));
+            if (tid < r) {
+                const float2 ml = L.ml[hx * r + tid];
+                ml_s[tid] = make_float2(ml.x, 1.0f / ml.y);
+                step_s[tid] = t - (((t - tid) % r) + r) % r;  // the step column tid holds
+            }
+            __syncthreads();
+
+            // scores and stratum counts; keys into shared memory
+            bool bad = false;
+            int nn = 0, nf = 0;
+            uint32_t alo = 0xffffffffu, ahi = 0u, blo = 0xffffffffu, bhi = 0u;
+            const bool strat = L.stratified != 0;
+            for (int b0 = 0; b0 < n; b0 += 2 * BT) {
+                int pv[2];
+                float4 la[2], lb[2];
+    #pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int q = b0 + u * BT + tid;
+                    if (q < n) {
+                        pv[u] = L.pos[slot0 + q];
+                        if (r == 8) {
+                            const float4* p4 = reinterpret_cast<const float4*>(L.logit + (slot0 + q) * 8);
+                            la[u] = p4[0];
+                            lb[u] = p4[1];
+                        }
                     }
                 }
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int base = b0 + u * 32;
-                if (base >= n) break;  // warp-uniform
-                const int q = base + lane;
-                const bool valid = q < n;
-                const int p = valid ? pv[u] : 0;
-                float acc = 0.f;
-                if (valid) {
+    #pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int q = b0 + u * BT + tid;
+                    if (q >= n) continue;
+                    const int p = pv[u];
+                    float acc = 0.f;
                     if (r == 8) {
                         const float v[8] = {la[u].x, la[u].y, la[u].z, la[u].w, lb[u].x, lb[u].y, lb[u].z, lb[u].w};
-#pragma unroll
+    #pragma unroll
                         for (int c = 0; c < 8; ++c)
                             if (p <= step_s[c]) acc += exp2f(v[c] - ml_s[c].x) * ml_s[c].y;
                     } else {
-                        const float* lg = L.logit + (slot0 + q) * r;
+                        const float* lp = L.logit + (slot0 + q) * r;
                         for (int c = 0; c < r; ++c)
-                            if (p <= step_s[c]) acc += exp2f(lg[c] - ml_s[c].x) * ml_s[c].y;
+                            if (p <= step_s[c]) acc += exp2f(lp[c] - ml_s[c].x) * ml_s[c].y;
                     }
                     if (isnan(acc)) bad = true;
-                    if (q >= target) top_pos[q - target] = p;
+                    const uint32_t sb = __float_as_uint(acc);
+                    keys[q] = ((uint64_t)sb << 32) | (uint32_t)p;
+                    const int delta = t - p;
+                    if (delta >= 1) {
+                        if (strat && delta <= L.D) { ++nn; alo = min(alo, sb); ahi = max(ahi, sb); }
+                        else { ++nf; blo = min(blo, sb); bhi = max(bhi, sb); }
+                    }
                 }
-                warp_partition_batch(sc, n, t, L.D, L.stratified, base, valid, __float_as_uint(acc), p, nn, nf);
             }
-        }
-        __syncwarp();
-        const int E = n - target;
-        warp_select_partitioned(sc, n, nn, nf, E / 2, E - E / 2, L.stratified);
-        if (__any_sync(FULL_MASK, bad) && lane == 0) latch_error(L, HKV_ERR_NUMERIC, (int)hx);
-        // holes: evicted slots below the budget; movers: survivors above it
-        int nh = 0, nm = 0;
-        for (int b0 = 0; b0 < n; b0 += 32) {
-            const int q = b0 + lane;
-            const bool ev = q < n && ((sc.evict_bits[q >> 5] >> (q & 31)) & 1u);
-            const bool hole = q < target && ev;
-            const bool mover = q >= target && q < n && !ev;
-            const unsigned bh = __ballot_sync(FULL_MASK, hole);
-            const unsigned bm = __ballot_sync(FULL_MASK, mover);
-            const unsigned lt = (1u << lane) - 1u;
-            if (hole) sc.moves[nh + __popc(bh & lt)] = (uint16_t)q;
-            if (mover) sc.moves[sc.n_max - 1 - (nm + __popc(bm & lt))] = (uint16_t)q;
-            nh += __popc(bh);
-            nm += __popc(bm);
-        }
-        __syncwarp();
-        bool ok = true;
-        if (top > 0) {
-            ok = ptx::mbar_wait(bar, phase, EVICT_WAIT_NS);
-            ok = __all_sync(FULL_MASK, ok);
-            phase ^= 1u;
-        }
-        if (!ok) {  // the prefetch never landed: stop before reusing its buffer
-            if (lane == 0) latch_error(L, HKV_ERR_TIMEOUT, (int)hx);
-            break;
-        }
-        if (nh != nm) {
-            if (lane == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
-            continue;
-        }
-        // move rows: each survivor's K and V rows from shared memory into a
-        // hole, in 16-byte pieces
-        const int pieces = nh * per_pair;
-        for (int w = lane; w < pieces; w += 32) {
-            const int mv = w / per_pair, pc = w % per_pair;
-            const int src = sc.moves[sc.n_max - 1 - mv] - target;
-            const size_t dst = (slot0 + sc.moves[mv]) * pair + pc * 16;
-            *reinterpret_cast<uint4*>(KVb + dst) =
-                *reinterpret_cast<const uint4*>(kvbuf + (size_t)src * pair + pc * 16);
-        }
-        for (int mv = lane; mv < nh; mv += 32)
-            L.pos[slot0 + sc.moves[mv]] = top_pos[sc.moves[sc.n_max - 1 - mv] - target];
-        __syncwarp();
-        if (lane == 0) {
-            L.base_len[hx] = target;
-            L.base_t[hx] = t;
-        }
-    }
-    // the last block out clears the list for the next step
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        if (atomicAdd(L.due_ctl + 1, 1) == (int)gridDim.x - 1) {
-            L.due_ctl[0] = 0;
-            L.due_ctl[1] = 0;
+            if (__syncthreads_or(bad) && tid == 0) latch_error(L, HKV_ERR_NUMERIC, (int)hx);
+            // block totals: counts and score-bit ranges of both strata
+            {
+                nn = __reduce_add_sync(FULL_MASK, nn);
+                nf = __reduce_add_sync(FULL_MASK, nf);
+                alo = __reduce_min_sync(FULL_MASK, alo);
+                ahi = __reduce_max_sync(FULL_MASK, ahi);
+                blo = __reduce_min_sync(FULL_MASK, blo);
+                bhi = __reduce_max_sync(FULL_MASK, bhi);
+                int (*rb)[32] = red[par];
+                if (lane == 0) {
+                    rb[warp][0] = nn; rb[warp][1] = nf;
+                    rb[warp][2] = (int)alo; rb[warp][3] = (int)ahi;
+                    rb[warp][4] = (int)blo; rb[warp][5] = (int)bhi;
+                }
+                __syncthreads();
+                nn = nf = 0;
+                alo = blo = 0xffffffffu;
+                ahi = bhi = 0u;
+                for (int w = 0; w < NW; ++w) {
+                    nn += rb[w][0]; nf += rb[w][1];
+                    alo = min(alo, (uint32_t)rb[w][2]); ahi = max(ahi, (uint32_t)rb[w][3]);
+                    blo = min(blo, (uint32_t)rb[w][4]); bhi = max(bhi, (uint32_t)rb[w][5]);
+                }
+                par ^= 1;
+            }
+            // shares of the strata (a stratum short of candidates hands its
+            // shortfall to the other); unstratified: one pool, all "far"
+            const int E = n - target;
+            int ka = E / 2, kb = E - E / 2;
+            if (strat) {
+                if (ka > nn) { kb += ka - nn; ka = nn; }
+                if (kb > nf) { ka += kb - nf; kb = nf; if (ka > nn) ka = nn; }
+            } else {
+                kb = E < nf ? E : nf;
+                ka = 0;
+            }
+            // threshold search: stratum x is active while 0 < k < m and its
+            // score range is not one value; thr = every key <= it is evicted
+            const bool a_part = ka > 0 && ka < nn, b_part = kb > 0 && kb < nf;
+            if (!a_part) alo = ahi = 0u;
+            if (!b_part) blo = bhi = 0u;
+            while (alo < ahi || blo < bhi) {
+                const int sa = bin_shift(alo, ahi), sbh = bin_shift(blo, bhi);
+                uint32_t ha[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u}, hb[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                int below_a = 0, below_b = 0;
+                for (int q = tid; q < n; q += BT) {
+                    const uint64_t key = keys[q];
+                    const uint32_t sb = (uint32_t)(key >> 32);
+                    const int delta = t - (int32_t)(uint32_t)key;
+                    if (delta < 1) continue;
+                    if (strat && delta <= L.D) bin_add(ha, below_a, sb, alo, ahi, sa);
+                    else bin_add(hb, below_b, sb, blo, bhi, sbh);
+                }
+                const int cum = block_bin_counts(ha, hb, below_a, below_b, red[par], NW);
+                par ^= 1;
+                // first bin whose cumulative count reaches the share
+                const unsigned ma = __ballot_sync(FULL_MASK, lane < 16 && cum >= ka);
+                const unsigned mb = __ballot_sync(FULL_MASK, lane >= 16 && cum >= kb);
+                if (alo < ahi) {
+                    const uint32_t j = (uint32_t)(__ffs(ma) - 1);  // exists: all of [lo, hi] reaches k
+                    const uint32_t nlo = alo + (j << sa);
+                    const uint64_t top = (uint64_t)alo + ((uint64_t)(j + 1) << sa) - 1;
+                    alo = nlo;
+                    ahi = top < ahi ? (uint32_t)top : ahi;
+                }
+                if (blo < bhi) {
+                    const uint32_t j = (uint32_t)(__ffs(mb >> 16) - 1);
+                    const uint32_t nlo = blo + (j << sbh);
+                    const uint64_t top = (uint64_t)blo + ((uint64_t)(j + 1) << sbh) - 1;
+                    blo = nlo;
+                    bhi = top < bhi ? (uint32_t)top : bhi;
+                }
+            }
+            // the position tie at each boundary score s*: need = k - (keys below
+            // s*) of the tied keys go, lowest positions first
+            uint64_t thr_a = a_part ? 0ull : (ka >= nn && ka > 0 ? ~0ull : 0ull);
+            uint64_t thr_b = b_part ? 0ull : (kb >= nf && kb > 0 ? ~0ull : 0ull);
+            bool none_a = ka <= 0, none_b = kb <= 0;
+            if (a_part || b_part) {
+                int c[4] = {0, 0, 0, 0};  // below s* and at s*, near then far
+                uint32_t plo_a = 0xffffffffu, phi_a = 0u, plo_b = 0xffffffffu, phi_b = 0u;
+                for (int q = tid; q < n; q += BT) {
+                    const uint64_t key = keys[q];
+                    const uint32_t sb = (uint32_t)(key >> 32), p = (uint32_t)key;
+                    const int delta = t - (int32_t)p;
+                    if (delta < 1) continue;
+                    if (strat && delta <= L.D) {
+                        c[0] += sb < alo;
+                        if (sb == alo) { ++c[1]; plo_a = min(plo_a, p); phi_a = max(phi_a, p); }
+                    } else {
+                        c[2] += sb < blo;
+                        if (sb == blo) { ++c[3]; plo_b = min(plo_b, p); phi_b = max(phi_b, p); }
+                    }
+                }
+                int (*rb)[32] = red[par];
+    #pragma unroll
+                for (int j = 0; j < 4; ++j) c[j] = __reduce_add_sync(FULL_MASK, c[j]);
+                plo_a = __reduce_min_sync(FULL_MASK, plo_a); phi_a = __reduce_max_sync(FULL_MASK, phi_a);
+                plo_b = __reduce_min_sync(FULL_MASK, plo_b); phi_b = __reduce_max_sync(FULL_MASK, phi_b);
+                if (lane == 0) {
+                    rb[warp][0] = c[0]; rb[warp][1] = c[1]; rb[warp][2] = c[2]; rb[warp][3] = c[3];
+                    rb[warp][4] = (int)plo_a; rb[warp][5] = (int)phi_a;
+                    rb[warp][6] = (int)plo_b; rb[warp][7] = (int)phi_b;
+                }
+                __syncthreads();
+                par ^= 1;
+                c[0] = c[1] = c[2] = c[3] = 0;
+                plo_a = plo_b = 0xffffffffu;
+                phi_a = phi_b = 0u;
+                for (int w = 0; w < NW; ++w) {
+                    c[0] += rb[w][0]; c[1] += rb[w][1]; c[2] += rb[w][2]; c[3] += rb[w][3];
+                    plo_a = min(plo_a, (uint32_t)rb[w][4]); phi_a = max(phi_a, (uint32_t)rb[w][5]);
+                    plo_b = min(plo_b, (uint32_t)rb[w][6]); phi_b = max(phi_b, (uint32_t)rb[w][7]);
+                }
+                const int need_a = ka - c[0], need_b = kb - c[2];  // 1 <= need <= eq
+                bool tie_a = a_part && need_a < c[1], tie_b = b_part && need_b < c[3];
+                if (a_part && !tie_a) plo_a = phi_a;  // every tied key goes
+                if (b_part && !tie_b) plo_b = phi_b;
+                // bisection on positions among the tied keys (rare: equal fp32 scores)
+                while ((tie_a && plo_a < phi_a) || (tie_b && plo_b < phi_b)) {
+                    const uint32_t mid_a = plo_a + ((phi_a - plo_a) >> 1);
+                    const uint32_t mid_b = plo_b + ((phi_b - plo_b) >> 1);
+                    int da = 0, db = 0;
+                    for (int q = tid; q < n; q += BT) {
+                        const uint64_t key = keys[q];
+                        const uint32_t sb = (uint32_t)(key >> 32), p = (uint32_t)key;
+                        const int delta = t - (int32_t)p;
+                        if (delta < 1) continue;
+                        if (strat && delta <= L.D) da += sb == alo && p <= mid_a;
+                        else db += sb == blo && p <= mid_b;
+                    }
+                    da = __reduce_add_sync(FULL_MASK, da);
+                    db = __reduce_add_sync(FULL_MASK, db);
+                    int (*rr)[32] = red[par];
+                    if (lane == 0) { rr[warp][0] = da; rr[warp][1] = db; }
+                    __syncthreads();
+                    par ^= 1;
+                    da = db = 0;
+                    for (int w = 0; w < NW; ++w) { da += rr[w][0]; db += rr[w][1]; }
+                    if (tie_a && plo_a < phi_a) { if (da >= need_a) phi_a = mid_a; else plo_a = mid_a + 1; }
+                    if (tie_b && plo_b < phi_b) { if (db >= need_b) phi_b = mid_b; else plo_b = mid_b + 1; }
+                }
+                if (a_part) thr_a = ((uint64_t)alo << 32) | plo_a;
+                if (b_part) thr_b = ((uint64_t)blo << 32) | plo_b;
+            }
+            // holes and movers, listed in (thread, token) order
+            int nh_mine = 0, nm_mine = 0;
+            for (int q = tid; q < n; q += BT) {
+                const uint64_t key = keys[q];
+                const int delta = t - (int32_t)(uint32_t)key;
+                bool ev = false;
+                if (delta >= 1) {
+                    if (strat && delta <= L.D) ev = !none_a && key <= thr_a;
+                    else ev = !none_b && key <= thr_b;
+                }
+                nh_mine += ev && q < target;
+                nm_mine += !ev && q >= target;
+            }
+            int xh = nh_mine, xm = nm_mine;  // inclusive scans over the warp
+    #pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int yh = __shfl_up_sync(FULL_MASK, xh, o), ym = __shfl_up_sync(FULL_MASK, xm, o);
+                if (lane >= o) { xh += yh; xm += ym; }
+            }
+            if (lane == 31) { lists[0][warp] = xh; lists[1][warp] = xm; }
+            __syncthreads();
+            int oh = xh - nh_mine, om = xm - nm_mine, nh = 0, nm = 0;
+            for (int w = 0; w < NW; ++w) {
+                if (w < warp) { oh += lists[0][w]; om += lists[1][w]; }
+                nh += lists[0][w];
+                nm += lists[1][w];
+            }
+            if (nh != nm || nh > M) {
+                if (tid == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
+                continue;
+            }
+            for (int q = tid; q < n; q += BT) {
+                const uint64_t key = keys[q];
+                const int delta = t - (int32_t)(uint32_t)key;
+                bool ev = false;
+                if (delta >= 1) {
+                    if (strat && delta <= L.D) ev = !none_a && key <= thr_a;
+                    else ev = !none_b && key <= thr_b;
+                }
+                if (ev && q < target) holes[oh++] = q;
+                if (!ev && q >= target) { movers[om] = q; mpos[om] = (int32_t)(uint32_t)key; ++om; }
+            }
+            __syncthreads();
+            // row moves: the i-th mover's K|V pair into the i-th hole, 16-byte
+            // pieces, up to 4 loads in flight per thread
+            const int pieces = nh * per_pair;
+            for (int w0 = 0; w0 < pieces; w0 += 4 * BT) {
+                uint4 x[4];
+    #pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int w = w0 + u * BT + tid;
+                    if (w < pieces) {
+                        const int i = w / per_pair, pc = w % per_pair;
+                        x[u] = *reinterpret_cast<const uint4*>(KVb + (slot0 + movers[i]) * pair + pc * 16);
+                    }
+                }
+    #pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int w = w0 + u * BT + tid;
+                    if (w < pieces) {
+                        const int i = w / per_pair, pc = w % per_pair;
+                        *reinterpret_cast<uint4*>(KVb + (slot0 + holes[i]) * pair + pc * 16) = x[u];
+                    }
+                }
+            }
+            for (int i = tid; i < nh; i += BT) L.pos[slot0 + holes[i]] = mpos[i];
+            if (tid == 0) {
+                atomicAdd(L.ev_stats + 0, 1ull);
+                atomicAdd(L.ev_stats + 1, (unsigned long long)n);
+                atomicAdd(L.ev_stats + 2, (unsigned long long)nh);
+            }
         }
     }
 }
@@ -284,30 +513,31 @@ __global__ void __launch_bounds__(128) select_batch_kernel(
 // launchers
 // ---------------------------------------------------------------------------
 
-static int evict_warps(size_t per) {
-    int w = (int)((200 * 1024) / per);
-    return w < 1 ? 1 : (w > EVICT_MAX_WARPS ? EVICT_MAX_WARPS : w);
+// Dynamic shared memory of an eviction block: keys of up to n_max tokens,
+// then the hole, mover and mover-position lists of up to M entries.
+static size_t evict_block_smem(int n_max, int M) { return (size_t)n_max * 8 + (size_t)M * 12; }
+
+int evict_blocks_per_sm(const Layout& L, int optin) {
+    const size_t sm = evict_block_smem(L.L, L.M) + 5120;  // + static
+    int by_threads = 3;  // registers: see the kernel's launch bounds
+    int by_smem = (int)((size_t)optin * 1 / sm);
+    int b = by_threads < by_smem ? by_threads : by_smem;
+    return b < 1 ? 1 : b;
 }
 
 cudaError_t launch_evict(const Layout& L, int l0, int l1, int grid, cudaStream_t st) {
-    const int heads = (l1 - l0) * L.S * L.H;
-    evict_scan_kernel<<<(heads + 255) / 256, 256, 0, st>>>(L, l0, l1);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
     const int n_max = L.L;
-    const size_t per = evict_warp_bytes(n_max, L.M, L.d * (L.dtype == HKV_DTYPE_F32 ? 4 : 2));
-    const int nw = evict_warps(per);
-    const size_t sm = (size_t)nw * per;
+    const size_t sm = evict_block_smem(n_max, L.M);
     if (L.dtype == HKV_DTYPE_BF16)
-        evict_run_kernel<__nv_bfloat16><<<grid, 32 * nw, sm, st>>>(L, n_max);
+        evict_block_kernel<__nv_bfloat16><<<grid, EVB_THREADS, sm, st>>>(L, l0, l1, n_max);
     else
-        evict_run_kernel<float><<<grid, 32 * nw, sm, st>>>(L, n_max);
+        evict_block_kernel<float><<<grid, EVB_THREADS, sm, st>>>(L, l0, l1, n_max);
     return cudaGetLastError();
 }
 
 cudaError_t prepare_evict(int smem) {
-    cudaError_t e = allow_max_dynamic_smem(evict_run_kernel<__nv_bfloat16>, smem);
-    if (e == cudaSuccess) e = allow_max_dynamic_smem(evict_run_kernel<float>, smem);
+    cudaError_t e = allow_max_dynamic_smem(evict_block_kernel<__nv_bfloat16>, smem);
+    if (e == cudaSuccess) e = allow_max_dynamic_smem(evict_block_kernel<float>, smem);
     if (e == cudaSuccess) e = allow_max_dynamic_smem(select_batch_kernel, smem);
     return e;
 }

@@ -130,7 +130,7 @@ size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Lay
     l.t_next = (int32_t*)take(Ly * 4);
     l.done_ctr = (int32_t*)take(Ly * 4);
     l.ticket = (int32_t*)take(2 * S * H * 4);  // two sets: consecutive decode launches alternate
-    l.due_ctl = (int32_t*)take(16);
+    l.ev_stats = (unsigned long long*)take(3 * 8);
     const size_t ctrl_end = o;
     l.off = (int32_t*)take(nh * 4);
     l.cap = (int32_t*)take(nh * 4);
@@ -146,7 +146,8 @@ size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Lay
     l.ml = (float2*)take(nh * r * 8);
     l.rows = (float*)take(S * H * r * Lmax * 4);
     l.partial = (float*)take(2 * 2 * (size_t)hkv::PLAN_MAX_WARPS * (d + 2) * 4);
-    l.due_list = (int32_t*)take(nh * 4);
+    l.unit_due = (int32_t*)take(Ly * S * 4);
+    l.unit_gmask = (uint32_t*)take(Ly * S * 4);
     l.plan_desc = (int4*)take(Ly * max_chunks * 16);
     l.plan_warp = (int4*)take(Ly * hkv::PLAN_MAX_WARPS * (1 + hkv::PLAN_WARP_DESC) * 16);
     l.S = c->num_seqs; l.Ly = c->num_layers; l.H = c->num_heads; l.d = c->head_dim;
@@ -161,13 +162,13 @@ size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Lay
 }
 
 size_t ctrl_bytes(const hkv_config* c) {
-    // status, t_next, done_ctr, ticket and due_ctl are laid out first (see carve)
+    // status, t_next, done_ctr, ticket and ev_stats are laid out first (see carve)
     size_t o = 0;
     o = align_up(o + 16);
     o = align_up(o + (size_t)c->num_layers * 4);
     o = align_up(o + (size_t)c->num_layers * 4);
     o = align_up(o + 2 * (size_t)c->num_seqs * c->num_heads * 4);
-    o = align_up(o + 16);
+    o = align_up(o + 3 * 8);
     return o;
 }
 
@@ -243,7 +244,7 @@ hkv_status hkv_create(const hkv_config* cfg, void* pool, size_t bytes, void* str
     c->lay.plan_gw = c->decode_grid * c->decode_sh.warps;
     c->lay.plan_nw = c->decode_sh.warps;
     c->plan_for.assign(cfg->num_layers, -1);
-    c->evict_grid = c->n_sm;
+    c->evict_grid = c->n_sm * hkv::evict_blocks_per_sm(c->lay, optin);
     *out = c;
     return HKV_OK;
 }
@@ -270,7 +271,7 @@ static hkv_status prefill_args(const hkv_ctx* c, int32_t layer, const void* q, c
 // Marks `layer` ready for appends and decodes at length P and enqueues its
 // first decode plan.
 static hkv_status prefill_done(hkv_ctx* c, int32_t layer, int P, void* stream) {
-    if (hkv::launch_plan(c->lay, layer, layer + 1, 1, (cudaStream_t)stream) != cudaSuccess)
+    if (hkv::launch_plan(c->lay, layer, layer + 1, 1, 0, (cudaStream_t)stream) != cudaSuccess)
         return HKV_ERR_CUDA;
     c->plan_for[layer] = P;
     c->classified[layer] = 1;
@@ -352,7 +353,7 @@ hkv_status hkv_decode_attend(hkv_ctx* c, int32_t layer, const void* q_t, void* o
     cudaError_t e = cudaSuccess;
     if (c->plan_for[layer] != t) {
         note_other(c, stream);
-        e = hkv::launch_plan(c->lay, layer, layer + 1, 0, (cudaStream_t)stream);
+        e = hkv::launch_plan(c->lay, layer, layer + 1, 0, 0, (cudaStream_t)stream);
         c->plan_for[layer] = t;
     }
     if (e == cudaSuccess) e = decode_launch(c, layer, q_t, nullptr, nullptr, o_t, 0, stream);
@@ -370,7 +371,7 @@ hkv_status hkv_decode_step(hkv_ctx* c, int32_t layer, const void* q_t, const voi
     cudaError_t e = cudaSuccess;
     if (c->plan_for[layer] != t) {
         note_other(c, stream);
-        e = hkv::launch_plan(c->lay, layer, layer + 1, 1, (cudaStream_t)stream);
+        e = hkv::launch_plan(c->lay, layer, layer + 1, 1, 0, (cudaStream_t)stream);
         c->plan_for[layer] = t;
     }
     if (e == cudaSuccess) e = decode_launch(c, layer, q_t, k_t, v_t, o_t, 1, stream);
@@ -388,9 +389,11 @@ hkv_status hkv_ste_evict(hkv_ctx* c, int32_t layer_begin, int32_t layer_end, voi
     note_other(c, stream);
     if (c->cfg.mode != HKV_MODE_FULL)
         e = hkv::launch_evict(c->lay, layer_begin, layer_end, c->evict_grid, (cudaStream_t)stream);
-    // plans of the next step, made once for all these layers
+    // plans of the next step, made once for all these layers, with the new
+    // lengths of the heads just evicted
     if (e == cudaSuccess)
-        e = hkv::launch_plan(c->lay, layer_begin, layer_end, 1, (cudaStream_t)stream);
+        e = hkv::launch_plan(c->lay, layer_begin, layer_end, 1, c->cfg.mode != HKV_MODE_FULL,
+                             (cudaStream_t)stream);
     if (e != cudaSuccess) return HKV_ERR_CUDA;
     for (int l = layer_begin; l < layer_end; ++l) c->plan_for[l] = c->t_host[l];
     return HKV_OK;
@@ -463,6 +466,11 @@ hkv_status hkv_get_kept(hkv_ctx* c, int32_t seq, int32_t layer, int32_t head, in
         pos_host[j + 1] = x;
     }
     return HKV_OK;
+}
+
+hkv_status hkv_get_evict_stats(hkv_ctx* c, int64_t* stats_host, void* stream) {
+    if (!c || !stats_host) return HKV_ERR_INVALID_ARG;
+    return copy_back(stats_host, c->lay.ev_stats, 3 * 8, stream);
 }
 
 hkv_status hkv_check(hkv_ctx* c, int32_t* detail_host, void* stream) {

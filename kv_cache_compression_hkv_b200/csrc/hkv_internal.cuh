@@ -33,6 +33,7 @@ struct Layout {
     int32_t* status;    // [0] first error code, [1] detail
     int32_t* t_next;    // [Ly] position the next append writes
     int32_t* done_ctr;  // [Ly] CTA arrivals of the running decode launch
+    unsigned long long* ev_stats;  // [3] heads evicted, tokens scored, rows moved
     // per (layer, sequence, head) metadata, index (l*S + s)*H + h
     int32_t* off;       // first slot of the head inside its region
     int32_t* cap;       // slots reserved for the head
@@ -52,8 +53,11 @@ struct Layout {
     float* rows;        // [S*H][r][prefill_len] weights of the last r prefill queries
     float* partial;     // [2][PLAN_MAX_WARPS][2][d + 2] split-K partial states
     int32_t* ticket;    // [2][S*H] arrivals per head of the running decode launch
-    int32_t* due_ctl;   // [0] due heads listed, [1] blocks of the eviction done
-    int32_t* due_list;  // [Ly*S*H] heads due for eviction this step
+    // per (layer, sequence) "unit", index l*S + s: the step at which its
+    // Global heads reach their capacity (INT32_MAX: none), kept by the plan
+    // kernel; the Global heads held here as a bit mask (H <= 32)
+    int32_t* unit_due;
+    uint32_t* unit_gmask;
     // decode plan per layer, for the step it was made for (see plan_kernel)
     int4* plan_desc;     // [Ly][max_chunks] one descriptor per chunk
     // [Ly][PLAN_MAX_WARPS][1 + PLAN_WARP_DESC]: per warp {first chunk, end

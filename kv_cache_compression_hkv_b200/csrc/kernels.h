@@ -34,7 +34,10 @@ cudaError_t launch_prefill_compress(const Layout& L, int layer, const void* k, c
 struct DecodeShape {
     int warps, nstage;
     size_t smem;
-    int per_sm;  // resident blocks per SM
+    int per_sm;    // resident blocks per SM
+    int prologue;  // stages a warp fills before its first chunk lands:
+                   // 0 one when the block has 8 or more warps, else all;
+                   // 1 one; 2 all
 };
 DecodeShape decode_shape(const Layout& L, size_t smem_limit);
 // early: the previous launch in `st` is a decode launch of another layer (the
@@ -43,7 +46,8 @@ DecodeShape decode_shape(const Layout& L, size_t smem_limit);
 cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void* k, const void* v,
                           void* o, int append, const DecodeShape& sh, int grid, int early, int buf,
                           cudaStream_t st);
-cudaError_t launch_plan(const Layout& L, int l0, int l1, int ahead, cudaStream_t st);
+// commit: the launch right after an eviction (see plan_kernel)
+cudaError_t launch_plan(const Layout& L, int l0, int l1, int ahead, int commit, cudaStream_t st);
 // Shared memory of the plan kernel: four words per head of a layer, two per
 // warp of the decode grid (and one more), two bytes per chunk.
 inline size_t plan_smem_bytes(int heads_per_layer, int max_chunks) {
@@ -54,6 +58,8 @@ cudaError_t launch_prefill_rows_simt(int dtype, int d, int n_blocks, const void*
                                      float* rows, cudaStream_t st);
 cudaError_t launch_append(const Layout& L, int layer, const void* k, const void* v, cudaStream_t st);
 cudaError_t launch_evict(const Layout& L, int l0, int l1, int grid, cudaStream_t st);
+// Eviction blocks one SM holds at once (the eviction grid is this times the SMs).
+int evict_blocks_per_sm(const Layout& L, int optin);
 cudaError_t launch_classify_groups(const float* rows, int n_units, int r, int nq, int n,
                                    const int32_t* partner, int W, double tau, int32_t* n_tau,
                                    uint8_t* label, cudaStream_t st);

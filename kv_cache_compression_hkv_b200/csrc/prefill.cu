@@ -105,12 +105,13 @@ __device__ void lay_out_heads(const Layout& L, int layer, int s, int P, const ui
     else if (L.mode == HKV_MODE_UNIFORM) bg = (int)(L.T_total / L.H_total);
     else bg = L.L;
     int o = 0;
+    uint32_t gmask = 0;
     for (int j = 0; j < L.H; ++j) {
         const size_t hi = head_index(L, layer, s, j);
         int cap, budget, len0;
         if (lab[j] == 1) { cap = L.W; budget = L.W; len0 = P < L.W ? P : L.W; }
         else if (lab[j] == 2) { cap = L.L; budget = L.L; len0 = P; }
-        else { cap = bg + L.M; budget = bg; len0 = P < bg ? P : bg; }
+        else { cap = bg + L.M; budget = bg; len0 = P < bg ? P : bg; gmask |= 1u << j; }
         L.off[hi] = o;
         L.cap[hi] = cap;
         L.budget[hi] = budget;
@@ -121,6 +122,11 @@ __device__ void lay_out_heads(const Layout& L, int layer, int s, int P, const ui
         o += cap;
     }
     if (o > L.R) latch_error(L, HKV_ERR_CAPACITY, layer * L.S + s);
+    // the Global heads of a unit share capacity and length: one due step
+    const size_t u = (size_t)layer * L.S + s;
+    L.unit_gmask[u] = gmask;
+    const int len0_g = P < bg ? P : bg;
+    L.unit_due[u] = gmask ? (P - 1) + (bg + L.M - len0_g) : INT32_MAX;
     if (s == 0) L.t_next[layer] = P;
 }
 

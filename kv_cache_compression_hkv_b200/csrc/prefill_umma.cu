@@ -2,19 +2,19 @@
 // cores (tcgen05) for bf16 caches (HeadKV technical summary, Methodology
 // step 1, cache prefilling: its weights feed step 2, head grouping).
 //
-// One CTA (4 warps) per (sequence*head block, 128-query tile).  TMA brings
-// the Q tile (128 x d) once and the K / V tiles (64 keys x d) per key tile,
-// all with the 128-byte swizzle the tensor cores read.  Two passes over the
-// key tiles (keys up to the tile's causal limit):
-//   pass 1: S = Q K^T (M=128, N=64) into TMEM; thread i owns query row i
-//           (TMEM lane i) and keeps its running max and sum;
-//   pass 2: S again; P = exp2(S - max) / sum exactly normalised, written as
-//           bf16 into shared memory in the canonical K-major layout; the
-//           last r query rows also store their fp32 weights for the
-//           grouping; O += P V (V as the MN-major operand) in TMEM.
-// The epilogue reads O from TMEM and stores bf16 rows.  Every wait on an
-// mbarrier is bounded in time; a wait that gives up latches HKV_ERR_TIMEOUT,
-// waits (bounded) for the block's own copies, frees TMEM and returns.
+// One CTA (6 warps) per (sequence*head block, 128-query tile), one pass
+// over the key tiles (64 keys each, up to the tile's causal limit) with the
+// work split by role: a TMA warp brings the Q tile once and the K / V tiles
+// into two stages (128-byte swizzle, the layout the tensor cores read); an
+// MMA warp issues S = Q K^T (M=128, N=64) into one of two TMEM slots and
+// O += P V (V as the MN-major operand) into a TMEM accumulator; four row
+// warps (thread i owns query row i = TMEM lane i) turn S into bf16 weights
+// P with an online maximum and sum.  The tensor cores work on tiles j and
+// j-1 while the rows work on tile j.  The epilogue reads O from TMEM and
+// stores bf16 rows, and normalises the fp32 weights of the last r query
+// rows over every key for the grouping.  Every wait on an mbarrier is
+// bounded in time; a wait that gives up latches HKV_ERR_TIMEOUT, the block
+// waits (bounded) for its own copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
 #include <math.h>
 
@@ -91,39 +91,91 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Roles of the 192 threads of a CTA: warps 0-3 own the 128 query rows
+// (TMEM lane = row) and do the softmax and the epilogue; warp 4's lane 0
+// issues the TMA copies; warp 5's lane 0 issues the MMAs.
+constexpr int NTHREADS = 192;
+constexpr int PRODUCER_WARP = 4;
+constexpr int MMA_WARP = 5;
+// A row's reference maximum (log2 domain) is raised, and O rescaled, only
+// when a logit passes it by more than this: the weights stay below 2^8.
+constexpr float RESCALE = 8.f;
+
+// Barriers of the pipeline (two stages each, a stage per key-tile parity).
+enum Bar {
+    B_Q = 0,
+    B_KFULL = 1,   // +stage: K tile landed
+    B_VFULL = 3,   // +stage: V tile landed
+    B_SFULL = 5,   // +stage: S = Q K^T of the stage's tile in TMEM
+    B_SFREE = 7,   // +stage: the softmax rows have read that S (128 arrivals)
+    B_PFULL = 9,   // +stage: P of the tile in shared memory, O rescaled (128 arrivals)
+    B_PVDONE = 11, // +stage: O += P V of the tile done: K, V and P of the stage free
+    B_COUNT = 13
+};
+
 struct Smem {
-    // 1024-byte aligned tiles (128B swizzle atoms)
+    // 1024-byte aligned tiles (128B swizzle atoms): Q, K[2], V[2], P[2]
     __host__ __device__ static constexpr int q_bytes(int d) { return QT * d * 2; }
     __host__ __device__ static constexpr int kv_bytes(int d) { return KT * d * 2; }
     __host__ __device__ static constexpr int p_bytes() { return QT * KT * 2; }
-    __host__ __device__ static constexpr int total(int d) { return 1024 + q_bytes(d) + 2 * kv_bytes(d) + p_bytes() + 64; }
+    __host__ __device__ static constexpr int total(int d) {
+        return 1024 + q_bytes(d) + 4 * kv_bytes(d) + 2 * p_bytes() + B_COUNT * 8 + 16;
+    }
 };
 
+// Causal attention of one (block, 128-query tile) in one pass over the key
+// tiles, pipelined over two stages:
+//   producer: K_j, V_j into stage j % 2 once O += P V of tile j-2 is done;
+//   MMA:      S_j = Q K_j^T into TMEM columns 64 (j % 2) (once the rows
+//             have read S_{j-2}), then O += P_{j-1} V_{j-1} into columns
+//             128.. (once the rows have written P_{j-1}), so the rows' work
+//             on tile j overlaps the tensor cores' work on tiles j and j-1;
+//   rows:     read S_j, raise the reference maximum m only when a logit
+//             passes it by more than RESCALE (then O, once P_{j-1} V_{j-1}
+//             is in, is rescaled in TMEM), P_j = exp2(S_j - m) as bf16 into
+//             stage j % 2 of P (once P_{j-2} V_{j-2} is done), running sum l.
+// Epilogue: O / l as bf16 rows; the last r rows' fp32 weights
+// exp2(s - m) / l over every key (their scaled logits were kept in `rows`
+// during the pass and are normalised in place).
 template <int D>
-__global__ void __launch_bounds__(128) prefill_attn_umma(
+__global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
     const __grid_constant__ CUtensorMap vmap, int P, int r, __nv_bfloat16* __restrict__ out,
     float* __restrict__ rows, int32_t* __restrict__ status) {
     extern __shared__ unsigned char raw[];
     unsigned char* base = reinterpret_cast<unsigned char*>(((uintptr_t)raw + 1023) & ~(uintptr_t)1023);
     unsigned char* q_s = base;
-    unsigned char* k_s = q_s + Smem::q_bytes(D);
-    unsigned char* v_s = k_s + Smem::kv_bytes(D);
-    unsigned char* p_s = v_s + Smem::kv_bytes(D);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(p_s + Smem::p_bytes());
-    uint64_t* bar_q = bars + 0;
-    uint64_t* bar_k = bars + 1;
-    uint64_t* bar_v = bars + 2;
-    uint64_t* bar_m = bars + 3;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+    unsigned char* k_s = q_s + Smem::q_bytes(D);        // [2] stages
+    unsigned char* v_s = k_s + 2 * Smem::kv_bytes(D);   // [2]
+    unsigned char* p_s = v_s + 2 * Smem::kv_bytes(D);   // [2]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(p_s + 2 * Smem::p_bytes());
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
 
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = blockIdx.x;            // sequence * H + head
     const int q0 = blockIdx.y * QT;      // first query of the tile
     const int n_keys = min(P, q0 + QT);  // causal limit of the tile
     const int nkt = (n_keys + KT - 1) / KT;
     constexpr int NSUB = D / 64;         // 64-column swizzle sub-tiles
     constexpr uint64_t WAIT_NS = 2000000000ull;
+    constexpr int KVB = Smem::kv_bytes(D), PB = Smem::p_bytes();
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -132,178 +184,210 @@ __global__ void __launch_bounds__(128) prefill_attn_umma(
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     if (tid == 0) {
-        mbar_init(bar_q, 1);
-        mbar_init(bar_k, 1);
-        mbar_init(bar_v, 1);
-        mbar_init(bar_m, 1);
+        for (int i = 0; i < B_COUNT; ++i) {
+            const bool rows_arrive = (i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL || i == B_PFULL + 1);
+            mbar_init(bars + i, rows_arrive ? QT : 1);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     fence_before();
     __syncthreads();
     fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's lane quarter
-
-    uint32_t ph_k = 0, ph_v = 0, ph_m = 0;
     bool fail = false;
-    int pending_k = 0, pending_v = 0, pending_q = 0;
 
-    if (tid == 0) {
-        mbar_expect_tx(bar_q, Smem::q_bytes(D));
-        for (int s = 0; s < NSUB; ++s) tma_load_3d(q_s + s * QT * 128, &qmap, bar_q, s * 64, q0, b);
-    }
-    pending_q = 1;
-
-    const float scale = LOG2E / sqrtf((float)D);
-    const int row = tid;  // query q0 + row, TMEM lane = row
-    const int qpos = q0 + row;
-    float m = -INFINITY, l = 0.f;
-    constexpr uint32_t IDESC_S = idesc_bf16(KT, false);
-    constexpr uint32_t IDESC_O = idesc_bf16(D, true);
-
-    for (int pass = 0; pass < 2 && !fail; ++pass) {
-        for (int j = 0; j < nkt; ++j) {
-            if (tid == 0) {
-                mbar_expect_tx(bar_k, Smem::kv_bytes(D));
-                for (int s = 0; s < NSUB; ++s) tma_load_3d(k_s + s * KT * 128, &kmap, bar_k, s * 64, j * KT, b);
-                if (pass == 1) {
-                    mbar_expect_tx(bar_v, Smem::kv_bytes(D));
-                    for (int s = 0; s < NSUB; ++s)
-                        tma_load_3d(v_s + s * KT * 128, &vmap, bar_v, s * 64, j * KT, b);
-                }
+    if (warp == PRODUCER_WARP) {
+        // --- TMA producer -------------------------------------------------
+        uint32_t issued = 0;  // bit s: stage s has a load that may be in flight
+        uint32_t last_par = 0;  // bit s: parity of that load's phase
+        if (lane == 0) {
+            mbar_expect_tx(bars + B_Q, Smem::q_bytes(D));
+            for (int sub = 0; sub < NSUB; ++sub)
+                tma_load_3d(q_s + sub * QT * 128, &qmap, bars + B_Q, sub * 64, q0, b);
+            for (int j = 0; j < nkt && !fail; ++j) {
+                const int st = j & 1, k = j >> 1;
+                if (j >= 2 && !mbar_wait(bars + B_PVDONE + st, (k - 1) & 1, WAIT_NS)) { fail = true; break; }
+                mbar_expect_tx(bars + B_KFULL + st, KVB);
+                for (int sub = 0; sub < NSUB; ++sub)
+                    tma_load_3d(k_s + st * KVB + sub * KT * 128, &kmap, bars + B_KFULL + st, sub * 64, j * KT, b);
+                mbar_expect_tx(bars + B_VFULL + st, KVB);
+                for (int sub = 0; sub < NSUB; ++sub)
+                    tma_load_3d(v_s + st * KVB + sub * KT * 128, &vmap, bars + B_VFULL + st, sub * 64, j * KT, b);
+                issued |= 1u << st;
+                last_par = (last_par & ~(1u << st)) | ((uint32_t)(k & 1) << st);
             }
-            pending_k = 1;
-            pending_v = pass == 1;
-            bool ok = true;
-            if (pending_q) { ok = mbar_wait(bar_q, 0, WAIT_NS); pending_q = 0; }
-            ok = ok && mbar_wait(bar_k, ph_k, WAIT_NS);
-            if (ok) { ph_k ^= 1; pending_k = 0; }
-            if (__syncthreads_or(!ok)) { fail = true; break; }
-            // S = Q K^T
-            if (tid == 0) {
-                fence_after();
+            if (fail) {
+                // the block's own copies land before its shared memory goes
+                mbar_wait(bars + B_Q, 0, WAIT_NS);
+                for (int st = 0; st < 2; ++st)
+                    if (issued & (1u << st)) {
+                        mbar_wait(bars + B_KFULL + st, (last_par >> st) & 1, WAIT_NS);
+                        mbar_wait(bars + B_VFULL + st, (last_par >> st) & 1, WAIT_NS);
+                    }
+            }
+        }
+    } else if (warp == MMA_WARP) {
+        // --- MMA issuer ---------------------------------------------------
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = idesc_bf16(KT, false);
+            constexpr uint32_t IDESC_O = idesc_bf16(D, true);
+            int committed = -1;  // last tile whose P V was committed
+            int s_issued = -1;   // last tile whose S was committed
+            if (!mbar_wait(bars + B_Q, 0, WAIT_NS)) fail = true;
+            for (int j = 0; j <= nkt && !fail; ++j) {
+                if (j < nkt) {
+                    const int st = j & 1, k = j >> 1;
+                    if (!mbar_wait(bars + B_KFULL + st, k & 1, WAIT_NS)) { fail = true; break; }
+                    if (j >= 2 && !mbar_wait(bars + B_SFREE + st, (k - 1) & 1, WAIT_NS)) { fail = true; break; }
+                    fence_after();
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t qa = smem_u32(q_s) + (kk / 4) * (QT * 128) + (kk % 4) * 32;
-                    const uint32_t ka = smem_u32(k_s) + (kk / 4) * (KT * 128) + (kk % 4) * 32;
-                    mma_bf16(tmem, sw128_desc(qa, 16, 1024), sw128_desc(ka, 16, 1024), IDESC_S, kk > 0);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t qa = smem_u32(q_s) + (kk / 4) * (QT * 128) + (kk % 4) * 32;
+                        const uint32_t ka = smem_u32(k_s + st * KVB) + (kk / 4) * (KT * 128) + (kk % 4) * 32;
+                        mma_bf16(tmem + st * KT, sw128_desc(qa, 16, 1024), sw128_desc(ka, 16, 1024), IDESC_S,
+                                 kk > 0);
+                    }
+                    mma_commit(bars + B_SFULL + st);
+                    s_issued = j;
                 }
-                mma_commit(bar_m);
+                if (j >= 1) {
+                    const int jp = j - 1, sp = jp & 1, kp = jp >> 1;
+                    if (!mbar_wait(bars + B_PFULL + sp, kp & 1, WAIT_NS) ||
+                        !mbar_wait(bars + B_VFULL + sp, kp & 1, WAIT_NS)) { fail = true; break; }
+                    fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < KT / 16; ++kk) {
+                        const uint32_t pa = smem_u32(p_s + sp * PB) + kk * 32;
+                        const uint32_t va = smem_u32(v_s + sp * KVB) + kk * 16 * 128;
+                        mma_bf16(tmem + O_COL, sw128_desc(pa, 16, 1024), sw128_desc(va, KT * 128, 1024),
+                                 IDESC_O, (jp > 0 || kk > 0));
+                    }
+                    mma_commit(bars + B_PVDONE + sp);
+                    committed = jp;
+                }
             }
-            ok = mbar_wait(bar_m, ph_m, WAIT_NS);
-            if (ok) ph_m ^= 1;
-            if (__syncthreads_or(!ok)) { fail = true; break; }
+            // the tensor cores finish what was issued before TMEM is freed
+            // (a commit covers every MMA issued before it)
+            if (s_issued > committed)
+                mbar_wait(bars + B_SFULL + (s_issued & 1), (s_issued >> 1) & 1, WAIT_NS);
+            else if (committed >= 0)
+                mbar_wait(bars + B_PVDONE + (committed & 1), (committed >> 1) & 1, WAIT_NS);
+        }
+    } else {
+        // --- rows: softmax and epilogue ------------------------------------
+        const int row = tid;  // query q0 + row, TMEM lane = row
+        const int qpos = q0 + row;
+        const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's lane quarter
+        const float scale = LOG2E / sqrtf((float)D);
+        const bool keep_row = qpos >= P - r && qpos < P;
+        float* rrow = keep_row ? rows + ((size_t)b * r + (qpos - (P - r))) * P : nullptr;
+        float m = -INFINITY, l = 0.f;
+        for (int j = 0; j < nkt; ++j) {
+            const int st = j & 1, k = j >> 1;
+            if (!mbar_wait(bars + B_SFULL + st, k & 1, WAIT_NS)) { fail = true; break; }
             fence_after();
             uint32_t sr[2][32];
-            tmem_ld32(t_row + 0, sr[0]);
-            tmem_ld32(t_row + 32, sr[1]);
+            tmem_ld32(t_row + st * KT, sr[0]);
+            tmem_ld32(t_row + st * KT + 32, sr[1]);
             tmem_ld_wait();
-            if (pass == 0) {
-                float mx = m;
+            fence_before();
+            mbar_arrive(bars + B_SFREE + st);
+            float x[KT];
+            float mt = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < KT; ++c) {
-                    const int key = j * KT + c;
-                    const float s = (key <= qpos && key < P) ? __uint_as_float(sr[c >> 5][c & 31]) * scale : -INFINITY;
-                    mx = fmaxf(mx, s);
-                }
-                float acc = l * exp2f(m - mx);
-                if (mx == -INFINITY) acc = 0.f;
-#pragma unroll
-                for (int c = 0; c < KT; ++c) {
-                    const int key = j * KT + c;
-                    if (key <= qpos && key < P) acc += exp2f(__uint_as_float(sr[c >> 5][c & 31]) * scale - mx);
-                }
-                l = acc;
-                m = mx;
-                fence_before();
-                __syncthreads();
-                continue;
+            for (int c = 0; c < KT; ++c) {
+                const int key = j * KT + c;
+                x[c] = (key <= qpos && key < P) ? __uint_as_float(sr[c >> 5][c & 31]) * scale : -INFINITY;
+                mt = fmaxf(mt, x[c]);
             }
-            // pass 2: exact weights -> bf16 P tile (K-major, 128B swizzle)
-            const float inv_l = 1.0f / l;
-            const bool keep_row = qpos >= P - r && qpos < P;
-            float* rrow = keep_row ? rows + ((size_t)b * r + (qpos - (P - r))) * P : nullptr;
+            if (rrow) {
+#pragma unroll
+                for (int c = 0; c < KT; ++c) {
+                    const int key = j * KT + c;
+                    if (key < P) rrow[key] = x[c];  // normalised in the epilogue
+                }
+            }
+            if (mt > m + RESCALE) {
+                const float alpha = exp2f(m - mt);  // 0 on the first tile
+                if (j > 0) {
+                    // O holds P V up to tile j-1: rescale it once that is in
+                    const int jp = j - 1;
+                    if (!mbar_wait(bars + B_PVDONE + (jp & 1), (jp >> 1) & 1, WAIT_NS)) { fail = true; break; }
+                    fence_after();
+#pragma unroll
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        uint32_t o[32];
+                        tmem_ld32(t_row + O_COL + c0, o);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(t_row + O_COL + c0, o);
+                    }
+                    tmem_st_wait();
+                }
+                l *= alpha;
+                m = mt;
+            }
+            // stage st of P is free once P V of tile j-2 is done
+            if (j >= 2 && !mbar_wait(bars + B_PVDONE + st, (k - 1) & 1, WAIT_NS)) { fail = true; break; }
+            unsigned char* pst = p_s + st * PB;
 #pragma unroll
             for (int ch = 0; ch < KT / 8; ++ch) {
                 uint32_t w[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    float pv[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int c = ch * 8 + e * 2 + u;
-                        const int key = j * KT + c;
-                        const bool valid = key <= qpos && key < P;
-                        pv[u] = valid ? exp2f(__uint_as_float(sr[c >> 5][c & 31]) * scale - m) * inv_l : 0.f;
-                        if (rrow && key < P) rrow[key] = pv[u];
-                    }
-                    __nv_bfloat162 h2 = __floats2bfloat162_rn(pv[0], pv[1]);
+                    const float p0 = exp2f(x[ch * 8 + 2 * e] - m), p1 = exp2f(x[ch * 8 + 2 * e + 1] - m);
+                    l += p0 + p1;
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
                     w[e] = *reinterpret_cast<uint32_t*>(&h2);
                 }
                 const uint32_t off = row * 128 + ((ch ^ (row & 7)) << 4);
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(p_s) + off),
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(pst) + off),
                              "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
                              : "memory");
             }
             fence_proxy_async();
             fence_before();
-            ok = mbar_wait(bar_v, ph_v, WAIT_NS);
-            if (ok) { ph_v ^= 1; pending_v = 0; }
-            if (__syncthreads_or(!ok)) { fail = true; break; }
-            // O += P V
-            if (tid == 0) {
-                fence_after();
-#pragma unroll
-                for (int kk = 0; kk < KT / 16; ++kk) {
-                    const uint32_t pa = smem_u32(p_s) + kk * 32;
-                    const uint32_t va = smem_u32(v_s) + kk * 16 * 128;
-                    mma_bf16(tmem + O_COL, sw128_desc(pa, 16, 1024), sw128_desc(va, KT * 128, 1024),
-                             IDESC_O, (j > 0 || kk > 0));
-                }
-                mma_commit(bar_m);
-            }
-            ok = mbar_wait(bar_m, ph_m, WAIT_NS);
-            if (ok) ph_m ^= 1;
-            if (__syncthreads_or(!ok)) { fail = true; break; }
+            mbar_arrive(bars + B_PFULL + st);
         }
-    }
-
-    if (!fail) {
-        // weights of the kept rows past this tile's causal limit are zero
-        if (qpos >= P - r && qpos < P)
-            for (int key = n_keys; key < P; ++key) rows[((size_t)b * r + (qpos - (P - r))) * P + key] = 0.f;
-        fence_after();
-        if (out != nullptr) {
+        if (!fail && nkt > 0) {
+            const int jl = nkt - 1;
+            if (!mbar_wait(bars + B_PVDONE + (jl & 1), (jl >> 1) & 1, WAIT_NS)) fail = true;
+        }
+        if (!fail) {
+            fence_after();
+            const float inv_l = 1.0f / l;
+            if (rrow) {
+                // the kept rows' weights over every key, exactly normalised
+                for (int key = 0; key < P; ++key)
+                    rrow[key] = key <= qpos ? exp2f(rrow[key] - m) * inv_l : 0.f;
+            }
+            if (out != nullptr) {
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t o[32];
-                tmem_ld32(t_row + O_COL + c0, o);
-                tmem_ld_wait();
-                if (qpos < P) {
-                    __nv_bfloat16* orow = out + ((size_t)b * P + qpos) * D + c0;
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(t_row + O_COL + c0, o);
+                    tmem_ld_wait();
+                    if (qpos < P) {
+                        __nv_bfloat16* orow = out + ((size_t)b * P + qpos) * D + c0;
 #pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        uint32_t w[4];
+                        for (int e = 0; e < 32; e += 8) {
+                            uint32_t w[4];
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[e + 2 * u]),
-                                                                      __uint_as_float(o[e + 2 * u + 1]));
-                            w[u] = *reinterpret_cast<uint32_t*>(&h2);
+                            for (int u = 0; u < 4; ++u) {
+                                __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[e + 2 * u]) * inv_l,
+                                                                          __uint_as_float(o[e + 2 * u + 1]) * inv_l);
+                                w[u] = *reinterpret_cast<uint32_t*>(&h2);
+                            }
+                            *reinterpret_cast<uint4*>(orow + e) = make_uint4(w[0], w[1], w[2], w[3]);
                         }
-                        *reinterpret_cast<uint4*>(orow + e) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 }
             }
         }
-    } else {
-        if (tid == 0) {
-            if (atomicCAS(status, 0, HKV_ERR_TIMEOUT) == 0) atomicExch(status + 1, b);
-            // let the block's own copies land before its shared memory is released
-            if (pending_q) mbar_wait(bar_q, 0, WAIT_NS);
-            if (pending_k) mbar_wait(bar_k, ph_k, WAIT_NS);
-            if (pending_v) mbar_wait(bar_v, ph_v, WAIT_NS);
-        }
     }
+    if (__syncthreads_or(fail) && tid == 0)
+        if (atomicCAS(status, 0, HKV_ERR_TIMEOUT) == 0) atomicExch(status + 1, b);
     fence_before();
     __syncthreads();
     fence_after();
@@ -360,10 +444,10 @@ cudaError_t launch_prefill_umma(const Layout& L, const void* q, const void* k, c
     dim3 grid(nblk, (P + umma::QT - 1) / umma::QT);
     const size_t sm = umma::Smem::total(L.d);
     if (L.d == 128)
-        umma::prefill_attn_umma<128><<<grid, 128, sm, st>>>(qm, km, vm, P, L.r, (__nv_bfloat16*)out,
+        umma::prefill_attn_umma<128><<<grid, umma::NTHREADS, sm, st>>>(qm, km, vm, P, L.r, (__nv_bfloat16*)out,
                                                            L.rows, L.status);
     else
-        umma::prefill_attn_umma<64><<<grid, 128, sm, st>>>(qm, km, vm, P, L.r, (__nv_bfloat16*)out,
+        umma::prefill_attn_umma<64><<<grid, umma::NTHREADS, sm, st>>>(qm, km, vm, P, L.r, (__nv_bfloat16*)out,
                                                           L.rows, L.status);
     return cudaGetLastError();
 }
