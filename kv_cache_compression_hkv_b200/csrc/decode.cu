@@ -456,6 +456,13 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
     constexpr int PB = 1 + PLAN_WARP_DESC;
     const int4* pw = L.plan_warp + (size_t)layer * PLAN_MAX_WARPS * PB;
     const int4 blk = lane < PB ? pw[(size_t)gw * PB + lane] : make_int4(0, 0, 0, 0);
+    // The same warp's plan block of the next layer (same step): once this
+    // warp's range is done, its first chunks are prefetched into L2 for the
+    // decode launch that usually follows (layer + 1), while slower warps
+    // finish.  Only a hint: a different call order merely wastes the copy.
+    const bool hint = append && layer + 1 < L.Ly;
+    const int4 nblk = hint && lane < PB ? pw[(size_t)PLAN_MAX_WARPS * PB + (size_t)gw * PB + lane]
+                                        : make_int4(0, 0, 0, 0);
     if (lane == 0) {
         for (int s = 0; s < nstage; ++s) ptx::mbar_init(&bars[s], 1);
         ptx::fence_mbar_init();
@@ -807,6 +814,17 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
     } else {
         if (early) ptx::grid_dep_wait();
         ptx::grid_dep_trigger();
+    }
+    if (hint) {
+        // L2 prefetch of the next layer's first chunks of this warp number
+        const int4 nrec = shfl_int4(nblk, 0);
+        const int nc = min(min(nrec.y - nrec.x, nstage), PLAN_WARP_DESC);
+        const size_t nrow = (size_t)(layer + 1) * L.S * L.R;
+        for (int k = 0; k < nc; ++k) {
+            const ChunkDesc c = ChunkDesc::of(shfl_int4(nblk, k + 1));
+            if (lane == 0 && c.n > 0)
+                ptx::bulk_prefetch_l2(KVp + (nrow + c.row) * 2 * D, (uint32_t)(c.n * KVR));
+        }
     }
     if (append) {
         __syncthreads();
