@@ -171,6 +171,28 @@ def test_llamagen_1layer_f32_full_config():
     assert stats[0]["n_events"] >= 1 and stats[0]["n_select"] > 0
 
 
+def test_evict_counters_match_the_events():
+    """hkv_get_evict_stats: every Global head evicts once per event, scoring
+    its whole cache (budget + M tokens) and moving at most M rows."""
+    w = WORKLOADS["llamagen_xl"].scaled(num_seqs=2, num_layers=2)
+    units = [(s, l) for s in range(2) for l in range(2)]
+    cfg = hkv.config_for(w)
+    data = generate(w, 31, DEV)
+    cache, rec, _ = run_gpu(w, cfg, data, units)
+    st = cache.evict_stats()
+    heads = tokens = 0
+    for (s, l) in units:
+        ln, bd = cache.lens(l)
+        glob = rec[(s, l)]["labels"] == 0
+        n_ev = sum(1 for t, _ in rec[(s, l)]["events"] if t >= w.prefill_len)
+        heads += n_ev * int(glob.sum())
+        tokens += n_ev * int((bd[s][glob] + w.ste_m).sum())
+    assert st["heads"] == heads and st["tokens"] == tokens, (st, heads, tokens)
+    assert 0 < st["rows_moved"] <= heads * w.ste_m
+    cache.reset()
+    assert cache.evict_stats() == {"heads": 0, "tokens": 0, "rows_moved": 0}
+
+
 @pytest.mark.parametrize("name", ["llamagen_xl", "janus_pro_1b", "janus_pro_7b_rho4",
                                   "janus_pro_7b_rho6", "janus_pro_7b_rho8", "lumina_mgpt_768"])
 def test_lockstep_scaled_stacks(name):
@@ -181,6 +203,19 @@ def test_lockstep_scaled_stacks(name):
     if w.max_len > 1000:
         units = units[:2]
     _lockstep(w, units, seed=11)
+
+
+def test_long_sequence_large_strata():
+    """A 4096-token sequence: Global caches of about 2000 tokens, so each
+    eviction selects 32 of ~1900 far keys and 32 of 128 near keys (the
+    block select's bins hold several keys per thread), in lock step."""
+    w = WORKLOADS["lumina_mgpt_768"].scaled(
+        name="long_4096", num_seqs=1, num_layers=1, num_heads=4, local_heads=2, head_dim=128,
+        prefix_len=64, image_tokens=4032, prefill_image=448, row_pitch=64, local_window=64,
+        rho=(1, 4), ste_m=64, near_dist=128, images=1)
+    assert w.max_len == 4096
+    stats = _lockstep(w, [(0, 0)], seed=41, tau=0.5)
+    assert stats[0]["n_events"] >= 2
 
 
 @pytest.mark.parametrize("name", ["llamagen_xl", "janus_pro_1b"])
