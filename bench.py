@@ -300,10 +300,17 @@ def timed_replays(g, n):
     return e0.elapsed_time(e1) / n  # ms per replay
 
 
+# workloads on which the pages compare whole-model speed and memory with
+# the full cache (LlamaGen-XL and Janus-Pro-7B at rho = 1/6): the
+# decoder-layer arm runs on these
+DECODER_LAYER_WORKLOADS = ("llamagen_xl", "janus_pro_7b_rho6")
+
+
 def gpu_arm(args, rank, world, dev, w, lite=False):
     """The timed GPU arm on workload w.  lite: the shorter run of the sweep
     (one warm-up and two timed passes, the full-cache comparator on one
-    timed pass, no end-to-end or decoder-layer arm, no clock sampling)."""
+    timed pass, no end-to-end arm, no clock sampling).  The decoder-layer
+    arm runs on DECODER_LAYER_WORKLOADS unless --no-decoder-layer."""
     import kv_cache_compression_hkv_b200 as hkv
 
     S, H, d, Ly = w.num_seqs, w.num_heads, w.head_dim, w.num_layers
@@ -435,7 +442,7 @@ def gpu_arm(args, rank, world, dev, w, lite=False):
         del g_full, cache_f
         torch.cuda.empty_cache()
 
-    if not lite and not args.no_decoder_layer:
+    if not args.no_decoder_layer and w.name in DECODER_LAYER_WORKLOADS:
         res["decoder_layer"] = decoder_layer_arm(args, w, cache, inp, outs, pre_out, dev)
 
     # end to end through the C ABI from pinned host buffers
@@ -469,6 +476,8 @@ def sweep_arm(args, dev, skip):
             "kv_pool_bytes": r["kv_pool_bytes"],
             "full_kv_pool_bytes": (r.get("full") or {}).get("kv_pool_bytes"),
             "labels_local_frac": r["labels_local_frac"]}
+        if r.get("decoder_layer"):
+            out[name]["decoder_layer"] = r["decoder_layer"]
         torch.cuda.empty_cache()
     return out
 
@@ -806,7 +815,10 @@ def main():
             "speedup_pass_vs_full": res.get("speedup_pass_vs_full"),
             "kv_pool_bytes": res["kv_pool_bytes"], "labels_local_frac": res["labels_local_frac"],
             "labels_planted": res["labels_planted"],
-            "decoder_layer": res.get("decoder_layer"),
+            # whole decoder layers, compressed vs full cache, on the shapes the
+            # pages compare end to end (the headline's own when it is one)
+            "decoder_layer": res.get("decoder_layer") or
+                {k: v["decoder_layer"] for k, v in (sweep or {}).items() if "decoder_layer" in v} or None,
             "all_configs": sweep,
         }
         print(json.dumps(line))
