@@ -420,8 +420,8 @@ def gpu_arm(args, rank, world, dev, w, lite=False):
         "labels_local_frac": float((labels == 1).mean()),
         "labels_planted": planted_recovery(w, labels, dist.rank_seed(args.seed, rank)),
         # per layer at prefill: attention, grouping, packing, plan; per
-        # step: one decode launch per layer, eviction scan and run, plan
-        "gpu_launches": args.steps * (4 * Ly + steps * (Ly + 3)),
+        # step: one decode launch per layer, the eviction, the plan
+        "gpu_launches": args.steps * (4 * Ly + steps * (Ly + 2)),
         "kv_pool_bytes": cache.nbytes,
     }
     del g_main
