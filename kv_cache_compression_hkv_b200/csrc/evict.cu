@@ -2,12 +2,12 @@
 // summary, Methodology step 3, global heads) and the standalone grouping and
 // selection primitives.
 //
-// One warp per due head (listed first by a scan): it turns the logits the decode kernel stored over
+// One block per due head: it turns the logits the decode kernel stored over
 // the last r steps into scores (summed softmax weights, each step normalised
 // by its own (max, sum) and counting only tokens already cached at that
 // step), selects the M/2 lowest (score, position) of the near and the far
-// strata with a warp bisection, and compacts the cache in place by moving
-// the surviving tail tokens into the holes below the budget.
+// strata by a block-wide threshold search, and compacts the cache in place
+// by moving the surviving tail tokens into the holes below the budget.
 #include <math.h>
 
 #include <mutex>
