@@ -282,9 +282,11 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
         const bool keep_row = qpos >= P - r && qpos < P;
         float* rrow = keep_row ? rows + ((size_t)b * r + (qpos - (P - r))) * P : nullptr;
         float m = -INFINITY, l = 0.f;
+        // every branch around the warp-wide tcgen05.ld / tcgen05.st below is
+        // taken by the whole warp: waits and decisions are warp votes
         for (int j = 0; j < nkt; ++j) {
             const int st = j & 1, k = j >> 1;
-            if (!mbar_wait(bars + B_SFULL + st, k & 1, WAIT_NS)) { fail = true; break; }
+            if (__any_sync(FULL_MASK, !mbar_wait(bars + B_SFULL + st, k & 1, WAIT_NS))) { fail = true; break; }
             fence_after();
             uint32_t sr[2][32];
             tmem_ld32(t_row + st * KT, sr[0]);
@@ -307,12 +309,18 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
                     if (key < P) rrow[key] = x[c];  // normalised in the epilogue
                 }
             }
-            if (mt > m + RESCALE) {
-                const float alpha = exp2f(m - mt);  // 0 on the first tile
+            if (__any_sync(FULL_MASK, mt > m + RESCALE)) {
+                // the warp raises its rows' references together (a row whose
+                // maximum did not grow keeps m: alpha = 1)
+                const float mn = fmaxf(m, mt);
+                const float alpha = mn == -INFINITY ? 1.f : exp2f(m - mn);  // 0 on the first tile
                 if (j > 0) {
                     // O holds P V up to tile j-1: rescale it once that is in
                     const int jp = j - 1;
-                    if (!mbar_wait(bars + B_PVDONE + (jp & 1), (jp >> 1) & 1, WAIT_NS)) { fail = true; break; }
+                    if (__any_sync(FULL_MASK, !mbar_wait(bars + B_PVDONE + (jp & 1), (jp >> 1) & 1, WAIT_NS))) {
+                        fail = true;
+                        break;
+                    }
                     fence_after();
 #pragma unroll
                     for (int c0 = 0; c0 < D; c0 += 32) {
@@ -326,10 +334,13 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
                     tmem_st_wait();
                 }
                 l *= alpha;
-                m = mt;
+                m = mn;
             }
             // stage st of P is free once P V of tile j-2 is done
-            if (j >= 2 && !mbar_wait(bars + B_PVDONE + st, (k - 1) & 1, WAIT_NS)) { fail = true; break; }
+            if (j >= 2 && __any_sync(FULL_MASK, !mbar_wait(bars + B_PVDONE + st, (k - 1) & 1, WAIT_NS))) {
+                fail = true;
+                break;
+            }
             unsigned char* pst = p_s + st * PB;
 #pragma unroll
             for (int ch = 0; ch < KT / 8; ++ch) {
@@ -352,7 +363,8 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
         }
         if (!fail && nkt > 0) {
             const int jl = nkt - 1;
-            if (!mbar_wait(bars + B_PVDONE + (jl & 1), (jl >> 1) & 1, WAIT_NS)) fail = true;
+            if (__any_sync(FULL_MASK, !mbar_wait(bars + B_PVDONE + (jl & 1), (jl >> 1) & 1, WAIT_NS)))
+                fail = true;
         }
         if (!fail) {
             fence_after();
