@@ -400,7 +400,7 @@ template <typename T, int DPL>
 __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
     decode_kernel(Layout L, int layer, const T* __restrict__ q_t, const T* __restrict__ k_t,
                   const T* __restrict__ v_t, T* __restrict__ o_t, int append, int nstage,
-                  int early, int buf, int prologue) {
+                  int early, int buf, int prologue, int l2_hint) {
     extern __shared__ __align__(128) unsigned char dsm[];
     const int n_heads = L.S * L.H;
     constexpr int D = DPL * 32;
@@ -460,7 +460,7 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
     // warp's range is done, its first chunks are prefetched into L2 for the
     // decode launch that usually follows (layer + 1), while slower warps
     // finish.  Only a hint: a different call order merely wastes the copy.
-    const bool hint = append && layer + 1 < L.Ly;
+    const bool hint = l2_hint && append && layer + 1 < L.Ly;
     const int4 nblk = hint && lane < PB ? pw[(size_t)PLAN_MAX_WARPS * PB + (size_t)gw * PB + lane]
                                         : make_int4(0, 0, 0, 0);
     if (lane == 0) {
@@ -892,12 +892,16 @@ DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
     // warp consumes chunks); a third stage only when it costs no warp.
     // Tuning overrides (read once per context): HKV_DECODE_WARPS caps the
     // warps per block, HKV_DECODE_STAGES fixes the stages per warp (2 ..
-    // MAX_STAGES), HKV_DECODE_PROLOGUE sets DecodeShape::prologue (1 or 2).
+    // MAX_STAGES), HKV_DECODE_PROLOGUE sets DecodeShape::prologue (1 or 2),
+    // HKV_DECODE_L2_HINT=0 turns the next-layer L2 prefetch off (any other
+    // value: on).
     const int es = L.dtype == HKV_DTYPE_F32 ? 4 : 2;
     const int max_w = env_int("HKV_DECODE_WARPS");
     const int fix_s = env_int("HKV_DECODE_STAGES");
     const int pro = env_int("HKV_DECODE_PROLOGUE");
-    DecodeShape best{0, 0, 0, 1, pro <= 2 ? pro : 0};
+    const char* hint_env = getenv("HKV_DECODE_L2_HINT");
+    const int hint = hint_env && hint_env[0] == '0' && hint_env[1] == 0 ? 0 : 1;
+    DecodeShape best{0, 0, 0, 1, pro <= 2 ? pro : 0, hint};
     for (int ns = 2; ns <= MAX_STAGES; ++ns) {
         if (fix_s && ns != fix_s) continue;
         // the per-warp tail regions are laid out for MAX_STAGES barriers
@@ -906,7 +910,7 @@ DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
         if (w > DECODE_MAX_WARPS) w = DECODE_MAX_WARPS;
         if (max_w && w > max_w) w = max_w;
         if (w >= 1 && w >= best.warps)
-            best = DecodeShape{w, ns, 1024 + (size_t)w * per, 1, best.prologue};
+            best = DecodeShape{w, ns, 1024 + (size_t)w * per, 1, best.prologue, hint};
     }
     return best;
 }
@@ -926,7 +930,8 @@ static cudaError_t launch_decode_t(const Layout& L, int layer, const void* q, co
     cfg.attrs = at;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, decode_kernel<T, DPL>, L, layer, (const T*)q, (const T*)k,
-                              (const T*)v, (T*)o, append, sh.nstage, early, buf, sh.prologue);
+                              (const T*)v, (T*)o, append, sh.nstage, early, buf, sh.prologue,
+                              sh.l2_hint);
 }
 
 cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void* k, const void* v,

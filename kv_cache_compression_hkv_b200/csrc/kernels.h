@@ -38,6 +38,7 @@ struct DecodeShape {
     int prologue;  // stages a warp fills before its first chunk lands:
                    // 0 one when the block has 8 or more warps, else all;
                    // 1 one; 2 all
+    int l2_hint;   // 1: finished warps prefetch the next layer's first chunks into L2
 };
 DecodeShape decode_shape(const Layout& L, size_t smem_limit);
 // early: the previous launch in `st` is a decode launch of another layer (the
