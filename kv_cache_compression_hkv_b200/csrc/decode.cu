@@ -194,12 +194,13 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead,
         for (int i = tid; i < n; i += blockDim.x) {
             const size_t hx = hbase + i;
             const int cap = L.cap[hx];
-            int bl = L.base_len[hx], bt = L.base_t[hx];
+            const uint64_t b = L.base[hx];
+            int bl = base_len_of(b), bt = base_t_of(b);
             if (L.label[hx] != 0 || L.mode == HKV_MODE_FULL) continue;
             if (bl + (te - bt) >= cap) {
                 bl = L.budget[hx];
                 bt = te;
-                if (part == 0) { L.base_len[hx] = bl; L.base_t[hx] = bt; }
+                if (part == 0) L.base[hx] = base_pack(bl, bt);
             }
             const int s = i / L.H;
             const uint32_t gm = L.unit_gmask[(size_t)layer * L.S + s];
@@ -214,8 +215,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead,
         const int cap = L.cap[hx];
         int len;
         {
-            int bl = L.base_len[hx], bt = L.base_t[hx];
-            // part 0 may already have written the committed values: either
+            const uint64_t b = L.base[hx];
+            int bl = base_len_of(b), bt = base_t_of(b);
+            // part 0 may already have written the committed pair: either
             // reading gives the same length
             if (commit && L.label[hx] == 0 && L.mode != HKV_MODE_FULL && bl + (te - bt) >= cap) {
                 bl = L.budget[hx];
@@ -891,7 +893,7 @@ DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
     // (one chunk in flight per warp covers the HBM latency at the rate a
     // warp consumes chunks); a third stage only when it costs no warp.
     // Tuning overrides (read once per context): HKV_DECODE_WARPS caps the
-    // warps per block, HKV_DECODE_STAGES fixes the stages per warp (2 ..
+    // warps per block, HKV_DECODE_STAGES fixes the stages per warp (1 ..
     // MAX_STAGES), HKV_DECODE_PROLOGUE sets DecodeShape::prologue (1 or 2),
     // HKV_DECODE_L2_HINT=0 turns the next-layer L2 prefetch off (any other
     // value: on).
@@ -902,7 +904,7 @@ DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
     const char* hint_env = getenv("HKV_DECODE_L2_HINT");
     const int hint = hint_env && hint_env[0] == '0' && hint_env[1] == 0 ? 0 : 1;
     DecodeShape best{0, 0, 0, 1, pro <= 2 ? pro : 0, hint};
-    for (int ns = 2; ns <= MAX_STAGES; ++ns) {
+    for (int ns = fix_s == 1 ? 1 : 2; ns <= MAX_STAGES; ++ns) {
         if (fix_s && ns != fix_s) continue;
         // the per-warp tail regions are laid out for MAX_STAGES barriers
         const size_t per = decode_warp_bytes(L.d, es, ns) + (MAX_STAGES - ns) * 8;

@@ -135,8 +135,7 @@ size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Lay
     l.off = (int32_t*)take(nh * 4);
     l.cap = (int32_t*)take(nh * 4);
     l.budget = (int32_t*)take(nh * 4);
-    l.base_len = (int32_t*)take(nh * 4);
-    l.base_t = (int32_t*)take(nh * 4);
+    l.base = (uint64_t*)take(nh * 8);
     l.n_tau = (int32_t*)take(nh * 4);
     l.label = (uint8_t*)take(nh);
     l.K = take(slots * 2 * d * es);  // K and V rows interleaved per slot
@@ -420,10 +419,10 @@ hkv_status hkv_get_lens(hkv_ctx* c, int32_t layer, int32_t* len_host, int32_t* b
     if (!c || !len_host || layer < 0 || layer >= c->cfg.num_layers) return HKV_ERR_INVALID_ARG;
     if (!c->classified[layer]) return HKV_ERR_STATE;
     const size_t nh = (size_t)c->cfg.num_seqs * c->cfg.num_heads;
-    std::vector<int32_t> bl(nh), bt(nh), cap(nh), tn(1);
+    std::vector<uint64_t> base(nh);
+    std::vector<int32_t> cap(nh), tn(1);
     std::vector<uint8_t> lab(nh);
-    hkv_status s = copy_back(bl.data(), c->lay.base_len + layer * nh, nh * 4, stream);
-    if (s == HKV_OK) s = copy_back(bt.data(), c->lay.base_t + layer * nh, nh * 4, stream);
+    hkv_status s = copy_back(base.data(), c->lay.base + layer * nh, nh * 8, stream);
     if (s == HKV_OK) s = copy_back(cap.data(), c->lay.cap + layer * nh, nh * 4, stream);
     if (s == HKV_OK) s = copy_back(lab.data(), c->lay.label + layer * nh, nh, stream);
     if (s == HKV_OK) s = copy_back(tn.data(), c->lay.t_next + layer, 4, stream);
@@ -431,7 +430,7 @@ hkv_status hkv_get_lens(hkv_ctx* c, int32_t layer, int32_t* len_host, int32_t* b
     if (s != HKV_OK) return s;
     const int t = tn[0] - 1;  // newest cached position
     for (size_t i = 0; i < nh; ++i) {
-        int n = bl[i] + (t - bt[i]);
+        int n = hkv::base_len_of(base[i]) + (t - hkv::base_t_of(base[i]));
         if (lab[i] == 1 && n > cap[i]) n = cap[i];
         len_host[i] = n;
     }

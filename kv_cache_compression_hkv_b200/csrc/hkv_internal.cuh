@@ -38,8 +38,10 @@ struct Layout {
     int32_t* off;       // first slot of the head inside its region
     int32_t* cap;       // slots reserved for the head
     int32_t* budget;    // tokens kept after an eviction (W for Local heads)
-    int32_t* base_len;  // cache length at step base_t
-    int32_t* base_t;    // the length grows by one per step after base_t
+    uint64_t* base;     // cache length at step t0 (low 32 bits) and t0 (high
+                        // 32 bits): the length grows by one per step after t0;
+                        // one 64-bit word, so a reader never sees half of an
+                        // update (see base_pack / base_len_of / base_t_of)
     uint8_t* label;     // 1 Local, 0 Global, 2 full cache
     int32_t* n_tau;
     // per (layer, sequence): step at which its Global heads reach their cap
@@ -68,6 +70,12 @@ struct Layout {
     int32_t max_chunks;
 };
 
+__host__ __device__ __forceinline__ uint64_t base_pack(int len, int t0) {
+    return (uint64_t)(uint32_t)len | ((uint64_t)(uint32_t)t0 << 32);
+}
+__host__ __device__ __forceinline__ int base_len_of(uint64_t b) { return (int)(uint32_t)b; }
+__host__ __device__ __forceinline__ int base_t_of(uint64_t b) { return (int)(uint32_t)(b >> 32); }
+
 __device__ __forceinline__ size_t head_index(const Layout& L, int l, int s, int h) {
     return ((size_t)l * L.S + s) * L.H + h;
 }
@@ -75,10 +83,11 @@ __device__ __forceinline__ size_t region_slot0(const Layout& L, int l, int s) {
     return ((size_t)l * L.S + s) * (size_t)L.R;
 }
 
-// Cache length of a head at step t: one token joins per step after base_t;
+// Cache length of a head at step t: one token joins per step after its t0;
 // a Local head's ring stops growing at its capacity W.
 __device__ __forceinline__ int len_at(const Layout& L, size_t hi, int t) {
-    int n = L.base_len[hi] + (t - L.base_t[hi]);
+    const uint64_t b = L.base[hi];
+    int n = base_len_of(b) + (t - base_t_of(b));
     if (L.label[hi] == 1 && n > L.cap[hi]) n = L.cap[hi];
     return n;
 }

@@ -115,8 +115,7 @@ __device__ void lay_out_heads(const Layout& L, int layer, int s, int P, const ui
         L.off[hi] = o;
         L.cap[hi] = cap;
         L.budget[hi] = budget;
-        L.base_len[hi] = len0;
-        L.base_t[hi] = P - 1;
+        L.base[hi] = base_pack(len0, P - 1);
         L.label[hi] = lab[j];
         L.n_tau[hi] = ntau[j];
         o += cap;
