@@ -203,9 +203,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead,
                 if (part == 0) L.base[hx] = base_pack(bl, bt);
             }
             const int s = i / L.H;
-            const uint32_t gm = L.unit_gmask[(size_t)layer * L.S + s];
-            if (part == 0 && gm && (i % L.H) == __ffs(gm) - 1)
-                L.unit_due[(size_t)layer * L.S + s] = bt + (cap - bl);
+            int4* ur = L.unit + (size_t)layer * L.S + s;
+            const uint32_t gm = (uint32_t)ur->y;
+            if (part == 0 && gm && (i % L.H) == __ffs(gm) - 1) ur->x = bt + (cap - bl);
         }
         __syncthreads();
     }

@@ -109,14 +109,15 @@ __device__ __forceinline__ int bin_shift(uint32_t lo, uint32_t hi) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(EVB_THREADS, 3) evict_block_kernel(Layout L, int l0, int l1, int n_max) {
+__global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, int l0, int l1, int n_max) {
     extern __shared__ __align__(16) unsigned char ebs[];
     __shared__ float2 ml_s[32];
     __shared__ int step_s[32];
     __shared__ int red[2][EVB_WARPS][32];
     __shared__ int lists[2][EVB_WARPS];
-    __shared__ int due_items[EVB_THREADS];
+    __shared__ int4 due_items[EVB_THREADS];  // {head, due step, budget, Global mask}
     __shared__ int n_due;
+    __shared__ bool head_ok;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int BT = blockDim.x, NW = BT >> 5;
     const int r = L.r, M = L.M;
@@ -133,18 +134,20 @@ __global__ void __launch_bounds__(EVB_THREADS, 3) evict_block_kernel(Layout L, i
     const int64_t G = gridDim.x;
 
     for (int64_t k0 = 0; (int64_t)blockIdx.x + k0 * G < items; k0 += BT) {
-        // this block's next BT items: the due ones, in item order
+        // this block's next BT items: the due ones, in item order, each with
+        // its unit's step, budget and Global mask (no per-head metadata)
         {
             const int64_t i = (int64_t)blockIdx.x + (k0 + tid) * G;
             bool due = false;
-            int hxi = 0;
+            int4 item = make_int4(0, 0, 0, 0);
             if (i < items) {
                 const int64_t u = i / L.H;  // unit within the range
                 const int h = (int)(i % L.H);
                 const int l = l0 + (int)(u / L.S), s = (int)(u % L.S);
                 const size_t uu = (size_t)l * L.S + s;
-                due = L.unit_due[uu] == L.t_next[l] - 1 && ((L.unit_gmask[uu] >> h) & 1u);
-                hxi = (int)(uu * L.H + h);
+                const int4 rec = L.unit[uu];
+                due = rec.x == L.t_next[l] - 1 && (((uint32_t)rec.y >> h) & 1u);
+                item = make_int4((int)(uu * L.H + h), rec.x, rec.z, rec.y);
             }
             const unsigned b = __ballot_sync(FULL_MASK, due);
             __syncthreads();  // the previous round's list is no longer read
@@ -155,62 +158,84 @@ __global__ void __launch_bounds__(EVB_THREADS, 3) evict_block_kernel(Layout L, i
                 if (w < warp) o += lists[0][w];
                 tot += lists[0][w];
             }
-            if (due) due_items[o] = hxi;
+            if (due) due_items[o] = item;
             if (tid == 0) n_due = tot;
             __syncthreads();
         }
         const int nd = n_due;
         for (int e = 0; e < nd; ++e) {
-            const size_t hx = (size_t)due_items[e];
+            const int4 item = due_items[e];
+            const size_t hx = (size_t)item.x;
             const int l = (int)(hx / n_heads);
             const int s = (int)(hx % n_heads) / L.H;
-            const int t = L.t_next[l] - 1;
-            const int n = len_at(L, hx, t);
-            const int target = L.budget[hx];
+            const int h = (int)(hx % L.H);
+            const int t = item.y;                 // the due step: the newest position
+            const int target = item.z;            // the budget
+            const int n = target + M;             // the capacity, reached at the due step
+            const uint32_t gm = (uint32_t)item.w, below = (1u << h) - 1u;
+            // first slot: Local heads before h hold W slots, Global ones n
+            const size_t slot0 = region_slot0(L, l, s) + (size_t)__popc(~gm & below) * L.W +
+                                 (size_t)__popc(gm & below) * n;
             __syncthreads();  // the previous head's lists and keys are no longer read
-            if (n > n_max || n != L.cap[hx] || n - target > M || n - target < 0) {
+            if (n > n_max) {
                 if (tid == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
                 continue;
             }
-            const size_t slot0 = region_slot0(L, l, s) + L.off[hx];
-            const int top = n - target;
-            if (tid == 0 && top > 0) ptx::bulk_prefetch_l2(KVb + (slot0 + target) * pair, (uint32_t)(top * pair));
+            // every load of the head at once: thread 0 the L2 prefetch of the
+            // rows a survivor may move from (slots budget .. n-1) and the
+            // head's length record (checked below), threads < r the (max, sum)
+            // of the scoring steps, every thread the positions and logits of
+            // its first two tokens
+            if (tid == 0) {
+                ptx::bulk_prefetch_l2(KVb + (slot0 + target) * pair, (uint32_t)(M * pair));
+                head_ok = len_at(L, hx, t) == n;
+            }
             if (tid < r) {
                 const float2 ml = L.ml[hx * r + tid];
                 ml_s[tid] = make_float2(ml.x, 1.0f / ml.y);
                 step_s[tid] = t - (((t - tid) % r) + r) % r;  // the step column tid holds
             }
-            __syncthreads();
-
-            // scores and stratum counts; keys into shared memory
-            bool bad = false;
-            int nn = 0, nf = 0;
-            uint32_t alo = 0xffffffffu, ahi = 0u, blo = 0xffffffffu, bhi = 0u;
             const bool strat = L.stratified != 0;
-            for (int b0 = 0; b0 < n; b0 += 2 * BT) {
-                int pv[2];
-                float4 la[2], lb[2];
-    #pragma unroll
+            // two tokens of this thread: position and r = 8 logits each
+            struct Two {
+                int p[2];
+                float4 a[2], b[2];
+            };
+            auto load2 = [&](int b0, Two& x) {
+#pragma unroll
                 for (int u = 0; u < 2; ++u) {
                     const int q = b0 + u * BT + tid;
                     if (q < n) {
-                        pv[u] = L.pos[slot0 + q];
+                        x.p[u] = L.pos[slot0 + q];
                         if (r == 8) {
                             const float4* p4 = reinterpret_cast<const float4*>(L.logit + (slot0 + q) * 8);
-                            la[u] = p4[0];
-                            lb[u] = p4[1];
+                            x.a[u] = p4[0];
+                            x.b[u] = p4[1];
                         }
                     }
                 }
-    #pragma unroll
+            };
+            Two cur, nxt;
+            load2(0, cur);
+            __syncthreads();  // ml_s, step_s
+
+            // scores and stratum counts; keys into shared memory; the next
+            // two tokens' loads go out before this pair is used
+            bool bad = false;
+            int nn = 0, nf = 0;
+            uint32_t alo = 0xffffffffu, ahi = 0u, blo = 0xffffffffu, bhi = 0u;
+            for (int b0 = 0; b0 < n; b0 += 2 * BT) {
+                if (b0 + 2 * BT < n) load2(b0 + 2 * BT, nxt);
+#pragma unroll
                 for (int u = 0; u < 2; ++u) {
                     const int q = b0 + u * BT + tid;
                     if (q >= n) continue;
-                    const int p = pv[u];
+                    const int p = cur.p[u];
                     float acc = 0.f;
                     if (r == 8) {
-                        const float v[8] = {la[u].x, la[u].y, la[u].z, la[u].w, lb[u].x, lb[u].y, lb[u].z, lb[u].w};
-    #pragma unroll
+                        const float v[8] = {cur.a[u].x, cur.a[u].y, cur.a[u].z, cur.a[u].w,
+                                            cur.b[u].x, cur.b[u].y, cur.b[u].z, cur.b[u].w};
+#pragma unroll
                         for (int c = 0; c < 8; ++c)
                             if (p <= step_s[c]) acc += exp2f(v[c] - ml_s[c].x) * ml_s[c].y;
                     } else {
@@ -227,8 +252,13 @@ __global__ void __launch_bounds__(EVB_THREADS, 3) evict_block_kernel(Layout L, i
                         else { ++nf; blo = min(blo, sb); bhi = max(bhi, sb); }
                     }
                 }
+                cur = nxt;
             }
             if (__syncthreads_or(bad) && tid == 0) latch_error(L, HKV_ERR_NUMERIC, (int)hx);
+            if (!head_ok) {  // the head's length disagrees with its unit's record
+                if (tid == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
+                continue;
+            }
             // block totals: counts and score-bit ranges of both strata
             {
                 nn = __reduce_add_sync(FULL_MASK, nn);
@@ -519,7 +549,7 @@ static size_t evict_block_smem(int n_max, int M) { return (size_t)n_max * 8 + (s
 
 int evict_blocks_per_sm(const Layout& L, int optin) {
     const size_t sm = evict_block_smem(L.L, L.M) + 5120;  // + static
-    int by_threads = 3;  // registers: see the kernel's launch bounds
+    int by_threads = 2;  // registers: see the kernel's launch bounds
     int by_smem = (int)((size_t)optin * 1 / sm);
     int b = by_threads < by_smem ? by_threads : by_smem;
     return b < 1 ? 1 : b;

@@ -145,8 +145,7 @@ size_t carve(const hkv_config* c, int64_t T, int32_t R, unsigned char* base, Lay
     l.ml = (float2*)take(nh * r * 8);
     l.rows = (float*)take(S * H * r * Lmax * 4);
     l.partial = (float*)take(2 * 2 * (size_t)hkv::PLAN_MAX_WARPS * (d + 2) * 4);
-    l.unit_due = (int32_t*)take(Ly * S * 4);
-    l.unit_gmask = (uint32_t*)take(Ly * S * 4);
+    l.unit = (int4*)take(Ly * S * 16);
     l.plan_desc = (int4*)take(Ly * max_chunks * 16);
     l.plan_warp = (int4*)take(Ly * hkv::PLAN_MAX_WARPS * (1 + hkv::PLAN_WARP_DESC) * 16);
     l.S = c->num_seqs; l.Ly = c->num_layers; l.H = c->num_heads; l.d = c->head_dim;

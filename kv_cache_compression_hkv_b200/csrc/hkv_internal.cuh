@@ -55,11 +55,13 @@ struct Layout {
     float* rows;        // [S*H][r][prefill_len] weights of the last r prefill queries
     float* partial;     // [2][PLAN_MAX_WARPS][2][d + 2] split-K partial states
     int32_t* ticket;    // [2][S*H] arrivals per head of the running decode launch
-    // per (layer, sequence) "unit", index l*S + s: the step at which its
-    // Global heads reach their capacity (INT32_MAX: none), kept by the plan
-    // kernel; the Global heads held here as a bit mask (H <= 32)
-    int32_t* unit_due;
-    uint32_t* unit_gmask;
+    // per (layer, sequence) "unit", index l*S + s: {x: the step at which its
+    // Global heads reach their capacity (INT32_MAX: none; advanced by the
+    // plan kernel after each eviction), y: the Global heads held here as a
+    // bit mask (H <= 32), z: their budget, w: their capacity}.  The Global
+    // heads of a unit share budget, capacity and length, and a head's first
+    // slot follows from the mask (Local heads hold W slots, Global ones w).
+    int4* unit;
     // decode plan per layer, for the step it was made for (see plan_kernel)
     int4* plan_desc;     // [Ly][max_chunks] one descriptor per chunk
     // [Ly][PLAN_MAX_WARPS][1 + PLAN_WARP_DESC]: per warp {first chunk, end

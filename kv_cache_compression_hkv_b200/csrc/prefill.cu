@@ -123,9 +123,8 @@ __device__ void lay_out_heads(const Layout& L, int layer, int s, int P, const ui
     if (o > L.R) latch_error(L, HKV_ERR_CAPACITY, layer * L.S + s);
     // the Global heads of a unit share capacity and length: one due step
     const size_t u = (size_t)layer * L.S + s;
-    L.unit_gmask[u] = gmask;
     const int len0_g = P < bg ? P : bg;
-    L.unit_due[u] = gmask ? (P - 1) + (bg + L.M - len0_g) : INT32_MAX;
+    L.unit[u] = make_int4(gmask ? (P - 1) + (bg + L.M - len0_g) : INT32_MAX, (int)gmask, bg, bg + L.M);
     if (s == 0) L.t_next[layer] = P;
 }
 
