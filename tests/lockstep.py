@@ -8,11 +8,13 @@ unit through the oracle with those decisions as hints: the oracle adopts a
 GPU decision only where its own differs by a near-tie inside the stated band,
 and counts every other difference as a hard mismatch.
 
-Bands: fp32 logits carry an absolute error of at
-most ~1e-4 on these inputs (sequential fp32 dot products of length <= 128),
-so softmax weights carry a relative error <= ~1e-4; labels compare
-sum-of-weights with tau (band 1e-3 absolute) and selections compare two
-scores (band 1e-3 relative).
+Bands: labels compare a sum of weights with tau (band absolute), selections
+compare two scores (band relative).  The GPU computes the weights in fp32
+from the same bf16/fp32 inputs as the fp64 oracle; typical relative errors
+are ~1e-6.  With bands of 1e-3, 75 lock-step units of the GPU suite (1676
+labels, 15196 selections) adopted no GPU decision at all; the bands are
+1e-5, and assert_lockstep bounds the adoptions to 1% of the decisions of a
+unit (one allowed in any unit).
 """
 from __future__ import annotations
 
@@ -25,8 +27,8 @@ import kv_cache_compression_hkv_b200 as hkv
 from kv_cache_compression_hkv_b200.inputs import generate_layer
 from oracle import hkv_oracle as O
 
-LABEL_BAND = 1e-3
-SELECT_BAND = 1e-3
+LABEL_BAND = 1e-5
+SELECT_BAND = 1e-5
 
 
 def oracle_params(w, mode=O.MODE_HEADKV, stratified=True, cls_queries=1,
@@ -212,6 +214,8 @@ def assert_lockstep(res, err, tol, n_events_gpu, unit=None):
     st = res.stats
     print("lockstep", json.dumps(tie_report(res, err, unit)))
     assert st["n_label_hard"] == 0, st
+    assert st["n_label_ties"] <= max(1, len(res.labels) // 100), st
+    assert st["n_select_ties"] <= max(1, st["n_select"] // 100), st
     assert st["n_select_hard"] == 0, st
     assert st["n_events"] == n_events_gpu, (st, n_events_gpu)
     assert err.max() <= tol, f"max relative output error {err.max():.3e} > {tol}"

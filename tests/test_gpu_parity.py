@@ -407,10 +407,10 @@ def test_prefill_shapes_against_oracle(d, P):
             got = out[s, h].double().cpu().numpy()
             assert np.abs(got - o).max() / np.abs(o).max() < 2e-2, (s, h)
             e_nt, e_lab, cw = O.classify(p[-1], w.local_window, 0.9)
-            if abs(cw - 0.9) > 1e-3:
+            if abs(cw - 0.9) > 1e-5:
                 assert lab[s, h] == e_lab, (s, h, cw)
-            if e_nt > 1 and abs(np.cumsum(p[-1][::-1])[e_nt - 2] - 0.9) > 1e-3 and \
-                    abs(np.cumsum(p[-1][::-1])[e_nt - 1] - 0.9) > 1e-3:
+            if e_nt > 1 and abs(np.cumsum(p[-1][::-1])[e_nt - 2] - 0.9) > 1e-5 and \
+                    abs(np.cumsum(p[-1][::-1])[e_nt - 1] - 0.9) > 1e-5:
                 assert ntau[s, h] == e_nt, (s, h)
 
 

@@ -65,7 +65,7 @@ def test_noalloc_matches_context_path_two_calls(name):
 def _check_against_oracle(w, q, k, v, out, n_tau, label, tol):
     """Every block against the oracle's causal attention and grouping of
     the last query's weights on the same bits: outputs within tol, labels
-    equal unless the sum of the W-1 newest weights lies within 1e-3 of tau,
+    equal unless the sum of the W-1 newest weights lies within 1e-5 of tau,
     n_tau equal unless a running sum next to the boundary does."""
     P, W = w.prefill_len, w.local_window
     S, H = q.shape[0], q.shape[1]
@@ -78,10 +78,10 @@ def _check_against_oracle(w, q, k, v, out, n_tau, label, tol):
             err = np.abs(got_out[s, h] - o).max() / np.abs(o).max()
             assert err <= tol, (s, h, err)
             e_nt, e_lab, cw = O.classify(p[-1], W, 0.9)
-            if abs(cw - 0.9) > 1e-3:
+            if abs(cw - 0.9) > 1e-5:
                 assert lab[s, h] == e_lab, (s, h, cw)
             c = np.cumsum(p[-1][::-1])
-            near = [abs(c[i] - 0.9) <= 1e-3 for i in (e_nt - 2, e_nt - 1) if 0 <= i < P]
+            near = [abs(c[i] - 0.9) <= 1e-5 for i in (e_nt - 2, e_nt - 1) if 0 <= i < P]
             if not any(near):
                 assert nt[s, h] == e_nt, (s, h)
 
