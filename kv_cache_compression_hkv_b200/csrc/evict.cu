@@ -46,17 +46,21 @@ namespace hkv {
 // ---------------------------------------------------------------------------
 constexpr int EVB_THREADS = 256;  // threads of an eviction block
 constexpr int EVB_WARPS = EVB_THREADS / 32;
+__host__ __device__ inline size_t evict_group_smem(int n_max, int M);
 
 // One round of the threshold search of both strata: every thread adds its
 // candidate keys with score bits in [lo, hi] of their stratum to 16 bins of
 // width 2^sh above lo (16-bit counters packed two to a word: a warp holds
-// far fewer than 65536 keys) and counts those below lo; the block's totals
-// are reduced through `red` (this round's buffer; rounds alternate between
-// two, so one barrier per round suffices).  Lane i of every warp returns the
-// number of keys at or below the top of bin i (i < 16: near stratum, else
-// bin i - 16 of the far stratum).
-__device__ __forceinline__ int block_bin_counts(const uint32_t (&ha)[8], const uint32_t (&hb)[8],
-                                                int below_a, int below_b, int (*red)[32], int NW) {
+// far fewer than 65536 keys) and counts those below lo; the totals of the
+// head's group of warps (w0 .. w0 + nw - 1) are reduced through `red` (this
+// round's buffer; rounds alternate between two, so one group barrier per
+// round suffices).  Lane i of every warp returns the number of keys at or
+// below the top of bin i (i < 16: near stratum, else bin i - 16 of the far
+// stratum).
+template <typename Sync>
+__device__ __forceinline__ int group_bin_counts(const uint32_t (&ha)[8], const uint32_t (&hb)[8],
+                                                int below_a, int below_b, int (*red)[32], int w0,
+                                                int nw, Sync gsync) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t w[16];
 #pragma unroll
@@ -72,11 +76,11 @@ __device__ __forceinline__ int block_bin_counts(const uint32_t (&ha)[8], const u
         red[warp][16] = below_a;
         red[warp][17] = below_b;
     }
-    __syncthreads();
-    // lane i: bin i & 15 of stratum i >> 4, summed over the warps
+    gsync();
+    // lane i: bin i & 15 of stratum i >> 4, summed over the group's warps
     int tot = 0, below = 0;
     const int word = lane >> 1, sh = 16 * (lane & 1);
-    for (int v = 0; v < NW; ++v) {
+    for (int v = w0; v < w0 + nw; ++v) {
         tot += ((uint32_t)red[v][word] >> sh) & 0xffffu;
         below += red[v][16 + (lane >> 4)];
     }
@@ -109,22 +113,44 @@ __device__ __forceinline__ int bin_shift(uint32_t lo, uint32_t hi) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, int l0, int l1, int n_max) {
+__global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, int l0, int l1, int n_max,
+                                                                    int GW) {
     extern __shared__ __align__(16) unsigned char ebs[];
-    __shared__ float2 ml_s[32];
-    __shared__ int step_s[32];
+    __shared__ float2 ml_all[EVB_WARPS][32];
+    __shared__ int step_all[EVB_WARPS][32];
     __shared__ int red[2][EVB_WARPS][32];
     __shared__ int lists[2][EVB_WARPS];
     __shared__ int4 due_items[EVB_THREADS];  // {head, due step, budget, Global mask}
     __shared__ int n_due;
-    __shared__ bool head_ok;
+    __shared__ int flag_all[EVB_WARPS];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int BT = blockDim.x, NW = BT >> 5;
+    // the block's warps work in groups of GW, one due head per group
+    const int GT = 32 * GW, ngroups = NW / GW, grp = warp / GW, gw0 = grp * GW, gtid = tid % GT;
     const int r = L.r, M = L.M;
-    uint64_t* keys = reinterpret_cast<uint64_t*>(ebs);            // [n_max]
+    unsigned char* gbase = ebs + (size_t)grp * evict_group_smem(n_max, M);
+    uint64_t* keys = reinterpret_cast<uint64_t*>(gbase);          // [n_max]
     int32_t* holes = reinterpret_cast<int32_t*>(keys + n_max);    // [M]
     int32_t* movers = holes + M;                                  // [M]
     int32_t* mpos = movers + M;                                   // [M]
+    float2* ml_s = ml_all[grp];
+    int* step_s = step_all[grp];
+    // barrier of the head's group (one warp: the warp itself)
+    auto gsync = [&]() {
+        if (GW == 1) __syncwarp();
+        else asm volatile("bar.sync %0, %1;" ::"r"(grp + 1), "r"(GT) : "memory");
+    };
+    // OR of a flag over the group
+    auto gany = [&](bool x) -> bool {
+        const bool wx = __any_sync(FULL_MASK, x);
+        if (GW == 1) return wx;
+        if (lane == 0) flag_all[warp] = wx;
+        gsync();
+        bool any = false;
+        for (int w = gw0; w < gw0 + GW; ++w) any |= flag_all[w] != 0;
+        gsync();  // the flags are read before they are written again
+        return any;
+    };
     const int n_heads = L.S * L.H;
     const int pair = 2 * L.d * (int)sizeof(T);                    // bytes of a K|V row pair
     const int per_pair = pair / 16;
@@ -163,7 +189,7 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
             __syncthreads();
         }
         const int nd = n_due;
-        for (int e = 0; e < nd; ++e) {
+        for (int e = grp; e < nd; e += ngroups) {
             const int4 item = due_items[e];
             const size_t hx = (size_t)item.x;
             const int l = (int)(hx / n_heads);
@@ -176,9 +202,9 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
             // first slot: Local heads before h hold W slots, Global ones n
             const size_t slot0 = region_slot0(L, l, s) + (size_t)__popc(~gm & below) * L.W +
                                  (size_t)__popc(gm & below) * n;
-            __syncthreads();  // the previous head's lists and keys are no longer read
+            gsync();  // the previous head's lists and keys are no longer read
             if (n > n_max) {
-                if (tid == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
+                if (gtid == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
                 continue;
             }
             // every load of the head at once: thread 0 the L2 prefetch of the
@@ -186,14 +212,15 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
             // head's length record (checked below), threads < r the (max, sum)
             // of the scoring steps, every thread the positions and logits of
             // its first two tokens
-            if (tid == 0) {
+            bool head_bad = false;
+            if (gtid == 0) {
                 ptx::bulk_prefetch_l2(KVb + (slot0 + target) * pair, (uint32_t)(M * pair));
-                head_ok = len_at(L, hx, t) == n;
+                head_bad = len_at(L, hx, t) != n;
             }
-            if (tid < r) {
-                const float2 ml = L.ml[hx * r + tid];
-                ml_s[tid] = make_float2(ml.x, 1.0f / ml.y);
-                step_s[tid] = t - (((t - tid) % r) + r) % r;  // the step column tid holds
+            if (gtid < r) {
+                const float2 ml = L.ml[hx * r + gtid];
+                ml_s[gtid] = make_float2(ml.x, 1.0f / ml.y);
+                step_s[gtid] = t - (((t - gtid) % r) + r) % r;  // the step column gtid holds
             }
             const bool strat = L.stratified != 0;
             // two tokens of this thread: position and r = 8 logits each
@@ -204,7 +231,7 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
             auto load2 = [&](int b0, Two& x) {
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
-                    const int q = b0 + u * BT + tid;
+                    const int q = b0 + u * GT + gtid;
                     if (q < n) {
                         x.p[u] = L.pos[slot0 + q];
                         if (r == 8) {
@@ -217,18 +244,18 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
             };
             Two cur, nxt;
             load2(0, cur);
-            __syncthreads();  // ml_s, step_s
+            gsync();  // ml_s, step_s
 
             // scores and stratum counts; keys into shared memory; the next
             // two tokens' loads go out before this pair is used
             bool bad = false;
             int nn = 0, nf = 0;
             uint32_t alo = 0xffffffffu, ahi = 0u, blo = 0xffffffffu, bhi = 0u;
-            for (int b0 = 0; b0 < n; b0 += 2 * BT) {
-                if (b0 + 2 * BT < n) load2(b0 + 2 * BT, nxt);
+            for (int b0 = 0; b0 < n; b0 += 2 * GT) {
+                if (b0 + 2 * GT < n) load2(b0 + 2 * GT, nxt);
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
-                    const int q = b0 + u * BT + tid;
+                    const int q = b0 + u * GT + gtid;
                     if (q >= n) continue;
                     const int p = cur.p[u];
                     float acc = 0.f;
@@ -254,9 +281,9 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
                 }
                 cur = nxt;
             }
-            if (__syncthreads_or(bad) && tid == 0) latch_error(L, HKV_ERR_NUMERIC, (int)hx);
-            if (!head_ok) {  // the head's length disagrees with its unit's record
-                if (tid == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
+            if (gany(bad) && gtid == 0) latch_error(L, HKV_ERR_NUMERIC, (int)hx);
+            if (gany(head_bad)) {  // the head's length disagrees with its unit's record
+                if (gtid == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
                 continue;
             }
             // block totals: counts and score-bit ranges of both strata
@@ -273,11 +300,11 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
                     rb[warp][2] = (int)alo; rb[warp][3] = (int)ahi;
                     rb[warp][4] = (int)blo; rb[warp][5] = (int)bhi;
                 }
-                __syncthreads();
+                gsync();
                 nn = nf = 0;
                 alo = blo = 0xffffffffu;
                 ahi = bhi = 0u;
-                for (int w = 0; w < NW; ++w) {
+                for (int w = gw0; w < gw0 + GW; ++w) {
                     nn += rb[w][0]; nf += rb[w][1];
                     alo = min(alo, (uint32_t)rb[w][2]); ahi = max(ahi, (uint32_t)rb[w][3]);
                     blo = min(blo, (uint32_t)rb[w][4]); bhi = max(bhi, (uint32_t)rb[w][5]);
@@ -304,7 +331,7 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
                 const int sa = bin_shift(alo, ahi), sbh = bin_shift(blo, bhi);
                 uint32_t ha[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u}, hb[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
                 int below_a = 0, below_b = 0;
-                for (int q = tid; q < n; q += BT) {
+                for (int q = gtid; q < n; q += GT) {
                     const uint64_t key = keys[q];
                     const uint32_t sb = (uint32_t)(key >> 32);
                     const int delta = t - (int32_t)(uint32_t)key;
@@ -312,7 +339,7 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
                     if (strat && delta <= L.D) bin_add(ha, below_a, sb, alo, ahi, sa);
                     else bin_add(hb, below_b, sb, blo, bhi, sbh);
                 }
-                const int cum = block_bin_counts(ha, hb, below_a, below_b, red[par], NW);
+                const int cum = group_bin_counts(ha, hb, below_a, below_b, red[par], gw0, GW, gsync);
                 par ^= 1;
                 // first bin whose cumulative count reaches the share
                 const unsigned ma = __ballot_sync(FULL_MASK, lane < 16 && cum >= ka);
@@ -340,7 +367,7 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
             if (a_part || b_part) {
                 int c[4] = {0, 0, 0, 0};  // below s* and at s*, near then far
                 uint32_t plo_a = 0xffffffffu, phi_a = 0u, plo_b = 0xffffffffu, phi_b = 0u;
-                for (int q = tid; q < n; q += BT) {
+                for (int q = gtid; q < n; q += GT) {
                     const uint64_t key = keys[q];
                     const uint32_t sb = (uint32_t)(key >> 32), p = (uint32_t)key;
                     const int delta = t - (int32_t)p;
@@ -363,12 +390,12 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
                     rb[warp][4] = (int)plo_a; rb[warp][5] = (int)phi_a;
                     rb[warp][6] = (int)plo_b; rb[warp][7] = (int)phi_b;
                 }
-                __syncthreads();
+                gsync();
                 par ^= 1;
                 c[0] = c[1] = c[2] = c[3] = 0;
                 plo_a = plo_b = 0xffffffffu;
                 phi_a = phi_b = 0u;
-                for (int w = 0; w < NW; ++w) {
+                for (int w = gw0; w < gw0 + GW; ++w) {
                     c[0] += rb[w][0]; c[1] += rb[w][1]; c[2] += rb[w][2]; c[3] += rb[w][3];
                     plo_a = min(plo_a, (uint32_t)rb[w][4]); phi_a = max(phi_a, (uint32_t)rb[w][5]);
                     plo_b = min(plo_b, (uint32_t)rb[w][6]); phi_b = max(phi_b, (uint32_t)rb[w][7]);
@@ -382,7 +409,7 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
                     const uint32_t mid_a = plo_a + ((phi_a - plo_a) >> 1);
                     const uint32_t mid_b = plo_b + ((phi_b - plo_b) >> 1);
                     int da = 0, db = 0;
-                    for (int q = tid; q < n; q += BT) {
+                    for (int q = gtid; q < n; q += GT) {
                         const uint64_t key = keys[q];
                         const uint32_t sb = (uint32_t)(key >> 32), p = (uint32_t)key;
                         const int delta = t - (int32_t)p;
@@ -394,10 +421,10 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
                     db = __reduce_add_sync(FULL_MASK, db);
                     int (*rr)[32] = red[par];
                     if (lane == 0) { rr[warp][0] = da; rr[warp][1] = db; }
-                    __syncthreads();
+                    gsync();
                     par ^= 1;
                     da = db = 0;
-                    for (int w = 0; w < NW; ++w) { da += rr[w][0]; db += rr[w][1]; }
+                    for (int w = gw0; w < gw0 + GW; ++w) { da += rr[w][0]; db += rr[w][1]; }
                     if (tie_a && plo_a < phi_a) { if (da >= need_a) phi_a = mid_a; else plo_a = mid_a + 1; }
                     if (tie_b && plo_b < phi_b) { if (db >= need_b) phi_b = mid_b; else plo_b = mid_b + 1; }
                 }
@@ -406,7 +433,7 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
             }
             // holes and movers, listed in (thread, token) order
             int nh_mine = 0, nm_mine = 0;
-            for (int q = tid; q < n; q += BT) {
+            for (int q = gtid; q < n; q += GT) {
                 const uint64_t key = keys[q];
                 const int delta = t - (int32_t)(uint32_t)key;
                 bool ev = false;
@@ -424,18 +451,18 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
                 if (lane >= o) { xh += yh; xm += ym; }
             }
             if (lane == 31) { lists[0][warp] = xh; lists[1][warp] = xm; }
-            __syncthreads();
+            gsync();
             int oh = xh - nh_mine, om = xm - nm_mine, nh = 0, nm = 0;
-            for (int w = 0; w < NW; ++w) {
+            for (int w = gw0; w < gw0 + GW; ++w) {
                 if (w < warp) { oh += lists[0][w]; om += lists[1][w]; }
                 nh += lists[0][w];
                 nm += lists[1][w];
             }
             if (nh != nm || nh > M) {
-                if (tid == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
+                if (gtid == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
                 continue;
             }
-            for (int q = tid; q < n; q += BT) {
+            for (int q = gtid; q < n; q += GT) {
                 const uint64_t key = keys[q];
                 const int delta = t - (int32_t)(uint32_t)key;
                 bool ev = false;
@@ -446,15 +473,15 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
                 if (ev && q < target) holes[oh++] = q;
                 if (!ev && q >= target) { movers[om] = q; mpos[om] = (int32_t)(uint32_t)key; ++om; }
             }
-            __syncthreads();
+            gsync();
             // row moves: the i-th mover's K|V pair into the i-th hole, 16-byte
             // pieces, up to 4 loads in flight per thread
             const int pieces = nh * per_pair;
-            for (int w0 = 0; w0 < pieces; w0 += 4 * BT) {
+            for (int w0 = 0; w0 < pieces; w0 += 4 * GT) {
                 uint4 x[4];
     #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int w = w0 + u * BT + tid;
+                    const int w = w0 + u * GT + gtid;
                     if (w < pieces) {
                         const int i = w / per_pair, pc = w % per_pair;
                         x[u] = *reinterpret_cast<const uint4*>(KVb + (slot0 + movers[i]) * pair + pc * 16);
@@ -462,15 +489,15 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
                 }
     #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int w = w0 + u * BT + tid;
+                    const int w = w0 + u * GT + gtid;
                     if (w < pieces) {
                         const int i = w / per_pair, pc = w % per_pair;
                         *reinterpret_cast<uint4*>(KVb + (slot0 + holes[i]) * pair + pc * 16) = x[u];
                     }
                 }
             }
-            for (int i = tid; i < nh; i += BT) L.pos[slot0 + holes[i]] = mpos[i];
-            if (tid == 0) {
+            for (int i = gtid; i < nh; i += GT) L.pos[slot0 + holes[i]] = mpos[i];
+            if (gtid == 0) {
                 atomicAdd(L.ev_stats + 0, 1ull);
                 atomicAdd(L.ev_stats + 1, (unsigned long long)n);
                 atomicAdd(L.ev_stats + 2, (unsigned long long)nh);
@@ -543,25 +570,44 @@ __global__ void __launch_bounds__(128) select_batch_kernel(
 // launchers
 // ---------------------------------------------------------------------------
 
-// Dynamic shared memory of an eviction block: keys of up to n_max tokens,
-// then the hole, mover and mover-position lists of up to M entries.
-static size_t evict_block_smem(int n_max, int M) { return (size_t)n_max * 8 + (size_t)M * 12; }
+// Shared memory of one group of an eviction block: keys of up to n_max
+// tokens, then the hole, mover and mover-position lists of up to M entries.
+__host__ __device__ inline size_t evict_group_smem(int n_max, int M) {
+    return ((size_t)n_max * 8 + (size_t)M * 12 + 15) / 16 * 16;
+}
+
+// Warps per head: enough for about 256 cached tokens per warp at the usual
+// Global capacity floor(H_total * L * rho) / H_total + M (a power of two,
+// 1 .. 8), more while the groups' shared memory would not fit two blocks per
+// SM.
+int evict_group_warps(const Layout& L) {
+    const int64_t cap = L.T_total / (L.H_total > 0 ? L.H_total : L.H) + L.M;
+    int gw = 1;
+    while (gw < EVB_WARPS && cap > 256 * gw) gw *= 2;
+    while (gw < EVB_WARPS && (EVB_WARPS / gw) * evict_group_smem(L.L, L.M) > 100 * 1024) gw *= 2;
+    return gw;
+}
+
+static size_t evict_block_smem(const Layout& L) {
+    return (size_t)(EVB_WARPS / evict_group_warps(L)) * evict_group_smem(L.L, L.M);
+}
 
 int evict_blocks_per_sm(const Layout& L, int optin) {
-    const size_t sm = evict_block_smem(L.L, L.M) + 5120;  // + static
+    const size_t sm = evict_block_smem(L) + 12 * 1024;  // + static
     int by_threads = 2;  // registers: see the kernel's launch bounds
-    int by_smem = (int)((size_t)optin * 1 / sm);
+    int by_smem = (int)((size_t)optin / sm);
     int b = by_threads < by_smem ? by_threads : by_smem;
     return b < 1 ? 1 : b;
 }
 
 cudaError_t launch_evict(const Layout& L, int l0, int l1, int grid, cudaStream_t st) {
     const int n_max = L.L;
-    const size_t sm = evict_block_smem(n_max, L.M);
+    const int gw = evict_group_warps(L);
+    const size_t sm = evict_block_smem(L);
     if (L.dtype == HKV_DTYPE_BF16)
-        evict_block_kernel<__nv_bfloat16><<<grid, EVB_THREADS, sm, st>>>(L, l0, l1, n_max);
+        evict_block_kernel<__nv_bfloat16><<<grid, EVB_THREADS, sm, st>>>(L, l0, l1, n_max, gw);
     else
-        evict_block_kernel<float><<<grid, EVB_THREADS, sm, st>>>(L, l0, l1, n_max);
+        evict_block_kernel<float><<<grid, EVB_THREADS, sm, st>>>(L, l0, l1, n_max, gw);
     return cudaGetLastError();
 }
 
