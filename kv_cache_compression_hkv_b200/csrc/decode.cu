@@ -895,15 +895,18 @@ DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
     // Tuning overrides (read once per context): HKV_DECODE_WARPS caps the
     // warps per block, HKV_DECODE_STAGES fixes the stages per warp (1 ..
     // MAX_STAGES), HKV_DECODE_PROLOGUE sets DecodeShape::prologue (1 or 2),
-    // HKV_DECODE_L2_HINT=0 turns the next-layer L2 prefetch off (any other
-    // value: on).
+    // HKV_DECODE_L2_HINT=0 / =1 turns the next-layer L2 prefetch off / on.
     const int es = L.dtype == HKV_DTYPE_F32 ? 4 : 2;
     const int max_w = env_int("HKV_DECODE_WARPS");
     const int fix_s = env_int("HKV_DECODE_STAGES");
     const int pro = env_int("HKV_DECODE_PROLOGUE");
+    // the next-layer L2 prefetch pays off with many warps per block
+    // (LlamaGen-XL shape: 11.15 against 12.05 us per launch) and not with
+    // the six of a d = 128 cache (Lumina-mGPT-768 shape: 25.04 against
+    // 24.75 us): on when the block has 8 or more warps, unless overridden
     const char* hint_env = getenv("HKV_DECODE_L2_HINT");
-    const int hint = hint_env && hint_env[0] == '0' && hint_env[1] == 0 ? 0 : 1;
-    DecodeShape best{0, 0, 0, 1, pro <= 2 ? pro : 0, hint};
+    const int hint_set = hint_env ? (hint_env[0] == '0' && hint_env[1] == 0 ? 0 : 1) : -1;
+    DecodeShape best{0, 0, 0, 1, pro <= 2 ? pro : 0, 0};
     for (int ns = fix_s == 1 ? 1 : 2; ns <= MAX_STAGES; ++ns) {
         if (fix_s && ns != fix_s) continue;
         // the per-warp tail regions are laid out for MAX_STAGES barriers
@@ -912,8 +915,9 @@ DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
         if (w > DECODE_MAX_WARPS) w = DECODE_MAX_WARPS;
         if (max_w && w > max_w) w = max_w;
         if (w >= 1 && w >= best.warps)
-            best = DecodeShape{w, ns, 1024 + (size_t)w * per, 1, best.prologue, hint};
+            best = DecodeShape{w, ns, 1024 + (size_t)w * per, 1, best.prologue, 0};
     }
+    best.l2_hint = hint_set >= 0 ? hint_set : (best.warps >= 8 ? 1 : 0);
     return best;
 }
 
