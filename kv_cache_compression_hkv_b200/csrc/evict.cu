@@ -153,7 +153,8 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
     };
     const int n_heads = L.S * L.H;
     const int pair = 2 * L.d * (int)sizeof(T);                    // bytes of a K|V row pair
-    const int per_pair = pair / 16;
+    const int per_pair = pair / 16;          // a power of two: 16 .. 64
+    const int pp_shift = __ffs(per_pair) - 1;
     unsigned char* KVb = reinterpret_cast<unsigned char*>(L.K);
     int par = 0;  // reduction buffer of the next round
     const int64_t items = (int64_t)(l1 - l0) * L.S * L.H;
@@ -245,6 +246,13 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
             Two cur, nxt;
             load2(0, cur);
             gsync();  // ml_s, step_s
+            // the r = 8 scoring steps' (max, 1/sum) and positions in registers
+            float mx[8], il[8];
+            int stp[8];
+            if (r == 8) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) { mx[c] = ml_s[c].x; il[c] = ml_s[c].y; stp[c] = step_s[c]; }
+            }
 
             // scores and stratum counts; keys into shared memory; the next
             // two tokens' loads go out before this pair is used
@@ -264,7 +272,7 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
                                             cur.b[u].x, cur.b[u].y, cur.b[u].z, cur.b[u].w};
 #pragma unroll
                         for (int c = 0; c < 8; ++c)
-                            if (p <= step_s[c]) acc += exp2f(v[c] - ml_s[c].x) * ml_s[c].y;
+                            if (p <= stp[c]) acc += exp2f(v[c] - mx[c]) * il[c];
                     } else {
                         const float* lp = L.logit + (slot0 + q) * r;
                         for (int c = 0; c < r; ++c)
@@ -483,7 +491,7 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
                 for (int u = 0; u < 4; ++u) {
                     const int w = w0 + u * GT + gtid;
                     if (w < pieces) {
-                        const int i = w / per_pair, pc = w % per_pair;
+                        const int i = w >> pp_shift, pc = w & (per_pair - 1);
                         x[u] = *reinterpret_cast<const uint4*>(KVb + (slot0 + movers[i]) * pair + pc * 16);
                     }
                 }
@@ -491,7 +499,7 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
                 for (int u = 0; u < 4; ++u) {
                     const int w = w0 + u * GT + gtid;
                     if (w < pieces) {
-                        const int i = w / per_pair, pc = w % per_pair;
+                        const int i = w >> pp_shift, pc = w & (per_pair - 1);
                         *reinterpret_cast<uint4*>(KVb + (slot0 + holes[i]) * pair + pc * 16) = x[u];
                     }
                 }
