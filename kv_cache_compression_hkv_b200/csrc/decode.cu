@@ -36,6 +36,9 @@ constexpr int DECODE_MAX_WARPS = 12;
 constexpr int CHUNK_COST = 3;
 // Most chunks a range starting a decode block moves to avoid cutting a head.
 constexpr int SNAP_MAX = 2;
+// Least cost of a warp's range (two chunks of one head): small layers use
+// fewer warps rather than thinner ranges.
+constexpr int MIN_RANGE_COST = 2 * CHUNK_COST + 1;
 
 // Packed storage of DPL consecutive elements of one row.
 template <typename T, int DPL> struct Raw;
@@ -278,21 +281,25 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead,
     // i + 1; the warps w whose boundary w * cost / GW falls in it start in
     // head i, at the first of its chunks whose cost starts at or after the
     // boundary.  (Every warp start found by arithmetic, no search.)
+    // A small layer uses only the first GWe warps, about two chunks of work
+    // each or more: ranges thinner than that would split its heads into
+    // one-chunk segments whose merges cost more than the chunks.
     const int64_t tcost = (int64_t)CHUNK_COST * total + n;
+    const int GWe = (int)min((int64_t)GW, max((int64_t)1, (tcost + MIN_RANGE_COST - 1) / MIN_RANGE_COST));
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
         const int c0 = i ? cnt[i - 1] : 0, c1 = cnt[i];
         const int64_t e0 = i ? (int64_t)CHUNK_COST * c0 + i : 0;
         const int64_t e1 = (int64_t)CHUNK_COST * c1 + i + 1;
-        const int w_lo = (int)((e0 * GW + tcost - 1) / tcost);
-        const int w_hi = min((int)((e1 * GW + tcost - 1) / tcost), GW);  // exclusive
+        const int w_lo = (int)((e0 * GWe + tcost - 1) / tcost);
+        const int w_hi = min((int)((e1 * GWe + tcost - 1) / tcost), GWe);  // exclusive
         for (int w = w_lo; w < w_hi; ++w) {
-            const int64_t bnd = (int64_t)w * tcost / GW;
+            const int64_t bnd = (int64_t)w * tcost / GWe;
             const int k = (int)((bnd - e0 + CHUNK_COST - 1) / CHUNK_COST);
             wbeg[w] = c0 + min(max(k, 0), c1 - c0);
             whead[w] = i;
         }
     }
-    if (threadIdx.x == 0) wbeg[GW] = total;
+    for (int w = GWe + threadIdx.x; w <= GW; w += blockDim.x) wbeg[w] = total;  // idle warps
     __syncthreads();
     // A range starting a decode block moves to the nearer end of the head
     // it would cut (at most SNAP_MAX chunks, staying between its neighbours'
@@ -301,7 +308,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead,
     // block starts, so the entries read here are not being written.
     const int NWB = L.plan_nw;
     if (NWB > 1)
-        for (int w = NWB * (threadIdx.x + 1); w < GW; w += NWB * blockDim.x) {
+        for (int w = NWB * (threadIdx.x + 1); w < GWe; w += NWB * blockDim.x) {
             const int lo = whead[w], c = wbeg[w];
             const int c0 = lo ? cnt[lo - 1] : 0, c1 = cnt[lo];
             if (c > c0 && c < c1) {
