@@ -174,7 +174,13 @@ __device__ __forceinline__ int4 shfl_int4(const int4& v, int src) {
 // Global heads that were due at that step get their new length first (the
 // budget, from that step on) and each unit its next due step; part 0 writes
 // them, every part plans with them.
-__global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead, int commit) {
+//
+// With after_evict, the launch may start while the eviction kernel ahead of
+// it still moves rows (programmatic dependent launch; the plan reads none of
+// what the eviction writes); it completes only after that kernel, so a
+// decode launch that waits for the plan sees the compacted cache too.
+__global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead, int commit,
+                                                    int after_evict) {
     extern __shared__ int32_t psm[];
     __shared__ int wsum[32];
     const int layer = l0 + blockIdx.x;
@@ -189,6 +195,13 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead,
     uint16_t* own = reinterpret_cast<uint16_t*>(whead + PLAN_MAX_WARPS);  // [total] warp of each chunk
     const int parts = gridDim.y, part = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, NW = blockDim.x >> 5;
+    // block (0, 0) completes only after the eviction kernel ahead of it
+    struct AfterEvict {
+        bool on;
+        __device__ ~AfterEvict() {
+            if (on) ptx::grid_dep_wait();
+        }
+    } after{after_evict && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0};
     const int te = L.t_next[layer] - 1;  // newest cached position
     const int t = te + ahead;
     const size_t hbase = (size_t)layer * n;
@@ -961,10 +974,19 @@ cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void*
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_plan(const Layout& L, int l0, int l1, int ahead, int commit, cudaStream_t st) {
-    plan_kernel<<<dim3(l1 - l0, PLAN_DESC_PARTS), 1024, plan_smem_bytes(L.S * L.H, L.max_chunks), st>>>(
-        L, l0, ahead, commit);
-    return cudaGetLastError();
+cudaError_t launch_plan(const Layout& L, int l0, int l1, int ahead, int commit, cudaStream_t st,
+                        int after_evict) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(l1 - l0, PLAN_DESC_PARTS);
+    cfg.blockDim = dim3(1024);
+    cfg.dynamicSmemBytes = plan_smem_bytes(L.S * L.H, L.max_chunks);
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = after_evict ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, plan_kernel, L, l0, ahead, commit, after_evict);
 }
 
 cudaError_t launch_append(const Layout& L, int layer, const void* k, const void* v, cudaStream_t st) {

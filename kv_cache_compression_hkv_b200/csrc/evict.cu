@@ -159,6 +159,7 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
     int par = 0;  // reduction buffer of the next round
     const int64_t items = (int64_t)(l1 - l0) * L.S * L.H;
     const int64_t G = gridDim.x;
+    if ((int64_t)blockIdx.x >= items) ptx::grid_dep_trigger();
 
     for (int64_t k0 = 0; (int64_t)blockIdx.x + k0 * G < items; k0 += BT) {
         // this block's next BT items: the due ones, in item order, each with
@@ -189,6 +190,10 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
             if (tid == 0) n_due = tot;
             __syncthreads();
         }
+        // every unit record this block reads has been read: the plan
+        // launched after this kernel (which commits the new lengths and due
+        // steps) may start
+        if ((int64_t)blockIdx.x + (k0 + BT) * G >= items) ptx::grid_dep_trigger();
         const int nd = n_due;
         for (int e = grp; e < nd; e += ngroups) {
             const int4 item = due_items[e];
@@ -216,7 +221,10 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
             bool head_bad = false;
             if (gtid == 0) {
                 ptx::bulk_prefetch_l2(KVb + (slot0 + target) * pair, (uint32_t)(M * pair));
-                head_bad = len_at(L, hx, t) != n;
+                // the head's length record, before or after the plan kernel
+                // running next to this one commits it
+                const uint64_t b = L.base[hx];
+                head_bad = !(base_len_of(b) + (t - base_t_of(b)) == n || b == base_pack(target, t));
             }
             if (gtid < r) {
                 const float2 ml = L.ml[hx * r + gtid];

@@ -391,7 +391,7 @@ hkv_status hkv_ste_evict(hkv_ctx* c, int32_t layer_begin, int32_t layer_end, voi
     // lengths of the heads just evicted
     if (e == cudaSuccess)
         e = hkv::launch_plan(c->lay, layer_begin, layer_end, 1, c->cfg.mode != HKV_MODE_FULL,
-                             (cudaStream_t)stream);
+                             (cudaStream_t)stream, c->cfg.mode != HKV_MODE_FULL);
     if (e != cudaSuccess) return HKV_ERR_CUDA;
     for (int l = layer_begin; l < layer_end; ++l) c->plan_for[l] = c->t_host[l];
     return HKV_OK;

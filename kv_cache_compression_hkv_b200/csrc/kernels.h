@@ -48,7 +48,10 @@ cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void*
                           void* o, int append, const DecodeShape& sh, int grid, int early, int buf,
                           cudaStream_t st);
 // commit: the launch right after an eviction (see plan_kernel)
-cudaError_t launch_plan(const Layout& L, int l0, int l1, int ahead, int commit, cudaStream_t st);
+// after_evict: launched right behind the eviction kernel, which it may
+// overlap (see plan_kernel)
+cudaError_t launch_plan(const Layout& L, int l0, int l1, int ahead, int commit, cudaStream_t st,
+                        int after_evict = 0);
 // Shared memory of the plan kernel: four words per head of a layer, two per
 // warp of the decode grid (and one more), two bytes per chunk.
 inline size_t plan_smem_bytes(int heads_per_layer, int max_chunks) {
