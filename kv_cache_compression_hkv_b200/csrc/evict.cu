@@ -47,6 +47,12 @@ namespace hkv {
 constexpr int EVB_THREADS = 256;  // threads of an eviction block
 constexpr int EVB_WARPS = EVB_THREADS / 32;
 __host__ __device__ inline size_t evict_group_smem(int n_max, int M);
+// A stratum whose search window holds at most this many keys is finished by
+// ranking those keys against each other.
+constexpr int RANK_WIN = 32;
+// Shared memory of the ranking: two candidate lists, their counters, the
+// two thresholds.
+constexpr int EVB_RANK_BYTES = 2 * RANK_WIN * 8 + 16 + 16;
 
 // One round of the threshold search of both strata: every thread adds its
 // candidate keys with score bits in [lo, hi] of their stratum to 16 bins of
@@ -54,11 +60,11 @@ __host__ __device__ inline size_t evict_group_smem(int n_max, int M);
 // far fewer than 65536 keys) and counts those below lo; the totals of the
 // head's group of warps (w0 .. w0 + nw - 1) are reduced through `red` (this
 // round's buffer; rounds alternate between two, so one group barrier per
-// round suffices).  Lane i of every warp returns the number of keys at or
-// below the top of bin i (i < 16: near stratum, else bin i - 16 of the far
-// stratum).
+// round suffices).  Lane i of every warp returns {the number of keys at or
+// below the top of bin i, the number below lo} (i < 16: near stratum, else
+// bin i - 16 of the far stratum).
 template <typename Sync>
-__device__ __forceinline__ int group_bin_counts(const uint32_t (&ha)[8], const uint32_t (&hb)[8],
+__device__ __forceinline__ int2 group_bin_counts(const uint32_t (&ha)[8], const uint32_t (&hb)[8],
                                                 int below_a, int below_b, int (*red)[32], int w0,
                                                 int nw, Sync gsync) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -90,7 +96,7 @@ __device__ __forceinline__ int group_bin_counts(const uint32_t (&ha)[8], const u
         const int y = __shfl_up_sync(FULL_MASK, tot, o);
         if ((lane & 15) >= o) tot += y;
     }
-    return tot + below;
+    return make_int2(tot + below, below);
 }
 
 // Adds one candidate key to its stratum's packed bins.
@@ -133,6 +139,9 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
     int32_t* holes = reinterpret_cast<int32_t*>(keys + n_max);    // [M]
     int32_t* movers = holes + M;                                  // [M]
     int32_t* mpos = movers + M;                                   // [M]
+    uint64_t* cand = reinterpret_cast<uint64_t*>(gbase + ((size_t)n_max * 8 + (size_t)M * 12 + 15) / 16 * 16);
+    int* ccnt = reinterpret_cast<int*>(cand + 2 * RANK_WIN);      // [2] (+ 2 spare)
+    uint64_t* thr_sm = reinterpret_cast<uint64_t*>(ccnt + 4);     // [2]
     float2* ml_s = ml_all[grp];
     int* step_s = step_all[grp];
     // barrier of the head's group (one warp: the warp itself)
@@ -338,12 +347,15 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
                 kb = E < nf ? E : nf;
                 ka = 0;
             }
-            // threshold search: stratum x is active while 0 < k < m and its
-            // score range is not one value; thr = every key <= it is evicted
+            // threshold of each partial stratum (0 < k < m): the k-th smallest
+            // key.  A window of score bits [lo, hi] that holds it shrinks
+            // 16-fold per round until it holds at most RANK_WIN keys (or one
+            // score value); those keys are then ranked against each other
             const bool a_part = ka > 0 && ka < nn, b_part = kb > 0 && kb < nf;
-            if (!a_part) alo = ahi = 0u;
-            if (!b_part) blo = bhi = 0u;
-            while (alo < ahi || blo < bhi) {
+            int bel_a = 0, win_a = nn, bel_b = 0, win_b = nf;  // keys below / inside the window
+            bool sa_on = a_part && alo < ahi && win_a > RANK_WIN;
+            bool sb_on = b_part && blo < bhi && win_b > RANK_WIN;
+            while (sa_on || sb_on) {
                 const int sa = bin_shift(alo, ahi), sbh = bin_shift(blo, bhi);
                 uint32_t ha[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u}, hb[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
                 int below_a = 0, below_b = 0;
@@ -352,36 +364,83 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
                     const uint32_t sb = (uint32_t)(key >> 32);
                     const int delta = t - (int32_t)(uint32_t)key;
                     if (delta < 1) continue;
-                    if (strat && delta <= L.D) bin_add(ha, below_a, sb, alo, ahi, sa);
-                    else bin_add(hb, below_b, sb, blo, bhi, sbh);
+                    if (strat && delta <= L.D) { if (sa_on) bin_add(ha, below_a, sb, alo, ahi, sa); }
+                    else if (sb_on) bin_add(hb, below_b, sb, blo, bhi, sbh);
                 }
-                const int cum = group_bin_counts(ha, hb, below_a, below_b, red[par], gw0, GW, gsync);
+                const int2 cb = group_bin_counts(ha, hb, below_a, below_b, red[par], gw0, GW, gsync);
                 par ^= 1;
-                // first bin whose cumulative count reaches the share
+                const int cum = cb.x;
+                // first bin whose cumulative count reaches the share; the keys
+                // before it (the bin before's total, or those below lo)
                 const unsigned ma = __ballot_sync(FULL_MASK, lane < 16 && cum >= ka);
                 const unsigned mb = __ballot_sync(FULL_MASK, lane >= 16 && cum >= kb);
-                if (alo < ahi) {
-                    const uint32_t j = (uint32_t)(__ffs(ma) - 1);  // exists: all of [lo, hi] reaches k
-                    const uint32_t nlo = alo + (j << sa);
-                    const uint64_t top = (uint64_t)alo + ((uint64_t)(j + 1) << sa) - 1;
-                    alo = nlo;
+                const int ja = ma ? __ffs(ma) - 1 : 0, jb = mb ? __ffs(mb >> 16) - 1 : 0;
+                const int at_a = __shfl_sync(FULL_MASK, cum, ja), at_b = __shfl_sync(FULL_MASK, cum, 16 + jb);
+                const int pre_a = __shfl_sync(FULL_MASK, ja ? cum : cb.y, ja ? ja - 1 : 0);
+                const int pre_b = __shfl_sync(FULL_MASK, jb ? cum : cb.y, jb ? 15 + jb : 16);
+                if (sa_on) {
+                    const uint64_t top = (uint64_t)alo + ((uint64_t)(ja + 1) << sa) - 1;
+                    alo = alo + ((uint32_t)ja << sa);
                     ahi = top < ahi ? (uint32_t)top : ahi;
+                    bel_a = pre_a;
+                    win_a = at_a - pre_a;
+                    sa_on = alo < ahi && win_a > RANK_WIN;
                 }
-                if (blo < bhi) {
-                    const uint32_t j = (uint32_t)(__ffs(mb >> 16) - 1);
-                    const uint32_t nlo = blo + (j << sbh);
-                    const uint64_t top = (uint64_t)blo + ((uint64_t)(j + 1) << sbh) - 1;
-                    blo = nlo;
+                if (sb_on) {
+                    const uint64_t top = (uint64_t)blo + ((uint64_t)(jb + 1) << sbh) - 1;
+                    blo = blo + ((uint32_t)jb << sbh);
                     bhi = top < bhi ? (uint32_t)top : bhi;
+                    bel_b = pre_b;
+                    win_b = at_b - pre_b;
+                    sb_on = blo < bhi && win_b > RANK_WIN;
                 }
             }
-            // the position tie at each boundary score s*: need = k - (keys below
-            // s*) of the tied keys go, lowest positions first
+            const int need_a = ka - bel_a, need_b = kb - bel_b;  // rank in the window, 1..win
+            // every key <= thr of its stratum is evicted
             uint64_t thr_a = a_part ? 0ull : (ka >= nn && ka > 0 ? ~0ull : 0ull);
             uint64_t thr_b = b_part ? 0ull : (kb >= nf && kb > 0 ? ~0ull : 0ull);
-            bool none_a = ka <= 0, none_b = kb <= 0;
-            if (a_part || b_part) {
-                int c[4] = {0, 0, 0, 0};  // below s* and at s*, near then far
+            const bool none_a = ka <= 0, none_b = kb <= 0;
+            const bool rank_a = a_part && win_a <= RANK_WIN, rank_b = b_part && win_b <= RANK_WIN;
+            if (rank_a || rank_b) {
+                // the window's keys into two lists, ranked by the group's first warp
+                if (gtid < 2) ccnt[gtid] = 0;
+                gsync();
+                for (int q = gtid; q < n; q += GT) {
+                    const uint64_t key = keys[q];
+                    const uint32_t sb = (uint32_t)(key >> 32);
+                    const int delta = t - (int32_t)(uint32_t)key;
+                    if (delta < 1) continue;
+                    if (strat && delta <= L.D) {
+                        if (rank_a && sb >= alo && sb <= ahi) {
+                            const int i = atomicAdd(&ccnt[0], 1);
+                            if (i < RANK_WIN) cand[i] = key;
+                        }
+                    } else if (rank_b && sb >= blo && sb <= bhi) {
+                        const int i = atomicAdd(&ccnt[1], 1);
+                        if (i < RANK_WIN) cand[RANK_WIN + i] = key;
+                    }
+                }
+                gsync();
+                if (warp == gw0) {
+#pragma unroll
+                    for (int x = 0; x < 2; ++x) {
+                        const bool on = x == 0 ? rank_a : rank_b;
+                        const int cnt = x == 0 ? win_a : win_b, need = x == 0 ? need_a : need_b;
+                        if (!on) continue;
+                        const uint64_t* cl = cand + x * RANK_WIN;
+                        const uint64_t mine = lane < cnt ? cl[lane] : ~0ull;
+                        int rk = 0;
+                        for (int j = 0; j < cnt; ++j) rk += cl[j] < mine;
+                        if (lane < cnt && rk == need - 1) thr_sm[x] = mine;
+                    }
+                }
+                gsync();
+                if (rank_a) thr_a = thr_sm[0];
+                if (rank_b) thr_b = thr_sm[1];
+            }
+            const bool tie_a = a_part && !rank_a, tie_b = b_part && !rank_b;  // one score, many keys
+            if (tie_a || tie_b) {
+                // the need lowest positions among the keys at the one score s*
                 uint32_t plo_a = 0xffffffffu, phi_a = 0u, plo_b = 0xffffffffu, phi_b = 0u;
                 for (int q = gtid; q < n; q += GT) {
                     const uint64_t key = keys[q];
@@ -389,38 +448,27 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
                     const int delta = t - (int32_t)p;
                     if (delta < 1) continue;
                     if (strat && delta <= L.D) {
-                        c[0] += sb < alo;
-                        if (sb == alo) { ++c[1]; plo_a = min(plo_a, p); phi_a = max(phi_a, p); }
-                    } else {
-                        c[2] += sb < blo;
-                        if (sb == blo) { ++c[3]; plo_b = min(plo_b, p); phi_b = max(phi_b, p); }
+                        if (sb == alo) { plo_a = min(plo_a, p); phi_a = max(phi_a, p); }
+                    } else if (sb == blo) {
+                        plo_b = min(plo_b, p); phi_b = max(phi_b, p);
                     }
                 }
                 int (*rb)[32] = red[par];
-    #pragma unroll
-                for (int j = 0; j < 4; ++j) c[j] = __reduce_add_sync(FULL_MASK, c[j]);
                 plo_a = __reduce_min_sync(FULL_MASK, plo_a); phi_a = __reduce_max_sync(FULL_MASK, phi_a);
                 plo_b = __reduce_min_sync(FULL_MASK, plo_b); phi_b = __reduce_max_sync(FULL_MASK, phi_b);
                 if (lane == 0) {
-                    rb[warp][0] = c[0]; rb[warp][1] = c[1]; rb[warp][2] = c[2]; rb[warp][3] = c[3];
                     rb[warp][4] = (int)plo_a; rb[warp][5] = (int)phi_a;
                     rb[warp][6] = (int)plo_b; rb[warp][7] = (int)phi_b;
                 }
                 gsync();
                 par ^= 1;
-                c[0] = c[1] = c[2] = c[3] = 0;
                 plo_a = plo_b = 0xffffffffu;
                 phi_a = phi_b = 0u;
                 for (int w = gw0; w < gw0 + GW; ++w) {
-                    c[0] += rb[w][0]; c[1] += rb[w][1]; c[2] += rb[w][2]; c[3] += rb[w][3];
                     plo_a = min(plo_a, (uint32_t)rb[w][4]); phi_a = max(phi_a, (uint32_t)rb[w][5]);
                     plo_b = min(plo_b, (uint32_t)rb[w][6]); phi_b = max(phi_b, (uint32_t)rb[w][7]);
                 }
-                const int need_a = ka - c[0], need_b = kb - c[2];  // 1 <= need <= eq
-                bool tie_a = a_part && need_a < c[1], tie_b = b_part && need_b < c[3];
-                if (a_part && !tie_a) plo_a = phi_a;  // every tied key goes
-                if (b_part && !tie_b) plo_b = phi_b;
-                // bisection on positions among the tied keys (rare: equal fp32 scores)
+                // bisection on positions (every key of the window has score s*)
                 while ((tie_a && plo_a < phi_a) || (tie_b && plo_b < phi_b)) {
                     const uint32_t mid_a = plo_a + ((phi_a - plo_a) >> 1);
                     const uint32_t mid_b = plo_b + ((phi_b - plo_b) >> 1);
@@ -444,8 +492,8 @@ __global__ void __launch_bounds__(EVB_THREADS, 2) evict_block_kernel(Layout L, i
                     if (tie_a && plo_a < phi_a) { if (da >= need_a) phi_a = mid_a; else plo_a = mid_a + 1; }
                     if (tie_b && plo_b < phi_b) { if (db >= need_b) phi_b = mid_b; else plo_b = mid_b + 1; }
                 }
-                if (a_part) thr_a = ((uint64_t)alo << 32) | plo_a;
-                if (b_part) thr_b = ((uint64_t)blo << 32) | plo_b;
+                if (tie_a) thr_a = ((uint64_t)alo << 32) | plo_a;
+                if (tie_b) thr_b = ((uint64_t)blo << 32) | plo_b;
             }
             // holes and movers, listed in (thread, token) order
             int nh_mine = 0, nm_mine = 0;
@@ -589,7 +637,7 @@ __global__ void __launch_bounds__(128) select_batch_kernel(
 // Shared memory of one group of an eviction block: keys of up to n_max
 // tokens, then the hole, mover and mover-position lists of up to M entries.
 __host__ __device__ inline size_t evict_group_smem(int n_max, int M) {
-    return ((size_t)n_max * 8 + (size_t)M * 12 + 15) / 16 * 16;
+    return ((size_t)n_max * 8 + (size_t)M * 12 + 15) / 16 * 16 + EVB_RANK_BYTES;
 }
 
 // Warps per head: enough for about 256 cached tokens per warp at the usual
