@@ -385,8 +385,12 @@ hkv_status hkv_ste_evict(hkv_ctx* c, int32_t layer_begin, int32_t layer_end, voi
         if (!c->classified[l]) return HKV_ERR_STATE;
     cudaError_t e = cudaSuccess;
     note_other(c, stream);
-    if (c->cfg.mode != HKV_MODE_FULL)
-        e = hkv::launch_evict(c->lay, layer_begin, layer_end, c->evict_grid, (cudaStream_t)stream);
+    if (c->cfg.mode != HKV_MODE_FULL) {
+        // no more blocks than (unit, head) items: a small cache launches few
+        const int64_t items = (int64_t)(layer_end - layer_begin) * c->cfg.num_seqs * c->cfg.num_heads;
+        const int grid = items < c->evict_grid ? (int)items : c->evict_grid;
+        e = hkv::launch_evict(c->lay, layer_begin, layer_end, grid, (cudaStream_t)stream);
+    }
     // plans of the next step, made once for all these layers, with the new
     // lengths of the heads just evicted
     if (e == cudaSuccess)

@@ -591,14 +591,19 @@ __device__ __forceinline__ int warp_group_need_rows(const float* ra, const float
 }
 
 // Allows `func` as much dynamic shared memory as the device's opt-in limit
-// leaves next to its static shared memory.
+// leaves next to its static shared memory, and asks for the largest shared
+// memory carve-out: the kernels of a decode step then all run under the same
+// L1 / shared split, and an SM does not repartition between them.
 template <typename F>
 inline cudaError_t allow_max_dynamic_smem(F* func, int optin) {
     cudaFuncAttributes a;
     cudaError_t e = cudaFuncGetAttributes(&a, func);
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                optin - (int)a.sharedSizeBytes);
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             optin - (int)a.sharedSizeBytes);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                (int)cudaSharedmemCarveoutMaxShared);
 }
 
 }  // namespace hkv
