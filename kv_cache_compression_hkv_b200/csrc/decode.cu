@@ -31,14 +31,10 @@ constexpr float RESCALE = 8.f;
 constexpr int MAX_STAGES = 4;
 // Most warps of one decode block (one block per SM).
 constexpr int DECODE_MAX_WARPS = 12;
-// Cost of a chunk, in units of the cost of a head's end, in the plan's
-// balancing of the warp ranges.
-constexpr int CHUNK_COST = 3;
+
 // Most chunks a range starting a decode block moves to avoid cutting a head.
 constexpr int SNAP_MAX = 2;
-// Least cost of a warp's range (two chunks of one head): small layers use
-// fewer warps rather than thinner ranges.
-constexpr int MIN_RANGE_COST = 2 * CHUNK_COST + 1;
+
 
 // Packed storage of DPL consecutive elements of one row.
 template <typename T, int DPL> struct Raw;

@@ -235,6 +235,16 @@ hkv_status hkv_create(const hkv_config* cfg, void* pool, size_t bytes, void* str
     }
     c->decode_sh = hkv::decode_shape(c->lay, (size_t)optin - 256);
     c->decode_grid = c->n_sm * c->decode_sh.per_sm;  // persistent: every block resident
+    {
+        // A small cache needs fewer blocks: the plan gives a warp at least
+        // MIN_RANGE_COST of work, and a layer holds at most
+        // max_chunks chunks (S heads' slot regions in 32-token chunks, one
+        // partial chunk per head).
+        const int64_t tcost = (int64_t)hkv::CHUNK_COST * c->lay.max_chunks + (int64_t)cfg->num_seqs * cfg->num_heads;
+        const int64_t warps = (tcost + hkv::MIN_RANGE_COST - 1) / hkv::MIN_RANGE_COST;
+        const int64_t blocks = (warps + c->decode_sh.warps - 1) / c->decode_sh.warps;
+        if (blocks < c->decode_grid) c->decode_grid = (int)(blocks < 1 ? 1 : blocks);
+    }
     if (c->decode_sh.warps == 0 || c->decode_grid * c->decode_sh.warps > hkv::PLAN_MAX_WARPS) {
         delete c;
         return HKV_ERR_INVALID_ARG;

@@ -17,6 +17,12 @@ constexpr int PLAN_MAX_WARPS = 2048;  // capacity of a decode plan's warp table
 constexpr int PLAN_WARP_DESC = 7;     // descriptors copied into each warp's plan block
 constexpr int PLAN_DESC_PARTS = 4;    // blocks per layer of the plan kernel
 constexpr int RANK_MAX = 32;          // strata up to this size are selected by ranking
+// Cost of a decode chunk, in units of the cost of a head's end, in the
+// plan's balancing of the warp ranges.
+constexpr int CHUNK_COST = 3;
+// Least cost of a warp's range (two chunks of one head): small layers use
+// fewer warps rather than thinner ranges, and a small cache fewer blocks.
+constexpr int MIN_RANGE_COST = 2 * CHUNK_COST + 1;
 
 // Everything a kernel needs to find the state of a (layer, sequence, head).
 // The pool is one caller-owned device buffer carved into these regions.
