@@ -169,8 +169,11 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int b = blockIdx.x;            // sequence * H + head
-    const int q0 = blockIdx.y * QT;      // first query of the tile
+    // the query tiles of one (sequence, head) block are neighbours in the
+    // grid, so its K and V tiles are read from HBM once and then from L2;
+    // the longest (last) tile first
+    const int b = blockIdx.y;                           // sequence * H + head
+    const int q0 = (gridDim.x - 1 - blockIdx.x) * QT;   // first query of the tile
     const int n_keys = min(P, q0 + QT);  // causal limit of the tile
     const int nkt = (n_keys + KT - 1) / KT;
     constexpr int NSUB = D / 64;         // 64-column swizzle sub-tiles
@@ -453,7 +456,8 @@ cudaError_t launch_prefill_umma(const Layout& L, const void* q, const void* k, c
         !make_map(&km, k, L.d, P, nblk, block_stride, umma::KT) ||
         !make_map(&vm, v, L.d, P, nblk, block_stride, umma::KT))
         return cudaErrorInvalidValue;
-    dim3 grid(nblk, (P + umma::QT - 1) / umma::QT);
+    if (nblk > 65535) return cudaErrorInvalidValue;
+    dim3 grid((P + umma::QT - 1) / umma::QT, nblk);
     const size_t sm = umma::Smem::total(L.d);
     if (L.d == 128)
         umma::prefill_attn_umma<128><<<grid, umma::NTHREADS, sm, st>>>(qm, km, vm, P, L.r, (__nv_bfloat16*)out,
