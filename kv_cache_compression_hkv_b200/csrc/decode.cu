@@ -281,24 +281,24 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead,
         if (tid == 0 && part == 0) latch_error(L, HKV_ERR_STATE, layer);
         return;
     }
-    // Warp ranges of equal cost: a chunk costs CHUNK_COST units and a head
-    // one more (its end: reductions, output, a merge when split), so that
-    // warps holding many short heads get fewer chunks.  Head i's cost ends
-    // at CHUNK_COST * cnt[i] + i + 1; warp w's range starts at the first
-    // chunk whose cost starts at or after w * cost / GW.
-    // Head i's cost interval is [E(i-1), E(i)), E(i) = CHUNK_COST * cnt[i] +
-    // i + 1; the warps w whose boundary w * cost / GW falls in it start in
-    // head i, at the first of its chunks whose cost starts at or after the
+    // Warp ranges of equal cost: a chunk costs CHUNK_COST units and the end
+    // of a head HC more (reductions, output, a merge when split), so that
+    // warps holding many short heads get fewer chunks.  Head i's cost
+    // interval is [E(i-1), E(i)), E(i) = CHUNK_COST * cnt[i] + HC (i + 1);
+    // the warps w whose boundary w * cost / GW falls in it start in head i,
+    // at the first of its chunks whose cost starts at or after the
     // boundary.  (Every warp start found by arithmetic, no search.)
     // A small layer uses only the first GWe warps, about two chunks of work
     // each or more: ranges thinner than that would split its heads into
     // one-chunk segments whose merges cost more than the chunks.
-    const int64_t tcost = (int64_t)CHUNK_COST * total + n;
-    const int GWe = (int)min((int64_t)GW, max((int64_t)1, (tcost + MIN_RANGE_COST - 1) / MIN_RANGE_COST));
+    const int HC = L.plan_hc;
+    const int64_t tcost = (int64_t)CHUNK_COST * total + (int64_t)HC * n;
+    const int64_t mrc = min_range_cost(HC);
+    const int GWe = (int)min((int64_t)GW, max((int64_t)1, (tcost + mrc - 1) / mrc));
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
         const int c0 = i ? cnt[i - 1] : 0, c1 = cnt[i];
-        const int64_t e0 = i ? (int64_t)CHUNK_COST * c0 + i : 0;
-        const int64_t e1 = (int64_t)CHUNK_COST * c1 + i + 1;
+        const int64_t e0 = (int64_t)CHUNK_COST * c0 + (int64_t)HC * i;
+        const int64_t e1 = (int64_t)CHUNK_COST * c1 + (int64_t)HC * (i + 1);
         const int w_lo = (int)((e0 * GWe + tcost - 1) / tcost);
         const int w_hi = min((int)((e1 * GWe + tcost - 1) / tcost), GWe);  // exclusive
         for (int w = w_lo; w < w_hi; ++w) {
@@ -911,7 +911,8 @@ DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
     // Tuning overrides (read once per context): HKV_DECODE_WARPS caps the
     // warps per block, HKV_DECODE_STAGES fixes the stages per warp (1 ..
     // MAX_STAGES), HKV_DECODE_PROLOGUE sets DecodeShape::prologue (1 or 2),
-    // HKV_DECODE_L2_HINT=0 / =1 turns the next-layer L2 prefetch off / on.
+    // HKV_DECODE_L2_HINT=0 / =1 turns the next-layer L2 prefetch off / on,
+    // HKV_DECODE_HEAD_COST (1 .. 4 CHUNK_COST) sets DecodeShape::head_cost.
     const int es = L.dtype == HKV_DTYPE_F32 ? 4 : 2;
     const int max_w = env_int("HKV_DECODE_WARPS");
     const int fix_s = env_int("HKV_DECODE_STAGES");
@@ -922,7 +923,7 @@ DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
     // 24.75 us): on when the block has 8 or more warps, unless overridden
     const char* hint_env = getenv("HKV_DECODE_L2_HINT");
     const int hint_set = hint_env ? (hint_env[0] == '0' && hint_env[1] == 0 ? 0 : 1) : -1;
-    DecodeShape best{0, 0, 0, 1, pro <= 2 ? pro : 0, 0};
+    DecodeShape best{0, 0, 0, 1, pro <= 2 ? pro : 0, 0, HEAD_COST};
     for (int ns = fix_s == 1 ? 1 : 2; ns <= MAX_STAGES; ++ns) {
         if (fix_s && ns != fix_s) continue;
         // the per-warp tail regions are laid out for MAX_STAGES barriers
@@ -931,9 +932,11 @@ DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
         if (w > DECODE_MAX_WARPS) w = DECODE_MAX_WARPS;
         if (max_w && w > max_w) w = max_w;
         if (w >= 1 && w >= best.warps)
-            best = DecodeShape{w, ns, 1024 + (size_t)w * per, 1, best.prologue, 0};
+            best = DecodeShape{w, ns, 1024 + (size_t)w * per, 1, best.prologue, 0, HEAD_COST};
     }
     best.l2_hint = hint_set >= 0 ? hint_set : (best.warps >= 8 ? 1 : 0);
+    const int hc = env_int("HKV_DECODE_HEAD_COST");
+    if (hc > 0 && hc <= 4 * CHUNK_COST) best.head_cost = hc;
     return best;
 }
 

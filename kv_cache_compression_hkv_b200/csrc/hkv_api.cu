@@ -237,11 +237,13 @@ hkv_status hkv_create(const hkv_config* cfg, void* pool, size_t bytes, void* str
     c->decode_grid = c->n_sm * c->decode_sh.per_sm;  // persistent: every block resident
     {
         // A small cache needs fewer blocks: the plan gives a warp at least
-        // MIN_RANGE_COST of work, and a layer holds at most
+        // min_range_cost of work, and a layer holds at most
         // max_chunks chunks (S heads' slot regions in 32-token chunks, one
         // partial chunk per head).
-        const int64_t tcost = (int64_t)hkv::CHUNK_COST * c->lay.max_chunks + (int64_t)cfg->num_seqs * cfg->num_heads;
-        const int64_t warps = (tcost + hkv::MIN_RANGE_COST - 1) / hkv::MIN_RANGE_COST;
+        const int hc = c->decode_sh.head_cost;
+        const int64_t tcost = (int64_t)hkv::CHUNK_COST * c->lay.max_chunks + (int64_t)hc * cfg->num_seqs * cfg->num_heads;
+        const int64_t mrc = hkv::min_range_cost(hc);
+        const int64_t warps = (tcost + mrc - 1) / mrc;
         const int64_t blocks = (warps + c->decode_sh.warps - 1) / c->decode_sh.warps;
         if (blocks < c->decode_grid) c->decode_grid = (int)(blocks < 1 ? 1 : blocks);
     }
@@ -251,6 +253,7 @@ hkv_status hkv_create(const hkv_config* cfg, void* pool, size_t bytes, void* str
     }
     c->lay.plan_gw = c->decode_grid * c->decode_sh.warps;
     c->lay.plan_nw = c->decode_sh.warps;
+    c->lay.plan_hc = c->decode_sh.head_cost;
     c->plan_for.assign(cfg->num_layers, -1);
     c->evict_grid = c->n_sm * hkv::evict_blocks_per_sm(c->lay, optin);
     *out = c;

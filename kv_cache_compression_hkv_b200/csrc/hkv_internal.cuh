@@ -17,12 +17,18 @@ constexpr int PLAN_MAX_WARPS = 2048;  // capacity of a decode plan's warp table
 constexpr int PLAN_WARP_DESC = 7;     // descriptors copied into each warp's plan block
 constexpr int PLAN_DESC_PARTS = 4;    // blocks per layer of the plan kernel
 constexpr int RANK_MAX = 32;          // strata up to this size are selected by ranking
-// Cost of a decode chunk, in units of the cost of a head's end, in the
-// plan's balancing of the warp ranges.
+// Costs in the plan's balancing of the warp ranges: a decode chunk costs
+// CHUNK_COST, the end of a head's segment (reductions, output, a merge
+// when split) HEAD_COST by default.  Per-warp timings of the decode launch
+// put a head's end at about two thirds of a chunk on average; launch times
+// are shortest with it weighted higher (the warps that end a launch are the
+// ones with many head ends: 5 / 3 gave 2-5% shorter launches than 1 / 3 on
+// the Lumina-mGPT-768 and LlamaGen-XL shapes).
 constexpr int CHUNK_COST = 3;
+constexpr int HEAD_COST = 5;
 // Least cost of a warp's range (two chunks of one head): small layers use
 // fewer warps rather than thinner ranges, and a small cache fewer blocks.
-constexpr int MIN_RANGE_COST = 2 * CHUNK_COST + 1;
+__host__ __device__ constexpr int min_range_cost(int head_cost) { return 2 * CHUNK_COST + head_cost; }
 
 // Everything a kernel needs to find the state of a (layer, sequence, head).
 // The pool is one caller-owned device buffer carved into these regions.
@@ -75,6 +81,7 @@ struct Layout {
     int4* plan_warp;
     int32_t plan_gw;     // warps of one decode launch
     int32_t plan_nw;     // warps of one decode block
+    int32_t plan_hc;     // cost of a head's end in the plan's balancing
     int32_t max_chunks;
 };
 

@@ -39,6 +39,7 @@ struct DecodeShape {
                    // 0 one when the block has 8 or more warps, else all;
                    // 1 one; 2 all
     int l2_hint;   // 1: finished warps prefetch the next layer's first chunks into L2
+    int head_cost; // cost of a head's end in the plan's balancing (CHUNK_COST per chunk)
 };
 DecodeShape decode_shape(const Layout& L, size_t smem_limit);
 // early: the previous launch in `st` is a decode launch of another layer (the

@@ -422,6 +422,14 @@ def test_full_size_sampled_units():
     _lockstep(w, units, seed=2024)
 
 
+def test_full_size_lumina_sampled_units():
+    """The default bench workload (Lumina-mGPT-768: 16 sequences, 32
+    layers) at full size and launch configuration; two sampled units go
+    through the oracle in lock step."""
+    w = WORKLOADS["lumina_mgpt_768"]
+    _lockstep(w, [(3, 0), (12, 31)], seed=2025)
+
+
 # ---------------------------------------------------------------------------
 # errors: argument checks, call order, device-side status
 # ---------------------------------------------------------------------------
