@@ -305,11 +305,20 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
                 x[c] = (key <= qpos && key < P) ? __uint_as_float(sr[c >> 5][c & 31]) * scale : -INFINITY;
                 mt = fmaxf(mt, x[c]);
             }
-            if (rrow) {
+            if (rrow) {  // normalised in the epilogue
+                if ((P & 3) == 0) {  // 16-byte rows: whole float4 groups
 #pragma unroll
-                for (int c = 0; c < KT; ++c) {
-                    const int key = j * KT + c;
-                    if (key < P) rrow[key] = x[c];  // normalised in the epilogue
+                    for (int c = 0; c < KT; c += 4) {
+                        const int key = j * KT + c;
+                        if (key < P)
+                            *reinterpret_cast<float4*>(rrow + key) = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < KT; ++c) {
+                        const int key = j * KT + c;
+                        if (key < P) rrow[key] = x[c];
+                    }
                 }
             }
             if (__any_sync(FULL_MASK, mt > m + RESCALE)) {
@@ -372,10 +381,18 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
         if (!fail) {
             fence_after();
             const float inv_l = 1.0f / l;
-            if (rrow) {
-                // the kept rows' weights over every key, exactly normalised
-                for (int key = 0; key < P; ++key)
-                    rrow[key] = key <= qpos ? exp2f(rrow[key] - m) * inv_l : 0.f;
+            // the kept rows' weights over every key, exactly normalised; the
+            // warp's lanes share each kept row's keys (coalesced, independent
+            // loads) instead of its own thread walking them one by one
+            for (unsigned keep = __ballot_sync(FULL_MASK, rrow != nullptr); keep; keep &= keep - 1) {
+                const int src = __ffs(keep) - 1;
+                const float ms = __shfl_sync(FULL_MASK, m, src);
+                const float il = __shfl_sync(FULL_MASK, inv_l, src);
+                const int qs = __shfl_sync(FULL_MASK, qpos, src);
+                float* rr = rows + ((size_t)b * r + (qs - (P - r))) * P;
+#pragma unroll 4
+                for (int key = lane; key < P; key += 32)
+                    rr[key] = key <= qs ? exp2f(rr[key] - ms) * il : 0.f;
             }
             if (out != nullptr) {
 #pragma unroll
