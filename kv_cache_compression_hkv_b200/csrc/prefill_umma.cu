@@ -136,7 +136,7 @@ struct Smem {
     __host__ __device__ static constexpr int kv_bytes(int d) { return KT * d * 2; }
     __host__ __device__ static constexpr int p_bytes() { return QT * KT * 2; }
     __host__ __device__ static constexpr int total(int d) {
-        return 1024 + q_bytes(d) + 4 * kv_bytes(d) + 2 * p_bytes() + B_COUNT * 8 + 16;
+        return 1024 + q_bytes(d) + 4 * kv_bytes(d) + 2 * p_bytes() + B_COUNT * 8 + 16 + QT * 8;
     }
 };
 
@@ -167,6 +167,7 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
     unsigned char* p_s = v_s + 2 * Smem::kv_bytes(D);   // [2]
     uint64_t* bars = reinterpret_cast<uint64_t*>(p_s + 2 * Smem::p_bytes());
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
+    float2* ml_s = reinterpret_cast<float2*>(tmem_slot + 4);  // [QT] kept rows' (max, 1 / sum)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // the query tiles of one (sequence, head) block are neighbours in the
@@ -381,19 +382,7 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
         if (!fail) {
             fence_after();
             const float inv_l = 1.0f / l;
-            // the kept rows' weights over every key, exactly normalised; the
-            // warp's lanes share each kept row's keys (coalesced, independent
-            // loads) instead of its own thread walking them one by one
-            for (unsigned keep = __ballot_sync(FULL_MASK, rrow != nullptr); keep; keep &= keep - 1) {
-                const int src = __ffs(keep) - 1;
-                const float ms = __shfl_sync(FULL_MASK, m, src);
-                const float il = __shfl_sync(FULL_MASK, inv_l, src);
-                const int qs = __shfl_sync(FULL_MASK, qpos, src);
-                float* rr = rows + ((size_t)b * r + (qs - (P - r))) * P;
-#pragma unroll 4
-                for (int key = lane; key < P; key += 32)
-                    rr[key] = key <= qs ? exp2f(rr[key] - ms) * il : 0.f;
-            }
+            if (rrow) ml_s[row] = make_float2(m, inv_l);  // normalised below, by the whole block
             if (out != nullptr) {
 #pragma unroll
                 for (int c0 = 0; c0 < D; c0 += 32) {
@@ -418,8 +407,42 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
             }
         }
     }
-    if (__syncthreads_or(fail) && tid == 0)
-        if (atomicCAS(status, 0, HKV_ERR_TIMEOUT) == 0) atomicExch(status + 1, b);
+    if (__syncthreads_or(fail)) {
+        if (tid == 0 && atomicCAS(status, 0, HKV_ERR_TIMEOUT) == 0) atomicExch(status + 1, b);
+    } else {
+        // The kept rows' weights over every key, exactly normalised: every
+        // thread of the block takes a share of the rows' keys (coalesced,
+        // independent loads of the logits the pass stored).  The kept rows
+        // of the tile are consecutive rows of `rows`.
+        const int k0 = max(q0, P - r), k1 = min(q0 + QT, P);
+        if (k0 < k1) {
+            float* kr0 = rows + ((size_t)b * r + (k0 - (P - r))) * P;
+            if ((P & 3) == 0) {
+                const int P4 = P >> 2, total = (k1 - k0) * P4;
+#pragma unroll 4
+                for (int e = tid; e < total; e += NTHREADS) {
+                    const int kr = e / P4, key = (e - kr * P4) * 4, qs = k0 + kr;
+                    const float2 mi = ml_s[qs - q0];
+                    float4* p4 = reinterpret_cast<float4*>(kr0 + (size_t)kr * P + key);
+                    float4 x4 = *p4;
+                    x4.x = key <= qs ? exp2f(x4.x - mi.x) * mi.y : 0.f;
+                    x4.y = key + 1 <= qs ? exp2f(x4.y - mi.x) * mi.y : 0.f;
+                    x4.z = key + 2 <= qs ? exp2f(x4.z - mi.x) * mi.y : 0.f;
+                    x4.w = key + 3 <= qs ? exp2f(x4.w - mi.x) * mi.y : 0.f;
+                    *p4 = x4;
+                }
+            } else {
+                const int total = (k1 - k0) * P;
+#pragma unroll 4
+                for (int e = tid; e < total; e += NTHREADS) {
+                    const int kr = e / P, key = e - kr * P, qs = k0 + kr;
+                    const float2 mi = ml_s[qs - q0];
+                    float* p1 = kr0 + (size_t)kr * P + key;
+                    *p1 = key <= qs ? exp2f(*p1 - mi.x) * mi.y : 0.f;
+                }
+            }
+        }
+    }
     fence_before();
     __syncthreads();
     fence_after();
