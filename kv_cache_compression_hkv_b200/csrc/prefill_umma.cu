@@ -5,7 +5,7 @@
 // One CTA (6 warps) per (sequence*head block, 128-query tile), one pass
 // over the key tiles (64 keys each, up to the tile's causal limit) with the
 // work split by role: a TMA warp brings the Q tile once and the K / V tiles
-// into two stages (128-byte swizzle, the layout the tensor cores read); an
+// into three stages (128-byte swizzle, the layout the tensor cores read); an
 // MMA warp issues S = Q K^T (M=128, N=64) into one of two TMEM slots and
 // O += P V (V as the MN-major operand) into a TMEM accumulator; four row
 // warps (thread i owns query row i = TMEM lane i) turn S into bf16 weights
@@ -118,31 +118,40 @@ constexpr int MMA_WARP = 5;
 // when a logit passes it by more than this: the weights stay below 2^8.
 constexpr float RESCALE = 8.f;
 
-// Barriers of the pipeline (two stages each, a stage per key-tile parity).
+// K / V tiles in flight: key tile j uses stage j % NKV.  (S slots in TMEM
+// and P tiles have two stages, j % 2.)  Three stages let the copies of
+// tile j + 2 start while tiles j and j + 1 are in the tensor cores and the
+// rows: with two, a stage came free only once P V of its tile was done,
+// and the copy's L2 latency sat in every other tile's critical path.
+constexpr int NKV = 3;
+
+// Barriers of the pipeline.
 enum Bar {
     B_Q = 0,
-    B_KFULL = 1,   // +stage: K tile landed
-    B_VFULL = 3,   // +stage: V tile landed
-    B_SFULL = 5,   // +stage: S = Q K^T of the stage's tile in TMEM
-    B_SFREE = 7,   // +stage: the softmax rows have read that S (128 arrivals)
-    B_PFULL = 9,   // +stage: P of the tile in shared memory, O rescaled (128 arrivals)
-    B_PVDONE = 11, // +stage: O += P V of the tile done: K, V and P of the stage free
-    B_COUNT = 13
+    B_KFULL = 1,                 // +kv stage: K tile landed
+    B_VFULL = B_KFULL + NKV,     // +kv stage: V tile landed
+    B_KVFREE = B_VFULL + NKV,    // +kv stage: P V of its tile done, K and V free
+    B_SFULL = B_KVFREE + NKV,    // +slot: S = Q K^T of the slot's tile in TMEM
+    B_SFREE = B_SFULL + 2,       // +slot: the softmax rows have read that S (128 arrivals)
+    B_PFULL = B_SFREE + 2,       // +p stage: P of the tile in shared memory, O rescaled (128 arrivals)
+    B_PVDONE = B_PFULL + 2,      // +p stage: O += P V of the tile done, P free
+    B_COUNT = B_PVDONE + 2
 };
 
 struct Smem {
-    // 1024-byte aligned tiles (128B swizzle atoms): Q, K[2], V[2], P[2]
+    // 1024-byte aligned tiles (128B swizzle atoms): Q, K[NKV], V[NKV], P[2]
     __host__ __device__ static constexpr int q_bytes(int d) { return QT * d * 2; }
     __host__ __device__ static constexpr int kv_bytes(int d) { return KT * d * 2; }
     __host__ __device__ static constexpr int p_bytes() { return QT * KT * 2; }
     __host__ __device__ static constexpr int total(int d) {
-        return 1024 + q_bytes(d) + 4 * kv_bytes(d) + 2 * p_bytes() + B_COUNT * 8 + 16 + QT * 8;
+        return 1024 + q_bytes(d) + 2 * NKV * kv_bytes(d) + 2 * p_bytes() + B_COUNT * 8 + 16 + QT * 8;
     }
 };
 
 // Causal attention of one (block, 128-query tile) in one pass over the key
-// tiles, pipelined over two stages:
-//   producer: K_j, V_j into stage j % 2 once O += P V of tile j-2 is done;
+// tiles, pipelined:
+//   producer: K_j, V_j into stage j % NKV once O += P V of tile j-NKV is
+//             done;
 //   MMA:      S_j = Q K_j^T into TMEM columns 64 (j % 2) (once the rows
 //             have read S_{j-2}), then O += P_{j-1} V_{j-1} into columns
 //             128.. (once the rows have written P_{j-1}), so the rows' work
@@ -153,7 +162,7 @@ struct Smem {
 //             stage j % 2 of P (once P_{j-2} V_{j-2} is done), running sum l.
 // Epilogue: O / l as bf16 rows; the last r rows' fp32 weights
 // exp2(s - m) / l over every key (their scaled logits were kept in `rows`
-// during the pass and are normalised in place).
+// during the pass and are normalised in place by the whole block).
 template <int D>
 __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
@@ -162,9 +171,9 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
     extern __shared__ unsigned char raw[];
     unsigned char* base = reinterpret_cast<unsigned char*>(((uintptr_t)raw + 1023) & ~(uintptr_t)1023);
     unsigned char* q_s = base;
-    unsigned char* k_s = q_s + Smem::q_bytes(D);        // [2] stages
-    unsigned char* v_s = k_s + 2 * Smem::kv_bytes(D);   // [2]
-    unsigned char* p_s = v_s + 2 * Smem::kv_bytes(D);   // [2]
+    unsigned char* k_s = q_s + Smem::q_bytes(D);          // [NKV] stages
+    unsigned char* v_s = k_s + NKV * Smem::kv_bytes(D);   // [NKV]
+    unsigned char* p_s = v_s + NKV * Smem::kv_bytes(D);   // [2]
     uint64_t* bars = reinterpret_cast<uint64_t*>(p_s + 2 * Smem::p_bytes());
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
     float2* ml_s = reinterpret_cast<float2*>(tmem_slot + 4);  // [QT] kept rows' (max, 1 / sum)
@@ -190,6 +199,7 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
     if (tid == 0) {
         for (int i = 0; i < B_COUNT; ++i) {
             const bool rows_arrive = (i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL || i == B_PFULL + 1);
+            // (every other barrier: one arrival, a copy's or a commit's)
             mbar_init(bars + i, rows_arrive ? QT : 1);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -202,15 +212,15 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
 
     if (warp == PRODUCER_WARP) {
         // --- TMA producer -------------------------------------------------
-        uint32_t issued = 0;  // bit s: stage s has a load that may be in flight
+        uint32_t issued = 0;    // bit s: kv stage s has a load that may be in flight
         uint32_t last_par = 0;  // bit s: parity of that load's phase
         if (lane == 0) {
             mbar_expect_tx(bars + B_Q, Smem::q_bytes(D));
             for (int sub = 0; sub < NSUB; ++sub)
                 tma_load_3d(q_s + sub * QT * 128, &qmap, bars + B_Q, sub * 64, q0, b);
             for (int j = 0; j < nkt && !fail; ++j) {
-                const int st = j & 1, k = j >> 1;
-                if (j >= 2 && !mbar_wait(bars + B_PVDONE + st, (k - 1) & 1, WAIT_NS)) { fail = true; break; }
+                const int st = j % NKV, u = j / NKV;
+                if (j >= NKV && !mbar_wait(bars + B_KVFREE + st, (u - 1) & 1, WAIT_NS)) { fail = true; break; }
                 mbar_expect_tx(bars + B_KFULL + st, KVB);
                 for (int sub = 0; sub < NSUB; ++sub)
                     tma_load_3d(k_s + st * KVB + sub * KT * 128, &kmap, bars + B_KFULL + st, sub * 64, j * KT, b);
@@ -218,12 +228,12 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
                 for (int sub = 0; sub < NSUB; ++sub)
                     tma_load_3d(v_s + st * KVB + sub * KT * 128, &vmap, bars + B_VFULL + st, sub * 64, j * KT, b);
                 issued |= 1u << st;
-                last_par = (last_par & ~(1u << st)) | ((uint32_t)(k & 1) << st);
+                last_par = (last_par & ~(1u << st)) | ((uint32_t)(u & 1) << st);
             }
             if (fail) {
                 // the block's own copies land before its shared memory goes
                 mbar_wait(bars + B_Q, 0, WAIT_NS);
-                for (int st = 0; st < 2; ++st)
+                for (int st = 0; st < NKV; ++st)
                     if (issued & (1u << st)) {
                         mbar_wait(bars + B_KFULL + st, (last_par >> st) & 1, WAIT_NS);
                         mbar_wait(bars + B_VFULL + st, (last_par >> st) & 1, WAIT_NS);
@@ -240,14 +250,15 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
             if (!mbar_wait(bars + B_Q, 0, WAIT_NS)) fail = true;
             for (int j = 0; j <= nkt && !fail; ++j) {
                 if (j < nkt) {
-                    const int st = j & 1, k = j >> 1;
-                    if (!mbar_wait(bars + B_KFULL + st, k & 1, WAIT_NS)) { fail = true; break; }
+                    const int st = j & 1, k = j >> 1;           // S slot
+                    const int kv = j % NKV, ku = j / NKV;       // K stage
+                    if (!mbar_wait(bars + B_KFULL + kv, ku & 1, WAIT_NS)) { fail = true; break; }
                     if (j >= 2 && !mbar_wait(bars + B_SFREE + st, (k - 1) & 1, WAIT_NS)) { fail = true; break; }
                     fence_after();
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t qa = smem_u32(q_s) + (kk / 4) * (QT * 128) + (kk % 4) * 32;
-                        const uint32_t ka = smem_u32(k_s + st * KVB) + (kk / 4) * (KT * 128) + (kk % 4) * 32;
+                        const uint32_t ka = smem_u32(k_s + kv * KVB) + (kk / 4) * (KT * 128) + (kk % 4) * 32;
                         mma_bf16(tmem + st * KT, sw128_desc(qa, 16, 1024), sw128_desc(ka, 16, 1024), IDESC_S,
                                  kk > 0);
                     }
@@ -255,27 +266,32 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
                     s_issued = j;
                 }
                 if (j >= 1) {
-                    const int jp = j - 1, sp = jp & 1, kp = jp >> 1;
+                    const int jp = j - 1, sp = jp & 1, kp = jp >> 1;  // P stage
+                    const int kv = jp % NKV, ku = jp / NKV;           // V stage
                     if (!mbar_wait(bars + B_PFULL + sp, kp & 1, WAIT_NS) ||
-                        !mbar_wait(bars + B_VFULL + sp, kp & 1, WAIT_NS)) { fail = true; break; }
+                        !mbar_wait(bars + B_VFULL + kv, ku & 1, WAIT_NS)) { fail = true; break; }
                     fence_after();
 #pragma unroll
                     for (int kk = 0; kk < KT / 16; ++kk) {
                         const uint32_t pa = smem_u32(p_s + sp * PB) + kk * 32;
-                        const uint32_t va = smem_u32(v_s + sp * KVB) + kk * 16 * 128;
+                        const uint32_t va = smem_u32(v_s + kv * KVB) + kk * 16 * 128;
                         mma_bf16(tmem + O_COL, sw128_desc(pa, 16, 1024), sw128_desc(va, KT * 128, 1024),
                                  IDESC_O, (jp > 0 || kk > 0));
                     }
                     mma_commit(bars + B_PVDONE + sp);
+                    mma_commit(bars + B_KVFREE + kv);
                     committed = jp;
                 }
             }
             // the tensor cores finish what was issued before TMEM is freed
-            // (a commit covers every MMA issued before it)
+            // (a commit covers every MMA issued before it), and the last
+            // commit's arrivals land before the shared memory goes
             if (s_issued > committed)
                 mbar_wait(bars + B_SFULL + (s_issued & 1), (s_issued >> 1) & 1, WAIT_NS);
-            else if (committed >= 0)
+            if (committed >= 0) {
                 mbar_wait(bars + B_PVDONE + (committed & 1), (committed >> 1) & 1, WAIT_NS);
+                mbar_wait(bars + B_KVFREE + committed % NKV, (committed / NKV) & 1, WAIT_NS);
+            }
         }
     } else {
         // --- rows: softmax and epilogue ------------------------------------
@@ -298,14 +314,20 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
             tmem_ld_wait();
             fence_before();
             mbar_arrive(bars + B_SFREE + st);
-            float x[KT];
-            float mt = -INFINITY;
+            // scaled logits and their maximum (eight independent chains and a
+            // tree: one warp per sub-partition has no other warp to hide a
+            // 64-long dependent chain behind)
+            float x[KT], mx[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
 #pragma unroll
             for (int c = 0; c < KT; ++c) {
                 const int key = j * KT + c;
                 x[c] = (key <= qpos && key < P) ? __uint_as_float(sr[c >> 5][c & 31]) * scale : -INFINITY;
-                mt = fmaxf(mt, x[c]);
+                mx[c & 7] = fmaxf(mx[c & 7], x[c]);
             }
+            const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
             if (rrow) {  // normalised in the epilogue
                 if ((P & 3) == 0) {  // 16-byte rows: whole float4 groups
 #pragma unroll
@@ -354,20 +376,24 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
                 fail = true;
                 break;
             }
+            // the weights as packed bf16 pairs (the sum over four chains),
+            // then the stores into the swizzled P tile
+            uint32_t w[KT / 2];
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int c2 = 0; c2 < KT / 2; ++c2) {
+                const float p0 = exp2f(x[2 * c2] - m), p1 = exp2f(x[2 * c2 + 1] - m);
+                ls[c2 & 3] += p0 + p1;
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                w[c2] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
             unsigned char* pst = p_s + st * PB;
 #pragma unroll
             for (int ch = 0; ch < KT / 8; ++ch) {
-                uint32_t w[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float p0 = exp2f(x[ch * 8 + 2 * e] - m), p1 = exp2f(x[ch * 8 + 2 * e + 1] - m);
-                    l += p0 + p1;
-                    __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                    w[e] = *reinterpret_cast<uint32_t*>(&h2);
-                }
                 const uint32_t off = row * 128 + ((ch ^ (row & 7)) << 4);
                 asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(pst) + off),
-                             "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                             "r"(w[4 * ch]), "r"(w[4 * ch + 1]), "r"(w[4 * ch + 2]), "r"(w[4 * ch + 3])
                              : "memory");
             }
             fence_proxy_async();
