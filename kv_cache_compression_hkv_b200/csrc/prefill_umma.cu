@@ -27,8 +27,7 @@ namespace umma {
 
 constexpr int QT = 128;   // query rows per CTA (MMA M)
 constexpr int KT = 64;    // keys per key tile (MMA N of S, K of P V)
-constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t O_COL = 128;  // O accumulator columns start here; S uses 0..63
+constexpr uint32_t O_COL = 128;  // O accumulators start here; S uses 0..127 (two slots)
 
 using ptx::smem_u32;
 using ptx::mbar_init;
@@ -108,12 +107,22 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Roles of the 192 threads of a CTA: warps 0-3 own the 128 query rows
-// (TMEM lane = row) and do the softmax and the epilogue; warp 4's lane 0
-// issues the TMA copies; warp 5's lane 0 issues the MMAs.
-constexpr int NTHREADS = 192;
-constexpr int PRODUCER_WARP = 4;
-constexpr int MMA_WARP = 5;
+// Roles of a CTA's warps: NH groups of four row warps own the 128 query
+// rows (TMEM lane = row; group g takes columns [g KT / NH, (g + 1) KT / NH)
+// of every S tile and has an O accumulator of its own) and do the softmax
+// and the epilogue; the next warp's lane 0 issues the TMA copies, the last
+// warp's lane 0 the MMAs.  d = 128 has two groups: its shared memory
+// allows one CTA per SM, and one row warp per SM sub-partition left the
+// softmax latency-bound (about 1.2 of the 1.4 us a key tile took); d = 64
+// has one group and two CTAs per SM.
+template <int D> struct Roles {
+    static constexpr int NH = D == 128 ? 2 : 1;
+    static constexpr int ROW_THREADS = 128 * NH;
+    static constexpr int PRODUCER_WARP = 4 * NH;
+    static constexpr int MMA_WARP = 4 * NH + 1;
+    static constexpr int NTHREADS = 32 * (4 * NH + 2);
+    static constexpr uint32_t TMEM_COLS = NH == 2 ? 512 : 256;  // S slots, then NH O accumulators
+};
 // A row's reference maximum (log2 domain) is raised, and O rescaled, only
 // when a logit passes it by more than this: the weights stay below 2^8.
 constexpr float RESCALE = 8.f;
@@ -132,10 +141,13 @@ enum Bar {
     B_VFULL = B_KFULL + NKV,     // +kv stage: V tile landed
     B_KVFREE = B_VFULL + NKV,    // +kv stage: P V of its tile done, K and V free
     B_SFULL = B_KVFREE + NKV,    // +slot: S = Q K^T of the slot's tile in TMEM
-    B_SFREE = B_SFULL + 2,       // +slot: the softmax rows have read that S (128 arrivals)
-    B_PFULL = B_SFREE + 2,       // +p stage: P of the tile in shared memory, O rescaled (128 arrivals)
-    B_PVDONE = B_PFULL + 2,      // +p stage: O += P V of the tile done, P free
-    B_COUNT = B_PVDONE + 2
+    B_SFREE = B_SFULL + 2,       // +slot: the row threads have read that S (ROW_THREADS arrivals)
+    B_PFULL = B_SFREE + 2,       // +2 group + p stage: the group's columns of P written, its O
+                                 // rescaled (128 arrivals)
+    B_PVDONE = B_PFULL + 4,      // +p stage: O += P V of the tile done, P free
+    B_XCH = B_PVDONE + 2,        // every row's (max, sum) of each group in shared memory
+                                 // (ROW_THREADS arrivals)
+    B_COUNT = B_XCH + 1
 };
 
 struct Smem {
@@ -144,7 +156,7 @@ struct Smem {
     __host__ __device__ static constexpr int kv_bytes(int d) { return KT * d * 2; }
     __host__ __device__ static constexpr int p_bytes() { return QT * KT * 2; }
     __host__ __device__ static constexpr int total(int d) {
-        return 1024 + q_bytes(d) + 2 * NKV * kv_bytes(d) + 2 * p_bytes() + B_COUNT * 8 + 16 + QT * 8;
+        return 1024 + q_bytes(d) + 2 * NKV * kv_bytes(d) + 2 * p_bytes() + B_COUNT * 8 + 16 + 3 * QT * 8;
     }
 };
 
@@ -164,7 +176,7 @@ struct Smem {
 // exp2(s - m) / l over every key (their scaled logits were kept in `rows`
 // during the pass and are normalised in place by the whole block).
 template <int D>
-__global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
+__global__ void __launch_bounds__(Roles<D>::NTHREADS) prefill_attn_umma(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
     const __grid_constant__ CUtensorMap vmap, int P, int r, __nv_bfloat16* __restrict__ out,
     float* __restrict__ rows, int32_t* __restrict__ status) {
@@ -177,6 +189,9 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
     uint64_t* bars = reinterpret_cast<uint64_t*>(p_s + 2 * Smem::p_bytes());
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
     float2* ml_s = reinterpret_cast<float2*>(tmem_slot + 4);  // [QT] kept rows' (max, 1 / sum)
+    float2* xch = ml_s + QT;                                  // [2][QT] groups' (max, sum)
+    using R = Roles<D>;
+    constexpr int NH = R::NH, CW = KT / NH;  // column groups, S columns per group
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // the query tiles of one (sequence, head) block are neighbours in the
@@ -193,14 +208,15 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tmem_slot)),
-                     "r"(TMEM_COLS));
+                     "r"(R::TMEM_COLS));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     if (tid == 0) {
         for (int i = 0; i < B_COUNT; ++i) {
-            const bool rows_arrive = (i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL || i == B_PFULL + 1);
-            // (every other barrier: one arrival, a copy's or a commit's)
-            mbar_init(bars + i, rows_arrive ? QT : 1);
+            // every other barrier: one arrival, a copy's or a commit's
+            const int n = (i == B_SFREE || i == B_SFREE + 1 || i == B_XCH) ? R::ROW_THREADS
+                          : (i >= B_PFULL && i < B_PFULL + 4) ? QT : 1;
+            mbar_init(bars + i, n);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -210,7 +226,7 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
     const uint32_t tmem = *tmem_slot;
     bool fail = false;
 
-    if (warp == PRODUCER_WARP) {
+    if (warp == R::PRODUCER_WARP) {
         // --- TMA producer -------------------------------------------------
         uint32_t issued = 0;    // bit s: kv stage s has a load that may be in flight
         uint32_t last_par = 0;  // bit s: parity of that load's phase
@@ -240,7 +256,7 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
                     }
             }
         }
-    } else if (warp == MMA_WARP) {
+    } else if (warp == R::MMA_WARP) {
         // --- MMA issuer ---------------------------------------------------
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16(KT, false);
@@ -268,19 +284,27 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
                 if (j >= 1) {
                     const int jp = j - 1, sp = jp & 1, kp = jp >> 1;  // P stage
                     const int kv = jp % NKV, ku = jp / NKV;           // V stage
-                    if (!mbar_wait(bars + B_PFULL + sp, kp & 1, WAIT_NS) ||
-                        !mbar_wait(bars + B_VFULL + kv, ku & 1, WAIT_NS)) { fail = true; break; }
-                    fence_after();
+                    if (!mbar_wait(bars + B_VFULL + kv, ku & 1, WAIT_NS)) { fail = true; break; }
+                    // group g's keys of the tile into its own O accumulator,
+                    // as soon as the group has written its columns of P
+                    bool ok = true;
 #pragma unroll
-                    for (int kk = 0; kk < KT / 16; ++kk) {
-                        const uint32_t pa = smem_u32(p_s + sp * PB) + kk * 32;
-                        const uint32_t va = smem_u32(v_s + kv * KVB) + kk * 16 * 128;
-                        mma_bf16(tmem + O_COL, sw128_desc(pa, 16, 1024), sw128_desc(va, KT * 128, 1024),
-                                 IDESC_O, (jp > 0 || kk > 0));
+                    for (int g = 0; g < NH; ++g) {
+                        if (!mbar_wait(bars + B_PFULL + 2 * g + sp, kp & 1, WAIT_NS)) { ok = false; break; }
+                        fence_after();
+#pragma unroll
+                        for (int kk = g * (CW / 16); kk < (g + 1) * (CW / 16); ++kk) {
+                            const uint32_t pa = smem_u32(p_s + sp * PB) + kk * 32;
+                            const uint32_t va = smem_u32(v_s + kv * KVB) + kk * 16 * 128;
+                            mma_bf16(tmem + O_COL + g * D, sw128_desc(pa, 16, 1024),
+                                     sw128_desc(va, KT * 128, 1024), IDESC_O, (jp > 0 || kk > g * (CW / 16)));
+                        }
                     }
+                    // (on a failed wait the commits still cover what was issued)
                     mma_commit(bars + B_PVDONE + sp);
                     mma_commit(bars + B_KVFREE + kv);
                     committed = jp;
+                    if (!ok) { fail = true; break; }
                 }
             }
             // the tensor cores finish what was issued before TMEM is freed
@@ -295,51 +319,55 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
         }
     } else {
         // --- rows: softmax and epilogue ------------------------------------
-        const int row = tid;  // query q0 + row, TMEM lane = row
+        const int grp = warp >> 2;             // column group
+        const int row = tid & (QT - 1);        // query q0 + row, TMEM lane = row
         const int qpos = q0 + row;
-        const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's lane quarter
+        const uint32_t t_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's lane quarter
+        const uint32_t o_col = O_COL + grp * D;  // the group's O accumulator
         const float scale = LOG2E / sqrtf((float)D);
         const bool keep_row = qpos >= P - r && qpos < P;
         float* rrow = keep_row ? rows + ((size_t)b * r + (qpos - (P - r))) * P : nullptr;
+        // m: the reference maximum of the row over the group's columns
+        // (-inf until one of them holds a key at or before the query)
         float m = -INFINITY, l = 0.f;
         // every branch around the warp-wide tcgen05.ld / tcgen05.st below is
         // taken by the whole warp: waits and decisions are warp votes
         for (int j = 0; j < nkt; ++j) {
             const int st = j & 1, k = j >> 1;
+            const int kb = j * KT + grp * CW;  // key of the group's first column
             if (__any_sync(FULL_MASK, !mbar_wait(bars + B_SFULL + st, k & 1, WAIT_NS))) { fail = true; break; }
             fence_after();
-            uint32_t sr[2][32];
-            tmem_ld32(t_row + st * KT, sr[0]);
-            tmem_ld32(t_row + st * KT + 32, sr[1]);
+            uint32_t sr[CW / 32][32];
+#pragma unroll
+            for (int u = 0; u < CW / 32; ++u) tmem_ld32(t_row + st * KT + grp * CW + u * 32, sr[u]);
             tmem_ld_wait();
             fence_before();
             mbar_arrive(bars + B_SFREE + st);
             // scaled logits and their maximum (eight independent chains and a
-            // tree: one warp per sub-partition has no other warp to hide a
-            // 64-long dependent chain behind)
-            float x[KT], mx[8];
+            // tree)
+            float x[CW], mx[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < KT; ++c) {
-                const int key = j * KT + c;
+            for (int c = 0; c < CW; ++c) {
+                const int key = kb + c;
                 x[c] = (key <= qpos && key < P) ? __uint_as_float(sr[c >> 5][c & 31]) * scale : -INFINITY;
                 mx[c & 7] = fmaxf(mx[c & 7], x[c]);
             }
             const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                    fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-            if (rrow) {  // normalised in the epilogue
+            if (rrow) {  // normalised after the pass
                 if ((P & 3) == 0) {  // 16-byte rows: whole float4 groups
 #pragma unroll
-                    for (int c = 0; c < KT; c += 4) {
-                        const int key = j * KT + c;
+                    for (int c = 0; c < CW; c += 4) {
+                        const int key = kb + c;
                         if (key < P)
                             *reinterpret_cast<float4*>(rrow + key) = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
                     }
                 } else {
 #pragma unroll
-                    for (int c = 0; c < KT; ++c) {
-                        const int key = j * KT + c;
+                    for (int c = 0; c < CW; ++c) {
+                        const int key = kb + c;
                         if (key < P) rrow[key] = x[c];
                     }
                 }
@@ -348,7 +376,7 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
                 // the warp raises its rows' references together (a row whose
                 // maximum did not grow keeps m: alpha = 1)
                 const float mn = fmaxf(m, mt);
-                const float alpha = mn == -INFINITY ? 1.f : exp2f(m - mn);  // 0 on the first tile
+                const float alpha = mn == -INFINITY ? 1.f : exp2f(m - mn);  // 0 while m is -inf
                 if (j > 0) {
                     // O holds P V up to tile j-1: rescale it once that is in
                     const int jp = j - 1;
@@ -360,11 +388,11 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
 #pragma unroll
                     for (int c0 = 0; c0 < D; c0 += 32) {
                         uint32_t o[32];
-                        tmem_ld32(t_row + O_COL + c0, o);
+                        tmem_ld32(t_row + o_col + c0, o);
                         tmem_ld_wait();
 #pragma unroll
                         for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st32(t_row + O_COL + c0, o);
+                        tmem_st32(t_row + o_col + c0, o);
                     }
                     tmem_st_wait();
                 }
@@ -377,12 +405,13 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
                 break;
             }
             // the weights as packed bf16 pairs (the sum over four chains),
-            // then the stores into the swizzled P tile
-            uint32_t w[KT / 2];
+            // then the stores into the group's chunks of the swizzled P tile
+            const float mb = m == -INFINITY ? 0.f : m;  // every logit is -inf then: weight 0
+            uint32_t w[CW / 2];
             float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c2 = 0; c2 < KT / 2; ++c2) {
-                const float p0 = exp2f(x[2 * c2] - m), p1 = exp2f(x[2 * c2 + 1] - m);
+            for (int c2 = 0; c2 < CW / 2; ++c2) {
+                const float p0 = exp2f(x[2 * c2] - mb), p1 = exp2f(x[2 * c2 + 1] - mb);
                 ls[c2 & 3] += p0 + p1;
                 __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
                 w[c2] = *reinterpret_cast<uint32_t*>(&h2);
@@ -390,31 +419,58 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
             l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
             unsigned char* pst = p_s + st * PB;
 #pragma unroll
-            for (int ch = 0; ch < KT / 8; ++ch) {
-                const uint32_t off = row * 128 + ((ch ^ (row & 7)) << 4);
+            for (int ch = 0; ch < CW / 8; ++ch) {
+                const int gch = grp * (CW / 8) + ch;  // 16-byte chunk of the 128-byte row
+                const uint32_t off = row * 128 + ((gch ^ (row & 7)) << 4);
                 asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(pst) + off),
                              "r"(w[4 * ch]), "r"(w[4 * ch + 1]), "r"(w[4 * ch + 2]), "r"(w[4 * ch + 3])
                              : "memory");
             }
             fence_proxy_async();
             fence_before();
-            mbar_arrive(bars + B_PFULL + st);
+            mbar_arrive(bars + B_PFULL + 2 * grp + st);
         }
         if (!fail && nkt > 0) {
             const int jl = nkt - 1;
             if (__any_sync(FULL_MASK, !mbar_wait(bars + B_PVDONE + (jl & 1), (jl >> 1) & 1, WAIT_NS)))
                 fail = true;
         }
+        // The row's maximum and sum over both groups (every row thread
+        // arrives once, even after a failed wait, so no wait here depends
+        // on a thread that left).
+        float M = m, fa = 1.f, fb = 0.f, Lsum = l;
+        if constexpr (NH == 2) {
+            xch[grp * QT + row] = make_float2(m, l);
+            mbar_arrive(bars + B_XCH);
+            if (!fail && __any_sync(FULL_MASK, !mbar_wait(bars + B_XCH, 0, WAIT_NS))) fail = true;
+            if (!fail) {
+                const float2 a = xch[row], c = xch[QT + row];  // group 0 holds key 0: a.x is finite
+                M = fmaxf(a.x, c.x);
+                fa = exp2f(a.x - M);
+                fb = c.x == -INFINITY ? 0.f : exp2f(c.x - M);
+                Lsum = a.y * fa + c.y * fb;
+            }
+        }
         if (!fail) {
             fence_after();
-            const float inv_l = 1.0f / l;
-            if (rrow) ml_s[row] = make_float2(m, inv_l);  // normalised below, by the whole block
+            const float inv_l = 1.0f / Lsum;
+            if (rrow && grp == 0) ml_s[row] = make_float2(M, inv_l);  // normalised below, by the whole block
             if (out != nullptr) {
+                // group g writes the output columns [g D / NH, (g + 1) D / NH)
 #pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
+                for (int c0 = grp * (D / NH); c0 < (grp + 1) * (D / NH); c0 += 32) {
                     uint32_t o[32];
                     tmem_ld32(t_row + O_COL + c0, o);
-                    tmem_ld_wait();
+                    if constexpr (NH == 2) {
+                        uint32_t o2[32];
+                        tmem_ld32(t_row + O_COL + D + c0, o2);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            o[e] = __float_as_uint(__uint_as_float(o[e]) * fa + __uint_as_float(o2[e]) * fb);
+                    } else {
+                        tmem_ld_wait();
+                    }
                     if (qpos < P) {
                         __nv_bfloat16* orow = out + ((size_t)b * P + qpos) * D + c0;
 #pragma unroll
@@ -446,7 +502,7 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
             if ((P & 3) == 0) {
                 const int P4 = P >> 2, total = (k1 - k0) * P4;
 #pragma unroll 4
-                for (int e = tid; e < total; e += NTHREADS) {
+                for (int e = tid; e < total; e += R::NTHREADS) {
                     const int kr = e / P4, key = (e - kr * P4) * 4, qs = k0 + kr;
                     const float2 mi = ml_s[qs - q0];
                     float4* p4 = reinterpret_cast<float4*>(kr0 + (size_t)kr * P + key);
@@ -460,7 +516,7 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
             } else {
                 const int total = (k1 - k0) * P;
 #pragma unroll 4
-                for (int e = tid; e < total; e += NTHREADS) {
+                for (int e = tid; e < total; e += R::NTHREADS) {
                     const int kr = e / P, key = e - kr * P, qs = k0 + kr;
                     const float2 mi = ml_s[qs - q0];
                     float* p1 = kr0 + (size_t)kr * P + key;
@@ -473,7 +529,7 @@ __global__ void __launch_bounds__(NTHREADS) prefill_attn_umma(
     __syncthreads();
     fence_after();
     if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(R::TMEM_COLS));
 }
 
 }  // namespace umma
@@ -526,10 +582,10 @@ cudaError_t launch_prefill_umma(const Layout& L, const void* q, const void* k, c
     dim3 grid((P + umma::QT - 1) / umma::QT, nblk);
     const size_t sm = umma::Smem::total(L.d);
     if (L.d == 128)
-        umma::prefill_attn_umma<128><<<grid, umma::NTHREADS, sm, st>>>(qm, km, vm, P, L.r, (__nv_bfloat16*)out,
+        umma::prefill_attn_umma<128><<<grid, umma::Roles<128>::NTHREADS, sm, st>>>(qm, km, vm, P, L.r, (__nv_bfloat16*)out,
                                                            L.rows, L.status);
     else
-        umma::prefill_attn_umma<64><<<grid, umma::NTHREADS, sm, st>>>(qm, km, vm, P, L.r, (__nv_bfloat16*)out,
+        umma::prefill_attn_umma<64><<<grid, umma::Roles<64>::NTHREADS, sm, st>>>(qm, km, vm, P, L.r, (__nv_bfloat16*)out,
                                                           L.rows, L.status);
     return cudaGetLastError();
 }
