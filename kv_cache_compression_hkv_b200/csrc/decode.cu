@@ -836,7 +836,7 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
     if (hint) {
         // L2 prefetch of the next layer's first chunks of this warp number
         const int4 nrec = shfl_int4(nblk, 0);
-        const int nc = min(min(nrec.y - nrec.x, nstage), PLAN_WARP_DESC);
+        const int nc = min(min(nrec.y - nrec.x, l2_hint == 1 ? nstage : l2_hint), PLAN_WARP_DESC);
         const size_t nrow = (size_t)(layer + 1) * L.S * L.R;
         for (int k = 0; k < nc; ++k) {
             const ChunkDesc c = ChunkDesc::of(shfl_int4(nblk, k + 1));
@@ -911,7 +911,8 @@ DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
     // Tuning overrides (read once per context): HKV_DECODE_WARPS caps the
     // warps per block, HKV_DECODE_STAGES fixes the stages per warp (1 ..
     // MAX_STAGES), HKV_DECODE_PROLOGUE sets DecodeShape::prologue (1 or 2),
-    // HKV_DECODE_L2_HINT=0 / =1 turns the next-layer L2 prefetch off / on,
+    // HKV_DECODE_L2_HINT=0 / =1 turns the next-layer L2 prefetch off / on
+    // (=k > 1: up to k chunks per warp instead of the stage count),
     // HKV_DECODE_HEAD_COST (1 .. 4 CHUNK_COST) sets DecodeShape::head_cost.
     const int es = L.dtype == HKV_DTYPE_F32 ? 4 : 2;
     const int max_w = env_int("HKV_DECODE_WARPS");
@@ -922,7 +923,8 @@ DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
     // the six of a d = 128 cache (Lumina-mGPT-768 shape: 25.04 against
     // 24.75 us): on when the block has 8 or more warps, unless overridden
     const char* hint_env = getenv("HKV_DECODE_L2_HINT");
-    const int hint_set = hint_env ? (hint_env[0] == '0' && hint_env[1] == 0 ? 0 : 1) : -1;
+    const int hint_val = hint_env ? atoi(hint_env) : 0;
+    const int hint_set = hint_env ? (hint_env[0] == '0' && hint_env[1] == 0 ? 0 : (hint_val > 1 ? hint_val : 1)) : -1;
     DecodeShape best{0, 0, 0, 1, pro <= 2 ? pro : 0, 0, HEAD_COST};
     for (int ns = fix_s == 1 ? 1 : 2; ns <= MAX_STAGES; ++ns) {
         if (fix_s && ns != fix_s) continue;

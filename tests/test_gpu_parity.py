@@ -414,6 +414,44 @@ def test_prefill_shapes_against_oracle(d, P):
                 assert ntau[s, h] == e_nt, (s, h)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_rescales_against_oracle(d):
+    """Logits that climb about 25 (log2) per 64-key tile along the keys, so
+    every row raises its reference maximum and rescales its O accumulator in
+    TMEM on every tile (and at d = 128 both column groups do, with the
+    second group's rows below key 32 starting from an empty maximum);
+    outputs and labels against the oracle."""
+    P, H = 300, 2
+    w = WORKLOADS["janus_pro_1b"].scaled(num_seqs=1, num_layers=1, num_heads=H, local_heads=1,
+                                          head_dim=d, prefix_len=1, prefill_image=P - 1,
+                                          image_tokens=P + 39, local_window=28)
+    cfg = hkv.config_for(w, mode=hkv.MODE_HEADKV)
+    g = torch.Generator().manual_seed(31 + d)
+    u = torch.ones(d) / d ** 0.5
+    slope = 0.4 / 1.4426950408889634  # per key, natural-log units of q.k / sqrt(d)
+    j = torch.arange(P, dtype=torch.float64)
+    q = u + 0.05 * torch.randn(1, H, P, d, generator=g)
+    k = (slope * j)[:, None] * u * d ** 0.5 + 0.05 * torch.randn(1, H, P, d, generator=g)
+    v = torch.randn(1, H, P, d, generator=g)
+    q, k, v = (x.to(torch.bfloat16).to(DEV).contiguous() for x in (q, k, v))
+    cache = hkv.HeadKVCache(cfg, device=DEV)
+    out = torch.empty(1, H, P, d, dtype=torch.bfloat16, device=DEV)
+    cache.prefill_classify(0, q, k, v, out=out)
+    lab, _ = cache.labels(0)
+    assert cache.check()[0] == 0
+    for h in range(H):
+        qq, kk, vv = (x[0, h].double().cpu().numpy() for x in (q, k, v))
+        o, p = O.causal_attention(qq, kk, vv)
+        # the logits do climb past the threshold within every tile
+        s_last = qq[-1] @ kk.T / d ** 0.5 * 1.4426950408889634
+        assert s_last[63] - s_last[0] > 16 and s_last[-1] - s_last[-65] > 16
+        got = out[0, h].double().cpu().numpy()
+        assert np.abs(got - o).max() / np.abs(o).max() < 2e-2, h
+        _, e_lab, cw = O.classify(p[-1], w.local_window, 0.9)
+        if abs(cw - 0.9) > 1e-5:
+            assert lab[0, h] == e_lab, (h, cw)
+
+
 def test_full_size_sampled_units():
     """The bench's workload at full size and launch configuration; two
     sampled units go through the oracle in lock step."""
