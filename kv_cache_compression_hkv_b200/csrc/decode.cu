@@ -978,7 +978,12 @@ cudaError_t launch_decode(const Layout& L, int layer, const void* q, const void*
 cudaError_t launch_plan(const Layout& L, int l0, int l1, int ahead, int commit, cudaStream_t st,
                         int after_evict) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(l1 - l0, PLAN_DESC_PARTS);
+    // blocks per layer: PLAN_DESC_PARTS, or HKV_PLAN_PARTS (1 .. 32; tuning)
+    static const int parts = [] {
+        const int v = env_int("HKV_PLAN_PARTS");
+        return v >= 1 && v <= 32 ? v : PLAN_DESC_PARTS;
+    }();
+    cfg.gridDim = dim3(l1 - l0, parts);
     cfg.blockDim = dim3(1024);
     cfg.dynamicSmemBytes = plan_smem_bytes(L.S * L.H, L.max_chunks);
     cfg.stream = st;

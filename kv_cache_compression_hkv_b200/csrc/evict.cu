@@ -9,6 +9,7 @@
 // strata by a block-wide threshold search, and compacts the cache in place
 // by moving the surviving tail tokens into the holes below the budget.
 #include <math.h>
+#include <stdlib.h>
 
 #include <mutex>
 
@@ -646,7 +647,13 @@ __host__ __device__ inline size_t evict_group_smem(int n_max, int M) {
 // SM.
 int evict_group_warps(const Layout& L) {
     const int64_t cap = L.T_total / (L.H_total > 0 ? L.H_total : L.H) + L.M;
-    int gw = 1;
+    // HKV_EVICT_WARPS (1, 2, 4 or 8) sets the least group size (tuning)
+    static const int least = [] {
+        const char* v = getenv("HKV_EVICT_WARPS");
+        const int x = v ? atoi(v) : 1;
+        return (x == 2 || x == 4 || x == 8) ? x : 1;
+    }();
+    int gw = least < EVB_WARPS ? least : EVB_WARPS;
     while (gw < EVB_WARPS && cap > 256 * gw) gw *= 2;
     while (gw < EVB_WARPS && (EVB_WARPS / gw) * evict_group_smem(L.L, L.M) > 100 * 1024) gw *= 2;
     return gw;
