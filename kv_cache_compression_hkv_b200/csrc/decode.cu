@@ -157,12 +157,35 @@ __device__ __forceinline__ int4 shfl_int4(const int4& v, int src) {
                      __shfl_sync(FULL_MASK, v.z, src), __shfl_sync(FULL_MASK, v.w, src));
 }
 
+// Warp ranges of equal cost over the chunk list (see plan_kernel): the
+// warps w whose boundary w * tcost / GWe falls in head i's cost interval
+// start in head i, at the first of its chunks whose cost starts at or
+// after the boundary.  U: an unsigned type that holds tcost * (GWe + 1).
+template <typename U>
+__device__ __forceinline__ void cut_ranges(const int32_t* cnt, int n, int HC, U tcost, int GWe,
+                                           int32_t* wbeg, int32_t* whead) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int c0 = i ? cnt[i - 1] : 0, c1 = cnt[i];
+        const U e0 = (U)CHUNK_COST * (U)c0 + (U)HC * (U)i;
+        const U e1 = (U)CHUNK_COST * (U)c1 + (U)HC * (U)(i + 1);
+        const int w_lo = (int)((e0 * (U)GWe + tcost - 1) / tcost);
+        const int w_hi = min((int)((e1 * (U)GWe + tcost - 1) / tcost), GWe);  // exclusive
+        for (int w = w_lo; w < w_hi; ++w) {
+            const U bnd = (U)w * tcost / (U)GWe;
+            // chunks of head i whose cost starts before the boundary
+            const int k = bnd > e0 ? (int)((bnd - e0 + CHUNK_COST - 1) / CHUNK_COST) : 0;
+            wbeg[w] = c0 + min(k, c1 - c0);
+            whead[w] = i;
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // The plan of a layer's decode launch at step t (ahead = 1: the step of the
 // next append, t_next; ahead = 0: the newest cached position, t_next - 1).
 // Blocks (layer, part): every block computes the layer's per-head facts,
 // the chunk-count prefix and the warp ranges in shared memory; part p then
-// writes the descriptors of the p-th slice of the heads and the records of
+// writes the descriptors of the p-th slice of the chunks and the records of
 // the p-th slice of the warps (each warp: its range and copies of the first
 // PLAN_WARP_DESC descriptors of its range).
 // ---------------------------------------------------------------------------
@@ -201,54 +224,43 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead,
     const int te = L.t_next[layer] - 1;  // newest cached position
     const int t = te + ahead;
     const size_t hbase = (size_t)layer * n;
-    if (commit) {
-        // heads evicted at te: length = budget from te on; due again M steps later
-        for (int i = tid; i < n; i += blockDim.x) {
-            const size_t hx = hbase + i;
-            const int cap = L.cap[hx];
-            const uint64_t b = L.base[hx];
-            int bl = base_len_of(b), bt = base_t_of(b);
-            if (L.label[hx] != 0 || L.mode == HKV_MODE_FULL) continue;
+    const bool complete = t >= L.L;  // the sequence is complete: no step left to plan
+    for (int i = tid; i < n; i += blockDim.x) {
+        const size_t hx = hbase + i;
+        const int cap = L.cap[hx];
+        const int lab = L.label[hx];
+        const uint64_t b = L.base[hx];
+        int bl = base_len_of(b), bt = base_t_of(b);
+        if (commit && lab == 0 && L.mode != HKV_MODE_FULL) {
+            // a head evicted at te: length = budget from te on (part 0 writes
+            // it; another part may read either pair: the same length), due
+            // again M steps later (written once per unit)
             if (bl + (te - bt) >= cap) {
                 bl = L.budget[hx];
                 bt = te;
                 if (part == 0) L.base[hx] = base_pack(bl, bt);
             }
-            const int s = i / L.H;
-            int4* ur = L.unit + (size_t)layer * L.S + s;
-            const uint32_t gm = (uint32_t)ur->y;
-            if (part == 0 && gm && (i % L.H) == __ffs(gm) - 1) ur->x = bt + (cap - bl);
-        }
-        __syncthreads();
-    }
-    if (t >= L.L) return;  // the sequence is complete: no step left to plan
-    for (int i = tid; i < n; i += blockDim.x) {
-        const size_t hx = hbase + i;
-        const int cap = L.cap[hx];
-        int len;
-        {
-            const uint64_t b = L.base[hx];
-            int bl = base_len_of(b), bt = base_t_of(b);
-            // part 0 may already have written the committed pair: either
-            // reading gives the same length
-            if (commit && L.label[hx] == 0 && L.mode != HKV_MODE_FULL && bl + (te - bt) >= cap) {
-                bl = L.budget[hx];
-                bt = te;
+            if (part == 0) {
+                int4* ur = L.unit + (size_t)layer * L.S + i / L.H;
+                const uint32_t gm = (uint32_t)ur->y;
+                if (gm && (i % L.H) == __ffs(gm) - 1) ur->x = bt + (cap - bl);
             }
-            len = bl + (t - bt);
-            if (L.label[hx] == 1 && len > cap) len = cap;
         }
+        if (complete) continue;
+        int len = bl + (t - bt);
+        if (lab == 1 && len > cap) len = cap;
         int c = (len + CHUNK - 1) / CHUNK;
         if (len > cap || len < 1) {
             if (part == 0) latch_error(L, HKV_ERR_CAPACITY, (int)hx);
             c = 0;
         }
-        const int jn = append_slot(L, hx, t, len);
-        hscore[i] = L.label[hx] == 0 && L.mode != HKV_MODE_FULL && len > cap - L.r;
+        const int jn = append_slot_of(lab, cap, t, len);
+        hscore[i] = lab == 0 && L.mode != HKV_MODE_FULL && len > cap - L.r;
         hslot[i] = (i / L.H) * L.R + L.off[hx];
         hlen[i] = (len << 16) | (jn & 0xffff);
         cnt[i] = c;
     }
+    if (complete) return;
     __syncthreads();
     // inclusive scan: contiguous runs per thread, then the warps
     const int per = (n + blockDim.x - 1) / blockDim.x;
@@ -295,19 +307,12 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead,
     const int64_t tcost = (int64_t)CHUNK_COST * total + (int64_t)HC * n;
     const int64_t mrc = min_range_cost(HC);
     const int GWe = (int)min((int64_t)GW, max((int64_t)1, (tcost + mrc - 1) / mrc));
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const int c0 = i ? cnt[i - 1] : 0, c1 = cnt[i];
-        const int64_t e0 = (int64_t)CHUNK_COST * c0 + (int64_t)HC * i;
-        const int64_t e1 = (int64_t)CHUNK_COST * c1 + (int64_t)HC * (i + 1);
-        const int w_lo = (int)((e0 * GWe + tcost - 1) / tcost);
-        const int w_hi = min((int)((e1 * GWe + tcost - 1) / tcost), GWe);  // exclusive
-        for (int w = w_lo; w < w_hi; ++w) {
-            const int64_t bnd = (int64_t)w * tcost / GWe;
-            const int k = (int)((bnd - e0 + CHUNK_COST - 1) / CHUNK_COST);
-            wbeg[w] = c0 + min(max(k, 0), c1 - c0);
-            whead[w] = i;
-        }
-    }
+    // (32-bit arithmetic whenever every product fits: the usual case, and
+    // 64-bit divisions cost several times more)
+    if ((uint64_t)tcost * (uint64_t)(GWe + 1) < (1ull << 32))
+        cut_ranges<uint32_t>(cnt, n, HC, (uint32_t)tcost, GWe, wbeg, whead);
+    else
+        cut_ranges<uint64_t>(cnt, n, HC, (uint64_t)tcost, GWe, wbeg, whead);
     for (int w = GWe + threadIdx.x; w <= GW; w += blockDim.x) wbeg[w] = total;  // idle warps
     __syncthreads();
     // A range starting a decode block moves to the nearer end of the head
@@ -336,29 +341,32 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead,
     constexpr int PB = 1 + PLAN_WARP_DESC;
     int4* dsc = L.plan_desc + (size_t)layer * L.max_chunks;
     int4* pw = L.plan_warp + (size_t)layer * PLAN_MAX_WARPS * PB;
-    const int h0 = (int)((int64_t)part * n / parts), h1 = (int)((int64_t)(part + 1) * n / parts);
-    for (int i = h0 + threadIdx.x; i < h1; i += blockDim.x) {
-        const int c1 = cnt[i], c0 = i ? cnt[i - 1] : 0;
-        if (c1 == c0) continue;
-        const int4 f = make_int4(hslot[i], hlen[i], hscore[i], 0);
-        const int wa = own[c0], wb = own[c1 - 1];
-        int segs = 0;
-        for (int w = wa; w <= wb; ++w) segs += wbeg[w] < wbeg[w + 1];
-        const int hw = wa | ((wb - wa) << 12);
-        const int len = f.y >> 16, jn = (int)(int16_t)(f.y & 0xffff);
-        int w = wa;  // the warp holding chunk c
-        for (int c = c0; c < c1; ++c) {
-            while (wbeg[w + 1] <= c) ++w;
-            const int k = c - c0;
-            const int tok0 = k * CHUNK;
-            const int nr = min(CHUNK, len - tok0);
-            const int a = jn - tok0;
-            const int z = nr | ((a >= 0 && a < nr ? a + 1 : 0) << 6) | ((k == 0) << 12) |
-                          ((c == c1 - 1) << 13) | (f.z << 14) | (segs << 16);
-            const int4 d = make_int4(f.x + tok0, i, z, hw);
-            dsc[c] = d;
-            if (c - wbeg[w] < PLAN_WARP_DESC) pw[PB * w + 1 + (c - wbeg[w])] = d;
+    // part p writes the descriptors of the p-th slice of the chunks, one
+    // chunk per thread (a head's chunks are spread over threads)
+    const int c_lo = (int)((int64_t)part * total / parts), c_hi = (int)((int64_t)(part + 1) * total / parts);
+    for (int c = c_lo + threadIdx.x; c < c_hi; c += blockDim.x) {
+        int i = 0;  // the head holding chunk c: the first with cnt[i] > c
+        for (int hi = n - 1; i < hi;) {
+            const int mid = (i + hi) >> 1;
+            if (cnt[mid] > c) hi = mid;
+            else i = mid + 1;
         }
+        const int c1 = cnt[i], c0 = i ? cnt[i - 1] : 0;
+        const int wa = own[c0], wb = own[c1 - 1], w = own[c];  // w: the warp holding chunk c
+        int segs = 0;
+        for (int u = wa; u <= wb; ++u) segs += wbeg[u] < wbeg[u + 1];
+        const int hw = wa | ((wb - wa) << 12);
+        const int hl = hlen[i];
+        const int len = hl >> 16, jn = (int)(int16_t)(hl & 0xffff);
+        const int k = c - c0;
+        const int tok0 = k * CHUNK;
+        const int nr = min(CHUNK, len - tok0);
+        const int a = jn - tok0;
+        const int z = nr | ((a >= 0 && a < nr ? a + 1 : 0) << 6) | ((k == 0) << 12) |
+                      ((c == c1 - 1) << 13) | (hscore[i] << 14) | (segs << 16);
+        const int4 d = make_int4(hslot[i] + tok0, i, z, hw);
+        dsc[c] = d;
+        if (c - wbeg[w] < PLAN_WARP_DESC) pw[PB * w + 1 + (c - wbeg[w])] = d;
     }
     const int w0 = (int)((int64_t)part * GW / parts), w1 = (int)((int64_t)(part + 1) * GW / parts);
     for (int w = w0 + threadIdx.x; w < w1; w += blockDim.x)

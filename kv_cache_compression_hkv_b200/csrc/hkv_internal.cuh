@@ -108,8 +108,11 @@ __device__ __forceinline__ int len_at(const Layout& L, size_t hi, int t) {
 }
 
 // Slot (within the head) that the token of position t occupies when appended.
+__device__ __forceinline__ int append_slot_of(int label, int cap, int t, int len_after) {
+    return label == 1 ? t % cap : len_after - 1;
+}
 __device__ __forceinline__ int append_slot(const Layout& L, size_t hi, int t, int len_after) {
-    return L.label[hi] == 1 ? t % L.cap[hi] : len_after - 1;
+    return append_slot_of(L.label[hi], L.cap[hi], t, len_after);
 }
 
 __device__ __forceinline__ void latch_error(const Layout& L, int code, int detail) {
