@@ -103,6 +103,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// 2^x by the SFU's approximation (PTX ex2.approx.ftz: relative error about
+// 2^-22, results below 2^-126 flushed to zero); the weights it makes are
+// rounded to bf16 right after.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -132,20 +140,23 @@ template <int D> struct Roles {
 // thousand.
 constexpr float RESCALE = 16.f;
 
-// K / V tiles in flight: key tile j uses stage j % NKV.  (S slots in TMEM
-// and P tiles have two stages, j % 2.)  Three stages let the copies of
-// tile j + 2 start while tiles j and j + 1 are in the tensor cores and the
-// rows: with two, a stage came free only once P V of its tile was done,
-// and the copy's L2 latency sat in every other tile's critical path.
-constexpr int NKV = 3;
+// K / V tiles in flight: key tile j uses stage j % nkv(d).  (S slots in
+// TMEM and P tiles have two stages, j % 2.)  With two, a stage came free only
+// once P V of its tile was done, and a copy's latency sat in every other
+// tile's critical path; three let the copies of tile j + 2 start while
+// tiles j and j + 1 are in the tensor cores and the rows, and at d = 128
+// (one CTA per SM, shared memory to spare) four cover the HBM latency of a
+// head's first query tile, whose K and V are not yet in L2.
+__host__ __device__ constexpr int nkv(int d) { return d == 128 ? 4 : 3; }
+constexpr int NKV_MAX = 4;
 
 // Barriers of the pipeline.
 enum Bar {
     B_Q = 0,
     B_KFULL = 1,                 // +kv stage: K tile landed
-    B_VFULL = B_KFULL + NKV,     // +kv stage: V tile landed
-    B_KVFREE = B_VFULL + NKV,    // +kv stage: P V of its tile done, K and V free
-    B_SFULL = B_KVFREE + NKV,    // +slot: S = Q K^T of the slot's tile in TMEM
+    B_VFULL = B_KFULL + NKV_MAX,   // +kv stage: V tile landed
+    B_KVFREE = B_VFULL + NKV_MAX,  // +kv stage: P V of its tile done, K and V free
+    B_SFULL = B_KVFREE + NKV_MAX,  // +slot: S = Q K^T of the slot's tile in TMEM
     B_SFREE = B_SFULL + 2,       // +slot: the row threads have read that S (ROW_THREADS arrivals)
     B_PFULL = B_SFREE + 2,       // +2 group + p stage: the group's columns of P written, its O
                                  // rescaled (128 arrivals)
@@ -156,12 +167,12 @@ enum Bar {
 };
 
 struct Smem {
-    // 1024-byte aligned tiles (128B swizzle atoms): Q, K[NKV], V[NKV], P[2]
+    // 1024-byte aligned tiles (128B swizzle atoms): Q, K[nkv], V[nkv], P[2]
     __host__ __device__ static constexpr int q_bytes(int d) { return QT * d * 2; }
     __host__ __device__ static constexpr int kv_bytes(int d) { return KT * d * 2; }
     __host__ __device__ static constexpr int p_bytes() { return QT * KT * 2; }
     __host__ __device__ static constexpr int total(int d) {
-        return 1024 + q_bytes(d) + 2 * NKV * kv_bytes(d) + 2 * p_bytes() + B_COUNT * 8 + 16 + 3 * QT * 8;
+        return 1024 + q_bytes(d) + 2 * nkv(d) * kv_bytes(d) + 2 * p_bytes() + B_COUNT * 8 + 16 + 3 * QT * 8;
     }
 };
 
@@ -188,6 +199,7 @@ __global__ void __launch_bounds__(Roles<D>::NTHREADS) prefill_attn_umma(
     extern __shared__ unsigned char raw[];
     unsigned char* base = reinterpret_cast<unsigned char*>(((uintptr_t)raw + 1023) & ~(uintptr_t)1023);
     unsigned char* q_s = base;
+    constexpr int NKV = nkv(D);
     unsigned char* k_s = q_s + Smem::q_bytes(D);          // [NKV] stages
     unsigned char* v_s = k_s + NKV * Smem::kv_bytes(D);   // [NKV]
     unsigned char* p_s = v_s + NKV * Smem::kv_bytes(D);   // [2]
@@ -350,14 +362,26 @@ __global__ void __launch_bounds__(Roles<D>::NTHREADS) prefill_attn_umma(
             mbar_arrive(bars + B_SFREE + st);
             // scaled logits and their maximum (eight independent chains and a
             // tree)
+            // (no per-key test where every key of the group's slice is at or
+            // before every query of the warp and inside P: all but the
+            // diagonal tiles)
+            const bool whole = kb + CW - 1 <= q0 + (warp & 3) * 32 && kb + CW <= P;
             float x[CW], mx[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
+            if (whole) {
 #pragma unroll
-            for (int c = 0; c < CW; ++c) {
-                const int key = kb + c;
-                x[c] = (key <= qpos && key < P) ? __uint_as_float(sr[c >> 5][c & 31]) * scale : -INFINITY;
-                mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+                for (int c = 0; c < CW; ++c) {
+                    x[c] = __uint_as_float(sr[c >> 5][c & 31]) * scale;
+                    mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < CW; ++c) {
+                    const int key = kb + c;
+                    x[c] = (key <= qpos && key < P) ? __uint_as_float(sr[c >> 5][c & 31]) * scale : -INFINITY;
+                    mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+                }
             }
             const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                    fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
@@ -416,7 +440,7 @@ __global__ void __launch_bounds__(Roles<D>::NTHREADS) prefill_attn_umma(
             float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c2 = 0; c2 < CW / 2; ++c2) {
-                const float p0 = exp2f(x[2 * c2] - mb), p1 = exp2f(x[2 * c2 + 1] - mb);
+                const float p0 = ex2_approx(x[2 * c2] - mb), p1 = ex2_approx(x[2 * c2 + 1] - mb);
                 ls[c2 & 3] += p0 + p1;
                 __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
                 w[c2] = *reinterpret_cast<uint32_t*>(&h2);
