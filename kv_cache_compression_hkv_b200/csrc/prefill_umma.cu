@@ -2,17 +2,19 @@
 // cores (tcgen05) for bf16 caches (HeadKV technical summary, Methodology
 // step 1, cache prefilling: its weights feed step 2, head grouping).
 //
-// One CTA (6 warps) per (sequence*head block, 128-query tile), one pass
-// over the key tiles (64 keys each, up to the tile's causal limit) with the
-// work split by role: a TMA warp brings the Q tile once and the K / V tiles
-// into three stages (128-byte swizzle, the layout the tensor cores read); an
+// One CTA per (sequence*head block, 128-query tile), one pass over the key
+// tiles (64 keys each, up to the tile's causal limit) with the work split
+// by role: a TMA warp brings the Q tile once and the K / V tiles into three
+// or four stages (128-byte swizzle, the layout the tensor cores read); an
 // MMA warp issues S = Q K^T (M=128, N=64) into one of two TMEM slots and
-// O += P V (V as the MN-major operand) into a TMEM accumulator; four row
-// warps (thread i owns query row i = TMEM lane i) turn S into bf16 weights
-// P with an online maximum and sum.  The tensor cores work on tiles j and
-// j-1 while the rows work on tile j.  The epilogue reads O from TMEM and
-// stores bf16 rows, and normalises the fp32 weights of the last r query
-// rows over every key for the grouping.  Every wait on an mbarrier is
+// O += P V (V as the MN-major operand) into TMEM accumulators; one or two
+// groups of four row warps (thread i of a group owns query row i = TMEM
+// lane i; a group takes its share of every S tile's columns and has its
+// own O) turn S into bf16 weights P with an online maximum and sum.  The
+// tensor cores work on tiles j and j-1 while the rows work on tile j.  The
+// epilogue combines the groups, reads O from TMEM and stores bf16 rows, and
+// the whole block normalises the fp32 weights of the last r query rows over
+// every key for the grouping.  Every wait on an mbarrier is
 // bounded in time; a wait that gives up latches HKV_ERR_TIMEOUT, the block
 // waits (bounded) for its own copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -181,16 +183,19 @@ struct Smem {
 //   producer: K_j, V_j into stage j % NKV once O += P V of tile j-NKV is
 //             done;
 //   MMA:      S_j = Q K_j^T into TMEM columns 64 (j % 2) (once the rows
-//             have read S_{j-2}), then O += P_{j-1} V_{j-1} into columns
-//             128.. (once the rows have written P_{j-1}), so the rows' work
-//             on tile j overlaps the tensor cores' work on tiles j and j-1;
-//   rows:     read S_j, raise the reference maximum m only when a logit
-//             passes it by more than RESCALE (then O, once P_{j-1} V_{j-1}
-//             is in, is rescaled in TMEM), P_j = exp2(S_j - m) as bf16 into
-//             stage j % 2 of P (once P_{j-2} V_{j-2} is done), running sum l.
-// Epilogue: O / l as bf16 rows; the last r rows' fp32 weights
-// exp2(s - m) / l over every key (their scaled logits were kept in `rows`
-// during the pass and are normalised in place by the whole block).
+//             have read S_{j-2}), then, group by group, O_g += P_{j-1} V_{j-1}
+//             over the group's keys into its columns 128 + g d .. (once the
+//             group has written its part of P_{j-1}), so the rows' work on
+//             tile j overlaps the tensor cores' work on tiles j and j-1;
+//   rows:     read their columns of S_j, raise the reference maximum m only
+//             when a logit passes it by more than RESCALE (then O_g, once
+//             P_{j-1} V_{j-1} is in, is rescaled in TMEM), P_j = exp2(S_j - m)
+//             as bf16 into stage j % 2 of P (once P_{j-2} V_{j-2} is done),
+//             running sum l.
+// Epilogue: per row, M = max of the groups' m and O = sum of O_g 2^(m_g - M)
+// over L = sum of l_g 2^(m_g - M), as bf16 rows; the last r rows' fp32
+// weights exp2(s - M) / L over every key (their scaled logits were kept in
+// `rows` during the pass and are normalised in place by the whole block).
 template <int D>
 __global__ void __launch_bounds__(Roles<D>::NTHREADS) prefill_attn_umma(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
