@@ -157,10 +157,11 @@ __device__ __forceinline__ int4 shfl_int4(const int4& v, int src) {
                      __shfl_sync(FULL_MASK, v.z, src), __shfl_sync(FULL_MASK, v.w, src));
 }
 
-// Warp ranges of equal cost over the chunk list (see plan_kernel): the
-// warps w whose boundary w * tcost / GWe falls in head i's cost interval
-// start in head i, at the first of its chunks whose cost starts at or
-// after the boundary.  U: an unsigned type that holds tcost * (GWe + 1).
+// Warp ranges over the chunk list (see plan_kernel): the warps w whose
+// boundary falls in head i's cost interval start in head i, at the first of
+// its chunks whose cost starts at or after the boundary.  Equal shares: the
+// boundary of warp w is w * tcost / GWe.  U: an unsigned type that holds
+// tcost * (GWe + 1).
 template <typename U>
 __device__ __forceinline__ void cut_ranges(const int32_t* cnt, int n, int HC, U tcost, int GWe,
                                            int32_t* wbeg, int32_t* whead) {
@@ -176,6 +177,40 @@ __device__ __forceinline__ void cut_ranges(const int32_t* cnt, int n, int HC, U 
             const int k = bnd > e0 ? (int)((bnd - e0 + CHUNK_COST - 1) / CHUNK_COST) : 0;
             wbeg[w] = c0 + min(k, c1 - c0);
             whead[w] = i;
+        }
+    }
+}
+
+// Weighted shares: warp k of a block (NW warps) weighs wt[k]; warp w =
+// b NW + k starts at unit u(w) = b S + pre[k] of U = (GW / NW) S units
+// (S = the block's total weight, pre = the prefix of wt), i.e. at cost
+// u(w) tcost / U.  The heads' cost intervals, scaled to units, cut [0, U)
+// into consecutive pieces, so every warp gets exactly one start.
+__device__ __forceinline__ void cut_ranges_weighted(const int32_t* cnt, int n, int HC, uint64_t tcost,
+                                                    int GW, int NW, const int* pre, int32_t* wbeg,
+                                                    int32_t* whead) {
+    const int S = pre[NW];
+    const uint64_t U = (uint64_t)(GW / NW) * S;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int c0 = i ? cnt[i - 1] : 0, c1 = cnt[i];
+        const uint64_t e0 = (uint64_t)CHUNK_COST * c0 + (uint64_t)HC * i;
+        const uint64_t e1 = (uint64_t)CHUNK_COST * c1 + (uint64_t)HC * (i + 1);
+        const uint64_t x_lo = (e0 * U + tcost - 1) / tcost;  // first unit whose cost is >= e0
+        const uint64_t x_hi = min((e1 * U + tcost - 1) / tcost, U);
+        if (x_lo >= x_hi) continue;
+        int b = (int)(x_lo / S), k = 0;
+        const int r = (int)(x_lo - (uint64_t)b * S);
+        while (k < NW && pre[k] < r) ++k;
+        if (k == NW) { ++b; k = 0; }
+        for (;;) {
+            const uint64_t u = (uint64_t)b * S + pre[k];
+            if (u >= x_hi) break;
+            const int w = b * NW + k;
+            const uint64_t bnd = u * tcost / U;
+            const int kk = bnd > e0 ? (int)((bnd - e0 + CHUNK_COST - 1) / CHUNK_COST) : 0;
+            wbeg[w] = c0 + min(kk, c1 - c0);
+            whead[w] = i;
+            if (++k == NW) { ++b; k = 0; }
         }
     }
 }
@@ -307,9 +342,28 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead,
     const int64_t tcost = (int64_t)CHUNK_COST * total + (int64_t)HC * n;
     const int64_t mrc = min_range_cost(HC);
     const int GWe = (int)min((int64_t)GW, max((int64_t)1, (tcost + mrc - 1) / mrc));
-    // (32-bit arithmetic whenever every product fits: the usual case, and
-    // 64-bit divisions cost several times more)
-    if ((uint64_t)tcost * (uint64_t)(GWe + 1) < (1ull << 32))
+    // A full grid whose blocks load the SM's sub-partitions unevenly weighs
+    // its warps (LONE_WEIGHT / SHARED_WEIGHT); otherwise equal shares, in
+    // 32-bit arithmetic whenever every product fits (the usual case: 64-bit
+    // divisions cost several times more).
+    int pre[DECODE_MAX_WARPS + 1];
+    bool weighted = false;
+    {
+        const int NWb = L.plan_nw;
+        if (GWe == GW && NWb > 0 && NWb <= DECODE_MAX_WARPS && GW % NWb == 0 && L.plan_lw != SHARED_WEIGHT) {
+            int per[4] = {0, 0, 0, 0}, top = 0;
+            for (int k = 0; k < NWb; ++k) ++per[k & 3];
+            for (int q = 0; q < 4; ++q) top = max(top, per[q]);
+            pre[0] = 0;
+            for (int k = 0; k < NWb; ++k) {
+                pre[k + 1] = pre[k] + (per[k & 3] < top ? L.plan_lw : SHARED_WEIGHT);
+                weighted |= per[k & 3] < top;
+            }
+        }
+    }
+    if (weighted)
+        cut_ranges_weighted(cnt, n, HC, (uint64_t)tcost, GW, L.plan_nw, pre, wbeg, whead);
+    else if ((uint64_t)tcost * (uint64_t)(GWe + 1) < (1ull << 32))
         cut_ranges<uint32_t>(cnt, n, HC, (uint32_t)tcost, GWe, wbeg, whead);
     else
         cut_ranges<uint64_t>(cnt, n, HC, (uint64_t)tcost, GWe, wbeg, whead);
@@ -921,7 +975,9 @@ DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
     // MAX_STAGES), HKV_DECODE_PROLOGUE sets DecodeShape::prologue (1 or 2),
     // HKV_DECODE_L2_HINT=0 / =1 turns the next-layer L2 prefetch off / on
     // (=k > 1: up to k chunks per warp instead of the stage count),
-    // HKV_DECODE_HEAD_COST (1 .. 4 CHUNK_COST) sets DecodeShape::head_cost.
+    // HKV_DECODE_HEAD_COST (1 .. 4 CHUNK_COST) sets DecodeShape::head_cost,
+    // HKV_DECODE_LONE_WEIGHT (SHARED_WEIGHT .. 2 SHARED_WEIGHT; SHARED_WEIGHT:
+    // equal shares) DecodeShape::lone_weight.
     const int es = L.dtype == HKV_DTYPE_F32 ? 4 : 2;
     const int max_w = env_int("HKV_DECODE_WARPS");
     const int fix_s = env_int("HKV_DECODE_STAGES");
@@ -945,6 +1001,9 @@ DecodeShape decode_shape(const Layout& L, size_t smem_limit) {
             best = DecodeShape{w, ns, 1024 + (size_t)w * per, 1, best.prologue, 0, HEAD_COST};
     }
     best.l2_hint = hint_set >= 0 ? hint_set : (best.warps >= 8 ? 1 : 0);
+    best.lone_weight = LONE_WEIGHT;
+    const int lw = env_int("HKV_DECODE_LONE_WEIGHT");
+    if (lw >= SHARED_WEIGHT && lw <= 2 * SHARED_WEIGHT) best.lone_weight = lw;
     const int hc = env_int("HKV_DECODE_HEAD_COST");
     if (hc > 0 && hc <= 4 * CHUNK_COST) best.head_cost = hc;
     return best;

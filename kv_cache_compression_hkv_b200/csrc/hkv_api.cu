@@ -254,6 +254,7 @@ hkv_status hkv_create(const hkv_config* cfg, void* pool, size_t bytes, void* str
     c->lay.plan_gw = c->decode_grid * c->decode_sh.warps;
     c->lay.plan_nw = c->decode_sh.warps;
     c->lay.plan_hc = c->decode_sh.head_cost;
+    c->lay.plan_lw = c->decode_sh.lone_weight;
     c->plan_for.assign(cfg->num_layers, -1);
     c->evict_grid = c->n_sm * hkv::evict_blocks_per_sm(c->lay, optin);
     *out = c;

@@ -29,6 +29,15 @@ constexpr int HEAD_COST = 5;
 // Least cost of a warp's range (two chunks of one head): small layers use
 // fewer warps rather than thinner ranges, and a small cache fewer blocks.
 __host__ __device__ constexpr int min_range_cost(int head_cost) { return 2 * CHUNK_COST + head_cost; }
+// Weights of a decode warp's share of a layer when a block's warps do not
+// spread evenly over the SM's four sub-partitions (six warps: two share
+// each of sub-partitions 0 and 1, two are alone on 2 and 3).  Per-warp
+// timestamps of the decode launch on a d = 128 cache: 2.14 us per chunk
+// for a warp alone, 2.33 for one that shares (about 12 : 11); launch times
+// on the Lumina-mGPT-768 shape: 22.68 / 22.48 / 22.36 / 22.39 us at 11 /
+// 12 / 13 / 14 against 11 (13 counts the warp's share of the block's end).
+constexpr int SHARED_WEIGHT = 11;
+constexpr int LONE_WEIGHT = 13;
 
 // Everything a kernel needs to find the state of a (layer, sequence, head).
 // The pool is one caller-owned device buffer carved into these regions.
@@ -82,6 +91,8 @@ struct Layout {
     int32_t plan_gw;     // warps of one decode launch
     int32_t plan_nw;     // warps of one decode block
     int32_t plan_hc;     // cost of a head's end in the plan's balancing
+    int32_t plan_lw;     // weight of a warp alone on its SM sub-partition
+                         // (the others weigh SHARED_WEIGHT) in the plan
     int32_t max_chunks;
 };
 

@@ -40,6 +40,7 @@ struct DecodeShape {
                    // 1 one; 2 all
     int l2_hint;   // 1: finished warps prefetch the next layer's first chunks into L2
     int head_cost; // cost of a head's end in the plan's balancing (CHUNK_COST per chunk)
+    int lone_weight;  // plan weight of a warp alone on its SM sub-partition
 };
 DecodeShape decode_shape(const Layout& L, size_t smem_limit);
 // early: the previous launch in `st` is a decode launch of another layer (the
