@@ -185,28 +185,29 @@ __device__ __forceinline__ void cut_ranges(const int32_t* cnt, int n, int HC, U 
 // b NW + k starts at unit u(w) = b S + pre[k] of U = (GW / NW) S units
 // (S = the block's total weight, pre = the prefix of wt), i.e. at cost
 // u(w) tcost / U.  The heads' cost intervals, scaled to units, cut [0, U)
-// into consecutive pieces, so every warp gets exactly one start.
-__device__ __forceinline__ void cut_ranges_weighted(const int32_t* cnt, int n, int HC, uint64_t tcost,
-                                                    int GW, int NW, const int* pre, int32_t* wbeg,
+// into consecutive pieces, so every warp gets exactly one start.  V: an
+// unsigned type that holds tcost * (U + 1).
+template <typename V>
+__device__ __forceinline__ void cut_ranges_weighted(const int32_t* cnt, int n, int HC, V tcost, V U,
+                                                    int NW, const int* pre, int32_t* wbeg,
                                                     int32_t* whead) {
     const int S = pre[NW];
-    const uint64_t U = (uint64_t)(GW / NW) * S;
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
         const int c0 = i ? cnt[i - 1] : 0, c1 = cnt[i];
-        const uint64_t e0 = (uint64_t)CHUNK_COST * c0 + (uint64_t)HC * i;
-        const uint64_t e1 = (uint64_t)CHUNK_COST * c1 + (uint64_t)HC * (i + 1);
-        const uint64_t x_lo = (e0 * U + tcost - 1) / tcost;  // first unit whose cost is >= e0
-        const uint64_t x_hi = min((e1 * U + tcost - 1) / tcost, U);
+        const V e0 = (V)CHUNK_COST * (V)c0 + (V)HC * (V)i;
+        const V e1 = (V)CHUNK_COST * (V)c1 + (V)HC * (V)(i + 1);
+        const V x_lo = (e0 * U + tcost - 1) / tcost;  // first unit whose cost is >= e0
+        const V x_hi = min((e1 * U + tcost - 1) / tcost, U);
         if (x_lo >= x_hi) continue;
-        int b = (int)(x_lo / S), k = 0;
-        const int r = (int)(x_lo - (uint64_t)b * S);
+        int b = (int)(x_lo / (V)S), k = 0;
+        const int r = (int)(x_lo - (V)b * (V)S);
         while (k < NW && pre[k] < r) ++k;
         if (k == NW) { ++b; k = 0; }
         for (;;) {
-            const uint64_t u = (uint64_t)b * S + pre[k];
+            const V u = (V)b * (V)S + (V)pre[k];
             if (u >= x_hi) break;
             const int w = b * NW + k;
-            const uint64_t bnd = u * tcost / U;
+            const V bnd = u * tcost / U;
             const int kk = bnd > e0 ? (int)((bnd - e0 + CHUNK_COST - 1) / CHUNK_COST) : 0;
             wbeg[w] = c0 + min(kk, c1 - c0);
             whead[w] = i;
@@ -361,9 +362,13 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead,
             }
         }
     }
-    if (weighted)
-        cut_ranges_weighted(cnt, n, HC, (uint64_t)tcost, GW, L.plan_nw, pre, wbeg, whead);
-    else if ((uint64_t)tcost * (uint64_t)(GWe + 1) < (1ull << 32))
+    if (weighted) {
+        const uint64_t U = (uint64_t)(GW / L.plan_nw) * pre[L.plan_nw];
+        if ((uint64_t)tcost * (U + 1) < (1ull << 32))
+            cut_ranges_weighted<uint32_t>(cnt, n, HC, (uint32_t)tcost, (uint32_t)U, L.plan_nw, pre, wbeg, whead);
+        else
+            cut_ranges_weighted<uint64_t>(cnt, n, HC, (uint64_t)tcost, U, L.plan_nw, pre, wbeg, whead);
+    } else if ((uint64_t)tcost * (uint64_t)(GWe + 1) < (1ull << 32))
         cut_ranges<uint32_t>(cnt, n, HC, (uint32_t)tcost, GWe, wbeg, whead);
     else
         cut_ranges<uint64_t>(cnt, n, HC, (uint64_t)tcost, GWe, wbeg, whead);
