@@ -250,6 +250,18 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead,
     uint16_t* own = reinterpret_cast<uint16_t*>(whead + PLAN_MAX_WARPS);  // [total] warp of each chunk
     const int parts = gridDim.y, part = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, NW = blockDim.x >> 5;
+    // per-warp weights of a decode block (see the range cutting below)
+    __shared__ int pre[DECODE_MAX_WARPS + 1];
+    const int NWb = L.plan_nw;
+    const bool uneven = NWb > 0 && NWb <= DECODE_MAX_WARPS && L.plan_gw % NWb == 0 &&
+                        L.plan_lw != SHARED_WEIGHT && NWb >= 4 && NWb % 4 != 0;
+    if (tid == 0 && uneven) {
+        int per[4] = {0, 0, 0, 0}, top = 0;
+        for (int k = 0; k < NWb; ++k) ++per[k & 3];
+        for (int q = 0; q < 4; ++q) top = max(top, per[q]);
+        pre[0] = 0;
+        for (int k = 0; k < NWb; ++k) pre[k + 1] = pre[k] + (per[k & 3] < top ? L.plan_lw : SHARED_WEIGHT);
+    }
     // block (0, 0) completes only after the eviction kernel ahead of it
     struct AfterEvict {
         bool on;
@@ -344,24 +356,10 @@ __global__ void __launch_bounds__(1024) plan_kernel(Layout L, int l0, int ahead,
     const int64_t mrc = min_range_cost(HC);
     const int GWe = (int)min((int64_t)GW, max((int64_t)1, (tcost + mrc - 1) / mrc));
     // A full grid whose blocks load the SM's sub-partitions unevenly weighs
-    // its warps (LONE_WEIGHT / SHARED_WEIGHT); otherwise equal shares, in
-    // 32-bit arithmetic whenever every product fits (the usual case: 64-bit
-    // divisions cost several times more).
-    int pre[DECODE_MAX_WARPS + 1];
-    bool weighted = false;
-    {
-        const int NWb = L.plan_nw;
-        if (GWe == GW && NWb > 0 && NWb <= DECODE_MAX_WARPS && GW % NWb == 0 && L.plan_lw != SHARED_WEIGHT) {
-            int per[4] = {0, 0, 0, 0}, top = 0;
-            for (int k = 0; k < NWb; ++k) ++per[k & 3];
-            for (int q = 0; q < 4; ++q) top = max(top, per[q]);
-            pre[0] = 0;
-            for (int k = 0; k < NWb; ++k) {
-                pre[k + 1] = pre[k] + (per[k & 3] < top ? L.plan_lw : SHARED_WEIGHT);
-                weighted |= per[k & 3] < top;
-            }
-        }
-    }
+    // its warps (the prefix `pre` of LONE_WEIGHT / SHARED_WEIGHT, made at the
+    // start); otherwise equal shares, in 32-bit arithmetic whenever every
+    // product fits (the usual case: 64-bit divisions cost several times more).
+    const bool weighted = uneven && GWe == GW;
     if (weighted) {
         const uint64_t U = (uint64_t)(GW / L.plan_nw) * pre[L.plan_nw];
         if ((uint64_t)tcost * (U + 1) < (1ull << 32))
